@@ -1,0 +1,478 @@
+#!/usr/bin/env python
+"""Throughput of the EfficientQAT fake-quantized linear hot path on B200.
+
+One step = one pass of the whole path over one batch of synthetic tokens, on the
+Llama-2-7B q_proj workload (M = 4096 tokens, W [4096, 4096] bf16, w2g64):
+
+  min-max init (s, z)                      HBM-bound
+  Block-AP forward  Y = X W-hat^T          quantizer prepass + tcgen05 GEMM
+  Block-AP backward dX = dY W-hat          quantizer prepass + tcgen05 GEMM
+                    dW, ds, dz             tcgen05 GEMM dY^T X with the fused
+                                           straight-through epilogue
+  pack to 2-bit codes                      HBM-bound
+  E2E-QP forward    Y = X ((W_q - z) s)^T  dequant prepass + tcgen05 GEMM
+  E2E-QP backward   dX, ds                 dequant prepass + GEMM; GEMM with the
+                                           fused ds epilogue
+
+value = (6 M N K for Block-AP + 6 M N K for E2E-QP) / step time, in TFLOP/s.
+L2 is flushed (a 512 MiB write) before every timed step.  Under torchrun (N > 1)
+every rank runs the same step on its own token batch (weak scaling) and the
+weight gradients dW, ds, dz and the E2E ds are summed over ranks with NCCL
+all-reduce inside the step (data-parallel training).
+
+--impl reference times the CPU oracle (the only other arm) on a
+bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import weight_quantization_aware_b200 as eqat  # noqa: E402
+from weight_quantization_aware_b200 import synthetic  # noqa: E402
+
+WORKLOAD = synthetic.WORKLOADS[2]
+METRIC = "fake-quant linear fwd+bwd TFLOP/s & % bf16 peak (w2g64); init/pack HBM GB/s"
+PHASES = ["init", "fq_fwd", "fq_bwd_dx", "fq_bwd_w", "pack", "dq_fwd", "dq_bwd_dx", "dq_bwd_ds"]
+LAUNCHES_PER_STEP = {"init": 1, "fq_fwd": 2, "fq_bwd_dx": 2, "fq_bwd_w": 1, "pack": 1,
+                     "dq_fwd": 2, "dq_bwd_dx": 2, "dq_bwd_ds": 1}
+DOMINANT = "fq_bwd_w"  # one kernel: dY^T X with the fused straight-through epilogue
+DOMINANT_KERNEL_SOURCES = ["weight_quantization_aware_b200/csrc/eqat_gemm_tc.cu",
+                           "weight_quantization_aware_b200/csrc/eqat_ptx.cuh",
+                           "weight_quantization_aware_b200/csrc/eqat_qmath.cuh"]
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    for p in DOMINANT_KERNEL_SOURCES:
+        with open(os.path.join(ROOT, p), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return {"hbm_gbs": d["hbm_gbs"], "bf16_tflops": d["bf16_tflops"],
+                "bf16_tflops_sustained": d.get("bf16_tflops_sustained", d["bf16_tflops"]),
+                "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+def load_traffic():
+    """dram bytes per launch of the dominant kernel from the committed ncu summary,
+    if it was taken on the current kernel source."""
+    path = os.path.join(ROOT, "profiles", "gemm_dwhat_fused_ste_llama2-7b-q_proj_traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        d = json.load(f)
+    if d.get("kernel_source_hash") != kernel_source_hash():
+        return None
+    return d.get("dram_bytes_per_launch")
+
+
+# ------------------------------------------------------------------------------ clocks
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc:
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                out, _ = self.proc.communicate()
+            self.lines = [l for l in out.splitlines() if l.strip()]
+        else:
+            self.lines = []
+
+    def summary(self):
+        sm, smax, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for l in self.lines:
+            f = [x.strip() for x in l.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                smax = float(f[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": smax, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ------------------------------------------------------------------------------ our arm
+
+class Step:
+    """Holds the device buffers of one rank and runs the hot path through the C ABI."""
+
+    def __init__(self, wl, rank, bits, group, dev):
+        lin = wl.linears[0]
+        self.M, self.N, self.K = wl.m, lin.n, lin.k
+        self.bits, self.group = bits, group
+        rng = synthetic.rng_for(wl.index, 0)
+        d = synthetic.draw_linear(rng, wl.m, lin.n, lin.k, wl.sigma, wl.dtype, wl.outliers)
+        if rank:  # each data-parallel rank sees its own tokens; W is shared
+            d2 = synthetic.draw_linear(synthetic.rng_for(wl.index, 1000 + rank), wl.m, lin.n, lin.k,
+                                       wl.sigma, wl.dtype, wl.outliers)
+            d["X"], d["dY"] = d2["X"], d2["dY"]
+        self.host = {k: v.pin_memory() for k, v in d.items()}
+        self.X = self.host["X"].to(dev)
+        self.W = self.host["W"].to(dev)
+        self.dY = self.host["dY"].to(dev)
+        M, N, K, G = self.M, self.N, self.K, self.K // group
+        bf = torch.bfloat16
+        self.ws = eqat.workspace(M, N, K, bits, group, bf, dev)
+        self.s = torch.empty((N, G), dtype=torch.float32, device=dev)
+        self.z = torch.empty_like(self.s)
+        self.Y = torch.empty((M, N), dtype=bf, device=dev)
+        self.dX = torch.empty((M, K), dtype=bf, device=dev)
+        self.dW = torch.empty((N, K), dtype=bf, device=dev)
+        self.ds = torch.empty_like(self.s)
+        self.dz = torch.empty_like(self.s)
+        self.codes = torch.empty((N, eqat.packed_row_bytes(K, bits)), dtype=torch.uint8, device=dev)
+        self.zq = torch.empty((N, G), dtype=torch.uint8, device=dev)
+        self.Y2 = torch.empty_like(self.Y)
+        self.dX2 = torch.empty_like(self.dX)
+        self.ds2 = torch.empty_like(self.s)
+
+    def outputs(self):
+        return [self.s, self.z, self.Y, self.dX, self.dW, self.ds, self.dz, self.codes, self.zq,
+                self.Y2, self.dX2, self.ds2]
+
+    def run(self, events=None, allreduce=None):
+        b, g = self.bits, self.group
+
+        def mark(i):
+            if events is not None:
+                events[i].record()
+
+        mark(0)
+        eqat.minmax_init(self.W, b, g, s=self.s, z=self.z)
+        mark(1)
+        eqat.fq_linear_fwd(self.X, self.W, self.s, self.z, b, g, ws=self.ws, Y=self.Y)
+        mark(2)
+        eqat.fq_linear_bwd(self.X, self.W, self.s, self.z, self.dY, b, g, ws=self.ws,
+                           out=(self.dX, None, None, None))
+        mark(3)
+        eqat.fq_linear_bwd(self.X, self.W, self.s, self.z, self.dY, b, g, ws=self.ws,
+                           out=(None, self.dW, self.ds, self.dz))
+        mark(4)
+        eqat.pack_codes(self.W, self.s, self.z, b, g, codes=self.codes, zq=self.zq)
+        mark(5)
+        eqat.dq_linear_fwd(self.X, self.codes, self.zq, self.s, b, g, ws=self.ws, Y=self.Y2)
+        mark(6)
+        eqat.dq_linear_bwd_s(self.X, self.codes, self.zq, self.s, self.dY, b, g, ws=self.ws,
+                             out=(self.dX2, None))
+        mark(7)
+        eqat.dq_linear_bwd_s(self.X, self.codes, self.zq, self.s, self.dY, b, g, ws=self.ws,
+                             out=(None, self.ds2))
+        mark(8)
+        if allreduce is not None:
+            allreduce([self.dW, self.ds, self.dz, self.ds2])
+
+
+def phase_bytes(M, N, K, bits, group):
+    """Algorithmic HBM bytes of the two HBM-bound phases (bf16 W)."""
+    G = K // group
+    init = N * K * 2 + 8 * N * G
+    pack = N * K * 2 + 8 * N * G + N * K * bits // 8 + N * G
+    if bits == 3:
+        pack = N * K * 2 + 8 * N * G + N * K + N * G
+    return init, pack
+
+
+def flush_l2(buf):
+    buf.zero_()
+
+
+def run_ours(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus:
+        raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE={world}")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    dist = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+
+    eqat.load_library()
+    wl = WORKLOAD
+    step = Step(wl, rank, wl.bits, wl.group, dev)
+    M, N, K = step.M, step.N, step.K
+    flush = torch.empty(512 << 20, dtype=torch.uint8, device=dev)
+
+    allreduce = None
+    if dist is not None:
+        def allreduce(ts):
+            for t in ts:
+                dist.all_reduce(t)
+
+    for _ in range(args.warmup):
+        flush_l2(flush)
+        step.run(allreduce=allreduce)
+    torch.cuda.synchronize()
+    if eqat.device_error() != 0:
+        raise RuntimeError("device error word set during warm-up")
+
+    nph = len(PHASES)
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(nph + 2)] for _ in range(args.steps)]
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        t_wall = time.perf_counter()
+        for i in range(args.steps):
+            flush_l2(flush)
+            step.run(events=ev[i], allreduce=allreduce)
+            ev[i][nph + 1].record()
+        torch.cuda.synchronize()
+        t_wall = time.perf_counter() - t_wall
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize()
+    if eqat.device_error() != 0:
+        raise RuntimeError("device error word set during the timed region")
+
+    step_ms = [ev[i][0].elapsed_time(ev[i][nph + 1]) for i in range(args.steps)]
+    phase_ms = {p: [ev[i][j].elapsed_time(ev[i][j + 1]) for i in range(args.steps)] for j, p in enumerate(PHASES)}
+    total_ms = sum(step_ms)
+    if dist is not None:
+        t = torch.tensor([total_ms], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = float(t.item())
+    ms_per_step = total_ms / args.steps
+    flops_step = 12 * M * N * K
+    value = flops_step * world / (ms_per_step * 1e-3) / 1e12
+
+    peaks = load_peaks()
+    mean = {p: sum(v) / len(v) for p, v in phase_ms.items()}
+    dom_ms = mean[DOMINANT]
+    dom_flops = 2 * M * N * K
+    achieved = dom_flops / (dom_ms * 1e-3) / 1e12
+    peak = peaks["bf16_tflops_sustained"]
+    init_b, pack_b = phase_bytes(M, N, K, wl.bits, wl.group)
+    traffic = load_traffic()
+    clocks = clk.summary()
+
+    # --------------------------------------------------------------------- e2e (host buffers)
+    e2e = None
+    if not args.no_e2e:
+        outs = step.outputs()
+        host_out = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in outs]
+        ins = [(step.host["X"], step.X), (step.host["W"], step.W), (step.host["dY"], step.dY)]
+        h2d = sum(h.numel() * h.element_size() for h, _ in ins)
+        d2h = sum(t.numel() * t.element_size() for t in outs)
+        n_e2e = max(3, min(args.steps, 20))
+        for it in range(2):  # warm
+            for h, d in ins:
+                d.copy_(h, non_blocking=True)
+            step.run(allreduce=allreduce)
+            for d, h in zip(outs, host_out):
+                h.copy_(d, non_blocking=True)
+        torch.cuda.synchronize()
+        if dist is not None:
+            dist.barrier()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for it in range(n_e2e):
+            for h, d in ins:
+                d.copy_(h, non_blocking=True)
+            step.run(allreduce=allreduce)
+            for d, h in zip(outs, host_out):
+                h.copy_(d, non_blocking=True)
+        e1.record()
+        torch.cuda.synchronize()
+        e2e_ms = e0.elapsed_time(e1) / n_e2e
+        if dist is not None:
+            t = torch.tensor([e2e_ms], device=dev, dtype=torch.float64)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            e2e_ms = float(t.item())
+        e2e = {"value": round(flops_step * world / (e2e_ms * 1e-3) / 1e12, 3), "unit": "TFLOP/s",
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_ms, 4),
+               "steps": n_e2e}
+
+    line = {
+        "metric": METRIC,
+        "value": round(value, 3),
+        "unit": "TFLOP/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(ms_per_step, 4),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic (seeded N(0,1) activations and gradients, N(0,0.02) weights with 0.1% x10 outliers)",
+        "config": {"workload": wl.name, "M": M, "N": N, "K": K, "bits": wl.bits, "group": wl.group,
+                   "flops_per_step": flops_step, "l2": "flushed before every step (512 MiB write)",
+                   "parallelism": f"dp{world}" if world > 1 else "single-gpu",
+                   "step": "+".join(PHASES)},
+        "roofline": {"bound": "tensor", "kernel": "k_gemm_tc dW-hat = dY^T X + fused straight-through epilogue",
+                     "achieved": round(achieved, 2), "peak": peak, "unit": "TFLOP/s",
+                     "frac": round(achieved / peak, 4), "traffic": traffic,
+                     "peak_kind": f"bf16 dense, sustained, {peaks['source']}"},
+        "phases_ms": {p: round(v, 4) for p, v in mean.items()},
+        "phase_rates": {
+            "init_GBps": round(init_b / (mean["init"] * 1e-3) / 1e9, 1),
+            "pack_GBps": round(pack_b / (mean["pack"] * 1e-3) / 1e9, 1),
+            "init_frac_hbm": round(init_b / (mean["init"] * 1e-3) / 1e9 / peaks["hbm_gbs"], 4),
+            "pack_frac_hbm": round(pack_b / (mean["pack"] * 1e-3) / 1e9 / peaks["hbm_gbs"], 4),
+            "blockap_fwd_bwd_TFLOPs": round(6 * M * N * K / ((mean["fq_fwd"] + mean["fq_bwd_dx"] + mean["fq_bwd_w"]) * 1e-3) / 1e12, 2),
+            "e2e_fwd_bwd_TFLOPs": round(6 * M * N * K / ((mean["dq_fwd"] + mean["dq_bwd_dx"] + mean["dq_bwd_ds"]) * 1e-3) / 1e12, 2),
+            "hbm_peak_GBps": peaks["hbm_gbs"],
+        },
+        "gpu_launches": sum(LAUNCHES_PER_STEP.values()) * args.steps,
+        "clocks": clocks,
+        "wall_s_timed": round(t_wall, 3),
+        "e2e": e2e,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(target_s=args.cpu_seconds)
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+# ------------------------------------------------------------------------------ oracle arm
+
+def oracle_sample(rows: int):
+    """The oracle's hot path on a bounded sample of the workload: min-max init and
+    pack of the whole W; Block-AP and E2E-QP forward (Y rows), input gradient (dX
+    rows) and weight-side gradients (dW, ds, dz / ds rows) for `rows` token rows
+    and `rows` weight rows.  Returns (seconds, flops, description)."""
+    import oracle
+    wl = WORKLOAD
+    lin = wl.linears[0]
+    d = synthetic.workload_linear(wl, 0)
+    X, W, dY = (synthetic.as_f32_numpy(d[k]) for k in ("X", "W", "dY"))
+    M, N, K = wl.m, lin.n, lin.k
+    b, g = wl.bits, wl.group
+    rng = np.random.default_rng(5)
+    r = np.sort(rng.choice(M, rows, replace=False))
+    wr = np.sort(rng.choice(N, rows, replace=False))
+    t0 = time.perf_counter()
+    s, z = oracle.minmax_init(W, b, g)
+    oracle.fq_linear_fwd(X, W, s, z, b, g, rows=r)
+    oracle.fq_linear_bwd(X, W, s, z, dY, b, g, rows=r, wrows=wr)
+    packed, zq = oracle.pack(W, s, z, b, g)
+    oracle.dq_linear_fwd(X, packed, zq, s, b, g, rows=r)
+    oracle.dq_linear_bwd_s(X, packed, zq, s, dY, b, g, rows=r, wrows=wr)
+    dt = time.perf_counter() - t0
+    flops = 2 * (2 * rows * N * K + 2 * rows * N * K + 2 * rows * M * K)  # per mode: Y, dX rows; dW-hat rows
+    desc = (f"{wl.name}: init+pack of all {N}x{K} weights; fwd and dX for {rows} of {M} token rows; "
+            f"dW-hat/dW/ds/dz for {rows} of {N} weight rows; both Block-AP and E2E-QP")
+    return dt, flops, desc
+
+
+def calibrate_rows(target_s: float) -> int:
+    """Rows of the sample so that one oracle_sample() takes about target_s seconds:
+    the cost is a fixed part (init, pack, W-hat) plus a part linear in the rows."""
+    t4, _, _ = oracle_sample(4)
+    t20, _, _ = oracle_sample(20)
+    per_row = max((t20 - t4) / 16, 1e-5)
+    fixed = max(t4 - 4 * per_row, 0.0)
+    return int(max(4, min(WORKLOAD.m, (target_s - fixed) / per_row)))
+
+
+def cpu_baseline(target_s: float = 15.0):
+    import oracle
+    rows = calibrate_rows(target_s)
+    dt, flops, desc = oracle_sample(rows)
+    return {"value": round(flops / dt / 1e12, 6), "unit": "TFLOP/s", "cores": oracle.num_threads(),
+            "kind": "oracle", "sample": desc, "seconds": round(dt, 2)}
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    import oracle
+    wl = WORKLOAD
+    lin = wl.linears[0]
+    per_step = max(1.0, min(8.0, 150.0 / max(1, args.steps + args.warmup)))
+    rows = calibrate_rows(per_step)
+    for _ in range(args.warmup):
+        oracle_sample(rows)
+    times, flops, desc = [], 0, ""
+    for _ in range(args.steps):
+        dt, flops, desc = oracle_sample(rows)
+        times.append(dt)
+    sec = sum(times) / len(times)
+    value = flops / sec / 1e12
+    line = {"impl": "reference", "metric": METRIC, "value": round(value, 6), "unit": "TFLOP/s", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(sec * 1e3, 2),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic",
+            "config": {"workload": wl.name, "M": wl.m, "N": lin.n, "K": lin.k, "bits": wl.bits, "group": wl.group},
+            "cpu_baseline": {"value": round(value, 6), "unit": "TFLOP/s", "cores": oracle.num_threads(),
+                             "kind": "oracle", "sample": desc},
+            "e2e": {"value": round(value, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", default="eqat", choices=["eqat", "reference"])
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    args = ap.parse_args()
+    args.warmup = max(3, args.warmup)  # timing rule: at least 3 untimed warm-up steps
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,182 @@
+/*
+ * eqat.h: C ABI of the B200 (sm_100a) fake-quantized linear layer of
+ * EfficientQAT (Efficient Quantization-Aware Training for LLMs, arXiv 2407.11062).
+ *
+ * The layer quantizes each group of g consecutive in-features of an output row
+ * with a step s and a zero point z (paperlayer.ai summary, appendix D):
+ *   W_int = clamp(round(W / s) + z, 0, 2^b - 1)        (Eq. 1)
+ *   W-hat = (W_int - z) * s                            (Eq. 2)
+ * (zhaoyang97 ACL2025 notes, "Block-AP"), initialised per group by min-max
+ * (modelfoundations.com note "EfficientQAT, low-bit training on a single GPU",
+ * Phase 1), trained with a straight-through backward in Block-AP (paperlayer
+ * appendix A) and, on frozen packed codes, with the exact scale gradient
+ * dW-hat/ds = W_q - z in E2E-QP (modelfoundations Phase 2).
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ * Layout: all matrices are dense, row-major and contiguous.
+ *   X, dX      [M, K]  tokens x in-features
+ *   W, dW, W-hat [N, K] out-features x in-features
+ *   Y, dY      [M, N]
+ *   s, z, ds, dz, zq [N, G], G = K / group  (group j of row n covers columns
+ *              j*group .. j*group + group - 1)
+ *   codes      [N, K/4] bytes for 2-bit (code of column k in bits 2*(k%4)),
+ *              [N, K/2] for 4-bit (bits 4*(k%2)), [N, K] for 3-bit (one code
+ *              per byte, unpacked).
+ * Dtypes: X, W, Y, dY, dX, dW, W-hat share `dt` (EQAT_BF16 or EQAT_F32); s, z, ds,
+ *   dz are fp32; codes and zq are uint8.  In EQAT_BF16 mode the contractions run
+ *   on tcgen05 tensor cores with bf16 operands (W-hat rounded to bf16 to nearest
+ *   even) and fp32 accumulation; in EQAT_F32 mode they run in fp32 on the CUDA
+ *   cores.  The quantizer's element arithmetic is IEEE fp32 in both modes:
+ *   W / s is a correctly rounded division and round() is half-to-even.
+ * Quantizer readings (the pages leave these open): z is a float that every
+ *   forward rounds (zr = round(z)); s = (xmax - xmin) / (2^b - 1) is floored at
+ *   EQAT_S_MIN; the straight-through backward gives round an identity gradient
+ *   and lets clamp pass the gradient only where 0 <= round(W/s) + zr <= 2^b - 1
+ *   (bounds included).
+ * Supported: bits in {2, 3, 4}; group in {32, 64, 128}; K % group == 0;
+ *   N % 8 == 0; M, N, K >= 0 (empty problems are valid and write only what has
+ *   a defined value, e.g. zero gradients when M == 0).
+ * Pointers: device memory (cudaMalloc / PyTorch CUDA tensors) of the current
+ *   device, 16-byte aligned, not overlapping one another.  The caller owns every
+ *   buffer; the library allocates nothing and keeps no state beyond cached
+ *   device attributes.  Outputs are overwritten (gradients are not accumulated).
+ *   NULL optional outputs skip their work.
+ * Workspace: entry points that take (ws, ws_bytes) need at least
+ *   eqat_workspace_bytes(...) bytes of device scratch, 256-byte aligned; it
+ *   holds W-hat between the quantizer prepass and the contractions.
+ * Streams: every call enqueues its kernels on `stream` (a cudaStream_t; NULL is
+ *   the legacy default stream) and returns without synchronising.
+ * Errors: argument errors are detected on the host before anything is launched
+ *   and return EQAT_ERR_NULL / _SHAPE / _ALIGN / _DTYPE / _UNSUPPORTED /
+ *   _WORKSPACE.  A launch failure returns EQAT_ERR_CUDA.  Kernels that wait on
+ *   on-chip barriers bound every wait; a wait that runs out records
+ *   EQAT_ERR_TIMEOUT in a device error word, the kernel releases what it holds
+ *   and returns, and eqat_device_error() reports it.  No call aborts the process
+ *   or lets an exception escape.
+ */
+#ifndef EQAT_H
+#define EQAT_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define EQAT_VERSION 1
+#define EQAT_S_MIN 1e-5f
+
+typedef struct CUstream_st *eqat_stream_t; /* same type as cudaStream_t */
+
+typedef enum {
+    EQAT_OK = 0,
+    EQAT_ERR_NULL = 1,        /* a required pointer is NULL */
+    EQAT_ERR_SHAPE = 2,       /* negative size, K % group, N % 8, size overflow */
+    EQAT_ERR_ALIGN = 3,       /* a pointer is not 16-byte aligned (ws: 256) */
+    EQAT_ERR_DTYPE = 4,       /* unknown eqat_dtype */
+    EQAT_ERR_UNSUPPORTED = 5, /* bits or group outside the supported set; no sm_100 device */
+    EQAT_ERR_WORKSPACE = 6,   /* ws NULL or smaller than eqat_workspace_bytes() */
+    EQAT_ERR_CUDA = 7,        /* a CUDA runtime / launch error */
+    EQAT_ERR_TIMEOUT = 8      /* a bounded on-chip wait ran out (see eqat_device_error) */
+} eqat_status;
+
+typedef enum { EQAT_F32 = 0, EQAT_BF16 = 1 } eqat_dtype;
+
+/* Human-readable name of a status; never NULL. */
+const char *eqat_status_string(int status);
+
+/* Detail of the last error returned on the calling thread (empty if none). */
+const char *eqat_last_error_detail(void);
+
+/* Library ABI version (EQAT_VERSION). */
+int eqat_version(void);
+
+/* Bytes of device workspace that the linear entry points need for this shape
+ * (0 when none).  Depends only on N, K and dt; M, bits and group are accepted
+ * so that later versions may add split-K partials without an ABI change. */
+size_t eqat_workspace_bytes(int64_t M, int64_t N, int64_t K, int bits, int group, int dt);
+
+/* a1. Per-group min-max initialisation (modelfoundations note, Phase 1):
+ *   s[n,j] = max((xmax - xmin) / (2^b - 1), EQAT_S_MIN)   fp32, IEEE division
+ *   z[n,j] = round(-xmin / s[n,j])                        fp32, integer-valued
+ * W [N,K] of dtype wdt (bf16 or fp32); s, z [N,G] fp32 outputs. */
+eqat_status eqat_minmax_init(const void *W, int wdt, int64_t N, int64_t K, int bits, int group,
+                             float *s, float *z, eqat_stream_t stream);
+
+/* a2. The quantizer prepass on its own (Eq. 1 with round(z), Eq. 2):
+ *   u = W/s, q = round(u) + round(z), code = clamp(q, 0, 2^b-1),
+ *   mask = [0 <= q <= 2^b-1], W_hat = (code - round(z)) * s.
+ * W_hat [N,K] has dtype wdt (bf16: rounded to nearest even); code and mask
+ * [N,K] uint8 are optional (NULL skips).  W_hat may be NULL too. */
+eqat_status eqat_fake_quant(const void *W, int wdt, const float *s, const float *z, int64_t N,
+                            int64_t K, int bits, int group, void *W_hat, uint8_t *code,
+                            uint8_t *mask, eqat_stream_t stream);
+
+/* a7. Pack to low-bit integers (modelfoundations note, "Paper vs. code": z is
+ * hard-rounded at pack time; Phase 2: the weights become real integers):
+ *   zq = clamp(round(z), 0, 2^b-1) (uint8 [N,G]),
+ *   codes = clamp(round(W/s) + zq, 0, 2^b-1) packed as described above. */
+eqat_status eqat_pack_codes(const void *W, int wdt, const float *s, const float *z, int64_t N,
+                            int64_t K, int bits, int group, uint8_t *codes, uint8_t *zq,
+                            eqat_stream_t stream);
+
+/* a3 (E2E-QP). Eq. 2 on frozen codes: W_hat = (W_q - zq) * s, dtype dt. */
+eqat_status eqat_dequant_codes(const uint8_t *codes, const uint8_t *zq, const float *s, int64_t N,
+                               int64_t K, int bits, int group, void *W_hat, int dt,
+                               eqat_stream_t stream);
+
+/* a2-a4. Block-AP forward: Y = X W_hat^T with W_hat from (W, s, z) as in
+ * eqat_fake_quant (paperlayer section 3: quantization and dequantization sit
+ * inside the computation graph).  Y [M,N] of dtype dt. */
+eqat_status eqat_fq_linear_fwd(const void *X, const void *W, int dt, const float *s,
+                               const float *z, void *Y, int64_t M, int64_t N, int64_t K,
+                               int bits, int group, void *ws, size_t ws_bytes,
+                               eqat_stream_t stream);
+
+/* a5-a6. Block-AP straight-through backward (paperlayer appendix A):
+ *   dX = dY W_hat                                   [M,K], dtype dt   (nullable)
+ *   dW = (dY^T X) * mask                            [N,K], dtype dt   (nullable)
+ *   ds = sum_group (dY^T X) ((code - zr) - mask*u)  [N,G], fp32       (nullable)
+ *   dz = sum_group (dY^T X) s (mask - 1)            [N,G], fp32       (nullable)
+ * with u, code, mask, zr as in eqat_fake_quant.  dY^T X is formed in fp32 on
+ * chip and never stored; the mask, ds and dz reductions run in the epilogue of
+ * that contraction. */
+eqat_status eqat_fq_linear_bwd(const void *X, const void *W, int dt, const float *s,
+                               const float *z, const void *dY, void *dX, void *dW, float *ds,
+                               float *dz, int64_t M, int64_t N, int64_t K, int bits, int group,
+                               void *ws, size_t ws_bytes, eqat_stream_t stream);
+
+/* a8. E2E-QP forward on frozen codes (modelfoundations Phase 2: only
+ * dequantization in the graph): Y = X ((W_q - zq) s)^T. */
+eqat_status eqat_dq_linear_fwd(const void *X, int dt, const uint8_t *codes, const uint8_t *zq,
+                               const float *s, void *Y, int64_t M, int64_t N, int64_t K, int bits,
+                               int group, void *ws, size_t ws_bytes, eqat_stream_t stream);
+
+/* a9. E2E-QP backward, scales only (modelfoundations Phase 2; zhaoyang97 notes,
+ * E2E-QP: dW-hat/ds = w_q - z, no straight-through estimator):
+ *   dX = dY W_hat (nullable),  ds = sum_group (dY^T X) (W_q - zq). */
+eqat_status eqat_dq_linear_bwd_s(const void *X, int dt, const uint8_t *codes, const uint8_t *zq,
+                                 const float *s, const void *dY, void *dX, float *ds, int64_t M,
+                                 int64_t N, int64_t K, int bits, int group, void *ws,
+                                 size_t ws_bytes, eqat_stream_t stream);
+
+/* Synchronises `stream`, then reads and clears the device error word of the
+ * current device.  Returns EQAT_OK, EQAT_ERR_TIMEOUT if a bounded wait ran out
+ * since the last call, or EQAT_ERR_CUDA if the synchronisation failed.  If
+ * where != NULL it receives the raw error word (0 when clean). */
+eqat_status eqat_device_error(int *where, eqat_stream_t stream);
+
+/* Failure-detection self-test: launches one block whose single thread waits on
+ * an on-chip barrier that nothing arrives on, with a bound of timeout_ns
+ * nanoseconds (1e5 .. 1e10).  The wait runs out, records EQAT_ERR_TIMEOUT in
+ * the device error word and the kernel returns normally; the context stays
+ * usable.  Used by the tests of the bounded-wait path. */
+eqat_status eqat_selftest_bounded_wait(int64_t timeout_ns, eqat_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* EQAT_H */

@@ -1,0 +1,118 @@
+"""The C-ABI library loads, exports every entry point its header declares, and
+rejects bad arguments on the host before any CUDA call (CPU only: every call
+here fails validation or has nothing to do, so no kernel is launched)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import weight_quantization_aware_b200 as eqat
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "eqat.h")
+
+OK, NULL, SHAPE, ALIGN, DTYPE, UNSUP, WS, CUDA, TIMEOUT = range(9)
+FAKE = 0x10  # aligned, never dereferenced: each call below fails validation first
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(eqat_[a-z0-9_]+)\s*\(", text)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from weight_quantization_aware_b200 import build
+    build.build()
+    return eqat.load_library()
+
+
+def test_every_declared_entry_point_is_exported(lib):
+    names = declared_functions()
+    assert len(names) >= 14
+    for n in names:
+        assert hasattr(lib, n), f"{n} declared in eqat.h but not exported"
+
+
+def test_status_strings_and_version(lib):
+    for code, name in [(OK, "EQAT_OK"), (NULL, "EQAT_ERR_NULL"), (SHAPE, "EQAT_ERR_SHAPE"),
+                       (ALIGN, "EQAT_ERR_ALIGN"), (DTYPE, "EQAT_ERR_DTYPE"),
+                       (UNSUP, "EQAT_ERR_UNSUPPORTED"), (WS, "EQAT_ERR_WORKSPACE"),
+                       (CUDA, "EQAT_ERR_CUDA"), (TIMEOUT, "EQAT_ERR_TIMEOUT")]:
+        assert eqat.status_name(code) == name
+    assert eqat.status_name(99) == "EQAT_ERR_UNKNOWN"
+    assert lib.eqat_version() == 1
+
+
+def test_workspace_bytes(lib):
+    assert lib.eqat_workspace_bytes(4096, 4096, 4096, 2, 64, 1) == 4096 * 4096 * 2
+    assert lib.eqat_workspace_bytes(128, 512, 256, 2, 64, 0) == 512 * 256 * 8
+    assert lib.eqat_workspace_bytes(1, 8, 32, 2, 32, 1) == 512  # rounded up to 256 B
+    assert lib.eqat_workspace_bytes(1, 0, 32, 2, 32, 1) == 0
+    assert lib.eqat_workspace_bytes(1, 8, 32, 2, 32, 7) == 0
+
+
+def P(v):
+    return ctypes.c_void_p(v)
+
+
+def fwd(lib, X=FAKE, W=FAKE, dt=1, s=FAKE, z=FAKE, Y=FAKE, M=16, N=16, K=64, bits=2, group=64,
+        ws=FAKE, ws_bytes=1 << 20):
+    return lib.eqat_fq_linear_fwd(P(X), P(W), dt, P(s), P(z), P(Y), M, N, K, bits, group, P(ws), ws_bytes, None)
+
+
+def test_fq_fwd_argument_errors(lib):
+    assert fwd(lib, bits=5) == UNSUP
+    assert fwd(lib, bits=1) == UNSUP
+    assert fwd(lib, group=48, K=96) == UNSUP
+    assert fwd(lib, K=96, group=64) == SHAPE
+    assert fwd(lib, N=12) == SHAPE
+    assert fwd(lib, M=-1) == SHAPE
+    assert fwd(lib, M=1 << 31) == SHAPE
+    assert fwd(lib, dt=3) == DTYPE
+    assert fwd(lib, X=0) == NULL
+    assert fwd(lib, W=0) == NULL
+    assert fwd(lib, s=0) == NULL
+    assert fwd(lib, Y=0) == NULL
+    assert fwd(lib, X=FAKE + 4) == ALIGN
+    assert fwd(lib, Y=FAKE + 8) == ALIGN
+    assert fwd(lib, ws=0) == WS
+    assert fwd(lib, ws_bytes=100) == WS
+    assert fwd(lib, ws=FAKE + 16) == ALIGN  # 16-aligned but not 256-aligned
+    assert b"256" in lib.eqat_last_error_detail()
+    # empty problems have nothing to do and touch no device
+    assert fwd(lib, M=0) == OK
+    assert fwd(lib, N=0) == OK
+
+
+def test_other_entry_points_argument_errors(lib):
+    st = None
+    assert lib.eqat_minmax_init(P(FAKE), 1, 16, 96, 2, 64, P(FAKE), P(FAKE), st) == SHAPE
+    assert lib.eqat_minmax_init(P(FAKE), 1, 16, 64, 2, 64, P(0), P(FAKE), st) == NULL
+    assert lib.eqat_minmax_init(P(FAKE), 1, 0, 64, 2, 64, P(0), P(0), st) == OK
+    assert lib.eqat_fake_quant(P(FAKE), 1, P(FAKE), P(FAKE), 16, 64, 2, 64, P(FAKE + 2), P(0), P(0), st) == ALIGN
+    assert lib.eqat_fake_quant(P(FAKE), 1, P(FAKE), P(FAKE), 16, 64, 2, 64, P(0), P(0), P(0), st) == OK
+    assert lib.eqat_pack_codes(P(FAKE), 1, P(FAKE), P(FAKE), 16, 64, 2, 64, P(0), P(FAKE), st) == NULL
+    assert lib.eqat_pack_codes(P(FAKE), 1, P(FAKE), P(FAKE), 16, 64, 6, 64, P(FAKE), P(FAKE), st) == UNSUP
+    assert lib.eqat_dequant_codes(P(FAKE), P(FAKE), P(FAKE), 16, 64, 2, 64, P(FAKE), 2, st) == DTYPE
+    assert lib.eqat_fq_linear_bwd(P(FAKE), P(FAKE), 1, P(FAKE), P(FAKE), P(0), P(FAKE), P(0), P(0), P(0),
+                                  16, 16, 64, 2, 64, P(FAKE), 1 << 20, st) == NULL
+    # nothing requested -> nothing to do
+    assert lib.eqat_fq_linear_bwd(P(FAKE), P(FAKE), 1, P(FAKE), P(FAKE), P(FAKE), P(0), P(0), P(0), P(0),
+                                  16, 16, 64, 2, 64, P(0), 0, st) == OK
+    assert lib.eqat_fq_linear_bwd(P(FAKE), P(FAKE), 1, P(FAKE), P(FAKE), P(FAKE), P(FAKE), P(0), P(0), P(0),
+                                  16, 16, 64, 2, 64, P(FAKE), 10, st) == WS
+    assert lib.eqat_dq_linear_fwd(P(FAKE), 1, P(FAKE), P(FAKE), P(FAKE), P(FAKE), 16, 16, 64, 3, 128,
+                                  P(FAKE), 1 << 20, st) == SHAPE
+    assert lib.eqat_dq_linear_bwd_s(P(FAKE), 1, P(FAKE), P(FAKE), P(FAKE), P(FAKE), P(0), P(0),
+                                    16, 16, 64, 2, 64, P(0), 0, st) == OK
+    assert lib.eqat_selftest_bounded_wait(10, st) == SHAPE
+
+
+def test_binding_refuses_cpu_tensors():
+    import torch
+    W = torch.zeros(16, 64, dtype=torch.bfloat16)
+    with pytest.raises(ValueError):
+        eqat.minmax_init(W, 2, 64)

@@ -1,0 +1,225 @@
+"""GPU parity: the CUDA path (through the Python binding and the C ABI) against the
+CPU oracle on the same seeded inputs, at sizes that span several tiles and end in
+ragged tails, in both quantizer states (min-max init, where nothing is clamped,
+and a "trained" state with shrunk steps and shifted zero points, where a few
+percent of the weights are clamped)."""
+import numpy as np
+import pytest
+import torch
+
+import weight_quantization_aware_b200 as eqat
+from weight_quantization_aware_b200 import synthetic
+from parity import TOL_GEMM, TOL_RED, assert_bits_equal, assert_close, bf16_round, to_np
+
+pytestmark = pytest.mark.gpu
+
+BF16_SHAPES = [  # (M, N, K, bits, group)
+    (300, 392, 384, 2, 64),
+    (128, 256, 256, 3, 128),
+    (200, 136, 160, 4, 32),
+    (1, 8, 32, 2, 32),
+    (257, 520, 640, 2, 128),
+]
+
+
+@pytest.fixture(scope="module", autouse=True)
+def built():
+    from weight_quantization_aware_b200 import build
+    build.build()
+    eqat.load_library()
+    assert torch.cuda.is_available()
+    yield
+    assert eqat.device_error() == 0
+
+
+def inputs(M, N, K, bits, g, dtype, seed, trained, orc):
+    d = synthetic.draw_linear(np.random.default_rng(seed), M, N, K, 0.02, dtype)
+    Xn, Wn, dYn = (synthetic.as_f32_numpy(d[k]) for k in ("X", "W", "dY"))
+    s, z = orc.minmax_init(Wn, bits, g)
+    if trained:
+        s, z = synthetic.perturb_quant_params(s, z, seed)
+        z = z + np.float32(0.375)  # non-integer zero points: round(z) in every forward
+    dev = {k: v.cuda() for k, v in d.items()}
+    dev["s"] = torch.from_numpy(s).cuda()
+    dev["z"] = torch.from_numpy(z).cuda()
+    return dev, Xn, Wn, dYn, s, z
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+@pytest.mark.parametrize("bits,g", [(2, 32), (2, 64), (2, 128), (3, 128), (3, 64), (4, 32)])
+def test_minmax_init_bit_exact(orc, dtype, bits, g):
+    rng = np.random.default_rng(bits * 1000 + g)
+    d = synthetic.draw_linear(rng, 1, 264, 1024, 0.02, dtype)
+    Wn = synthetic.as_f32_numpy(d["W"])
+    s_ref, z_ref = orc.minmax_init(Wn, bits, g)
+    s, z = eqat.minmax_init(d["W"].cuda(), bits, g)
+    assert_bits_equal(to_np(s), s_ref, "s")
+    assert_bits_equal(to_np(z), z_ref, "z")
+
+
+def test_minmax_init_degenerate_groups(orc):
+    W = np.zeros((8, 128), np.float32)
+    W[0, :64] = 0.25          # constant group: step floor
+    W[1, :64] = -0.5          # all negative
+    W[1, 64:] = np.linspace(0.1, 0.9, 64)  # all positive
+    W[2, :] = np.linspace(-1, 1, 128)
+    W[3, ::2] = 1e-3
+    Wt = torch.from_numpy(W)
+    for dtype in (torch.float32, torch.bfloat16):
+        Wd = Wt.to(dtype)
+        Wn = Wd.float().numpy()
+        s_ref, z_ref = orc.minmax_init(Wn, 2, 64)
+        s, z = eqat.minmax_init(Wd.cuda(), 2, 64)
+        assert_bits_equal(to_np(s), s_ref, "s")
+        assert_bits_equal(to_np(z), z_ref, "z")
+        wh_ref, c_ref, m_ref, _ = orc.fake_quant(Wn, s_ref, z_ref, 2, 64)
+        wh, c, m = eqat.fake_quant(Wd.cuda(), s, z, 2, 64)
+        assert_bits_equal(to_np(c), c_ref, "code")
+        assert_bits_equal(to_np(m), m_ref, "mask")
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+@pytest.mark.parametrize("trained", [False, True])
+@pytest.mark.parametrize("bits,g", [(2, 64), (3, 128), (4, 32)])
+def test_fake_quant_and_pack_bit_exact(orc, dtype, trained, bits, g):
+    dev, Xn, Wn, dYn, s, z = inputs(4, 136, 512, bits, g, dtype, 31 + bits, trained, orc)
+    wh_ref, c_ref, m_ref, _ = orc.fake_quant(Wn, s, z, bits, g)
+    wh, c, m = eqat.fake_quant(dev["W"], dev["s"], dev["z"], bits, g)
+    assert_bits_equal(to_np(c), c_ref, "code")
+    assert_bits_equal(to_np(m), m_ref, "mask")
+    exp_wh = wh_ref if dtype == "f32" else bf16_round(wh_ref)
+    assert_bits_equal(to_np(wh), exp_wh, "W_hat")
+    if trained:
+        assert 0 < m_ref.mean() < 1
+    p_ref, zq_ref = orc.pack(Wn, s, z, bits, g)
+    p, zq = eqat.pack_codes(dev["W"], dev["s"], dev["z"], bits, g)
+    assert_bits_equal(to_np(p), p_ref, "packed codes")
+    assert_bits_equal(to_np(zq), zq_ref, "zq")
+    dq_ref = orc.dequant_packed(p_ref, zq_ref, s, 512, bits, g)
+    for odt in (torch.float32, torch.bfloat16):
+        dq = eqat.dequant_codes(p, zq, dev["s"], 512, bits, g, odt)
+        assert_bits_equal(to_np(dq), dq_ref if odt == torch.float32 else bf16_round(dq_ref), "dequant")
+
+
+def check_fq(orc, M, N, K, bits, g, dtype, seed, trained):
+    dev, Xn, Wn, dYn, s, z = inputs(M, N, K, bits, g, dtype, seed, trained, orc)
+    Y = eqat.fq_linear_fwd(dev["X"], dev["W"], dev["s"], dev["z"], bits, g)
+    dX, dW, ds, dz = eqat.fq_linear_bwd(dev["X"], dev["W"], dev["s"], dev["z"], dev["dY"], bits, g)
+    Y_ref = orc.fq_linear_fwd(Xn, Wn, s, z, bits, g)
+    dX_ref, dW_ref, ds_ref, dz_ref = orc.fq_linear_bwd(Xn, Wn, s, z, dYn, bits, g)
+    assert_close(to_np(Y), Y_ref, TOL_GEMM, "Y")
+    assert_close(to_np(dX), dX_ref, TOL_GEMM, "dX")
+    assert_close(to_np(dW), dW_ref, TOL_GEMM, "dW")
+    # the straight-through mask is an integer decision: clamped weights get exactly 0
+    _, _, m_ref, _ = orc.fake_quant(Wn, s, z, bits, g)
+    assert (to_np(dW)[m_ref == 0] == 0).all()
+    assert_close(to_np(ds), ds_ref, TOL_RED, "ds")
+    if np.abs(dz_ref).max() == 0:
+        assert (to_np(dz) == 0).all()
+    else:
+        assert_close(to_np(dz), dz_ref, TOL_RED, "dz")
+    return m_ref
+
+
+@pytest.mark.parametrize("trained", [False, True])
+@pytest.mark.parametrize("shape", BF16_SHAPES, ids=lambda s: "x".join(map(str, s)))
+def test_fq_linear_bf16_tensor_core(orc, shape, trained):
+    M, N, K, bits, g = shape
+    check_fq(orc, M, N, K, bits, g, "bf16", 100 + M + K, trained)
+
+
+@pytest.mark.parametrize("trained", [False, True])
+@pytest.mark.parametrize("shape", [(128, 512, 256, 2, 64), (77, 24, 96, 3, 32), (5, 64, 128, 4, 128)],
+                         ids=lambda s: "x".join(map(str, s)))
+def test_fq_linear_f32(orc, shape, trained):
+    M, N, K, bits, g = shape
+    check_fq(orc, M, N, K, bits, g, "f32", 200 + M, trained)
+
+
+def check_dq(orc, M, N, K, bits, g, dtype, seed):
+    dev, Xn, Wn, dYn, s, z = inputs(M, N, K, bits, g, dtype, seed, False, orc)
+    p_ref, zq_ref = orc.pack(Wn, s, z, bits, g)
+    s2, _ = synthetic.perturb_quant_params(s, z, seed)  # E2E-QP has moved the steps
+    codes = torch.from_numpy(p_ref).cuda()
+    zq = torch.from_numpy(zq_ref).cuda()
+    s2d = torch.from_numpy(s2).cuda()
+    Y = eqat.dq_linear_fwd(dev["X"], codes, zq, s2d, bits, g)
+    dX, ds = eqat.dq_linear_bwd_s(dev["X"], codes, zq, s2d, dev["dY"], bits, g)
+    Y_ref = orc.dq_linear_fwd(Xn, p_ref, zq_ref, s2, bits, g)
+    dX_ref, ds_ref = orc.dq_linear_bwd_s(Xn, p_ref, zq_ref, s2, dYn, bits, g)
+    assert_close(to_np(Y), Y_ref, TOL_GEMM, "Y")
+    assert_close(to_np(dX), dX_ref, TOL_GEMM, "dX")
+    assert_close(to_np(ds), ds_ref, TOL_RED, "ds")
+
+
+@pytest.mark.parametrize("shape", BF16_SHAPES, ids=lambda s: "x".join(map(str, s)))
+def test_dq_linear_bf16_tensor_core(orc, shape):
+    M, N, K, bits, g = shape
+    check_dq(orc, M, N, K, bits, g, "bf16", 300 + M)
+
+
+@pytest.mark.parametrize("shape", [(128, 512, 256, 2, 64), (33, 40, 96, 3, 32)], ids=lambda s: "x".join(map(str, s)))
+def test_dq_linear_f32(orc, shape):
+    M, N, K, bits, g = shape
+    check_dq(orc, M, N, K, bits, g, "f32", 400 + M)
+
+
+def test_persistent_tiles_wrap_accumulator_ring(orc):
+    """More than two output tiles per CTA (the double-buffered accumulator ring wraps
+    several times), checked on sampled rows."""
+    M, N, K, bits, g = 4864, 4096, 256, 2, 64  # fwd: 38 x 16 = 608 tiles on 148 SMs
+    dev, Xn, Wn, dYn, s, z = inputs(M, N, K, bits, g, "bf16", 77, True, orc)
+    Y = eqat.fq_linear_fwd(dev["X"], dev["W"], dev["s"], dev["z"], bits, g)
+    dX, dW, ds, dz = eqat.fq_linear_bwd(dev["X"], dev["W"], dev["s"], dev["z"], dev["dY"], bits, g)
+    rows = np.r_[0, 1, 127, 128, 2047, 2048, np.random.default_rng(0).integers(0, M, 40), M - 1]
+    wrows = np.r_[0, 255, 256, 1000, N - 1, np.random.default_rng(1).integers(0, N, 27)]
+    wh = orc.fake_quant(Wn, s, z, bits, g)[0]
+    assert_close(to_np(Y)[rows], orc.linear_fwd(Xn, wh, rows), TOL_GEMM, "Y rows")
+    assert_close(to_np(dX)[rows], orc.linear_dx(dYn, wh, rows), TOL_GEMM, "dX rows")
+    dwh = orc.linear_dwhat(dYn, Xn, wrows)
+    dW_ref, ds_ref, dz_ref = orc.ste_grads(Wn, s, z, dwh, bits, g, wrows)
+    assert_close(to_np(dW)[wrows], dW_ref, TOL_GEMM, "dW rows")
+    assert_close(to_np(ds)[wrows], ds_ref, TOL_RED, "ds rows")
+    assert_close(to_np(dz)[wrows], dz_ref, TOL_RED, "dz rows")
+
+
+def test_empty_and_degenerate_problems(orc):
+    dev = "cuda"
+    bf = torch.bfloat16
+    # M == 0: Y and dX are empty; the weight gradients are exact zeros
+    X = torch.empty(0, 64, dtype=bf, device=dev)
+    W = torch.randn(16, 64, device=dev).to(bf)
+    s, z = eqat.minmax_init(W, 2, 64)
+    dY = torch.empty(0, 16, dtype=bf, device=dev)
+    assert eqat.fq_linear_fwd(X, W, s, z, 2, 64).shape == (0, 16)
+    dX, dW, ds, dz = eqat.fq_linear_bwd(X, W, s, z, dY, 2, 64)
+    assert dX.shape == (0, 64)
+    assert (dW == 0).all() and (ds == 0).all() and (dz == 0).all()
+    dX2, ds2 = eqat.dq_linear_bwd_s(X, *eqat.pack_codes(W, s, z, 2, 64), s, dY, 2, 64)
+    assert (ds2 == 0).all()
+    # N == 0: Y empty, dX exact zeros
+    X = torch.randn(8, 64, device=dev).to(bf)
+    W0 = torch.empty(0, 64, dtype=bf, device=dev)
+    s0, z0 = eqat.minmax_init(W0, 2, 64)
+    dY0 = torch.empty(8, 0, dtype=bf, device=dev)
+    assert eqat.fq_linear_fwd(X, W0, s0, z0, 2, 64).shape == (8, 0)
+    dX, dW, ds, dz = eqat.fq_linear_bwd(X, W0, s0, z0, dY0, 2, 64)
+    assert (dX == 0).all()
+    # optional outputs skipped
+    dX, dW, ds, dz = eqat.fq_linear_bwd(X, W, s, z, torch.randn(8, 16, device=dev).to(bf), 2, 64,
+                                        need_dx=False, need_dw=False, need_dz=False)
+    assert dX is None and dW is None and dz is None and ds is not None
+    torch.cuda.synchronize()
+
+
+def test_bounded_wait_reports_timeout_and_context_survives():
+    assert eqat.device_error() == 0
+    eqat.selftest_bounded_wait(50_000_000)  # 50 ms
+    with pytest.raises(eqat.EqatError) as ei:
+        eqat.device_error()
+    assert ei.value.status == eqat.EQAT_ERR_TIMEOUT
+    assert eqat.device_error() == 0  # read-and-clear
+    W = torch.randn(8, 64, device="cuda").to(torch.bfloat16)
+    s, z = eqat.minmax_init(W, 2, 64)
+    torch.cuda.synchronize()
+    assert torch.isfinite(s).all()

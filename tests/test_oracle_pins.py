@@ -94,12 +94,16 @@ def test_golden_worked_examples(orc, case):
 
 # ---------------------------------------------------------------- init invariants
 
+@pytest.mark.parametrize("bf16", [False, True])
 @pytest.mark.parametrize("bits,g", [(2, 32), (2, 64), (2, 128), (3, 128), (3, 64), (4, 64)])
-def test_minmax_endpoints_land_on_first_and_last_codes(orc, bits, g):
+def test_minmax_endpoints_land_on_first_and_last_codes(orc, bits, g, bf16):
     """Phase 1 init: group min lands on code 0, group max on code 2^N-1 (or Q-1 at an
-    exact half-way tie), both within s/2 of the grid."""
+    exact half-way tie), both within s/2 of the grid.  bf16 weights sit on a coarse
+    grid, so exact ties of W/s at .5 are common there."""
     Q = (1 << bits) - 1
     W = rand_w(96, 512, 11 + bits + g)
+    if bf16:
+        W = synthetic.as_f32_numpy(synthetic.to_dtype(W, "bf16"))
     s, z = orc.minmax_init(W, bits, g)
     wh, code, mask, u = orc.fake_quant(W, s, z, bits, g)
     G = 512 // g
@@ -116,13 +120,21 @@ def test_minmax_endpoints_land_on_first_and_last_codes(orc, bits, g):
     tie = np.abs(umax - np.floor(umax) - 0.5) == 0
     assert ((cmax == Q) | (tie & (cmax == Q - 1))).all()
     assert (s > 0).all()
-    tol = s * 0.5 * (1 + 2.0 ** -20)
+    # s/2, plus Q times the one rounding of s = (xmax - xmin)/Q (relative 2^-24), doubled
+    tol = s * (0.5 + Q * 2.0 ** -23)
     assert (np.abs(take(whg, imin) - Wg.min(-1)) <= tol).all()
     assert (np.abs(take(whg, imax) - Wg.max(-1)) <= tol).all()
-    # with xmin < 0 < xmax nothing is clamped after min-max init
+    # With xmin < 0 < xmax, min-max init clamps nothing except, at a half-way tie, the
+    # group maximum: xmax/s - xmin/s is Q up to one rounding of s, and when one of the
+    # two quotients sits exactly on .5 and rounds up (to even) while the other also
+    # rounds up, round(xmax/s) + round(-xmin/s) reaches Q + 1.
     mixed = (Wg.min(-1) < 0) & (Wg.max(-1) > 0)
-    assert mask.reshape(96, G, g)[mixed].all()
     assert ((z >= 0) & (z <= Q))[mixed].all()
+    q = np.rint(ui) + z[..., None]
+    clamped = (mask.reshape(96, G, g) == 0) & mixed[..., None]
+    assert (q[clamped] == Q + 1).all()
+    assert (Wg[clamped] == np.broadcast_to(Wg.max(-1, keepdims=True), Wg.shape)[clamped]).all()
+    assert clamped.sum() <= mixed.sum()
 
 
 def test_init_matches_numpy_fp32_brute_force(orc):

@@ -1,0 +1,255 @@
+"""Python binding of libeqat, the B200 (sm_100a) fake-quantized linear layer of
+EfficientQAT.
+
+Argument marshalling only: every function checks tensor placement, dtype and
+contiguity, allocates the outputs with PyTorch (the library itself allocates
+nothing), passes raw pointers and the current CUDA stream to the C ABI
+(``include/eqat.h``) and raises :class:`EqatError` on a non-zero status.  All the
+arithmetic runs in the library's CUDA kernels; there is no CPU path.  If
+``libeqat.so`` has not been built, loading fails loudly.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libeqat.so")
+
+EQAT_F32 = 0
+EQAT_BF16 = 1
+EQAT_ERR_TIMEOUT = 8
+
+_lib = None
+
+
+class EqatError(RuntimeError):
+    def __init__(self, fn, status, detail):
+        self.status = status
+        super().__init__(f"{fn}: {status_name(status)} ({status}): {detail}")
+
+
+def load_library():
+    """Loads libeqat.so (built in-tree by ``weight_quantization_aware_b200.build``)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise RuntimeError(
+            f"{LIB_PATH} is missing: build it with `python -m weight_quantization_aware_b200.build`"
+            " (there is no fallback implementation)")
+    lib = ctypes.CDLL(LIB_PATH)
+    P, I, I64, SZ = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_size_t
+    sigs = {
+        "eqat_minmax_init": [P, I, I64, I64, I, I, P, P, P],
+        "eqat_fake_quant": [P, I, P, P, I64, I64, I, I, P, P, P, P],
+        "eqat_pack_codes": [P, I, P, P, I64, I64, I, I, P, P, P],
+        "eqat_dequant_codes": [P, P, P, I64, I64, I, I, P, I, P],
+        "eqat_fq_linear_fwd": [P, P, I, P, P, P, I64, I64, I64, I, I, P, SZ, P],
+        "eqat_fq_linear_bwd": [P, P, I, P, P, P, P, P, P, P, I64, I64, I64, I, I, P, SZ, P],
+        "eqat_dq_linear_fwd": [P, I, P, P, P, P, I64, I64, I64, I, I, P, SZ, P],
+        "eqat_dq_linear_bwd_s": [P, I, P, P, P, P, P, P, I64, I64, I64, I, I, P, SZ, P],
+        "eqat_device_error": [P, P],
+        "eqat_selftest_bounded_wait": [I64, P],
+    }
+    for name, args in sigs.items():
+        fn = getattr(lib, name)
+        fn.argtypes = args
+        fn.restype = I
+    lib.eqat_status_string.argtypes = [I]
+    lib.eqat_status_string.restype = ctypes.c_char_p
+    lib.eqat_last_error_detail.argtypes = []
+    lib.eqat_last_error_detail.restype = ctypes.c_char_p
+    lib.eqat_version.restype = I
+    lib.eqat_workspace_bytes.argtypes = [I64, I64, I64, I, I, I]
+    lib.eqat_workspace_bytes.restype = SZ
+    _lib = lib
+    return lib
+
+
+def status_name(status: int) -> str:
+    return load_library().eqat_status_string(int(status)).decode()
+
+
+def _call(name, *args):
+    lib = load_library()
+    st = getattr(lib, name)(*args)
+    if st != 0:
+        raise EqatError(name, st, lib.eqat_last_error_detail().decode())
+
+
+def _p(t):
+    if t is None:
+        return None
+    return ctypes.c_void_p(t.data_ptr()) if t.numel() > 0 else None
+
+
+def _stream():
+    return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+
+
+def _dt(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return EQAT_BF16
+    if t.dtype == torch.float32:
+        return EQAT_F32
+    raise TypeError(f"unsupported dtype {t.dtype}; use torch.bfloat16 or torch.float32")
+
+
+def _req(t, name, dtype=None):
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    return t
+
+
+def packed_row_bytes(K: int, bits: int) -> int:
+    return K // 4 if bits == 2 else K // 2 if bits == 4 else K
+
+
+def workspace_bytes(M: int, N: int, K: int, bits: int, group: int, dtype: torch.dtype) -> int:
+    dt = EQAT_BF16 if dtype == torch.bfloat16 else EQAT_F32
+    return int(load_library().eqat_workspace_bytes(M, N, K, bits, group, dt))
+
+
+def workspace(M, N, K, bits, group, dtype, device=None) -> torch.Tensor:
+    """A uint8 CUDA buffer of eqat_workspace_bytes() bytes (PyTorch blocks are 512-byte aligned)."""
+    n = workspace_bytes(M, N, K, bits, group, dtype)
+    return torch.empty(max(n, 1), dtype=torch.uint8, device=device or "cuda")
+
+
+def _ws(ws, M, N, K, bits, group, dtype, device):
+    if ws is None:
+        ws = workspace(M, N, K, bits, group, dtype, device)
+    _req(ws, "ws", torch.uint8)
+    return ws
+
+
+def minmax_init(W, bits, group, s=None, z=None):
+    """Per-group min-max init: returns (s, z) fp32 [N, K/group]."""
+    _req(W, "W")
+    N, K = W.shape
+    G = K // group if group else 0
+    s = torch.empty((N, G), dtype=torch.float32, device=W.device) if s is None else _req(s, "s", torch.float32)
+    z = torch.empty((N, G), dtype=torch.float32, device=W.device) if z is None else _req(z, "z", torch.float32)
+    _call("eqat_minmax_init", _p(W), _dt(W), N, K, bits, group, _p(s), _p(z), _stream())
+    return s, z
+
+
+def fake_quant(W, s, z, bits, group, want_w_hat=True, want_code=True, want_mask=True):
+    """Quantizer prepass: returns (W_hat (W's dtype), code uint8, mask uint8), None where not wanted."""
+    _req(W, "W"); _req(s, "s", torch.float32); _req(z, "z", torch.float32)
+    N, K = W.shape
+    wh = torch.empty_like(W) if want_w_hat else None
+    code = torch.empty((N, K), dtype=torch.uint8, device=W.device) if want_code else None
+    mask = torch.empty((N, K), dtype=torch.uint8, device=W.device) if want_mask else None
+    _call("eqat_fake_quant", _p(W), _dt(W), _p(s), _p(z), N, K, bits, group, _p(wh), _p(code), _p(mask),
+          _stream())
+    return wh, code, mask
+
+
+def pack_codes(W, s, z, bits, group, codes=None, zq=None):
+    """Pack to low-bit integers: returns (codes uint8 [N, row_bytes], zq uint8 [N, K/group])."""
+    _req(W, "W"); _req(s, "s", torch.float32); _req(z, "z", torch.float32)
+    N, K = W.shape
+    if codes is None:
+        codes = torch.empty((N, packed_row_bytes(K, bits)), dtype=torch.uint8, device=W.device)
+    if zq is None:
+        zq = torch.empty((N, K // group), dtype=torch.uint8, device=W.device)
+    _req(codes, "codes", torch.uint8); _req(zq, "zq", torch.uint8)
+    _call("eqat_pack_codes", _p(W), _dt(W), _p(s), _p(z), N, K, bits, group, _p(codes), _p(zq), _stream())
+    return codes, zq
+
+
+def dequant_codes(codes, zq, s, K, bits, group, dtype=torch.bfloat16):
+    """E2E-QP dequant of frozen codes: W_hat = (W_q - zq) s, [N, K] of `dtype`."""
+    _req(codes, "codes", torch.uint8); _req(zq, "zq", torch.uint8); _req(s, "s", torch.float32)
+    N = codes.shape[0]
+    wh = torch.empty((N, K), dtype=dtype, device=codes.device)
+    _call("eqat_dequant_codes", _p(codes), _p(zq), _p(s), N, K, bits, group, _p(wh), _dt(wh), _stream())
+    return wh
+
+
+def fq_linear_fwd(X, W, s, z, bits, group, ws=None, Y=None):
+    """Block-AP forward Y = X W_hat^T."""
+    _req(X, "X"); _req(W, "W", X.dtype); _req(s, "s", torch.float32); _req(z, "z", torch.float32)
+    M, K = X.shape
+    N = W.shape[0]
+    Y = torch.empty((M, N), dtype=X.dtype, device=X.device) if Y is None else _req(Y, "Y", X.dtype)
+    ws = _ws(ws, M, N, K, bits, group, X.dtype, X.device)
+    _call("eqat_fq_linear_fwd", _p(X), _p(W), _dt(X), _p(s), _p(z), _p(Y), M, N, K, bits, group,
+          _p(ws), ws.numel(), _stream())
+    return Y
+
+
+def fq_linear_bwd(X, W, s, z, dY, bits, group, need_dx=True, need_dw=True, need_ds=True, need_dz=True,
+                  ws=None, out=None):
+    """Block-AP straight-through backward: returns (dX, dW, ds, dz), None where not requested."""
+    _req(X, "X"); _req(W, "W", X.dtype); _req(s, "s", torch.float32); _req(z, "z", torch.float32)
+    _req(dY, "dY", X.dtype)
+    M, K = X.shape
+    N = W.shape[0]
+    G = K // group
+    if out is None:
+        dev = X.device
+        dX = torch.empty((M, K), dtype=X.dtype, device=dev) if need_dx else None
+        dW = torch.empty((N, K), dtype=X.dtype, device=dev) if need_dw else None
+        ds = torch.empty((N, G), dtype=torch.float32, device=dev) if need_ds else None
+        dz = torch.empty((N, G), dtype=torch.float32, device=dev) if need_dz else None
+    else:
+        dX, dW, ds, dz = out
+    ws = _ws(ws, M, N, K, bits, group, X.dtype, X.device)
+    _call("eqat_fq_linear_bwd", _p(X), _p(W), _dt(X), _p(s), _p(z), _p(dY), _p(dX), _p(dW), _p(ds), _p(dz),
+          M, N, K, bits, group, _p(ws), ws.numel(), _stream())
+    return dX, dW, ds, dz
+
+
+def dq_linear_fwd(X, codes, zq, s, bits, group, ws=None, Y=None):
+    """E2E-QP forward on frozen codes: Y = X ((W_q - zq) s)^T."""
+    _req(X, "X"); _req(codes, "codes", torch.uint8); _req(zq, "zq", torch.uint8); _req(s, "s", torch.float32)
+    M, K = X.shape
+    N = codes.shape[0]
+    Y = torch.empty((M, N), dtype=X.dtype, device=X.device) if Y is None else _req(Y, "Y", X.dtype)
+    ws = _ws(ws, M, N, K, bits, group, X.dtype, X.device)
+    _call("eqat_dq_linear_fwd", _p(X), _dt(X), _p(codes), _p(zq), _p(s), _p(Y), M, N, K, bits, group,
+          _p(ws), ws.numel(), _stream())
+    return Y
+
+
+def dq_linear_bwd_s(X, codes, zq, s, dY, bits, group, need_dx=True, need_ds=True, ws=None, out=None):
+    """E2E-QP backward (scales only): returns (dX, ds)."""
+    _req(X, "X"); _req(codes, "codes", torch.uint8); _req(zq, "zq", torch.uint8); _req(s, "s", torch.float32)
+    _req(dY, "dY", X.dtype)
+    M, K = X.shape
+    N = codes.shape[0]
+    if out is None:
+        dX = torch.empty((M, K), dtype=X.dtype, device=X.device) if need_dx else None
+        ds = torch.empty((N, K // group), dtype=torch.float32, device=X.device) if need_ds else None
+    else:
+        dX, ds = out
+    ws = _ws(ws, M, N, K, bits, group, X.dtype, X.device)
+    _call("eqat_dq_linear_bwd_s", _p(X), _dt(X), _p(codes), _p(zq), _p(s), _p(dY), _p(dX), _p(ds),
+          M, N, K, bits, group, _p(ws), ws.numel(), _stream())
+    return dX, ds
+
+
+def device_error():
+    """Synchronises the current stream and returns the raw device error word (0 when clean).
+    Raises EqatError(EQAT_ERR_TIMEOUT) if a bounded on-chip wait ran out."""
+    where = ctypes.c_int(0)
+    lib = load_library()
+    st = lib.eqat_device_error(ctypes.byref(where), _stream())
+    if st != 0:
+        raise EqatError("eqat_device_error", st, lib.eqat_last_error_detail().decode())
+    return where.value
+
+
+def selftest_bounded_wait(timeout_ns: int):
+    _call("eqat_selftest_bounded_wait", int(timeout_ns), _stream())

@@ -1,0 +1,464 @@
+// extern "C" entry points of libeqat: argument validation on the host, then
+// kernel launches on the caller's stream.  No entry point allocates memory,
+// synchronises (except eqat_device_error) or falls back to another device.
+#include <cuda_runtime.h>
+
+#include <cstdint>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+
+#include "../../include/eqat.h"
+#include "eqat_internal.h"
+
+namespace eqat {
+
+cudaError_t current_device_info(DeviceInfo &info) {
+    static std::mutex mu;
+    static DeviceInfo cache[64];
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+    std::lock_guard<std::mutex> lock(mu);
+    if (cache[dev].device != dev) {
+        DeviceInfo d;
+        d.device = dev;
+        if ((e = cudaDeviceGetAttribute(&d.sm_count, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
+        if ((e = cudaDeviceGetAttribute(&d.major, cudaDevAttrComputeCapabilityMajor, dev)) != cudaSuccess) return e;
+        if ((e = cudaDeviceGetAttribute(&d.minor, cudaDevAttrComputeCapabilityMinor, dev)) != cudaSuccess) return e;
+        cache[dev] = d;
+    }
+    info = cache[dev];
+    return cudaSuccess;
+}
+
+}  // namespace eqat
+
+namespace {
+
+using eqat::DeviceInfo;
+using eqat::Epi;
+using eqat::EpiArgs;
+using eqat::Operand;
+
+thread_local char g_detail[256] = "";
+
+void set_detail(const char *msg) {
+    std::snprintf(g_detail, sizeof(g_detail), "%s", msg);
+}
+
+eqat_status fail(eqat_status st, const char *msg) {
+    set_detail(msg);
+    return st;
+}
+
+eqat_status cuda_fail(cudaError_t e, const char *where) {
+    std::snprintf(g_detail, sizeof(g_detail), "%s: %s", where, cudaGetErrorString(e));
+    return EQAT_ERR_CUDA;
+}
+
+bool aligned(const void *p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
+
+// Validates bits, group and sizes (no CUDA call).
+eqat_status check_common(int64_t M, int64_t N, int64_t K, int bits, int group) {
+    if (bits != 2 && bits != 3 && bits != 4) return fail(EQAT_ERR_UNSUPPORTED, "bits must be 2, 3 or 4");
+    if (group != 32 && group != 64 && group != 128)
+        return fail(EQAT_ERR_UNSUPPORTED, "group must be 32, 64 or 128");
+    if (M < 0 || N < 0 || K < 0) return fail(EQAT_ERR_SHAPE, "negative size");
+    if (K % group != 0) return fail(EQAT_ERR_SHAPE, "K must be a multiple of group");
+    if (N % 8 != 0) return fail(EQAT_ERR_SHAPE, "N must be a multiple of 8");
+    const int64_t lim = int64_t(1) << 31;
+    if (M >= lim || N >= lim || K >= lim) return fail(EQAT_ERR_SHAPE, "a dimension is 2^31 or more");
+    if ((N > 0 && K > (int64_t(1) << 60) / N) || (M > 0 && K > (int64_t(1) << 60) / M) ||
+        (M > 0 && N > (int64_t(1) << 60) / M))
+        return fail(EQAT_ERR_SHAPE, "size product overflows");
+    return EQAT_OK;
+}
+
+// The current device must be an sm_100 part; fills dev.  Called after every
+// argument check, right before the first launch.
+eqat_status get_device(DeviceInfo &dev) {
+    cudaError_t e = eqat::current_device_info(dev);
+    if (e != cudaSuccess) return cuda_fail(e, "device query");
+    if (dev.major != 10) return fail(EQAT_ERR_UNSUPPORTED, "needs an sm_100 (B200) device");
+    return EQAT_OK;
+}
+
+// A pointer must be non-NULL when its buffer has elements, and 16-byte aligned.
+eqat_status check_ptr(const void *p, int64_t elems, const char *name) {
+    static thread_local char msg[128];
+    if (elems > 0 && p == nullptr) {
+        std::snprintf(msg, sizeof(msg), "%s is NULL", name);
+        return fail(EQAT_ERR_NULL, msg);
+    }
+    if (p && !aligned(p, 16)) {
+        std::snprintf(msg, sizeof(msg), "%s is not 16-byte aligned", name);
+        return fail(EQAT_ERR_ALIGN, msg);
+    }
+    return EQAT_OK;
+}
+
+eqat_status check_dtype(int dt) {
+    if (dt != EQAT_F32 && dt != EQAT_BF16) return fail(EQAT_ERR_DTYPE, "dtype must be EQAT_F32 or EQAT_BF16");
+    return EQAT_OK;
+}
+
+size_t esize(int dt) { return dt == EQAT_F32 ? 4 : 2; }
+
+int64_t code_bytes(int64_t N, int64_t K, int bits) {
+    return bits == 2 ? N * (K / 4) : bits == 4 ? N * (K / 2) : N * K;
+}
+
+size_t ws_need(int64_t N, int64_t K, int dt) {
+    const size_t per = dt == EQAT_F32 ? 8 : 2;  // W-hat (+ fp32 dW-hat in fp32 mode)
+    const size_t b = static_cast<size_t>(N) * static_cast<size_t>(K) * per;
+    return (b + 255) & ~static_cast<size_t>(255);
+}
+
+eqat_status check_ws(const void *ws, size_t ws_bytes, int64_t N, int64_t K, int dt) {
+    const size_t need = ws_need(N, K, dt);
+    if (need == 0) return EQAT_OK;
+    if (!ws || ws_bytes < need) return fail(EQAT_ERR_WORKSPACE, "workspace missing or smaller than eqat_workspace_bytes()");
+    if (!aligned(ws, 256)) return fail(EQAT_ERR_ALIGN, "workspace is not 256-byte aligned");
+    return EQAT_OK;
+}
+
+#define EQAT_TRY(expr)                       \
+    do {                                     \
+        eqat_status _s = (expr);             \
+        if (_s != EQAT_OK) return _s;        \
+    } while (0)
+
+#define EQAT_CUDA(expr, where)                 \
+    do {                                       \
+        cudaError_t _e = (expr);               \
+        if (_e != cudaSuccess) return cuda_fail(_e, where); \
+    } while (0)
+
+cudaError_t zero(void *p, size_t bytes, cudaStream_t st) {
+    if (!p || bytes == 0) return cudaSuccess;
+    return cudaMemsetAsync(p, 0, bytes, st);
+}
+
+// Y[GM, GN] = A . B^T with the dtype's engine.
+cudaError_t contract(int dt, const Operand &A, const Operand &B, int64_t GM, int64_t GN, int64_t GK,
+                     const EpiArgs &epi, float *f32_scratch, const DeviceInfo &dev, cudaStream_t st) {
+    if (dt == EQAT_BF16) return eqat::launch_gemm_tc(A, B, GM, GN, GK, epi, dev, st);
+    return eqat::launch_gemm_f32(A, B, GM, GN, GK, epi, f32_scratch, dev, st);
+}
+
+}  // namespace
+
+extern "C" {
+
+const char *eqat_status_string(int status) {
+    switch (status) {
+        case EQAT_OK: return "EQAT_OK";
+        case EQAT_ERR_NULL: return "EQAT_ERR_NULL";
+        case EQAT_ERR_SHAPE: return "EQAT_ERR_SHAPE";
+        case EQAT_ERR_ALIGN: return "EQAT_ERR_ALIGN";
+        case EQAT_ERR_DTYPE: return "EQAT_ERR_DTYPE";
+        case EQAT_ERR_UNSUPPORTED: return "EQAT_ERR_UNSUPPORTED";
+        case EQAT_ERR_WORKSPACE: return "EQAT_ERR_WORKSPACE";
+        case EQAT_ERR_CUDA: return "EQAT_ERR_CUDA";
+        case EQAT_ERR_TIMEOUT: return "EQAT_ERR_TIMEOUT";
+        default: return "EQAT_ERR_UNKNOWN";
+    }
+}
+
+const char *eqat_last_error_detail(void) { return g_detail; }
+
+int eqat_version(void) { return EQAT_VERSION; }
+
+size_t eqat_workspace_bytes(int64_t M, int64_t N, int64_t K, int bits, int group, int dt) {
+    (void)M;
+    (void)bits;
+    (void)group;
+    if (N <= 0 || K <= 0 || (dt != EQAT_F32 && dt != EQAT_BF16)) return 0;
+    return ws_need(N, K, dt);
+}
+
+eqat_status eqat_minmax_init(const void *W, int wdt, int64_t N, int64_t K, int bits, int group, float *s,
+                             float *z, eqat_stream_t stream) {
+    DeviceInfo dev;
+    EQAT_TRY(check_dtype(wdt));
+    EQAT_TRY(check_common(0, N, K, bits, group));
+    const int64_t ng = N * (K / group);
+    EQAT_TRY(check_ptr(W, N * K, "W"));
+    EQAT_TRY(check_ptr(s, ng, "s"));
+    EQAT_TRY(check_ptr(z, ng, "z"));
+    if (ng == 0) return EQAT_OK;
+    EQAT_TRY(get_device(dev));
+    EQAT_CUDA(eqat::launch_minmax_init(W, wdt == EQAT_F32, N, K, bits, group, s, z, dev,
+                                       reinterpret_cast<cudaStream_t>(stream)),
+              "minmax_init");
+    return EQAT_OK;
+}
+
+eqat_status eqat_fake_quant(const void *W, int wdt, const float *s, const float *z, int64_t N, int64_t K,
+                            int bits, int group, void *W_hat, uint8_t *code, uint8_t *mask,
+                            eqat_stream_t stream) {
+    DeviceInfo dev;
+    EQAT_TRY(check_dtype(wdt));
+    EQAT_TRY(check_common(0, N, K, bits, group));
+    const int64_t ng = N * (K / group);
+    EQAT_TRY(check_ptr(W, N * K, "W"));
+    EQAT_TRY(check_ptr(s, ng, "s"));
+    EQAT_TRY(check_ptr(z, ng, "z"));
+    EQAT_TRY(check_ptr(W_hat, 0, "W_hat"));
+    EQAT_TRY(check_ptr(code, 0, "code"));
+    EQAT_TRY(check_ptr(mask, 0, "mask"));
+    if (!W_hat && !code && !mask) return EQAT_OK;
+    if (N * K == 0) return EQAT_OK;
+    EQAT_TRY(get_device(dev));
+    EQAT_CUDA(eqat::launch_fake_quant(W, wdt == EQAT_F32, s, z, N, K, bits, group, W_hat, wdt == EQAT_F32,
+                                      code, mask, dev, reinterpret_cast<cudaStream_t>(stream)),
+              "fake_quant");
+    return EQAT_OK;
+}
+
+eqat_status eqat_pack_codes(const void *W, int wdt, const float *s, const float *z, int64_t N, int64_t K,
+                            int bits, int group, uint8_t *codes, uint8_t *zq, eqat_stream_t stream) {
+    DeviceInfo dev;
+    EQAT_TRY(check_dtype(wdt));
+    EQAT_TRY(check_common(0, N, K, bits, group));
+    const int64_t ng = N * (K / group);
+    EQAT_TRY(check_ptr(W, N * K, "W"));
+    EQAT_TRY(check_ptr(s, ng, "s"));
+    EQAT_TRY(check_ptr(z, ng, "z"));
+    EQAT_TRY(check_ptr(codes, code_bytes(N, K, bits), "codes"));
+    EQAT_TRY(check_ptr(zq, ng, "zq"));
+    if (N * K == 0) return EQAT_OK;
+    EQAT_TRY(get_device(dev));
+    EQAT_CUDA(eqat::launch_pack(W, wdt == EQAT_F32, s, z, N, K, bits, group, codes, zq, dev,
+                                reinterpret_cast<cudaStream_t>(stream)),
+              "pack_codes");
+    return EQAT_OK;
+}
+
+eqat_status eqat_dequant_codes(const uint8_t *codes, const uint8_t *zq, const float *s, int64_t N, int64_t K,
+                               int bits, int group, void *W_hat, int dt, eqat_stream_t stream) {
+    DeviceInfo dev;
+    EQAT_TRY(check_dtype(dt));
+    EQAT_TRY(check_common(0, N, K, bits, group));
+    const int64_t ng = N * (K / group);
+    EQAT_TRY(check_ptr(codes, code_bytes(N, K, bits), "codes"));
+    EQAT_TRY(check_ptr(zq, ng, "zq"));
+    EQAT_TRY(check_ptr(s, ng, "s"));
+    EQAT_TRY(check_ptr(W_hat, N * K, "W_hat"));
+    if (N * K == 0) return EQAT_OK;
+    EQAT_TRY(get_device(dev));
+    EQAT_CUDA(eqat::launch_dequant(codes, zq, s, N, K, bits, group, W_hat, dt == EQAT_F32, dev,
+                                   reinterpret_cast<cudaStream_t>(stream)),
+              "dequant_codes");
+    return EQAT_OK;
+}
+
+eqat_status eqat_fq_linear_fwd(const void *X, const void *W, int dt, const float *s, const float *z, void *Y,
+                               int64_t M, int64_t N, int64_t K, int bits, int group, void *ws, size_t ws_bytes,
+                               eqat_stream_t stream) {
+    DeviceInfo dev;
+    EQAT_TRY(check_dtype(dt));
+    EQAT_TRY(check_common(M, N, K, bits, group));
+    const int64_t ng = N * (K / group);
+    EQAT_TRY(check_ptr(X, M * K, "X"));
+    EQAT_TRY(check_ptr(W, N * K, "W"));
+    EQAT_TRY(check_ptr(s, ng, "s"));
+    EQAT_TRY(check_ptr(z, ng, "z"));
+    EQAT_TRY(check_ptr(Y, M * N, "Y"));
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    if (M * N == 0) return EQAT_OK;
+    if (K > 0) EQAT_TRY(check_ws(ws, ws_bytes, N, K, dt));
+    EQAT_TRY(get_device(dev));
+    if (K == 0) {
+        EQAT_CUDA(zero(Y, static_cast<size_t>(M * N) * esize(dt), st), "memset Y");
+        return EQAT_OK;
+    }
+    const bool f32 = dt == EQAT_F32;
+    EQAT_CUDA(eqat::launch_fake_quant(W, f32, s, z, N, K, bits, group, ws, f32, nullptr, nullptr, dev, st),
+              "fq prepass");
+    EpiArgs epi;
+    epi.kind = Epi::kStore;
+    epi.out = Y;
+    epi.ldo = N;
+    epi.out_f32 = f32;
+    EQAT_CUDA(contract(dt, Operand{X, K, false}, Operand{ws, K, false}, M, N, K, epi, nullptr, dev, st),
+              "fq forward contraction");
+    return EQAT_OK;
+}
+
+eqat_status eqat_fq_linear_bwd(const void *X, const void *W, int dt, const float *s, const float *z,
+                               const void *dY, void *dX, void *dW, float *ds, float *dz, int64_t M, int64_t N,
+                               int64_t K, int bits, int group, void *ws, size_t ws_bytes, eqat_stream_t stream) {
+    DeviceInfo dev;
+    EQAT_TRY(check_dtype(dt));
+    EQAT_TRY(check_common(M, N, K, bits, group));
+    const int64_t ng = N * (K / group);
+    EQAT_TRY(check_ptr(X, M * K, "X"));
+    EQAT_TRY(check_ptr(W, N * K, "W"));
+    EQAT_TRY(check_ptr(s, ng, "s"));
+    EQAT_TRY(check_ptr(z, ng, "z"));
+    EQAT_TRY(check_ptr(dY, M * N, "dY"));
+    EQAT_TRY(check_ptr(dX, 0, "dX"));
+    EQAT_TRY(check_ptr(dW, 0, "dW"));
+    EQAT_TRY(check_ptr(ds, 0, "ds"));
+    EQAT_TRY(check_ptr(dz, 0, "dz"));
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    const bool f32 = dt == EQAT_F32;
+    const size_t es = esize(dt);
+    const bool want_w = dW || ds || dz;
+    if (!dX && !want_w) return EQAT_OK;
+    if (N * K > 0) EQAT_TRY(check_ws(ws, ws_bytes, N, K, dt));
+    EQAT_TRY(get_device(dev));
+    if (dX && M * K > 0) {
+        if (N == 0) {
+            EQAT_CUDA(zero(dX, static_cast<size_t>(M * K) * es, st), "memset dX");
+        } else {
+            EQAT_CUDA(eqat::launch_fake_quant(W, f32, s, z, N, K, bits, group, ws, f32, nullptr, nullptr, dev, st),
+                      "fq prepass");
+            EpiArgs epi;
+            epi.kind = Epi::kStore;
+            epi.out = dX;
+            epi.ldo = K;
+            epi.out_f32 = f32;
+            EQAT_CUDA(contract(dt, Operand{dY, N, false}, Operand{ws, K, true}, M, K, N, epi, nullptr, dev, st),
+                      "dX contraction");
+        }
+    }
+    if (want_w && N * K > 0) {
+        if (M == 0) {
+            EQAT_CUDA(zero(dW, static_cast<size_t>(N * K) * es, st), "memset dW");
+            EQAT_CUDA(zero(ds, static_cast<size_t>(ng) * 4, st), "memset ds");
+            EQAT_CUDA(zero(dz, static_cast<size_t>(ng) * 4, st), "memset dz");
+        } else {
+            EpiArgs epi;
+            epi.kind = Epi::kFqGrad;
+            epi.W = W;
+            epi.w_f32 = f32;
+            epi.s = s;
+            epi.z = z;
+            epi.dW = dW;
+            epi.ds = ds;
+            epi.dz = dz;
+            epi.bits = bits;
+            epi.group = group;
+            float *scratch = f32 ? reinterpret_cast<float *>(static_cast<uint8_t *>(ws) + static_cast<size_t>(N * K) * 4)
+                                 : nullptr;
+            EQAT_CUDA(contract(dt, Operand{dY, N, true}, Operand{X, K, true}, N, K, M, epi, scratch, dev, st),
+                      "dW-hat contraction");
+        }
+    }
+    return EQAT_OK;
+}
+
+eqat_status eqat_dq_linear_fwd(const void *X, int dt, const uint8_t *codes, const uint8_t *zq, const float *s,
+                               void *Y, int64_t M, int64_t N, int64_t K, int bits, int group, void *ws,
+                               size_t ws_bytes, eqat_stream_t stream) {
+    DeviceInfo dev;
+    EQAT_TRY(check_dtype(dt));
+    EQAT_TRY(check_common(M, N, K, bits, group));
+    const int64_t ng = N * (K / group);
+    EQAT_TRY(check_ptr(X, M * K, "X"));
+    EQAT_TRY(check_ptr(codes, code_bytes(N, K, bits), "codes"));
+    EQAT_TRY(check_ptr(zq, ng, "zq"));
+    EQAT_TRY(check_ptr(s, ng, "s"));
+    EQAT_TRY(check_ptr(Y, M * N, "Y"));
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    if (M * N == 0) return EQAT_OK;
+    if (K > 0) EQAT_TRY(check_ws(ws, ws_bytes, N, K, dt));
+    EQAT_TRY(get_device(dev));
+    if (K == 0) {
+        EQAT_CUDA(zero(Y, static_cast<size_t>(M * N) * esize(dt), st), "memset Y");
+        return EQAT_OK;
+    }
+    const bool f32 = dt == EQAT_F32;
+    EQAT_CUDA(eqat::launch_dequant(codes, zq, s, N, K, bits, group, ws, f32, dev, st), "dequant prepass");
+    EpiArgs epi;
+    epi.kind = Epi::kStore;
+    epi.out = Y;
+    epi.ldo = N;
+    epi.out_f32 = f32;
+    EQAT_CUDA(contract(dt, Operand{X, K, false}, Operand{ws, K, false}, M, N, K, epi, nullptr, dev, st),
+              "dq forward contraction");
+    return EQAT_OK;
+}
+
+eqat_status eqat_dq_linear_bwd_s(const void *X, int dt, const uint8_t *codes, const uint8_t *zq, const float *s,
+                                 const void *dY, void *dX, float *ds, int64_t M, int64_t N, int64_t K, int bits,
+                                 int group, void *ws, size_t ws_bytes, eqat_stream_t stream) {
+    DeviceInfo dev;
+    EQAT_TRY(check_dtype(dt));
+    EQAT_TRY(check_common(M, N, K, bits, group));
+    const int64_t ng = N * (K / group);
+    EQAT_TRY(check_ptr(X, M * K, "X"));
+    EQAT_TRY(check_ptr(codes, code_bytes(N, K, bits), "codes"));
+    EQAT_TRY(check_ptr(zq, ng, "zq"));
+    EQAT_TRY(check_ptr(s, ng, "s"));
+    EQAT_TRY(check_ptr(dY, M * N, "dY"));
+    EQAT_TRY(check_ptr(dX, 0, "dX"));
+    EQAT_TRY(check_ptr(ds, 0, "ds"));
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    const bool f32 = dt == EQAT_F32;
+    if (!dX && !ds) return EQAT_OK;
+    if (N * K > 0) EQAT_TRY(check_ws(ws, ws_bytes, N, K, dt));
+    EQAT_TRY(get_device(dev));
+    if (dX && M * K > 0) {
+        if (N == 0) {
+            EQAT_CUDA(zero(dX, static_cast<size_t>(M * K) * esize(dt), st), "memset dX");
+        } else {
+            EQAT_CUDA(eqat::launch_dequant(codes, zq, s, N, K, bits, group, ws, f32, dev, st), "dequant prepass");
+            EpiArgs epi;
+            epi.kind = Epi::kStore;
+            epi.out = dX;
+            epi.ldo = K;
+            epi.out_f32 = f32;
+            EQAT_CUDA(contract(dt, Operand{dY, N, false}, Operand{ws, K, true}, M, K, N, epi, nullptr, dev, st),
+                      "dX contraction");
+        }
+    }
+    if (ds && ng > 0) {
+        if (M == 0) {
+            EQAT_CUDA(zero(ds, static_cast<size_t>(ng) * 4, st), "memset ds");
+        } else {
+            EpiArgs epi;
+            epi.kind = Epi::kE2eDs;
+            epi.codes = codes;
+            epi.zq = zq;
+            epi.ds = ds;
+            epi.bits = bits;
+            epi.group = group;
+            float *scratch = f32 ? reinterpret_cast<float *>(static_cast<uint8_t *>(ws) + static_cast<size_t>(N * K) * 4)
+                                 : nullptr;
+            EQAT_CUDA(contract(dt, Operand{dY, N, true}, Operand{X, K, true}, N, K, M, epi, scratch, dev, st),
+                      "dW-hat contraction (E2E)");
+        }
+    }
+    return EQAT_OK;
+}
+
+eqat_status eqat_device_error(int *where, eqat_stream_t stream) {
+    cudaError_t e = cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "stream synchronize");
+    int v = 0;
+    e = eqat::read_and_clear_device_error(v);
+    if (e != cudaSuccess) return cuda_fail(e, "read device error word");
+    if (where) *where = v;
+    if (v != 0) return fail(EQAT_ERR_TIMEOUT, "a bounded on-chip wait ran out");
+    return EQAT_OK;
+}
+
+eqat_status eqat_selftest_bounded_wait(int64_t timeout_ns, eqat_stream_t stream) {
+    if (timeout_ns < 100000 || timeout_ns > 10000000000ll)
+        return fail(EQAT_ERR_SHAPE, "timeout_ns must be within 1e5 .. 1e10");
+    DeviceInfo dev;
+    cudaError_t e = eqat::current_device_info(dev);
+    if (e != cudaSuccess) return cuda_fail(e, "device query");
+    if (dev.major != 10) return fail(EQAT_ERR_UNSUPPORTED, "needs an sm_100 (B200) device");
+    EQAT_CUDA(eqat::launch_selftest_bounded_wait(static_cast<uint64_t>(timeout_ns),
+                                                 reinterpret_cast<cudaStream_t>(stream)),
+              "selftest launch");
+    return EQAT_OK;
+}
+
+}  // extern "C"

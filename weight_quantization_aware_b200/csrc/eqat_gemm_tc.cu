@@ -1,0 +1,558 @@
+// The three contractions of the fake-quantized linear layer on sm_100a tensor
+// cores (tcgen05), with the straight-through and E2E-QP reductions fused into
+// the epilogue:
+//   forward        Y[M,N]  = X[M,K]  . W-hat[N,K]^T   A = X  (K-major), B = W-hat (K-major)
+//   input grad     dX[M,K] = dY[M,N] . W-hat[N,K]     A = dY (K-major), B = W-hat (MN-major)
+//   weight grad    dW-hat[N,K] = dY^T . X             A = dY (MN-major), B = X (MN-major)
+// dW-hat stays in tensor memory: the epilogue turns it into dW (masked), ds and
+// dz (Block-AP, paperlayer appendix A) or ds = sum dW-hat (W_q - zq) (E2E-QP,
+// modelfoundations note Phase 2) and never writes it to HBM.
+//
+// Kernel structure (one CTA per SM, persistent over output tiles):
+//   warp 0       TMA producer: 128x64 A and 256x64 B bf16 tiles, 128-byte
+//                swizzle, into a 4-stage shared-memory ring (48 KB per stage)
+//   warp 1       MMA issuer: one thread issues tcgen05.mma 128x256x16 into one
+//                of two 256-column fp32 accumulators in tensor memory
+//   warp 2       allocates / frees the 512 tensor-memory columns
+//   warps 4..    epilogue: tcgen05.ld 32 columns at a time (thread i of warp w
+//                owns accumulator row 32*(w%4)+i), then the fused epilogue
+// The two accumulators let the epilogue of tile i overlap the main loop of
+// tile i+1.  Every mbarrier wait is bounded (see eqat_ptx.cuh).
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <algorithm>
+#include <atomic>
+#include <cstdint>
+#include <mutex>
+
+#include "eqat_internal.h"
+#include "eqat_ptx.cuh"
+#include "eqat_qmath.cuh"
+
+namespace eqat {
+
+__device__ int g_dev_error = 0;
+
+namespace {
+
+constexpr int BM = 128;
+constexpr int BN = 256;
+constexpr int BK = 64;  // one 128-byte swizzle row of bf16
+constexpr int UK = 16;  // K of one tcgen05.mma kind::f16
+constexpr int STAGES = 4;
+constexpr int A_BYTES = BM * BK * 2;
+constexpr int B_BYTES = BN * BK * 2;
+constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+constexpr int ACC_COLS = BN;
+constexpr int TMEM_COLS = 2 * ACC_COLS;
+constexpr int MN_BOX = 64;                  // MN extent of one MN-major TMA box
+constexpr int MN_BOX_BYTES = MN_BOX * 2 * BK;  // 64 columns x 64 k-rows of bf16
+constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + 256;
+constexpr uint64_t kWaitLimitNs = 4000000000ull;  // 4 s: far above any legitimate wait
+
+struct KParams {
+    int GM, GN, GK;
+    int tiles_m, tiles_n, num_tiles, m_fast;
+    // epilogue
+    void *out;
+    int64_t ldo;
+    const void *W;
+    const float *s;
+    const float *z;
+    void *dW;
+    float *ds;
+    float *dz;
+    const uint8_t *codes;
+    const uint8_t *zq;
+    int group;
+    float Q;
+    int *err;
+    uint64_t wait_limit_ns;
+};
+
+struct SharedCtl {
+    uint64_t full[STAGES];
+    uint64_t empty[STAGES];
+    uint64_t acc_full[2];
+    uint64_t acc_empty[2];
+    uint64_t drain;
+    uint32_t tmem_base;
+    int abort_flag;
+};
+
+__device__ __forceinline__ void tile_coords(const KParams &p, int t, int &tm, int &tn) {
+    if (p.m_fast) {
+        tm = t % p.tiles_m;
+        tn = t / p.tiles_m;
+    } else {
+        tn = t % p.tiles_n;
+        tm = t / p.tiles_n;
+    }
+}
+
+// Epilogue chunk: 32 consecutive accumulator columns of one row.
+template <int EPI, int BITS, bool W_F32>
+struct Epilogue;
+
+// D -> bf16 output.
+template <int BITS, bool W_F32>
+struct Epilogue<0, BITS, W_F32> {
+    float acc_s = 0.0f, acc_z = 0.0f;
+    __device__ __forceinline__ void chunk(const KParams &p, int row, int col, const float (&v)[32]) {
+        if (row >= p.GM) return;
+        __nv_bfloat16 *out = static_cast<__nv_bfloat16 *>(p.out) + static_cast<int64_t>(row) * p.ldo + col;
+        if (col + 32 <= p.GN) {
+            uint4 *o = reinterpret_cast<uint4 *>(out);
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                uint4 r;
+                r.x = pack_bf16x2(v[8 * q + 0], v[8 * q + 1]);
+                r.y = pack_bf16x2(v[8 * q + 2], v[8 * q + 3]);
+                r.z = pack_bf16x2(v[8 * q + 4], v[8 * q + 5]);
+                r.w = pack_bf16x2(v[8 * q + 6], v[8 * q + 7]);
+                o[q] = r;
+            }
+        } else {
+#pragma unroll
+            for (int j = 0; j < 32; ++j)
+                if (col + j < p.GN) out[j] = __float2bfloat16_rn(v[j]);
+        }
+    }
+};
+
+// Block-AP straight-through: D is dW-hat[N, K]; row = n, col = k.
+template <int BITS, bool W_F32>
+struct Epilogue<1, BITS, W_F32> {
+    float acc_s = 0.0f, acc_z = 0.0f;
+    __device__ __forceinline__ void chunk(const KParams &p, int row, int col, const float (&v)[32]) {
+        if (row >= p.GM || col >= p.GN) return;
+        const int64_t K = p.GN;
+        const int64_t G = K / p.group;
+        const int64_t gi = static_cast<int64_t>(row) * G + col / p.group;
+        const float sc = __ldg(p.s + gi);
+        const float zr = rintf(__ldg(p.z + gi));
+        const int64_t e0 = static_cast<int64_t>(row) * K + col;
+        float dwv[32];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            float w[8];
+            if (W_F32)
+                load8<float>(static_cast<const float *>(p.W) + e0 + 8 * q, w);
+            else
+                load8<__nv_bfloat16>(static_cast<const __nv_bfloat16 *>(p.W) + e0 + 8 * q, w);
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                const float d = v[8 * q + j];
+                const QuantElem e = quant_elem(w[j], sc, zr, p.Q);
+                const float dwds = __fsub_rn(__fsub_rn(e.c, zr), e.inside ? e.u : 0.0f);
+                acc_s = fmaf(d, dwds, acc_s);
+                acc_z += e.inside ? 0.0f : d;
+                dwv[8 * q + j] = e.inside ? d : 0.0f;
+            }
+        }
+        if (p.dW) {
+            if (W_F32) {
+                float *o = static_cast<float *>(p.dW) + e0;
+#pragma unroll
+                for (int q = 0; q < 4; ++q)
+                    store8<float>(o + 8 * q, *reinterpret_cast<const float(*)[8]>(&dwv[8 * q]));
+            } else {
+                __nv_bfloat16 *o = static_cast<__nv_bfloat16 *>(p.dW) + e0;
+#pragma unroll
+                for (int q = 0; q < 4; ++q)
+                    store8<__nv_bfloat16>(o + 8 * q, *reinterpret_cast<const float(*)[8]>(&dwv[8 * q]));
+            }
+        }
+        if (((col + 32) % p.group) == 0) {
+            if (p.ds) p.ds[gi] = acc_s;
+            if (p.dz) p.dz[gi] = -sc * acc_z;
+            acc_s = 0.0f;
+            acc_z = 0.0f;
+        }
+    }
+};
+
+// E2E-QP: D is dW-hat[N, K]; ds = sum_group D * (W_q - zq).
+template <int BITS, bool W_F32>
+struct Epilogue<2, BITS, W_F32> {
+    float acc_s = 0.0f, acc_z = 0.0f;
+    __device__ __forceinline__ void chunk(const KParams &p, int row, int col, const float (&v)[32]) {
+        if (row >= p.GM || col >= p.GN) return;
+        const int64_t K = p.GN;
+        const int64_t G = K / p.group;
+        const int64_t gi = static_cast<int64_t>(row) * G + col / p.group;
+        const float zf = static_cast<float>(__ldg(p.zq + gi));
+        uint32_t c[32];
+        if (BITS == 2) {
+            const uint2 r = __ldg(reinterpret_cast<const uint2 *>(p.codes + (static_cast<int64_t>(row) * K + col) / 4));
+#pragma unroll
+            for (int j = 0; j < 16; ++j) c[j] = (r.x >> (2 * j)) & 3u;
+#pragma unroll
+            for (int j = 0; j < 16; ++j) c[16 + j] = (r.y >> (2 * j)) & 3u;
+        } else if (BITS == 4) {
+            const uint4 r = __ldg(reinterpret_cast<const uint4 *>(p.codes + (static_cast<int64_t>(row) * K + col) / 2));
+            const uint32_t w4[4] = {r.x, r.y, r.z, r.w};
+#pragma unroll
+            for (int j = 0; j < 32; ++j) c[j] = (w4[j / 8] >> (4 * (j % 8))) & 15u;
+        } else {
+            const uint4 *src = reinterpret_cast<const uint4 *>(p.codes + static_cast<int64_t>(row) * K + col);
+            const uint4 r0 = __ldg(src), r1 = __ldg(src + 1);
+            const uint32_t w8[8] = {r0.x, r0.y, r0.z, r0.w, r1.x, r1.y, r1.z, r1.w};
+#pragma unroll
+            for (int j = 0; j < 32; ++j) c[j] = (w8[j / 4] >> (8 * (j % 4))) & 0xFFu;
+        }
+#pragma unroll
+        for (int j = 0; j < 32; ++j) acc_s = fmaf(v[j], __fsub_rn(static_cast<float>(c[j]), zf), acc_s);
+        if (((col + 32) % p.group) == 0) {
+            p.ds[gi] = acc_s;
+            acc_s = 0.0f;
+        }
+    }
+};
+
+template <bool A_MN, bool B_MN, int EPI, int BITS, bool W_F32, int EPI_WARPS>
+__global__ void __launch_bounds__((4 + EPI_WARPS) * 32, 1)
+    k_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+              const KParams p) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                                ~static_cast<uintptr_t>(1023));
+    SharedCtl *ctl = reinterpret_cast<SharedCtl *>(smem + STAGES * STAGE_BYTES);
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    constexpr int EPI_THREADS = EPI_WARPS * 32;
+
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < STAGES; ++i) {
+            mbar_init(&ctl->full[i], 1);
+            mbar_init(&ctl->empty[i], 1);
+        }
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&ctl->acc_full[i], 1);
+            mbar_init(&ctl->acc_empty[i], EPI_THREADS);
+        }
+        mbar_init(&ctl->drain, 1);
+        ctl->abort_flag = 0;
+        fence_mbarrier_init();
+        tma_prefetch_desc(&tmA);
+        tma_prefetch_desc(&tmB);
+    }
+    if (warp == 2) {
+        tmem_alloc(&ctl->tmem_base, TMEM_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = ctl->tmem_base;
+    volatile int *abort_flag = &ctl->abort_flag;
+    const int nkb = (p.GK + BK - 1) / BK;
+
+    if (warp == 0) {
+        // ---------------------------------------------------------- TMA producer
+        if (elect_one_sync()) {
+            uint32_t it = 0;
+            uint32_t armed = 0;           // stages with a load issued
+            uint32_t armed_parity = 0;    // parity of the last phase armed per stage
+            bool ok = true;
+            for (int t = blockIdx.x; ok && t < p.num_tiles; t += gridDim.x) {
+                int tm, tn;
+                tile_coords(p, t, tm, tn);
+                const int m0 = tm * BM, n0 = tn * BN;
+                for (int kb = 0; kb < nkb; ++kb, ++it) {
+                    const int st = it % STAGES;
+                    const uint32_t ph = (it / STAGES) & 1u;
+                    if (!mbar_wait_bounded(&ctl->empty[st], ph ^ 1u, abort_flag, p.err, p.wait_limit_ns)) {
+                        ok = false;
+                        break;
+                    }
+                    uint8_t *sa = smem + st * STAGE_BYTES;
+                    uint8_t *sb = sa + A_BYTES;
+                    mbar_arrive_expect_tx(&ctl->full[st], STAGE_BYTES);
+                    armed |= 1u << st;
+                    armed_parity = (armed_parity & ~(1u << st)) | (ph << st);
+                    const int k0 = kb * BK;
+                    if (A_MN) {
+#pragma unroll
+                        for (int b = 0; b < BM / MN_BOX; ++b)
+                            tma_load_2d(sa + b * MN_BOX_BYTES, &tmA, &ctl->full[st], m0 + b * MN_BOX, k0);
+                    } else {
+                        tma_load_2d(sa, &tmA, &ctl->full[st], k0, m0);
+                    }
+                    if (B_MN) {
+#pragma unroll
+                        for (int b = 0; b < BN / MN_BOX; ++b)
+                            tma_load_2d(sb + b * MN_BOX_BYTES, &tmB, &ctl->full[st], n0 + b * MN_BOX, k0);
+                    } else {
+                        tma_load_2d(sb, &tmB, &ctl->full[st], k0, n0);
+                    }
+                }
+            }
+            if (!ok) {
+                // Let the copies already issued land before the block exits.
+                for (int st = 0; st < STAGES; ++st)
+                    if (armed & (1u << st)) {
+                        const uint32_t a = smem_u32(&ctl->full[st]);
+                        const uint64_t t0 = globaltimer_ns();
+                        while (!mbar_try_wait(a, (armed_parity >> st) & 1u) &&
+                               globaltimer_ns() - t0 < 100000000ull) {
+                        }
+                    }
+            }
+        }
+        __syncwarp();
+    } else if (warp == 1) {
+        // ---------------------------------------------------------- MMA issuer
+        if (elect_one_sync()) {
+            constexpr uint32_t idesc = idesc_bf16_f32(BM, BN, A_MN, B_MN);
+            uint32_t it = 0;
+            uint32_t local = 0;
+            bool ok = true;
+            bool issued = false;
+            for (int t = blockIdx.x; ok && t < p.num_tiles; t += gridDim.x, ++local) {
+                const uint32_t acc = local & 1u;
+                const uint32_t aph = (local >> 1) & 1u;
+                if (!mbar_wait_bounded(&ctl->acc_empty[acc], aph ^ 1u, abort_flag, p.err, p.wait_limit_ns)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t d_tmem = tmem_base + acc * ACC_COLS;
+                for (int kb = 0; kb < nkb; ++kb, ++it) {
+                    const int st = it % STAGES;
+                    const uint32_t ph = (it / STAGES) & 1u;
+                    if (!mbar_wait_bounded(&ctl->full[st], ph, abort_flag, p.err, p.wait_limit_ns)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t sa = smem_u32(smem + st * STAGE_BYTES);
+                    const uint32_t sb = sa + A_BYTES;
+#pragma unroll
+                    for (int kk = 0; kk < BK / UK; ++kk) {
+                        const uint64_t ad = A_MN ? smem_desc_sw128(sa + kk * (UK * 128), MN_BOX_BYTES, 1024)
+                                                 : smem_desc_sw128(sa + kk * (UK * 2), 16, 1024);
+                        const uint64_t bd = B_MN ? smem_desc_sw128(sb + kk * (UK * 128), MN_BOX_BYTES, 1024)
+                                                 : smem_desc_sw128(sb + kk * (UK * 2), 16, 1024);
+                        tc_mma_f16(d_tmem, ad, bd, idesc, (kb > 0 || kk > 0) ? 1u : 0u);
+                    }
+                    issued = true;
+                    tc_commit(&ctl->empty[st]);
+                }
+                if (!ok) break;
+                tc_commit(&ctl->acc_full[acc]);
+            }
+            if (!ok && issued) {
+                // Wait for the MMAs already issued before tensor memory is freed.
+                tc_commit(&ctl->drain);
+                const uint32_t a = smem_u32(&ctl->drain);
+                const uint64_t t0 = globaltimer_ns();
+                while (!mbar_try_wait(a, 0) && globaltimer_ns() - t0 < 100000000ull) {
+                }
+            }
+        }
+        __syncwarp();
+    } else if (warp >= 4) {
+        // ---------------------------------------------------------- epilogue
+        const int ew = warp - 4;
+        const int quad = warp & 3;                   // tensor-memory lane quadrant
+        const int half = ew >> 2;                    // column slice of the accumulator
+        constexpr int SLICES = EPI_WARPS / 4;
+        constexpr int COLS = ACC_COLS / SLICES;
+        uint32_t local = 0;
+        for (int t = blockIdx.x; t < p.num_tiles; t += gridDim.x, ++local) {
+            const uint32_t acc = local & 1u;
+            const uint32_t aph = (local >> 1) & 1u;
+            // Every lane waits; the warp leaves together (tcgen05.ld below is .sync.aligned).
+            const bool ok = mbar_wait_bounded(&ctl->acc_full[acc], aph, abort_flag, p.err, p.wait_limit_ns);
+            if (!__all_sync(0xffffffffu, ok)) break;
+            tc_fence_after();
+            int tm, tn;
+            tile_coords(p, t, tm, tn);
+            const int row = tm * BM + quad * 32 + lane;
+            Epilogue<EPI, BITS, W_F32> epi;
+#pragma unroll 1
+            for (int c0 = half * COLS; c0 < (half + 1) * COLS; c0 += 32) {
+                float v[32];
+                tmem_ld_32cols(tmem_base + acc * ACC_COLS + c0 + ((quad * 32) << 16), v);
+                epi.chunk(p, row, tn * BN + c0, v);
+            }
+            tc_fence_before();
+            mbar_arrive(&ctl->acc_empty[acc]);
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 2) {
+        tc_fence_after();
+        tmem_dealloc(tmem_base, TMEM_COLS);
+    }
+}
+
+// ---------------------------------------------------------------------------- host side
+
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+std::once_flag g_encode_once;
+
+cudaError_t get_encode() {
+    std::call_once(g_encode_once, [] {
+        void *fn = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+    });
+    return g_encode ? cudaSuccess : cudaErrorNotSupported;
+}
+
+// K-major operand stored [rows][GK] (row stride ld): box {64 k, box_rows}.
+// MN-major operand stored [GK][rows] (row stride ld): box {64 mn, 64 k}.
+cudaError_t make_map(CUtensorMap &map, const Operand &op, int64_t rows, int64_t GK, int box_rows) {
+    cuuint64_t dims[2];
+    cuuint32_t box[2];
+    if (op.mn_major) {
+        dims[0] = static_cast<cuuint64_t>(rows);
+        dims[1] = static_cast<cuuint64_t>(GK);
+        box[0] = MN_BOX;
+        box[1] = BK;
+    } else {
+        dims[0] = static_cast<cuuint64_t>(GK);
+        dims[1] = static_cast<cuuint64_t>(rows);
+        box[0] = BK;
+        box[1] = static_cast<cuuint32_t>(box_rows);
+    }
+    cuuint64_t strides[1] = {static_cast<cuuint64_t>(op.ld) * 2};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = g_encode(&map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(op.ptr), dims,
+                          strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                          CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
+template <bool A_MN, bool B_MN, int EPI, int BITS, bool W_F32, int EPI_WARPS>
+cudaError_t launch_variant(const CUtensorMap &ma, const CUtensorMap &mb, const KParams &p, int grid,
+                           int dev_id, cudaStream_t st) {
+    auto kern = k_gemm_tc<A_MN, B_MN, EPI, BITS, W_F32, EPI_WARPS>;
+    // The shared-memory opt-in is a per-device function attribute; setting it
+    // twice from racing threads is harmless.
+    static std::atomic<uint64_t> done{0};
+    const uint64_t bit = 1ull << (dev_id & 63);
+    if (!(done.load() & bit)) {
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+        if (e != cudaSuccess) return e;
+        done.fetch_or(bit);
+    }
+    kern<<<grid, (4 + EPI_WARPS) * 32, SMEM_BYTES, st>>>(ma, mb, p);
+    return cudaGetLastError();
+}
+
+int *device_error_ptr() {
+    int *ptr = nullptr;
+    if (cudaGetSymbolAddress(reinterpret_cast<void **>(&ptr), g_dev_error) != cudaSuccess) return nullptr;
+    return ptr;
+}
+
+}  // namespace
+
+cudaError_t launch_gemm_tc(const Operand &A, const Operand &B, int64_t GM, int64_t GN, int64_t GK,
+                           const EpiArgs &epi, const DeviceInfo &dev, cudaStream_t st) {
+    if (GM <= 0 || GN <= 0 || GK <= 0) return cudaSuccess;
+    if (GM > INT32_MAX - BM || GN > INT32_MAX - BN || GK > INT32_MAX - BK) return cudaErrorInvalidValue;
+    cudaError_t e = get_encode();
+    if (e != cudaSuccess) return e;
+    CUtensorMap ma, mb;
+    if ((e = make_map(ma, A, GM, GK, BM)) != cudaSuccess) return e;
+    if ((e = make_map(mb, B, GN, GK, BN)) != cudaSuccess) return e;
+    int *err = device_error_ptr();
+    if (!err) return cudaErrorInvalidSymbol;
+
+    KParams p{};
+    p.GM = static_cast<int>(GM);
+    p.GN = static_cast<int>(GN);
+    p.GK = static_cast<int>(GK);
+    p.tiles_m = static_cast<int>((GM + BM - 1) / BM);
+    p.tiles_n = static_cast<int>((GN + BN - 1) / BN);
+    p.num_tiles = p.tiles_m * p.tiles_n;
+    // Consecutive CTAs share the operand whose tiles are the larger total, so
+    // that one stays hot in L2 while the other streams once.
+    p.m_fast = (GM * GK <= GN * GK) ? 1 : 0;
+    p.out = epi.out;
+    p.ldo = epi.ldo;
+    p.W = epi.W;
+    p.s = epi.s;
+    p.z = epi.z;
+    p.dW = epi.dW;
+    p.ds = epi.ds;
+    p.dz = epi.dz;
+    p.codes = epi.codes;
+    p.zq = epi.zq;
+    p.group = epi.group;
+    p.Q = static_cast<float>((1 << epi.bits) - 1);
+    p.err = err;
+    p.wait_limit_ns = kWaitLimitNs;
+    const int grid = std::min(p.num_tiles, dev.sm_count);
+
+    const bool am = A.mn_major, bm = B.mn_major;
+    switch (epi.kind) {
+        case Epi::kStore:
+            if (epi.out_f32) return cudaErrorInvalidValue;
+            if (!am && !bm) return launch_variant<false, false, 0, 2, false, 4>(ma, mb, p, grid, dev.device, st);
+            if (!am && bm) return launch_variant<false, true, 0, 2, false, 4>(ma, mb, p, grid, dev.device, st);
+            return cudaErrorInvalidValue;
+        case Epi::kFqGrad:
+            if (!(am && bm) || epi.w_f32) return cudaErrorInvalidValue;
+            return launch_variant<true, true, 1, 2, false, 8>(ma, mb, p, grid, dev.device, st);
+        case Epi::kE2eDs:
+            if (!(am && bm)) return cudaErrorInvalidValue;
+            switch (epi.bits) {
+                case 2: return launch_variant<true, true, 2, 2, false, 4>(ma, mb, p, grid, dev.device, st);
+                case 3: return launch_variant<true, true, 2, 3, false, 4>(ma, mb, p, grid, dev.device, st);
+                case 4: return launch_variant<true, true, 2, 4, false, 4>(ma, mb, p, grid, dev.device, st);
+                default: return cudaErrorInvalidValue;
+            }
+    }
+    return cudaErrorInvalidValue;
+}
+
+// ---------------------------------------------------------------------------- error word
+
+cudaError_t read_and_clear_device_error(int &value) {
+    value = 0;
+    cudaError_t e = cudaMemcpyFromSymbol(&value, g_dev_error, sizeof(int));
+    if (e != cudaSuccess) return e;
+    if (value != 0) {
+        const int zero = 0;
+        e = cudaMemcpyToSymbol(g_dev_error, &zero, sizeof(int));
+    }
+    return e;
+}
+
+namespace {
+// One thread waits on a barrier that nothing arrives on; the bounded wait runs
+// out, records the timeout and the kernel returns.
+__global__ void k_selftest_bounded_wait(int *err, uint64_t limit_ns) {
+    __shared__ uint64_t bar;
+    __shared__ int abort_flag;
+    if (threadIdx.x == 0) {
+        abort_flag = 0;
+        mbar_init(&bar, 1);
+        fence_mbarrier_init();
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) (void)mbar_wait_bounded(&bar, 0, &abort_flag, err, limit_ns);
+}
+}  // namespace
+
+cudaError_t launch_selftest_bounded_wait(uint64_t timeout_ns, cudaStream_t st) {
+    int *err = device_error_ptr();
+    if (!err) return cudaErrorInvalidSymbol;
+    k_selftest_bounded_wait<<<1, 32, 0, st>>>(err, timeout_ns);
+    return cudaGetLastError();
+}
+
+}  // namespace eqat

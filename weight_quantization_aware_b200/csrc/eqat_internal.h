@@ -1,0 +1,86 @@
+// Host-side declarations shared by the library's translation units.
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+#include <cuda_runtime.h>
+
+namespace eqat {
+
+struct DeviceInfo {
+    int device = -1;
+    int sm_count = 0;
+    int major = 0;
+    int minor = 0;
+};
+
+// Cached attributes of the current device (thread-safe, one query per device).
+cudaError_t current_device_info(DeviceInfo &info);
+
+// ---------------------------------------------------------------- HBM kernels
+// All element counts are validated by the caller; every launch goes on `st`.
+cudaError_t launch_minmax_init(const void *W, bool w_f32, int64_t N, int64_t K, int bits, int group,
+                               float *s, float *z, const DeviceInfo &dev, cudaStream_t st);
+cudaError_t launch_fake_quant(const void *W, bool w_f32, const float *s, const float *z, int64_t N,
+                              int64_t K, int bits, int group, void *W_hat, bool out_f32,
+                              uint8_t *code, uint8_t *mask, const DeviceInfo &dev,
+                              cudaStream_t st);
+cudaError_t launch_pack(const void *W, bool w_f32, const float *s, const float *z, int64_t N,
+                        int64_t K, int bits, int group, uint8_t *codes, uint8_t *zq,
+                        const DeviceInfo &dev, cudaStream_t st);
+cudaError_t launch_dequant(const uint8_t *codes, const uint8_t *zq, const float *s, int64_t N,
+                           int64_t K, int bits, int group, void *W_hat, bool out_f32,
+                           const DeviceInfo &dev, cudaStream_t st);
+
+// ---------------------------------------------------------------- contractions
+// D[GM, GN] = sum_k A(m, k) B(n, k).  An operand is "K-major" when its reduction
+// index is contiguous in memory (stored as [rows][GK]) and "MN-major" when its
+// row index is ([GK][rows]).  `ld` is the row stride of the stored matrix in
+// elements.
+struct Operand {
+    const void *ptr;
+    int64_t ld;
+    bool mn_major;
+};
+
+enum class Epi : int {
+    kStore = 0,   // D -> out (bf16 or fp32), row stride ldo
+    kFqGrad = 1,  // Block-AP straight-through: dW = D*mask, ds, dz per group
+    kE2eDs = 2,   // E2E-QP: ds = sum_group D * (W_q - zq)
+};
+
+struct EpiArgs {
+    Epi kind = Epi::kStore;
+    void *out = nullptr;
+    int64_t ldo = 0;
+    bool out_f32 = false;
+    // kFqGrad: quantizer inputs of the rows of D (D is [N, K] = dW-hat)
+    const void *W = nullptr;
+    bool w_f32 = false;
+    const float *s = nullptr;
+    const float *z = nullptr;
+    void *dW = nullptr;
+    float *ds = nullptr;
+    float *dz = nullptr;
+    // kE2eDs
+    const uint8_t *codes = nullptr;
+    const uint8_t *zq = nullptr;
+    int bits = 2;
+    int group = 64;
+};
+
+// bf16 operands on tcgen05 tensor cores, fp32 accumulation in tensor memory.
+cudaError_t launch_gemm_tc(const Operand &A, const Operand &B, int64_t GM, int64_t GN, int64_t GK,
+                           const EpiArgs &epi, const DeviceInfo &dev, cudaStream_t st);
+
+// fp32 operands on the CUDA cores; epilogues run as a separate pass over an
+// fp32 D held in `d_scratch` (GM x GN floats) when epi.kind != kStore.
+cudaError_t launch_gemm_f32(const Operand &A, const Operand &B, int64_t GM, int64_t GN, int64_t GK,
+                            const EpiArgs &epi, float *d_scratch, const DeviceInfo &dev,
+                            cudaStream_t st);
+
+// Device error word (bounded waits): read-and-clear on the current device.
+cudaError_t read_and_clear_device_error(int &value);
+cudaError_t launch_selftest_bounded_wait(uint64_t timeout_ns, cudaStream_t st);
+
+}  // namespace eqat

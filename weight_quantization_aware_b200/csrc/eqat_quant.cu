@@ -1,0 +1,308 @@
+// HBM-bound kernels of the quantizer: per-group min-max init, the fake-quant
+// prepass (codes, mask, W-hat), packing to low-bit integers and the E2E-QP
+// dequantization of frozen codes.
+//
+// Every kernel streams its input once with 16-byte loads; a group (g in
+// {32, 64, 128} consecutive in-features of one row) is never split across
+// warps, so per-group reductions are warp shuffles and per-group parameters are
+// read once per thread from L1.  Grids are grid-stride loops sized to a whole
+// number of waves of the SMs.
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cstdint>
+
+#include "eqat_internal.h"
+#include "eqat_qmath.cuh"
+
+namespace eqat {
+namespace {
+
+constexpr int kThreads = 256;
+constexpr int kBlocksPerSm = 8;
+
+inline int grid_for(int64_t work_items, const DeviceInfo &dev, int per_thread = 1) {
+    const int64_t threads = (work_items + per_thread - 1) / per_thread;
+    const int64_t blocks = (threads + kThreads - 1) / kThreads;
+    const int64_t cap = static_cast<int64_t>(dev.sm_count) * kBlocksPerSm;
+    return static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(blocks, cap)));
+}
+
+// ------------------------------------------------------------------ min-max init
+// A thread holds 8 consecutive weights of one group; TPG = G/8 threads cover a
+// group and reduce min/max with xor shuffles; UNROLL independent groups per
+// thread keep 64 bytes of loads in flight per thread.
+template <typename T, int G>
+__global__ void __launch_bounds__(kThreads) k_minmax_init(const T *__restrict__ W, int64_t n_groups,
+                                                          float Q, float *__restrict__ s,
+                                                          float *__restrict__ z) {
+    constexpr int TPG = G / 8;
+    constexpr int GPW = 32 / TPG;  // groups per warp per unrolled slot
+    constexpr int UNROLL = 4;
+    const int lane = threadIdx.x & 31;
+    const int sub = lane % TPG;
+    const int slot = lane / TPG;
+    const int64_t warp = (static_cast<int64_t>(blockIdx.x) * kThreads + threadIdx.x) >> 5;
+    const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * kThreads) >> 5;
+    for (int64_t base = warp * (GPW * UNROLL); base < n_groups; base += nwarps * (GPW * UNROLL)) {
+        float v[UNROLL][8];
+#pragma unroll
+        for (int u = 0; u < UNROLL; ++u) {
+            const int64_t g = base + u * GPW + slot;
+            if (g < n_groups) {
+                load8<T>(W + g * G + sub * 8, v[u]);
+            } else {
+#pragma unroll
+                for (int i = 0; i < 8; ++i) v[u][i] = 0.0f;
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < UNROLL; ++u) {
+            float mn = v[u][0], mx = v[u][0];
+#pragma unroll
+            for (int i = 1; i < 8; ++i) {
+                mn = fminf(mn, v[u][i]);
+                mx = fmaxf(mx, v[u][i]);
+            }
+#pragma unroll
+            for (int off = TPG / 2; off > 0; off >>= 1) {
+                mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, off));
+                mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+            }
+            const int64_t g = base + u * GPW + slot;
+            if (sub == 0 && g < n_groups) {
+                float sc, zz;
+                minmax_step_zero(mn, mx, Q, sc, zz);
+                s[g] = sc;
+                z[g] = zz;
+            }
+        }
+    }
+}
+
+// ------------------------------------------------------------------ fake-quant prepass
+// One thread per 8 consecutive weights (same group): code, mask and W-hat.
+template <typename T, typename O>
+__global__ void __launch_bounds__(kThreads)
+    k_fake_quant(const T *__restrict__ W, const float *__restrict__ s, const float *__restrict__ z,
+                 int64_t n_chunks, int group, float Q, O *__restrict__ W_hat,
+                 uint8_t *__restrict__ code, uint8_t *__restrict__ mask) {
+    const int64_t stride = static_cast<int64_t>(gridDim.x) * kThreads;
+    for (int64_t i = static_cast<int64_t>(blockIdx.x) * kThreads + threadIdx.x; i < n_chunks;
+         i += stride) {
+        const int64_t e0 = i * 8;
+        const int64_t g = e0 / group;
+        const float sc = __ldg(s + g);
+        const float zr = rintf(__ldg(z + g));
+        float w[8], wh[8];
+        load8<T>(W + e0, w);
+        uint32_t c_lo = 0, c_hi = 0, m_lo = 0, m_hi = 0;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            const QuantElem q = quant_elem(w[j], sc, zr, Q);
+            wh[j] = dequant_elem(q.c, zr, sc);
+            const uint32_t cb = static_cast<uint32_t>(q.c);
+            const uint32_t mb = q.inside ? 1u : 0u;
+            if (j < 4) {
+                c_lo |= cb << (8 * j);
+                m_lo |= mb << (8 * j);
+            } else {
+                c_hi |= cb << (8 * (j - 4));
+                m_hi |= mb << (8 * (j - 4));
+            }
+        }
+        if (W_hat) store8<O>(W_hat + e0, wh);
+        if (code) *reinterpret_cast<uint2 *>(code + e0) = make_uint2(c_lo, c_hi);
+        if (mask) *reinterpret_cast<uint2 *>(mask + e0) = make_uint2(m_lo, m_hi);
+    }
+}
+
+// ------------------------------------------------------------------ pack
+// One thread per 16 consecutive weights (same group).  zq = clamp(round(z), 0, Q)
+// and the codes use zr := zq (z hard-rounded at pack time).  Output per thread:
+// 4 bytes (2-bit), 8 bytes (4-bit) or 16 bytes (3-bit, one code per byte).
+template <typename T, int BITS>
+__global__ void __launch_bounds__(kThreads)
+    k_pack(const T *__restrict__ W, const float *__restrict__ s, const float *__restrict__ z,
+           int64_t n_chunks, int group, float Q, uint8_t *__restrict__ codes,
+           uint8_t *__restrict__ zq) {
+    const int64_t stride = static_cast<int64_t>(gridDim.x) * kThreads;
+    for (int64_t i = static_cast<int64_t>(blockIdx.x) * kThreads + threadIdx.x; i < n_chunks;
+         i += stride) {
+        const int64_t e0 = i * 16;
+        const int64_t g = e0 / group;
+        const float sc = __ldg(s + g);
+        const float zr = fminf(fmaxf(rintf(__ldg(z + g)), 0.0f), Q);
+        if (e0 % group == 0) zq[g] = static_cast<uint8_t>(zr);
+        float w[16];
+        load8<T>(W + e0, *reinterpret_cast<float(*)[8]>(&w[0]));
+        load8<T>(W + e0 + 8, *reinterpret_cast<float(*)[8]>(&w[8]));
+        uint32_t c[16];
+#pragma unroll
+        for (int j = 0; j < 16; ++j) c[j] = static_cast<uint32_t>(quant_elem(w[j], sc, zr, Q).c);
+        if (BITS == 2) {
+            uint32_t word = 0;
+#pragma unroll
+            for (int j = 0; j < 16; ++j) word |= c[j] << (2 * j);
+            *reinterpret_cast<uint32_t *>(codes + e0 / 4) = word;
+        } else if (BITS == 4) {
+            uint32_t lo = 0, hi = 0;
+#pragma unroll
+            for (int j = 0; j < 8; ++j) lo |= c[j] << (4 * j);
+#pragma unroll
+            for (int j = 0; j < 8; ++j) hi |= c[8 + j] << (4 * j);
+            *reinterpret_cast<uint2 *>(codes + e0 / 2) = make_uint2(lo, hi);
+        } else {
+            uint4 r;
+            r.x = c[0] | (c[1] << 8) | (c[2] << 16) | (c[3] << 24);
+            r.y = c[4] | (c[5] << 8) | (c[6] << 16) | (c[7] << 24);
+            r.z = c[8] | (c[9] << 8) | (c[10] << 16) | (c[11] << 24);
+            r.w = c[12] | (c[13] << 8) | (c[14] << 16) | (c[15] << 24);
+            *reinterpret_cast<uint4 *>(codes + e0) = r;
+        }
+    }
+}
+
+// ------------------------------------------------------------------ E2E dequant
+// One thread per 16 consecutive codes: W-hat = (W_q - zq) * s (Eq. 2).
+template <int BITS>
+__device__ __forceinline__ void unpack16(const uint8_t *codes, int64_t e0, uint32_t (&c)[16]) {
+    if (BITS == 2) {
+        const uint32_t word = __ldg(reinterpret_cast<const uint32_t *>(codes + e0 / 4));
+#pragma unroll
+        for (int j = 0; j < 16; ++j) c[j] = (word >> (2 * j)) & 3u;
+    } else if (BITS == 4) {
+        const uint2 r = __ldg(reinterpret_cast<const uint2 *>(codes + e0 / 2));
+#pragma unroll
+        for (int j = 0; j < 8; ++j) c[j] = (r.x >> (4 * j)) & 15u;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) c[8 + j] = (r.y >> (4 * j)) & 15u;
+    } else {
+        const uint4 r = __ldg(reinterpret_cast<const uint4 *>(codes + e0));
+        const uint32_t w4[4] = {r.x, r.y, r.z, r.w};
+#pragma unroll
+        for (int j = 0; j < 16; ++j) c[j] = (w4[j / 4] >> (8 * (j % 4))) & 0xFFu;
+    }
+}
+
+template <int BITS, typename O>
+__global__ void __launch_bounds__(kThreads)
+    k_dequant(const uint8_t *__restrict__ codes, const uint8_t *__restrict__ zq,
+              const float *__restrict__ s, int64_t n_chunks, int group, O *__restrict__ W_hat) {
+    const int64_t stride = static_cast<int64_t>(gridDim.x) * kThreads;
+    for (int64_t i = static_cast<int64_t>(blockIdx.x) * kThreads + threadIdx.x; i < n_chunks;
+         i += stride) {
+        const int64_t e0 = i * 16;
+        const int64_t g = e0 / group;
+        const float sc = __ldg(s + g);
+        const float zf = static_cast<float>(__ldg(zq + g));
+        uint32_t c[16];
+        unpack16<BITS>(codes, e0, c);
+        float a[8], b[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) a[j] = dequant_elem(static_cast<float>(c[j]), zf, sc);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) b[j] = dequant_elem(static_cast<float>(c[8 + j]), zf, sc);
+        store8<O>(W_hat + e0, a);
+        store8<O>(W_hat + e0 + 8, b);
+    }
+}
+
+template <typename T>
+cudaError_t minmax_dispatch(const T *W, int64_t n_groups, int group, float Q, float *s, float *z,
+                            const DeviceInfo &dev, cudaStream_t st) {
+    const int grid = grid_for(n_groups * group, dev, 8 * 4);
+    switch (group) {
+        case 32: k_minmax_init<T, 32><<<grid, kThreads, 0, st>>>(W, n_groups, Q, s, z); break;
+        case 64: k_minmax_init<T, 64><<<grid, kThreads, 0, st>>>(W, n_groups, Q, s, z); break;
+        case 128: k_minmax_init<T, 128><<<grid, kThreads, 0, st>>>(W, n_groups, Q, s, z); break;
+        default: return cudaErrorInvalidValue;
+    }
+    return cudaGetLastError();
+}
+
+template <typename T>
+cudaError_t pack_dispatch(const T *W, const float *s, const float *z, int64_t n, int bits, int group,
+                          uint8_t *codes, uint8_t *zq, const DeviceInfo &dev, cudaStream_t st) {
+    const int64_t chunks = n / 16;
+    const int grid = grid_for(chunks, dev);
+    const float Q = static_cast<float>((1 << bits) - 1);
+    switch (bits) {
+        case 2: k_pack<T, 2><<<grid, kThreads, 0, st>>>(W, s, z, chunks, group, Q, codes, zq); break;
+        case 3: k_pack<T, 3><<<grid, kThreads, 0, st>>>(W, s, z, chunks, group, Q, codes, zq); break;
+        case 4: k_pack<T, 4><<<grid, kThreads, 0, st>>>(W, s, z, chunks, group, Q, codes, zq); break;
+        default: return cudaErrorInvalidValue;
+    }
+    return cudaGetLastError();
+}
+
+template <typename O>
+cudaError_t dequant_dispatch(const uint8_t *codes, const uint8_t *zq, const float *s, int64_t n,
+                             int bits, int group, O *W_hat, const DeviceInfo &dev,
+                             cudaStream_t st) {
+    const int64_t chunks = n / 16;
+    const int grid = grid_for(chunks, dev);
+    switch (bits) {
+        case 2: k_dequant<2, O><<<grid, kThreads, 0, st>>>(codes, zq, s, chunks, group, W_hat); break;
+        case 3: k_dequant<3, O><<<grid, kThreads, 0, st>>>(codes, zq, s, chunks, group, W_hat); break;
+        case 4: k_dequant<4, O><<<grid, kThreads, 0, st>>>(codes, zq, s, chunks, group, W_hat); break;
+        default: return cudaErrorInvalidValue;
+    }
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_minmax_init(const void *W, bool w_f32, int64_t N, int64_t K, int bits, int group,
+                               float *s, float *z, const DeviceInfo &dev, cudaStream_t st) {
+    const int64_t n_groups = N * (K / group);
+    if (n_groups == 0) return cudaSuccess;
+    const float Q = static_cast<float>((1 << bits) - 1);
+    if (w_f32) return minmax_dispatch(static_cast<const float *>(W), n_groups, group, Q, s, z, dev, st);
+    return minmax_dispatch(static_cast<const __nv_bfloat16 *>(W), n_groups, group, Q, s, z, dev, st);
+}
+
+cudaError_t launch_fake_quant(const void *W, bool w_f32, const float *s, const float *z, int64_t N,
+                              int64_t K, int bits, int group, void *W_hat, bool out_f32,
+                              uint8_t *code, uint8_t *mask, const DeviceInfo &dev,
+                              cudaStream_t st) {
+    const int64_t chunks = N * K / 8;
+    if (chunks == 0) return cudaSuccess;
+    const int grid = grid_for(chunks, dev);
+    const float Q = static_cast<float>((1 << bits) - 1);
+    using bf = __nv_bfloat16;
+    if (w_f32 && out_f32)
+        k_fake_quant<float, float><<<grid, kThreads, 0, st>>>(
+            static_cast<const float *>(W), s, z, chunks, group, Q, static_cast<float *>(W_hat), code, mask);
+    else if (w_f32)
+        k_fake_quant<float, bf><<<grid, kThreads, 0, st>>>(
+            static_cast<const float *>(W), s, z, chunks, group, Q, static_cast<bf *>(W_hat), code, mask);
+    else if (out_f32)
+        k_fake_quant<bf, float><<<grid, kThreads, 0, st>>>(
+            static_cast<const bf *>(W), s, z, chunks, group, Q, static_cast<float *>(W_hat), code, mask);
+    else
+        k_fake_quant<bf, bf><<<grid, kThreads, 0, st>>>(
+            static_cast<const bf *>(W), s, z, chunks, group, Q, static_cast<bf *>(W_hat), code, mask);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_pack(const void *W, bool w_f32, const float *s, const float *z, int64_t N,
+                        int64_t K, int bits, int group, uint8_t *codes, uint8_t *zq,
+                        const DeviceInfo &dev, cudaStream_t st) {
+    const int64_t n = N * K;
+    if (n == 0) return cudaSuccess;
+    if (w_f32) return pack_dispatch(static_cast<const float *>(W), s, z, n, bits, group, codes, zq, dev, st);
+    return pack_dispatch(static_cast<const __nv_bfloat16 *>(W), s, z, n, bits, group, codes, zq, dev, st);
+}
+
+cudaError_t launch_dequant(const uint8_t *codes, const uint8_t *zq, const float *s, int64_t N,
+                           int64_t K, int bits, int group, void *W_hat, bool out_f32,
+                           const DeviceInfo &dev, cudaStream_t st) {
+    const int64_t n = N * K;
+    if (n == 0) return cudaSuccess;
+    if (out_f32) return dequant_dispatch(codes, zq, s, n, bits, group, static_cast<float *>(W_hat), dev, st);
+    return dequant_dispatch(codes, zq, s, n, bits, group, static_cast<__nv_bfloat16 *>(W_hat), dev, st);
+}
+
+}  // namespace eqat

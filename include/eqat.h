@@ -162,6 +162,26 @@ eqat_status eqat_dq_linear_bwd_s(const void *X, int dt, const uint8_t *codes, co
                                  int64_t N, int64_t K, int bits, int group, void *ws,
                                  size_t ws_bytes, eqat_stream_t stream);
 
+/* Block-AP forward (as eqat_fq_linear_fwd) that allocates nothing and takes no
+ * workspace: the paper has no counterpart; this entry point exists for callers of
+ * the library that cannot allocate device memory or pass a scratch buffer (a
+ * plugin or custom-operator interface that hands over only inputs and outputs, a
+ * process that must not call cudaMalloc once running because it can stall the
+ * whole device, memory owned by an allocator the library cannot reach).
+ * W_hat lives in a static device array of EQAT_NOALLOC_SCRATCH_BYTES (32 MiB)
+ * that the library holds on every GPU that loads it, until the process exits.
+ * Limit: N * K * sizeof(dtype) <= EQAT_NOALLOC_SCRATCH_BYTES (16 Mi bf16 or 8 Mi
+ * fp32 weights); larger layers are rejected with EQAT_ERR_WORKSPACE before
+ * anything is launched.  The first call on a device looks up the array's device
+ * address (cudaGetSymbolAddress), so make that first call before any stream
+ * capture.  Every call shares the one array: calls whose kernels overlap on the
+ * GPU (other streams, other host threads) race on it and must be serialised by
+ * the caller.  Arguments, layout and the result are those of eqat_fq_linear_fwd. */
+#define EQAT_NOALLOC_SCRATCH_BYTES 33554432u
+eqat_status eqat_fq_linear_fwd_noalloc(const void *X, const void *W, int dt, const float *s,
+                                       const float *z, void *Y, int64_t M, int64_t N, int64_t K,
+                                       int bits, int group, eqat_stream_t stream);
+
 /* Synchronises `stream`, then reads and clears the device error word of the
  * current device.  Returns EQAT_OK, EQAT_ERR_TIMEOUT if a bounded wait ran out
  * since the last call, or EQAT_ERR_CUDA if the synchronisation failed.  If

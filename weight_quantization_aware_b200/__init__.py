@@ -51,6 +51,7 @@ def load_library():
         "eqat_fq_linear_bwd": [P, P, I, P, P, P, P, P, P, P, I64, I64, I64, I, I, P, SZ, P],
         "eqat_dq_linear_fwd": [P, I, P, P, P, P, I64, I64, I64, I, I, P, SZ, P],
         "eqat_dq_linear_bwd_s": [P, I, P, P, P, P, P, P, I64, I64, I64, I, I, P, SZ, P],
+        "eqat_fq_linear_fwd_noalloc": [P, P, I, P, P, P, I64, I64, I64, I, I, P],
         "eqat_device_error": [P, P],
         "eqat_selftest_bounded_wait": [I64, P],
     }
@@ -186,6 +187,20 @@ def fq_linear_fwd(X, W, s, z, bits, group, ws=None, Y=None):
     ws = _ws(ws, M, N, K, bits, group, X.dtype, X.device)
     _call("eqat_fq_linear_fwd", _p(X), _p(W), _dt(X), _p(s), _p(z), _p(Y), M, N, K, bits, group,
           _p(ws), ws.numel(), _stream())
+    return Y
+
+
+def fq_linear_fwd_noalloc(X, W, s, z, bits, group, Y):
+    """Block-AP forward for callers that cannot allocate: no workspace, W-hat lives in
+    the library's static 32 MiB device scratch (N*K*sizeof(dtype) must fit).  The
+    output Y is the caller's.  Calls that overlap on the GPU share that scratch and
+    race; serialise them."""
+    _req(X, "X"); _req(W, "W", X.dtype); _req(s, "s", torch.float32); _req(z, "z", torch.float32)
+    _req(Y, "Y", X.dtype)
+    M, K = X.shape
+    N = W.shape[0]
+    _call("eqat_fq_linear_fwd_noalloc", _p(X), _p(W), _dt(X), _p(s), _p(z), _p(Y), M, N, K, bits, group,
+          _stream())
     return Y
 
 

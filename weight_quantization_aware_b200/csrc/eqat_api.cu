@@ -36,13 +36,19 @@ cudaError_t current_device_info(DeviceInfo &info) {
 }  // namespace eqat
 
 namespace {
+thread_local char g_detail[256] = "";
+}  // namespace
+
+namespace eqat {
+void set_error_detail(const char *msg) { std::snprintf(g_detail, sizeof(g_detail), "%s", msg); }
+}  // namespace eqat
+
+namespace {
 
 using eqat::DeviceInfo;
 using eqat::Epi;
 using eqat::EpiArgs;
 using eqat::Operand;
-
-thread_local char g_detail[256] = "";
 
 void set_detail(const char *msg) {
     std::snprintf(g_detail, sizeof(g_detail), "%s", msg);

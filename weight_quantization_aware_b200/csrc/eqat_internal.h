@@ -79,6 +79,9 @@ cudaError_t launch_gemm_f32(const Operand &A, const Operand &B, int64_t GM, int6
                             const EpiArgs &epi, float *d_scratch, const DeviceInfo &dev,
                             cudaStream_t st);
 
+// Records the message that eqat_last_error_detail() returns on this thread.
+void set_error_detail(const char *msg);
+
 // Device error word (bounded waits): read-and-clear on the current device.
 cudaError_t read_and_clear_device_error(int &value);
 cudaError_t launch_selftest_bounded_wait(uint64_t timeout_ns, cudaStream_t st);

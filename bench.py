@@ -2,17 +2,18 @@
 """Throughput of the EfficientQAT fake-quantized linear hot path on B200.
 
 One step = one pass of the whole path over one batch of synthetic tokens, on the
-Llama-2-7B q_proj workload (M = 4096 tokens, W [4096, 4096] bf16, w2g64):
+Llama-2-7B q_proj workload (M = 4096 tokens, W [4096, 4096] bf16, w2g64), in the
+order of a training step (the backward reuses the W-hat its forward left in the
+workspace):
 
-  min-max init (s, z)                      HBM-bound
-  Block-AP forward  Y = X W-hat^T          quantizer prepass + tcgen05 GEMM
-  Block-AP backward dX = dY W-hat          quantizer prepass + tcgen05 GEMM
-                    dW, ds, dz             tcgen05 GEMM dY^T X with the fused
-                                           straight-through epilogue
-  pack to 2-bit codes                      HBM-bound
-  E2E-QP forward    Y = X ((W_q - z) s)^T  dequant prepass + tcgen05 GEMM
-  E2E-QP backward   dX, ds                 dequant prepass + GEMM; GEMM with the
-                                           fused ds epilogue
+  init      min-max init (s, z)                       HBM-bound, 1 kernel
+  fq_fwd    Block-AP forward  Y = X W-hat^T           quantizer prepass + tcgen05 GEMM
+  fq_bwd    Block-AP backward dX = dY W-hat and       one grouped tcgen05 launch; the
+            dW, ds, dz from dY^T X                    dW-hat tiles run the fused
+                                                      straight-through epilogue
+  pack      2-bit codes + zq                          HBM-bound, 1 kernel
+  dq_fwd    E2E-QP forward Y = X ((W_q - z) s)^T      dequant prepass + tcgen05 GEMM
+  dq_bwd    E2E-QP backward dX and ds                 one grouped tcgen05 launch
 
 value = (6 M N K for Block-AP + 6 M N K for E2E-QP) / step time, in TFLOP/s.
 L2 is flushed (a 512 MiB write) before every timed step.  Under torchrun (N > 1)
@@ -45,10 +46,11 @@ from weight_quantization_aware_b200 import synthetic  # noqa: E402
 
 WORKLOAD = synthetic.WORKLOADS[2]
 METRIC = "fake-quant linear fwd+bwd TFLOP/s & % bf16 peak (w2g64); init/pack HBM GB/s"
-PHASES = ["init", "fq_fwd", "fq_bwd_dx", "fq_bwd_w", "pack", "dq_fwd", "dq_bwd_dx", "dq_bwd_ds"]
-LAUNCHES_PER_STEP = {"init": 1, "fq_fwd": 2, "fq_bwd_dx": 2, "fq_bwd_w": 1, "pack": 1,
-                     "dq_fwd": 2, "dq_bwd_dx": 2, "dq_bwd_ds": 1}
-DOMINANT = "fq_bwd_w"  # one kernel: dY^T X with the fused straight-through epilogue
+PHASES = ["init", "fq_fwd", "fq_bwd", "pack", "dq_fwd", "dq_bwd"]
+LAUNCHES_PER_STEP = {"init": 1, "fq_fwd": 2, "fq_bwd": 1, "pack": 1, "dq_fwd": 2, "dq_bwd": 1}
+# One launch: the grouped backward GEMM (dY W-hat tiles and dY^T X tiles with the
+# fused straight-through epilogue), 4 M N K flops.
+DOMINANT = "fq_bwd"
 DOMINANT_KERNEL_SOURCES = ["weight_quantization_aware_b200/csrc/eqat_gemm_tc.cu",
                            "weight_quantization_aware_b200/csrc/eqat_ptx.cuh",
                            "weight_quantization_aware_b200/csrc/eqat_qmath.cuh"]
@@ -76,7 +78,7 @@ def load_peaks():
 def load_traffic():
     """dram bytes per launch of the dominant kernel from the committed ncu summary,
     if it was taken on the current kernel source."""
-    path = os.path.join(ROOT, "profiles", "gemm_dwhat_fused_ste_llama2-7b-q_proj_traffic.json")
+    path = os.path.join(ROOT, "profiles", "gemm_bwd_grouped_fused_ste_llama2-7b-q_proj_traffic.json")
     if not os.path.exists(path):
         return None
     with open(path) as f:
@@ -191,21 +193,15 @@ class Step:
         eqat.fq_linear_fwd(self.X, self.W, self.s, self.z, b, g, ws=self.ws, Y=self.Y)
         mark(2)
         eqat.fq_linear_bwd(self.X, self.W, self.s, self.z, self.dY, b, g, ws=self.ws,
-                           out=(self.dX, None, None, None))
+                           out=(self.dX, self.dW, self.ds, self.dz), w_hat_in_ws=True)
         mark(3)
-        eqat.fq_linear_bwd(self.X, self.W, self.s, self.z, self.dY, b, g, ws=self.ws,
-                           out=(None, self.dW, self.ds, self.dz))
-        mark(4)
         eqat.pack_codes(self.W, self.s, self.z, b, g, codes=self.codes, zq=self.zq)
-        mark(5)
+        mark(4)
         eqat.dq_linear_fwd(self.X, self.codes, self.zq, self.s, b, g, ws=self.ws, Y=self.Y2)
+        mark(5)
+        eqat.dq_linear_bwd_s(self.X, self.codes, self.zq, self.s, self.dY, b, g, ws=self.ws,
+                             out=(self.dX2, self.ds2), w_hat_in_ws=True)
         mark(6)
-        eqat.dq_linear_bwd_s(self.X, self.codes, self.zq, self.s, self.dY, b, g, ws=self.ws,
-                             out=(self.dX2, None))
-        mark(7)
-        eqat.dq_linear_bwd_s(self.X, self.codes, self.zq, self.s, self.dY, b, g, ws=self.ws,
-                             out=(None, self.ds2))
-        mark(8)
         if allreduce is not None:
             allreduce([self.dW, self.ds, self.dz, self.ds2])
 
@@ -291,7 +287,7 @@ def run_ours(args):
     peaks = load_peaks()
     mean = {p: sum(v) / len(v) for p, v in phase_ms.items()}
     dom_ms = mean[DOMINANT]
-    dom_flops = 2 * M * N * K
+    dom_flops = 4 * M * N * K
     achieved = dom_flops / (dom_ms * 1e-3) / 1e12
     peak = peaks["bf16_tflops_sustained"]
     init_b, pack_b = phase_bytes(M, N, K, wl.bits, wl.group)
@@ -352,7 +348,8 @@ def run_ours(args):
                    "flops_per_step": flops_step, "l2": "flushed before every step (512 MiB write)",
                    "parallelism": f"dp{world}" if world > 1 else "single-gpu",
                    "step": "+".join(PHASES)},
-        "roofline": {"bound": "tensor", "kernel": "k_gemm_tc dW-hat = dY^T X + fused straight-through epilogue",
+        "roofline": {"bound": "tensor",
+                     "kernel": "k_gemm_tc grouped backward: dY W-hat + dY^T X with the fused straight-through epilogue",
                      "achieved": round(achieved, 2), "peak": peak, "unit": "TFLOP/s",
                      "frac": round(achieved / peak, 4), "traffic": traffic,
                      "peak_kind": f"bf16 dense, sustained, {peaks['source']}"},
@@ -362,8 +359,8 @@ def run_ours(args):
             "pack_GBps": round(pack_b / (mean["pack"] * 1e-3) / 1e9, 1),
             "init_frac_hbm": round(init_b / (mean["init"] * 1e-3) / 1e9 / peaks["hbm_gbs"], 4),
             "pack_frac_hbm": round(pack_b / (mean["pack"] * 1e-3) / 1e9 / peaks["hbm_gbs"], 4),
-            "blockap_fwd_bwd_TFLOPs": round(6 * M * N * K / ((mean["fq_fwd"] + mean["fq_bwd_dx"] + mean["fq_bwd_w"]) * 1e-3) / 1e12, 2),
-            "e2e_fwd_bwd_TFLOPs": round(6 * M * N * K / ((mean["dq_fwd"] + mean["dq_bwd_dx"] + mean["dq_bwd_ds"]) * 1e-3) / 1e12, 2),
+            "blockap_fwd_bwd_TFLOPs": round(6 * M * N * K / ((mean["fq_fwd"] + mean["fq_bwd"]) * 1e-3) / 1e12, 2),
+            "e2e_fwd_bwd_TFLOPs": round(6 * M * N * K / ((mean["dq_fwd"] + mean["dq_bwd"]) * 1e-3) / 1e12, 2),
             "hbm_peak_GBps": peaks["hbm_gbs"],
         },
         "gpu_launches": sum(LAUNCHES_PER_STEP.values()) * args.steps,
@@ -371,6 +368,11 @@ def run_ours(args):
         "wall_s_timed": round(t_wall, 3),
         "e2e": e2e,
     }
+    if not args.no_initpack70b:
+        ip = initpack_70b_block(dev)
+        ip["init_frac_hbm"] = round(ip["init_GBps"] / peaks["hbm_gbs"], 4)
+        ip["pack_frac_hbm"] = round(ip["pack_GBps"] / peaks["hbm_gbs"], 4)
+        line["initpack_70b_block"] = ip
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(target_s=args.cpu_seconds)
     if dist is not None:
@@ -378,6 +380,53 @@ def run_ours(args):
         dist.destroy_process_group()
     if rank == 0:
         print(json.dumps(line), flush=True)
+
+
+def initpack_70b_block(dev, reps=5):
+    """HBM throughput of min-max init and pack over all seven linears of the
+    Llama-2-70B block (855.6 M bf16 weights, w2g64): algorithmic bytes / event time,
+    L2 flushed before each launch.  Weights are seeded N(0, 0.015) with 0.1% x10
+    outliers, drawn on the device."""
+    wl = synthetic.WORKLOADS[5]
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(1005)
+    flush = torch.empty(512 << 20, dtype=torch.uint8, device=dev)
+    t_init = t_pack = 0.0
+    b_init = b_pack = 0
+    for lin in wl.linears:
+        N, K = lin.n, lin.k
+        W = torch.randn(N, K, generator=gen, device=dev).mul_(wl.sigma)
+        idx = torch.randint(0, N * K, ((N * K) // 1000,), generator=gen, device=dev)
+        W.view(-1)[idx] *= 10.0
+        W = W.to(torch.bfloat16)
+        G = K // wl.group
+        s = torch.empty((N, G), dtype=torch.float32, device=dev)
+        z = torch.empty_like(s)
+        codes = torch.empty((N, eqat.packed_row_bytes(K, wl.bits)), dtype=torch.uint8, device=dev)
+        zq = torch.empty((N, G), dtype=torch.uint8, device=dev)
+        bi, bp = phase_bytes(1, N, K, wl.bits, wl.group)
+        for r in range(reps + 1):
+            e = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+            flush.zero_()
+            e[0].record()
+            eqat.minmax_init(W, wl.bits, wl.group, s=s, z=z)
+            e[1].record()
+            flush.zero_()
+            e[2].record()
+            eqat.pack_codes(W, s, z, wl.bits, wl.group, codes=codes, zq=zq)
+            e[3].record()
+            torch.cuda.synchronize()
+            if r:  # first round is warm-up
+                t_init += e[0].elapsed_time(e[1]) / reps
+                t_pack += e[2].elapsed_time(e[3]) / reps
+        b_init += bi
+        b_pack += bp
+        del W, s, z, codes, zq
+    return {"workload": wl.name + " (init+pack of all 7 linears, 855.6 M weights)",
+            "init_GBps": round(b_init / (t_init * 1e-3) / 1e9, 1),
+            "pack_GBps": round(b_pack / (t_pack * 1e-3) / 1e9, 1),
+            "init_ms": round(t_init, 4), "pack_ms": round(t_pack, 4),
+            "init_bytes": b_init, "pack_bytes": b_pack}
 
 
 # ------------------------------------------------------------------------------ oracle arm
@@ -465,6 +514,7 @@ def main():
     ap.add_argument("--impl", default="eqat", choices=["eqat", "reference"])
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-initpack70b", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)  # timing rule: at least 3 untimed warm-up steps

@@ -142,11 +142,15 @@ eqat_status eqat_fq_linear_fwd(const void *X, const void *W, int dt, const float
  *   dz = sum_group (dY^T X) s (mask - 1)            [N,G], fp32       (nullable)
  * with u, code, mask, zr as in eqat_fake_quant.  dY^T X is formed in fp32 on
  * chip and never stored; the mask, ds and dz reductions run in the epilogue of
- * that contraction. */
+ * that contraction.  In EQAT_BF16 mode both contractions run in one grouped
+ * persistent launch.  w_hat_in_ws != 0 promises that ws already holds W_hat for
+ * these (W, s, z, bits, group), as eqat_fq_linear_fwd leaves it on the same
+ * stream, and skips the quantizer prepass (training: forward, then backward with
+ * the same workspace). */
 eqat_status eqat_fq_linear_bwd(const void *X, const void *W, int dt, const float *s,
                                const float *z, const void *dY, void *dX, void *dW, float *ds,
                                float *dz, int64_t M, int64_t N, int64_t K, int bits, int group,
-                               void *ws, size_t ws_bytes, eqat_stream_t stream);
+                               void *ws, size_t ws_bytes, int w_hat_in_ws, eqat_stream_t stream);
 
 /* a8. E2E-QP forward on frozen codes (modelfoundations Phase 2: only
  * dequantization in the graph): Y = X ((W_q - zq) s)^T. */
@@ -156,11 +160,12 @@ eqat_status eqat_dq_linear_fwd(const void *X, int dt, const uint8_t *codes, cons
 
 /* a9. E2E-QP backward, scales only (modelfoundations Phase 2; zhaoyang97 notes,
  * E2E-QP: dW-hat/ds = w_q - z, no straight-through estimator):
- *   dX = dY W_hat (nullable),  ds = sum_group (dY^T X) (W_q - zq). */
+ *   dX = dY W_hat (nullable),  ds = sum_group (dY^T X) (W_q - zq).
+ * w_hat_in_ws as for eqat_fq_linear_bwd (ws holds W_hat from eqat_dq_linear_fwd). */
 eqat_status eqat_dq_linear_bwd_s(const void *X, int dt, const uint8_t *codes, const uint8_t *zq,
                                  const float *s, const void *dY, void *dX, float *ds, int64_t M,
                                  int64_t N, int64_t K, int bits, int group, void *ws,
-                                 size_t ws_bytes, eqat_stream_t stream);
+                                 size_t ws_bytes, int w_hat_in_ws, eqat_stream_t stream);
 
 /* Block-AP forward (as eqat_fq_linear_fwd) that allocates nothing and takes no
  * workspace: the paper has no counterpart; this entry point exists for callers of

@@ -98,16 +98,16 @@ def test_other_entry_points_argument_errors(lib):
     assert lib.eqat_pack_codes(P(FAKE), 1, P(FAKE), P(FAKE), 16, 64, 6, 64, P(FAKE), P(FAKE), st) == UNSUP
     assert lib.eqat_dequant_codes(P(FAKE), P(FAKE), P(FAKE), 16, 64, 2, 64, P(FAKE), 2, st) == DTYPE
     assert lib.eqat_fq_linear_bwd(P(FAKE), P(FAKE), 1, P(FAKE), P(FAKE), P(0), P(FAKE), P(0), P(0), P(0),
-                                  16, 16, 64, 2, 64, P(FAKE), 1 << 20, st) == NULL
+                                  16, 16, 64, 2, 64, P(FAKE), 1 << 20, 0, st) == NULL
     # nothing requested -> nothing to do
     assert lib.eqat_fq_linear_bwd(P(FAKE), P(FAKE), 1, P(FAKE), P(FAKE), P(FAKE), P(0), P(0), P(0), P(0),
-                                  16, 16, 64, 2, 64, P(0), 0, st) == OK
+                                  16, 16, 64, 2, 64, P(0), 0, 0, st) == OK
     assert lib.eqat_fq_linear_bwd(P(FAKE), P(FAKE), 1, P(FAKE), P(FAKE), P(FAKE), P(FAKE), P(0), P(0), P(0),
-                                  16, 16, 64, 2, 64, P(FAKE), 10, st) == WS
+                                  16, 16, 64, 2, 64, P(FAKE), 10, 1, st) == WS
     assert lib.eqat_dq_linear_fwd(P(FAKE), 1, P(FAKE), P(FAKE), P(FAKE), P(FAKE), 16, 16, 64, 3, 128,
                                   P(FAKE), 1 << 20, st) == SHAPE
     assert lib.eqat_dq_linear_bwd_s(P(FAKE), 1, P(FAKE), P(FAKE), P(FAKE), P(FAKE), P(0), P(0),
-                                    16, 16, 64, 2, 64, P(0), 0, st) == OK
+                                    16, 16, 64, 2, 64, P(0), 0, 0, st) == OK
     assert lib.eqat_selftest_bounded_wait(10, st) == SHAPE
 
 

@@ -101,10 +101,13 @@ def test_fake_quant_and_pack_bit_exact(orc, dtype, trained, bits, g):
         assert_bits_equal(to_np(dq), dq_ref if odt == torch.float32 else bf16_round(dq_ref), "dequant")
 
 
-def check_fq(orc, M, N, K, bits, g, dtype, seed, trained):
+def check_fq(orc, M, N, K, bits, g, dtype, seed, trained, reuse=False):
     dev, Xn, Wn, dYn, s, z = inputs(M, N, K, bits, g, dtype, seed, trained, orc)
-    Y = eqat.fq_linear_fwd(dev["X"], dev["W"], dev["s"], dev["z"], bits, g)
-    dX, dW, ds, dz = eqat.fq_linear_bwd(dev["X"], dev["W"], dev["s"], dev["z"], dev["dY"], bits, g)
+    tdt = torch.bfloat16 if dtype == "bf16" else torch.float32
+    ws = eqat.workspace(M, N, K, bits, g, tdt) if reuse else None
+    Y = eqat.fq_linear_fwd(dev["X"], dev["W"], dev["s"], dev["z"], bits, g, ws=ws)
+    dX, dW, ds, dz = eqat.fq_linear_bwd(dev["X"], dev["W"], dev["s"], dev["z"], dev["dY"], bits, g,
+                                        ws=ws, w_hat_in_ws=reuse)
     Y_ref = orc.fq_linear_fwd(Xn, Wn, s, z, bits, g)
     dX_ref, dW_ref, ds_ref, dz_ref = orc.fq_linear_bwd(Xn, Wn, s, z, dYn, bits, g)
     assert_close(to_np(Y), Y_ref, TOL_GEMM, "Y")
@@ -136,15 +139,17 @@ def test_fq_linear_f32(orc, shape, trained):
     check_fq(orc, M, N, K, bits, g, "f32", 200 + M, trained)
 
 
-def check_dq(orc, M, N, K, bits, g, dtype, seed):
+def check_dq(orc, M, N, K, bits, g, dtype, seed, reuse=False):
     dev, Xn, Wn, dYn, s, z = inputs(M, N, K, bits, g, dtype, seed, False, orc)
     p_ref, zq_ref = orc.pack(Wn, s, z, bits, g)
     s2, _ = synthetic.perturb_quant_params(s, z, seed)  # E2E-QP has moved the steps
     codes = torch.from_numpy(p_ref).cuda()
     zq = torch.from_numpy(zq_ref).cuda()
     s2d = torch.from_numpy(s2).cuda()
-    Y = eqat.dq_linear_fwd(dev["X"], codes, zq, s2d, bits, g)
-    dX, ds = eqat.dq_linear_bwd_s(dev["X"], codes, zq, s2d, dev["dY"], bits, g)
+    tdt = torch.bfloat16 if dtype == "bf16" else torch.float32
+    ws = eqat.workspace(M, N, K, bits, g, tdt) if reuse else None
+    Y = eqat.dq_linear_fwd(dev["X"], codes, zq, s2d, bits, g, ws=ws)
+    dX, ds = eqat.dq_linear_bwd_s(dev["X"], codes, zq, s2d, dev["dY"], bits, g, ws=ws, w_hat_in_ws=reuse)
     Y_ref = orc.dq_linear_fwd(Xn, p_ref, zq_ref, s2, bits, g)
     dX_ref, ds_ref = orc.dq_linear_bwd_s(Xn, p_ref, zq_ref, s2, dYn, bits, g)
     assert_close(to_np(Y), Y_ref, TOL_GEMM, "Y")
@@ -162,6 +167,41 @@ def test_dq_linear_bf16_tensor_core(orc, shape):
 def test_dq_linear_f32(orc, shape):
     M, N, K, bits, g = shape
     check_dq(orc, M, N, K, bits, g, "f32", 400 + M)
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+@pytest.mark.parametrize("shape", [(300, 392, 384, 2, 64), (96, 136, 256, 3, 128)], ids=lambda s: "x".join(map(str, s)))
+def test_backward_reuses_forward_w_hat(orc, shape, dtype):
+    """Training flow: the backward skips its prepass and reads the W-hat the forward
+    left in the shared workspace."""
+    M, N, K, bits, g = shape
+    check_fq(orc, M, N, K, bits, g, dtype, 500 + M, True, reuse=True)
+    check_dq(orc, M, N, K, bits, g, dtype, 600 + M, reuse=True)
+
+
+def test_backward_single_contraction_paths(orc):
+    """dX alone and the weight side alone each launch one contraction."""
+    M, N, K, bits, g = 200, 264, 320, 2, 64
+    dev, Xn, Wn, dYn, s, z = inputs(M, N, K, bits, g, "bf16", 9, True, orc)
+    dX_ref, dW_ref, ds_ref, dz_ref = orc.fq_linear_bwd(Xn, Wn, s, z, dYn, bits, g)
+    dX, dW, ds, dz = eqat.fq_linear_bwd(dev["X"], dev["W"], dev["s"], dev["z"], dev["dY"], bits, g,
+                                        need_dw=False, need_ds=False, need_dz=False)
+    assert dW is None and ds is None and dz is None
+    assert_close(to_np(dX), dX_ref, TOL_GEMM, "dX only")
+    dX, dW, ds, dz = eqat.fq_linear_bwd(dev["X"], dev["W"], dev["s"], dev["z"], dev["dY"], bits, g,
+                                        need_dx=False, need_dw=False)
+    assert dX is None and dW is None
+    assert_close(to_np(ds), ds_ref, TOL_RED, "ds only")
+    assert_close(to_np(dz), dz_ref, TOL_RED, "dz only")
+    p_ref, zq_ref = orc.pack(Wn, s, z, bits, g)
+    codes, zq = torch.from_numpy(p_ref).cuda(), torch.from_numpy(zq_ref).cuda()
+    dX2_ref, ds2_ref = orc.dq_linear_bwd_s(Xn, p_ref, zq_ref, s, dYn, bits, g)
+    dX2, ds2 = eqat.dq_linear_bwd_s(dev["X"], codes, zq, dev["s"], dev["dY"], bits, g, need_ds=False)
+    assert ds2 is None
+    assert_close(to_np(dX2), dX2_ref, TOL_GEMM, "E2E dX only")
+    dX2, ds2 = eqat.dq_linear_bwd_s(dev["X"], codes, zq, dev["s"], dev["dY"], bits, g, need_dx=False)
+    assert dX2 is None
+    assert_close(to_np(ds2), ds2_ref, TOL_RED, "E2E ds only")
 
 
 def test_persistent_tiles_wrap_accumulator_ring(orc):

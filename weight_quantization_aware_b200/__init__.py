@@ -48,9 +48,9 @@ def load_library():
         "eqat_pack_codes": [P, I, P, P, I64, I64, I, I, P, P, P],
         "eqat_dequant_codes": [P, P, P, I64, I64, I, I, P, I, P],
         "eqat_fq_linear_fwd": [P, P, I, P, P, P, I64, I64, I64, I, I, P, SZ, P],
-        "eqat_fq_linear_bwd": [P, P, I, P, P, P, P, P, P, P, I64, I64, I64, I, I, P, SZ, P],
+        "eqat_fq_linear_bwd": [P, P, I, P, P, P, P, P, P, P, I64, I64, I64, I, I, P, SZ, I, P],
         "eqat_dq_linear_fwd": [P, I, P, P, P, P, I64, I64, I64, I, I, P, SZ, P],
-        "eqat_dq_linear_bwd_s": [P, I, P, P, P, P, P, P, I64, I64, I64, I, I, P, SZ, P],
+        "eqat_dq_linear_bwd_s": [P, I, P, P, P, P, P, P, I64, I64, I64, I, I, P, SZ, I, P],
         "eqat_fq_linear_fwd_noalloc": [P, P, I, P, P, P, I64, I64, I64, I, I, P],
         "eqat_device_error": [P, P],
         "eqat_selftest_bounded_wait": [I64, P],
@@ -205,8 +205,9 @@ def fq_linear_fwd_noalloc(X, W, s, z, bits, group, Y):
 
 
 def fq_linear_bwd(X, W, s, z, dY, bits, group, need_dx=True, need_dw=True, need_ds=True, need_dz=True,
-                  ws=None, out=None):
-    """Block-AP straight-through backward: returns (dX, dW, ds, dz), None where not requested."""
+                  ws=None, out=None, w_hat_in_ws=False):
+    """Block-AP straight-through backward: returns (dX, dW, ds, dz), None where not requested.
+    w_hat_in_ws=True reuses the W-hat that fq_linear_fwd left in `ws` (same W, s, z)."""
     _req(X, "X"); _req(W, "W", X.dtype); _req(s, "s", torch.float32); _req(z, "z", torch.float32)
     _req(dY, "dY", X.dtype)
     M, K = X.shape
@@ -221,8 +222,10 @@ def fq_linear_bwd(X, W, s, z, dY, bits, group, need_dx=True, need_dw=True, need_
     else:
         dX, dW, ds, dz = out
     ws = _ws(ws, M, N, K, bits, group, X.dtype, X.device)
+    if w_hat_in_ws and ws is None:
+        raise ValueError("w_hat_in_ws needs the workspace of the forward call")
     _call("eqat_fq_linear_bwd", _p(X), _p(W), _dt(X), _p(s), _p(z), _p(dY), _p(dX), _p(dW), _p(ds), _p(dz),
-          M, N, K, bits, group, _p(ws), ws.numel(), _stream())
+          M, N, K, bits, group, _p(ws), ws.numel(), int(bool(w_hat_in_ws)), _stream())
     return dX, dW, ds, dz
 
 
@@ -238,8 +241,10 @@ def dq_linear_fwd(X, codes, zq, s, bits, group, ws=None, Y=None):
     return Y
 
 
-def dq_linear_bwd_s(X, codes, zq, s, dY, bits, group, need_dx=True, need_ds=True, ws=None, out=None):
-    """E2E-QP backward (scales only): returns (dX, ds)."""
+def dq_linear_bwd_s(X, codes, zq, s, dY, bits, group, need_dx=True, need_ds=True, ws=None, out=None,
+                    w_hat_in_ws=False):
+    """E2E-QP backward (scales only): returns (dX, ds).  w_hat_in_ws=True reuses the
+    W-hat that dq_linear_fwd left in `ws`."""
     _req(X, "X"); _req(codes, "codes", torch.uint8); _req(zq, "zq", torch.uint8); _req(s, "s", torch.float32)
     _req(dY, "dY", X.dtype)
     M, K = X.shape
@@ -250,8 +255,10 @@ def dq_linear_bwd_s(X, codes, zq, s, dY, bits, group, need_dx=True, need_ds=True
     else:
         dX, ds = out
     ws = _ws(ws, M, N, K, bits, group, X.dtype, X.device)
+    if w_hat_in_ws and ws is None:
+        raise ValueError("w_hat_in_ws needs the workspace of the forward call")
     _call("eqat_dq_linear_bwd_s", _p(X), _dt(X), _p(codes), _p(zq), _p(s), _p(dY), _p(dX), _p(ds),
-          M, N, K, bits, group, _p(ws), ws.numel(), _stream())
+          M, N, K, bits, group, _p(ws), ws.numel(), int(bool(w_hat_in_ws)), _stream())
     return dX, ds
 
 

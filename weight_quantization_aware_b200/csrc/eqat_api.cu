@@ -296,7 +296,8 @@ eqat_status eqat_fq_linear_fwd(const void *X, const void *W, int dt, const float
 
 eqat_status eqat_fq_linear_bwd(const void *X, const void *W, int dt, const float *s, const float *z,
                                const void *dY, void *dX, void *dW, float *ds, float *dz, int64_t M, int64_t N,
-                               int64_t K, int bits, int group, void *ws, size_t ws_bytes, eqat_stream_t stream) {
+                               int64_t K, int bits, int group, void *ws, size_t ws_bytes, int w_hat_in_ws,
+                               eqat_stream_t stream) {
     DeviceInfo dev;
     EQAT_TRY(check_dtype(dt));
     EQAT_TRY(check_common(M, N, K, bits, group));
@@ -317,21 +318,12 @@ eqat_status eqat_fq_linear_bwd(const void *X, const void *W, int dt, const float
     if (!dX && !want_w) return EQAT_OK;
     if (N * K > 0) EQAT_TRY(check_ws(ws, ws_bytes, N, K, dt));
     EQAT_TRY(get_device(dev));
-    if (dX && M * K > 0) {
-        if (N == 0) {
-            EQAT_CUDA(zero(dX, static_cast<size_t>(M * K) * es, st), "memset dX");
-        } else {
-            EQAT_CUDA(eqat::launch_fake_quant(W, f32, s, z, N, K, bits, group, ws, f32, nullptr, nullptr, dev, st),
-                      "fq prepass");
-            EpiArgs epi;
-            epi.kind = Epi::kStore;
-            epi.out = dX;
-            epi.ldo = K;
-            epi.out_f32 = f32;
-            EQAT_CUDA(contract(dt, Operand{dY, N, false}, Operand{ws, K, true}, M, K, N, epi, nullptr, dev, st),
-                      "dX contraction");
-        }
-    }
+
+    // Contractions to run: the weight side dY^T X (fused straight-through
+    // epilogue) and the input side dY W-hat.  On the tensor cores both run in one
+    // grouped persistent launch.
+    eqat::GemmProblem probs[2];
+    int np = 0;
     if (want_w && N * K > 0) {
         if (M == 0) {
             EQAT_CUDA(zero(dW, static_cast<size_t>(N * K) * es, st), "memset dW");
@@ -349,11 +341,33 @@ eqat_status eqat_fq_linear_bwd(const void *X, const void *W, int dt, const float
             epi.dz = dz;
             epi.bits = bits;
             epi.group = group;
-            float *scratch = f32 ? reinterpret_cast<float *>(static_cast<uint8_t *>(ws) + static_cast<size_t>(N * K) * 4)
-                                 : nullptr;
-            EQAT_CUDA(contract(dt, Operand{dY, N, true}, Operand{X, K, true}, N, K, M, epi, scratch, dev, st),
-                      "dW-hat contraction");
+            probs[np++] = eqat::GemmProblem{Operand{dY, N, true}, Operand{X, K, true}, N, K, M, epi};
         }
+    }
+    if (dX && M * K > 0) {
+        if (N == 0) {
+            EQAT_CUDA(zero(dX, static_cast<size_t>(M * K) * es, st), "memset dX");
+        } else {
+            if (!w_hat_in_ws)
+                EQAT_CUDA(eqat::launch_fake_quant(W, f32, s, z, N, K, bits, group, ws, f32, nullptr, nullptr, dev, st),
+                          "fq prepass");
+            EpiArgs epi;
+            epi.kind = Epi::kStore;
+            epi.out = dX;
+            epi.ldo = K;
+            epi.out_f32 = f32;
+            probs[np++] = eqat::GemmProblem{Operand{dY, N, false}, Operand{ws, K, true}, M, K, N, epi};
+        }
+    }
+    if (np == 0) return EQAT_OK;
+    if (!f32) {
+        EQAT_CUDA(eqat::launch_gemm_tc_group(probs, np, dev, st), "backward contractions");
+    } else {
+        float *scratch = reinterpret_cast<float *>(static_cast<uint8_t *>(ws) + static_cast<size_t>(N * K) * 4);
+        for (int i = 0; i < np; ++i)
+            EQAT_CUDA(eqat::launch_gemm_f32(probs[i].A, probs[i].B, probs[i].GM, probs[i].GN, probs[i].GK,
+                                            probs[i].epi, scratch, dev, st),
+                      "backward contraction (fp32)");
     }
     return EQAT_OK;
 }
@@ -392,7 +406,7 @@ eqat_status eqat_dq_linear_fwd(const void *X, int dt, const uint8_t *codes, cons
 
 eqat_status eqat_dq_linear_bwd_s(const void *X, int dt, const uint8_t *codes, const uint8_t *zq, const float *s,
                                  const void *dY, void *dX, float *ds, int64_t M, int64_t N, int64_t K, int bits,
-                                 int group, void *ws, size_t ws_bytes, eqat_stream_t stream) {
+                                 int group, void *ws, size_t ws_bytes, int w_hat_in_ws, eqat_stream_t stream) {
     DeviceInfo dev;
     EQAT_TRY(check_dtype(dt));
     EQAT_TRY(check_common(M, N, K, bits, group));
@@ -409,20 +423,9 @@ eqat_status eqat_dq_linear_bwd_s(const void *X, int dt, const uint8_t *codes, co
     if (!dX && !ds) return EQAT_OK;
     if (N * K > 0) EQAT_TRY(check_ws(ws, ws_bytes, N, K, dt));
     EQAT_TRY(get_device(dev));
-    if (dX && M * K > 0) {
-        if (N == 0) {
-            EQAT_CUDA(zero(dX, static_cast<size_t>(M * K) * esize(dt), st), "memset dX");
-        } else {
-            EQAT_CUDA(eqat::launch_dequant(codes, zq, s, N, K, bits, group, ws, f32, dev, st), "dequant prepass");
-            EpiArgs epi;
-            epi.kind = Epi::kStore;
-            epi.out = dX;
-            epi.ldo = K;
-            epi.out_f32 = f32;
-            EQAT_CUDA(contract(dt, Operand{dY, N, false}, Operand{ws, K, true}, M, K, N, epi, nullptr, dev, st),
-                      "dX contraction");
-        }
-    }
+
+    eqat::GemmProblem probs[2];
+    int np = 0;
     if (ds && ng > 0) {
         if (M == 0) {
             EQAT_CUDA(zero(ds, static_cast<size_t>(ng) * 4, st), "memset ds");
@@ -434,11 +437,32 @@ eqat_status eqat_dq_linear_bwd_s(const void *X, int dt, const uint8_t *codes, co
             epi.ds = ds;
             epi.bits = bits;
             epi.group = group;
-            float *scratch = f32 ? reinterpret_cast<float *>(static_cast<uint8_t *>(ws) + static_cast<size_t>(N * K) * 4)
-                                 : nullptr;
-            EQAT_CUDA(contract(dt, Operand{dY, N, true}, Operand{X, K, true}, N, K, M, epi, scratch, dev, st),
-                      "dW-hat contraction (E2E)");
+            probs[np++] = eqat::GemmProblem{Operand{dY, N, true}, Operand{X, K, true}, N, K, M, epi};
         }
+    }
+    if (dX && M * K > 0) {
+        if (N == 0) {
+            EQAT_CUDA(zero(dX, static_cast<size_t>(M * K) * esize(dt), st), "memset dX");
+        } else {
+            if (!w_hat_in_ws)
+                EQAT_CUDA(eqat::launch_dequant(codes, zq, s, N, K, bits, group, ws, f32, dev, st), "dequant prepass");
+            EpiArgs epi;
+            epi.kind = Epi::kStore;
+            epi.out = dX;
+            epi.ldo = K;
+            epi.out_f32 = f32;
+            probs[np++] = eqat::GemmProblem{Operand{dY, N, false}, Operand{ws, K, true}, M, K, N, epi};
+        }
+    }
+    if (np == 0) return EQAT_OK;
+    if (!f32) {
+        EQAT_CUDA(eqat::launch_gemm_tc_group(probs, np, dev, st), "E2E backward contractions");
+    } else {
+        float *scratch = reinterpret_cast<float *>(static_cast<uint8_t *>(ws) + static_cast<size_t>(N * K) * 4);
+        for (int i = 0; i < np; ++i)
+            EQAT_CUDA(eqat::launch_gemm_f32(probs[i].A, probs[i].B, probs[i].GM, probs[i].GN, probs[i].GK,
+                                            probs[i].epi, scratch, dev, st),
+                      "E2E backward contraction (fp32)");
     }
     return EQAT_OK;
 }

@@ -53,9 +53,12 @@ constexpr int MN_BOX_BYTES = MN_BOX * 2 * BK;  // 64 columns x 64 k-rows of bf16
 constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + 256;
 constexpr uint64_t kWaitLimitNs = 4000000000ull;  // 4 s: far above any legitimate wait
 
-struct KParams {
+// One contraction of a grouped launch.  Tiles of problem 0 come first in the
+// global tile order, then those of problem 1.
+struct Prob {
     int GM, GN, GK;
-    int tiles_m, tiles_n, num_tiles, m_fast;
+    int tiles_m, tiles_n, tile_begin, m_fast;
+    int a_mn, b_mn;  // operand majorness (1 = MN-major)
     // epilogue
     void *out;
     int64_t ldo;
@@ -69,6 +72,12 @@ struct KParams {
     const uint8_t *zq;
     int group;
     float Q;
+};
+
+struct KParams {
+    Prob pr[2];
+    int nprob;
+    int total_tiles;
     int *err;
     uint64_t wait_limit_ns;
 };
@@ -83,25 +92,32 @@ struct SharedCtl {
     int abort_flag;
 };
 
-__device__ __forceinline__ void tile_coords(const KParams &p, int t, int &tm, int &tn) {
-    if (p.m_fast) {
-        tm = t % p.tiles_m;
-        tn = t / p.tiles_m;
+// Problem index and tile coordinates of global tile t.
+__device__ __forceinline__ int tile_coords(const KParams &p, int t, int &tm, int &tn) {
+    const int pi = (p.nprob > 1 && t >= p.pr[1].tile_begin) ? 1 : 0;
+    const int lt = t - (pi ? p.pr[1].tile_begin : 0);
+    const int tiles_m = pi ? p.pr[1].tiles_m : p.pr[0].tiles_m;
+    const int tiles_n = pi ? p.pr[1].tiles_n : p.pr[0].tiles_n;
+    const int m_fast = pi ? p.pr[1].m_fast : p.pr[0].m_fast;
+    if (m_fast) {
+        tm = lt % tiles_m;
+        tn = lt / tiles_m;
     } else {
-        tn = t % p.tiles_n;
-        tm = t / p.tiles_n;
+        tn = lt % tiles_n;
+        tm = lt / tiles_n;
     }
+    return pi;
 }
 
 // Epilogue chunk: 32 consecutive accumulator columns of one row.
-template <int EPI, int BITS, bool W_F32>
+template <int EPI, int BITS>
 struct Epilogue;
 
 // D -> bf16 output.
-template <int BITS, bool W_F32>
-struct Epilogue<0, BITS, W_F32> {
+template <int BITS>
+struct Epilogue<0, BITS> {
     float acc_s = 0.0f, acc_z = 0.0f;
-    __device__ __forceinline__ void chunk(const KParams &p, int row, int col, const float (&v)[32]) {
+    __device__ __forceinline__ void chunk(const Prob &p, int row, int col, const float (&v)[32]) {
         if (row >= p.GM) return;
         __nv_bfloat16 *out = static_cast<__nv_bfloat16 *>(p.out) + static_cast<int64_t>(row) * p.ldo + col;
         if (col + 32 <= p.GN) {
@@ -123,11 +139,12 @@ struct Epilogue<0, BITS, W_F32> {
     }
 };
 
-// Block-AP straight-through: D is dW-hat[N, K]; row = n, col = k.
-template <int BITS, bool W_F32>
-struct Epilogue<1, BITS, W_F32> {
+// Block-AP straight-through: D is dW-hat[N, K] (bf16 W); row = n, col = k.
+//   dW = D * mask,  ds += D ((code - zr) - mask * u),  dz = -s * sum_{clamped} D.
+template <int BITS>
+struct Epilogue<1, BITS> {
     float acc_s = 0.0f, acc_z = 0.0f;
-    __device__ __forceinline__ void chunk(const KParams &p, int row, int col, const float (&v)[32]) {
+    __device__ __forceinline__ void chunk(const Prob &p, int row, int col, const float (&v)[32]) {
         if (row >= p.GM || col >= p.GN) return;
         const int64_t K = p.GN;
         const int64_t G = K / p.group;
@@ -139,10 +156,7 @@ struct Epilogue<1, BITS, W_F32> {
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
             float w[8];
-            if (W_F32)
-                load8<float>(static_cast<const float *>(p.W) + e0 + 8 * q, w);
-            else
-                load8<__nv_bfloat16>(static_cast<const __nv_bfloat16 *>(p.W) + e0 + 8 * q, w);
+            load8<__nv_bfloat16>(static_cast<const __nv_bfloat16 *>(p.W) + e0 + 8 * q, w);
 #pragma unroll
             for (int j = 0; j < 8; ++j) {
                 const float d = v[8 * q + j];
@@ -154,17 +168,10 @@ struct Epilogue<1, BITS, W_F32> {
             }
         }
         if (p.dW) {
-            if (W_F32) {
-                float *o = static_cast<float *>(p.dW) + e0;
+            __nv_bfloat16 *o = static_cast<__nv_bfloat16 *>(p.dW) + e0;
 #pragma unroll
-                for (int q = 0; q < 4; ++q)
-                    store8<float>(o + 8 * q, *reinterpret_cast<const float(*)[8]>(&dwv[8 * q]));
-            } else {
-                __nv_bfloat16 *o = static_cast<__nv_bfloat16 *>(p.dW) + e0;
-#pragma unroll
-                for (int q = 0; q < 4; ++q)
-                    store8<__nv_bfloat16>(o + 8 * q, *reinterpret_cast<const float(*)[8]>(&dwv[8 * q]));
-            }
+            for (int q = 0; q < 4; ++q)
+                store8<__nv_bfloat16>(o + 8 * q, *reinterpret_cast<const float(*)[8]>(&dwv[8 * q]));
         }
         if (((col + 32) % p.group) == 0) {
             if (p.ds) p.ds[gi] = acc_s;
@@ -176,10 +183,10 @@ struct Epilogue<1, BITS, W_F32> {
 };
 
 // E2E-QP: D is dW-hat[N, K]; ds = sum_group D * (W_q - zq).
-template <int BITS, bool W_F32>
-struct Epilogue<2, BITS, W_F32> {
+template <int BITS>
+struct Epilogue<2, BITS> {
     float acc_s = 0.0f, acc_z = 0.0f;
-    __device__ __forceinline__ void chunk(const KParams &p, int row, int col, const float (&v)[32]) {
+    __device__ __forceinline__ void chunk(const Prob &p, int row, int col, const float (&v)[32]) {
         if (row >= p.GM || col >= p.GN) return;
         const int64_t K = p.GN;
         const int64_t G = K / p.group;
@@ -213,9 +220,26 @@ struct Epilogue<2, BITS, W_F32> {
     }
 };
 
-template <bool A_MN, bool B_MN, int EPI, int BITS, bool W_F32, int EPI_WARPS>
+// Drains one accumulator (this warp's 32 rows, columns [c_begin, c_end)) through
+// the epilogue of kind EPI.
+template <int EPI, int BITS>
+__device__ __forceinline__ void drain_accumulator(const Prob &pr, uint32_t taddr, int row, int col0,
+                                                  int c_begin, int c_end) {
+    Epilogue<EPI, BITS> epi;
+#pragma unroll 1
+    for (int c0 = c_begin; c0 < c_end; c0 += 32) {
+        float v[32];
+        tmem_ld_32cols(taddr + c0, v);
+        epi.chunk(pr, row, col0 + c0, v);
+    }
+}
+
+// Persistent grouped GEMM: problem 0 uses epilogue EPI0, problem 1 (if any)
+// EPI1; operand majorness is a per-problem runtime property.
+template <int EPI0, int EPI1, int BITS, int EPI_WARPS>
 __global__ void __launch_bounds__((4 + EPI_WARPS) * 32, 1)
-    k_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+    k_gemm_tc(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUtensorMap tmB0,
+              const __grid_constant__ CUtensorMap tmA1, const __grid_constant__ CUtensorMap tmB1,
               const KParams p) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -237,8 +261,12 @@ __global__ void __launch_bounds__((4 + EPI_WARPS) * 32, 1)
         mbar_init(&ctl->drain, 1);
         ctl->abort_flag = 0;
         fence_mbarrier_init();
-        tma_prefetch_desc(&tmA);
-        tma_prefetch_desc(&tmB);
+        tma_prefetch_desc(&tmA0);
+        tma_prefetch_desc(&tmB0);
+        if (p.nprob > 1) {
+            tma_prefetch_desc(&tmA1);
+            tma_prefetch_desc(&tmB1);
+        }
     }
     if (warp == 2) {
         tmem_alloc(&ctl->tmem_base, TMEM_COLS);
@@ -249,18 +277,22 @@ __global__ void __launch_bounds__((4 + EPI_WARPS) * 32, 1)
     tc_fence_after();
     const uint32_t tmem_base = ctl->tmem_base;
     volatile int *abort_flag = &ctl->abort_flag;
-    const int nkb = (p.GK + BK - 1) / BK;
 
     if (warp == 0) {
         // ---------------------------------------------------------- TMA producer
         if (elect_one_sync()) {
             uint32_t it = 0;
-            uint32_t armed = 0;           // stages with a load issued
-            uint32_t armed_parity = 0;    // parity of the last phase armed per stage
+            uint32_t armed = 0;         // stages with a load issued
+            uint32_t armed_parity = 0;  // parity of the last phase armed per stage
             bool ok = true;
-            for (int t = blockIdx.x; ok && t < p.num_tiles; t += gridDim.x) {
+            for (int t = blockIdx.x; ok && t < p.total_tiles; t += gridDim.x) {
                 int tm, tn;
-                tile_coords(p, t, tm, tn);
+                const int pi = tile_coords(p, t, tm, tn);
+                const CUtensorMap *ma = pi ? &tmA1 : &tmA0;
+                const CUtensorMap *mb = pi ? &tmB1 : &tmB0;
+                const int a_mn = pi ? p.pr[1].a_mn : p.pr[0].a_mn;
+                const int b_mn = pi ? p.pr[1].b_mn : p.pr[0].b_mn;
+                const int nkb = ((pi ? p.pr[1].GK : p.pr[0].GK) + BK - 1) / BK;
                 const int m0 = tm * BM, n0 = tn * BN;
                 for (int kb = 0; kb < nkb; ++kb, ++it) {
                     const int st = it % STAGES;
@@ -275,19 +307,19 @@ __global__ void __launch_bounds__((4 + EPI_WARPS) * 32, 1)
                     armed |= 1u << st;
                     armed_parity = (armed_parity & ~(1u << st)) | (ph << st);
                     const int k0 = kb * BK;
-                    if (A_MN) {
+                    if (a_mn) {
 #pragma unroll
                         for (int b = 0; b < BM / MN_BOX; ++b)
-                            tma_load_2d(sa + b * MN_BOX_BYTES, &tmA, &ctl->full[st], m0 + b * MN_BOX, k0);
+                            tma_load_2d(sa + b * MN_BOX_BYTES, ma, &ctl->full[st], m0 + b * MN_BOX, k0);
                     } else {
-                        tma_load_2d(sa, &tmA, &ctl->full[st], k0, m0);
+                        tma_load_2d(sa, ma, &ctl->full[st], k0, m0);
                     }
-                    if (B_MN) {
+                    if (b_mn) {
 #pragma unroll
                         for (int b = 0; b < BN / MN_BOX; ++b)
-                            tma_load_2d(sb + b * MN_BOX_BYTES, &tmB, &ctl->full[st], n0 + b * MN_BOX, k0);
+                            tma_load_2d(sb + b * MN_BOX_BYTES, mb, &ctl->full[st], n0 + b * MN_BOX, k0);
                     } else {
-                        tma_load_2d(sb, &tmB, &ctl->full[st], k0, n0);
+                        tma_load_2d(sb, mb, &ctl->full[st], k0, n0);
                     }
                 }
             }
@@ -307,12 +339,22 @@ __global__ void __launch_bounds__((4 + EPI_WARPS) * 32, 1)
     } else if (warp == 1) {
         // ---------------------------------------------------------- MMA issuer
         if (elect_one_sync()) {
-            constexpr uint32_t idesc = idesc_bf16_f32(BM, BN, A_MN, B_MN);
             uint32_t it = 0;
             uint32_t local = 0;
             bool ok = true;
             bool issued = false;
-            for (int t = blockIdx.x; ok && t < p.num_tiles; t += gridDim.x, ++local) {
+            for (int t = blockIdx.x; ok && t < p.total_tiles; t += gridDim.x, ++local) {
+                int tm, tn;
+                const int pi = tile_coords(p, t, tm, tn);
+                const int a_mn = pi ? p.pr[1].a_mn : p.pr[0].a_mn;
+                const int b_mn = pi ? p.pr[1].b_mn : p.pr[0].b_mn;
+                const int nkb = ((pi ? p.pr[1].GK : p.pr[0].GK) + BK - 1) / BK;
+                const uint32_t idesc = idesc_bf16_f32(BM, BN, a_mn != 0, b_mn != 0);
+                // K-major: advance 16 elements (32 B) inside the 128 B swizzle row,
+                // LBO unused (16), SBO = 8 rows x 128 B.  MN-major: advance 16 k-rows
+                // (2 KB), LBO = next 64-wide MN box, SBO = 8 k-rows x 128 B.
+                const uint32_t a_step = a_mn ? UK * 128 : UK * 2, a_lbo = a_mn ? MN_BOX_BYTES : 16;
+                const uint32_t b_step = b_mn ? UK * 128 : UK * 2, b_lbo = b_mn ? MN_BOX_BYTES : 16;
                 const uint32_t acc = local & 1u;
                 const uint32_t aph = (local >> 1) & 1u;
                 if (!mbar_wait_bounded(&ctl->acc_empty[acc], aph ^ 1u, abort_flag, p.err, p.wait_limit_ns)) {
@@ -333,10 +375,8 @@ __global__ void __launch_bounds__((4 + EPI_WARPS) * 32, 1)
                     const uint32_t sb = sa + A_BYTES;
 #pragma unroll
                     for (int kk = 0; kk < BK / UK; ++kk) {
-                        const uint64_t ad = A_MN ? smem_desc_sw128(sa + kk * (UK * 128), MN_BOX_BYTES, 1024)
-                                                 : smem_desc_sw128(sa + kk * (UK * 2), 16, 1024);
-                        const uint64_t bd = B_MN ? smem_desc_sw128(sb + kk * (UK * 128), MN_BOX_BYTES, 1024)
-                                                 : smem_desc_sw128(sb + kk * (UK * 2), 16, 1024);
+                        const uint64_t ad = smem_desc_sw128(sa + kk * a_step, a_lbo, 1024);
+                        const uint64_t bd = smem_desc_sw128(sb + kk * b_step, b_lbo, 1024);
                         tc_mma_f16(d_tmem, ad, bd, idesc, (kb > 0 || kk > 0) ? 1u : 0u);
                     }
                     issued = true;
@@ -358,28 +398,26 @@ __global__ void __launch_bounds__((4 + EPI_WARPS) * 32, 1)
     } else if (warp >= 4) {
         // ---------------------------------------------------------- epilogue
         const int ew = warp - 4;
-        const int quad = warp & 3;                   // tensor-memory lane quadrant
-        const int half = ew >> 2;                    // column slice of the accumulator
+        const int quad = warp & 3;  // tensor-memory lane quadrant of this warp
+        const int half = ew >> 2;   // column slice of the accumulator
         constexpr int SLICES = EPI_WARPS / 4;
         constexpr int COLS = ACC_COLS / SLICES;
         uint32_t local = 0;
-        for (int t = blockIdx.x; t < p.num_tiles; t += gridDim.x, ++local) {
+        for (int t = blockIdx.x; t < p.total_tiles; t += gridDim.x, ++local) {
             const uint32_t acc = local & 1u;
             const uint32_t aph = (local >> 1) & 1u;
-            // Every lane waits; the warp leaves together (tcgen05.ld below is .sync.aligned).
+            // Every lane waits; the warp leaves together (tcgen05.ld is .sync.aligned).
             const bool ok = mbar_wait_bounded(&ctl->acc_full[acc], aph, abort_flag, p.err, p.wait_limit_ns);
             if (!__all_sync(0xffffffffu, ok)) break;
             tc_fence_after();
             int tm, tn;
-            tile_coords(p, t, tm, tn);
+            const int pi = tile_coords(p, t, tm, tn);
             const int row = tm * BM + quad * 32 + lane;
-            Epilogue<EPI, BITS, W_F32> epi;
-#pragma unroll 1
-            for (int c0 = half * COLS; c0 < (half + 1) * COLS; c0 += 32) {
-                float v[32];
-                tmem_ld_32cols(tmem_base + acc * ACC_COLS + c0 + ((quad * 32) << 16), v);
-                epi.chunk(p, row, tn * BN + c0, v);
-            }
+            const uint32_t taddr = tmem_base + acc * ACC_COLS + ((quad * 32) << 16);
+            if (pi == 0)
+                drain_accumulator<EPI0, BITS>(p.pr[0], taddr, row, tn * BN, half * COLS, (half + 1) * COLS);
+            else
+                drain_accumulator<EPI1, BITS>(p.pr[1], taddr, row, tn * BN, half * COLS, (half + 1) * COLS);
             tc_fence_before();
             mbar_arrive(&ctl->acc_empty[acc]);
         }
@@ -434,10 +472,12 @@ cudaError_t make_map(CUtensorMap &map, const Operand &op, int64_t rows, int64_t 
     return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 
-template <bool A_MN, bool B_MN, int EPI, int BITS, bool W_F32, int EPI_WARPS>
-cudaError_t launch_variant(const CUtensorMap &ma, const CUtensorMap &mb, const KParams &p, int grid,
-                           int dev_id, cudaStream_t st) {
-    auto kern = k_gemm_tc<A_MN, B_MN, EPI, BITS, W_F32, EPI_WARPS>;
+constexpr int kEpiWarps = 8;
+
+template <int EPI0, int EPI1, int BITS>
+cudaError_t launch_variant(const CUtensorMap (&maps)[4], const KParams &p, int grid, int dev_id,
+                           cudaStream_t st) {
+    auto kern = k_gemm_tc<EPI0, EPI1, BITS, kEpiWarps>;
     // The shared-memory opt-in is a per-device function attribute; setting it
     // twice from racing threads is harmless.
     static std::atomic<uint64_t> done{0};
@@ -447,7 +487,7 @@ cudaError_t launch_variant(const CUtensorMap &ma, const CUtensorMap &mb, const K
         if (e != cudaSuccess) return e;
         done.fetch_or(bit);
     }
-    kern<<<grid, (4 + EPI_WARPS) * 32, SMEM_BYTES, st>>>(ma, mb, p);
+    kern<<<grid, (4 + kEpiWarps) * 32, SMEM_BYTES, st>>>(maps[0], maps[1], maps[2], maps[3], p);
     return cudaGetLastError();
 }
 
@@ -457,66 +497,95 @@ int *device_error_ptr() {
     return ptr;
 }
 
+cudaError_t fill_prob(Prob &q, const GemmProblem &g, int tile_begin, CUtensorMap &ma, CUtensorMap &mb) {
+    const int64_t GM = g.GM, GN = g.GN, GK = g.GK;
+    if (GM <= 0 || GN <= 0 || GK <= 0) return cudaErrorInvalidValue;
+    if (GM > INT32_MAX - BM || GN > INT32_MAX - BN || GK > INT32_MAX - BK) return cudaErrorInvalidValue;
+    cudaError_t e;
+    if ((e = make_map(ma, g.A, GM, GK, BM)) != cudaSuccess) return e;
+    if ((e = make_map(mb, g.B, GN, GK, BN)) != cudaSuccess) return e;
+    q = Prob{};
+    q.GM = static_cast<int>(GM);
+    q.GN = static_cast<int>(GN);
+    q.GK = static_cast<int>(GK);
+    q.tiles_m = static_cast<int>((GM + BM - 1) / BM);
+    q.tiles_n = static_cast<int>((GN + BN - 1) / BN);
+    q.tile_begin = tile_begin;
+    // Consecutive CTAs share the operand whose tiles are the larger total, so
+    // that the smaller one stays hot in L2 while the larger streams once.
+    q.m_fast = (GM <= GN) ? 1 : 0;
+    q.a_mn = g.A.mn_major ? 1 : 0;
+    q.b_mn = g.B.mn_major ? 1 : 0;
+    const EpiArgs &epi = g.epi;
+    q.out = epi.out;
+    q.ldo = epi.ldo;
+    q.W = epi.W;
+    q.s = epi.s;
+    q.z = epi.z;
+    q.dW = epi.dW;
+    q.ds = epi.ds;
+    q.dz = epi.dz;
+    q.codes = epi.codes;
+    q.zq = epi.zq;
+    q.group = epi.group;
+    q.Q = static_cast<float>((1 << epi.bits) - 1);
+    return cudaSuccess;
+}
+
 }  // namespace
 
-cudaError_t launch_gemm_tc(const Operand &A, const Operand &B, int64_t GM, int64_t GN, int64_t GK,
-                           const EpiArgs &epi, const DeviceInfo &dev, cudaStream_t st) {
-    if (GM <= 0 || GN <= 0 || GK <= 0) return cudaSuccess;
-    if (GM > INT32_MAX - BM || GN > INT32_MAX - BN || GK > INT32_MAX - BK) return cudaErrorInvalidValue;
+cudaError_t launch_gemm_tc_group(const GemmProblem *probs, int nprob, const DeviceInfo &dev,
+                                 cudaStream_t st) {
+    if (nprob < 1 || nprob > 2) return cudaErrorInvalidValue;
+    for (int i = 0; i < nprob; ++i) {
+        const EpiArgs &e = probs[i].epi;
+        if (e.kind == Epi::kStore && e.out_f32) return cudaErrorInvalidValue;
+        if (e.kind == Epi::kFqGrad && e.w_f32) return cudaErrorInvalidValue;
+        if (i == 1 && e.kind != Epi::kStore) return cudaErrorInvalidValue;
+    }
     cudaError_t e = get_encode();
     if (e != cudaSuccess) return e;
-    CUtensorMap ma, mb;
-    if ((e = make_map(ma, A, GM, GK, BM)) != cudaSuccess) return e;
-    if ((e = make_map(mb, B, GN, GK, BN)) != cudaSuccess) return e;
-    int *err = device_error_ptr();
-    if (!err) return cudaErrorInvalidSymbol;
-
+    CUtensorMap maps[4];
     KParams p{};
-    p.GM = static_cast<int>(GM);
-    p.GN = static_cast<int>(GN);
-    p.GK = static_cast<int>(GK);
-    p.tiles_m = static_cast<int>((GM + BM - 1) / BM);
-    p.tiles_n = static_cast<int>((GN + BN - 1) / BN);
-    p.num_tiles = p.tiles_m * p.tiles_n;
-    // Consecutive CTAs share the operand whose tiles are the larger total, so
-    // that one stays hot in L2 while the other streams once.
-    p.m_fast = (GM * GK <= GN * GK) ? 1 : 0;
-    p.out = epi.out;
-    p.ldo = epi.ldo;
-    p.W = epi.W;
-    p.s = epi.s;
-    p.z = epi.z;
-    p.dW = epi.dW;
-    p.ds = epi.ds;
-    p.dz = epi.dz;
-    p.codes = epi.codes;
-    p.zq = epi.zq;
-    p.group = epi.group;
-    p.Q = static_cast<float>((1 << epi.bits) - 1);
-    p.err = err;
+    int tiles = 0;
+    for (int i = 0; i < nprob; ++i) {
+        if ((e = fill_prob(p.pr[i], probs[i], tiles, maps[2 * i], maps[2 * i + 1])) != cudaSuccess) return e;
+        const int64_t t = static_cast<int64_t>(p.pr[i].tiles_m) * p.pr[i].tiles_n;
+        if (tiles + t > INT32_MAX) return cudaErrorInvalidValue;
+        tiles += static_cast<int>(t);
+    }
+    if (nprob == 1) {  // unused slots still travel as kernel parameters
+        maps[2] = maps[0];
+        maps[3] = maps[1];
+    }
+    p.nprob = nprob;
+    p.total_tiles = tiles;
+    p.err = device_error_ptr();
+    if (!p.err) return cudaErrorInvalidSymbol;
     p.wait_limit_ns = kWaitLimitNs;
-    const int grid = std::min(p.num_tiles, dev.sm_count);
-
-    const bool am = A.mn_major, bm = B.mn_major;
-    switch (epi.kind) {
+    const int grid = std::min(tiles, dev.sm_count);
+    switch (probs[0].epi.kind) {
         case Epi::kStore:
-            if (epi.out_f32) return cudaErrorInvalidValue;
-            if (!am && !bm) return launch_variant<false, false, 0, 2, false, 4>(ma, mb, p, grid, dev.device, st);
-            if (!am && bm) return launch_variant<false, true, 0, 2, false, 4>(ma, mb, p, grid, dev.device, st);
-            return cudaErrorInvalidValue;
+            if (nprob > 1) return cudaErrorInvalidValue;  // two plain contractions: launch separately
+            return launch_variant<0, 0, 2>(maps, p, grid, dev.device, st);
         case Epi::kFqGrad:
-            if (!(am && bm) || epi.w_f32) return cudaErrorInvalidValue;
-            return launch_variant<true, true, 1, 2, false, 8>(ma, mb, p, grid, dev.device, st);
+            return launch_variant<1, 0, 2>(maps, p, grid, dev.device, st);
         case Epi::kE2eDs:
-            if (!(am && bm)) return cudaErrorInvalidValue;
-            switch (epi.bits) {
-                case 2: return launch_variant<true, true, 2, 2, false, 4>(ma, mb, p, grid, dev.device, st);
-                case 3: return launch_variant<true, true, 2, 3, false, 4>(ma, mb, p, grid, dev.device, st);
-                case 4: return launch_variant<true, true, 2, 4, false, 4>(ma, mb, p, grid, dev.device, st);
+            switch (probs[0].epi.bits) {
+                case 2: return launch_variant<2, 0, 2>(maps, p, grid, dev.device, st);
+                case 3: return launch_variant<2, 0, 3>(maps, p, grid, dev.device, st);
+                case 4: return launch_variant<2, 0, 4>(maps, p, grid, dev.device, st);
                 default: return cudaErrorInvalidValue;
             }
     }
     return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_gemm_tc(const Operand &A, const Operand &B, int64_t GM, int64_t GN, int64_t GK,
+                           const EpiArgs &epi, const DeviceInfo &dev, cudaStream_t st) {
+    if (GM <= 0 || GN <= 0 || GK <= 0) return cudaSuccess;
+    GemmProblem g{A, B, GM, GN, GK, epi};
+    return launch_gemm_tc_group(&g, 1, dev, st);
 }
 
 // ---------------------------------------------------------------------------- error word

@@ -69,7 +69,18 @@ struct EpiArgs {
     int group = 64;
 };
 
+struct GemmProblem {
+    Operand A;
+    Operand B;
+    int64_t GM, GN, GK;
+    EpiArgs epi;
+};
+
 // bf16 operands on tcgen05 tensor cores, fp32 accumulation in tensor memory.
+// A grouped launch runs the tiles of up to two contractions in one persistent
+// kernel (problem 0 first); problem 1, if present, must use the kStore epilogue.
+cudaError_t launch_gemm_tc_group(const GemmProblem *probs, int nprob, const DeviceInfo &dev,
+                                 cudaStream_t st);
 cudaError_t launch_gemm_tc(const Operand &A, const Operand &B, int64_t GM, int64_t GN, int64_t GK,
                            const EpiArgs &epi, const DeviceInfo &dev, cudaStream_t st);
 

@@ -32,14 +32,14 @@ inline int grid_for(int64_t work_items, const DeviceInfo &dev, int per_thread = 
 // ------------------------------------------------------------------ min-max init
 // A thread holds 8 consecutive weights of one group; TPG = G/8 threads cover a
 // group and reduce min/max with xor shuffles; UNROLL independent groups per
-// thread keep 64 bytes of loads in flight per thread.
+// thread keep 128 bytes (bf16) of loads in flight per thread.
 template <typename T, int G>
 __global__ void __launch_bounds__(kThreads) k_minmax_init(const T *__restrict__ W, int64_t n_groups,
                                                           float Q, float *__restrict__ s,
                                                           float *__restrict__ z) {
     constexpr int TPG = G / 8;
     constexpr int GPW = 32 / TPG;  // groups per warp per unrolled slot
-    constexpr int UNROLL = 4;
+    constexpr int UNROLL = 8;
     const int lane = threadIdx.x & 31;
     const int sub = lane % TPG;
     const int slot = lane / TPG;
@@ -82,39 +82,59 @@ __global__ void __launch_bounds__(kThreads) k_minmax_init(const T *__restrict__ 
 }
 
 // ------------------------------------------------------------------ fake-quant prepass
-// One thread per 8 consecutive weights (same group): code, mask and W-hat.
+// A thread handles U = 2 chunks of 8 consecutive weights (each chunk inside one
+// group) per iteration and issues both loads before any arithmetic.
+template <typename T, typename O>
+__device__ __forceinline__ void fake_quant_chunk(const float (&w)[8], float sc, float zr, float Q,
+                                                 int64_t e0, O *__restrict__ W_hat,
+                                                 uint8_t *__restrict__ code, uint8_t *__restrict__ mask) {
+    float wh[8];
+    uint32_t c_lo = 0, c_hi = 0, m_lo = 0, m_hi = 0;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+        const QuantElem q = quant_elem(w[j], sc, zr, Q);
+        wh[j] = dequant_elem(q.c, zr, sc);
+        const uint32_t cb = static_cast<uint32_t>(q.c);
+        const uint32_t mb = q.inside ? 1u : 0u;
+        if (j < 4) {
+            c_lo |= cb << (8 * j);
+            m_lo |= mb << (8 * j);
+        } else {
+            c_hi |= cb << (8 * (j - 4));
+            m_hi |= mb << (8 * (j - 4));
+        }
+    }
+    if (W_hat) store8<O>(W_hat + e0, wh);
+    if (code) *reinterpret_cast<uint2 *>(code + e0) = make_uint2(c_lo, c_hi);
+    if (mask) *reinterpret_cast<uint2 *>(mask + e0) = make_uint2(m_lo, m_hi);
+}
+
 template <typename T, typename O>
 __global__ void __launch_bounds__(kThreads)
     k_fake_quant(const T *__restrict__ W, const float *__restrict__ s, const float *__restrict__ z,
                  int64_t n_chunks, int group, float Q, O *__restrict__ W_hat,
                  uint8_t *__restrict__ code, uint8_t *__restrict__ mask) {
-    const int64_t stride = static_cast<int64_t>(gridDim.x) * kThreads;
-    for (int64_t i = static_cast<int64_t>(blockIdx.x) * kThreads + threadIdx.x; i < n_chunks;
-         i += stride) {
-        const int64_t e0 = i * 8;
-        const int64_t g = e0 / group;
-        const float sc = __ldg(s + g);
-        const float zr = rintf(__ldg(z + g));
-        float w[8], wh[8];
-        load8<T>(W + e0, w);
-        uint32_t c_lo = 0, c_hi = 0, m_lo = 0, m_hi = 0;
+    constexpr int U = 2;
+    const int64_t nthreads = static_cast<int64_t>(gridDim.x) * kThreads;
+    for (int64_t base = static_cast<int64_t>(blockIdx.x) * kThreads + threadIdx.x; base < n_chunks;
+         base += nthreads * U) {
+        float w[U][8];
+        float sc[U], zr[U];
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
-            const QuantElem q = quant_elem(w[j], sc, zr, Q);
-            wh[j] = dequant_elem(q.c, zr, sc);
-            const uint32_t cb = static_cast<uint32_t>(q.c);
-            const uint32_t mb = q.inside ? 1u : 0u;
-            if (j < 4) {
-                c_lo |= cb << (8 * j);
-                m_lo |= mb << (8 * j);
-            } else {
-                c_hi |= cb << (8 * (j - 4));
-                m_hi |= mb << (8 * (j - 4));
+        for (int u = 0; u < U; ++u) {
+            const int64_t i = base + u * nthreads;
+            if (i < n_chunks) {
+                load8<T>(W + i * 8, w[u]);
+                const int64_t g = (i * 8) / group;
+                sc[u] = __ldg(s + g);
+                zr[u] = rintf(__ldg(z + g));
             }
         }
-        if (W_hat) store8<O>(W_hat + e0, wh);
-        if (code) *reinterpret_cast<uint2 *>(code + e0) = make_uint2(c_lo, c_hi);
-        if (mask) *reinterpret_cast<uint2 *>(mask + e0) = make_uint2(m_lo, m_hi);
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const int64_t i = base + u * nthreads;
+            if (i < n_chunks) fake_quant_chunk<T, O>(w[u], sc[u], zr[u], Q, i * 8, W_hat, code, mask);
+        }
     }
 }
 
@@ -122,44 +142,68 @@ __global__ void __launch_bounds__(kThreads)
 // One thread per 16 consecutive weights (same group).  zq = clamp(round(z), 0, Q)
 // and the codes use zr := zq (z hard-rounded at pack time).  Output per thread:
 // 4 bytes (2-bit), 8 bytes (4-bit) or 16 bytes (3-bit, one code per byte).
+template <int BITS>
+__device__ __forceinline__ void pack_chunk(const float (&w)[16], float sc, float zr, float Q, int64_t e0,
+                                           uint8_t *__restrict__ codes) {
+    uint32_t c[16];
+#pragma unroll
+    for (int j = 0; j < 16; ++j) c[j] = static_cast<uint32_t>(quant_elem(w[j], sc, zr, Q).c);
+    if (BITS == 2) {
+        uint32_t word = 0;
+#pragma unroll
+        for (int j = 0; j < 16; ++j) word |= c[j] << (2 * j);
+        *reinterpret_cast<uint32_t *>(codes + e0 / 4) = word;
+    } else if (BITS == 4) {
+        uint32_t lo = 0, hi = 0;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) lo |= c[j] << (4 * j);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) hi |= c[8 + j] << (4 * j);
+        *reinterpret_cast<uint2 *>(codes + e0 / 2) = make_uint2(lo, hi);
+    } else {
+        uint4 r;
+        r.x = c[0] | (c[1] << 8) | (c[2] << 16) | (c[3] << 24);
+        r.y = c[4] | (c[5] << 8) | (c[6] << 16) | (c[7] << 24);
+        r.z = c[8] | (c[9] << 8) | (c[10] << 16) | (c[11] << 24);
+        r.w = c[12] | (c[13] << 8) | (c[14] << 16) | (c[15] << 24);
+        *reinterpret_cast<uint4 *>(codes + e0) = r;
+    }
+}
+
+// A thread handles U = 2 chunks of 16 consecutive weights (each inside one group)
+// per iteration, loads first.  zq = clamp(round(z), 0, Q) and the codes use
+// zr := zq (z hard-rounded at pack time).  Output per chunk: 4 bytes (2-bit), 8
+// bytes (4-bit) or 16 bytes (3-bit, one code per byte).
 template <typename T, int BITS>
 __global__ void __launch_bounds__(kThreads)
     k_pack(const T *__restrict__ W, const float *__restrict__ s, const float *__restrict__ z,
            int64_t n_chunks, int group, float Q, uint8_t *__restrict__ codes,
            uint8_t *__restrict__ zq) {
-    const int64_t stride = static_cast<int64_t>(gridDim.x) * kThreads;
-    for (int64_t i = static_cast<int64_t>(blockIdx.x) * kThreads + threadIdx.x; i < n_chunks;
-         i += stride) {
-        const int64_t e0 = i * 16;
-        const int64_t g = e0 / group;
-        const float sc = __ldg(s + g);
-        const float zr = fminf(fmaxf(rintf(__ldg(z + g)), 0.0f), Q);
-        if (e0 % group == 0) zq[g] = static_cast<uint8_t>(zr);
-        float w[16];
-        load8<T>(W + e0, *reinterpret_cast<float(*)[8]>(&w[0]));
-        load8<T>(W + e0 + 8, *reinterpret_cast<float(*)[8]>(&w[8]));
-        uint32_t c[16];
+    constexpr int U = 2;
+    const int64_t nthreads = static_cast<int64_t>(gridDim.x) * kThreads;
+    for (int64_t base = static_cast<int64_t>(blockIdx.x) * kThreads + threadIdx.x; base < n_chunks;
+         base += nthreads * U) {
+        float w[U][16];
+        float sc[U], zr[U];
 #pragma unroll
-        for (int j = 0; j < 16; ++j) c[j] = static_cast<uint32_t>(quant_elem(w[j], sc, zr, Q).c);
-        if (BITS == 2) {
-            uint32_t word = 0;
+        for (int u = 0; u < U; ++u) {
+            const int64_t i = base + u * nthreads;
+            if (i < n_chunks) {
+                load8<T>(W + i * 16, *reinterpret_cast<float(*)[8]>(&w[u][0]));
+                load8<T>(W + i * 16 + 8, *reinterpret_cast<float(*)[8]>(&w[u][8]));
+                const int64_t g = (i * 16) / group;
+                sc[u] = __ldg(s + g);
+                zr[u] = fminf(fmaxf(rintf(__ldg(z + g)), 0.0f), Q);
+            }
+        }
 #pragma unroll
-            for (int j = 0; j < 16; ++j) word |= c[j] << (2 * j);
-            *reinterpret_cast<uint32_t *>(codes + e0 / 4) = word;
-        } else if (BITS == 4) {
-            uint32_t lo = 0, hi = 0;
-#pragma unroll
-            for (int j = 0; j < 8; ++j) lo |= c[j] << (4 * j);
-#pragma unroll
-            for (int j = 0; j < 8; ++j) hi |= c[8 + j] << (4 * j);
-            *reinterpret_cast<uint2 *>(codes + e0 / 2) = make_uint2(lo, hi);
-        } else {
-            uint4 r;
-            r.x = c[0] | (c[1] << 8) | (c[2] << 16) | (c[3] << 24);
-            r.y = c[4] | (c[5] << 8) | (c[6] << 16) | (c[7] << 24);
-            r.z = c[8] | (c[9] << 8) | (c[10] << 16) | (c[11] << 24);
-            r.w = c[12] | (c[13] << 8) | (c[14] << 16) | (c[15] << 24);
-            *reinterpret_cast<uint4 *>(codes + e0) = r;
+        for (int u = 0; u < U; ++u) {
+            const int64_t i = base + u * nthreads;
+            if (i < n_chunks) {
+                const int64_t e0 = i * 16;
+                if (e0 % group == 0) zq[e0 / group] = static_cast<uint8_t>(zr[u]);
+                pack_chunk<BITS>(w[u], sc[u], zr[u], Q, e0, codes);
+            }
         }
     }
 }
@@ -212,7 +256,7 @@ __global__ void __launch_bounds__(kThreads)
 template <typename T>
 cudaError_t minmax_dispatch(const T *W, int64_t n_groups, int group, float Q, float *s, float *z,
                             const DeviceInfo &dev, cudaStream_t st) {
-    const int grid = grid_for(n_groups * group, dev, 8 * 4);
+    const int grid = grid_for(n_groups * group, dev, 8 * 8);
     switch (group) {
         case 32: k_minmax_init<T, 32><<<grid, kThreads, 0, st>>>(W, n_groups, Q, s, z); break;
         case 64: k_minmax_init<T, 64><<<grid, kThreads, 0, st>>>(W, n_groups, Q, s, z); break;

@@ -515,9 +515,15 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-initpack70b", action="store_true")
+    ap.add_argument("--initpack70b-only", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)  # timing rule: at least 3 untimed warm-up steps
+    if args.initpack70b_only:  # profiling aid: just the 70B-block init/pack measurement
+        torch.cuda.set_device(0)
+        eqat.load_library()
+        print(json.dumps(initpack_70b_block(torch.device("cuda", 0), reps=1)), flush=True)
+        return
     if args.impl == "reference":
         run_reference(args)
     else:

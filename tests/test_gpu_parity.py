@@ -101,6 +101,56 @@ def test_fake_quant_and_pack_bit_exact(orc, dtype, trained, bits, g):
         assert_bits_equal(to_np(dq), dq_ref if odt == torch.float32 else bf16_round(dq_ref), "dequant")
 
 
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("bits", [2, 3, 4])
+def test_codes_at_and_around_rounding_boundaries_bit_exact(orc, dtype, bits):
+    """Weights on, and one or two ulps either side of, half-integer multiples of s:
+    the cases where the kernels' reciprocal-multiply decision must hand over to the
+    IEEE division to reproduce round(W/s)."""
+    Q = (1 << bits) - 1
+    rng = np.random.default_rng(4321 + bits)
+    N, K, g = 64, 512, 32
+    z = rng.integers(-1, Q + 2, size=(N, K // g)).astype(np.float32)
+    j = rng.integers(-Q - 3, Q + 3, size=(N, K)).astype(np.float32)
+    off = rng.integers(-2, 3, size=(N, K))
+    if dtype == "f32":
+        s = rng.uniform(1e-3, 0.1, size=(N, K // g)).astype(np.float32)
+        W = ((j + np.float32(0.5)) * np.repeat(s, g, 1)).astype(np.float32)
+        for step in (1, 2):
+            W = np.where(off >= step, np.nextafter(W, np.float32(np.inf)), W)
+            W = np.where(off <= -step, np.nextafter(W, np.float32(-np.inf)), W)
+        Wt = torch.from_numpy(W.astype(np.float32))
+    else:
+        # s with at most two significant bits keeps (j + 1/2) s exact in bf16; the
+        # offsets then step the bf16 bit pattern by one or two units.
+        s = (rng.choice([1.0, 3.0], size=(N, K // g)) * 2.0 ** rng.integers(-12, -4, size=(N, K // g))).astype(np.float32)
+        W = ((j + np.float32(0.5)) * np.repeat(s, g, 1)).astype(np.float32)
+        Wb = torch.from_numpy(W).to(torch.bfloat16)
+        assert np.array_equal(Wb.float().numpy(), W)
+        pattern = Wb.view(torch.int16).numpy().astype(np.int32) + off
+        Wt = torch.from_numpy(pattern.astype(np.int16)).view(torch.bfloat16)
+    Wn = Wt.float().numpy()
+    _, c_ref, m_ref, u_ref = orc.fake_quant(Wn, s, z, bits, g)
+    frac = np.abs(u_ref - np.floor(u_ref) - 0.5)
+    assert (frac == 0).sum() > 50  # exact ties present
+    sd, zd = torch.from_numpy(s).cuda(), torch.from_numpy(z).cuda()
+    _, c, m = eqat.fake_quant(Wt.cuda(), sd, zd, bits, g, want_w_hat=False)
+    assert_bits_equal(to_np(c), c_ref, "codes")
+    assert_bits_equal(to_np(m), m_ref, "mask")
+    p_ref, zq_ref = orc.pack(Wn, s, z, bits, g)
+    p, zq = eqat.pack_codes(Wt.cuda(), sd, zd, bits, g)
+    assert_bits_equal(to_np(p), p_ref, "packed")
+    if dtype == "bf16":
+        X = torch.randn(64, K).to(torch.bfloat16)
+        dY = torch.randn(64, N).to(torch.bfloat16)
+        dX, dW, ds, dz = eqat.fq_linear_bwd(X.cuda(), Wt.cuda(), sd, zd, dY.cuda(), bits, g)
+        dX_r, dW_r, ds_r, dz_r = orc.fq_linear_bwd(X.float().numpy(), Wn, s, z, dY.float().numpy(), bits, g)
+        assert (to_np(dW)[m_ref == 0] == 0).all() and (dW_r[m_ref == 0] == 0).all()
+        assert ((to_np(dW) != 0) == (dW_r != 0)).mean() > 0.999
+        assert_close(to_np(ds), ds_r, TOL_RED, "ds")
+        assert_close(to_np(dz), dz_r, TOL_RED, "dz")
+
+
 def check_fq(orc, M, N, K, bits, g, dtype, seed, trained, reuse=False):
     dev, Xn, Wn, dYn, s, z = inputs(M, N, K, bits, g, dtype, seed, trained, orc)
     tdt = torch.bfloat16 if dtype == "bf16" else torch.float32

@@ -76,12 +76,13 @@ __global__ void k_ste_epilogue_f32(const float *__restrict__ W, const float *__r
     const int64_t gi = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
     if (gi >= n_groups) return;
     const float sc = s[gi];
+    const float rcp = __frcp_rn(sc);
     const float zr = rintf(z[gi]);
     float acc_s = 0.0f, acc_z = 0.0f;
     const int64_t e0 = gi * group;
     for (int i = 0; i < group; ++i) {
         const float d = dwh[e0 + i];
-        const QuantElem e = quant_elem(W[e0 + i], sc, zr, Q);
+        const QuantElem e = quant_elem(W[e0 + i], sc, rcp, zr, Q);
         acc_s = fmaf(d, __fsub_rn(__fsub_rn(e.c, zr), e.inside ? e.u : 0.0f), acc_s);
         acc_z += e.inside ? 0.0f : d;
         if (dW) dW[e0 + i] = e.inside ? d : 0.0f;

@@ -26,6 +26,7 @@
 #include <algorithm>
 #include <atomic>
 #include <cstdint>
+#include <cstdlib>
 #include <mutex>
 
 #include "eqat_internal.h"
@@ -39,7 +40,7 @@ __device__ int g_dev_error = 0;
 namespace {
 
 constexpr int BM = 128;
-constexpr int BN = 256;
+constexpr int BN = 256;  // widest N tile; a problem may use 128 (Prob::bn)
 constexpr int BK = 64;  // one 128-byte swizzle row of bf16
 constexpr int UK = 16;  // K of one tcgen05.mma kind::f16
 constexpr int STAGES = 4;
@@ -58,6 +59,7 @@ constexpr uint64_t kWaitLimitNs = 4000000000ull;  // 4 s: far above any legitima
 struct Prob {
     int GM, GN, GK;
     int tiles_m, tiles_n, tile_begin, m_fast;
+    int bn;  // N-tile width of this problem: 256 or 128
     int a_mn, b_mn;  // operand majorness (1 = MN-major)
     // epilogue
     void *out;
@@ -150,6 +152,7 @@ struct Epilogue<1, BITS> {
         const int64_t G = K / p.group;
         const int64_t gi = static_cast<int64_t>(row) * G + col / p.group;
         const float sc = __ldg(p.s + gi);
+        const float rcp = __frcp_rn(sc);
         const float zr = rintf(__ldg(p.z + gi));
         const int64_t e0 = static_cast<int64_t>(row) * K + col;
         float dwv[32];
@@ -157,14 +160,18 @@ struct Epilogue<1, BITS> {
         for (int q = 0; q < 4; ++q) {
             float w[8];
             load8<__nv_bfloat16>(static_cast<const __nv_bfloat16 *>(p.W) + e0 + 8 * q, w);
+            float r[8], u[8];
+            round_quotients<8>(w, sc, rcp, r, u);
 #pragma unroll
             for (int j = 0; j < 8; ++j) {
                 const float d = v[8 * q + j];
-                const QuantElem e = quant_elem(w[j], sc, zr, p.Q);
-                const float dwds = __fsub_rn(__fsub_rn(e.c, zr), e.inside ? e.u : 0.0f);
+                const float qv = __fadd_rn(r[j], zr);
+                const bool inside = (qv >= 0.0f) && (qv <= p.Q);
+                const float c = fminf(fmaxf(qv, 0.0f), p.Q);
+                const float dwds = __fsub_rn(__fsub_rn(c, zr), inside ? u[j] : 0.0f);
                 acc_s = fmaf(d, dwds, acc_s);
-                acc_z += e.inside ? 0.0f : d;
-                dwv[8 * q + j] = e.inside ? d : 0.0f;
+                acc_z += inside ? 0.0f : d;
+                dwv[8 * q + j] = inside ? d : 0.0f;
             }
         }
         if (p.dW) {
@@ -293,7 +300,8 @@ __global__ void __launch_bounds__((4 + EPI_WARPS) * 32, 1)
                 const int a_mn = pi ? p.pr[1].a_mn : p.pr[0].a_mn;
                 const int b_mn = pi ? p.pr[1].b_mn : p.pr[0].b_mn;
                 const int nkb = ((pi ? p.pr[1].GK : p.pr[0].GK) + BK - 1) / BK;
-                const int m0 = tm * BM, n0 = tn * BN;
+                const int bn = pi ? p.pr[1].bn : p.pr[0].bn;
+                const int m0 = tm * BM, n0 = tn * bn;
                 for (int kb = 0; kb < nkb; ++kb, ++it) {
                     const int st = it % STAGES;
                     const uint32_t ph = (it / STAGES) & 1u;
@@ -303,7 +311,7 @@ __global__ void __launch_bounds__((4 + EPI_WARPS) * 32, 1)
                     }
                     uint8_t *sa = smem + st * STAGE_BYTES;
                     uint8_t *sb = sa + A_BYTES;
-                    mbar_arrive_expect_tx(&ctl->full[st], STAGE_BYTES);
+                    mbar_arrive_expect_tx(&ctl->full[st], A_BYTES + bn * BK * 2);
                     armed |= 1u << st;
                     armed_parity = (armed_parity & ~(1u << st)) | (ph << st);
                     const int k0 = kb * BK;
@@ -316,7 +324,7 @@ __global__ void __launch_bounds__((4 + EPI_WARPS) * 32, 1)
                     }
                     if (b_mn) {
 #pragma unroll
-                        for (int b = 0; b < BN / MN_BOX; ++b)
+                        for (int b = 0; b < bn / MN_BOX; ++b)
                             tma_load_2d(sb + b * MN_BOX_BYTES, mb, &ctl->full[st], n0 + b * MN_BOX, k0);
                     } else {
                         tma_load_2d(sb, mb, &ctl->full[st], k0, n0);
@@ -349,7 +357,8 @@ __global__ void __launch_bounds__((4 + EPI_WARPS) * 32, 1)
                 const int a_mn = pi ? p.pr[1].a_mn : p.pr[0].a_mn;
                 const int b_mn = pi ? p.pr[1].b_mn : p.pr[0].b_mn;
                 const int nkb = ((pi ? p.pr[1].GK : p.pr[0].GK) + BK - 1) / BK;
-                const uint32_t idesc = idesc_bf16_f32(BM, BN, a_mn != 0, b_mn != 0);
+                const int bn = pi ? p.pr[1].bn : p.pr[0].bn;
+                const uint32_t idesc = idesc_bf16_f32(BM, bn, a_mn != 0, b_mn != 0);
                 // K-major: advance 16 elements (32 B) inside the 128 B swizzle row,
                 // LBO unused (16), SBO = 8 rows x 128 B.  MN-major: advance 16 k-rows
                 // (2 KB), LBO = next 64-wide MN box, SBO = 8 k-rows x 128 B.
@@ -401,7 +410,7 @@ __global__ void __launch_bounds__((4 + EPI_WARPS) * 32, 1)
         const int quad = warp & 3;  // tensor-memory lane quadrant of this warp
         const int half = ew >> 2;   // column slice of the accumulator
         constexpr int SLICES = EPI_WARPS / 4;
-        constexpr int COLS = ACC_COLS / SLICES;
+
         uint32_t local = 0;
         for (int t = blockIdx.x; t < p.total_tiles; t += gridDim.x, ++local) {
             const uint32_t acc = local & 1u;
@@ -414,10 +423,12 @@ __global__ void __launch_bounds__((4 + EPI_WARPS) * 32, 1)
             const int pi = tile_coords(p, t, tm, tn);
             const int row = tm * BM + quad * 32 + lane;
             const uint32_t taddr = tmem_base + acc * ACC_COLS + ((quad * 32) << 16);
+            const int bn = pi ? p.pr[1].bn : p.pr[0].bn;
+            const int cols = bn / SLICES;  // a multiple of 64, hence of every group size
             if (pi == 0)
-                drain_accumulator<EPI0, BITS>(p.pr[0], taddr, row, tn * BN, half * COLS, (half + 1) * COLS);
+                drain_accumulator<EPI0, BITS>(p.pr[0], taddr, row, tn * bn, half * cols, (half + 1) * cols);
             else
-                drain_accumulator<EPI1, BITS>(p.pr[1], taddr, row, tn * BN, half * COLS, (half + 1) * COLS);
+                drain_accumulator<EPI1, BITS>(p.pr[1], taddr, row, tn * bn, half * cols, (half + 1) * cols);
             tc_fence_before();
             mbar_arrive(&ctl->acc_empty[acc]);
         }
@@ -497,19 +508,20 @@ int *device_error_ptr() {
     return ptr;
 }
 
-cudaError_t fill_prob(Prob &q, const GemmProblem &g, int tile_begin, CUtensorMap &ma, CUtensorMap &mb) {
+cudaError_t fill_prob(Prob &q, const GemmProblem &g, int tile_begin, int bn, CUtensorMap &ma, CUtensorMap &mb) {
     const int64_t GM = g.GM, GN = g.GN, GK = g.GK;
     if (GM <= 0 || GN <= 0 || GK <= 0) return cudaErrorInvalidValue;
     if (GM > INT32_MAX - BM || GN > INT32_MAX - BN || GK > INT32_MAX - BK) return cudaErrorInvalidValue;
     cudaError_t e;
     if ((e = make_map(ma, g.A, GM, GK, BM)) != cudaSuccess) return e;
-    if ((e = make_map(mb, g.B, GN, GK, BN)) != cudaSuccess) return e;
+    if ((e = make_map(mb, g.B, GN, GK, bn)) != cudaSuccess) return e;
     q = Prob{};
     q.GM = static_cast<int>(GM);
     q.GN = static_cast<int>(GN);
     q.GK = static_cast<int>(GK);
     q.tiles_m = static_cast<int>((GM + BM - 1) / BM);
-    q.tiles_n = static_cast<int>((GN + BN - 1) / BN);
+    q.tiles_n = static_cast<int>((GN + bn - 1) / bn);
+    q.bn = bn;
     q.tile_begin = tile_begin;
     // Consecutive CTAs share the operand whose tiles are the larger total, so
     // that the smaller one stays hot in L2 while the larger streams once.
@@ -532,6 +544,37 @@ cudaError_t fill_prob(Prob &q, const GemmProblem &g, int tile_begin, CUtensorMap
     return cudaSuccess;
 }
 
+// N-tile width for a launch.  A 128-wide tile does half the work of a 256-wide
+// one at a somewhat lower tensor-pipe efficiency (more operand traffic per FLOP),
+// but halves the granularity of the last wave.  Estimated time = waves x tile cost;
+// the narrower tile wins when it removes enough of a partial last wave.  Group
+// reductions need a whole group inside one epilogue slice (bn / 2 columns).
+// EQAT_GEMM_BN=128|256 forces a width (measurement aid).
+int choose_bn(const GemmProblem *probs, int nprob, int sms) {
+    bool narrow_ok = true;
+    for (int i = 0; i < nprob; ++i)
+        if (probs[i].epi.kind != Epi::kStore && probs[i].epi.group > 64) narrow_ok = false;
+    static const int forced = [] {
+        const char *v = std::getenv("EQAT_GEMM_BN");
+        return v ? std::atoi(v) : 0;
+    }();
+    if (forced == 256) return 256;
+    if (forced == 128 && narrow_ok) return 128;
+    if (!narrow_ok) return 256;
+    auto estimate = [&](int bn, double tile_cost) {
+        int64_t tiles = 0;
+        for (int i = 0; i < nprob; ++i)
+            tiles += ((probs[i].GM + BM - 1) / BM) * ((probs[i].GN + bn - 1) / bn);
+        const int64_t waves = (tiles + sms - 1) / sms;
+        return static_cast<double>(waves) * tile_cost;
+    };
+    // Measured on B200 (4096^3 forward, bench.py): a wave of 128-wide tiles takes
+    // 0.71 of a wave of 256-wide ones, i.e. 42% more time per FLOP, in line with
+    // the operand bytes per FLOP the tensor core reads from shared memory.
+    constexpr double kNarrowTileCost = 0.72;
+    return estimate(128, kNarrowTileCost) < estimate(256, 1.0) ? 128 : 256;
+}
+
 }  // namespace
 
 cudaError_t launch_gemm_tc_group(const GemmProblem *probs, int nprob, const DeviceInfo &dev,
@@ -548,8 +591,9 @@ cudaError_t launch_gemm_tc_group(const GemmProblem *probs, int nprob, const Devi
     CUtensorMap maps[4];
     KParams p{};
     int tiles = 0;
+    const int bn = choose_bn(probs, nprob, dev.sm_count);
     for (int i = 0; i < nprob; ++i) {
-        if ((e = fill_prob(p.pr[i], probs[i], tiles, maps[2 * i], maps[2 * i + 1])) != cudaSuccess) return e;
+        if ((e = fill_prob(p.pr[i], probs[i], tiles, bn, maps[2 * i], maps[2 * i + 1])) != cudaSuccess) return e;
         const int64_t t = static_cast<int64_t>(p.pr[i].tiles_m) * p.pr[i].tiles_n;
         if (tiles + t > INT32_MAX) return cudaErrorInvalidValue;
         tiles += static_cast<int>(t);

@@ -14,15 +14,59 @@ namespace eqat {
 constexpr float kStepMin = 1e-5f;  // floor of s for constant groups (EQAT_S_MIN)
 
 struct QuantElem {
-    float u;      // W / s, correctly rounded
+    float u;      // W / s (see round_quotient for its accuracy)
     float c;      // clamped code, integer-valued
-    bool inside;  // 0 <= round(u) + zr <= Q
+    bool inside;  // 0 <= round(W/s) + zr <= Q
 };
 
-__device__ __forceinline__ QuantElem quant_elem(float w, float s, float zr, float Q) {
+// round(RN(W/s)) without a division per weight.  With rcp = RN(1/s),
+// q = RN(W * rcp) satisfies |q - RN(W/s)| < |W/s| 2^-22 (two roundings of the
+// quotient against one), so round(q) can differ from round(RN(W/s)) only if q
+// lies within |q| 2^-21 of a half-integer, a rounding boundary of round().
+// There the IEEE division decides; elsewhere the product does.  The returned
+// integer is therefore always round(RN(W/s)); u is RN(W/s) on the exact path
+// and q (within 2^-22 relative) otherwise.
+__device__ __forceinline__ float round_quotient(float w, float s, float rcp, float &u) {
+    const float q = __fmul_rn(w, rcp);
+    const float r = rintf(q);
+    const float to_half = __fsub_rn(0.5f, fabsf(__fsub_rn(q, r)));  // distance to nearest half-integer
+    if (to_half <= fabsf(q) * 0x1p-21f) {
+        u = __fdiv_rn(w, s);
+        return rintf(u);
+    }
+    u = q;
+    return r;
+}
+
+// round_quotient for N weights of one group with a single branch: the fast
+// decisions for all N first, then, only if one of them lies within the bound of a
+// rounding boundary, the IEEE division for those.  r[j] = round(RN(w[j]/s)); u[j]
+// as in round_quotient.
+template <int N>
+__device__ __forceinline__ void round_quotients(const float (&w)[N], float s, float rcp, float (&r)[N],
+                                                float (&u)[N]) {
+    bool near = false;
+#pragma unroll
+    for (int j = 0; j < N; ++j) {
+        u[j] = __fmul_rn(w[j], rcp);
+        r[j] = rintf(u[j]);
+        near |= __fsub_rn(0.5f, fabsf(__fsub_rn(u[j], r[j]))) <= fabsf(u[j]) * 0x1p-21f;
+    }
+    if (near) {
+#pragma unroll
+        for (int j = 0; j < N; ++j) {
+            if (__fsub_rn(0.5f, fabsf(__fsub_rn(u[j], r[j]))) <= fabsf(u[j]) * 0x1p-21f) {
+                u[j] = __fdiv_rn(w[j], s);
+                r[j] = rintf(u[j]);
+            }
+        }
+    }
+}
+
+// Eq. 1 and the straight-through mask for one weight; rcp = __frcp_rn(s).
+__device__ __forceinline__ QuantElem quant_elem(float w, float s, float rcp, float zr, float Q) {
     QuantElem e;
-    e.u = __fdiv_rn(w, s);
-    const float q = __fadd_rn(rintf(e.u), zr);
+    const float q = __fadd_rn(round_quotient(w, s, rcp, e.u), zr);
     e.inside = (q >= 0.0f) && (q <= Q);
     e.c = fminf(fmaxf(q, 0.0f), Q);
     return e;
@@ -49,6 +93,54 @@ __device__ __forceinline__ float bf16_hi(uint32_t v) { return __uint_as_float(v 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);  // .x = lo (low half), .y = hi
     return *reinterpret_cast<uint32_t *>(&h);
+}
+
+// 8 consecutive elements as stored: one 16-byte word of bf16, two of fp32.
+template <typename T>
+struct Raw8;
+template <>
+struct Raw8<__nv_bfloat16> {
+    uint4 v;
+};
+template <>
+struct Raw8<float> {
+    float4 a, b;
+};
+
+template <typename T>
+__device__ __forceinline__ Raw8<T> load_raw8(const T *p);
+template <>
+__device__ __forceinline__ Raw8<__nv_bfloat16> load_raw8<__nv_bfloat16>(const __nv_bfloat16 *p) {
+    return Raw8<__nv_bfloat16>{__ldg(reinterpret_cast<const uint4 *>(p))};
+}
+template <>
+__device__ __forceinline__ Raw8<float> load_raw8<float>(const float *p) {
+    return Raw8<float>{__ldg(reinterpret_cast<const float4 *>(p)), __ldg(reinterpret_cast<const float4 *>(p) + 1)};
+}
+
+__device__ __forceinline__ void unpack8(const Raw8<__nv_bfloat16> &r, float (&v)[8]) {
+    v[0] = bf16_lo(r.v.x); v[1] = bf16_hi(r.v.x);
+    v[2] = bf16_lo(r.v.y); v[3] = bf16_hi(r.v.y);
+    v[4] = bf16_lo(r.v.z); v[5] = bf16_hi(r.v.z);
+    v[6] = bf16_lo(r.v.w); v[7] = bf16_hi(r.v.w);
+}
+__device__ __forceinline__ void unpack8(const Raw8<float> &r, float (&v)[8]) {
+    v[0] = r.a.x; v[1] = r.a.y; v[2] = r.a.z; v[3] = r.a.w;
+    v[4] = r.b.x; v[5] = r.b.y; v[6] = r.b.z; v[7] = r.b.w;
+}
+
+// Exact min and max of the 8 elements (bf16 min/max on packed pairs; the
+// widening to fp32 is exact).
+__device__ __forceinline__ void minmax8(const Raw8<__nv_bfloat16> &r, float &mn, float &mx) {
+    const __nv_bfloat162 *h = reinterpret_cast<const __nv_bfloat162 *>(&r.v);
+    __nv_bfloat162 lo = __hmin2(__hmin2(h[0], h[1]), __hmin2(h[2], h[3]));
+    __nv_bfloat162 hi = __hmax2(__hmax2(h[0], h[1]), __hmax2(h[2], h[3]));
+    mn = fminf(__low2float(lo), __high2float(lo));
+    mx = fmaxf(__low2float(hi), __high2float(hi));
+}
+__device__ __forceinline__ void minmax8(const Raw8<float> &r, float &mn, float &mx) {
+    mn = fminf(fminf(fminf(r.a.x, r.a.y), fminf(r.a.z, r.a.w)), fminf(fminf(r.b.x, r.b.y), fminf(r.b.z, r.b.w)));
+    mx = fmaxf(fmaxf(fmaxf(r.a.x, r.a.y), fmaxf(r.a.z, r.a.w)), fmaxf(fmaxf(r.b.x, r.b.y), fmaxf(r.b.z, r.b.w)));
 }
 
 // Loads 8 consecutive elements (16 bytes of bf16, 32 bytes of fp32) as floats.

@@ -34,46 +34,59 @@ inline int grid_for(int64_t work_items, const DeviceInfo &dev, int per_thread = 
 // group and reduce min/max with xor shuffles; UNROLL independent groups per
 // thread keep 128 bytes (bf16) of loads in flight per thread.
 template <typename T, int G>
-__global__ void __launch_bounds__(kThreads) k_minmax_init(const T *__restrict__ W, int64_t n_groups,
-                                                          float Q, float *__restrict__ s,
-                                                          float *__restrict__ z) {
+__global__ void __launch_bounds__(kThreads, 4) k_minmax_init(const T *__restrict__ W, int64_t n_groups,
+                                                             float Q, float *__restrict__ s,
+                                                             float *__restrict__ z) {
     constexpr int TPG = G / 8;
     constexpr int GPW = 32 / TPG;  // groups per warp per unrolled slot
-    constexpr int UNROLL = 8;
+    constexpr int UNROLL = 4;  // 16-byte words in flight per thread
     const int lane = threadIdx.x & 31;
     const int sub = lane % TPG;
     const int slot = lane / TPG;
     const int64_t warp = (static_cast<int64_t>(blockIdx.x) * kThreads + threadIdx.x) >> 5;
     const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * kThreads) >> 5;
     for (int64_t base = warp * (GPW * UNROLL); base < n_groups; base += nwarps * (GPW * UNROLL)) {
-        float v[UNROLL][8];
+        Raw8<T> raw[UNROLL];
 #pragma unroll
         for (int u = 0; u < UNROLL; ++u) {
             const int64_t g = base + u * GPW + slot;
-            if (g < n_groups) {
-                load8<T>(W + g * G + sub * 8, v[u]);
-            } else {
+            if (g < n_groups) raw[u] = load_raw8<T>(W + g * G + sub * 8);
+        }
+        // Reduce every chunk to (min, max) first so the raw words die before the
+        // shuffles and the per-group divisions.
+        float mn[UNROLL], mx[UNROLL];
 #pragma unroll
-                for (int i = 0; i < 8; ++i) v[u][i] = 0.0f;
-            }
+        for (int u = 0; u < UNROLL; ++u) {
+            mn[u] = 0.0f;
+            mx[u] = 0.0f;
+            if (base + u * GPW + slot < n_groups) minmax8(raw[u], mn[u], mx[u]);
         }
 #pragma unroll
         for (int u = 0; u < UNROLL; ++u) {
-            float mn = v[u][0], mx = v[u][0];
-#pragma unroll
-            for (int i = 1; i < 8; ++i) {
-                mn = fminf(mn, v[u][i]);
-                mx = fmaxf(mx, v[u][i]);
-            }
 #pragma unroll
             for (int off = TPG / 2; off > 0; off >>= 1) {
-                mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, off));
-                mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+                mn[u] = fminf(mn[u], __shfl_xor_sync(0xffffffffu, mn[u], off));
+                mx[u] = fmaxf(mx[u], __shfl_xor_sync(0xffffffffu, mx[u], off));
             }
-            const int64_t g = base + u * GPW + slot;
-            if (sub == 0 && g < n_groups) {
+        }
+        // After the xor-shuffles every lane of a group holds its (min, max): lane
+        // `sub` finishes chunks sub, sub + TPG, ... so the divisions spread over
+        // the group's lanes instead of running one after another on one lane.
+        constexpr int PER_LANE = (UNROLL + TPG - 1) / TPG;
+#pragma unroll
+        for (int k = 0; k < PER_LANE; ++k) {
+            const int uu = sub + k * TPG;
+            float a = 0.0f, b = 0.0f;
+#pragma unroll
+            for (int u = 0; u < UNROLL; ++u)
+                if (u == uu) {
+                    a = mn[u];
+                    b = mx[u];
+                }
+            const int64_t g = base + uu * GPW + slot;
+            if (uu < UNROLL && g < n_groups) {
                 float sc, zz;
-                minmax_step_zero(mn, mx, Q, sc, zz);
+                minmax_step_zero(a, b, Q, sc, zz);
                 s[g] = sc;
                 z[g] = zz;
             }
@@ -84,18 +97,21 @@ __global__ void __launch_bounds__(kThreads) k_minmax_init(const T *__restrict__ 
 // ------------------------------------------------------------------ fake-quant prepass
 // A thread handles U = 2 chunks of 8 consecutive weights (each chunk inside one
 // group) per iteration and issues both loads before any arithmetic.
-template <typename T, typename O>
+template <typename T, typename O, bool CODES>
 __device__ __forceinline__ void fake_quant_chunk(const float (&w)[8], float sc, float zr, float Q,
                                                  int64_t e0, O *__restrict__ W_hat,
                                                  uint8_t *__restrict__ code, uint8_t *__restrict__ mask) {
-    float wh[8];
+    float wh[8], r[8], u[8];
+    round_quotients<8>(w, sc, __frcp_rn(sc), r, u);
     uint32_t c_lo = 0, c_hi = 0, m_lo = 0, m_hi = 0;
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
-        const QuantElem q = quant_elem(w[j], sc, zr, Q);
-        wh[j] = dequant_elem(q.c, zr, sc);
-        const uint32_t cb = static_cast<uint32_t>(q.c);
-        const uint32_t mb = q.inside ? 1u : 0u;
+        const float q = __fadd_rn(r[j], zr);
+        const bool inside = (q >= 0.0f) && (q <= Q);
+        const float c = fminf(fmaxf(q, 0.0f), Q);
+        wh[j] = dequant_elem(c, zr, sc);
+        const uint32_t cb = static_cast<uint32_t>(c);
+        const uint32_t mb = inside ? 1u : 0u;
         if (j < 4) {
             c_lo |= cb << (8 * j);
             m_lo |= mb << (8 * j);
@@ -105,12 +121,14 @@ __device__ __forceinline__ void fake_quant_chunk(const float (&w)[8], float sc, 
         }
     }
     if (W_hat) store8<O>(W_hat + e0, wh);
-    if (code) *reinterpret_cast<uint2 *>(code + e0) = make_uint2(c_lo, c_hi);
-    if (mask) *reinterpret_cast<uint2 *>(mask + e0) = make_uint2(m_lo, m_hi);
+    if (CODES) {
+        if (code) *reinterpret_cast<uint2 *>(code + e0) = make_uint2(c_lo, c_hi);
+        if (mask) *reinterpret_cast<uint2 *>(mask + e0) = make_uint2(m_lo, m_hi);
+    }
 }
 
-template <typename T, typename O>
-__global__ void __launch_bounds__(kThreads)
+template <typename T, typename O, bool CODES>
+__global__ void __launch_bounds__(kThreads, 4)
     k_fake_quant(const T *__restrict__ W, const float *__restrict__ s, const float *__restrict__ z,
                  int64_t n_chunks, int group, float Q, O *__restrict__ W_hat,
                  uint8_t *__restrict__ code, uint8_t *__restrict__ mask) {
@@ -118,13 +136,13 @@ __global__ void __launch_bounds__(kThreads)
     const int64_t nthreads = static_cast<int64_t>(gridDim.x) * kThreads;
     for (int64_t base = static_cast<int64_t>(blockIdx.x) * kThreads + threadIdx.x; base < n_chunks;
          base += nthreads * U) {
-        float w[U][8];
+        Raw8<T> raw[U];
         float sc[U], zr[U];
 #pragma unroll
         for (int u = 0; u < U; ++u) {
             const int64_t i = base + u * nthreads;
             if (i < n_chunks) {
-                load8<T>(W + i * 8, w[u]);
+                raw[u] = load_raw8<T>(W + i * 8);
                 const int64_t g = (i * 8) / group;
                 sc[u] = __ldg(s + g);
                 zr[u] = rintf(__ldg(z + g));
@@ -133,7 +151,11 @@ __global__ void __launch_bounds__(kThreads)
 #pragma unroll
         for (int u = 0; u < U; ++u) {
             const int64_t i = base + u * nthreads;
-            if (i < n_chunks) fake_quant_chunk<T, O>(w[u], sc[u], zr[u], Q, i * 8, W_hat, code, mask);
+            if (i < n_chunks) {
+                float w[8];
+                unpack8(raw[u], w);
+                fake_quant_chunk<T, O, CODES>(w, sc[u], zr[u], Q, i * 8, W_hat, code, mask);
+            }
         }
     }
 }
@@ -145,28 +167,27 @@ __global__ void __launch_bounds__(kThreads)
 template <int BITS>
 __device__ __forceinline__ void pack_chunk(const float (&w)[16], float sc, float zr, float Q, int64_t e0,
                                            uint8_t *__restrict__ codes) {
-    uint32_t c[16];
+    const float rcp = __frcp_rn(sc);
+    uint32_t word[4] = {0u, 0u, 0u, 0u};  // 2-bit: word[0]; 4-bit: word[0..1]; 3-bit: word[0..3]
 #pragma unroll
-    for (int j = 0; j < 16; ++j) c[j] = static_cast<uint32_t>(quant_elem(w[j], sc, zr, Q).c);
+    for (int h = 0; h < 2; ++h) {  // two batches of 8 keep the rare division path small
+        float r[8], u[8];
+        round_quotients<8>(*reinterpret_cast<const float(*)[8]>(&w[8 * h]), sc, rcp, r, u);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            const uint32_t c = static_cast<uint32_t>(fminf(fmaxf(__fadd_rn(r[j], zr), 0.0f), Q));
+            const int k = 8 * h + j;
+            if (BITS == 2) word[0] |= c << (2 * k);
+            else if (BITS == 4) word[k / 8] |= c << (4 * (k % 8));
+            else word[k / 4] |= c << (8 * (k % 4));
+        }
+    }
     if (BITS == 2) {
-        uint32_t word = 0;
-#pragma unroll
-        for (int j = 0; j < 16; ++j) word |= c[j] << (2 * j);
-        *reinterpret_cast<uint32_t *>(codes + e0 / 4) = word;
+        *reinterpret_cast<uint32_t *>(codes + e0 / 4) = word[0];
     } else if (BITS == 4) {
-        uint32_t lo = 0, hi = 0;
-#pragma unroll
-        for (int j = 0; j < 8; ++j) lo |= c[j] << (4 * j);
-#pragma unroll
-        for (int j = 0; j < 8; ++j) hi |= c[8 + j] << (4 * j);
-        *reinterpret_cast<uint2 *>(codes + e0 / 2) = make_uint2(lo, hi);
+        *reinterpret_cast<uint2 *>(codes + e0 / 2) = make_uint2(word[0], word[1]);
     } else {
-        uint4 r;
-        r.x = c[0] | (c[1] << 8) | (c[2] << 16) | (c[3] << 24);
-        r.y = c[4] | (c[5] << 8) | (c[6] << 16) | (c[7] << 24);
-        r.z = c[8] | (c[9] << 8) | (c[10] << 16) | (c[11] << 24);
-        r.w = c[12] | (c[13] << 8) | (c[14] << 16) | (c[15] << 24);
-        *reinterpret_cast<uint4 *>(codes + e0) = r;
+        *reinterpret_cast<uint4 *>(codes + e0) = make_uint4(word[0], word[1], word[2], word[3]);
     }
 }
 
@@ -175,7 +196,7 @@ __device__ __forceinline__ void pack_chunk(const float (&w)[16], float sc, float
 // zr := zq (z hard-rounded at pack time).  Output per chunk: 4 bytes (2-bit), 8
 // bytes (4-bit) or 16 bytes (3-bit, one code per byte).
 template <typename T, int BITS>
-__global__ void __launch_bounds__(kThreads)
+__global__ void __launch_bounds__(kThreads, 4)
     k_pack(const T *__restrict__ W, const float *__restrict__ s, const float *__restrict__ z,
            int64_t n_chunks, int group, float Q, uint8_t *__restrict__ codes,
            uint8_t *__restrict__ zq) {
@@ -183,14 +204,14 @@ __global__ void __launch_bounds__(kThreads)
     const int64_t nthreads = static_cast<int64_t>(gridDim.x) * kThreads;
     for (int64_t base = static_cast<int64_t>(blockIdx.x) * kThreads + threadIdx.x; base < n_chunks;
          base += nthreads * U) {
-        float w[U][16];
+        Raw8<T> raw[U][2];
         float sc[U], zr[U];
 #pragma unroll
         for (int u = 0; u < U; ++u) {
             const int64_t i = base + u * nthreads;
             if (i < n_chunks) {
-                load8<T>(W + i * 16, *reinterpret_cast<float(*)[8]>(&w[u][0]));
-                load8<T>(W + i * 16 + 8, *reinterpret_cast<float(*)[8]>(&w[u][8]));
+                raw[u][0] = load_raw8<T>(W + i * 16);
+                raw[u][1] = load_raw8<T>(W + i * 16 + 8);
                 const int64_t g = (i * 16) / group;
                 sc[u] = __ldg(s + g);
                 zr[u] = fminf(fmaxf(rintf(__ldg(z + g)), 0.0f), Q);
@@ -202,7 +223,10 @@ __global__ void __launch_bounds__(kThreads)
             if (i < n_chunks) {
                 const int64_t e0 = i * 16;
                 if (e0 % group == 0) zq[e0 / group] = static_cast<uint8_t>(zr[u]);
-                pack_chunk<BITS>(w[u], sc[u], zr[u], Q, e0, codes);
+                float w[16];
+                unpack8(raw[u][0], *reinterpret_cast<float(*)[8]>(&w[0]));
+                unpack8(raw[u][1], *reinterpret_cast<float(*)[8]>(&w[8]));
+                pack_chunk<BITS>(w, sc[u], zr[u], Q, e0, codes);
             }
         }
     }
@@ -256,7 +280,7 @@ __global__ void __launch_bounds__(kThreads)
 template <typename T>
 cudaError_t minmax_dispatch(const T *W, int64_t n_groups, int group, float Q, float *s, float *z,
                             const DeviceInfo &dev, cudaStream_t st) {
-    const int grid = grid_for(n_groups * group, dev, 8 * 8);
+    const int grid = grid_for(n_groups * group, dev, 8 * 4);
     switch (group) {
         case 32: k_minmax_init<T, 32><<<grid, kThreads, 0, st>>>(W, n_groups, Q, s, z); break;
         case 64: k_minmax_init<T, 64><<<grid, kThreads, 0, st>>>(W, n_groups, Q, s, z); break;
@@ -316,18 +340,25 @@ cudaError_t launch_fake_quant(const void *W, bool w_f32, const float *s, const f
     const int grid = grid_for(chunks, dev);
     const float Q = static_cast<float>((1 << bits) - 1);
     using bf = __nv_bfloat16;
+    const bool codes = code || mask;
+#define EQAT_FQ_LAUNCH(TW, TO)                                                                          \
+    do {                                                                                                \
+        if (codes)                                                                                      \
+            k_fake_quant<TW, TO, true><<<grid, kThreads, 0, st>>>(static_cast<const TW *>(W), s, z, chunks, \
+                                                                 group, Q, static_cast<TO *>(W_hat), code, mask); \
+        else                                                                                            \
+            k_fake_quant<TW, TO, false><<<grid, kThreads, 0, st>>>(static_cast<const TW *>(W), s, z, chunks, \
+                                                                  group, Q, static_cast<TO *>(W_hat), code, mask); \
+    } while (0)
     if (w_f32 && out_f32)
-        k_fake_quant<float, float><<<grid, kThreads, 0, st>>>(
-            static_cast<const float *>(W), s, z, chunks, group, Q, static_cast<float *>(W_hat), code, mask);
+        EQAT_FQ_LAUNCH(float, float);
     else if (w_f32)
-        k_fake_quant<float, bf><<<grid, kThreads, 0, st>>>(
-            static_cast<const float *>(W), s, z, chunks, group, Q, static_cast<bf *>(W_hat), code, mask);
+        EQAT_FQ_LAUNCH(float, bf);
     else if (out_f32)
-        k_fake_quant<bf, float><<<grid, kThreads, 0, st>>>(
-            static_cast<const bf *>(W), s, z, chunks, group, Q, static_cast<float *>(W_hat), code, mask);
+        EQAT_FQ_LAUNCH(bf, float);
     else
-        k_fake_quant<bf, bf><<<grid, kThreads, 0, st>>>(
-            static_cast<const bf *>(W), s, z, chunks, group, Q, static_cast<bf *>(W_hat), code, mask);
+        EQAT_FQ_LAUNCH(bf, bf);
+#undef EQAT_FQ_LAUNCH
     return cudaGetLastError();
 }
 

@@ -42,7 +42,7 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 import weight_quantization_aware_b200 as eqat  # noqa: E402
-from weight_quantization_aware_b200 import synthetic  # noqa: E402
+from weight_quantization_aware_b200 import dp, synthetic  # noqa: E402
 
 WORKLOAD = synthetic.WORKLOADS[2]
 METRIC = "fake-quant linear fwd+bwd TFLOP/s & % bf16 peak (w2g64); init/pack HBM GB/s"
@@ -150,12 +150,7 @@ class Step:
         lin = wl.linears[0]
         self.M, self.N, self.K = wl.m, lin.n, lin.k
         self.bits, self.group = bits, group
-        rng = synthetic.rng_for(wl.index, 0)
-        d = synthetic.draw_linear(rng, wl.m, lin.n, lin.k, wl.sigma, wl.dtype, wl.outliers)
-        if rank:  # each data-parallel rank sees its own tokens; W is shared
-            d2 = synthetic.draw_linear(synthetic.rng_for(wl.index, 1000 + rank), wl.m, lin.n, lin.k,
-                                       wl.sigma, wl.dtype, wl.outliers)
-            d["X"], d["dY"] = d2["X"], d2["dY"]
+        d = dp.rank_batch(wl, 0, rank)  # each data-parallel rank sees its own tokens; W is shared
         self.host = {k: v.pin_memory() for k, v in d.items()}
         self.X = self.host["X"].to(dev)
         self.W = self.host["W"].to(dev)
@@ -244,8 +239,7 @@ def run_ours(args):
     allreduce = None
     if dist is not None:
         def allreduce(ts):
-            for t in ts:
-                dist.all_reduce(t)
+            dp.allreduce_weight_grads(ts, dist)
 
     for _ in range(args.warmup):
         flush_l2(flush)

@@ -254,6 +254,25 @@ def test_backward_single_contraction_paths(orc):
     assert_close(to_np(ds2), ds2_ref, TOL_RED, "E2E ds only")
 
 
+@pytest.mark.parametrize("shape", [
+    (1024, 520, 2048, 2, 64),    # fewer tiles than SMs, long K
+    (1024, 1024, 1024, 3, 128),  # grouped backward with one partial wave
+    (520, 256, 1536, 2, 32),     # ragged M and N tails, long K
+], ids=lambda s: "x".join(map(str, s)))
+def test_long_k_partial_wave_launches(orc, shape):
+    """Launches of fewer tiles than SMs with long reductions, twice in a row on one
+    workspace (store, straight-through and E2E-QP ds epilogues)."""
+    M, N, K, bits, g = shape
+    check_fq(orc, M, N, K, bits, g, "bf16", 700 + M, True)
+    check_dq(orc, M, N, K, bits, g, "bf16", 800 + M)
+    dev, Xn, Wn, dYn, s, z = inputs(M, N, K, bits, g, "bf16", 900 + M, True, orc)
+    ws = eqat.workspace(M, N, K, bits, g, torch.bfloat16)
+    ref = orc.fq_linear_fwd(Xn, Wn, s, z, bits, g)
+    for _ in range(2):
+        Y = eqat.fq_linear_fwd(dev["X"], dev["W"], dev["s"], dev["z"], bits, g, ws=ws)
+        assert_close(to_np(Y), ref, TOL_GEMM, "Y (repeat)")
+
+
 def test_persistent_tiles_wrap_accumulator_ring(orc):
     """More than two output tiles per CTA (the double-buffered accumulator ring wraps
     several times), checked on sampled rows."""

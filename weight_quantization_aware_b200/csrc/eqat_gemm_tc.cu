@@ -73,6 +73,7 @@ struct Prob {
     const uint8_t *codes;
     const uint8_t *zq;
     int group;
+    int gshift;  // log2(group)
     float Q;
 };
 
@@ -149,8 +150,8 @@ struct Epilogue<1, BITS> {
     __device__ __forceinline__ void chunk(const Prob &p, int row, int col, const float (&v)[32]) {
         if (row >= p.GM || col >= p.GN) return;
         const int64_t K = p.GN;
-        const int64_t G = K / p.group;
-        const int64_t gi = static_cast<int64_t>(row) * G + col / p.group;
+        const int64_t G = K >> p.gshift;
+        const int64_t gi = static_cast<int64_t>(row) * G + (col >> p.gshift);
         const float sc = __ldg(p.s + gi);
         const float rcp = __frcp_rn(sc);
         const float zr = rintf(__ldg(p.z + gi));
@@ -180,7 +181,7 @@ struct Epilogue<1, BITS> {
             for (int q = 0; q < 4; ++q)
                 store8<__nv_bfloat16>(o + 8 * q, *reinterpret_cast<const float(*)[8]>(&dwv[8 * q]));
         }
-        if (((col + 32) % p.group) == 0) {
+        if (((col + 32) & (p.group - 1)) == 0) {
             if (p.ds) p.ds[gi] = acc_s;
             if (p.dz) p.dz[gi] = -sc * acc_z;
             acc_s = 0.0f;
@@ -196,8 +197,8 @@ struct Epilogue<2, BITS> {
     __device__ __forceinline__ void chunk(const Prob &p, int row, int col, const float (&v)[32]) {
         if (row >= p.GM || col >= p.GN) return;
         const int64_t K = p.GN;
-        const int64_t G = K / p.group;
-        const int64_t gi = static_cast<int64_t>(row) * G + col / p.group;
+        const int64_t G = K >> p.gshift;
+        const int64_t gi = static_cast<int64_t>(row) * G + (col >> p.gshift);
         const float zf = static_cast<float>(__ldg(p.zq + gi));
         uint32_t c[32];
         if (BITS == 2) {
@@ -220,7 +221,7 @@ struct Epilogue<2, BITS> {
         }
 #pragma unroll
         for (int j = 0; j < 32; ++j) acc_s = fmaf(v[j], __fsub_rn(static_cast<float>(c[j]), zf), acc_s);
-        if (((col + 32) % p.group) == 0) {
+        if (((col + 32) & (p.group - 1)) == 0) {
             p.ds[gi] = acc_s;
             acc_s = 0.0f;
         }
@@ -540,6 +541,7 @@ cudaError_t fill_prob(Prob &q, const GemmProblem &g, int tile_begin, int bn, CUt
     q.codes = epi.codes;
     q.zq = epi.zq;
     q.group = epi.group;
+    q.gshift = epi.group == 32 ? 5 : epi.group == 64 ? 6 : 7;
     q.Q = static_cast<float>((1 << epi.bits) - 1);
     return cudaSuccess;
 }

@@ -42,6 +42,20 @@ __device__ __forceinline__ float round_quotient(float w, float s, float rcp, flo
 // decisions for all N first, then, only if one of them lies within the bound of a
 // rounding boundary, the IEEE division for those.  r[j] = round(RN(w[j]/s)); u[j]
 // as in round_quotient.
+// Round-half-to-even with two full-rate additions: for |x| < 2^22,
+// RN(RN(x + 1.5 * 2^23) - 1.5 * 2^23) == rint(x), because x + 1.5 * 2^23 lies in
+// [2^23, 2^24) where the spacing of fp32 is 1.  (For larger |x| the callers'
+// near-boundary test always fires and the exact path decides.)  Unlike rintf this
+// keeps the work off the quarter-rate conversion pipe.
+constexpr float kRoundMagic = 12582912.0f;  // 1.5 * 2^23
+
+__device__ __forceinline__ float rint_small(float x) { return __fsub_rn(__fadd_rn(x, kRoundMagic), kRoundMagic); }
+
+// A clamped code c in [0, 255] as an integer: the low mantissa bits of c + 1.5 * 2^23.
+__device__ __forceinline__ uint32_t code_bits(float c) {
+    return static_cast<uint32_t>(__float_as_int(__fadd_rn(c, kRoundMagic))) & 0xFFu;
+}
+
 template <int N>
 __device__ __forceinline__ void round_quotients(const float (&w)[N], float s, float rcp, float (&r)[N],
                                                 float (&u)[N]) {
@@ -49,13 +63,15 @@ __device__ __forceinline__ void round_quotients(const float (&w)[N], float s, fl
 #pragma unroll
     for (int j = 0; j < N; ++j) {
         u[j] = __fmul_rn(w[j], rcp);
-        r[j] = rintf(u[j]);
-        near |= __fsub_rn(0.5f, fabsf(__fsub_rn(u[j], r[j]))) <= fabsf(u[j]) * 0x1p-21f;
+        r[j] = rint_small(u[j]);
+        // near a half-integer: |u - r| >= 1/2 - |u| 2^-21 (one rounding of the
+        // threshold, far inside the factor-2 margin of the bound)
+        near |= fabsf(__fsub_rn(u[j], r[j])) >= __fmaf_rn(fabsf(u[j]), -0x1p-21f, 0.5f);
     }
     if (near) {
 #pragma unroll
         for (int j = 0; j < N; ++j) {
-            if (__fsub_rn(0.5f, fabsf(__fsub_rn(u[j], r[j]))) <= fabsf(u[j]) * 0x1p-21f) {
+            if (fabsf(__fsub_rn(u[j], r[j])) >= __fmaf_rn(fabsf(u[j]), -0x1p-21f, 0.5f)) {
                 u[j] = __fdiv_rn(w[j], s);
                 r[j] = rintf(u[j]);
             }

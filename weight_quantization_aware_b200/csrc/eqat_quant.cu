@@ -22,6 +22,9 @@ namespace {
 constexpr int kThreads = 256;
 constexpr int kBlocksPerSm = 8;
 
+// log2 of the group size (32, 64 or 128): index arithmetic by shifts, not division.
+inline int group_shift(int group) { return group == 32 ? 5 : group == 64 ? 6 : 7; }
+
 inline int grid_for(int64_t work_items, const DeviceInfo &dev, int per_thread = 1) {
     const int64_t threads = (work_items + per_thread - 1) / per_thread;
     const int64_t blocks = (threads + kThreads - 1) / kThreads;
@@ -110,7 +113,7 @@ __device__ __forceinline__ void fake_quant_chunk(const float (&w)[8], float sc, 
         const bool inside = (q >= 0.0f) && (q <= Q);
         const float c = fminf(fmaxf(q, 0.0f), Q);
         wh[j] = dequant_elem(c, zr, sc);
-        const uint32_t cb = static_cast<uint32_t>(c);
+        const uint32_t cb = CODES ? code_bits(c) : 0u;
         const uint32_t mb = inside ? 1u : 0u;
         if (j < 4) {
             c_lo |= cb << (8 * j);
@@ -130,7 +133,7 @@ __device__ __forceinline__ void fake_quant_chunk(const float (&w)[8], float sc, 
 template <typename T, typename O, bool CODES>
 __global__ void __launch_bounds__(kThreads, 4)
     k_fake_quant(const T *__restrict__ W, const float *__restrict__ s, const float *__restrict__ z,
-                 int64_t n_chunks, int group, float Q, O *__restrict__ W_hat,
+                 int64_t n_chunks, int gshift, float Q, O *__restrict__ W_hat,
                  uint8_t *__restrict__ code, uint8_t *__restrict__ mask) {
     constexpr int U = 2;
     const int64_t nthreads = static_cast<int64_t>(gridDim.x) * kThreads;
@@ -143,7 +146,7 @@ __global__ void __launch_bounds__(kThreads, 4)
             const int64_t i = base + u * nthreads;
             if (i < n_chunks) {
                 raw[u] = load_raw8<T>(W + i * 8);
-                const int64_t g = (i * 8) / group;
+                const int64_t g = (i * 8) >> gshift;
                 sc[u] = __ldg(s + g);
                 zr[u] = rintf(__ldg(z + g));
             }
@@ -175,7 +178,7 @@ __device__ __forceinline__ void pack_chunk(const float (&w)[16], float sc, float
         round_quotients<8>(*reinterpret_cast<const float(*)[8]>(&w[8 * h]), sc, rcp, r, u);
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
-            const uint32_t c = static_cast<uint32_t>(fminf(fmaxf(__fadd_rn(r[j], zr), 0.0f), Q));
+            const uint32_t c = code_bits(fminf(fmaxf(__fadd_rn(r[j], zr), 0.0f), Q));
             const int k = 8 * h + j;
             if (BITS == 2) word[0] |= c << (2 * k);
             else if (BITS == 4) word[k / 8] |= c << (4 * (k % 8));
@@ -198,7 +201,7 @@ __device__ __forceinline__ void pack_chunk(const float (&w)[16], float sc, float
 template <typename T, int BITS>
 __global__ void __launch_bounds__(kThreads, 4)
     k_pack(const T *__restrict__ W, const float *__restrict__ s, const float *__restrict__ z,
-           int64_t n_chunks, int group, float Q, uint8_t *__restrict__ codes,
+           int64_t n_chunks, int gshift, float Q, uint8_t *__restrict__ codes,
            uint8_t *__restrict__ zq) {
     constexpr int U = 2;
     const int64_t nthreads = static_cast<int64_t>(gridDim.x) * kThreads;
@@ -212,7 +215,7 @@ __global__ void __launch_bounds__(kThreads, 4)
             if (i < n_chunks) {
                 raw[u][0] = load_raw8<T>(W + i * 16);
                 raw[u][1] = load_raw8<T>(W + i * 16 + 8);
-                const int64_t g = (i * 16) / group;
+                const int64_t g = (i * 16) >> gshift;
                 sc[u] = __ldg(s + g);
                 zr[u] = fminf(fmaxf(rintf(__ldg(z + g)), 0.0f), Q);
             }
@@ -222,7 +225,7 @@ __global__ void __launch_bounds__(kThreads, 4)
             const int64_t i = base + u * nthreads;
             if (i < n_chunks) {
                 const int64_t e0 = i * 16;
-                if (e0 % group == 0) zq[e0 / group] = static_cast<uint8_t>(zr[u]);
+                if ((e0 & ((int64_t(1) << gshift) - 1)) == 0) zq[e0 >> gshift] = static_cast<uint8_t>(zr[u]);
                 float w[16];
                 unpack8(raw[u][0], *reinterpret_cast<float(*)[8]>(&w[0]));
                 unpack8(raw[u][1], *reinterpret_cast<float(*)[8]>(&w[8]));
@@ -257,12 +260,12 @@ __device__ __forceinline__ void unpack16(const uint8_t *codes, int64_t e0, uint3
 template <int BITS, typename O>
 __global__ void __launch_bounds__(kThreads)
     k_dequant(const uint8_t *__restrict__ codes, const uint8_t *__restrict__ zq,
-              const float *__restrict__ s, int64_t n_chunks, int group, O *__restrict__ W_hat) {
+              const float *__restrict__ s, int64_t n_chunks, int gshift, O *__restrict__ W_hat) {
     const int64_t stride = static_cast<int64_t>(gridDim.x) * kThreads;
     for (int64_t i = static_cast<int64_t>(blockIdx.x) * kThreads + threadIdx.x; i < n_chunks;
          i += stride) {
         const int64_t e0 = i * 16;
-        const int64_t g = e0 / group;
+        const int64_t g = e0 >> gshift;
         const float sc = __ldg(s + g);
         const float zf = static_cast<float>(__ldg(zq + g));
         uint32_t c[16];
@@ -293,13 +296,14 @@ cudaError_t minmax_dispatch(const T *W, int64_t n_groups, int group, float Q, fl
 template <typename T>
 cudaError_t pack_dispatch(const T *W, const float *s, const float *z, int64_t n, int bits, int group,
                           uint8_t *codes, uint8_t *zq, const DeviceInfo &dev, cudaStream_t st) {
+    const int gshift = group_shift(group);
     const int64_t chunks = n / 16;
     const int grid = grid_for(chunks, dev);
     const float Q = static_cast<float>((1 << bits) - 1);
     switch (bits) {
-        case 2: k_pack<T, 2><<<grid, kThreads, 0, st>>>(W, s, z, chunks, group, Q, codes, zq); break;
-        case 3: k_pack<T, 3><<<grid, kThreads, 0, st>>>(W, s, z, chunks, group, Q, codes, zq); break;
-        case 4: k_pack<T, 4><<<grid, kThreads, 0, st>>>(W, s, z, chunks, group, Q, codes, zq); break;
+        case 2: k_pack<T, 2><<<grid, kThreads, 0, st>>>(W, s, z, chunks, gshift, Q, codes, zq); break;
+        case 3: k_pack<T, 3><<<grid, kThreads, 0, st>>>(W, s, z, chunks, gshift, Q, codes, zq); break;
+        case 4: k_pack<T, 4><<<grid, kThreads, 0, st>>>(W, s, z, chunks, gshift, Q, codes, zq); break;
         default: return cudaErrorInvalidValue;
     }
     return cudaGetLastError();
@@ -309,12 +313,13 @@ template <typename O>
 cudaError_t dequant_dispatch(const uint8_t *codes, const uint8_t *zq, const float *s, int64_t n,
                              int bits, int group, O *W_hat, const DeviceInfo &dev,
                              cudaStream_t st) {
+    const int gshift = group_shift(group);
     const int64_t chunks = n / 16;
     const int grid = grid_for(chunks, dev);
     switch (bits) {
-        case 2: k_dequant<2, O><<<grid, kThreads, 0, st>>>(codes, zq, s, chunks, group, W_hat); break;
-        case 3: k_dequant<3, O><<<grid, kThreads, 0, st>>>(codes, zq, s, chunks, group, W_hat); break;
-        case 4: k_dequant<4, O><<<grid, kThreads, 0, st>>>(codes, zq, s, chunks, group, W_hat); break;
+        case 2: k_dequant<2, O><<<grid, kThreads, 0, st>>>(codes, zq, s, chunks, gshift, W_hat); break;
+        case 3: k_dequant<3, O><<<grid, kThreads, 0, st>>>(codes, zq, s, chunks, gshift, W_hat); break;
+        case 4: k_dequant<4, O><<<grid, kThreads, 0, st>>>(codes, zq, s, chunks, gshift, W_hat); break;
         default: return cudaErrorInvalidValue;
     }
     return cudaGetLastError();
@@ -341,14 +346,15 @@ cudaError_t launch_fake_quant(const void *W, bool w_f32, const float *s, const f
     const float Q = static_cast<float>((1 << bits) - 1);
     using bf = __nv_bfloat16;
     const bool codes = code || mask;
+    const int gshift = group_shift(group);
 #define EQAT_FQ_LAUNCH(TW, TO)                                                                          \
     do {                                                                                                \
         if (codes)                                                                                      \
             k_fake_quant<TW, TO, true><<<grid, kThreads, 0, st>>>(static_cast<const TW *>(W), s, z, chunks, \
-                                                                 group, Q, static_cast<TO *>(W_hat), code, mask); \
+                                                                 gshift, Q, static_cast<TO *>(W_hat), code, mask); \
         else                                                                                            \
             k_fake_quant<TW, TO, false><<<grid, kThreads, 0, st>>>(static_cast<const TW *>(W), s, z, chunks, \
-                                                                  group, Q, static_cast<TO *>(W_hat), code, mask); \
+                                                                  gshift, Q, static_cast<TO *>(W_hat), code, mask); \
     } while (0)
     if (w_f32 && out_f32)
         EQAT_FQ_LAUNCH(float, float);

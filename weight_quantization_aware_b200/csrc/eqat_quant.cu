@@ -104,27 +104,44 @@ template <typename T, typename O, bool CODES>
 __device__ __forceinline__ void fake_quant_chunk(const float (&w)[8], float sc, float zr, float Q,
                                                  int64_t e0, O *__restrict__ W_hat,
                                                  uint8_t *__restrict__ code, uint8_t *__restrict__ mask) {
-    float wh[8], r[8], u[8];
-    round_quotients<8>(w, sc, __frcp_rn(sc), r, u);
-    uint32_t c_lo = 0, c_hi = 0, m_lo = 0, m_hi = 0;
+    const float rcp = __frcp_rn(sc);
+    const float lo = kRoundMagic, hi = __fadd_rn(kRoundMagic, Q);
+    const float mz = __fadd_rn(kRoundMagic, zr);  // W-hat = (M + code - (M + zr)) s
+    float qm[8];
+    bool inside[8];
+    bool near = false;
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
-        const float q = __fadd_rn(r[j], zr);
-        const bool inside = (q >= 0.0f) && (q <= Q);
-        const float c = fminf(fmaxf(q, 0.0f), Q);
-        wh[j] = dequant_elem(c, zr, sc);
-        const uint32_t cb = CODES ? code_bits(c) : 0u;
-        const uint32_t mb = inside ? 1u : 0u;
-        if (j < 4) {
-            c_lo |= cb << (8 * j);
-            m_lo |= mb << (8 * j);
-        } else {
-            c_hi |= cb << (8 * (j - 4));
-            m_hi |= mb << (8 * (j - 4));
+        const float t = magic_decision(w[j], rcp, zr, near);  // M + round(u) + zr
+        inside[j] = (t >= lo) && (t <= hi);
+        qm[j] = fminf(fmaxf(t, lo), hi);
+    }
+    if (near) {
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            bool nj = false;
+            (void)magic_decision(w[j], rcp, zr, nj);
+            if (nj) qm[j] = exact_decision(w[j], sc, zr, Q, inside[j]);
         }
     }
+    float wh[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) wh[j] = __fmul_rn(__fsub_rn(qm[j], mz), sc);
     if (W_hat) store8<O>(W_hat + e0, wh);
     if (CODES) {
+        uint32_t c_lo = 0, c_hi = 0, m_lo = 0, m_hi = 0;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            const uint32_t cb = static_cast<uint32_t>(__float_as_int(qm[j])) & 0xFFu;
+            const uint32_t mb = inside[j] ? 1u : 0u;
+            if (j < 4) {
+                c_lo |= cb << (8 * j);
+                m_lo |= mb << (8 * j);
+            } else {
+                c_hi |= cb << (8 * (j - 4));
+                m_hi |= mb << (8 * (j - 4));
+            }
+        }
         if (code) *reinterpret_cast<uint2 *>(code + e0) = make_uint2(c_lo, c_hi);
         if (mask) *reinterpret_cast<uint2 *>(mask + e0) = make_uint2(m_lo, m_hi);
     }
@@ -171,26 +188,41 @@ template <int BITS>
 __device__ __forceinline__ void pack_chunk(const float (&w)[16], float sc, float zr, float Q, int64_t e0,
                                            uint8_t *__restrict__ codes) {
     const float rcp = __frcp_rn(sc);
+    const float lo = kRoundMagic, hi = __fadd_rn(kRoundMagic, Q);
+    // Each code enters its word as the raw bits of M + code (one multiply-add);
+    // the bits of M are taken out once per word at the end.
     uint32_t word[4] = {0u, 0u, 0u, 0u};  // 2-bit: word[0]; 4-bit: word[0..1]; 3-bit: word[0..3]
 #pragma unroll
-    for (int h = 0; h < 2; ++h) {  // two batches of 8 keep the rare division path small
-        float r[8], u[8];
-        round_quotients<8>(*reinterpret_cast<const float(*)[8]>(&w[8 * h]), sc, rcp, r, u);
+    for (int h = 0; h < 2; ++h) {
+        float cm[8];
+        bool near = false;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) cm[j] = fminf(fmaxf(magic_decision(w[8 * h + j], rcp, zr, near), lo), hi);
+        if (near) {
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                bool nj = false, inside;
+                (void)magic_decision(w[8 * h + j], rcp, zr, nj);
+                if (nj) cm[j] = exact_decision(w[8 * h + j], sc, zr, Q, inside);
+            }
+        }
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
-            const uint32_t c = code_bits(fminf(fmaxf(__fadd_rn(r[j], zr), 0.0f), Q));
+            const uint32_t b = static_cast<uint32_t>(__float_as_int(cm[j]));
             const int k = 8 * h + j;
-            if (BITS == 2) word[0] |= c << (2 * k);
-            else if (BITS == 4) word[k / 8] |= c << (4 * (k % 8));
-            else word[k / 4] |= c << (8 * (k % 4));
+            if (BITS == 2) word[0] += b << (2 * k);
+            else if (BITS == 4) word[k / 8] += b << (4 * (k % 8));
+            else word[k / 4] += b << (8 * (k % 4));
         }
     }
     if (BITS == 2) {
-        *reinterpret_cast<uint32_t *>(codes + e0 / 4) = word[0];
+        *reinterpret_cast<uint32_t *>(codes + e0 / 4) = word[0] - magic_word(2, 16);
     } else if (BITS == 4) {
-        *reinterpret_cast<uint2 *>(codes + e0 / 2) = make_uint2(word[0], word[1]);
+        *reinterpret_cast<uint2 *>(codes + e0 / 2) =
+            make_uint2(word[0] - magic_word(4, 8), word[1] - magic_word(4, 8));
     } else {
-        *reinterpret_cast<uint4 *>(codes + e0) = make_uint4(word[0], word[1], word[2], word[3]);
+        constexpr uint32_t m = magic_word(8, 4);
+        *reinterpret_cast<uint4 *>(codes + e0) = make_uint4(word[0] - m, word[1] - m, word[2] - m, word[3] - m);
     }
 }
 

@@ -95,6 +95,16 @@ struct SharedCtl {
     int abort_flag;
 };
 
+struct SharedCtl2 {
+    uint64_t full[6];
+    uint64_t empty[6];
+    uint64_t acc_full[2];
+    uint64_t acc_empty[2];
+    uint64_t drain;
+    uint32_t tmem_base;
+    int abort_flag;
+};
+
 // Problem index and tile coordinates of global tile t.
 __device__ __forceinline__ int tile_coords(const KParams &p, int t, int &tm, int &tn) {
     const int pi = (p.nprob > 1 && t >= p.pr[1].tile_begin) ? 1 : 0;
@@ -443,6 +453,232 @@ __global__ void __launch_bounds__((4 + EPI_WARPS) * 32, 1)
     }
 }
 
+// ---------------------------------------------------------------------------- CTA pairs
+// The same grouped GEMM on pairs of SMs (cta_group::2, cluster of two CTAs):
+// one tcgen05.mma covers a 256-row tile, each CTA stages its 128 rows of A and
+// half of the tile's B columns, the even CTA issues the MMAs, and each CTA's
+// tensor memory holds its 128 accumulator rows.  Per SM, a 256 x bn pair tile
+// reads a third less operand data from shared memory per FLOP than a 128 x bn
+// tile of one CTA (B is split between the two SMs), the limiter of the one-CTA
+// kernel.  Protocol:
+//   full[s]      the leader's: armed by the leader with both CTAs' bytes, completed
+//                by both CTAs' TMA loads (each into its own shared memory)
+//   empty[s]     each CTA's: the leader's MMA commit arrives on both (multicast)
+//   acc_full[a]  each CTA's: the leader's commit after a tile's last MMA (multicast)
+//   acc_empty[a] the leader's: both CTAs' epilogue threads arrive after draining
+constexpr int BM2 = 256;              // rows of a pair tile
+constexpr int STAGES2 = 6;
+constexpr int A_HALF = 128 * BK * 2;  // this CTA's 128 rows of A per stage
+constexpr int STAGE2_BYTES = A_HALF + 128 * BK * 2;  // + up to 128 rows of B
+constexpr int SMEM2_BYTES = 1024 + STAGES2 * STAGE2_BYTES + 256;
+
+template <int EPI0, int EPI1, int BITS, int EPI_WARPS>
+__global__ void __launch_bounds__((4 + EPI_WARPS) * 32, 1)
+    k_gemm_tc2(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUtensorMap tmB0,
+               const __grid_constant__ CUtensorMap tmA1, const __grid_constant__ CUtensorMap tmB1,
+               const KParams p) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                                ~static_cast<uintptr_t>(1023));
+    SharedCtl2 *ctl = reinterpret_cast<SharedCtl2 *>(smem + STAGES2 * STAGE2_BYTES);
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const uint32_t rank = cluster_rank();
+    const bool leader = rank == 0;
+    constexpr int EPI_THREADS = EPI_WARPS * 32;
+
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < STAGES2; ++i) {
+            mbar_init(&ctl->full[i], 1);
+            mbar_init(&ctl->empty[i], 1);
+        }
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&ctl->acc_full[i], 1);
+            mbar_init(&ctl->acc_empty[i], 2 * EPI_THREADS);
+        }
+        mbar_init(&ctl->drain, 1);
+        ctl->abort_flag = 0;
+        fence_mbarrier_init();
+        tma_prefetch_desc(&tmA0);
+        tma_prefetch_desc(&tmB0);
+        if (p.nprob > 1) {
+            tma_prefetch_desc(&tmA1);
+            tma_prefetch_desc(&tmB1);
+        }
+    }
+    if (warp == 2) {
+        tmem_alloc_pair(&ctl->tmem_base, TMEM_COLS);
+        tmem_relinquish_pair();
+    }
+    tc_fence_before();
+    cluster_sync();  // both CTAs' barriers are initialised and the pair's tensor memory is allocated
+    tc_fence_after();
+    const uint32_t tmem_base = ctl->tmem_base;
+    volatile int *abort_flag = &ctl->abort_flag;
+    const int pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
+    const uint32_t full0 = map_to_rank(&ctl->full[0], 0);           // the leader's full barriers
+    const uint32_t acc_empty0 = map_to_rank(&ctl->acc_empty[0], 0);  // the leader's accumulator-empty barriers
+
+    if (warp == 0) {
+        // ---------------------------------------------------------- TMA producer (both CTAs)
+        if (elect_one_sync()) {
+            uint32_t it = 0;
+            uint32_t armed = 0, armed_parity = 0;
+            bool ok = true;
+            for (int t = pair; ok && t < p.total_tiles; t += npairs) {
+                int tm, tn;
+                const int pi = tile_coords(p, t, tm, tn);
+                const CUtensorMap *ma = pi ? &tmA1 : &tmA0;
+                const CUtensorMap *mb = pi ? &tmB1 : &tmB0;
+                const int a_mn = pi ? p.pr[1].a_mn : p.pr[0].a_mn;
+                const int b_mn = pi ? p.pr[1].b_mn : p.pr[0].b_mn;
+                const int nkb = ((pi ? p.pr[1].GK : p.pr[0].GK) + BK - 1) / BK;
+                const int bn = pi ? p.pr[1].bn : p.pr[0].bn;
+                const int half = bn / 2;
+                const int m0 = tm * BM2 + 128 * static_cast<int>(rank);
+                const int n0 = tn * bn + half * static_cast<int>(rank);
+                for (int kb = 0; kb < nkb; ++kb, ++it) {
+                    const int st = it % STAGES2;
+                    const uint32_t ph = (it / STAGES2) & 1u;
+                    if (!mbar_wait_bounded(&ctl->empty[st], ph ^ 1u, abort_flag, p.err, p.wait_limit_ns)) {
+                        ok = false;
+                        break;
+                    }
+                    uint8_t *sa = smem + st * STAGE2_BYTES;
+                    uint8_t *sb = sa + A_HALF;
+                    if (leader) {
+                        mbar_arrive_expect_tx(&ctl->full[st], 2 * (A_HALF + half * BK * 2));
+                        armed |= 1u << st;
+                        armed_parity = (armed_parity & ~(1u << st)) | (ph << st);
+                    }
+                    const uint32_t bar = full0 + 8u * static_cast<uint32_t>(st);
+                    const int k0 = kb * BK;
+                    if (a_mn) {
+#pragma unroll
+                        for (int b = 0; b < 128 / MN_BOX; ++b)
+                            tma_load_2d_pair(sa + b * MN_BOX_BYTES, ma, bar, m0 + b * MN_BOX, k0);
+                    } else {
+                        tma_load_2d_pair(sa, ma, bar, k0, m0);
+                    }
+                    if (b_mn) {
+                        for (int b = 0; b < half / MN_BOX; ++b)
+                            tma_load_2d_pair(sb + b * MN_BOX_BYTES, mb, bar, n0 + b * MN_BOX, k0);
+                    } else {
+                        tma_load_2d_pair(sb, mb, bar, k0, n0);
+                    }
+                }
+            }
+            if (!ok) {
+                // Copies this CTA issued for stages the leader has not armed count on
+                // no phase that can complete: give them a fixed 2 ms to land.
+                const uint64_t t0 = globaltimer_ns();
+                while (globaltimer_ns() - t0 < 2000000ull) {
+                }
+            }
+            if (!ok && leader) {
+                // Let the pair's copies already issued land before the blocks exit.
+                for (int st = 0; st < STAGES2; ++st)
+                    if (armed & (1u << st)) {
+                        const uint32_t a = smem_u32(&ctl->full[st]);
+                        const uint64_t t0 = globaltimer_ns();
+                        while (!mbar_try_wait(a, (armed_parity >> st) & 1u) &&
+                               globaltimer_ns() - t0 < 100000000ull) {
+                        }
+                    }
+            }
+        }
+        __syncwarp();
+    } else if (warp == 1) {
+        // ---------------------------------------------------------- MMA issuer (the leader)
+        if (leader && elect_one_sync()) {
+            uint32_t it = 0, local = 0;
+            bool ok = true, issued = false;
+            for (int t = pair; ok && t < p.total_tiles; t += npairs, ++local) {
+                int tm, tn;
+                const int pi = tile_coords(p, t, tm, tn);
+                const int a_mn = pi ? p.pr[1].a_mn : p.pr[0].a_mn;
+                const int b_mn = pi ? p.pr[1].b_mn : p.pr[0].b_mn;
+                const int nkb = ((pi ? p.pr[1].GK : p.pr[0].GK) + BK - 1) / BK;
+                const int bn = pi ? p.pr[1].bn : p.pr[0].bn;
+                const uint32_t idesc = idesc_bf16_f32(BM2, bn, a_mn != 0, b_mn != 0);
+                const uint32_t a_step = a_mn ? UK * 128 : UK * 2, a_lbo = a_mn ? MN_BOX_BYTES : 16;
+                const uint32_t b_step = b_mn ? UK * 128 : UK * 2, b_lbo = b_mn ? MN_BOX_BYTES : 16;
+                const uint32_t acc = local & 1u;
+                const uint32_t aph = (local >> 1) & 1u;
+                if (!mbar_wait_bounded(&ctl->acc_empty[acc], aph ^ 1u, abort_flag, p.err, p.wait_limit_ns)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t d_tmem = tmem_base + acc * ACC_COLS;
+                for (int kb = 0; kb < nkb; ++kb, ++it) {
+                    const int st = it % STAGES2;
+                    const uint32_t ph = (it / STAGES2) & 1u;
+                    if (!mbar_wait_bounded(&ctl->full[st], ph, abort_flag, p.err, p.wait_limit_ns)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t sa = smem_u32(smem + st * STAGE2_BYTES);
+                    const uint32_t sb = sa + A_HALF;
+#pragma unroll
+                    for (int kk = 0; kk < BK / UK; ++kk) {
+                        const uint64_t ad = smem_desc_sw128(sa + kk * a_step, a_lbo, 1024);
+                        const uint64_t bd = smem_desc_sw128(sb + kk * b_step, b_lbo, 1024);
+                        tc_mma_f16_pair(d_tmem, ad, bd, idesc, (kb > 0 || kk > 0) ? 1u : 0u);
+                    }
+                    issued = true;
+                    tc_commit_pair(&ctl->empty[st], 0x3);
+                }
+                if (!ok) break;
+                tc_commit_pair(&ctl->acc_full[acc], 0x3);
+            }
+            if (!ok && issued) {
+                tc_commit_pair(&ctl->drain, 0x1);
+                const uint32_t a = smem_u32(&ctl->drain);
+                const uint64_t t0 = globaltimer_ns();
+                while (!mbar_try_wait(a, 0) && globaltimer_ns() - t0 < 100000000ull) {
+                }
+            }
+        }
+        __syncwarp();
+    } else if (warp >= 4) {
+        // ---------------------------------------------------------- epilogue (both CTAs)
+        const int ew = warp - 4;
+        const int quad = warp & 3;
+        const int half_slice = ew >> 2;
+        constexpr int SLICES = EPI_WARPS / 4;
+        uint32_t local = 0;
+        for (int t = pair; t < p.total_tiles; t += npairs, ++local) {
+            const uint32_t acc = local & 1u;
+            const uint32_t aph = (local >> 1) & 1u;
+            const bool ok = mbar_wait_bounded(&ctl->acc_full[acc], aph, abort_flag, p.err, p.wait_limit_ns);
+            if (!__all_sync(0xffffffffu, ok)) break;
+            tc_fence_after();
+            int tm, tn;
+            const int pi = tile_coords(p, t, tm, tn);
+            const int row = tm * BM2 + 128 * static_cast<int>(rank) + quad * 32 + lane;
+            const uint32_t taddr = tmem_base + acc * ACC_COLS + ((quad * 32) << 16);
+            const int bn = pi ? p.pr[1].bn : p.pr[0].bn;
+            const int cols = bn / SLICES;
+            if (pi == 0)
+                drain_accumulator<EPI0, BITS>(p.pr[0], taddr, row, tn * bn, half_slice * cols, (half_slice + 1) * cols);
+            else
+                drain_accumulator<EPI1, BITS>(p.pr[1], taddr, row, tn * bn, half_slice * cols, (half_slice + 1) * cols);
+            tc_fence_before();
+            mbar_arrive_cluster(acc_empty0 + 8u * acc);
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    cluster_sync();  // neither CTA leaves while the pair's MMAs may still read its shared memory
+    if (warp == 2) {
+        tc_fence_after();
+        tmem_dealloc_pair(tmem_base, TMEM_COLS);
+    }
+}
+
 // ---------------------------------------------------------------------------- host side
 
 PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
@@ -503,24 +739,64 @@ cudaError_t launch_variant(const CUtensorMap (&maps)[4], const KParams &p, int g
     return cudaGetLastError();
 }
 
+template <int EPI0, int EPI1, int BITS>
+cudaError_t launch_pair_variant(const CUtensorMap (&maps)[4], const KParams &p, int grid, int dev_id,
+                                cudaStream_t st) {
+    auto kern = k_gemm_tc2<EPI0, EPI1, BITS, kEpiWarps>;
+    static std::atomic<uint64_t> done{0};
+    const uint64_t bit = 1ull << (dev_id & 63);
+    if (!(done.load() & bit)) {
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM2_BYTES);
+        if (e != cudaSuccess) return e;
+        done.fetch_or(bit);
+    }
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(grid), 1, 1);
+    cfg.blockDim = dim3((4 + kEpiWarps) * 32, 1, 1);
+    cfg.dynamicSmemBytes = SMEM2_BYTES;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    // Persistent pairs: no more clusters than can be resident at once.
+    static std::atomic<int> resident[64];
+    int n = resident[dev_id & 63].load();
+    if (n == 0) {
+        cudaError_t e = cudaOccupancyMaxActiveClusters(&n, kern, &cfg);
+        if (e != cudaSuccess) return e;
+        if (n <= 0) return cudaErrorInvalidConfiguration;
+        resident[dev_id & 63].store(n);
+    }
+    cfg.gridDim.x = static_cast<unsigned>(std::min(grid, 2 * n));
+    return cudaLaunchKernelEx(&cfg, kern, maps[0], maps[1], maps[2], maps[3], p);
+}
+
 int *device_error_ptr() {
     int *ptr = nullptr;
     if (cudaGetSymbolAddress(reinterpret_cast<void **>(&ptr), g_dev_error) != cudaSuccess) return nullptr;
     return ptr;
 }
 
-cudaError_t fill_prob(Prob &q, const GemmProblem &g, int tile_begin, int bn, CUtensorMap &ma, CUtensorMap &mb) {
+// tile_m: rows of an output tile (128 for one CTA, 256 for a CTA pair, where each
+// CTA loads 128 rows of A and bn / 2 rows of B).
+cudaError_t fill_prob(Prob &q, const GemmProblem &g, int tile_begin, int bn, int tile_m, CUtensorMap &ma,
+                      CUtensorMap &mb) {
     const int64_t GM = g.GM, GN = g.GN, GK = g.GK;
     if (GM <= 0 || GN <= 0 || GK <= 0) return cudaErrorInvalidValue;
-    if (GM > INT32_MAX - BM || GN > INT32_MAX - BN || GK > INT32_MAX - BK) return cudaErrorInvalidValue;
+    if (GM > INT32_MAX - BM2 || GN > INT32_MAX - BN || GK > INT32_MAX - BK) return cudaErrorInvalidValue;
     cudaError_t e;
+    const bool pair = tile_m == BM2;
     if ((e = make_map(ma, g.A, GM, GK, BM)) != cudaSuccess) return e;
-    if ((e = make_map(mb, g.B, GN, GK, bn)) != cudaSuccess) return e;
+    if ((e = make_map(mb, g.B, GN, GK, pair ? bn / 2 : bn)) != cudaSuccess) return e;
     q = Prob{};
     q.GM = static_cast<int>(GM);
     q.GN = static_cast<int>(GN);
     q.GK = static_cast<int>(GK);
-    q.tiles_m = static_cast<int>((GM + BM - 1) / BM);
+    q.tiles_m = static_cast<int>((GM + tile_m - 1) / tile_m);
     q.tiles_n = static_cast<int>((GN + bn - 1) / bn);
     q.bn = bn;
     q.tile_begin = tile_begin;
@@ -546,35 +822,59 @@ cudaError_t fill_prob(Prob &q, const GemmProblem &g, int tile_begin, int bn, CUt
     return cudaSuccess;
 }
 
-// N-tile width for a launch.  A 128-wide tile does half the work of a 256-wide
-// one at a somewhat lower tensor-pipe efficiency (more operand traffic per FLOP),
-// but halves the granularity of the last wave.  Estimated time = waves x tile cost;
-// the narrower tile wins when it removes enough of a partial last wave.  Group
+struct Tiling {
+    bool pair;  // 256-row tiles on CTA pairs, else 128-row tiles on one CTA
+    int bn;     // N-tile width, 128 or 256
+};
+
+// Tile shape for a launch, from a wave model: estimated time = waves x the time
+// one wave of that shape takes, relative to a wave of 128 x 256 tiles on single
+// CTAs.  Measured on B200 (4096^3 forward, CUDA events):
+//   one CTA,  128 x 128: 0.72  (42% more time per FLOP: operand bytes per FLOP
+//                               read from shared memory)
+//   CTA pair, 256 x 256: 0.89  (B split over the two SMs: a third fewer operand
+//                               bytes per FLOP; the same per-SM work per wave)
+//   CTA pair, 256 x 128: 0.89 x 0.66 (0.64-0.69 of a 256 x 256 pair wave on four shapes)
+// A pair covers 256 rows, so concurrent tiles are half the SM count.  Group
 // reductions need a whole group inside one epilogue slice (bn / 2 columns).
-// EQAT_GEMM_BN=128|256 forces a width (measurement aid).
-int choose_bn(const GemmProblem *probs, int nprob, int sms) {
+// EQAT_GEMM_BN=128|256 and EQAT_GEMM_PAIR=0|1 force a choice (measurement aid).
+Tiling choose_tiling(const GemmProblem *probs, int nprob, int sms) {
     bool narrow_ok = true;
     for (int i = 0; i < nprob; ++i)
         if (probs[i].epi.kind != Epi::kStore && probs[i].epi.group > 64) narrow_ok = false;
-    static const int forced = [] {
+    static const int forced_bn = [] {
         const char *v = std::getenv("EQAT_GEMM_BN");
         return v ? std::atoi(v) : 0;
     }();
-    if (forced == 256) return 256;
-    if (forced == 128 && narrow_ok) return 128;
-    if (!narrow_ok) return 256;
-    auto estimate = [&](int bn, double tile_cost) {
+    static const int forced_pair = [] {
+        const char *v = std::getenv("EQAT_GEMM_PAIR");
+        return v ? std::atoi(v) : -1;
+    }();
+    auto estimate = [&](bool pair, int bn) {
+        const int64_t tile_m = pair ? BM2 : BM;
+        const int64_t units = pair ? sms / 2 : sms;
         int64_t tiles = 0;
         for (int i = 0; i < nprob; ++i)
-            tiles += ((probs[i].GM + BM - 1) / BM) * ((probs[i].GN + bn - 1) / bn);
-        const int64_t waves = (tiles + sms - 1) / sms;
-        return static_cast<double>(waves) * tile_cost;
+            tiles += ((probs[i].GM + tile_m - 1) / tile_m) * ((probs[i].GN + bn - 1) / bn);
+        const int64_t waves = (tiles + units - 1) / units;
+        const double cost = pair ? (bn == 256 ? 0.89 : 0.89 * 0.66) : (bn == 256 ? 1.0 : 0.72);
+        return static_cast<double>(waves) * cost;
     };
-    // Measured on B200 (4096^3 forward, bench.py): a wave of 128-wide tiles takes
-    // 0.71 of a wave of 256-wide ones, i.e. 42% more time per FLOP, in line with
-    // the operand bytes per FLOP the tensor core reads from shared memory.
-    constexpr double kNarrowTileCost = 0.72;
-    return estimate(128, kNarrowTileCost) < estimate(256, 1.0) ? 128 : 256;
+    Tiling best{false, 256};
+    double best_t = 1e300;
+    for (int pair = 0; pair < 2; ++pair) {
+        if (forced_pair >= 0 && pair != (forced_pair != 0)) continue;
+        for (int bn = 256; bn >= 128; bn -= 128) {
+            if (bn == 128 && (!narrow_ok || forced_bn == 256)) continue;
+            if (bn == 256 && forced_bn == 128 && narrow_ok) continue;
+            const double t = estimate(pair != 0, bn);
+            if (t < best_t) {
+                best_t = t;
+                best = Tiling{pair != 0, bn};
+            }
+        }
+    }
+    return best;
 }
 
 }  // namespace
@@ -593,9 +893,14 @@ cudaError_t launch_gemm_tc_group(const GemmProblem *probs, int nprob, const Devi
     CUtensorMap maps[4];
     KParams p{};
     int tiles = 0;
-    const int bn = choose_bn(probs, nprob, dev.sm_count);
+    const Tiling tiling = choose_tiling(probs, nprob, dev.sm_count);
+    const bool pair = tiling.pair;
+    const int tile_m = pair ? BM2 : BM;
+    const int units = pair ? dev.sm_count / 2 : dev.sm_count;  // concurrent tiles
+    const int bn = tiling.bn;
     for (int i = 0; i < nprob; ++i) {
-        if ((e = fill_prob(p.pr[i], probs[i], tiles, bn, maps[2 * i], maps[2 * i + 1])) != cudaSuccess) return e;
+        if ((e = fill_prob(p.pr[i], probs[i], tiles, bn, tile_m, maps[2 * i], maps[2 * i + 1])) != cudaSuccess)
+            return e;
         const int64_t t = static_cast<int64_t>(p.pr[i].tiles_m) * p.pr[i].tiles_n;
         if (tiles + t > INT32_MAX) return cudaErrorInvalidValue;
         tiles += static_cast<int>(t);
@@ -609,6 +914,24 @@ cudaError_t launch_gemm_tc_group(const GemmProblem *probs, int nprob, const Devi
     p.err = device_error_ptr();
     if (!p.err) return cudaErrorInvalidSymbol;
     p.wait_limit_ns = kWaitLimitNs;
+    if (pair) {
+        const int grid = 2 * std::min(tiles, units);
+        switch (probs[0].epi.kind) {
+            case Epi::kStore:
+                if (nprob > 1) return cudaErrorInvalidValue;
+                return launch_pair_variant<0, 0, 2>(maps, p, grid, dev.device, st);
+            case Epi::kFqGrad:
+                return launch_pair_variant<1, 0, 2>(maps, p, grid, dev.device, st);
+            case Epi::kE2eDs:
+                switch (probs[0].epi.bits) {
+                    case 2: return launch_pair_variant<2, 0, 2>(maps, p, grid, dev.device, st);
+                    case 3: return launch_pair_variant<2, 0, 3>(maps, p, grid, dev.device, st);
+                    case 4: return launch_pair_variant<2, 0, 4>(maps, p, grid, dev.device, st);
+                    default: return cudaErrorInvalidValue;
+                }
+        }
+        return cudaErrorInvalidValue;
+    }
     const int grid = std::min(tiles, dev.sm_count);
     switch (probs[0].epi.kind) {
         case Epi::kStore:

@@ -64,6 +64,8 @@ def _load():
             "orc_linear_dwhat": [P, P, I64, I64, I64, P, I64, P],
             "orc_ste_grads": [P, P, P, P, P, I64, I64, I64, I, I, P, P, P],
             "orc_e2e_ds": [P, P, P, P, I64, I64, I64, I, I, P],
+            "orc_ste_grads_clamp_pass": [P, P, P, P, P, I64, I64, I64, I, I, P, P, P],
+            "orc_e2e_dz": [P, P, P, I64, I64, I64, I, P],
         }
         for name, args in sig.items():
             fn = getattr(lib, name)
@@ -141,6 +143,8 @@ def pack(W, s, z, bits, group):
 
 
 def dequant_packed(packed, zq, s, K, bits, group):
+    """W-hat = (W_q - zq) s in fp32.  s may be float16 (the pages' fp16 step-size
+    storage); widening it to fp32 is exact."""
     packed = np.ascontiguousarray(packed, dtype=np.uint8)
     zq = np.ascontiguousarray(zq, dtype=np.uint8)
     s = _f32(s)
@@ -181,8 +185,9 @@ def linear_dwhat(dY, X, wrows=None):
     return out
 
 
-def ste_grads(W, s, z, dWhat, bits, group, wrows=None):
-    """Block-AP straight-through grads for the weight rows `wrows` (rows of dWhat)."""
+def ste_grads(W, s, z, dWhat, bits, group, wrows=None, clamp_pass=False):
+    """Block-AP straight-through grads for the weight rows `wrows` (rows of dWhat).
+    clamp_pass=True: the clamp is straight-through as well (all-pass variant)."""
     W, s, z = _f32(W), _f32(s), _f32(z)
     dWhat = np.ascontiguousarray(dWhat, dtype=np.float64)
     N, K = W.shape
@@ -194,8 +199,8 @@ def ste_grads(W, s, z, dWhat, bits, group, wrows=None):
     dW = np.empty((n_out, K), np.float64)
     ds = np.empty((n_out, G), np.float64)
     dz = np.empty((n_out, G), np.float64)
-    _load().orc_ste_grads(_p(W), _p(s), _p(z), _p(dWhat), _p(r), nr, N, K, bits, group,
-                          _p(dW), _p(ds), _p(dz))
+    fn = _load().orc_ste_grads_clamp_pass if clamp_pass else _load().orc_ste_grads
+    fn(_p(W), _p(s), _p(z), _p(dWhat), _p(r), nr, N, K, bits, group, _p(dW), _p(ds), _p(dz))
     return dW, ds, dz
 
 
@@ -213,6 +218,20 @@ def e2e_ds(packed, zq, dWhat, K, bits, group, wrows=None):
     return ds
 
 
+def e2e_dz(s, dWhat, K, group, wrows=None):
+    """E2E-QP zero-point gradient dz = -s * sum_group dW-hat (z trained as a float)."""
+    s = _f32(s)
+    dWhat = np.ascontiguousarray(dWhat, dtype=np.float64)
+    N = s.shape[0]
+    _check(N, K, 2, group)
+    r, nr = _rows(wrows)
+    n_out = N if r is None else nr
+    assert dWhat.shape == (n_out, K)
+    dz = np.empty((n_out, K // group), np.float64)
+    _load().orc_e2e_dz(_p(s), _p(dWhat), _p(r), nr, N, K, group, _p(dz))
+    return dz
+
+
 # ----------------------------------------------------------------------------
 # The layer, step by step in the pages' order.
 # ----------------------------------------------------------------------------
@@ -223,12 +242,12 @@ def fq_linear_fwd(X, W, s, z, bits, group, rows=None):
     return linear_fwd(X, wh, rows)
 
 
-def fq_linear_bwd(X, W, s, z, dY, bits, group, rows=None, wrows=None):
+def fq_linear_bwd(X, W, s, z, dY, bits, group, rows=None, wrows=None, clamp_pass=False):
     """Block-AP backward: dX (token rows `rows`), dW, ds, dz (weight rows `wrows`)."""
     wh = fake_quant(W, s, z, bits, group)[0]
     dX = linear_dx(dY, wh, rows)
     dwh = linear_dwhat(dY, X, wrows)
-    dW, ds, dz = ste_grads(W, s, z, dwh, bits, group, wrows)
+    dW, ds, dz = ste_grads(W, s, z, dwh, bits, group, wrows, clamp_pass=clamp_pass)
     return dX, dW, ds, dz
 
 
@@ -240,9 +259,18 @@ def dq_linear_fwd(X, packed, zq, s, bits, group, rows=None):
 
 def dq_linear_bwd_s(X, packed, zq, s, dY, bits, group, rows=None, wrows=None):
     """E2E-QP backward: dX (token rows `rows`) and ds (weight rows `wrows`)."""
+    dX, ds, _ = dq_linear_bwd(X, packed, zq, s, dY, bits, group, rows, wrows)
+    return dX, ds
+
+
+def dq_linear_bwd(X, packed, zq, s, dY, bits, group, rows=None, wrows=None):
+    """E2E-QP backward with the zero-point gradient: dX (token rows `rows`), ds and
+    dz (weight rows `wrows`).  s may be float16 (fp16 step-size storage); widening
+    it to fp32 is exact."""
     K = np.asarray(X).shape[1]
     wh = dequant_packed(packed, zq, s, K, bits, group)
     dX = linear_dx(dY, wh, rows)
     dwh = linear_dwhat(dY, X, wrows)
     ds = e2e_ds(packed, zq, dwh, K, bits, group, wrows)
-    return dX, ds
+    dz = e2e_dz(s, dwh, K, group, wrows)
+    return dX, ds, dz

@@ -33,6 +33,9 @@
  *   z during Block-AP  = a float that is rounded (zr = rint(z)) in every forward;
  *   clamp gradient     = passes only where 0 <= round(W/s) + zr <= 2^N - 1
  *                        (inclusive bounds); round has identity gradient;
+ *                        orc_ste_grads_clamp_pass is the all-pass variant;
+ *   E2E zero point     = dz of W-hat = (W_q - z) s at z = zq (z as a float);
+ *   fp16 step storage  = s widened exactly to fp32 before any arithmetic;
  *   pack               = zq = clamp(rint(z), 0, Q) as uint8, codes recomputed
  *                        with zr := zq; 2-bit: 4 codes per byte, code k at bits
  *                        2*(k%4); 4-bit: 2 per byte at bits 4*(k%2); 3-bit: one
@@ -296,6 +299,63 @@ void orc_e2e_ds(const uint8_t *packed, const uint8_t *zq, const double *dWhat,
                 acc += dWhat[r * K + k] * diff;
             }
             ds[r * G + j] = acc;
+        }
+    }
+}
+
+/* Variant of orc_ste_grads in which the clamp is straight-through as well (the
+ * all-pass clamp_ste that [MF] "Paper vs. code" finds defined in the quantizer
+ * but whose use the pages leave unstated).  With round and clamp both identity
+ * in the backward pass, W-hat = (clamp(round(W/s) + zr, 0, Q) - zr) s gives
+ *   dW-hat/dW  = (1/s) s                  = 1,
+ *   dW-hat/ds  = (c - zr) + s (-W / s^2)  = (c - zr) - u,
+ *   dW-hat/dzr = s (1 - 1)                = 0,
+ * for every element, clamped or not. */
+void orc_ste_grads_clamp_pass(const float *W, const float *s, const float *z, const double *dWhat,
+                              const int64_t *wrows, int64_t nw, int64_t N, int64_t K, int bits,
+                              int group, double *dW, double *ds, double *dz)
+{
+    const int64_t G = K / group;
+    const float Q = orc_qmax(bits);
+    if (!wrows) nw = N;
+#pragma omp parallel for schedule(static)
+    for (int64_t r = 0; r < nw; ++r) {
+        const int64_t n = wrows ? wrows[r] : r;
+        for (int64_t j = 0; j < G; ++j) {
+            const float sc = s[n * G + j];
+            const float zr = rintf(z[n * G + j]);
+            double acc_s = 0.0;
+            for (int i = 0; i < group; ++i) {
+                const int64_t k = j * group + i;
+                const float u = W[n * K + k] / sc;
+                float c = rintf(u) + zr;
+                if (c < 0.0f) c = 0.0f;
+                if (c > Q) c = Q;
+                const double g = dWhat[r * K + k];
+                if (dW) dW[r * K + k] = g;
+                acc_s += g * ((double)(c - zr) - (double)u);
+            }
+            if (ds) ds[r * G + j] = acc_s;
+            if (dz) dz[r * G + j] = 0.0;
+        }
+    }
+}
+
+/* E2E-QP with the zero point trained too (a float z evaluated at the frozen zq):
+ * W-hat = (W_q - z) s ([ZN] Eq. 2, [MF] Phase 2) is linear in z with
+ * dW-hat/dz = -s, so dz[n,j] = -s[n,j] * sum_{k in j} dWhat[n,k]. */
+void orc_e2e_dz(const float *s, const double *dWhat, const int64_t *wrows, int64_t nw, int64_t N,
+                int64_t K, int group, double *dz)
+{
+    const int64_t G = K / group;
+    if (!wrows) nw = N;
+#pragma omp parallel for schedule(static)
+    for (int64_t r = 0; r < nw; ++r) {
+        const int64_t n = wrows ? wrows[r] : r;
+        for (int64_t j = 0; j < G; ++j) {
+            double acc = 0.0;
+            for (int i = 0; i < group; ++i) acc += dWhat[r * K + j * group + i];
+            dz[r * G + j] = -(double)s[n * G + j] * acc;
         }
     }
 }

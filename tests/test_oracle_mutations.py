@@ -33,6 +33,13 @@ MUTANTS = {
     "dx_transposed_operand": ("out[k] += g * (double)What[n * K + k];",
                               "out[k] += g * (double)What[(k % N) * K + (n % K)];"),
     "round_half_away": ("const float r = rintf(u);", "const float r = roundf(u);"),
+    "clamp_pass_drops_u_term": ("acc_s += g * ((double)(c - zr) - (double)u);",
+                                "acc_s += g * (double)(c - zr);"),
+    "clamp_pass_masks_dw": ("if (dW) dW[r * K + k] = g;",
+                            "if (dW) dW[r * K + k] = (c == rintf(u) + zr) ? g : 0.0;"),
+    "e2e_dz_wrong_sign": ("dz[r * G + j] = -(double)s[n * G + j] * acc;",
+                          "dz[r * G + j] = (double)s[n * G + j] * acc;"),
+    "e2e_dz_drops_scale": ("dz[r * G + j] = -(double)s[n * G + j] * acc;", "dz[r * G + j] = -acc;"),
     "e2e_ds_ignores_zero_point": ("const double diff = (double)orc_code_at(packed, K, bits, n, k) - (double)zq[n * G + j];",
                                   "const double diff = (double)orc_code_at(packed, K, bits, n, k);"),
 }

@@ -292,7 +292,19 @@ class _RoundSTE(torch.autograd.Function):
         return grad, None
 
 
-def _surrogate_torch(X, W, s, z, dY, bits, g):
+class _ClampSTE(torch.autograd.Function):
+    """clamp_ste: the value of clamp, the gradient of the identity."""
+
+    @staticmethod
+    def forward(ctx, x, lo, hi):
+        return torch.clamp(x, lo, hi)
+
+    @staticmethod
+    def backward(ctx, grad):
+        return grad, None, None
+
+
+def _surrogate_torch(X, W, s, z, dY, bits, g, clamp_pass=False):
     """Independent autograd re-derivation of Eq. 1-2 with round_ste on both round(W/s)
     and round(z), and torch.clamp (whose own backward passes the gradient only inside
     [0, Q], bounds included), in fp64.  The rounded values come from fp32 arithmetic
@@ -307,7 +319,7 @@ def _surrogate_torch(X, W, s, z, dY, bits, g):
     srep = st.repeat_interleave(g, dim=1)
     zr = _RoundSTE.apply(zt, zr_val).repeat_interleave(g, dim=1)
     q = _RoundSTE.apply(Wt / srep, r) + zr
-    c = torch.clamp(q, 0, Q)
+    c = _ClampSTE.apply(q, 0, Q) if clamp_pass else torch.clamp(q, 0, Q)
     wh = (c - zr) * srep
     Xt = torch.tensor(X, dtype=torch.float64, requires_grad=True)
     Y = Xt @ wh.T
@@ -424,6 +436,95 @@ def test_ste_no_clamping_special_case(orc):
     np.testing.assert_allclose(ds, ref, rtol=1e-9, atol=1e-12)
 
 
+# ---------------------------------------------------------------- all-pass clamp variant
+
+@pytest.mark.parametrize("bits,g", [(2, 4), (3, 8), (4, 16)])
+def test_clamp_pass_backward_matches_autograd_rederivation(orc, bits, g):
+    """With the clamp straight-through too (clamp_ste), autograd of Eq. 1-2 gives
+    dW = dW-hat everywhere, dz = 0, ds = sum dW-hat ((c - zr) - u)."""
+    rng = np.random.default_rng(31 + bits)
+    M, N, K = 3, 6, 4 * g
+    X = rng.standard_normal((M, K)).astype(np.float32)
+    dY = rng.standard_normal((M, N)).astype(np.float32)
+    W = rand_w(N, K, 37 + g)
+    s, z = orc.minmax_init(W, bits, g)
+    s, z = synthetic.perturb_quant_params(s, z, seed=g + 1)
+    _, _, mask, u = orc.fake_quant(W, s, z, bits, g)
+    assert 0 < mask.mean() < 1, "the case must clamp some weights"
+    _, dX_ref, dW_ref, ds_ref, dz_ref = _surrogate_torch(X, W, s, z, dY, bits, g, clamp_pass=True)
+    dX, dW, ds, dz = orc.fq_linear_bwd(X, W, s, z, dY, bits, g, clamp_pass=True)
+    np.testing.assert_allclose(dX, dX_ref, rtol=1e-5, atol=1e-6)
+    np.testing.assert_allclose(dW, dW_ref, rtol=1e-12, atol=1e-12)
+    dwh = dY.astype(np.float64).T @ X.astype(np.float64)
+    bound = (np.abs(dwh) * np.abs(u.astype(np.float64)) * 2.0 ** -23).reshape(N, -1, g).sum(-1)
+    assert (np.abs(ds - ds_ref) <= bound + 1e-12).all()
+    np.testing.assert_allclose(dz_ref, 0.0, atol=1e-12)
+    assert (dz == 0).all()
+    # the variant differs from the default convention exactly on the clamped weights
+    _, dW0, ds0, _ = orc.fq_linear_bwd(X, W, s, z, dY, bits, g)
+    assert (dW0[mask == 1] == dW[mask == 1]).all() and (dW0[mask == 0] == 0).all()
+    assert np.abs(ds - ds0).max() > 0
+
+
+def test_clamp_pass_matches_finite_differences_of_frozen_offset_surrogate(orc):
+    """What the all-pass variant differentiates: W-hat = (W/s + delta + zr + eps - zr) s
+    with the rounding offset delta and the clamp offset eps = clamp(q0) - q0 frozen at
+    the base point.  The surrogate is linear in W and z and smooth in s, so central
+    differences pin every weight and every group, on the clamp kinks too."""
+    bits, g, Q = 2, 4, 3
+    rng = np.random.default_rng(9)
+    M, N, K = 2, 16, 16
+    X = rng.standard_normal((M, K)).astype(np.float32)
+    dY = rng.standard_normal((M, N)).astype(np.float32)
+    W = rand_w(N, K, 43)
+    s, z = orc.minmax_init(W, bits, g)
+    s, z = synthetic.perturb_quant_params(s, z, seed=43)
+    u32 = (W / np.repeat(s, g, 1)).astype(np.float32)
+    delta = (np.rint(u32) - u32).astype(np.float64)
+    zr0 = np.rint(z).astype(np.float64)
+    q0 = np.rint(u32).astype(np.float64) + np.repeat(zr0, g, 1)
+    eps = np.clip(q0, 0, Q) - q0
+    assert (eps != 0).any()
+    X64, dY64 = X.astype(np.float64), dY.astype(np.float64)
+
+    def loss(Wv, sv, zv):
+        srep = np.repeat(sv, g, 1)
+        zr = np.repeat(zv - z.astype(np.float64) + zr0, g, 1)
+        wh = (Wv / srep + delta + zr + eps - zr) * srep
+        return float(np.sum(dY64 * (X64 @ wh.T)))
+
+    _, dW, ds, dz = orc.fq_linear_bwd(X, W, s, z, dY, bits, g, clamp_pass=True)
+    W64, s64, z64 = W.astype(np.float64), s.astype(np.float64), z.astype(np.float64)
+    h = 1e-7
+    for n, k in [(n, k) for n in range(N) for k in range(0, K, 3)]:
+        e = np.zeros_like(W64); e[n, k] = h
+        fd = (loss(W64 + e, s64, z64) - loss(W64 - e, s64, z64)) / (2 * h)
+        assert abs(fd - dW[n, k]) <= 1e-6 * max(1.0, abs(fd))
+    for n in range(N):
+        for j in range(K // g):
+            hs = 1e-7 * s64[n, j]
+            e = np.zeros_like(s64); e[n, j] = hs
+            fd = (loss(W64, s64 + e, z64) - loss(W64, s64 - e, z64)) / (2 * hs)
+            assert abs(fd - ds[n, j]) <= 1e-5 * max(1.0, abs(fd))
+            e = np.zeros_like(z64); e[n, j] = h
+            fd = (loss(W64, s64, z64 + e) - loss(W64, s64, z64 - e)) / (2 * h)
+            assert abs(fd - dz[n, j]) <= 1e-6
+
+
+def test_clamp_pass_equals_default_when_nothing_is_clamped(orc):
+    rng = np.random.default_rng(5)
+    M, N, K, g, bits = 4, 8, 128, 32, 3
+    X = rng.standard_normal((M, K)).astype(np.float32)
+    dY = rng.standard_normal((M, N)).astype(np.float32)
+    W = rand_w(N, K, 5)
+    s, z = orc.minmax_init(W, bits, g)
+    assert orc.fake_quant(W, s, z, bits, g)[2].all()
+    a = orc.fq_linear_bwd(X, W, s, z, dY, bits, g)
+    b = orc.fq_linear_bwd(X, W, s, z, dY, bits, g, clamp_pass=True)
+    for x, y in zip(a, b):
+        assert (x == y).all()
+
+
 # ---------------------------------------------------------------- E2E-QP
 
 def test_e2e_ds_is_exact_gradient_finite_differences(orc):
@@ -455,6 +556,55 @@ def test_e2e_ds_is_exact_gradient_finite_differences(orc):
     wh = orc.dequant_packed(packed, zq, s, K, bits, g).astype(np.float64)
     np.testing.assert_allclose(dX, dY64 @ wh, rtol=1e-12, atol=1e-12)
     np.testing.assert_allclose(orc.dq_linear_fwd(X, packed, zq, s, bits, g), X64 @ wh.T, rtol=1e-12, atol=1e-12)
+
+
+@pytest.mark.parametrize("s_dtype", [np.float32, np.float16])
+def test_e2e_dz_is_exact_gradient_finite_differences(orc, s_dtype):
+    """With z trained as a float at the frozen codes, W-hat = (W_q - z) s is linear in z:
+    central differences of L(z) equal dz = -s sum dW-hat to ~1e-10.  With fp16 step
+    storage the oracle widens s exactly, so the same holds with s = float(s16)."""
+    bits, g = 3, 8
+    rng = np.random.default_rng(14)
+    M, N, K = 5, 4, 32
+    X = rng.standard_normal((M, K)).astype(np.float32)
+    dY = rng.standard_normal((M, N)).astype(np.float32)
+    W = rand_w(N, K, 14)
+    s, z = orc.minmax_init(W, bits, g)
+    packed, zq = orc.pack(W, s, z, bits, g)
+    s = s.astype(s_dtype)
+    codes = unpack_codes(packed, K, bits).astype(np.float64)
+    X64, dY64 = X.astype(np.float64), dY.astype(np.float64)
+    s64 = s.astype(np.float64)
+
+    def loss(zv):
+        wh = (codes - np.repeat(zv, g, 1)) * np.repeat(s64, g, 1)
+        return float(np.sum(dY64 * (X64 @ wh.T)))
+
+    dX, ds, dz = orc.dq_linear_bwd(X, packed, zq, s, dY, bits, g)
+    z64 = zq.astype(np.float64)
+    for n in range(N):
+        for j in range(K // g):
+            e = np.zeros_like(z64); e[n, j] = 0.5
+            fd = (loss(z64 + e) - loss(z64 - e)) / 1.0
+            assert abs(fd - dz[n, j]) <= 1e-10 * max(1.0, abs(dz).max())
+    _, ds_s = orc.dq_linear_bwd_s(X, packed, zq, s, dY, bits, g)
+    assert (ds == ds_s).all()
+
+
+def test_fp16_step_storage_dequant_is_exact(orc):
+    """(W_q - zq) is an integer of at most 5 bits and an fp16 s has an 11-bit
+    significand, so with fp16 step storage W-hat = (W_q - zq) s is exact in fp32: it
+    equals the fp64 product with the fp16 value of s (numpy's float16 conversion)."""
+    bits, g = 4, 16
+    W = rand_w(8, 64, 15)
+    s, z = orc.minmax_init(W, bits, g)
+    packed, zq = orc.pack(W, s, z, bits, g)
+    s16 = s.astype(np.float16)
+    wh = orc.dequant_packed(packed, zq, s16, 64, bits, g)
+    codes = unpack_codes(packed, 64, bits).astype(np.float64)
+    ref = (codes - np.repeat(zq.astype(np.float64), g, 1)) * np.repeat(s16.astype(np.float64), g, 1)
+    assert (wh.astype(np.float64) == ref).all()
+    assert not (s16.astype(np.float32) == s).all()
 
 
 def test_effective_bits_closed_form():

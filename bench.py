@@ -369,6 +369,8 @@ def run_ours(args):
         ip["init_frac_hbm"] = round(ip["init_GBps"] / peaks["hbm_gbs"], 4)
         ip["pack_frac_hbm"] = round(ip["pack_GBps"] / peaks["hbm_gbs"], 4)
         line["initpack_70b_block"] = ip
+    if not args.no_variants:
+        line["variants"] = quantizer_variants(step, dev)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(target_s=args.cpu_seconds)
     if dist is not None:
@@ -376,6 +378,56 @@ def run_ours(args):
         dist.destroy_process_group()
     if rank == 0:
         print(json.dumps(line), flush=True)
+
+
+def quantizer_variants(step, dev, reps=50):
+    """Backward throughput of the quantizer variants on the step's workload, each
+    beside its default (same buffers, W-hat reused from the workspace, L2 flushed
+    before every call): the all-pass clamp gradient of the Block-AP backward, and
+    the E2E-QP backward with dz and fp32 / fp16 step sizes.  TFLOP/s = 4MNK / event
+    time of the call."""
+    b, g = step.bits, step.group
+    M, N, K = step.M, step.N, step.K
+    flush = torch.empty(512 << 20, dtype=torch.uint8, device=dev)
+    s16 = step.s.to(torch.float16)
+    dz2 = torch.empty_like(step.ds2)
+    eqat.fq_linear_fwd(step.X, step.W, step.s, step.z, b, g, ws=step.ws, Y=step.Y)
+    calls = {
+        "fq_bwd": lambda: eqat.fq_linear_bwd(step.X, step.W, step.s, step.z, step.dY, b, g, ws=step.ws,
+                                             out=(step.dX, step.dW, step.ds, step.dz), w_hat_in_ws=True),
+        "fq_bwd_clamp_pass": lambda: eqat.fq_linear_bwd(step.X, step.W, step.s, step.z, step.dY, b, g,
+                                                        ws=step.ws, out=(step.dX, step.dW, step.ds, step.dz),
+                                                        w_hat_in_ws=True, clamp_pass=True),
+    }
+    e2e = {
+        "dq_bwd_ds": lambda s_: eqat.dq_linear_bwd(step.X, step.codes, step.zq, s_, step.dY, b, g, ws=step.ws,
+                                                   out=(step.dX2, step.ds2, None), w_hat_in_ws=True),
+        "dq_bwd_ds_dz": lambda s_: eqat.dq_linear_bwd(step.X, step.codes, step.zq, s_, step.dY, b, g, ws=step.ws,
+                                                     out=(step.dX2, step.ds2, dz2), w_hat_in_ws=True),
+    }
+
+    def timed(fn):
+        tot = 0.0
+        for r in range(reps + 3):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            flush.zero_()
+            e0.record()
+            fn()
+            e1.record()
+            torch.cuda.synchronize()
+            if r >= 3:
+                tot += e0.elapsed_time(e1)
+        return tot / reps
+
+    out = {}
+    for name, fn in calls.items():
+        out[name + "_TFLOPs"] = round(4 * M * N * K / (timed(fn) * 1e-3) / 1e12, 1)
+    for sname, s_ in (("s32", step.s), ("s16", s16)):
+        eqat.dq_linear_fwd(step.X, step.codes, step.zq, s_, b, g, ws=step.ws, Y=step.Y2)
+        for name, fn in e2e.items():
+            out[f"{name}_{sname}_TFLOPs"] = round(4 * M * N * K / (timed(lambda: fn(s_)) * 1e-3) / 1e12, 1)
+    out["note"] = "4MNK per backward call, L2 flushed before each call, W-hat reused from the forward"
+    return out
 
 
 def initpack_70b_block(dev, reps=5):
@@ -511,6 +563,7 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-initpack70b", action="store_true")
+    ap.add_argument("--no-variants", action="store_true")
     ap.add_argument("--initpack70b-only", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     args = ap.parse_args()

@@ -82,7 +82,13 @@ typedef enum {
     EQAT_ERR_TIMEOUT = 8      /* a bounded on-chip wait ran out (see eqat_device_error) */
 } eqat_status;
 
-typedef enum { EQAT_F32 = 0, EQAT_BF16 = 1 } eqat_dtype;
+/* EQAT_F16 is accepted only for the step size s of the E2E-QP entry points
+ * that take an `sdt` argument (the pages' fp16 step-size storage). */
+typedef enum { EQAT_F32 = 0, EQAT_BF16 = 1, EQAT_F16 = 2 } eqat_dtype;
+
+/* Flags of eqat_fq_linear_bwd_ex. */
+#define EQAT_GRAD_CLAMP_PASS 1u /* clamp straight-through too: dW = dY^T X, dz = 0,
+                                   ds = sum_group (dY^T X) ((code - zr) - u) */
 
 /* Human-readable name of a status; never NULL. */
 const char *eqat_status_string(int status);
@@ -166,6 +172,42 @@ eqat_status eqat_dq_linear_bwd_s(const void *X, int dt, const uint8_t *codes, co
                                  const float *s, const void *dY, void *dX, float *ds, int64_t M,
                                  int64_t N, int64_t K, int bits, int group, void *ws,
                                  size_t ws_bytes, int w_hat_in_ws, eqat_stream_t stream);
+
+/* Quantizer variants (the pages leave these open or mention them in passing).
+ *
+ * eqat_fq_linear_bwd_ex: eqat_fq_linear_bwd with `flags`.  flags == 0 is
+ * eqat_fq_linear_bwd.  EQAT_GRAD_CLAMP_PASS gives the clamp an identity
+ * gradient as well (the all-pass clamp_ste of the modelfoundations note, "Paper
+ * vs. code"): dW = dY^T X, ds = sum_group (dY^T X) ((code - zr) - u), dz = 0.
+ * Unknown flag bits return EQAT_ERR_UNSUPPORTED. */
+eqat_status eqat_fq_linear_bwd_ex(const void *X, const void *W, int dt, const float *s,
+                                  const float *z, const void *dY, void *dX, void *dW, float *ds,
+                                  float *dz, int64_t M, int64_t N, int64_t K, int bits, int group,
+                                  uint32_t flags, void *ws, size_t ws_bytes, int w_hat_in_ws,
+                                  eqat_stream_t stream);
+
+/* eqat_dequant_codes / eqat_dq_linear_fwd with the step size s of dtype sdt:
+ * EQAT_F32 or EQAT_F16 (paperlayer appendix D: a shared FP16 step size per
+ * group).  An fp16 s is widened exactly to fp32 before any arithmetic. */
+eqat_status eqat_dequant_codes_ex(const uint8_t *codes, const uint8_t *zq, const void *s, int sdt,
+                                  int64_t N, int64_t K, int bits, int group, void *W_hat, int dt,
+                                  eqat_stream_t stream);
+eqat_status eqat_dq_linear_fwd_ex(const void *X, int dt, const uint8_t *codes, const uint8_t *zq,
+                                  const void *s, int sdt, void *Y, int64_t M, int64_t N, int64_t K,
+                                  int bits, int group, void *ws, size_t ws_bytes,
+                                  eqat_stream_t stream);
+
+/* E2E-QP backward with the zero point trained as well (z a float evaluated at
+ * the frozen zq): W_hat = (W_q - z) s gives
+ *   dX = dY W_hat                          (nullable)
+ *   ds = sum_group (dY^T X) (W_q - zq)     (nullable)
+ *   dz = -s * sum_group (dY^T X)           (nullable)
+ * s of dtype sdt (EQAT_F32 or EQAT_F16); ds and dz fp32.  With dz == NULL and
+ * sdt == EQAT_F32 this is eqat_dq_linear_bwd_s. */
+eqat_status eqat_dq_linear_bwd(const void *X, int dt, const uint8_t *codes, const uint8_t *zq,
+                               const void *s, int sdt, const void *dY, void *dX, float *ds,
+                               float *dz, int64_t M, int64_t N, int64_t K, int bits, int group,
+                               void *ws, size_t ws_bytes, int w_hat_in_ws, eqat_stream_t stream);
 
 /* Block-AP forward (as eqat_fq_linear_fwd) that allocates nothing and takes no
  * workspace: the paper has no counterpart; this entry point exists for callers of

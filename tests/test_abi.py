@@ -111,6 +111,30 @@ def test_other_entry_points_argument_errors(lib):
     assert lib.eqat_selftest_bounded_wait(10, st) == SHAPE
 
 
+def test_variant_entry_points_argument_errors(lib):
+    st = None
+    U = ctypes.c_uint32
+    # unknown gradient flag bits are refused; flags 0 and EQAT_GRAD_CLAMP_PASS pass validation
+    assert lib.eqat_fq_linear_bwd_ex(P(FAKE), P(FAKE), 1, P(FAKE), P(FAKE), P(FAKE), P(FAKE), P(0), P(0), P(0),
+                                     16, 16, 64, 2, 64, U(2), P(FAKE), 1 << 20, 0, st) == UNSUP
+    for flags in (0, 1):
+        assert lib.eqat_fq_linear_bwd_ex(P(FAKE), P(FAKE), 1, P(FAKE), P(FAKE), P(FAKE), P(0), P(0), P(0), P(0),
+                                         16, 16, 64, 2, 64, U(flags), P(0), 0, 0, st) == OK
+    # step-size dtype: fp32 or fp16 only
+    assert lib.eqat_dequant_codes_ex(P(FAKE), P(FAKE), P(FAKE), 1, 16, 64, 2, 64, P(FAKE), 1, st) == DTYPE
+    assert lib.eqat_dequant_codes_ex(P(FAKE), P(FAKE), P(FAKE), 2, 0, 64, 2, 64, P(FAKE), 1, st) == OK
+    assert lib.eqat_dq_linear_fwd_ex(P(FAKE), 1, P(FAKE), P(FAKE), P(FAKE), 3, P(FAKE), 16, 16, 64, 2, 64,
+                                     P(FAKE), 1 << 20, st) == DTYPE
+    assert lib.eqat_dq_linear_fwd_ex(P(FAKE), 2, P(FAKE), P(FAKE), P(FAKE), 2, P(FAKE), 16, 16, 64, 2, 64,
+                                     P(FAKE), 1 << 20, st) == DTYPE
+    assert lib.eqat_dq_linear_bwd(P(FAKE), 1, P(FAKE), P(FAKE), P(FAKE), 2, P(FAKE), P(0), P(0), P(FAKE + 4),
+                                  16, 16, 64, 2, 64, P(FAKE), 1 << 20, 0, st) == ALIGN
+    assert lib.eqat_dq_linear_bwd(P(FAKE), 1, P(FAKE), P(FAKE), P(0), 2, P(FAKE), P(0), P(0), P(FAKE),
+                                  16, 16, 64, 2, 64, P(FAKE), 1 << 20, 0, st) == NULL
+    assert lib.eqat_dq_linear_bwd(P(FAKE), 1, P(FAKE), P(FAKE), P(FAKE), 2, P(FAKE), P(0), P(0), P(0),
+                                  16, 16, 64, 2, 64, P(0), 0, 0, st) == OK
+
+
 def test_binding_refuses_cpu_tensors():
     import torch
     W = torch.zeros(16, 64, dtype=torch.bfloat16)

@@ -20,6 +20,8 @@ LIB_PATH = os.path.join(HERE, "libeqat.so")
 
 EQAT_F32 = 0
 EQAT_BF16 = 1
+EQAT_F16 = 2  # step sizes of the E2E-QP calls only
+EQAT_GRAD_CLAMP_PASS = 1
 EQAT_ERR_TIMEOUT = 8
 
 _lib = None
@@ -42,6 +44,7 @@ def load_library():
             " (there is no fallback implementation)")
     lib = ctypes.CDLL(LIB_PATH)
     P, I, I64, SZ = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_size_t
+    U32 = ctypes.c_uint32
     sigs = {
         "eqat_minmax_init": [P, I, I64, I64, I, I, P, P, P],
         "eqat_fake_quant": [P, I, P, P, I64, I64, I, I, P, P, P, P],
@@ -52,6 +55,10 @@ def load_library():
         "eqat_dq_linear_fwd": [P, I, P, P, P, P, I64, I64, I64, I, I, P, SZ, P],
         "eqat_dq_linear_bwd_s": [P, I, P, P, P, P, P, P, I64, I64, I64, I, I, P, SZ, I, P],
         "eqat_fq_linear_fwd_noalloc": [P, P, I, P, P, P, I64, I64, I64, I, I, P],
+        "eqat_fq_linear_bwd_ex": [P, P, I, P, P, P, P, P, P, P, I64, I64, I64, I, I, U32, P, SZ, I, P],
+        "eqat_dequant_codes_ex": [P, P, P, I, I64, I64, I, I, P, I, P],
+        "eqat_dq_linear_fwd_ex": [P, I, P, P, P, I, P, I64, I64, I64, I, I, P, SZ, P],
+        "eqat_dq_linear_bwd": [P, I, P, P, P, I, P, P, P, P, I64, I64, I64, I, I, P, SZ, I, P],
         "eqat_device_error": [P, P],
         "eqat_selftest_bounded_wait": [I64, P],
     }
@@ -97,6 +104,15 @@ def _dt(t: torch.Tensor) -> int:
     if t.dtype == torch.float32:
         return EQAT_F32
     raise TypeError(f"unsupported dtype {t.dtype}; use torch.bfloat16 or torch.float32")
+
+
+def _sdt(s: torch.Tensor) -> int:
+    """Step-size dtype of the E2E-QP calls: fp32, or fp16 storage."""
+    if s.dtype == torch.float32:
+        return EQAT_F32
+    if s.dtype == torch.float16:
+        return EQAT_F16
+    raise TypeError(f"s must be torch.float32 or torch.float16, got {s.dtype}")
 
 
 def _req(t, name, dtype=None):
@@ -170,11 +186,13 @@ def pack_codes(W, s, z, bits, group, codes=None, zq=None):
 
 
 def dequant_codes(codes, zq, s, K, bits, group, dtype=torch.bfloat16):
-    """E2E-QP dequant of frozen codes: W_hat = (W_q - zq) s, [N, K] of `dtype`."""
-    _req(codes, "codes", torch.uint8); _req(zq, "zq", torch.uint8); _req(s, "s", torch.float32)
+    """E2E-QP dequant of frozen codes: W_hat = (W_q - zq) s, [N, K] of `dtype`.
+    s is fp32 or fp16 (fp16 step-size storage)."""
+    _req(codes, "codes", torch.uint8); _req(zq, "zq", torch.uint8); _req(s, "s")
     N = codes.shape[0]
     wh = torch.empty((N, K), dtype=dtype, device=codes.device)
-    _call("eqat_dequant_codes", _p(codes), _p(zq), _p(s), N, K, bits, group, _p(wh), _dt(wh), _stream())
+    _call("eqat_dequant_codes_ex", _p(codes), _p(zq), _p(s), _sdt(s), N, K, bits, group, _p(wh), _dt(wh),
+          _stream())
     return wh
 
 
@@ -205,9 +223,10 @@ def fq_linear_fwd_noalloc(X, W, s, z, bits, group, Y):
 
 
 def fq_linear_bwd(X, W, s, z, dY, bits, group, need_dx=True, need_dw=True, need_ds=True, need_dz=True,
-                  ws=None, out=None, w_hat_in_ws=False):
+                  ws=None, out=None, w_hat_in_ws=False, clamp_pass=False):
     """Block-AP straight-through backward: returns (dX, dW, ds, dz), None where not requested.
-    w_hat_in_ws=True reuses the W-hat that fq_linear_fwd left in `ws` (same W, s, z)."""
+    w_hat_in_ws=True reuses the W-hat that fq_linear_fwd left in `ws` (same W, s, z).
+    clamp_pass=True lets the clamp pass the gradient too (EQAT_GRAD_CLAMP_PASS)."""
     _req(X, "X"); _req(W, "W", X.dtype); _req(s, "s", torch.float32); _req(z, "z", torch.float32)
     _req(dY, "dY", X.dtype)
     M, K = X.shape
@@ -224,20 +243,21 @@ def fq_linear_bwd(X, W, s, z, dY, bits, group, need_dx=True, need_dw=True, need_
     ws = _ws(ws, M, N, K, bits, group, X.dtype, X.device)
     if w_hat_in_ws and ws is None:
         raise ValueError("w_hat_in_ws needs the workspace of the forward call")
-    _call("eqat_fq_linear_bwd", _p(X), _p(W), _dt(X), _p(s), _p(z), _p(dY), _p(dX), _p(dW), _p(ds), _p(dz),
-          M, N, K, bits, group, _p(ws), ws.numel(), int(bool(w_hat_in_ws)), _stream())
+    flags = EQAT_GRAD_CLAMP_PASS if clamp_pass else 0
+    _call("eqat_fq_linear_bwd_ex", _p(X), _p(W), _dt(X), _p(s), _p(z), _p(dY), _p(dX), _p(dW), _p(ds),
+          _p(dz), M, N, K, bits, group, flags, _p(ws), ws.numel(), int(bool(w_hat_in_ws)), _stream())
     return dX, dW, ds, dz
 
 
 def dq_linear_fwd(X, codes, zq, s, bits, group, ws=None, Y=None):
-    """E2E-QP forward on frozen codes: Y = X ((W_q - zq) s)^T."""
-    _req(X, "X"); _req(codes, "codes", torch.uint8); _req(zq, "zq", torch.uint8); _req(s, "s", torch.float32)
+    """E2E-QP forward on frozen codes: Y = X ((W_q - zq) s)^T; s fp32 or fp16."""
+    _req(X, "X"); _req(codes, "codes", torch.uint8); _req(zq, "zq", torch.uint8); _req(s, "s")
     M, K = X.shape
     N = codes.shape[0]
     Y = torch.empty((M, N), dtype=X.dtype, device=X.device) if Y is None else _req(Y, "Y", X.dtype)
     ws = _ws(ws, M, N, K, bits, group, X.dtype, X.device)
-    _call("eqat_dq_linear_fwd", _p(X), _dt(X), _p(codes), _p(zq), _p(s), _p(Y), M, N, K, bits, group,
-          _p(ws), ws.numel(), _stream())
+    _call("eqat_dq_linear_fwd_ex", _p(X), _dt(X), _p(codes), _p(zq), _p(s), _sdt(s), _p(Y), M, N, K, bits,
+          group, _p(ws), ws.numel(), _stream())
     return Y
 
 
@@ -260,6 +280,29 @@ def dq_linear_bwd_s(X, codes, zq, s, dY, bits, group, need_dx=True, need_ds=True
     _call("eqat_dq_linear_bwd_s", _p(X), _dt(X), _p(codes), _p(zq), _p(s), _p(dY), _p(dX), _p(ds),
           M, N, K, bits, group, _p(ws), ws.numel(), int(bool(w_hat_in_ws)), _stream())
     return dX, ds
+
+
+def dq_linear_bwd(X, codes, zq, s, dY, bits, group, need_dx=True, need_ds=True, need_dz=True, ws=None,
+                  out=None, w_hat_in_ws=False):
+    """E2E-QP backward with the zero-point gradient: returns (dX, ds, dz), None where not
+    requested; dz = -s sum_group dY^T X.  s fp32 or fp16."""
+    _req(X, "X"); _req(codes, "codes", torch.uint8); _req(zq, "zq", torch.uint8); _req(s, "s")
+    _req(dY, "dY", X.dtype)
+    M, K = X.shape
+    N = codes.shape[0]
+    G = K // group
+    if out is None:
+        dX = torch.empty((M, K), dtype=X.dtype, device=X.device) if need_dx else None
+        ds = torch.empty((N, G), dtype=torch.float32, device=X.device) if need_ds else None
+        dz = torch.empty((N, G), dtype=torch.float32, device=X.device) if need_dz else None
+    else:
+        dX, ds, dz = out
+    ws = _ws(ws, M, N, K, bits, group, X.dtype, X.device)
+    if w_hat_in_ws and ws is None:
+        raise ValueError("w_hat_in_ws needs the workspace of the forward call")
+    _call("eqat_dq_linear_bwd", _p(X), _dt(X), _p(codes), _p(zq), _p(s), _sdt(s), _p(dY), _p(dX), _p(ds),
+          _p(dz), M, N, K, bits, group, _p(ws), ws.numel(), int(bool(w_hat_in_ws)), _stream())
+    return dX, ds, dz
 
 
 def device_error():

@@ -110,6 +110,12 @@ eqat_status check_dtype(int dt) {
     return EQAT_OK;
 }
 
+// Step-size dtype of the E2E-QP entry points: fp32, or fp16 storage.
+eqat_status check_sdtype(int sdt) {
+    if (sdt != EQAT_F32 && sdt != EQAT_F16) return fail(EQAT_ERR_DTYPE, "sdt must be EQAT_F32 or EQAT_F16");
+    return EQAT_OK;
+}
+
 size_t esize(int dt) { return dt == EQAT_F32 ? 4 : 2; }
 
 int64_t code_bytes(int64_t N, int64_t K, int bits) {
@@ -245,8 +251,14 @@ eqat_status eqat_pack_codes(const void *W, int wdt, const float *s, const float 
 
 eqat_status eqat_dequant_codes(const uint8_t *codes, const uint8_t *zq, const float *s, int64_t N, int64_t K,
                                int bits, int group, void *W_hat, int dt, eqat_stream_t stream) {
+    return eqat_dequant_codes_ex(codes, zq, s, EQAT_F32, N, K, bits, group, W_hat, dt, stream);
+}
+
+eqat_status eqat_dequant_codes_ex(const uint8_t *codes, const uint8_t *zq, const void *s, int sdt, int64_t N,
+                                  int64_t K, int bits, int group, void *W_hat, int dt, eqat_stream_t stream) {
     DeviceInfo dev;
     EQAT_TRY(check_dtype(dt));
+    EQAT_TRY(check_sdtype(sdt));
     EQAT_TRY(check_common(0, N, K, bits, group));
     const int64_t ng = N * (K / group);
     EQAT_TRY(check_ptr(codes, code_bytes(N, K, bits), "codes"));
@@ -255,7 +267,7 @@ eqat_status eqat_dequant_codes(const uint8_t *codes, const uint8_t *zq, const fl
     EQAT_TRY(check_ptr(W_hat, N * K, "W_hat"));
     if (N * K == 0) return EQAT_OK;
     EQAT_TRY(get_device(dev));
-    EQAT_CUDA(eqat::launch_dequant(codes, zq, s, N, K, bits, group, W_hat, dt == EQAT_F32, dev,
+    EQAT_CUDA(eqat::launch_dequant(codes, zq, s, sdt == EQAT_F16, N, K, bits, group, W_hat, dt == EQAT_F32, dev,
                                    reinterpret_cast<cudaStream_t>(stream)),
               "dequant_codes");
     return EQAT_OK;
@@ -298,8 +310,17 @@ eqat_status eqat_fq_linear_bwd(const void *X, const void *W, int dt, const float
                                const void *dY, void *dX, void *dW, float *ds, float *dz, int64_t M, int64_t N,
                                int64_t K, int bits, int group, void *ws, size_t ws_bytes, int w_hat_in_ws,
                                eqat_stream_t stream) {
+    return eqat_fq_linear_bwd_ex(X, W, dt, s, z, dY, dX, dW, ds, dz, M, N, K, bits, group, 0u, ws, ws_bytes,
+                                 w_hat_in_ws, stream);
+}
+
+eqat_status eqat_fq_linear_bwd_ex(const void *X, const void *W, int dt, const float *s, const float *z,
+                                  const void *dY, void *dX, void *dW, float *ds, float *dz, int64_t M, int64_t N,
+                                  int64_t K, int bits, int group, uint32_t flags, void *ws, size_t ws_bytes,
+                                  int w_hat_in_ws, eqat_stream_t stream) {
     DeviceInfo dev;
     EQAT_TRY(check_dtype(dt));
+    if (flags & ~EQAT_GRAD_CLAMP_PASS) return fail(EQAT_ERR_UNSUPPORTED, "unknown flag bits");
     EQAT_TRY(check_common(M, N, K, bits, group));
     const int64_t ng = N * (K / group);
     EQAT_TRY(check_ptr(X, M * K, "X"));
@@ -339,6 +360,7 @@ eqat_status eqat_fq_linear_bwd(const void *X, const void *W, int dt, const float
             epi.dW = dW;
             epi.ds = ds;
             epi.dz = dz;
+            epi.clamp_pass = (flags & EQAT_GRAD_CLAMP_PASS) != 0;
             epi.bits = bits;
             epi.group = group;
             probs[np++] = eqat::GemmProblem{Operand{dY, N, true}, Operand{X, K, true}, N, K, M, epi};
@@ -375,8 +397,15 @@ eqat_status eqat_fq_linear_bwd(const void *X, const void *W, int dt, const float
 eqat_status eqat_dq_linear_fwd(const void *X, int dt, const uint8_t *codes, const uint8_t *zq, const float *s,
                                void *Y, int64_t M, int64_t N, int64_t K, int bits, int group, void *ws,
                                size_t ws_bytes, eqat_stream_t stream) {
+    return eqat_dq_linear_fwd_ex(X, dt, codes, zq, s, EQAT_F32, Y, M, N, K, bits, group, ws, ws_bytes, stream);
+}
+
+eqat_status eqat_dq_linear_fwd_ex(const void *X, int dt, const uint8_t *codes, const uint8_t *zq, const void *s,
+                                  int sdt, void *Y, int64_t M, int64_t N, int64_t K, int bits, int group, void *ws,
+                                  size_t ws_bytes, eqat_stream_t stream) {
     DeviceInfo dev;
     EQAT_TRY(check_dtype(dt));
+    EQAT_TRY(check_sdtype(sdt));
     EQAT_TRY(check_common(M, N, K, bits, group));
     const int64_t ng = N * (K / group);
     EQAT_TRY(check_ptr(X, M * K, "X"));
@@ -393,7 +422,8 @@ eqat_status eqat_dq_linear_fwd(const void *X, int dt, const uint8_t *codes, cons
         return EQAT_OK;
     }
     const bool f32 = dt == EQAT_F32;
-    EQAT_CUDA(eqat::launch_dequant(codes, zq, s, N, K, bits, group, ws, f32, dev, st), "dequant prepass");
+    EQAT_CUDA(eqat::launch_dequant(codes, zq, s, sdt == EQAT_F16, N, K, bits, group, ws, f32, dev, st),
+              "dequant prepass");
     EpiArgs epi;
     epi.kind = Epi::kStore;
     epi.out = Y;
@@ -407,8 +437,17 @@ eqat_status eqat_dq_linear_fwd(const void *X, int dt, const uint8_t *codes, cons
 eqat_status eqat_dq_linear_bwd_s(const void *X, int dt, const uint8_t *codes, const uint8_t *zq, const float *s,
                                  const void *dY, void *dX, float *ds, int64_t M, int64_t N, int64_t K, int bits,
                                  int group, void *ws, size_t ws_bytes, int w_hat_in_ws, eqat_stream_t stream) {
+    return eqat_dq_linear_bwd(X, dt, codes, zq, s, EQAT_F32, dY, dX, ds, nullptr, M, N, K, bits, group, ws,
+                              ws_bytes, w_hat_in_ws, stream);
+}
+
+eqat_status eqat_dq_linear_bwd(const void *X, int dt, const uint8_t *codes, const uint8_t *zq, const void *s,
+                               int sdt, const void *dY, void *dX, float *ds, float *dz, int64_t M, int64_t N,
+                               int64_t K, int bits, int group, void *ws, size_t ws_bytes, int w_hat_in_ws,
+                               eqat_stream_t stream) {
     DeviceInfo dev;
     EQAT_TRY(check_dtype(dt));
+    EQAT_TRY(check_sdtype(sdt));
     EQAT_TRY(check_common(M, N, K, bits, group));
     const int64_t ng = N * (K / group);
     EQAT_TRY(check_ptr(X, M * K, "X"));
@@ -418,23 +457,28 @@ eqat_status eqat_dq_linear_bwd_s(const void *X, int dt, const uint8_t *codes, co
     EQAT_TRY(check_ptr(dY, M * N, "dY"));
     EQAT_TRY(check_ptr(dX, 0, "dX"));
     EQAT_TRY(check_ptr(ds, 0, "ds"));
+    EQAT_TRY(check_ptr(dz, 0, "dz"));
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     const bool f32 = dt == EQAT_F32;
-    if (!dX && !ds) return EQAT_OK;
+    if (!dX && !ds && !dz) return EQAT_OK;
     if (N * K > 0) EQAT_TRY(check_ws(ws, ws_bytes, N, K, dt));
     EQAT_TRY(get_device(dev));
 
     eqat::GemmProblem probs[2];
     int np = 0;
-    if (ds && ng > 0) {
+    if ((ds || dz) && ng > 0) {
         if (M == 0) {
             EQAT_CUDA(zero(ds, static_cast<size_t>(ng) * 4, st), "memset ds");
+            EQAT_CUDA(zero(dz, static_cast<size_t>(ng) * 4, st), "memset dz");
         } else {
             EpiArgs epi;
             epi.kind = Epi::kE2eDs;
             epi.codes = codes;
             epi.zq = zq;
             epi.ds = ds;
+            epi.dz = dz;
+            epi.s_e2e = s;
+            epi.s_f16 = sdt == EQAT_F16;
             epi.bits = bits;
             epi.group = group;
             probs[np++] = eqat::GemmProblem{Operand{dY, N, true}, Operand{X, K, true}, N, K, M, epi};
@@ -445,7 +489,8 @@ eqat_status eqat_dq_linear_bwd_s(const void *X, int dt, const uint8_t *codes, co
             EQAT_CUDA(zero(dX, static_cast<size_t>(M * K) * esize(dt), st), "memset dX");
         } else {
             if (!w_hat_in_ws)
-                EQAT_CUDA(eqat::launch_dequant(codes, zq, s, N, K, bits, group, ws, f32, dev, st), "dequant prepass");
+                EQAT_CUDA(eqat::launch_dequant(codes, zq, s, sdt == EQAT_F16, N, K, bits, group, ws, f32, dev, st),
+                          "dequant prepass");
             EpiArgs epi;
             epi.kind = Epi::kStore;
             epi.out = dX;

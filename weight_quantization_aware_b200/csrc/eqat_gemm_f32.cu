@@ -6,6 +6,7 @@
 // D[GM, GN] = sum_k A(m, k) B(n, k) with 64x64 output tiles, 16-deep k slices
 // staged in shared memory and a 4x4 register block per thread.  Non-store
 // epilogues run as a second pass over D kept in fp32 scratch.
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 
 #include <algorithm>
@@ -72,7 +73,8 @@ __global__ void __launch_bounds__(256)
 __global__ void k_ste_epilogue_f32(const float *__restrict__ W, const float *__restrict__ s,
                                    const float *__restrict__ z, const float *__restrict__ dwh,
                                    float *__restrict__ dW, float *__restrict__ ds,
-                                   float *__restrict__ dz, int64_t n_groups, int group, float Q) {
+                                   float *__restrict__ dz, int64_t n_groups, int group, float Q,
+                                   bool clamp_pass) {
     const int64_t gi = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
     if (gi >= n_groups) return;
     const float sc = s[gi];
@@ -83,9 +85,10 @@ __global__ void k_ste_epilogue_f32(const float *__restrict__ W, const float *__r
     for (int i = 0; i < group; ++i) {
         const float d = dwh[e0 + i];
         const QuantElem e = quant_elem(W[e0 + i], sc, rcp, zr, Q);
-        acc_s = fmaf(d, __fsub_rn(__fsub_rn(e.c, zr), e.inside ? e.u : 0.0f), acc_s);
-        acc_z += e.inside ? 0.0f : d;
-        if (dW) dW[e0 + i] = e.inside ? d : 0.0f;
+        const bool keep = e.inside || clamp_pass;
+        acc_s = fmaf(d, __fsub_rn(__fsub_rn(e.c, zr), keep ? e.u : 0.0f), acc_s);
+        acc_z += keep ? 0.0f : d;
+        if (dW) dW[e0 + i] = keep ? d : 0.0f;
     }
     if (ds) ds[gi] = acc_s;
     if (dz) dz[gi] = -sc * acc_z;
@@ -97,18 +100,27 @@ __device__ __forceinline__ uint32_t code_at(const uint8_t *codes, int64_t e, int
     return codes[e];
 }
 
-// E2E-QP epilogue: ds = sum_group dW-hat (W_q - zq); one thread per group.
+// E2E-QP epilogue: ds = sum_group dW-hat (W_q - zq), dz = -s sum_group dW-hat
+// (both nullable; s fp32 or fp16, read for dz only); one thread per group.
 __global__ void k_e2e_ds_epilogue_f32(const uint8_t *__restrict__ codes, const uint8_t *__restrict__ zq,
                                       const float *__restrict__ dwh, float *__restrict__ ds,
+                                      float *__restrict__ dz, const void *__restrict__ s, bool s_f16,
                                       int64_t n_groups, int group, int bits) {
     const int64_t gi = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
     if (gi >= n_groups) return;
     const float zf = static_cast<float>(zq[gi]);
-    float acc = 0.0f;
+    float acc = 0.0f, sum = 0.0f;
     const int64_t e0 = gi * group;
-    for (int i = 0; i < group; ++i)
-        acc = fmaf(dwh[e0 + i], __fsub_rn(static_cast<float>(code_at(codes, e0 + i, bits)), zf), acc);
-    ds[gi] = acc;
+    for (int i = 0; i < group; ++i) {
+        const float d = dwh[e0 + i];
+        acc = fmaf(d, __fsub_rn(static_cast<float>(code_at(codes, e0 + i, bits)), zf), acc);
+        sum += d;
+    }
+    if (ds) ds[gi] = acc;
+    if (dz) {
+        const float sc = s_f16 ? __half2float(static_cast<const __half *>(s)[gi]) : static_cast<const float *>(s)[gi];
+        dz[gi] = -sc * sum;
+    }
 }
 
 }  // namespace
@@ -146,10 +158,10 @@ cudaError_t launch_gemm_f32(const Operand &A, const Operand &B, int64_t GM, int6
         if (!epi.w_f32) return cudaErrorInvalidValue;
         k_ste_epilogue_f32<<<blocks, threads, 0, st>>>(
             static_cast<const float *>(epi.W), epi.s, epi.z, d_scratch, static_cast<float *>(epi.dW),
-            epi.ds, epi.dz, n_groups, epi.group, static_cast<float>((1 << epi.bits) - 1));
+            epi.ds, epi.dz, n_groups, epi.group, static_cast<float>((1 << epi.bits) - 1), epi.clamp_pass);
     } else {
-        k_e2e_ds_epilogue_f32<<<blocks, threads, 0, st>>>(epi.codes, epi.zq, d_scratch, epi.ds, n_groups,
-                                                          epi.group, epi.bits);
+        k_e2e_ds_epilogue_f32<<<blocks, threads, 0, st>>>(epi.codes, epi.zq, d_scratch, epi.ds, epi.dz, epi.s_e2e,
+                                                          epi.s_f16, n_groups, epi.group, epi.bits);
     }
     return cudaGetLastError();
 }

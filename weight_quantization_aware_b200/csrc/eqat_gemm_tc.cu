@@ -20,6 +20,7 @@
 // tile i+1.  Every mbarrier wait is bounded (see eqat_ptx.cuh).
 #include <cuda.h>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 #include <cudaTypedefs.h>
 
@@ -72,6 +73,9 @@ struct Prob {
     float *dz;
     const uint8_t *codes;
     const uint8_t *zq;
+    const void *s_e2e;  // E2E step sizes (read for dz only), fp32 or fp16
+    int s_f16;
+    int clamp_pass;     // Block-AP: the clamp is straight-through as well
     int group;
     int gshift;  // log2(group)
     float Q;
@@ -154,6 +158,7 @@ struct Epilogue<0, BITS> {
 
 // Block-AP straight-through: D is dW-hat[N, K] (bf16 W); row = n, col = k.
 //   dW = D * mask,  ds += D ((code - zr) - mask * u),  dz = -s * sum_{clamped} D.
+// With clamp_pass the mask is 1 everywhere (the clamp is straight-through too).
 template <int BITS>
 struct Epilogue<1, BITS> {
     float acc_s = 0.0f, acc_z = 0.0f;
@@ -177,7 +182,7 @@ struct Epilogue<1, BITS> {
             for (int j = 0; j < 8; ++j) {
                 const float d = v[8 * q + j];
                 const float qv = __fadd_rn(r[j], zr);
-                const bool inside = (qv >= 0.0f) && (qv <= p.Q);
+                const bool inside = ((qv >= 0.0f) && (qv <= p.Q)) || p.clamp_pass;
                 const float c = fminf(fmaxf(qv, 0.0f), p.Q);
                 const float dwds = __fsub_rn(__fsub_rn(c, zr), inside ? u[j] : 0.0f);
                 acc_s = fmaf(d, dwds, acc_s);
@@ -200,7 +205,8 @@ struct Epilogue<1, BITS> {
     }
 };
 
-// E2E-QP: D is dW-hat[N, K]; ds = sum_group D * (W_q - zq).
+// E2E-QP: D is dW-hat[N, K]; ds = sum_group D * (W_q - zq), dz = -s sum_group D
+// (the zero point trained as a float at zq).
 template <int BITS>
 struct Epilogue<2, BITS> {
     float acc_s = 0.0f, acc_z = 0.0f;
@@ -231,9 +237,19 @@ struct Epilogue<2, BITS> {
         }
 #pragma unroll
         for (int j = 0; j < 32; ++j) acc_s = fmaf(v[j], __fsub_rn(static_cast<float>(c[j]), zf), acc_s);
+        if (p.dz) {
+#pragma unroll
+            for (int j = 0; j < 32; ++j) acc_z += v[j];
+        }
         if (((col + 32) & (p.group - 1)) == 0) {
-            p.ds[gi] = acc_s;
+            if (p.ds) p.ds[gi] = acc_s;
+            if (p.dz) {
+                const float sc = p.s_f16 ? __half2float(static_cast<const __half *>(p.s_e2e)[gi])
+                                         : static_cast<const float *>(p.s_e2e)[gi];
+                p.dz[gi] = -sc * acc_z;
+            }
             acc_s = 0.0f;
+            acc_z = 0.0f;
         }
     }
 };
@@ -816,6 +832,9 @@ cudaError_t fill_prob(Prob &q, const GemmProblem &g, int tile_begin, int bn, int
     q.dz = epi.dz;
     q.codes = epi.codes;
     q.zq = epi.zq;
+    q.s_e2e = epi.s_e2e;
+    q.s_f16 = epi.s_f16 ? 1 : 0;
+    q.clamp_pass = epi.clamp_pass ? 1 : 0;
     q.group = epi.group;
     q.gshift = epi.group == 32 ? 5 : epi.group == 64 ? 6 : 7;
     q.Q = static_cast<float>((1 << epi.bits) - 1);

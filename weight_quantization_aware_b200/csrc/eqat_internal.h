@@ -28,7 +28,8 @@ cudaError_t launch_fake_quant(const void *W, bool w_f32, const float *s, const f
 cudaError_t launch_pack(const void *W, bool w_f32, const float *s, const float *z, int64_t N,
                         int64_t K, int bits, int group, uint8_t *codes, uint8_t *zq,
                         const DeviceInfo &dev, cudaStream_t st);
-cudaError_t launch_dequant(const uint8_t *codes, const uint8_t *zq, const float *s, int64_t N,
+// s is fp32, or fp16 when s_f16 (widened exactly before use).
+cudaError_t launch_dequant(const uint8_t *codes, const uint8_t *zq, const void *s, bool s_f16, int64_t N,
                            int64_t K, int bits, int group, void *W_hat, bool out_f32,
                            const DeviceInfo &dev, cudaStream_t st);
 
@@ -46,7 +47,7 @@ struct Operand {
 enum class Epi : int {
     kStore = 0,   // D -> out (bf16 or fp32), row stride ldo
     kFqGrad = 1,  // Block-AP straight-through: dW = D*mask, ds, dz per group
-    kE2eDs = 2,   // E2E-QP: ds = sum_group D * (W_q - zq)
+    kE2eDs = 2,   // E2E-QP: ds = sum_group D * (W_q - zq), dz = -s sum_group D
 };
 
 struct EpiArgs {
@@ -62,9 +63,12 @@ struct EpiArgs {
     void *dW = nullptr;
     float *ds = nullptr;
     float *dz = nullptr;
-    // kE2eDs
+    bool clamp_pass = false;  // kFqGrad: clamp straight-through as well
+    // kE2eDs (ds and dz nullable; s_e2e is read only for dz)
     const uint8_t *codes = nullptr;
     const uint8_t *zq = nullptr;
+    const void *s_e2e = nullptr;
+    bool s_f16 = false;
     int bits = 2;
     int group = 64;
 };

@@ -8,6 +8,7 @@
 // read once per thread from L1.  Grids are grid-stride loops sized to a whole
 // number of waves of the SMs.
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 
 #include <algorithm>
@@ -289,16 +290,20 @@ __device__ __forceinline__ void unpack16(const uint8_t *codes, int64_t e0, uint3
     }
 }
 
-template <int BITS, typename O>
+__device__ __forceinline__ float step_value(const float *s, int64_t g) { return __ldg(s + g); }
+__device__ __forceinline__ float step_value(const __half *s, int64_t g) { return __half2float(__ldg(s + g)); }
+
+// S: fp32 step sizes, or fp16 ones (fp16 step-size storage), widened exactly.
+template <int BITS, typename O, typename S>
 __global__ void __launch_bounds__(kThreads)
     k_dequant(const uint8_t *__restrict__ codes, const uint8_t *__restrict__ zq,
-              const float *__restrict__ s, int64_t n_chunks, int gshift, O *__restrict__ W_hat) {
+              const S *__restrict__ s, int64_t n_chunks, int gshift, O *__restrict__ W_hat) {
     const int64_t stride = static_cast<int64_t>(gridDim.x) * kThreads;
     for (int64_t i = static_cast<int64_t>(blockIdx.x) * kThreads + threadIdx.x; i < n_chunks;
          i += stride) {
         const int64_t e0 = i * 16;
         const int64_t g = e0 >> gshift;
-        const float sc = __ldg(s + g);
+        const float sc = step_value(s, g);
         const float zf = static_cast<float>(__ldg(zq + g));
         uint32_t c[16];
         unpack16<BITS>(codes, e0, c);
@@ -341,17 +346,17 @@ cudaError_t pack_dispatch(const T *W, const float *s, const float *z, int64_t n,
     return cudaGetLastError();
 }
 
-template <typename O>
-cudaError_t dequant_dispatch(const uint8_t *codes, const uint8_t *zq, const float *s, int64_t n,
+template <typename O, typename S>
+cudaError_t dequant_dispatch(const uint8_t *codes, const uint8_t *zq, const S *s, int64_t n,
                              int bits, int group, O *W_hat, const DeviceInfo &dev,
                              cudaStream_t st) {
     const int gshift = group_shift(group);
     const int64_t chunks = n / 16;
     const int grid = grid_for(chunks, dev);
     switch (bits) {
-        case 2: k_dequant<2, O><<<grid, kThreads, 0, st>>>(codes, zq, s, chunks, gshift, W_hat); break;
-        case 3: k_dequant<3, O><<<grid, kThreads, 0, st>>>(codes, zq, s, chunks, gshift, W_hat); break;
-        case 4: k_dequant<4, O><<<grid, kThreads, 0, st>>>(codes, zq, s, chunks, gshift, W_hat); break;
+        case 2: k_dequant<2, O, S><<<grid, kThreads, 0, st>>>(codes, zq, s, chunks, gshift, W_hat); break;
+        case 3: k_dequant<3, O, S><<<grid, kThreads, 0, st>>>(codes, zq, s, chunks, gshift, W_hat); break;
+        case 4: k_dequant<4, O, S><<<grid, kThreads, 0, st>>>(codes, zq, s, chunks, gshift, W_hat); break;
         default: return cudaErrorInvalidValue;
     }
     return cudaGetLastError();
@@ -409,13 +414,20 @@ cudaError_t launch_pack(const void *W, bool w_f32, const float *s, const float *
     return pack_dispatch(static_cast<const __nv_bfloat16 *>(W), s, z, n, bits, group, codes, zq, dev, st);
 }
 
-cudaError_t launch_dequant(const uint8_t *codes, const uint8_t *zq, const float *s, int64_t N,
+cudaError_t launch_dequant(const uint8_t *codes, const uint8_t *zq, const void *s, bool s_f16, int64_t N,
                            int64_t K, int bits, int group, void *W_hat, bool out_f32,
                            const DeviceInfo &dev, cudaStream_t st) {
     const int64_t n = N * K;
     if (n == 0) return cudaSuccess;
-    if (out_f32) return dequant_dispatch(codes, zq, s, n, bits, group, static_cast<float *>(W_hat), dev, st);
-    return dequant_dispatch(codes, zq, s, n, bits, group, static_cast<__nv_bfloat16 *>(W_hat), dev, st);
+    const float *s32 = static_cast<const float *>(s);
+    const __half *s16 = static_cast<const __half *>(s);
+    float *o32 = static_cast<float *>(W_hat);
+    __nv_bfloat16 *o16 = static_cast<__nv_bfloat16 *>(W_hat);
+    if (s_f16)
+        return out_f32 ? dequant_dispatch(codes, zq, s16, n, bits, group, o32, dev, st)
+                       : dequant_dispatch(codes, zq, s16, n, bits, group, o16, dev, st);
+    return out_f32 ? dequant_dispatch(codes, zq, s32, n, bits, group, o32, dev, st)
+                   : dequant_dispatch(codes, zq, s32, n, bits, group, o16, dev, st);
 }
 
 }  // namespace eqat

@@ -371,6 +371,8 @@ def run_ours(args):
         line["initpack_70b_block"] = ip
     if not args.no_variants:
         line["variants"] = quantizer_variants(step, dev)
+    if not args.no_gemv:
+        line["decode_gemv"] = decode_gemv(dev, peaks)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(target_s=args.cpu_seconds)
     if dist is not None:
@@ -427,6 +429,71 @@ def quantizer_variants(step, dev, reps=50):
         for name, fn in e2e.items():
             out[f"{name}_{sname}_TFLOPs"] = round(4 * M * N * K / (timed(lambda: fn(s_)) * 1e-3) / 1e12, 1)
     out["note"] = "4MNK per backward call, L2 flushed before each call, W-hat reused from the forward"
+    return out
+
+
+def decode_gemv(dev, peaks, budget_bytes=300_000_000):
+    """Batch-1 inference on frozen 2-bit codes (eqat_dq_linear_fwd at M = 1, the
+    decode-size path), against a bf16 matvec (torch.matmul) of the same shape.
+    Back-to-back calls over enough distinct layers that their bytes exceed L2,
+    captured in a CUDA graph so that host launch cost is excluded; CUDA events
+    around three replays.  GB/s = algorithmic bytes (codes + s + zq + X + Y) /
+    time per call."""
+    out = {}
+    side = torch.cuda.Stream(device=dev)
+    for name, N, K in (("llama2-70b-gate_proj", 28672, 8192), ("llama2-7b-q_proj", 4096, 4096)):
+        b, g, M = 2, 64, 1
+        G = K // g
+        per = N * K * b // 8 + N * G * 5
+        L = max(2, -(-budget_bytes // per))
+        gen = torch.Generator(device=dev)
+        gen.manual_seed(2000 + N)
+        layers = [(torch.randint(0, 256, (N, K * b // 8), generator=gen, device=dev, dtype=torch.uint8),
+                   torch.randint(0, 1 << b, (N, G), generator=gen, device=dev, dtype=torch.uint8),
+                   torch.rand(N, G, generator=gen, device=dev) * 0.01 + 1e-3) for _ in range(L)]
+        X = torch.randn(M, K, generator=gen, device=dev).to(torch.bfloat16)
+        ws = eqat.workspace(M, N, K, b, g, torch.bfloat16, dev)
+        Y = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
+
+        def timed_graph(fn, n_calls):
+            fn()
+            torch.cuda.synchronize()
+            gr = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(gr, stream=side):
+                fn()
+            gr.replay()
+            torch.cuda.synchronize()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            for _ in range(3):
+                gr.replay()
+            e1.record()
+            torch.cuda.synchronize()
+            return e0.elapsed_time(e1) * 1e3 / (3 * n_calls)
+
+        def run():
+            for c, z, s_ in layers:
+                eqat.dq_linear_fwd(X, c, z, s_, b, g, ws=ws, Y=Y)
+
+        t = timed_graph(run, L)
+        del layers
+        Lb = max(2, -(-budget_bytes // (N * K * 2)))
+        Ws = [torch.randn(N, K, generator=gen, device=dev).to(torch.bfloat16) for _ in range(Lb)]
+
+        def runb():
+            for W in Ws:
+                torch.matmul(X, W.t(), out=Y)
+
+        tb = timed_graph(runb, Lb)
+        del Ws
+        torch.cuda.empty_cache()
+        byts = per + M * K * 2 + M * N * 2
+        gbs = byts / (t * 1e-6) / 1e9
+        out[name] = {"N": N, "K": K, "M": M, "bits": b, "group": g, "us": round(t, 2), "GBps": round(gbs, 1),
+                     "frac_hbm": round(gbs / peaks["hbm_gbs"], 4), "bf16_matvec_us": round(tb, 2),
+                     "speedup_vs_bf16_matvec": round(tb / t, 2), "layers_cycled": L}
+    out["note"] = ("GPU time per call from a CUDA graph of back-to-back calls (3 kernels per call: X fragments, "
+                   "the streaming kernel, the partial sum); bf16 matvec = torch.matmul on bf16 weights, same method")
     return out
 
 
@@ -564,10 +631,31 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-initpack70b", action="store_true")
     ap.add_argument("--no-variants", action="store_true")
+    ap.add_argument("--no-gemv", action="store_true")
+    ap.add_argument("--gemv-only", action="store_true")
     ap.add_argument("--initpack70b-only", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)  # timing rule: at least 3 untimed warm-up steps
+    if args.gemv_only:  # profiling aid: four plain decode GEMV calls, Llama-2-70B gate_proj w2g64, M = 1
+        torch.cuda.set_device(0)
+        eqat.load_library()
+        dev = torch.device("cuda", 0)
+        N, K, b, g = 28672, 8192, 2, 64
+        gen = torch.Generator(device=dev)
+        gen.manual_seed(2000 + N)
+        c = torch.randint(0, 256, (N, K * b // 8), generator=gen, device=dev, dtype=torch.uint8)
+        z = torch.randint(0, 1 << b, (N, K // g), generator=gen, device=dev, dtype=torch.uint8)
+        s_ = torch.rand(N, K // g, generator=gen, device=dev) * 0.01 + 1e-3
+        X = torch.randn(1, K, generator=gen, device=dev).to(torch.bfloat16)
+        ws = eqat.workspace(1, N, K, b, g, torch.bfloat16, dev)
+        for _ in range(4):
+            eqat.dq_linear_fwd(X, c, z, s_, b, g, ws=ws)
+        torch.cuda.synchronize()
+        if eqat.device_error() != 0:
+            raise RuntimeError("device error word set")
+        print(json.dumps({"gemv_only": "ok"}), flush=True)
+        return
     if args.initpack70b_only:  # profiling aid: just the 70B-block init/pack measurement
         torch.cuda.set_device(0)
         eqat.load_library()

@@ -100,8 +100,11 @@ const char *eqat_last_error_detail(void);
 int eqat_version(void);
 
 /* Bytes of device workspace that the linear entry points need for this shape
- * (0 when none).  Depends only on N, K and dt; M, bits and group are accepted
- * so that later versions may add split-K partials without an ABI change. */
+ * (0 when none): W-hat (N K elements of dt; fp32 mode also an fp32 N K scratch),
+ * and for eqat_dq_linear_fwd at decode sizes (bf16, 1 <= M <= 8, group 64 or
+ * 128) the larger of that and the decode path's scratch (X's fragments, group
+ * sums of X and per-row-tile partials).  A workspace of only N K * sizeof(dt)
+ * bytes still works there: the call then dequantizes W-hat and runs the GEMM. */
 size_t eqat_workspace_bytes(int64_t M, int64_t N, int64_t K, int bits, int group, int dt);
 
 /* a1. Per-group min-max initialisation (modelfoundations note, Phase 1):
@@ -159,7 +162,10 @@ eqat_status eqat_fq_linear_bwd(const void *X, const void *W, int dt, const float
                                void *ws, size_t ws_bytes, int w_hat_in_ws, eqat_stream_t stream);
 
 /* a8. E2E-QP forward on frozen codes (modelfoundations Phase 2: only
- * dequantization in the graph): Y = X ((W_q - zq) s)^T. */
+ * dequantization in the graph): Y = X ((W_q - zq) s)^T.  At decode sizes (bf16,
+ * 1 <= M <= 8, group 64 or 128, workspace of eqat_workspace_bytes()) the codes are
+ * streamed once and W-hat is never written: the inference GEMV of the packed
+ * model. */
 eqat_status eqat_dq_linear_fwd(const void *X, int dt, const uint8_t *codes, const uint8_t *zq,
                                const float *s, void *Y, int64_t M, int64_t N, int64_t K, int bits,
                                int group, void *ws, size_t ws_bytes, eqat_stream_t stream);

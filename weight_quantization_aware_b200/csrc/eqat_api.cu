@@ -3,8 +3,10 @@
 // synchronises (except eqat_device_error) or falls back to another device.
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <cstdint>
 #include <cstdio>
+#include <cstdlib>
 #include <cstring>
 #include <mutex>
 
@@ -118,6 +120,16 @@ eqat_status check_sdtype(int sdt) {
 
 size_t esize(int dt) { return dt == EQAT_F32 ? 4 : 2; }
 
+// The decode-size path of eqat_dq_linear_fwd; EQAT_DQ_GEMV=0 turns it off
+// (measurement aid: the dequant + GEMM path at the same sizes).
+bool gemv_enabled() {
+    static const bool on = [] {
+        const char *v = std::getenv("EQAT_DQ_GEMV");
+        return !(v && v[0] == '0');
+    }();
+    return on;
+}
+
 int64_t code_bytes(int64_t N, int64_t K, int bits) {
     return bits == 2 ? N * (K / 4) : bits == 4 ? N * (K / 2) : N * K;
 }
@@ -184,11 +196,12 @@ const char *eqat_last_error_detail(void) { return g_detail; }
 int eqat_version(void) { return EQAT_VERSION; }
 
 size_t eqat_workspace_bytes(int64_t M, int64_t N, int64_t K, int bits, int group, int dt) {
-    (void)M;
-    (void)bits;
-    (void)group;
     if (N <= 0 || K <= 0 || (dt != EQAT_F32 && dt != EQAT_BF16)) return 0;
-    return ws_need(N, K, dt);
+    size_t need = ws_need(N, K, dt);
+    // the decode path (bf16, M <= 8) keeps X's fragments and partials here
+    if (dt == EQAT_BF16 && M >= 1 && M <= 8 && (group == 64 || group == 128) && bits >= 2 && bits <= 4)
+        need = std::max(need, (eqat::gemv_workspace_bound(M, N, K, bits, group) + 255) & ~static_cast<size_t>(255));
+    return need;
 }
 
 eqat_status eqat_minmax_init(const void *W, int wdt, int64_t N, int64_t K, int bits, int group, float *s,
@@ -422,6 +435,14 @@ eqat_status eqat_dq_linear_fwd_ex(const void *X, int dt, const uint8_t *codes, c
         return EQAT_OK;
     }
     const bool f32 = dt == EQAT_F32;
+    if (!f32 && M <= 8 && (group == 64 || group == 128) && gemv_enabled() &&
+        eqat::gemv_workspace_bytes(M, N, K, bits, group, dev.sm_count) <= ws_bytes) {
+        // decode sizes: stream the codes once, no W-hat in memory (a workspace
+        // sized for W-hat only, below eqat_workspace_bytes, takes the path below)
+        EQAT_CUDA(eqat::launch_dq_gemv(X, codes, zq, s, sdt == EQAT_F16, Y, M, N, K, bits, group, ws, dev, st),
+                  "dq GEMV");
+        return EQAT_OK;
+    }
     EQAT_CUDA(eqat::launch_dequant(codes, zq, s, sdt == EQAT_F16, N, K, bits, group, ws, f32, dev, st),
               "dequant prepass");
     EpiArgs epi;

@@ -898,6 +898,23 @@ Tiling choose_tiling(const GemmProblem *probs, int nprob, int sms) {
 
 }  // namespace
 
+int *device_error_word() { return device_error_ptr(); }
+
+cudaError_t encode_map_2d(CUtensorMap &map, CUtensorMapDataType type, const void *base, uint64_t inner,
+                          uint64_t outer, uint64_t stride_bytes, uint32_t box_inner, uint32_t box_outer,
+                          CUtensorMapSwizzle swizzle) {
+    cudaError_t e = get_encode();
+    if (e != cudaSuccess) return e;
+    cuuint64_t dims[2] = {inner, outer};
+    cuuint64_t strides[1] = {stride_bytes};
+    cuuint32_t box[2] = {box_inner, box_outer};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = g_encode(&map, type, 2, const_cast<void *>(base), dims, strides, box, estr,
+                          CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
 cudaError_t launch_gemm_tc_group(const GemmProblem *probs, int nprob, const DeviceInfo &dev,
                                  cudaStream_t st) {
     if (nprob < 1 || nprob > 2) return cudaErrorInvalidValue;

@@ -1,0 +1,735 @@
+// Batch-1..8 inference on frozen codes (E2E-QP forward at decode sizes):
+//   Y[m, n] = sum_k X[m, k] (W_q[n, k] - zq[n, g]) s[n, g]
+// (zhaoyang97 ACL2025 notes, Eq. 2; modelfoundations note, Phase 2: only
+// dequantization is left in the graph), read straight from the packed codes.
+//
+// At M <= 8 the layer is bound by HBM: 2-bit codes are 0.25 B per weight plus
+// 5/g B of s and zq, against 2 B per weight for a bf16 matrix.  The codes are
+// streamed once and W-hat is never formed in memory:
+//   - k_gemv_xprep turns X into the B-operand fragments of mma.sync m16n8k16,
+//     permuted and pre-scaled to match the A registers below, plus the per-group
+//     sums that remove the conversion offset and the zero point (a few KB per
+//     token octet, read from L2 afterwards);
+//   - in k_dq_gemv a producer warp moves 128-row x 128-byte code tiles into a
+//     shared-memory ring with TMA (128-byte swizzle, so the per-lane reads hit
+//     distinct banks), with the matching fragment slice by bulk copy;
+//   - eight consumer warps each own 16 rows.  A lane turns 16 codes of a row into
+//     eight bf16x2 registers with one AND-OR per register (the "magic number"
+//     conversion: code bits placed in the mantissa of 128.0 give 128 + code * 4^j
+//     exactly) and feeds them to mma.sync as the A operand:
+//       sum_k (c_k - zq) x_k = [sum_k (128 + c_k 4^j) (x_k 4^-j)] - xoff_g - zq xsum_g.
+// The tensor core is only a multiply-add engine for register-resident operands;
+// the roofline is HBM.
+//
+// Work: the stages (row tile, 128-byte column slab) in row-major order are split
+// into equal contiguous ranges, one per CTA, so each CTA streams along K of the
+// same rows (whole DRAM pages, s / zq sectors reused at once).  A CTA writes one
+// fp32 partial per row tile it touches; k_gemv_reduce sums the partials of each
+// row tile in CTA order (deterministic).
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <atomic>
+#include <cstdint>
+#include <cstdlib>
+
+#include "eqat_internal.h"
+#include "eqat_ptx.cuh"
+
+namespace eqat {
+namespace {
+
+constexpr int kConsumers = 8;              // consumer warps, 16 rows each
+constexpr int kRows = 16 * kConsumers;     // rows of a tile
+constexpr int kThreads = (kConsumers + 1) * 32;
+constexpr int kRowBytes = 128;             // code bytes of one row per stage
+constexpr int kCodeTile = kRows * kRowBytes;
+constexpr int kMaxSets = 8;                // 64-column sets per stage, at most (2-bit)
+constexpr int kMaxGps = 8;                 // groups per stage, at most (2-bit, g = 64)
+constexpr int kTableSlice = kMaxSets * 1024;  // B fragments of one stage
+constexpr int kXoSlice = kMaxGps * 64;        // {xoff, xsum} x 8 tokens of one stage
+// codes at the start of a stage: 1024-byte aligned for the 128-byte swizzle
+constexpr int kStageBytes = (kCodeTile + kTableSlice + kXoSlice + 1023) / 1024 * 1024;
+constexpr int kStages = 6;
+constexpr int kSlots = 2;                  // s / zq staging slots per consumer warp
+constexpr uint64_t kWaitLimitNs = 4000000000ull;
+
+// Shared-memory layout (after 1024-byte alignment): the stage ring, then the
+// s / zq slots, then the barriers.
+constexpr int kOffSz = kStages * kStageBytes;
+constexpr int kSzBytes = kConsumers * kSlots * 16 * kMaxGps * 8;
+constexpr int kOffBar = kOffSz + kSzBytes;
+constexpr int kSmemBytes = 1024 + kOffBar + 256;
+
+// Codes of one lane for one 64-column set of a row: 16 codes (columns 16t..16t+15
+// of the set).  extract() produces eight bf16x2 registers; register e holds codes
+// lo(e) (low half) and hi(e) (high half), scaled by 4^scale_exp(e), plus 128.
+constexpr uint32_t kMagic = 0x43004300u;  // bf16x2 {128.0, 128.0}
+
+template <int BITS>
+struct Codes;
+
+// 2-bit: one 32-bit word, code q at bits 2q.  Only mantissa bits 0..5 of each
+// half are usable, so three codes per half are taken per shift.
+template <>
+struct Codes<2> {
+    static constexpr int kBytes = 4;         // per lane per set
+    static constexpr int kCodeBits = 2;
+    __device__ static void extract(const uint32_t *w, uint32_t (&a)[8]) {
+        const uint32_t w0 = w[0], w6 = w[0] >> 6, w12 = w[0] >> 12;
+        a[0] = (w0 & 0x00030003u) | kMagic;
+        a[1] = (w0 & 0x000C000Cu) | kMagic;
+        a[2] = (w0 & 0x00300030u) | kMagic;
+        a[3] = (w6 & 0x00030003u) | kMagic;
+        a[4] = (w6 & 0x000C000Cu) | kMagic;
+        a[5] = (w6 & 0x00300030u) | kMagic;
+        a[6] = (w12 & 0x00030003u) | kMagic;
+        a[7] = (w12 & 0x000C000Cu) | kMagic;
+    }
+    __host__ __device__ static constexpr int lo(int e) { return e; }
+    __host__ __device__ static constexpr int hi(int e) { return e + 8; }
+    __host__ __device__ static constexpr int scale_exp(int e) { return e % 3; }
+    // scale exponent of the code at position q (0..15) of the lane's 16
+    __host__ __device__ static constexpr int pos_exp(int q) { return (q % 8) % 3; }
+};
+
+// 4-bit: two words, code q at bits 4(q % 8) of word q / 8.
+template <>
+struct Codes<4> {
+    static constexpr int kBytes = 8;
+    static constexpr int kCodeBits = 4;
+    __device__ static void extract(const uint32_t *w, uint32_t (&a)[8]) {
+#pragma unroll
+        for (int p = 0; p < 2; ++p) {
+            const uint32_t v = w[p];
+            a[4 * p + 0] = (v & 0x000F000Fu) | kMagic;
+            a[4 * p + 1] = ((v >> 4) & 0x000F000Fu) | kMagic;
+            a[4 * p + 2] = ((v >> 8) & 0x000F000Fu) | kMagic;
+            a[4 * p + 3] = ((v >> 12) & 0x000F000Fu) | kMagic;
+        }
+    }
+    __host__ __device__ static constexpr int lo(int e) { return e < 4 ? e : e + 4; }
+    __host__ __device__ static constexpr int hi(int e) { return lo(e) + 4; }
+    __host__ __device__ static constexpr int scale_exp(int) { return 0; }
+    __host__ __device__ static constexpr int pos_exp(int) { return 0; }
+};
+
+// 3-bit codes stored one per byte: four words, byte q = code q.  Seven mantissa
+// bits are taken so that any byte below 128 converts exactly.
+template <>
+struct Codes<3> {
+    static constexpr int kBytes = 16;
+    static constexpr int kCodeBits = 8;
+    __device__ static void extract(const uint32_t *w, uint32_t (&a)[8]) {
+#pragma unroll
+        for (int p = 0; p < 4; ++p) {
+            a[2 * p] = (w[p] & 0x007F007Fu) | kMagic;
+            a[2 * p + 1] = ((w[p] >> 8) & 0x007F007Fu) | kMagic;
+        }
+    }
+    __host__ __device__ static constexpr int lo(int e) { return 4 * (e / 2) + (e % 2); }
+    __host__ __device__ static constexpr int hi(int e) { return lo(e) + 2; }
+    __host__ __device__ static constexpr int scale_exp(int) { return 0; }
+    __host__ __device__ static constexpr int pos_exp(int) { return 0; }
+};
+
+// Codes per stage along K: one 128-byte row segment.
+template <int BITS>
+constexpr int stage_codes() {
+    return kRowBytes * 8 / Codes<BITS>::kCodeBits;
+}
+
+
+// Contiguous global -> shared copy whose completion is counted on `bar` (both
+// addresses 16-byte aligned, size a multiple of 16).
+__device__ __forceinline__ void bulk_load(void *smem_dst, const void *src, uint32_t bytes, uint64_t *bar) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+            smem_u32(smem_dst)),
+        "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(smem_u32(bar))
+        : "memory");
+}
+
+struct GemvParams {
+    const uint8_t *zq;
+    const void *s;
+    const uint4 *table;  // B fragments of X: [sets_pad][2][32]
+    const float2 *xso;   // {xoff, xsum}: [groups_pad][8 tokens]
+    float *partials;     // [row_tiles][maxseg][M][kRows]
+    int M, N, G;
+    int64_t K;
+    int spr;             // stages per row tile (along K)
+    int row_tiles;
+    int maxseg;          // partial slots per row tile
+    int vec;             // s / zq rows allow vector loads (G a multiple of the per-thread run)
+    int64_t total_stages;
+    int *err;
+    uint64_t wait_limit_ns;
+};
+
+// The CTA whose stage range holds stage x, for ranges [c S / grid, (c+1) S / grid).
+__host__ __device__ __forceinline__ int cta_of_stage(int64_t x, int64_t S, int grid) {
+    return static_cast<int>(((x + 1) * grid - 1) / S);
+}
+
+// Programmatic dependent launch: a kernel launched with programmatic stream
+// serialization may start before its predecessor ends; pdl_wait() blocks the
+// calling thread until the predecessor has completed and its writes are visible.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_allow_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
+// Stage x = rt * spr + ks, advanced without divisions.
+struct StageCursor {
+    int64_t x;
+    int rt, ks;
+    __device__ __forceinline__ void init(int64_t x0, int spr) {
+        x = x0;
+        rt = static_cast<int>(x0 / spr);
+        ks = static_cast<int>(x0 - static_cast<int64_t>(rt) * spr);
+    }
+    __device__ __forceinline__ void next(int spr) {
+        ++x;
+        if (++ks == spr) {
+            ks = 0;
+            ++rt;
+        }
+    }
+};
+
+__device__ __forceinline__ uint32_t bf16x2_bits(float lo, float hi) {
+    const __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<const uint32_t *>(&v);
+}
+
+// X -> B fragments and per-group sums, for the whole of K (padded with zeros to
+// whole stages).  One block per group, GROUP threads.  Thread i builds entry
+// (set j, ip, l) of the group's sets = {mma 2ip: b0b1, b2b3; mma 2ip+1: b0b1,
+// b2b3} for token l / 4 and column quad l % 4 (b0b1 of mma i pair with A register
+// 2i: columns lo, hi scaled by 4^-scale_exp; b2b3 with register 2i + 1).  It also
+// reads column i of the group for the 8 tokens, and the block sums them into
+// xoff = sum 128 x 4^-j and xsum = sum x per token.
+template <int BITS, int GROUP>
+__global__ void __launch_bounds__(GROUP) k_gemv_xprep(const __nv_bfloat16 *__restrict__ X, int M, int64_t K,
+                                                        uint4 *__restrict__ table, float2 *__restrict__ xso) {
+    using C = Codes<BITS>;
+    constexpr int WARPS = GROUP / 32;
+    __shared__ float red[WARPS][16];
+    pdl_allow_dependents();
+    const int gidx = blockIdx.x;
+    auto xv = [&](int tok, int64_t k) -> float {
+        return (tok < M && k < K) ? __bfloat162float(X[static_cast<int64_t>(tok) * K + k]) : 0.0f;
+    };
+    {
+        const int j = gidx * (GROUP / 64) + (threadIdx.x >> 6);
+        const int ip = (threadIdx.x >> 5) & 1, l = threadIdx.x & 31;
+        const int n = l >> 2, t = l & 3;
+        const int64_t kb = 64 * static_cast<int64_t>(j) + 16 * t;
+        uint32_t r[4];
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+#pragma unroll
+            for (int sl = 0; sl < 2; ++sl) {
+                const int e = 2 * (2 * ip + h) + sl;
+                const float sc = (C::scale_exp(e) == 0) ? 1.0f : (C::scale_exp(e) == 1 ? 0.25f : 0.0625f);
+                r[2 * h + sl] = bf16x2_bits(xv(n, kb + C::lo(e)) * sc, xv(n, kb + C::hi(e)) * sc);
+            }
+        }
+        table[(static_cast<int64_t>(j) * 2 + ip) * 32 + l] = make_uint4(r[0], r[1], r[2], r[3]);
+    }
+    // column sums
+    const int64_t k = static_cast<int64_t>(gidx) * GROUP + threadIdx.x;
+    const int ex = C::pos_exp(threadIdx.x & 15);
+    const float w = ex == 0 ? 128.0f : (ex == 1 ? 32.0f : 8.0f);
+    float so[8], ss[8];
+#pragma unroll
+    for (int tok = 0; tok < 8; ++tok) {
+        ss[tok] = xv(tok, k);
+        so[tok] = ss[tok] * w;
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) {
+#pragma unroll
+        for (int tok = 0; tok < 8; ++tok) {
+            ss[tok] += __shfl_xor_sync(0xffffffffu, ss[tok], off);
+            so[tok] += __shfl_xor_sync(0xffffffffu, so[tok], off);
+        }
+    }
+    const int warp = threadIdx.x >> 5;
+    if ((threadIdx.x & 31) == 0) {
+#pragma unroll
+        for (int tok = 0; tok < 8; ++tok) {
+            red[warp][tok] = so[tok];
+            red[warp][8 + tok] = ss[tok];
+        }
+    }
+    __syncthreads();
+    if (threadIdx.x < 8) {
+        float a = 0.0f, b = 0.0f;
+#pragma unroll
+        for (int w2 = 0; w2 < WARPS; ++w2) {
+            a += red[w2][threadIdx.x];
+            b += red[w2][8 + threadIdx.x];
+        }
+        xso[static_cast<int64_t>(gidx) * 8 + threadIdx.x] = make_float2(a, b);
+    }
+}
+
+// s and zq of one stage (128 rows x GPS groups), four values per consumer thread
+// at most, loaded into registers two stages ahead of their use.
+struct SzRegs {
+    float s[4], z[4];
+};
+
+// Each consumer warp stages the s and zq of its own 16 rows: lane l takes row
+// l / 2 and VPT = GPS / 2 consecutive groups (GPS = 1: lanes 0..15, one each).
+// When the row strides allow it (p.vec: G a multiple of VPT) and the stage lies
+// inside K, s and zq come in one vector load each.
+template <int BITS, int GROUP>
+struct SzShape {
+    static constexpr int GPS = stage_codes<BITS>() / GROUP;
+    static constexpr int VPT = GPS >= 2 ? GPS / 2 : 1;
+    static constexpr int TPR = GPS >= 2 ? 2 : 1;  // lanes per row
+    static constexpr int SLOT = 16 * GPS;         // float2 entries of one warp slot
+};
+
+template <int BITS, int GROUP, bool S16>
+__device__ __forceinline__ void load_sz(const GemvParams &p, const StageCursor &c, int64_t x_end, int row0,
+                                        int lane, SzRegs &r) {
+    using Sh = SzShape<BITS, GROUP>;
+    constexpr int VPT = Sh::VPT, TPR = Sh::TPR;
+#pragma unroll
+    for (int v = 0; v < 4; ++v) {
+        r.s[v] = 0.0f;
+        r.z[v] = 0.0f;
+    }
+    const int row = lane / TPR, part = lane % TPR;
+    if (c.x >= x_end || row >= 16) return;
+    const int64_t n = static_cast<int64_t>(c.rt) * kRows + row0 + row;
+    const int64_t g = static_cast<int64_t>(c.ks) * Sh::GPS + part * VPT;
+    if (n >= p.N) return;
+    const int64_t i = n * p.G + g;
+    if (p.vec && g + VPT <= p.G) {
+        if (VPT == 4) {
+            if (S16) {
+                const uint2 h = __ldg(reinterpret_cast<const uint2 *>(static_cast<const __half *>(p.s) + i));
+                const __half2 h0 = *reinterpret_cast<const __half2 *>(&h.x), h1 = *reinterpret_cast<const __half2 *>(&h.y);
+                r.s[0] = __low2float(h0); r.s[1] = __high2float(h0); r.s[2] = __low2float(h1); r.s[3] = __high2float(h1);
+            } else {
+                const float4 f = __ldg(reinterpret_cast<const float4 *>(static_cast<const float *>(p.s) + i));
+                r.s[0] = f.x; r.s[1] = f.y; r.s[2] = f.z; r.s[3] = f.w;
+            }
+            const uint32_t z = __ldg(reinterpret_cast<const uint32_t *>(p.zq + i));
+#pragma unroll
+            for (int v = 0; v < 4; ++v) r.z[v] = static_cast<float>((z >> (8 * v)) & 0xFFu);
+        } else if (VPT == 2) {
+            if (S16) {
+                const __half2 h = __ldg(reinterpret_cast<const __half2 *>(static_cast<const __half *>(p.s) + i));
+                r.s[0] = __low2float(h); r.s[1] = __high2float(h);
+            } else {
+                const float2 f = __ldg(reinterpret_cast<const float2 *>(static_cast<const float *>(p.s) + i));
+                r.s[0] = f.x; r.s[1] = f.y;
+            }
+            const uint32_t z = __ldg(reinterpret_cast<const unsigned short *>(p.zq + i));
+            r.z[0] = static_cast<float>(z & 0xFFu);
+            r.z[1] = static_cast<float>(z >> 8);
+        } else {
+            r.s[0] = S16 ? __half2float(__ldg(static_cast<const __half *>(p.s) + i))
+                         : __ldg(static_cast<const float *>(p.s) + i);
+            r.z[0] = static_cast<float>(__ldg(p.zq + i));
+        }
+        return;
+    }
+#pragma unroll
+    for (int v = 0; v < VPT; ++v) {
+        if (g + v < p.G) {
+            r.s[v] = S16 ? __half2float(__ldg(static_cast<const __half *>(p.s) + i + v))
+                         : __ldg(static_cast<const float *>(p.s) + i + v);
+            r.z[v] = static_cast<float>(__ldg(p.zq + i + v));
+        }
+    }
+}
+
+// Into the warp's slot, entry row * GPS + group (rows local to the warp).
+template <int BITS, int GROUP>
+__device__ __forceinline__ void store_sz(float2 *slot, int lane, const SzRegs &r) {
+    using Sh = SzShape<BITS, GROUP>;
+    const int row = lane / Sh::TPR, part = lane % Sh::TPR;
+    if (row >= 16) return;
+    float2 *d = slot + row * Sh::GPS + part * Sh::VPT;
+#pragma unroll
+    for (int v = 0; v < Sh::VPT; ++v) d[v] = make_float2(r.s[v], r.z[v]);
+}
+
+__device__ __forceinline__ void mma_bf16(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                         uint32_t b0, uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+        "{%0, %1, %2, %3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// Byte b of row r of a 128-byte-swizzled code tile.
+__device__ __forceinline__ uint32_t swz(int r, int b) {
+    return static_cast<uint32_t>(r * kRowBytes + ((((b >> 4) ^ (r & 7))) << 4) + (b & 15));
+}
+
+template <int BITS>
+__device__ __forceinline__ void load_codes(const uint8_t *tile, int row, int byte, uint32_t *w) {
+    const uint8_t *ptr = tile + swz(row, byte);
+    if (Codes<BITS>::kBytes == 4) {
+        w[0] = *reinterpret_cast<const uint32_t *>(ptr);
+    } else if (Codes<BITS>::kBytes == 8) {
+        const uint2 v = *reinterpret_cast<const uint2 *>(ptr);
+        w[0] = v.x;
+        w[1] = v.y;
+    } else {
+        const uint4 v = *reinterpret_cast<const uint4 *>(ptr);
+        w[0] = v.x;
+        w[1] = v.y;
+        w[2] = v.z;
+        w[3] = v.w;
+    }
+}
+
+
+template <int BITS, int GROUP, bool S16>
+__global__ void __launch_bounds__(kThreads, 1)
+    k_dq_gemv(const __grid_constant__ CUtensorMap tm_codes, const GemvParams p) {
+    using C = Codes<BITS>;
+    constexpr int KS = stage_codes<BITS>();
+    constexpr int SETS = KS / 64;                     // 64-column sets per stage
+    constexpr int SET_BYTES = 64 * C::kCodeBits / 8;  // code bytes of a set in one row
+    constexpr int SPG = GROUP / 64;                   // sets per group
+    constexpr int GPS = KS / GROUP;                   // groups per stage
+    constexpr uint32_t TABLE_BYTES = SETS * 1024;
+    constexpr uint32_t XO_BYTES = GPS * 64;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                                ~static_cast<uintptr_t>(1023));
+    float2 *sz = reinterpret_cast<float2 *>(smem + kOffSz);
+    uint64_t *full = reinterpret_cast<uint64_t *>(smem + kOffBar);
+    uint64_t *empty = full + kStages;
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(empty + kStages);
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < kStages; ++i) {
+            mbar_init(&full[i], 1);
+            mbar_init(&empty[i], kConsumers);
+        }
+        *abort_flag = 0;
+        fence_mbarrier_init();
+        tma_prefetch_desc(&tm_codes);
+        pdl_allow_dependents();
+    }
+    __syncthreads();
+
+    const int64_t S = p.total_stages;
+    const int64_t x_begin = static_cast<int64_t>(blockIdx.x) * S / gridDim.x;
+    const int64_t x_end = static_cast<int64_t>(blockIdx.x + 1) * S / gridDim.x;
+
+    if (warp == kConsumers) {
+        // ------------------------------------------------------------ producer
+        if (elect_one_sync()) {
+            // X's fragments and sums come from the preceding k_gemv_xprep
+            pdl_wait();
+            uint32_t armed = 0, armed_parity = 0;
+            bool ok = true;
+            uint32_t it = 0;
+            StageCursor c;
+            c.init(x_begin, p.spr);
+            for (; c.x < x_end; c.next(p.spr), ++it) {
+                const int st = it % kStages;
+                const uint32_t ph = (it / kStages) & 1u;
+                if (!mbar_wait_bounded(&empty[st], ph ^ 1u, abort_flag, p.err, p.wait_limit_ns)) {
+                    ok = false;
+                    break;
+                }
+                const int rt = c.rt, ks = c.ks;
+                uint8_t *stage = smem + st * kStageBytes;
+                mbar_arrive_expect_tx(&full[st], kCodeTile + TABLE_BYTES + XO_BYTES);
+                armed |= 1u << st;
+                armed_parity = (armed_parity & ~(1u << st)) | (ph << st);
+                tma_load_2d(stage, &tm_codes, &full[st], ks * kRowBytes, rt * kRows);
+                bulk_load(stage + kCodeTile, p.table + static_cast<int64_t>(ks) * SETS * 64, TABLE_BYTES, &full[st]);
+                bulk_load(stage + kCodeTile + kTableSlice, p.xso + static_cast<int64_t>(ks) * GPS * 8, XO_BYTES,
+                          &full[st]);
+            }
+            if (!ok) {
+                // let issued copies land before the block can exit
+                for (int st = 0; st < kStages; ++st)
+                    if (armed & (1u << st)) {
+                        const uint32_t a = smem_u32(&full[st]);
+                        const uint64_t t0 = globaltimer_ns();
+                        while (!mbar_try_wait(a, (armed_parity >> st) & 1u) &&
+                               globaltimer_ns() - t0 < 100000000ull) {
+                        }
+                    }
+            }
+        }
+        __syncwarp();
+        return;
+    }
+
+    // ---------------------------------------------------------------- consumers
+    const int r0 = lane >> 2, t = lane & 3;
+    const int row_a = warp * 16 + r0, row_b = row_a + 8;
+    // this warp's s / zq slots: [kSlots][16 rows][GPS] float2
+    float2 *szw = sz + warp * (kSlots * 16 * kMaxGps);
+
+    // s / zq pipeline, per warp: stage x's values are loaded at the start of stage
+    // x - 3 into one of three register sets and stored to the warp's slot at the
+    // end of stage x - 1.
+    SzRegs sa_, sb_, sc_;
+    StageCursor cur, pf;
+    cur.init(x_begin, p.spr);
+    pf = cur;
+    load_sz<BITS, GROUP, S16>(p, pf, x_end, warp * 16, lane, sa_);
+    pf.next(p.spr);
+    store_sz<BITS, GROUP>(szw, lane, sa_);
+    load_sz<BITS, GROUP, S16>(p, pf, x_end, warp * 16, lane, sb_);
+    pf.next(p.spr);
+    load_sz<BITS, GROUP, S16>(p, pf, x_end, warp * 16, lane, sc_);
+    pf.next(p.spr);
+    float y[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+    bool ok = true;
+    __syncwarp();
+
+    uint32_t it = 0;
+    auto stage = [&](SzRegs &load_into, const SzRegs &store_from) {
+        load_sz<BITS, GROUP, S16>(p, pf, x_end, warp * 16, lane, load_into);
+        pf.next(p.spr);
+        const int st = it % kStages;
+        const uint32_t ph = (it / kStages) & 1u;
+        ok = mbar_wait_bounded(&full[st], ph, abort_flag, p.err, p.wait_limit_ns) && ok;
+        const uint8_t *tile = smem + st * kStageBytes;
+        const uint4 *table = reinterpret_cast<const uint4 *>(tile + kCodeTile);
+        const float2 *xo = reinterpret_cast<const float2 *>(tile + kCodeTile + kTableSlice);
+        const float2 *szs = szw + (it % kSlots) * (16 * kMaxGps);
+        // Groups of the stage are independent: two accumulator chains per group
+        // (mmas 0, 2 and 1, 3 of each set), so the unrolled groups overlap.
+#pragma unroll
+        for (int gi = 0; gi < GPS; ++gi) {
+            float a0[4] = {0.0f, 0.0f, 0.0f, 0.0f}, a1[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+#pragma unroll
+            for (int q = 0; q < SPG; ++q) {
+                const int m = gi * SPG + q;
+                uint32_t wa[C::kBytes / 4], wb[C::kBytes / 4];
+                load_codes<BITS>(tile, row_a, m * SET_BYTES + t * C::kBytes, wa);
+                load_codes<BITS>(tile, row_b, m * SET_BYTES + t * C::kBytes, wb);
+                uint32_t ea[8], eb[8];
+                C::extract(wa, ea);
+                C::extract(wb, eb);
+                const uint4 b01 = table[(m * 2 + 0) * 32 + lane];
+                const uint4 b23 = table[(m * 2 + 1) * 32 + lane];
+                mma_bf16(a0, ea[0], eb[0], ea[1], eb[1], b01.x, b01.y);
+                mma_bf16(a1, ea[2], eb[2], ea[3], eb[3], b01.z, b01.w);
+                mma_bf16(a0, ea[4], eb[4], ea[5], eb[5], b23.x, b23.y);
+                mma_bf16(a1, ea[6], eb[6], ea[7], eb[7], b23.z, b23.w);
+            }
+            const float2 sa = szs[r0 * GPS + gi], sb = szs[(r0 + 8) * GPS + gi];
+            const float4 ox = *reinterpret_cast<const float4 *>(xo + gi * 8 + 2 * t);  // tokens 2t, 2t+1
+            // ox = {xoff(2t), xsum(2t), xoff(2t+1), xsum(2t+1)}
+            y[0] = fmaf(sa.x, (a0[0] + a1[0]) - fmaf(sa.y, ox.y, ox.x), y[0]);
+            y[1] = fmaf(sa.x, (a0[1] + a1[1]) - fmaf(sa.y, ox.w, ox.z), y[1]);
+            y[2] = fmaf(sb.x, (a0[2] + a1[2]) - fmaf(sb.y, ox.y, ox.x), y[2]);
+            y[3] = fmaf(sb.x, (a0[3] + a1[3]) - fmaf(sb.y, ox.w, ox.z), y[3]);
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty[st]);
+
+        // s / zq of the next stage into its slot
+        store_sz<BITS, GROUP>(szw + ((it + 1) % kSlots) * (16 * kMaxGps), lane, store_from);
+
+        const int rt = cur.rt;
+        cur.next(p.spr);
+        ++it;
+        if (cur.x == x_end || cur.ks == 0) {
+            // this CTA is done with row tile rt: its partial goes to slot
+            // (rt, cta - first cta of rt); rows rt*128 + row_a / row_b, tokens 2t, 2t+1
+            const int seg = static_cast<int>(blockIdx.x) -
+                            cta_of_stage(static_cast<int64_t>(rt) * p.spr, S, static_cast<int>(gridDim.x));
+            float *P = p.partials + (static_cast<int64_t>(rt) * p.maxseg + seg) * p.M * kRows;
+            const int m0 = 2 * t, m1 = m0 + 1;
+            if (m0 < p.M) {
+                P[m0 * kRows + row_a] = y[0];
+                P[m0 * kRows + row_b] = y[2];
+            }
+            if (m1 < p.M) {
+                P[m1 * kRows + row_a] = y[1];
+                P[m1 * kRows + row_b] = y[3];
+            }
+            y[0] = y[1] = y[2] = y[3] = 0.0f;
+        }
+        __syncwarp();  // the next stage's slot is written
+    };
+    while (cur.x < x_end) {
+        stage(sa_, sb_);
+        if (cur.x >= x_end) break;
+        stage(sb_, sc_);
+        if (cur.x >= x_end) break;
+        stage(sc_, sa_);
+    }
+    (void)ok;
+}
+
+// Y[m][n] = sum over the CTAs that touched row tile n / kRows, in CTA order, of
+// their partials.
+__global__ void k_gemv_reduce(const float *__restrict__ partials, int M, int N, int spr, int maxseg,
+                              int64_t S, int grid, __nv_bfloat16 *__restrict__ Y) {
+    pdl_wait();  // the partials of the preceding k_dq_gemv
+    const int64_t MN = static_cast<int64_t>(M) * N;
+    for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < MN;
+         i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+        const int m = static_cast<int>(i / N), n = static_cast<int>(i % N);
+        const int rt = n / kRows, row = n % kRows;
+        const int c0 = cta_of_stage(static_cast<int64_t>(rt) * spr, S, grid);
+        const int c1 = cta_of_stage(static_cast<int64_t>(rt) * spr + spr - 1, S, grid);
+        float a = 0.0f;
+        for (int c = c0; c <= c1; ++c)
+            a += partials[((static_cast<int64_t>(rt) * maxseg + (c - c0)) * M + m) * kRows + row];
+        Y[i] = __float2bfloat16_rn(a);
+    }
+}
+
+// Launch with programmatic stream serialization (may overlap the predecessor).
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st, Args... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, args...);
+}
+
+struct Plan {
+    int spr, row_tiles, maxseg, grid;
+    int64_t S;
+    size_t table_bytes, xso_bytes, partial_bytes;
+};
+
+Plan make_plan(int64_t M, int64_t N, int64_t K, int bits, int group, int sms) {
+    Plan pl{};
+    const int ks = bits == 2 ? stage_codes<2>() : bits == 4 ? stage_codes<4>() : stage_codes<3>();
+    pl.spr = static_cast<int>((K + ks - 1) / ks);
+    pl.row_tiles = static_cast<int>((N + kRows - 1) / kRows);
+    pl.S = static_cast<int64_t>(pl.spr) * pl.row_tiles;
+    pl.grid = static_cast<int>(std::min<int64_t>(pl.S, sms));
+    pl.maxseg = 1;
+    for (int rt = 0; rt < pl.row_tiles; ++rt) {
+        const int c0 = cta_of_stage(static_cast<int64_t>(rt) * pl.spr, pl.S, pl.grid);
+        const int c1 = cta_of_stage(static_cast<int64_t>(rt) * pl.spr + pl.spr - 1, pl.S, pl.grid);
+        pl.maxseg = std::max(pl.maxseg, c1 - c0 + 1);
+    }
+    const int64_t sets = static_cast<int64_t>(pl.spr) * (ks / 64);
+    const int64_t groups = static_cast<int64_t>(pl.spr) * (ks / group);
+    pl.table_bytes = static_cast<size_t>(sets) * 1024;
+    pl.xso_bytes = (static_cast<size_t>(groups) * 64 + 255) / 256 * 256;
+    pl.partial_bytes = static_cast<size_t>(pl.row_tiles) * pl.maxseg * M * kRows * 4;
+    return pl;
+}
+
+template <int BITS, int GROUP, bool S16>
+cudaError_t launch_main(const CUtensorMap &map, const GemvParams &p, int grid, int dev_id, cudaStream_t st) {
+    auto kern = k_dq_gemv<BITS, GROUP, S16>;
+    static std::atomic<uint64_t> done{0};
+    const uint64_t bit = 1ull << (dev_id & 63);
+    if (!(done.load() & bit)) {
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+        if (e != cudaSuccess) return e;
+        done.fetch_or(bit);
+    }
+    return launch_pdl(kern, dim3(grid), dim3(kThreads), kSmemBytes, st, map, p);
+}
+
+template <int BITS, int GROUP>
+cudaError_t launch_all(const CUtensorMap &map, const __nv_bfloat16 *X, GemvParams p, const Plan &pl, bool s_f16,
+                       __nv_bfloat16 *Y, const DeviceInfo &dev, cudaStream_t st) {
+    const int64_t groups = static_cast<int64_t>(pl.spr) * (stage_codes<BITS>() / GROUP);
+    k_gemv_xprep<BITS, GROUP><<<static_cast<unsigned>(groups), GROUP, 0, st>>>(
+        X, p.M, p.K, const_cast<uint4 *>(p.table), const_cast<float2 *>(p.xso));
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    e = s_f16 ? launch_main<BITS, GROUP, true>(map, p, pl.grid, dev.device, st)
+              : launch_main<BITS, GROUP, false>(map, p, pl.grid, dev.device, st);
+    if (e != cudaSuccess) return e;
+    const int64_t MN = static_cast<int64_t>(p.M) * p.N;
+    const unsigned rblocks = static_cast<unsigned>(std::min<int64_t>((MN + 255) / 256, 2 * dev.sm_count));
+    return launch_pdl(k_gemv_reduce, dim3(rblocks), dim3(256), 0, st, static_cast<const float *>(p.partials), p.M,
+                      p.N, pl.spr, pl.maxseg, pl.S, pl.grid, Y);
+}
+
+}  // namespace
+
+size_t gemv_workspace_bytes(int64_t M, int64_t N, int64_t K, int bits, int group, int sm_count) {
+    const Plan pl = make_plan(M, N, K, bits, group, sm_count);
+    return pl.table_bytes + pl.xso_bytes + pl.partial_bytes;
+}
+
+size_t gemv_workspace_bound(int64_t M, int64_t N, int64_t K, int bits, int group) {
+    // at most one CTA per stage, so at most S partial slots in all
+    const Plan pl = make_plan(M, N, K, bits, group, 1);
+    return pl.table_bytes + pl.xso_bytes + static_cast<size_t>(pl.S) * M * kRows * 4;
+}
+
+cudaError_t launch_dq_gemv(const void *X, const uint8_t *codes, const uint8_t *zq, const void *s, bool s_f16,
+                           void *Y, int64_t M, int64_t N, int64_t K, int bits, int group, void *ws,
+                           const DeviceInfo &dev, cudaStream_t st) {
+    if (M < 1 || M > 8 || N <= 0 || K <= 0 || (group != 64 && group != 128)) return cudaErrorInvalidValue;
+    if (bits != 2 && bits != 3 && bits != 4) return cudaErrorInvalidValue;
+    if (N > INT32_MAX - kRows || K > INT32_MAX) return cudaErrorInvalidValue;
+    const Plan pl = make_plan(M, N, K, bits, group, dev.sm_count);
+    const int code_bits = bits == 3 ? 8 : bits;
+    const uint64_t row_bytes = static_cast<uint64_t>(K) * code_bits / 8;
+    CUtensorMap map;
+    cudaError_t e = encode_map_2d(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, codes, row_bytes, static_cast<uint64_t>(N),
+                                  row_bytes, kRowBytes, kRows, CU_TENSOR_MAP_SWIZZLE_128B);
+    if (e != cudaSuccess) return e;
+    uint8_t *w = static_cast<uint8_t *>(ws);
+    GemvParams p{};
+    p.zq = zq;
+    p.s = s;
+    p.table = reinterpret_cast<const uint4 *>(w);
+    p.xso = reinterpret_cast<const float2 *>(w + pl.table_bytes);
+    p.partials = reinterpret_cast<float *>(w + pl.table_bytes + pl.xso_bytes);
+    p.M = static_cast<int>(M);
+    p.N = static_cast<int>(N);
+    p.G = static_cast<int>(K / group);
+    p.K = K;
+    p.spr = pl.spr;
+    p.row_tiles = pl.row_tiles;
+    p.maxseg = pl.maxseg;
+    {
+        const int gps = (bits == 2 ? stage_codes<2>() : bits == 4 ? stage_codes<4>() : stage_codes<3>()) / group;
+        const int vpt = gps >= 2 ? gps / 2 : 1;
+        p.vec = (p.G % vpt == 0) ? 1 : 0;
+    }
+    p.total_stages = pl.S;
+    p.err = device_error_word();
+    p.wait_limit_ns = kWaitLimitNs;
+    const __nv_bfloat16 *Xb = static_cast<const __nv_bfloat16 *>(X);
+    __nv_bfloat16 *Yb = static_cast<__nv_bfloat16 *>(Y);
+#define EQAT_GEMV_CASE(B, GR) \
+    if (bits == B && group == GR) return launch_all<B, GR>(map, Xb, p, pl, s_f16, Yb, dev, st);
+    EQAT_GEMV_CASE(2, 64)
+    EQAT_GEMV_CASE(2, 128)
+    EQAT_GEMV_CASE(3, 64)
+    EQAT_GEMV_CASE(3, 128)
+    EQAT_GEMV_CASE(4, 64)
+    EQAT_GEMV_CASE(4, 128)
+#undef EQAT_GEMV_CASE
+    return cudaErrorInvalidValue;
+}
+
+}  // namespace eqat

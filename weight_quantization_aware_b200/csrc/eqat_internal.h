@@ -3,6 +3,7 @@
 
 #include <cstddef>
 #include <cstdint>
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 namespace eqat {
@@ -93,6 +94,22 @@ cudaError_t launch_gemm_tc(const Operand &A, const Operand &B, int64_t GM, int64
 cudaError_t launch_gemm_f32(const Operand &A, const Operand &B, int64_t GM, int64_t GN, int64_t GK,
                             const EpiArgs &epi, float *d_scratch, const DeviceInfo &dev,
                             cudaStream_t st);
+
+// Batch-1..8 inference: Y[M, N] = X[M, K] ((W_q - zq) s)^T straight from packed
+// codes, bf16 X and Y, M in 1..8, group 64 or 128.  `ws` holds at least
+// gemv_workspace_bytes(...) bytes (256-byte aligned): X's fragments, the group
+// sums of X and the per-row-tile partials.
+size_t gemv_workspace_bytes(int64_t M, int64_t N, int64_t K, int bits, int group, int sm_count);
+size_t gemv_workspace_bound(int64_t M, int64_t N, int64_t K, int bits, int group);  // any SM count
+cudaError_t launch_dq_gemv(const void *X, const uint8_t *codes, const uint8_t *zq, const void *s, bool s_f16,
+                           void *Y, int64_t M, int64_t N, int64_t K, int bits, int group, void *ws,
+                           const DeviceInfo &dev, cudaStream_t st);
+
+// Shared by the kernels that use TMA and bounded waits.
+int *device_error_word();
+cudaError_t encode_map_2d(CUtensorMap &map, CUtensorMapDataType type, const void *base, uint64_t inner,
+                          uint64_t outer, uint64_t stride_bytes, uint32_t box_inner, uint32_t box_outer,
+                          CUtensorMapSwizzle swizzle);
 
 // Records the message that eqat_last_error_detail() returns on this thread.
 void set_error_detail(const char *msg);

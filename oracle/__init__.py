@@ -18,6 +18,7 @@ NumPy arrays; float outputs of the contractions are fp64.
 from __future__ import annotations
 
 import ctypes
+import math
 import os
 import subprocess
 
@@ -54,6 +55,7 @@ def _load():
         P = ctypes.c_void_p
         I64 = ctypes.c_int64
         I = ctypes.c_int
+        D = ctypes.c_double
         sig = {
             "orc_minmax_init": [P, I64, I64, I, I, P, P],
             "orc_fake_quant": [P, P, P, I64, I64, I, I, P, P, P, P],
@@ -66,6 +68,7 @@ def _load():
             "orc_e2e_ds": [P, P, P, P, I64, I64, I64, I, I, P],
             "orc_ste_grads_clamp_pass": [P, P, P, P, P, I64, I64, I64, I, I, P, P, P],
             "orc_e2e_dz": [P, P, P, I64, I64, I64, I, P],
+            "orc_adamw": [P, P, P, P, I64, D, D, D, D, D, I64],
         }
         for name, args in sig.items():
             fn = getattr(lib, name)
@@ -230,6 +233,31 @@ def e2e_dz(s, dWhat, K, group, wrows=None):
     dz = np.empty((n_out, K // group), np.float64)
     _load().orc_e2e_dz(_p(s), _p(dWhat), _p(r), nr, N, K, group, _p(dz))
     return dz
+
+
+def adamw(p, g, m, v, lr, b1, b2, eps, wd, t):
+    """One AdamW step (decoupled weight decay) on fp32 state; returns new (p, m, v)."""
+    p, m, v = (np.array(a, dtype=np.float32, copy=True) for a in (p, m, v))
+    g = _f32(g)
+    assert p.shape == g.shape == m.shape == v.shape and t >= 1
+    _load().orc_adamw(_p(p), _p(g), _p(m), _p(v), p.size, float(lr), float(b1), float(b2), float(eps),
+                      float(wd), int(t))
+    return p, m, v
+
+
+def cosine_lr(lr0, lr_min, t, total):
+    """Cosine annealing of the learning rate at step t of `total` ([MF] Phase 1: weights and
+    quantization parameters on separate cosine schedules): lr_min + (lr0 - lr_min)(1 + cos(pi t / total)) / 2."""
+    return lr_min + (lr0 - lr_min) * (1.0 + math.cos(math.pi * t / total)) / 2.0
+
+
+def mse_grad(Y, T):
+    """Reconstruction loss of Block-AP against the full-precision output ([MF] "Both phases": MSE
+    to FP block outputs), mean over all elements, and its gradient dL/dY = 2 (Y - T) / numel."""
+    Y = np.asarray(Y, dtype=np.float64)
+    T = np.asarray(T, dtype=np.float64)
+    R = Y - T
+    return float(np.sum(R * R) / R.size), 2.0 * R / R.size
 
 
 # ----------------------------------------------------------------------------

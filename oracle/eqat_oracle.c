@@ -360,6 +360,34 @@ void orc_e2e_dz(const float *s, const double *dWhat, const int64_t *wrows, int64
     }
 }
 
+/* One AdamW step (decoupled weight decay) at step t >= 1 over n parameters, for
+ * the Block-AP update of W, s and z ([MF] Phase 1 and "Paper vs. code": AdamW,
+ * weights and quantization parameters in separate learning-rate groups).  The
+ * pages print no formula; this is the textbook algorithm of Loshchilov & Hutter
+ * as PyTorch's AdamW states it:
+ *   p <- p (1 - lr wd)
+ *   m <- b1 m + (1 - b1) g,   v <- b2 v + (1 - b2) g^2
+ *   p <- p - lr (m / (1 - b1^t)) / (sqrt(v / (1 - b2^t)) + eps)
+ * in fp64 on fp32 state, each stored value rounded to fp32 once. */
+void orc_adamw(float *p, const float *g, float *m, float *v, int64_t n, double lr, double b1, double b2,
+               double eps, double wd, int64_t t)
+{
+    const double bc1 = 1.0 - pow(b1, (double)t);
+    const double bc2 = 1.0 - pow(b2, (double)t);
+#pragma omp parallel for schedule(static)
+    for (int64_t i = 0; i < n; ++i) {
+        const double gi = (double)g[i];
+        double pi = (double)p[i] * (1.0 - lr * wd);
+        const double mi = b1 * (double)m[i] + (1.0 - b1) * gi;
+        const double vi = b2 * (double)v[i] + (1.0 - b2) * gi * gi;
+        const float m32 = (float)mi, v32 = (float)vi;
+        pi -= lr * ((double)m32 / bc1) / (sqrt((double)v32 / bc2) + eps);
+        m[i] = m32;
+        v[i] = v32;
+        p[i] = (float)pi;
+    }
+}
+
 int orc_num_threads(void)
 {
 #ifdef _OPENMP

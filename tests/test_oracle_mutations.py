@@ -40,6 +40,9 @@ MUTANTS = {
     "e2e_dz_wrong_sign": ("dz[r * G + j] = -(double)s[n * G + j] * acc;",
                           "dz[r * G + j] = (double)s[n * G + j] * acc;"),
     "e2e_dz_drops_scale": ("dz[r * G + j] = -(double)s[n * G + j] * acc;", "dz[r * G + j] = -acc;"),
+    "adamw_bias_correction_outside_sqrt": ("pi -= lr * ((double)m32 / bc1) / (sqrt((double)v32 / bc2) + eps);",
+                                           "pi -= lr * ((double)m32 / bc1) / (sqrt((double)v32) / bc2 + eps);"),
+    "adamw_without_decoupled_decay": ("double pi = (double)p[i] * (1.0 - lr * wd);", "double pi = (double)p[i];"),
     "e2e_ds_ignores_zero_point": ("const double diff = (double)orc_code_at(packed, K, bits, n, k) - (double)zq[n * G + j];",
                                   "const double diff = (double)orc_code_at(packed, K, bits, n, k);"),
 }

@@ -615,3 +615,63 @@ def test_effective_bits_closed_form():
         extra = (16 + bits) / g
         assert 0.1 < extra < 0.3
     assert abs(1 / 64 - 0.0156) < 1e-3
+
+
+# ---------------------------------------------------------------- Block-AP optimizer step
+
+@pytest.mark.parametrize("wd", [0.0, 0.01])
+def test_adamw_matches_torch_optim_adamw(orc, wd):
+    """The oracle's AdamW against torch.optim.AdamW (fp64, CPU) with the two learning-rate
+    groups of Block-AP (weights 2e-5, quantization parameters 1e-4) over five steps."""
+    rng = np.random.default_rng(21)
+    shapes = {"W": (6, 16), "s": (6, 4)}
+    lrs = {"W": 2e-5, "s": 1e-4}
+    p0 = {k: (rng.standard_normal(sh) * (0.02 if k == "W" else 0.005) + (0 if k == "W" else 0.01)).astype(np.float32)
+          for k, sh in shapes.items()}
+    tp = {k: torch.tensor(p0[k].astype(np.float64), requires_grad=True) for k in shapes}
+    opt = torch.optim.AdamW([{"params": [tp["W"]], "lr": lrs["W"]}, {"params": [tp["s"]], "lr": lrs["s"]}],
+                            betas=(0.9, 0.999), eps=1e-8, weight_decay=wd)
+    st = {k: (p0[k].copy(), np.zeros_like(p0[k]), np.zeros_like(p0[k])) for k in shapes}
+    for t in range(1, 6):
+        grads = {k: (rng.standard_normal(sh) * 0.1).astype(np.float32) for k, sh in shapes.items()}
+        for k in shapes:
+            tp[k].grad = torch.tensor(grads[k].astype(np.float64))
+        opt.step()
+        for k in shapes:
+            p, m, v = st[k]
+            st[k] = orc.adamw(p, grads[k], m, v, lrs[k], 0.9, 0.999, 1e-8, wd, t)
+        for k in shapes:
+            ref = tp[k].detach().numpy()
+            got = st[k][0].astype(np.float64)
+            # fp32 storage of p, m and v: within a few ulps of p per step
+            assert np.abs(got - ref).max() <= 4 * t * np.spacing(np.abs(ref).max().astype(np.float32))
+            state = opt.state[tp[k]]
+            # m is a signed running sum: compare against its scale, not element-wise
+            m_ref, v_ref = state["exp_avg"].numpy(), state["exp_avg_sq"].numpy()
+            assert np.abs(st[k][1] - m_ref).max() <= 1e-6 * np.abs(m_ref).max()
+            np.testing.assert_allclose(st[k][2], v_ref, rtol=2e-6, atol=1e-16)
+        assert np.abs(st["W"][0] - p0["W"]).max() > 0
+
+
+def test_cosine_schedule_matches_torch_scheduler(orc):
+    """Closed form of cosine annealing against torch.optim.lr_scheduler.CosineAnnealingLR."""
+    T, lr0, lr_min = 37, 1e-4, 1e-6
+    p = torch.nn.Parameter(torch.zeros(1))
+    opt = torch.optim.AdamW([p], lr=lr0)
+    sch = torch.optim.lr_scheduler.CosineAnnealingLR(opt, T_max=T, eta_min=lr_min)
+    for t in range(T + 1):
+        assert abs(opt.param_groups[0]["lr"] - orc.cosine_lr(lr0, lr_min, t, T)) <= 1e-12 * lr0
+        opt.step()
+        sch.step()
+
+
+def test_mse_gradient_matches_autograd(orc):
+    rng = np.random.default_rng(3)
+    Y = rng.standard_normal((5, 7))
+    T = rng.standard_normal((5, 7))
+    Yt = torch.tensor(Y, requires_grad=True)
+    loss = ((Yt - torch.tensor(T)) ** 2).mean()
+    loss.backward()
+    l, dY = orc.mse_grad(Y, T)
+    assert abs(l - loss.item()) <= 1e-14
+    np.testing.assert_allclose(dY, Yt.grad.numpy(), rtol=1e-14, atol=1e-16)

@@ -215,6 +215,59 @@ eqat_status eqat_dq_linear_bwd(const void *X, int dt, const uint8_t *codes, cons
                                float *dz, int64_t M, int64_t N, int64_t K, int bits, int group,
                                void *ws, size_t ws_bytes, int w_hat_in_ws, eqat_stream_t stream);
 
+/* Block-AP step (modelfoundations note, Phase 1: each block is trained against the
+ * full-precision block's outputs with an MSE loss, by AdamW with the weights and
+ * the quantization parameters in separate learning-rate groups on cosine
+ * schedules).
+ *
+ * eqat_fq_linear_fwd_mse: the forward of eqat_fq_linear_fwd against a target T
+ * (the full-precision output, [M,N] of dtype dt), without storing Y:
+ *   dY = 2 (Y - T) / (M N)   [M,N], dtype dt (the loss gradient, input of eqat_fq_linear_bwd)
+ *   *loss = sum (Y - T)^2 / (M N)   one fp64 value in device memory, 8-byte aligned (overwritten)
+ * In EQAT_BF16 mode the subtraction runs on Y's fp32 accumulator in the GEMM
+ * epilogue; the loss is summed with atomics, so its last bits depend on order. */
+eqat_status eqat_fq_linear_fwd_mse(const void *X, const void *W, int dt, const float *s, const float *z,
+                                   const void *T, void *dY, double *loss, int64_t M, int64_t N, int64_t K,
+                                   int bits, int group, void *ws, size_t ws_bytes, eqat_stream_t stream);
+
+/* One AdamW step (decoupled weight decay, Loshchilov & Hutter; the pages print
+ * no formula) over up to 32 tensors in one launch, step >= 1:
+ *   p <- p (1 - lr wd);  m <- b1 m + (1 - b1) g;  v <- b2 v + (1 - b2) g^2
+ *   p <- p - lr / (1 - b1^step) * m / (sqrt(v) / sqrt(1 - b2^step) + eps)
+ * in fp32.  param, exp_avg, exp_avg_sq are fp32 device arrays updated in place;
+ * grad is EQAT_F32 or EQAT_BF16; param_copy (nullable) receives the updated
+ * parameter in copy_dtype (EQAT_BF16 for the weights the next forward reads, or
+ * EQAT_F32).  All pointers 16-byte aligned.  Hyperparameters come from
+ * groups[tensor.group] (double: 1 - beta2 is formed before rounding to the
+ * kernel's fp32 constants); the bias corrections are computed here in double. */
+typedef struct {
+    float *param;
+    const void *grad;
+    int grad_dtype;
+    float *exp_avg;
+    float *exp_avg_sq;
+    void *param_copy;
+    int copy_dtype;
+    int group;
+    int64_t numel;
+} eqat_adamw_tensor;
+
+typedef struct {
+    double lr;
+    double beta1;
+    double beta2;
+    double eps;
+    double weight_decay;
+} eqat_adamw_group;
+
+#define EQAT_ADAMW_MAX_TENSORS 32
+eqat_status eqat_adamw_step(const eqat_adamw_tensor *tensors, int n_tensors, const eqat_adamw_group *groups,
+                            int n_groups, int64_t step, eqat_stream_t stream);
+
+/* Cosine annealing (host): lr_min + (lr0 - lr_min) (1 + cos(pi step / total)) / 2,
+ * step in [0, total]; the learning rate of step `step` of a schedule of `total`. */
+double eqat_cosine_lr(double lr0, double lr_min, int64_t step, int64_t total);
+
 /* Block-AP forward (as eqat_fq_linear_fwd) that allocates nothing and takes no
  * workspace: the paper has no counterpart; this entry point exists for callers of
  * the library that cannot allocate device memory or pass a scratch buffer (a

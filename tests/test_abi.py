@@ -140,3 +140,32 @@ def test_binding_refuses_cpu_tensors():
     W = torch.zeros(16, 64, dtype=torch.bfloat16)
     with pytest.raises(ValueError):
         eqat.minmax_init(W, 2, 64)
+
+
+def test_blockap_entry_points_argument_errors(lib):
+    st = None
+    # loss must be 8-byte aligned and non-NULL; the rest as for the forward
+    assert lib.eqat_fq_linear_fwd_mse(P(FAKE), P(FAKE), 1, P(FAKE), P(FAKE), P(FAKE), P(FAKE), P(0),
+                                      16, 16, 64, 2, 64, P(FAKE), 1 << 20, st) == NULL
+    assert lib.eqat_fq_linear_fwd_mse(P(FAKE), P(FAKE), 1, P(FAKE), P(FAKE), P(FAKE), P(FAKE), P(FAKE + 4),
+                                      16, 16, 64, 2, 64, P(FAKE), 1 << 20, st) == ALIGN
+    assert lib.eqat_fq_linear_fwd_mse(P(FAKE), P(FAKE), 1, P(FAKE), P(FAKE), P(0), P(FAKE), P(FAKE),
+                                      16, 16, 64, 2, 64, P(FAKE), 1 << 20, st) == NULL
+    T = eqat.AdamwTensor(FAKE, FAKE, 1, FAKE, FAKE, None, 0, 0, 64)
+    G = eqat.AdamwGroup(1e-4, 0.9, 0.999, 1e-8, 0.0)
+    args = lambda t, ng, g, step: (ctypes.byref(t), 1, ctypes.byref(g), ng, step, st)
+    assert lib.eqat_adamw_step(*args(T, 1, G, 0)) == SHAPE          # step >= 1
+    assert lib.eqat_adamw_step(*args(T, 0, G, 1)) == SHAPE          # no groups
+    bad = eqat.AdamwGroup(1e-4, 1.0, 0.999, 1e-8, 0.0)
+    assert lib.eqat_adamw_step(*args(T, 1, bad, 1)) == UNSUP        # beta1 = 1
+    T2 = eqat.AdamwTensor(FAKE, FAKE, 7, FAKE, FAKE, None, 0, 0, 64)
+    assert lib.eqat_adamw_step(*args(T2, 1, G, 1)) == DTYPE
+    T3 = eqat.AdamwTensor(FAKE, FAKE, 1, FAKE, FAKE, None, 0, 3, 64)
+    assert lib.eqat_adamw_step(*args(T3, 1, G, 1)) == SHAPE         # group index
+    T4 = eqat.AdamwTensor(FAKE + 8, FAKE, 1, FAKE, FAKE, None, 0, 0, 64)
+    assert lib.eqat_adamw_step(*args(T4, 1, G, 1)) == ALIGN
+    T0 = eqat.AdamwTensor(FAKE, FAKE, 1, FAKE, FAKE, None, 0, 0, 0)
+    assert lib.eqat_adamw_step(*args(T0, 1, G, 1)) == OK            # nothing to do
+    assert abs(eqat.cosine_lr(1e-4, 0.0, 0, 10) - 1e-4) < 1e-18
+    assert abs(eqat.cosine_lr(1e-4, 0.0, 10, 10)) < 1e-18
+    assert abs(eqat.cosine_lr(1e-4, 1e-6, 5, 10) - (1e-6 + (1e-4 - 1e-6) / 2)) < 1e-15

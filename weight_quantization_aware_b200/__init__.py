@@ -59,6 +59,8 @@ def load_library():
         "eqat_dequant_codes_ex": [P, P, P, I, I64, I64, I, I, P, I, P],
         "eqat_dq_linear_fwd_ex": [P, I, P, P, P, I, P, I64, I64, I64, I, I, P, SZ, P],
         "eqat_dq_linear_bwd": [P, I, P, P, P, I, P, P, P, P, I64, I64, I64, I, I, P, SZ, I, P],
+        "eqat_fq_linear_fwd_mse": [P, P, I, P, P, P, P, P, I64, I64, I64, I, I, P, SZ, P],
+        "eqat_adamw_step": [P, I, P, I, I64, P],
         "eqat_device_error": [P, P],
         "eqat_selftest_bounded_wait": [I64, P],
     }
@@ -71,6 +73,8 @@ def load_library():
     lib.eqat_last_error_detail.argtypes = []
     lib.eqat_last_error_detail.restype = ctypes.c_char_p
     lib.eqat_version.restype = I
+    lib.eqat_cosine_lr.argtypes = [ctypes.c_double, ctypes.c_double, I64, I64]
+    lib.eqat_cosine_lr.restype = ctypes.c_double
     lib.eqat_workspace_bytes.argtypes = [I64, I64, I64, I, I, I]
     lib.eqat_workspace_bytes.restype = SZ
     _lib = lib
@@ -303,6 +307,57 @@ def dq_linear_bwd(X, codes, zq, s, dY, bits, group, need_dx=True, need_ds=True, 
     _call("eqat_dq_linear_bwd", _p(X), _dt(X), _p(codes), _p(zq), _p(s), _sdt(s), _p(dY), _p(dX), _p(ds),
           _p(dz), M, N, K, bits, group, _p(ws), ws.numel(), int(bool(w_hat_in_ws)), _stream())
     return dX, ds, dz
+
+
+def fq_linear_fwd_mse(X, W, s, z, T, bits, group, ws=None, dY=None, loss=None):
+    """Block-AP forward against the full-precision output T, Y not stored: returns
+    (dY = 2 (Y - T) / (M N), loss = mean (Y - T)^2 as a 1-element fp64 CUDA tensor)."""
+    _req(X, "X"); _req(W, "W", X.dtype); _req(s, "s", torch.float32); _req(z, "z", torch.float32)
+    _req(T, "T", X.dtype)
+    M, K = X.shape
+    N = W.shape[0]
+    dY = torch.empty((M, N), dtype=X.dtype, device=X.device) if dY is None else _req(dY, "dY", X.dtype)
+    loss = torch.empty(1, dtype=torch.float64, device=X.device) if loss is None else _req(loss, "loss", torch.float64)
+    ws = _ws(ws, M, N, K, bits, group, X.dtype, X.device)
+    _call("eqat_fq_linear_fwd_mse", _p(X), _p(W), _dt(X), _p(s), _p(z), _p(T), _p(dY), _p(loss), M, N, K, bits,
+          group, _p(ws), ws.numel(), _stream())
+    return dY, loss
+
+
+class AdamwTensor(ctypes.Structure):
+    _fields_ = [("param", ctypes.c_void_p), ("grad", ctypes.c_void_p), ("grad_dtype", ctypes.c_int),
+                ("exp_avg", ctypes.c_void_p), ("exp_avg_sq", ctypes.c_void_p), ("param_copy", ctypes.c_void_p),
+                ("copy_dtype", ctypes.c_int), ("group", ctypes.c_int), ("numel", ctypes.c_int64)]
+
+
+class AdamwGroup(ctypes.Structure):
+    _fields_ = [("lr", ctypes.c_double), ("beta1", ctypes.c_double), ("beta2", ctypes.c_double),
+                ("eps", ctypes.c_double), ("weight_decay", ctypes.c_double)]
+
+
+def adamw_step(entries, groups, step):
+    """One fused AdamW step.  entries: list of (param fp32, grad fp32|bf16, exp_avg, exp_avg_sq,
+    param_copy or None, group index); groups: list of dicts lr, beta1, beta2, eps, weight_decay."""
+    arr = (AdamwTensor * max(1, len(entries)))()
+    for i, (p, g, m, v, c, gi) in enumerate(entries):
+        _req(p, "param", torch.float32); _req(m, "exp_avg", torch.float32); _req(v, "exp_avg_sq", torch.float32)
+        _req(g, "grad")
+        if c is not None:
+            _req(c, "param_copy")
+        arr[i] = AdamwTensor(p.data_ptr(), g.data_ptr(), _dt(g), m.data_ptr(), v.data_ptr(),
+                             c.data_ptr() if c is not None else None, _dt(c) if c is not None else EQAT_F32,
+                             int(gi), p.numel())
+    garr = (AdamwGroup * len(groups))()
+    for i, gr in enumerate(groups):
+        garr[i] = AdamwGroup(gr["lr"], gr.get("beta1", 0.9), gr.get("beta2", 0.999), gr.get("eps", 1e-8),
+                             gr.get("weight_decay", 0.0))
+    _call("eqat_adamw_step", ctypes.cast(arr, ctypes.c_void_p), len(entries), ctypes.cast(garr, ctypes.c_void_p),
+          len(groups), int(step), _stream())
+
+
+def cosine_lr(lr0, lr_min, step, total):
+    """The learning rate at `step` of a cosine schedule of `total` steps."""
+    return float(load_library().eqat_cosine_lr(lr0, lr_min, int(step), int(total)))
 
 
 def device_error():

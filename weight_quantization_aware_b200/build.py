@@ -14,7 +14,7 @@ CSRC = os.path.join(HERE, "csrc")
 OUT_DIR = os.path.join(HERE, "_build")
 LIB = os.path.join(HERE, "libeqat.so")
 SOURCES = ["eqat_api.cu", "eqat_quant.cu", "eqat_gemm_tc.cu", "eqat_gemm_f32.cu", "eqat_noalloc.cu",
-           "eqat_gemv.cu"]
+           "eqat_gemv.cu", "eqat_optim.cu"]
 HEADERS = ["eqat_ptx.cuh", "eqat_qmath.cuh", "eqat_internal.h"]
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]

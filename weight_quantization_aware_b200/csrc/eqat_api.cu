@@ -4,6 +4,7 @@
 #include <cuda_runtime.h>
 
 #include <algorithm>
+#include <cmath>
 #include <cstdint>
 #include <cstdio>
 #include <cstdlib>
@@ -531,6 +532,125 @@ eqat_status eqat_dq_linear_bwd(const void *X, int dt, const uint8_t *codes, cons
                       "E2E backward contraction (fp32)");
     }
     return EQAT_OK;
+}
+
+eqat_status eqat_fq_linear_fwd_mse(const void *X, const void *W, int dt, const float *s, const float *z,
+                                   const void *T, void *dY, double *loss, int64_t M, int64_t N, int64_t K,
+                                   int bits, int group, void *ws, size_t ws_bytes, eqat_stream_t stream) {
+    DeviceInfo dev;
+    EQAT_TRY(check_dtype(dt));
+    EQAT_TRY(check_common(M, N, K, bits, group));
+    const int64_t ng = N * (K / group);
+    EQAT_TRY(check_ptr(X, M * K, "X"));
+    EQAT_TRY(check_ptr(W, N * K, "W"));
+    EQAT_TRY(check_ptr(s, ng, "s"));
+    EQAT_TRY(check_ptr(z, ng, "z"));
+    EQAT_TRY(check_ptr(T, M * N, "T"));
+    EQAT_TRY(check_ptr(dY, M * N, "dY"));
+    if (!loss) return fail(EQAT_ERR_NULL, "loss is NULL");
+    if (!aligned(loss, 8)) return fail(EQAT_ERR_ALIGN, "loss is not 8-byte aligned");
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    if (M * N > 0 && K > 0) EQAT_TRY(check_ws(ws, ws_bytes, N, K, dt));
+    EQAT_TRY(get_device(dev));
+    EQAT_CUDA(zero(loss, sizeof(double), st), "memset loss");
+    if (M * N == 0) return EQAT_OK;
+    const bool f32 = dt == EQAT_F32;
+    const float scale = static_cast<float>(2.0 / (static_cast<double>(M) * static_cast<double>(N)));
+    if (K == 0) {  // Y = 0
+        if (f32) {
+            EQAT_CUDA(zero(dY, static_cast<size_t>(M * N) * esize(dt), st), "memset dY");
+            EQAT_CUDA(eqat::launch_mse_f32(static_cast<float *>(dY), static_cast<const float *>(T), M * N, scale, loss,
+                                           dev, st),
+                      "mse (fp32)");
+            return EQAT_OK;
+        }
+        EQAT_CUDA(eqat::launch_mse_zero_bf16(dY, T, M * N, scale, loss, dev, st), "mse (K == 0)");
+        return EQAT_OK;
+    }
+    EQAT_CUDA(eqat::launch_fake_quant(W, f32, s, z, N, K, bits, group, ws, f32, nullptr, nullptr, dev, st),
+              "fq prepass");
+    EpiArgs epi;
+    if (f32) {
+        epi.kind = Epi::kStore;
+        epi.out = dY;
+        epi.ldo = N;
+        epi.out_f32 = true;
+        EQAT_CUDA(contract(dt, Operand{X, K, false}, Operand{ws, K, false}, M, N, K, epi, nullptr, dev, st),
+                  "fq forward contraction");
+        EQAT_CUDA(eqat::launch_mse_f32(static_cast<float *>(dY), static_cast<const float *>(T), M * N, scale, loss,
+                                       dev, st),
+                  "mse (fp32)");
+        return EQAT_OK;
+    }
+    epi.kind = Epi::kMse;
+    epi.out = dY;
+    epi.ldo = N;
+    epi.target = T;
+    epi.loss = loss;
+    epi.mse_scale = scale;
+    EQAT_CUDA(eqat::launch_gemm_tc(Operand{X, K, false}, Operand{ws, K, false}, M, N, K, epi, dev, st),
+              "fq forward contraction with the MSE epilogue");
+    return EQAT_OK;
+}
+
+eqat_status eqat_adamw_step(const eqat_adamw_tensor *tensors, int n_tensors, const eqat_adamw_group *groups,
+                            int n_groups, int64_t step, eqat_stream_t stream) {
+    DeviceInfo dev;
+    if (!tensors || !groups) return fail(EQAT_ERR_NULL, "tensors or groups is NULL");
+    if (n_tensors < 0 || n_tensors > EQAT_ADAMW_MAX_TENSORS || n_groups < 1)
+        return fail(EQAT_ERR_SHAPE, "n_tensors must be 0..32 and n_groups >= 1");
+    if (step < 1) return fail(EQAT_ERR_SHAPE, "step must be >= 1");
+    for (int i = 0; i < n_groups; ++i) {
+        const eqat_adamw_group &g = groups[i];
+        if (!(g.beta1 >= 0.0 && g.beta1 < 1.0 && g.beta2 >= 0.0 && g.beta2 < 1.0 && g.eps > 0.0 && g.lr >= 0.0 &&
+              g.weight_decay >= 0.0))
+            return fail(EQAT_ERR_UNSUPPORTED, "AdamW hyperparameters out of range");
+    }
+    eqat::AdamwSeg segs[EQAT_ADAMW_MAX_TENSORS];
+    int n = 0;
+    for (int i = 0; i < n_tensors; ++i) {
+        const eqat_adamw_tensor &t = tensors[i];
+        if (t.numel < 0) return fail(EQAT_ERR_SHAPE, "numel < 0");
+        if (t.group < 0 || t.group >= n_groups) return fail(EQAT_ERR_SHAPE, "group index out of range");
+        if (t.grad_dtype != EQAT_F32 && t.grad_dtype != EQAT_BF16) return fail(EQAT_ERR_DTYPE, "grad_dtype");
+        if (t.param_copy && t.copy_dtype != EQAT_F32 && t.copy_dtype != EQAT_BF16) return fail(EQAT_ERR_DTYPE, "copy_dtype");
+        EQAT_TRY(check_ptr(t.param, t.numel, "param"));
+        EQAT_TRY(check_ptr(t.grad, t.numel, "grad"));
+        EQAT_TRY(check_ptr(t.exp_avg, t.numel, "exp_avg"));
+        EQAT_TRY(check_ptr(t.exp_avg_sq, t.numel, "exp_avg_sq"));
+        EQAT_TRY(check_ptr(t.param_copy, 0, "param_copy"));
+        if (t.numel == 0) continue;
+        const eqat_adamw_group &g = groups[t.group];
+        const double bc1 = 1.0 - std::pow(g.beta1, static_cast<double>(step));
+        const double bc2 = 1.0 - std::pow(g.beta2, static_cast<double>(step));
+        eqat::AdamwSeg &sg = segs[n++];
+        sg.p = t.param;
+        sg.g = t.grad;
+        sg.m = t.exp_avg;
+        sg.v = t.exp_avg_sq;
+        sg.copy = t.param_copy;
+        sg.n = t.numel;
+        sg.g_bf16 = t.grad_dtype == EQAT_BF16;
+        sg.copy_bf16 = t.copy_dtype == EQAT_BF16;
+        sg.decay = static_cast<float>(1.0 - g.lr * g.weight_decay);
+        sg.b1 = static_cast<float>(g.beta1);
+        sg.b2 = static_cast<float>(g.beta2);
+        sg.omb1 = static_cast<float>(1.0 - g.beta1);
+        sg.omb2 = static_cast<float>(1.0 - g.beta2);
+        sg.step_size = static_cast<float>(g.lr / bc1);
+        sg.inv_sqrt_bc2 = static_cast<float>(1.0 / std::sqrt(bc2));
+        sg.eps = static_cast<float>(g.eps);
+    }
+    if (n == 0) return EQAT_OK;
+    EQAT_TRY(get_device(dev));
+    EQAT_CUDA(eqat::launch_adamw(segs, n, dev, reinterpret_cast<cudaStream_t>(stream)), "adamw");
+    return EQAT_OK;
+}
+
+double eqat_cosine_lr(double lr0, double lr_min, int64_t step, int64_t total) {
+    if (total <= 0) return lr0;
+    const double pi = 3.14159265358979323846;
+    return lr_min + (lr0 - lr_min) * (1.0 + std::cos(pi * static_cast<double>(step) / static_cast<double>(total))) / 2.0;
 }
 
 eqat_status eqat_device_error(int *where, eqat_stream_t stream) {

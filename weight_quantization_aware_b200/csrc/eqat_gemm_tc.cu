@@ -75,6 +75,9 @@ struct Prob {
     const uint8_t *zq;
     const void *s_e2e;  // E2E step sizes (read for dz only), fp32 or fp16
     int s_f16;
+    const void *target; // reconstruction target (bf16, row stride ldo)
+    double *loss;
+    float mse_scale;
     int clamp_pass;     // Block-AP: the clamp is straight-through as well
     int group;
     int gshift;  // log2(group)
@@ -254,6 +257,54 @@ struct Epilogue<2, BITS> {
     }
 };
 
+// Block-AP reconstruction loss against the full-precision output T: D is Y[M, N]
+// (fp32, never stored).  dY = mse_scale (D - T) in bf16, and the thread's sum of
+// (D - T)^2 goes to *loss (fp64) when the drain ends.
+template <int BITS>
+struct Epilogue<3, BITS> {
+    float acc_s = 0.0f, acc_z = 0.0f;
+    __device__ __forceinline__ void chunk(const Prob &p, int row, int col, const float (&v)[32]) {
+        if (row >= p.GM) return;
+        const int64_t off = static_cast<int64_t>(row) * p.ldo + col;
+        const __nv_bfloat16 *T = static_cast<const __nv_bfloat16 *>(p.target) + off;
+        __nv_bfloat16 *out = static_cast<__nv_bfloat16 *>(p.out) + off;
+        if (col + 32 <= p.GN) {
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                float t[8];
+                load8<__nv_bfloat16>(T + 8 * q, t);
+                float r[8];
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    const float d = __fsub_rn(v[8 * q + j], t[j]);
+                    acc_s = fmaf(d, d, acc_s);
+                    r[j] = __fmul_rn(d, p.mse_scale);
+                }
+                store8<__nv_bfloat16>(out + 8 * q, r);
+            }
+        } else {
+#pragma unroll
+            for (int j = 0; j < 32; ++j)
+                if (col + j < p.GN) {
+                    const float d = __fsub_rn(v[j], __bfloat162float(T[j]));
+                    acc_s = fmaf(d, d, acc_s);
+                    out[j] = __float2bfloat16_rn(__fmul_rn(d, p.mse_scale));
+                }
+        }
+    }
+};
+
+template <int EPI>
+__device__ __forceinline__ void finish_drain(const Prob &p, float acc) {
+    if (EPI == 3) {
+        double a = acc;
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) a += __shfl_xor_sync(0xffffffffu, a, off);
+        // mse_scale = 2 / (M N): the loss is the mean
+        if ((threadIdx.x & 31) == 0) atomicAdd(p.loss, a * (0.5 * static_cast<double>(p.mse_scale)));
+    }
+}
+
 // Drains one accumulator (this warp's 32 rows, columns [c_begin, c_end)) through
 // the epilogue of kind EPI.
 template <int EPI, int BITS>
@@ -266,6 +317,7 @@ __device__ __forceinline__ void drain_accumulator(const Prob &pr, uint32_t taddr
         tmem_ld_32cols(taddr + c0, v);
         epi.chunk(pr, row, col0 + c0, v);
     }
+    finish_drain<EPI>(pr, epi.acc_s);
 }
 
 // Persistent grouped GEMM: problem 0 uses epilogue EPI0, problem 1 (if any)
@@ -833,6 +885,9 @@ cudaError_t fill_prob(Prob &q, const GemmProblem &g, int tile_begin, int bn, int
     q.codes = epi.codes;
     q.zq = epi.zq;
     q.s_e2e = epi.s_e2e;
+    q.target = epi.target;
+    q.loss = epi.loss;
+    q.mse_scale = epi.mse_scale;
     q.s_f16 = epi.s_f16 ? 1 : 0;
     q.clamp_pass = epi.clamp_pass ? 1 : 0;
     q.group = epi.group;
@@ -965,6 +1020,9 @@ cudaError_t launch_gemm_tc_group(const GemmProblem *probs, int nprob, const Devi
                     case 4: return launch_pair_variant<2, 0, 4>(maps, p, grid, dev.device, st);
                     default: return cudaErrorInvalidValue;
                 }
+            case Epi::kMse:
+                if (nprob > 1) return cudaErrorInvalidValue;
+                return launch_pair_variant<3, 0, 2>(maps, p, grid, dev.device, st);
         }
         return cudaErrorInvalidValue;
     }
@@ -982,6 +1040,9 @@ cudaError_t launch_gemm_tc_group(const GemmProblem *probs, int nprob, const Devi
                 case 4: return launch_variant<2, 0, 4>(maps, p, grid, dev.device, st);
                 default: return cudaErrorInvalidValue;
             }
+        case Epi::kMse:
+            if (nprob > 1) return cudaErrorInvalidValue;
+            return launch_variant<3, 0, 2>(maps, p, grid, dev.device, st);
     }
     return cudaErrorInvalidValue;
 }

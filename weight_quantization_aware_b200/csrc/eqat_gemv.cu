@@ -292,7 +292,6 @@ struct SzShape {
     static constexpr int GPS = stage_codes<BITS>() / GROUP;
     static constexpr int VPT = GPS >= 2 ? GPS / 2 : 1;
     static constexpr int TPR = GPS >= 2 ? 2 : 1;  // lanes per row
-    static constexpr int SLOT = 16 * GPS;         // float2 entries of one warp slot
 };
 
 template <int BITS, int GROUP, bool S16>

@@ -49,6 +49,7 @@ enum class Epi : int {
     kStore = 0,   // D -> out (bf16 or fp32), row stride ldo
     kFqGrad = 1,  // Block-AP straight-through: dW = D*mask, ds, dz per group
     kE2eDs = 2,   // E2E-QP: ds = sum_group D * (W_q - zq), dz = -s sum_group D
+    kMse = 3,     // reconstruction MSE: out = mse_scale (D - target) (bf16), *loss += sum (D - target)^2
 };
 
 struct EpiArgs {
@@ -70,6 +71,10 @@ struct EpiArgs {
     const uint8_t *zq = nullptr;
     const void *s_e2e = nullptr;
     bool s_f16 = false;
+    // kMse (out, ldo: dY)
+    const void *target = nullptr;  // [GM, GN] bf16, row stride ldo
+    double *loss = nullptr;
+    float mse_scale = 0.0f;
     int bits = 2;
     int group = 64;
 };
@@ -110,6 +115,33 @@ int *device_error_word();
 cudaError_t encode_map_2d(CUtensorMap &map, CUtensorMapDataType type, const void *base, uint64_t inner,
                           uint64_t outer, uint64_t stride_bytes, uint32_t box_inner, uint32_t box_outer,
                           CUtensorMapSwizzle swizzle);
+
+// Multi-tensor AdamW (decoupled weight decay), fp32 math on fp32 state.
+struct AdamwSeg {
+    float *p;
+    const void *g;
+    float *m;
+    float *v;
+    void *copy;      // nullable: updated parameter in bf16 (copy_bf16) or fp32
+    int64_t n;
+    int g_bf16;
+    int copy_bf16;
+    float decay;     // 1 - lr wd
+    float b1, b2;
+    float omb1, omb2;  // 1 - b1, 1 - b2 (formed in double)
+    float step_size; // lr / (1 - b1^t)
+    float inv_sqrt_bc2;  // 1 / sqrt(1 - b2^t)
+    float eps;
+};
+constexpr int kAdamwMaxSegs = 32;
+cudaError_t launch_adamw(const AdamwSeg *segs, int nseg, const DeviceInfo &dev, cudaStream_t st);
+
+// fp32 reconstruction MSE in place: dY = scale (dY - target), *loss += sum (dY - target)^2.
+cudaError_t launch_mse_f32(float *dY, const float *target, int64_t n, float scale, double *loss,
+                           const DeviceInfo &dev, cudaStream_t st);
+// Y = 0 (K == 0), bf16: dY = scale (0 - T), *loss += sum T^2 scale / 2.
+cudaError_t launch_mse_zero_bf16(void *dY, const void *target, int64_t n, float scale, double *loss,
+                                 const DeviceInfo &dev, cudaStream_t st);
 
 // Records the message that eqat_last_error_detail() returns on this thread.
 void set_error_detail(const char *msg);

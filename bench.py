@@ -373,6 +373,8 @@ def run_ours(args):
         line["variants"] = quantizer_variants(step, dev)
     if not args.no_gemv:
         line["decode_gemv"] = decode_gemv(dev, peaks)
+    if not args.no_blockap:
+        line["blockap_block"] = blockap_block(dev, peaks)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(target_s=args.cpu_seconds)
     if dist is not None:
@@ -429,6 +431,76 @@ def quantizer_variants(step, dev, reps=50):
         for name, fn in e2e.items():
             out[f"{name}_{sname}_TFLOPs"] = round(4 * M * N * K / (timed(lambda: fn(s_)) * 1e-3) / 1e12, 1)
     out["note"] = "4MNK per backward call, L2 flushed before each call, W-hat reused from the forward"
+    return out
+
+
+def blockap_block(dev, peaks, steps=5):
+    """Block-AP step over the seven linears of one Llama-2-7B decoder block (q, k, v, o
+    4096x4096; gate, up 11008x4096; down 4096x11008), 2-bit g64, 4096 tokens (batch 2 x
+    2048): per linear the fake-quant forward with the fused MSE epilogue against the
+    full-precision output and the straight-through backward (dW, ds, dz; no dX: the
+    inputs are the step's data), then one AdamW launch over all 21 tensors.  Synthetic
+    seeded inputs; targets = X W_fp^T.  The weights and optimizer state (2.8 GB) exceed L2,
+    so no flush.  TFLOP/s = sum 4 M N K / step time; AdamW GB/s = its algorithmic bytes
+    (28 per weight, 32 per s/z entry) / its own event time."""
+    from weight_quantization_aware_b200.blockap import BlockAPConfig, QuantLinearState, blockap_step
+    M = 4096
+    shapes = {"q_proj": (4096, 4096), "k_proj": (4096, 4096), "v_proj": (4096, 4096), "o_proj": (4096, 4096),
+              "gate_proj": (11008, 4096), "up_proj": (11008, 4096), "down_proj": (4096, 11008)}
+    cfg = BlockAPConfig(bits=2, group=64, total_steps=4096)
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(3007)
+    X_in = {K: torch.randn(M, K, generator=gen, device=dev).to(torch.bfloat16) for K in (4096, 11008)}
+    lin, Xs, Ts = [], [], []
+    flops = 0
+    for name, (N, K) in shapes.items():
+        W = torch.randn(N, K, generator=gen, device=dev) * 0.02
+        L = QuantLinearState.from_weight(W, cfg.bits, cfg.group, M)
+        X = X_in[K]
+        Ts.append(torch.matmul(X, W.to(torch.bfloat16).t()))  # the full-precision output
+        lin.append(L)
+        Xs.append(X)
+        flops += 4 * M * N * K
+        del W
+    losses = torch.empty(len(lin), dtype=torch.float64, device=dev)
+    blockap_step(lin, Xs, Ts, cfg, 1, losses)
+    torch.cuda.synchronize()
+    e = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+    e[0].record()
+    for t in range(2, 2 + steps):
+        blockap_step(lin, Xs, Ts, cfg, t, losses)
+    e[1].record()
+    torch.cuda.synchronize()
+    step_ms = e[0].elapsed_time(e[1]) / steps
+    # AdamW alone, same tensors and gradients
+    groups = [dict(lr=cfg.lr_w, weight_decay=0.0), dict(lr=cfg.lr_q, weight_decay=0.0)]
+    entries = []
+    nw = nq = 0
+    for L in lin:
+        _, dW, ds, dz = L.grads
+        entries += [(L.W_master, dW, *L.moments["W"], L.W, 0), (L.s, ds, *L.moments["s"], None, 1),
+                    (L.z, dz, *L.moments["z"], None, 1)]
+        nw += L.W_master.numel()
+        nq += L.s.numel() + L.z.numel()
+    ea = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+    eqat.adamw_step(entries, groups, 10)
+    ea[0].record()
+    for t in range(3):
+        eqat.adamw_step(entries, groups, 11 + t)
+    ea[1].record()
+    torch.cuda.synchronize()
+    adamw_ms = ea[0].elapsed_time(ea[1]) / 3
+    adamw_bytes = 28 * nw + 32 * nq
+    out = {"workload": "llama2-7b-block-blockap-w2g64-m4096 (7 linears, 202.4 M weights)",
+           "step_ms": round(step_ms, 3), "TFLOPs": round(flops / (step_ms * 1e-3) / 1e12, 1),
+           "flops_per_step": flops, "adamw_ms": round(adamw_ms, 3),
+           "adamw_GBps": round(adamw_bytes / (adamw_ms * 1e-3) / 1e9, 1),
+           "adamw_frac_hbm": round(adamw_bytes / (adamw_ms * 1e-3) / 1e9 / peaks["hbm_gbs"], 4),
+           "loss_first_linear": float(losses[0].item()),
+           "launches_per_step": 7 * 2 + 7 + 1,
+           "note": "fq prepass + MSE-epilogue forward + grouped STE backward per linear, one AdamW launch"}
+    del lin, Xs, Ts, X_in
+    torch.cuda.empty_cache()
     return out
 
 
@@ -633,10 +705,17 @@ def main():
     ap.add_argument("--no-variants", action="store_true")
     ap.add_argument("--no-gemv", action="store_true")
     ap.add_argument("--gemv-only", action="store_true")
+    ap.add_argument("--no-blockap", action="store_true")
+    ap.add_argument("--blockap-only", action="store_true")
     ap.add_argument("--initpack70b-only", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)  # timing rule: at least 3 untimed warm-up steps
+    if args.blockap_only:  # profiling aid: the Block-AP block step measurement alone
+        torch.cuda.set_device(0)
+        eqat.load_library()
+        print(json.dumps(blockap_block(torch.device("cuda", 0), load_peaks(), steps=2)), flush=True)
+        return
     if args.gemv_only:  # profiling aid: four plain decode GEMV calls, Llama-2-70B gate_proj w2g64, M = 1
         torch.cuda.set_device(0)
         eqat.load_library()

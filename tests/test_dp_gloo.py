@@ -65,3 +65,36 @@ def test_allreduced_weight_grads_equal_full_batch_grads(orc):
         np.testing.assert_allclose(got[3], ds2, rtol=1e-12, atol=1e-12)
         # the input gradient is rank-local: rows r*M .. (r+1)*M of the full batch
         np.testing.assert_allclose(got[4], dX[r * WL.m:(r + 1) * WL.m], rtol=1e-12, atol=1e-12)
+
+
+def reducer_worker(rank, world, port, out):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        red = dp.OverlappedGradReducer(dist)
+        rng = np.random.default_rng(100 + rank)
+        layers = [[torch.from_numpy(rng.standard_normal(sh).astype(np.float32)) for sh in ((8, 16), (8, 2), (8, 2))]
+                  for _ in range(3)]
+        before = [[t.clone() for t in ts] for ts in layers]
+        for i, ts in enumerate(layers):
+            red.submit(ts + [None], tag=i)
+        red.wait()
+        out[rank] = ([[t.numpy() for t in ts] for ts in before], [[t.numpy() for t in ts] for ts in layers], red.order)
+    finally:
+        dist.destroy_process_group()
+
+
+def test_overlapped_reducer_averages_each_layer_in_order():
+    """The Block-AP step's exchange: each linear's (dW, ds, dz) averaged over ranks, in
+    submission order; None entries skipped."""
+    world = 2
+    out = mp.Manager().dict()
+    mp.spawn(reducer_worker, args=(world, free_port(), out), nprocs=world, join=True)
+    before = [out[r][0] for r in range(world)]
+    for r in range(world):
+        _, after, order = out[r]
+        assert order == [0, 1, 2]
+        for i in range(3):
+            for j in range(3):
+                mean = (before[0][i][j] + before[1][i][j]) / 2
+                np.testing.assert_allclose(after[i][j], mean, rtol=1e-6, atol=1e-7)

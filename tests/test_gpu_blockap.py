@@ -155,3 +155,50 @@ def test_blockap_steps_match_oracle(orc):
             assert err.max() <= 2.01 * 3 * lr
             assert np.mean(err <= 0.05 * 3 * lr) >= 0.95
         assert (to_np(L.W) == bf16_round(to_np(L.W_master))).all()
+
+
+def test_blockap_step_with_overlapped_reducer_single_rank():
+    """The NCCL stream plumbing of the overlapped gradient exchange, on one rank (the mean
+    over one rank is the identity): the step gives the same state as without it."""
+    import os
+    import subprocess
+    import sys
+    code = r'''
+import os, torch, numpy as np, torch.distributed as dist
+import weight_quantization_aware_b200 as eqat
+from weight_quantization_aware_b200 import dp
+from weight_quantization_aware_b200.blockap import BlockAPConfig, QuantLinearState, blockap_step
+os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=os.environ["PORT"])
+torch.cuda.set_device(0)
+dist.init_process_group("nccl", rank=0, world_size=1, device_id=torch.device("cuda", 0))
+cfg = BlockAPConfig(total_steps=10)
+g = torch.Generator(device="cuda"); g.manual_seed(5)
+def make():
+    Ls, Xs, Ts = [], [], []
+    for N, K in ((136, 256), (128, 384)):
+        g.manual_seed(N * K)
+        W = torch.randn(N, K, generator=g, device="cuda") * 0.02
+        X = torch.randn(64, K, generator=g, device="cuda").to(torch.bfloat16)
+        Ls.append(QuantLinearState.from_weight(W, 2, 64, 64)); Xs.append(X); Ts.append(X @ W.to(torch.bfloat16).t())
+    return Ls, Xs, Ts
+A = make(); B = make()
+red = dp.OverlappedGradReducer(dist, device="cuda")
+for t in range(1, 4):
+    blockap_step(*A, cfg, t)
+    blockap_step(*B, cfg, t, reducer=red)
+torch.cuda.synchronize()
+for a, b in zip(A[0], B[0]):
+    assert torch.equal(a.W_master, b.W_master) and torch.equal(a.s, b.s) and torch.equal(a.z, b.z)
+assert red.order == [0, 1] * 3
+dist.destroy_process_group()
+print("ok")
+'''
+    import socket
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        port = s.getsockname()[1]
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    r = subprocess.run([sys.executable, "-c", code], cwd=root, env=dict(os.environ, PORT=str(port), PYTHONPATH=root,
+                                                                         NCCL_NVLS_ENABLE="0"),
+                       capture_output=True, text=True, timeout=300)
+    assert r.returncode == 0 and "ok" in r.stdout, r.stdout[-2000:] + r.stderr[-3000:]

@@ -65,9 +65,11 @@ class BlockAPConfig:
     weight_decay: float = 0.0
 
 
-def blockap_step(linears, inputs, targets, cfg: BlockAPConfig, step: int, losses=None):
+def blockap_step(linears, inputs, targets, cfg: BlockAPConfig, step: int, losses=None, reducer=None):
     """One step (step >= 1).  linears: QuantLinearState per linear; inputs[i] X [M, K_i] bf16,
-    targets[i] T [M, N_i] bf16.  Returns the per-linear losses as one fp64 CUDA tensor."""
+    targets[i] T [M, N_i] bf16.  Returns the per-linear losses as one fp64 CUDA tensor.
+    With data parallelism over tokens, `reducer` (dp.OverlappedGradReducer) averages each
+    linear's dW, ds, dz over ranks while the next linear computes."""
     n = len(linears)
     if losses is None:
         losses = torch.empty(n, dtype=torch.float64, device=linears[0].W.device)
@@ -76,6 +78,10 @@ def blockap_step(linears, inputs, targets, cfg: BlockAPConfig, step: int, losses
         _, dW, ds, dz = fq_linear_bwd(X, L.W, L.s, L.z, dY, cfg.bits, cfg.group, need_dx=False, ws=L.ws,
                                       out=L.grads, w_hat_in_ws=True)
         L.grads = (None, dW, ds, dz)
+        if reducer is not None:
+            reducer.submit([dW, ds, dz], tag=i)
+    if reducer is not None:
+        reducer.wait()
     # the schedules are indexed from 0: step t uses the rate of position t - 1
     lr_w = cosine_lr(cfg.lr_w, cfg.lr_min, step - 1, cfg.total_steps)
     lr_q = cosine_lr(cfg.lr_q, cfg.lr_min, step - 1, cfg.total_steps)

@@ -27,3 +27,57 @@ def allreduce_weight_grads(tensors, dist, group=None) -> None:
     for t in tensors:
         if t is not None:
             dist.all_reduce(t, op=dist.ReduceOp.SUM, group=group)
+
+
+class OverlappedGradReducer:
+    """Averages the weight-side gradients over ranks while later work runs.
+
+    submit(tensors) starts the exchange of one layer's gradients as soon as the
+    kernels that produced them are done: on CUDA it records an event on the
+    compute stream, and a communication stream waits on it and all-reduces there,
+    so the next layer's forward and backward proceed meanwhile.  wait() makes the
+    compute stream wait for every exchange submitted (call it before the optimizer
+    step).  The Block-AP loss is a mean over tokens, so the exchange is a mean
+    over ranks (NCCL's AVG; SUM then a scale where the backend has no AVG).
+    On CPU tensors (gloo) the exchange runs at submit time."""
+
+    def __init__(self, dist, group=None, device=None):
+        import torch
+        self.dist = dist
+        self.group = group
+        self.world = dist.get_world_size(group)
+        self.cuda = device is not None and torch.device(device).type == "cuda"
+        self.stream = torch.cuda.Stream(device=device) if self.cuda else None
+        self.has_avg = dist.get_backend(group) == "nccl"
+        self.order = []  # submission order, for checks
+
+    def _reduce(self, tensors):
+        d = self.dist
+        for t in tensors:
+            if t is None:
+                continue
+            if self.has_avg:
+                d.all_reduce(t, op=d.ReduceOp.AVG, group=self.group)
+            else:
+                d.all_reduce(t, op=d.ReduceOp.SUM, group=self.group)
+                t.mul_(1.0 / self.world)
+
+    def submit(self, tensors, tag=None):
+        import torch
+        self.order.append(tag)
+        if not self.cuda:
+            self._reduce(tensors)
+            return
+        ev = torch.cuda.Event()
+        ev.record(torch.cuda.current_stream(self.stream.device))
+        with torch.cuda.stream(self.stream):
+            self.stream.wait_event(ev)
+            self._reduce(tensors)
+        for t in tensors:  # in use on the communication stream until wait()
+            if t is not None:
+                t.record_stream(self.stream)
+
+    def wait(self):
+        import torch
+        if self.cuda:
+            torch.cuda.current_stream(self.stream.device).wait_stream(self.stream)

@@ -88,6 +88,7 @@ struct KParams {
     Prob pr[2];
     int nprob;
     int total_tiles;
+    int split_begin;  // pair kernel, one problem: tiles from here on are halves (-1: none)
     int *err;
     uint64_t wait_limit_ns;
 };
@@ -127,6 +128,32 @@ __device__ __forceinline__ int tile_coords(const KParams &p, int t, int &tm, int
         tm = lt / tiles_n;
     }
     return pi;
+}
+
+// Tile t of a pair launch: problem, tile row, first column and width.  In a
+// one-problem launch the wide tiles from p.split_begin on (the last, partial wave)
+// are each split into two tiles of half the width, so that the wave ends sooner.
+struct TileInfo {
+    int pi, tm, n0, bn;
+    bool narrow;
+};
+
+__device__ __forceinline__ TileInfo tile_info(const KParams &p, int t) {
+    int tt = t, sub = -1;
+    if (p.split_begin >= 0 && t >= p.split_begin) {
+        const int r = t - p.split_begin;
+        tt = p.split_begin + (r >> 1);
+        sub = r & 1;
+    }
+    int tm, tn;
+    TileInfo ti;
+    ti.pi = tile_coords(p, tt, tm, tn);
+    const int bn = ti.pi ? p.pr[1].bn : p.pr[0].bn;
+    ti.tm = tm;
+    ti.narrow = sub >= 0;
+    ti.bn = ti.narrow ? bn / 2 : bn;
+    ti.n0 = tn * bn + (ti.narrow ? sub * (bn / 2) : 0);
+    return ti;
 }
 
 // Epilogue chunk: 32 consecutive accumulator columns of one row.
@@ -594,17 +621,17 @@ __global__ void __launch_bounds__((4 + EPI_WARPS) * 32, 1)
             uint32_t armed = 0, armed_parity = 0;
             bool ok = true;
             for (int t = pair; ok && t < p.total_tiles; t += npairs) {
-                int tm, tn;
-                const int pi = tile_coords(p, t, tm, tn);
+                const TileInfo ti = tile_info(p, t);
+                const int pi = ti.pi;
                 const CUtensorMap *ma = pi ? &tmA1 : &tmA0;
-                const CUtensorMap *mb = pi ? &tmB1 : &tmB0;
+                // the halves of a split wave take B through the second map (half the box rows)
+                const CUtensorMap *mb = (pi || ti.narrow) ? &tmB1 : &tmB0;
                 const int a_mn = pi ? p.pr[1].a_mn : p.pr[0].a_mn;
                 const int b_mn = pi ? p.pr[1].b_mn : p.pr[0].b_mn;
                 const int nkb = ((pi ? p.pr[1].GK : p.pr[0].GK) + BK - 1) / BK;
-                const int bn = pi ? p.pr[1].bn : p.pr[0].bn;
-                const int half = bn / 2;
-                const int m0 = tm * BM2 + 128 * static_cast<int>(rank);
-                const int n0 = tn * bn + half * static_cast<int>(rank);
+                const int half = ti.bn / 2;
+                const int m0 = ti.tm * BM2 + 128 * static_cast<int>(rank);
+                const int n0 = ti.n0 + half * static_cast<int>(rank);
                 for (int kb = 0; kb < nkb; ++kb, ++it) {
                     const int st = it % STAGES2;
                     const uint32_t ph = (it / STAGES2) & 1u;
@@ -662,13 +689,12 @@ __global__ void __launch_bounds__((4 + EPI_WARPS) * 32, 1)
             uint32_t it = 0, local = 0;
             bool ok = true, issued = false;
             for (int t = pair; ok && t < p.total_tiles; t += npairs, ++local) {
-                int tm, tn;
-                const int pi = tile_coords(p, t, tm, tn);
+                const TileInfo ti = tile_info(p, t);
+                const int pi = ti.pi;
                 const int a_mn = pi ? p.pr[1].a_mn : p.pr[0].a_mn;
                 const int b_mn = pi ? p.pr[1].b_mn : p.pr[0].b_mn;
                 const int nkb = ((pi ? p.pr[1].GK : p.pr[0].GK) + BK - 1) / BK;
-                const int bn = pi ? p.pr[1].bn : p.pr[0].bn;
-                const uint32_t idesc = idesc_bf16_f32(BM2, bn, a_mn != 0, b_mn != 0);
+                const uint32_t idesc = idesc_bf16_f32(BM2, ti.bn, a_mn != 0, b_mn != 0);
                 const uint32_t a_step = a_mn ? UK * 128 : UK * 2, a_lbo = a_mn ? MN_BOX_BYTES : 16;
                 const uint32_t b_step = b_mn ? UK * 128 : UK * 2, b_lbo = b_mn ? MN_BOX_BYTES : 16;
                 const uint32_t acc = local & 1u;
@@ -723,16 +749,14 @@ __global__ void __launch_bounds__((4 + EPI_WARPS) * 32, 1)
             const bool ok = mbar_wait_bounded(&ctl->acc_full[acc], aph, abort_flag, p.err, p.wait_limit_ns);
             if (!__all_sync(0xffffffffu, ok)) break;
             tc_fence_after();
-            int tm, tn;
-            const int pi = tile_coords(p, t, tm, tn);
-            const int row = tm * BM2 + 128 * static_cast<int>(rank) + quad * 32 + lane;
+            const TileInfo ti = tile_info(p, t);
+            const int row = ti.tm * BM2 + 128 * static_cast<int>(rank) + quad * 32 + lane;
             const uint32_t taddr = tmem_base + acc * ACC_COLS + ((quad * 32) << 16);
-            const int bn = pi ? p.pr[1].bn : p.pr[0].bn;
-            const int cols = bn / SLICES;
-            if (pi == 0)
-                drain_accumulator<EPI0, BITS>(p.pr[0], taddr, row, tn * bn, half_slice * cols, (half_slice + 1) * cols);
+            const int cols = ti.bn / SLICES;
+            if (ti.pi == 0)
+                drain_accumulator<EPI0, BITS>(p.pr[0], taddr, row, ti.n0, half_slice * cols, (half_slice + 1) * cols);
             else
-                drain_accumulator<EPI1, BITS>(p.pr[1], taddr, row, tn * bn, half_slice * cols, (half_slice + 1) * cols);
+                drain_accumulator<EPI1, BITS>(p.pr[1], taddr, row, ti.n0, half_slice * cols, (half_slice + 1) * cols);
             tc_fence_before();
             mbar_arrive_cluster(acc_empty0 + 8u * acc);
         }
@@ -841,6 +865,15 @@ cudaError_t launch_pair_variant(const CUtensorMap (&maps)[4], const KParams &p, 
     }
     cfg.gridDim.x = static_cast<unsigned>(std::min(grid, 2 * n));
     return cudaLaunchKernelEx(&cfg, kern, maps[0], maps[1], maps[2], maps[3], p);
+}
+
+// EQAT_GEMM_SPLIT_TAIL=0 keeps the last wave whole (measurement aid).
+bool split_tail_enabled() {
+    static const bool on = [] {
+        const char *v = std::getenv("EQAT_GEMM_SPLIT_TAIL");
+        return !(v && v[0] == '0');
+    }();
+    return on;
 }
 
 int *device_error_ptr() {
@@ -1002,11 +1035,25 @@ cudaError_t launch_gemm_tc_group(const GemmProblem *probs, int nprob, const Devi
     }
     p.nprob = nprob;
     p.total_tiles = tiles;
+    p.split_begin = -1;
+    // A one-problem pair launch whose last wave is partial, at most half full: split
+    // that wave's 256-wide tiles into 128-wide halves (one wave of narrow tiles costs
+    // about 0.66 of a wide one).  B must be K-major (one box per half) and the
+    // epilogue's groups must fit a 64-column slice.
+    if (pair && nprob == 1 && bn == 256 && !probs[0].B.mn_major && split_tail_enabled() &&
+        (probs[0].epi.kind == Epi::kStore || probs[0].epi.kind == Epi::kMse || probs[0].epi.group <= 64)) {
+        const int full = tiles / units, tail = tiles % units;
+        if (full >= 1 && tail > 0 && 2 * tail <= units) {
+            if ((e = make_map(maps[3], probs[0].B, probs[0].GN, probs[0].GK, bn / 4)) != cudaSuccess) return e;
+            p.split_begin = full * units;
+            p.total_tiles = full * units + 2 * tail;
+        }
+    }
     p.err = device_error_ptr();
     if (!p.err) return cudaErrorInvalidSymbol;
     p.wait_limit_ns = kWaitLimitNs;
     if (pair) {
-        const int grid = 2 * std::min(tiles, units);
+        const int grid = 2 * std::min(p.total_tiles, units);
         switch (probs[0].epi.kind) {
             case Epi::kStore:
                 if (nprob > 1) return cudaErrorInvalidValue;

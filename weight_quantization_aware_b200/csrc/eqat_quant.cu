@@ -190,6 +190,10 @@ __device__ __forceinline__ void pack_chunk(const float (&w)[16], float sc, float
                                            uint8_t *__restrict__ codes) {
     const float rcp = __frcp_rn(sc);
     const float lo = kRoundMagic, hi = __fadd_rn(kRoundMagic, Q);
+    // M + zr is exact; one add of it gives M + zr + round(u) for every u that is
+    // not an exact tie (ties may break toward an odd total, but a tie lies in the
+    // near band below and takes the exact path).
+    const float mz = __fadd_rn(kRoundMagic, zr);
     // Each code enters its word as the raw bits of M + code (one multiply-add);
     // the bits of M are taken out once per word at the end.
     uint32_t word[4] = {0u, 0u, 0u, 0u};  // 2-bit: word[0]; 4-bit: word[0..1]; 3-bit: word[0..3]
@@ -198,7 +202,15 @@ __device__ __forceinline__ void pack_chunk(const float (&w)[16], float sc, float
         float cm[8];
         bool near = false;
 #pragma unroll
-        for (int j = 0; j < 8; ++j) cm[j] = fminf(fmaxf(magic_decision(w[8 * h + j], rcp, zr, near), lo), hi);
+        for (int j = 0; j < 8; ++j) {
+            const float u = __fmul_rn(w[8 * h + j], rcp);
+            const float t = __fadd_rn(u, mz);
+            // |u - RN(w / s)| < |u| 2^-22: only a u within that of a half-integer can
+            // round differently.  A code that is not clamped has |u| <= Q + zr + 1/2 < 64,
+            // so a band of 2^-16 covers it; a clamped code does not depend on it.
+            near |= fabsf(__fsub_rn(u, __fsub_rn(t, mz))) >= 0.5f - 0x1p-16f;
+            cm[j] = fminf(fmaxf(t, lo), hi);
+        }
         if (near) {
 #pragma unroll
             for (int j = 0; j < 8; ++j) {

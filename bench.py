@@ -411,6 +411,8 @@ def run_ours(args):
         line["decode_gemv"] = decode_gemv(dev, peaks)
     if not args.no_blockap:
         line["blockap_block"] = blockap_block(dev, peaks)
+    if not args.no_configs:
+        line["per_config"] = per_config(dev, peaks)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(target_s=args.cpu_seconds)
     if dist is not None:
@@ -467,6 +469,65 @@ def quantizer_variants(step, dev, reps=50):
         for name, fn in e2e.items():
             out[f"{name}_{sname}_TFLOPs"] = round(4 * M * N * K / (timed(lambda: fn(s_)) * 1e-3) / 1e12, 1)
     out["note"] = "4MNK per backward call, L2 flushed before each call, W-hat reused from the forward"
+    return out
+
+
+def per_config(dev, peaks, reps=10):
+    """Fake-quant linear forward + backward throughput per linear and per config, for the
+    bf16 workloads (Llama-2 7B q_proj; 7B MLP w3g128; 13B E2E-QP w2g64 on packed codes;
+    70B block w2g64).  Block-AP: fq_linear_fwd then fq_linear_bwd (dX, dW, ds, dz, W-hat
+    reused); E2E-QP: dq_linear_fwd then dq_linear_bwd_s (dX, ds).  6 M N K per linear;
+    CUDA events around `reps` back-to-back fwd+bwd pairs after 2 warm ones.  Inputs are
+    drawn on the device (seeded); the per-linear bytes exceed L2 for all but the smallest."""
+    out = {}
+    gen = torch.Generator(device=dev)
+    for idx in (2, 3, 4, 5):
+        wl = synthetic.WORKLOADS[idx]
+        M, b, g = wl.m, wl.bits, wl.group
+        lines, tot_flops, tot_ms = {}, 0, 0.0
+        for lin in wl.linears:
+            N, K = lin.n, lin.k
+            gen.manual_seed(4000 + 10 * idx + len(lines))
+            X = torch.randn(M, K, generator=gen, device=dev).to(torch.bfloat16)
+            W = (torch.randn(N, K, generator=gen, device=dev) * wl.sigma).to(torch.bfloat16)
+            dY = torch.randn(M, N, generator=gen, device=dev).to(torch.bfloat16)
+            s, z = eqat.minmax_init(W, b, g)
+            ws = eqat.workspace(M, N, K, b, g, torch.bfloat16, dev)
+            Y = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
+            if wl.mode == "e2e_qp":
+                codes, zq = eqat.pack_codes(W, s, z, b, g)
+                out_b = (torch.empty_like(X), torch.empty_like(s))
+
+                def fb():
+                    eqat.dq_linear_fwd(X, codes, zq, s, b, g, ws=ws, Y=Y)
+                    eqat.dq_linear_bwd_s(X, codes, zq, s, dY, b, g, ws=ws, out=out_b, w_hat_in_ws=True)
+            else:
+                out_b = (torch.empty_like(X), torch.empty_like(W), torch.empty_like(s), torch.empty_like(s))
+
+                def fb():
+                    eqat.fq_linear_fwd(X, W, s, z, b, g, ws=ws, Y=Y)
+                    eqat.fq_linear_bwd(X, W, s, z, dY, b, g, ws=ws, out=out_b, w_hat_in_ws=True)
+            fb(); fb()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            for _ in range(reps):
+                fb()
+            e1.record()
+            torch.cuda.synchronize()
+            ms = e0.elapsed_time(e1) / reps
+            fl = 6 * M * N * K
+            lines[lin.name] = {"N": N, "K": K, "us": round(ms * 1e3, 1),
+                               "TFLOPs": round(fl / (ms * 1e-3) / 1e12, 1),
+                               "frac_bf16_sustained": round(fl / (ms * 1e-3) / 1e12 / peaks["bf16_tflops_sustained"], 3)}
+            tot_flops += fl
+            tot_ms += ms
+            del X, W, dY, ws, Y, out_b
+            torch.cuda.empty_cache()
+        out[wl.name] = {"M": M, "bits": b, "group": g, "mode": wl.mode, "linears": lines,
+                        "TFLOPs": round(tot_flops / (tot_ms * 1e-3) / 1e12, 1),
+                        "frac_bf16_sustained": round(tot_flops / (tot_ms * 1e-3) / 1e12 /
+                                                     peaks["bf16_tflops_sustained"], 3)}
+    out["note"] = "6 M N K per linear (forward + dX + dW-hat), prepasses included; no L2 flush between calls"
     return out
 
 
@@ -743,10 +804,17 @@ def main():
     ap.add_argument("--gemv-only", action="store_true")
     ap.add_argument("--no-blockap", action="store_true")
     ap.add_argument("--blockap-only", action="store_true")
+    ap.add_argument("--no-configs", action="store_true")
+    ap.add_argument("--configs-only", action="store_true")
     ap.add_argument("--initpack70b-only", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)  # timing rule: at least 3 untimed warm-up steps
+    if args.configs_only:  # the per-config table alone
+        torch.cuda.set_device(0)
+        eqat.load_library()
+        print(json.dumps(per_config(torch.device("cuda", 0), load_peaks())), flush=True)
+        return
     if args.blockap_only:  # profiling aid: the Block-AP block step measurement alone
         torch.cuda.set_device(0)
         eqat.load_library()

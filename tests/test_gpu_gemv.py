@@ -53,6 +53,15 @@ CASES = [  # (M, N, K, bits, group)
     (8, 520, 1600, 3, 64),
     (2, 96, 768, 3, 128),
     (7, 1024, 8192, 2, 64),
+    # groups of a stage sharing the mma columns: every (bits, group, slots) layout
+    (1, 200, 1664, 2, 128),     # 4 slots, 2 token columns (one empty)
+    (2, 136, 1088, 2, 64),      # 4 slots x 2 tokens
+    (4, 264, 2048, 2, 64),      # 2 slots x 4 tokens
+    (1, 392, 1344, 4, 64),      # 4 slots
+    (2, 136, 2304, 4, 128),     # 2 slots x 4 columns (two empty)
+    (4, 128, 512, 4, 64),       # 2 slots x 4 tokens
+    (1, 72, 704, 3, 64),        # 2 slots
+    (1, 136, 384, 3, 128),      # 1 slot, 7 empty columns
 ]
 
 

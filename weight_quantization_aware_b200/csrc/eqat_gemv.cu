@@ -18,6 +18,12 @@
 //     conversion: code bits placed in the mantissa of 128.0 give 128 + code * 4^j
 //     exactly) and feeds them to mma.sync as the A operand:
 //       sum_k (c_k - zq) x_k = [sum_k (128 + c_k 4^j) (x_k 4^-j)] - xoff_g - zq xsum_g.
+//   - the eight mma columns carry (group slot, token) pairs: with M padded to a
+//     power of two MP, SL = 8 / MP consecutive groups of a stage (at most the
+//     stage's group count) accumulate side by side in the same registers, each
+//     in its own columns, so the per-group correction above, the accumulator
+//     reset and the s / zq reads run once per SL groups.  At M = 1 that is once
+//     per stage instead of once per group.
 // The tensor core is only a multiply-add engine for register-resident operands;
 // the roofline is HBM.
 //
@@ -211,9 +217,14 @@ __device__ __forceinline__ uint32_t bf16x2_bits(float lo, float hi) {
 // 2i: columns lo, hi scaled by 4^-scale_exp; b2b3 with register 2i + 1).  It also
 // reads column i of the group for the 8 tokens, and the block sums them into
 // xoff = sum 128 x 4^-j and xsum = sum x per token.
+//
+// Column n of the fragments is (slot n / MPC, token n % MPC), MPC = 8 / slots:
+// a set's entries are nonzero only in the columns of its group's slot (the
+// group's index within its stage, modulo `slots`).
 template <int BITS, int GROUP>
 __global__ void __launch_bounds__(GROUP) k_gemv_xprep(const __nv_bfloat16 *__restrict__ X, int M, int64_t K,
-                                                        uint4 *__restrict__ table, float2 *__restrict__ xso) {
+                                                        int slots, uint4 *__restrict__ table,
+                                                        float2 *__restrict__ xso) {
     using C = Codes<BITS>;
     constexpr int WARPS = GROUP / 32;
     __shared__ float red[WARPS][16];
@@ -226,6 +237,9 @@ __global__ void __launch_bounds__(GROUP) k_gemv_xprep(const __nv_bfloat16 *__res
         const int j = gidx * (GROUP / 64) + (threadIdx.x >> 6);
         const int ip = (threadIdx.x >> 5) & 1, l = threadIdx.x & 31;
         const int n = l >> 2, t = l & 3;
+        const int mpc = 8 / slots;
+        const int gs = (j % (stage_codes<BITS>() / 64)) / (GROUP / 64);  // the set's group within its stage
+        const int tok = (n / mpc == gs % slots) ? n % mpc : 8;           // 8: no token, zeros
         const int64_t kb = 64 * static_cast<int64_t>(j) + 16 * t;
         uint32_t r[4];
 #pragma unroll
@@ -234,7 +248,7 @@ __global__ void __launch_bounds__(GROUP) k_gemv_xprep(const __nv_bfloat16 *__res
             for (int sl = 0; sl < 2; ++sl) {
                 const int e = 2 * (2 * ip + h) + sl;
                 const float sc = (C::scale_exp(e) == 0) ? 1.0f : (C::scale_exp(e) == 1 ? 0.25f : 0.0625f);
-                r[2 * h + sl] = bf16x2_bits(xv(n, kb + C::lo(e)) * sc, xv(n, kb + C::hi(e)) * sc);
+                r[2 * h + sl] = bf16x2_bits(xv(tok, kb + C::lo(e)) * sc, xv(tok, kb + C::hi(e)) * sc);
             }
         }
         table[(static_cast<int64_t>(j) * 2 + ip) * 32 + l] = make_uint4(r[0], r[1], r[2], r[3]);
@@ -278,9 +292,12 @@ __global__ void __launch_bounds__(GROUP) k_gemv_xprep(const __nv_bfloat16 *__res
 }
 
 // s and zq of one stage (128 rows x GPS groups), four values per consumer thread
-// at most, loaded into registers two stages ahead of their use.
+// at most, loaded into registers two stages ahead of their use.  The registers
+// hold the raw bits; they are converted only when stored to shared memory, so
+// that nothing waits for the loads before then.
 struct SzRegs {
-    float s[4], z[4];
+    uint32_t s[4];  // fp32 value v in word v, or fp16 value v in half v % 2 of word v / 2
+    uint32_t z;     // zq value v in byte v
 };
 
 // Each consumer warp stages the s and zq of its own 16 rows: lane l takes row
@@ -300,66 +317,70 @@ __device__ __forceinline__ void load_sz(const GemvParams &p, const StageCursor &
     using Sh = SzShape<BITS, GROUP>;
     constexpr int VPT = Sh::VPT, TPR = Sh::TPR;
 #pragma unroll
-    for (int v = 0; v < 4; ++v) {
-        r.s[v] = 0.0f;
-        r.z[v] = 0.0f;
-    }
+    for (int v = 0; v < 4; ++v) r.s[v] = 0u;
+    r.z = 0u;
     const int row = lane / TPR, part = lane % TPR;
     if (c.x >= x_end || row >= 16) return;
     const int64_t n = static_cast<int64_t>(c.rt) * kRows + row0 + row;
     const int64_t g = static_cast<int64_t>(c.ks) * Sh::GPS + part * VPT;
     if (n >= p.N) return;
     const int64_t i = n * p.G + g;
+    const uint32_t *s32 = static_cast<const uint32_t *>(p.s);
+    const unsigned short *s16 = static_cast<const unsigned short *>(p.s);
     if (p.vec && g + VPT <= p.G) {
         if (VPT == 4) {
             if (S16) {
-                const uint2 h = __ldg(reinterpret_cast<const uint2 *>(static_cast<const __half *>(p.s) + i));
-                const __half2 h0 = *reinterpret_cast<const __half2 *>(&h.x), h1 = *reinterpret_cast<const __half2 *>(&h.y);
-                r.s[0] = __low2float(h0); r.s[1] = __high2float(h0); r.s[2] = __low2float(h1); r.s[3] = __high2float(h1);
+                const uint2 h = __ldg(reinterpret_cast<const uint2 *>(s16 + i));
+                r.s[0] = h.x;
+                r.s[1] = h.y;
             } else {
-                const float4 f = __ldg(reinterpret_cast<const float4 *>(static_cast<const float *>(p.s) + i));
-                r.s[0] = f.x; r.s[1] = f.y; r.s[2] = f.z; r.s[3] = f.w;
+                const uint4 f = __ldg(reinterpret_cast<const uint4 *>(s32 + i));
+                r.s[0] = f.x;
+                r.s[1] = f.y;
+                r.s[2] = f.z;
+                r.s[3] = f.w;
             }
-            const uint32_t z = __ldg(reinterpret_cast<const uint32_t *>(p.zq + i));
-#pragma unroll
-            for (int v = 0; v < 4; ++v) r.z[v] = static_cast<float>((z >> (8 * v)) & 0xFFu);
+            r.z = __ldg(reinterpret_cast<const uint32_t *>(p.zq + i));
         } else if (VPT == 2) {
             if (S16) {
-                const __half2 h = __ldg(reinterpret_cast<const __half2 *>(static_cast<const __half *>(p.s) + i));
-                r.s[0] = __low2float(h); r.s[1] = __high2float(h);
+                r.s[0] = __ldg(reinterpret_cast<const uint32_t *>(s16 + i));
             } else {
-                const float2 f = __ldg(reinterpret_cast<const float2 *>(static_cast<const float *>(p.s) + i));
-                r.s[0] = f.x; r.s[1] = f.y;
+                const uint2 f = __ldg(reinterpret_cast<const uint2 *>(s32 + i));
+                r.s[0] = f.x;
+                r.s[1] = f.y;
             }
-            const uint32_t z = __ldg(reinterpret_cast<const unsigned short *>(p.zq + i));
-            r.z[0] = static_cast<float>(z & 0xFFu);
-            r.z[1] = static_cast<float>(z >> 8);
+            r.z = __ldg(reinterpret_cast<const unsigned short *>(p.zq + i));
         } else {
-            r.s[0] = S16 ? __half2float(__ldg(static_cast<const __half *>(p.s) + i))
-                         : __ldg(static_cast<const float *>(p.s) + i);
-            r.z[0] = static_cast<float>(__ldg(p.zq + i));
+            r.s[0] = S16 ? static_cast<uint32_t>(__ldg(s16 + i)) : __ldg(s32 + i);
+            r.z = __ldg(p.zq + i);
         }
         return;
     }
 #pragma unroll
     for (int v = 0; v < VPT; ++v) {
         if (g + v < p.G) {
-            r.s[v] = S16 ? __half2float(__ldg(static_cast<const __half *>(p.s) + i + v))
-                         : __ldg(static_cast<const float *>(p.s) + i + v);
-            r.z[v] = static_cast<float>(__ldg(p.zq + i + v));
+            if (S16)
+                r.s[v / 2] |= static_cast<uint32_t>(__ldg(s16 + i + v)) << (16 * (v % 2));
+            else
+                r.s[v] = __ldg(s32 + i + v);
+            r.z |= static_cast<uint32_t>(__ldg(p.zq + i + v)) << (8 * v);
         }
     }
 }
 
 // Into the warp's slot, entry row * GPS + group (rows local to the warp).
-template <int BITS, int GROUP>
+template <int BITS, int GROUP, bool S16>
 __device__ __forceinline__ void store_sz(float2 *slot, int lane, const SzRegs &r) {
     using Sh = SzShape<BITS, GROUP>;
     const int row = lane / Sh::TPR, part = lane % Sh::TPR;
     if (row >= 16) return;
     float2 *d = slot + row * Sh::GPS + part * Sh::VPT;
 #pragma unroll
-    for (int v = 0; v < Sh::VPT; ++v) d[v] = make_float2(r.s[v], r.z[v]);
+    for (int v = 0; v < Sh::VPT; ++v) {
+        const float sv = S16 ? __half2float(__ushort_as_half(static_cast<unsigned short>(r.s[v / 2] >> (16 * (v % 2)))))
+                             : __uint_as_float(r.s[v]);
+        d[v] = make_float2(sv, static_cast<float>((r.z >> (8 * v)) & 0xFFu));
+    }
 }
 
 __device__ __forceinline__ void mma_bf16(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
@@ -369,6 +390,16 @@ __device__ __forceinline__ void mma_bf16(float (&d)[4], uint32_t a0, uint32_t a1
         "{%0, %1, %2, %3};"
         : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
         : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// The same with a zero accumulator in.
+__device__ __forceinline__ void mma_bf16_z(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                           uint32_t b0, uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+        "{%10, %10, %10, %10};"
+        : "=f"(d[0]), "=f"(d[1]), "=f"(d[2]), "=f"(d[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1), "f"(0.0f));
 }
 
 // Byte b of row r of a 128-byte-swizzled code tile.
@@ -395,7 +426,7 @@ __device__ __forceinline__ void load_codes(const uint8_t *tile, int row, int byt
 }
 
 
-template <int BITS, int GROUP, bool S16>
+template <int BITS, int GROUP, bool S16, int SL>
 __global__ void __launch_bounds__(kThreads, 1)
     k_dq_gemv(const __grid_constant__ CUtensorMap tm_codes, const GemvParams p) {
     using C = Codes<BITS>;
@@ -406,6 +437,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     constexpr int GPS = KS / GROUP;                   // groups per stage
     constexpr uint32_t TABLE_BYTES = SETS * 1024;
     constexpr uint32_t XO_BYTES = GPS * 64;
+    constexpr int MPC = 8 / SL;  // token columns per slot
+    static_assert(SL >= 1 && SL <= 8 && GPS % SL == 0, "slots divide the stage's groups");
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                 ~static_cast<uintptr_t>(1023));
@@ -476,8 +509,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
 
     // ---------------------------------------------------------------- consumers
+    // Lane (r0, t) holds the accumulators of rows row_a, row_b and columns 2t,
+    // 2t + 1, i.e. slot slot0 with tokens tok0, tok0 + 1 (MPC >= 2), or slots
+    // 2t, 2t + 1 of token 0 (MPC = 1).
     const int r0 = lane >> 2, t = lane & 3;
     const int row_a = warp * 16 + r0, row_b = row_a + 8;
+    const int slot0 = (2 * t) / MPC, tok0 = (2 * t) % MPC;
     // this warp's s / zq slots: [kSlots][16 rows][GPS] float2
     float2 *szw = sz + warp * (kSlots * 16 * kMaxGps);
 
@@ -490,7 +527,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     pf = cur;
     load_sz<BITS, GROUP, S16>(p, pf, x_end, warp * 16, lane, sa_);
     pf.next(p.spr);
-    store_sz<BITS, GROUP>(szw, lane, sa_);
+    store_sz<BITS, GROUP, S16>(szw, lane, sa_);
     load_sz<BITS, GROUP, S16>(p, pf, x_end, warp * 16, lane, sb_);
     pf.next(p.spr);
     load_sz<BITS, GROUP, S16>(p, pf, x_end, warp * 16, lane, sc_);
@@ -510,58 +547,100 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint4 *table = reinterpret_cast<const uint4 *>(tile + kCodeTile);
         const float2 *xo = reinterpret_cast<const float2 *>(tile + kCodeTile + kTableSlice);
         const float2 *szs = szw + (it % kSlots) * (16 * kMaxGps);
-        // Groups of the stage are independent: two accumulator chains per group
-        // (mmas 0, 2 and 1, 3 of each set), so the unrolled groups overlap.
+        // Runs of SL groups: the four mmas of a set go to four accumulator chains,
+        // and the run's groups share them (each in its own columns).
 #pragma unroll
-        for (int gi = 0; gi < GPS; ++gi) {
-            float a0[4] = {0.0f, 0.0f, 0.0f, 0.0f}, a1[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+        for (int g0 = 0; g0 < GPS; g0 += SL) {
+            float acc[4][4];
 #pragma unroll
-            for (int q = 0; q < SPG; ++q) {
-                const int m = gi * SPG + q;
-                uint32_t wa[C::kBytes / 4], wb[C::kBytes / 4];
-                load_codes<BITS>(tile, row_a, m * SET_BYTES + t * C::kBytes, wa);
-                load_codes<BITS>(tile, row_b, m * SET_BYTES + t * C::kBytes, wb);
-                uint32_t ea[8], eb[8];
-                C::extract(wa, ea);
-                C::extract(wb, eb);
-                const uint4 b01 = table[(m * 2 + 0) * 32 + lane];
-                const uint4 b23 = table[(m * 2 + 1) * 32 + lane];
-                mma_bf16(a0, ea[0], eb[0], ea[1], eb[1], b01.x, b01.y);
-                mma_bf16(a1, ea[2], eb[2], ea[3], eb[3], b01.z, b01.w);
-                mma_bf16(a0, ea[4], eb[4], ea[5], eb[5], b23.x, b23.y);
-                mma_bf16(a1, ea[6], eb[6], ea[7], eb[7], b23.z, b23.w);
+            for (int gs = 0; gs < SL; ++gs) {
+#pragma unroll
+                for (int q = 0; q < SPG; ++q) {
+                    const int m = (g0 + gs) * SPG + q;
+                    uint32_t wa[C::kBytes / 4], wb[C::kBytes / 4];
+                    load_codes<BITS>(tile, row_a, m * SET_BYTES + t * C::kBytes, wa);
+                    load_codes<BITS>(tile, row_b, m * SET_BYTES + t * C::kBytes, wb);
+                    uint32_t ea[8], eb[8];
+                    C::extract(wa, ea);
+                    C::extract(wb, eb);
+                    const uint4 b01 = table[(m * 2 + 0) * 32 + lane];
+                    const uint4 b23 = table[(m * 2 + 1) * 32 + lane];
+                    if (gs == 0 && q == 0) {
+                        mma_bf16_z(acc[0], ea[0], eb[0], ea[1], eb[1], b01.x, b01.y);
+                        mma_bf16_z(acc[1], ea[2], eb[2], ea[3], eb[3], b01.z, b01.w);
+                        mma_bf16_z(acc[2], ea[4], eb[4], ea[5], eb[5], b23.x, b23.y);
+                        mma_bf16_z(acc[3], ea[6], eb[6], ea[7], eb[7], b23.z, b23.w);
+                    } else {
+                        mma_bf16(acc[0], ea[0], eb[0], ea[1], eb[1], b01.x, b01.y);
+                        mma_bf16(acc[1], ea[2], eb[2], ea[3], eb[3], b01.z, b01.w);
+                        mma_bf16(acc[2], ea[4], eb[4], ea[5], eb[5], b23.x, b23.y);
+                        mma_bf16(acc[3], ea[6], eb[6], ea[7], eb[7], b23.z, b23.w);
+                    }
+                }
             }
-            const float2 sa = szs[r0 * GPS + gi], sb = szs[(r0 + 8) * GPS + gi];
-            const float4 ox = *reinterpret_cast<const float4 *>(xo + gi * 8 + 2 * t);  // tokens 2t, 2t+1
-            // ox = {xoff(2t), xsum(2t), xoff(2t+1), xsum(2t+1)}
-            y[0] = fmaf(sa.x, (a0[0] + a1[0]) - fmaf(sa.y, ox.y, ox.x), y[0]);
-            y[1] = fmaf(sa.x, (a0[1] + a1[1]) - fmaf(sa.y, ox.w, ox.z), y[1]);
-            y[2] = fmaf(sb.x, (a0[2] + a1[2]) - fmaf(sb.y, ox.y, ox.x), y[2]);
-            y[3] = fmaf(sb.x, (a0[3] + a1[3]) - fmaf(sb.y, ox.w, ox.z), y[3]);
+            float c[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) c[i] = (acc[0][i] + acc[1][i]) + (acc[2][i] + acc[3][i]);
+            // c = {row_a col 2t, row_a col 2t+1, row_b col 2t, row_b col 2t+1}
+            if constexpr (MPC == 1) {
+                // columns 2t, 2t + 1 are groups g0 + 2t, g0 + 2t + 1 of token 0
+                const float4 sa = *reinterpret_cast<const float4 *>(szs + r0 * GPS + g0 + 2 * t);
+                const float4 sb = *reinterpret_cast<const float4 *>(szs + (r0 + 8) * GPS + g0 + 2 * t);
+                const float2 o0 = xo[(g0 + 2 * t) * 8], o1 = xo[(g0 + 2 * t + 1) * 8];
+                y[0] = fmaf(sa.x, c[0] - fmaf(sa.y, o0.y, o0.x), y[0]);
+                y[1] = fmaf(sa.z, c[1] - fmaf(sa.w, o1.y, o1.x), y[1]);
+                y[2] = fmaf(sb.x, c[2] - fmaf(sb.y, o0.y, o0.x), y[2]);
+                y[3] = fmaf(sb.z, c[3] - fmaf(sb.w, o1.y, o1.x), y[3]);
+            } else {
+                // both columns are group g0 + slot0; tokens tok0, tok0 + 1
+                const float2 sa = szs[r0 * GPS + g0 + slot0], sb = szs[(r0 + 8) * GPS + g0 + slot0];
+                const float4 o = *reinterpret_cast<const float4 *>(xo + (g0 + slot0) * 8 + tok0);
+                y[0] = fmaf(sa.x, c[0] - fmaf(sa.y, o.y, o.x), y[0]);
+                y[1] = fmaf(sa.x, c[1] - fmaf(sa.y, o.w, o.z), y[1]);
+                y[2] = fmaf(sb.x, c[2] - fmaf(sb.y, o.y, o.x), y[2]);
+                y[3] = fmaf(sb.x, c[3] - fmaf(sb.y, o.w, o.z), y[3]);
+            }
         }
         __syncwarp();
         if (lane == 0) mbar_arrive(&empty[st]);
 
         // s / zq of the next stage into its slot
-        store_sz<BITS, GROUP>(szw + ((it + 1) % kSlots) * (16 * kMaxGps), lane, store_from);
+        store_sz<BITS, GROUP, S16>(szw + ((it + 1) % kSlots) * (16 * kMaxGps), lane, store_from);
 
         const int rt = cur.rt;
         cur.next(p.spr);
         ++it;
         if (cur.x == x_end || cur.ks == 0) {
             // this CTA is done with row tile rt: its partial goes to slot
-            // (rt, cta - first cta of rt); rows rt*128 + row_a / row_b, tokens 2t, 2t+1
+            // (rt, cta - first cta of rt).  The lanes of a quad that hold the
+            // same tokens in different slots are summed first.
             const int seg = static_cast<int>(blockIdx.x) -
                             cta_of_stage(static_cast<int64_t>(rt) * p.spr, S, static_cast<int>(gridDim.x));
             float *P = p.partials + (static_cast<int64_t>(rt) * p.maxseg + seg) * p.M * kRows;
-            const int m0 = 2 * t, m1 = m0 + 1;
-            if (m0 < p.M) {
-                P[m0 * kRows + row_a] = y[0];
-                P[m0 * kRows + row_b] = y[2];
+            float v[4] = {y[0], y[1], y[2], y[3]};
+            if constexpr (MPC == 1) {
+                v[0] += v[1];
+                v[2] += v[3];
             }
-            if (m1 < p.M) {
-                P[m1 * kRows + row_a] = y[1];
-                P[m1 * kRows + row_b] = y[3];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                if (MPC <= 2) {
+                    v[i] += __shfl_xor_sync(0xffffffffu, v[i], 1);
+                    v[i] += __shfl_xor_sync(0xffffffffu, v[i], 2);
+                } else if (MPC == 4) {
+                    v[i] += __shfl_xor_sync(0xffffffffu, v[i], 2);
+                }
+            }
+            if (slot0 == 0) {
+                const int m0 = tok0, m1 = tok0 + 1;
+                if (m0 < p.M) {
+                    P[m0 * kRows + row_a] = v[0];
+                    P[m0 * kRows + row_b] = v[2];
+                }
+                if (MPC > 1 && m1 < p.M) {
+                    P[m1 * kRows + row_a] = v[1];
+                    P[m1 * kRows + row_b] = v[3];
+                }
             }
             y[0] = y[1] = y[2] = y[3] = 0.0f;
         }
@@ -639,9 +718,9 @@ Plan make_plan(int64_t M, int64_t N, int64_t K, int bits, int group, int sms) {
     return pl;
 }
 
-template <int BITS, int GROUP, bool S16>
+template <int BITS, int GROUP, bool S16, int SL>
 cudaError_t launch_main(const CUtensorMap &map, const GemvParams &p, int grid, int dev_id, cudaStream_t st) {
-    auto kern = k_dq_gemv<BITS, GROUP, S16>;
+    auto kern = k_dq_gemv<BITS, GROUP, S16, SL>;
     static std::atomic<uint64_t> done{0};
     const uint64_t bit = 1ull << (dev_id & 63);
     if (!(done.load() & bit)) {
@@ -652,16 +731,39 @@ cudaError_t launch_main(const CUtensorMap &map, const GemvParams &p, int grid, i
     return launch_pdl(kern, dim3(grid), dim3(kThreads), kSmemBytes, st, map, p);
 }
 
+template <int BITS, int GROUP, bool S16>
+cudaError_t launch_slots(int slots, const CUtensorMap &map, const GemvParams &p, int grid, int dev_id,
+                         cudaStream_t st) {
+    constexpr int GPS = stage_codes<BITS>() / GROUP;
+    if (slots == 1) return launch_main<BITS, GROUP, S16, 1>(map, p, grid, dev_id, st);
+    if constexpr (GPS >= 2)
+        if (slots == 2) return launch_main<BITS, GROUP, S16, 2>(map, p, grid, dev_id, st);
+    if constexpr (GPS >= 4)
+        if (slots == 4) return launch_main<BITS, GROUP, S16, 4>(map, p, grid, dev_id, st);
+    if constexpr (GPS >= 8)
+        if (slots == 8) return launch_main<BITS, GROUP, S16, 8>(map, p, grid, dev_id, st);
+    return cudaErrorInvalidValue;
+}
+
+// Slots per run: 8 / MP groups share the mma columns (MP = M rounded up to a
+// power of two), at most the stage's groups.
+inline int gemv_slots(int M, int gps) {
+    const int mp = M <= 1 ? 1 : M <= 2 ? 2 : M <= 4 ? 4 : 8;
+    return std::min(8 / mp, gps);
+}
+
 template <int BITS, int GROUP>
 cudaError_t launch_all(const CUtensorMap &map, const __nv_bfloat16 *X, GemvParams p, const Plan &pl, bool s_f16,
                        __nv_bfloat16 *Y, const DeviceInfo &dev, cudaStream_t st) {
-    const int64_t groups = static_cast<int64_t>(pl.spr) * (stage_codes<BITS>() / GROUP);
+    constexpr int GPS = stage_codes<BITS>() / GROUP;
+    const int slots = gemv_slots(p.M, GPS);
+    const int64_t groups = static_cast<int64_t>(pl.spr) * GPS;
     k_gemv_xprep<BITS, GROUP><<<static_cast<unsigned>(groups), GROUP, 0, st>>>(
-        X, p.M, p.K, const_cast<uint4 *>(p.table), const_cast<float2 *>(p.xso));
+        X, p.M, p.K, slots, const_cast<uint4 *>(p.table), const_cast<float2 *>(p.xso));
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
-    e = s_f16 ? launch_main<BITS, GROUP, true>(map, p, pl.grid, dev.device, st)
-              : launch_main<BITS, GROUP, false>(map, p, pl.grid, dev.device, st);
+    e = s_f16 ? launch_slots<BITS, GROUP, true>(slots, map, p, pl.grid, dev.device, st)
+              : launch_slots<BITS, GROUP, false>(slots, map, p, pl.grid, dev.device, st);
     if (e != cudaSuccess) return e;
     const int64_t MN = static_cast<int64_t>(p.M) * p.N;
     const unsigned rblocks = static_cast<unsigned>(std::min<int64_t>((MN + 255) / 256, 2 * dev.sm_count));

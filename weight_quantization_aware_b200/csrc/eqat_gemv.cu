@@ -75,6 +75,14 @@ constexpr int kSmemBytes = 1024 + kOffBar + 256;
 // lo(e) (low half) and hi(e) (high half), scaled by 4^scale_exp(e), plus 128.
 constexpr uint32_t kMagic = 0x43004300u;  // bf16x2 {128.0, 128.0}
 
+// (w & MASK) | magic in one logic op (truth table 0xEA = (a & b) | c).
+template <uint32_t MASK>
+__device__ __forceinline__ uint32_t and_or(uint32_t w, uint32_t magic) {
+    uint32_t d;
+    asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(d) : "r"(w), "n"(MASK), "r"(magic));
+    return d;
+}
+
 template <int BITS>
 struct Codes;
 
@@ -84,16 +92,16 @@ template <>
 struct Codes<2> {
     static constexpr int kBytes = 4;         // per lane per set
     static constexpr int kCodeBits = 2;
-    __device__ static void extract(const uint32_t *w, uint32_t (&a)[8]) {
+    __device__ static void extract(const uint32_t *w, uint32_t (&a)[8], uint32_t mg) {
         const uint32_t w0 = w[0], w6 = w[0] >> 6, w12 = w[0] >> 12;
-        a[0] = (w0 & 0x00030003u) | kMagic;
-        a[1] = (w0 & 0x000C000Cu) | kMagic;
-        a[2] = (w0 & 0x00300030u) | kMagic;
-        a[3] = (w6 & 0x00030003u) | kMagic;
-        a[4] = (w6 & 0x000C000Cu) | kMagic;
-        a[5] = (w6 & 0x00300030u) | kMagic;
-        a[6] = (w12 & 0x00030003u) | kMagic;
-        a[7] = (w12 & 0x000C000Cu) | kMagic;
+        a[0] = and_or<0x00030003u>(w0, mg);
+        a[1] = and_or<0x000C000Cu>(w0, mg);
+        a[2] = and_or<0x00300030u>(w0, mg);
+        a[3] = and_or<0x00030003u>(w6, mg);
+        a[4] = and_or<0x000C000Cu>(w6, mg);
+        a[5] = and_or<0x00300030u>(w6, mg);
+        a[6] = and_or<0x00030003u>(w12, mg);
+        a[7] = and_or<0x000C000Cu>(w12, mg);
     }
     __host__ __device__ static constexpr int lo(int e) { return e; }
     __host__ __device__ static constexpr int hi(int e) { return e + 8; }
@@ -107,14 +115,14 @@ template <>
 struct Codes<4> {
     static constexpr int kBytes = 8;
     static constexpr int kCodeBits = 4;
-    __device__ static void extract(const uint32_t *w, uint32_t (&a)[8]) {
+    __device__ static void extract(const uint32_t *w, uint32_t (&a)[8], uint32_t mg) {
 #pragma unroll
         for (int p = 0; p < 2; ++p) {
             const uint32_t v = w[p];
-            a[4 * p + 0] = (v & 0x000F000Fu) | kMagic;
-            a[4 * p + 1] = ((v >> 4) & 0x000F000Fu) | kMagic;
-            a[4 * p + 2] = ((v >> 8) & 0x000F000Fu) | kMagic;
-            a[4 * p + 3] = ((v >> 12) & 0x000F000Fu) | kMagic;
+            a[4 * p + 0] = and_or<0x000F000Fu>(v, mg);
+            a[4 * p + 1] = and_or<0x000F000Fu>(v >> 4, mg);
+            a[4 * p + 2] = and_or<0x000F000Fu>(v >> 8, mg);
+            a[4 * p + 3] = and_or<0x000F000Fu>(v >> 12, mg);
         }
     }
     __host__ __device__ static constexpr int lo(int e) { return e < 4 ? e : e + 4; }
@@ -129,11 +137,11 @@ template <>
 struct Codes<3> {
     static constexpr int kBytes = 16;
     static constexpr int kCodeBits = 8;
-    __device__ static void extract(const uint32_t *w, uint32_t (&a)[8]) {
+    __device__ static void extract(const uint32_t *w, uint32_t (&a)[8], uint32_t mg) {
 #pragma unroll
         for (int p = 0; p < 4; ++p) {
-            a[2 * p] = (w[p] & 0x007F007Fu) | kMagic;
-            a[2 * p + 1] = ((w[p] >> 8) & 0x007F007Fu) | kMagic;
+            a[2 * p] = and_or<0x007F007Fu>(w[p], mg);
+            a[2 * p + 1] = and_or<0x007F007Fu>(w[p] >> 8, mg);
         }
     }
     __host__ __device__ static constexpr int lo(int e) { return 4 * (e / 2) + (e % 2); }
@@ -440,8 +448,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     constexpr int MPC = 8 / SL;  // token columns per slot
     static_assert(SL >= 1 && SL <= 8 && GPS % SL == 0, "slots divide the stage's groups");
     extern __shared__ uint8_t smem_raw[];
-    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                                ~static_cast<uintptr_t>(1023));
+    // aligned by an offset from the array itself, so that every pointer below
+    // stays in the shared window (shared loads, 32-bit addresses)
+    uint8_t *smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     float2 *sz = reinterpret_cast<float2 *>(smem + kOffSz);
     uint64_t *full = reinterpret_cast<uint64_t *>(smem + kOffBar);
     uint64_t *empty = full + kStages;
@@ -515,6 +524,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int r0 = lane >> 2, t = lane & 3;
     const int row_a = warp * 16 + r0, row_b = row_a + 8;
     const int slot0 = (2 * t) / MPC, tok0 = (2 * t) % MPC;
+    const uint32_t magic = kMagic;
     // this warp's s / zq slots: [kSlots][16 rows][GPS] float2
     float2 *szw = sz + warp * (kSlots * 16 * kMaxGps);
 
@@ -561,8 +571,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                     load_codes<BITS>(tile, row_a, m * SET_BYTES + t * C::kBytes, wa);
                     load_codes<BITS>(tile, row_b, m * SET_BYTES + t * C::kBytes, wb);
                     uint32_t ea[8], eb[8];
-                    C::extract(wa, ea);
-                    C::extract(wb, eb);
+                    C::extract(wa, ea, magic);
+                    C::extract(wb, eb, magic);
                     const uint4 b01 = table[(m * 2 + 0) * 32 + lane];
                     const uint4 b23 = table[(m * 2 + 1) * 32 + lane];
                     if (gs == 0 && q == 0) {

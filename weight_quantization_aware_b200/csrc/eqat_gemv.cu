@@ -236,6 +236,8 @@ __global__ void __launch_bounds__(GROUP) k_gemv_xprep(const __nv_bfloat16 *__res
     using C = Codes<BITS>;
     constexpr int WARPS = GROUP / 32;
     __shared__ float red[WARPS][16];
+    // the workspace may still be read by the preceding call's kernels
+    pdl_wait();
     pdl_allow_dependents();
     const int gidx = blockIdx.x;
     auto xv = [&](int tok, int64_t k) -> float {
@@ -477,13 +479,30 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (warp == kConsumers) {
         // ------------------------------------------------------------ producer
         if (elect_one_sync()) {
-            // X's fragments and sums come from the preceding k_gemv_xprep
-            pdl_wait();
             uint32_t armed = 0, armed_parity = 0;
             bool ok = true;
             uint32_t it = 0;
             StageCursor c;
             c.init(x_begin, p.spr);
+            // The code tiles do not depend on X: the first ring's worth is requested
+            // before waiting for the preceding k_gemv_xprep; the stages' fragments
+            // and sums follow once it has completed.
+            const int pre = static_cast<int>(x_end - x_begin < kStages ? x_end - x_begin : kStages);
+            {
+                StageCursor cp = c;
+                for (int i = 0; i < pre; ++i, cp.next(p.spr)) {
+                    mbar_arrive_expect_tx(&full[i], kCodeTile + TABLE_BYTES + XO_BYTES);
+                    tma_load_2d(smem + i * kStageBytes, &tm_codes, &full[i], cp.ks * kRowBytes, cp.rt * kRows);
+                }
+                armed = (1u << pre) - 1u;  // parity 0
+            }
+            pdl_wait();
+            for (; static_cast<int>(it) < pre; c.next(p.spr), ++it) {
+                uint8_t *stage = smem + it * kStageBytes;
+                bulk_load(stage + kCodeTile, p.table + static_cast<int64_t>(c.ks) * SETS * 64, TABLE_BYTES, &full[it]);
+                bulk_load(stage + kCodeTile + kTableSlice, p.xso + static_cast<int64_t>(c.ks) * GPS * 8, XO_BYTES,
+                          &full[it]);
+            }
             for (; c.x < x_end; c.next(p.spr), ++it) {
                 const int st = it % kStages;
                 const uint32_t ph = (it / kStages) & 1u;
@@ -671,6 +690,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 __global__ void k_gemv_reduce(const float *__restrict__ partials, int M, int N, int spr, int maxseg,
                               int64_t S, int grid, __nv_bfloat16 *__restrict__ Y) {
     pdl_wait();  // the partials of the preceding k_dq_gemv
+    pdl_allow_dependents();
     const int64_t MN = static_cast<int64_t>(M) * N;
     for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < MN;
          i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
@@ -768,9 +788,8 @@ cudaError_t launch_all(const CUtensorMap &map, const __nv_bfloat16 *X, GemvParam
     constexpr int GPS = stage_codes<BITS>() / GROUP;
     const int slots = gemv_slots(p.M, GPS);
     const int64_t groups = static_cast<int64_t>(pl.spr) * GPS;
-    k_gemv_xprep<BITS, GROUP><<<static_cast<unsigned>(groups), GROUP, 0, st>>>(
-        X, p.M, p.K, slots, const_cast<uint4 *>(p.table), const_cast<float2 *>(p.xso));
-    cudaError_t e = cudaGetLastError();
+    cudaError_t e = launch_pdl(k_gemv_xprep<BITS, GROUP>, dim3(static_cast<unsigned>(groups)), dim3(GROUP), 0, st, X,
+                               p.M, p.K, slots, const_cast<uint4 *>(p.table), const_cast<float2 *>(p.xso));
     if (e != cudaSuccess) return e;
     e = s_f16 ? launch_slots<BITS, GROUP, true>(slots, map, p, pl.grid, dev.device, st)
               : launch_slots<BITS, GROUP, false>(slots, map, p, pl.grid, dev.device, st);

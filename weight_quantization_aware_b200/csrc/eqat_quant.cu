@@ -185,6 +185,32 @@ __global__ void __launch_bounds__(kThreads, 4)
 // One thread per 16 consecutive weights (same group).  zq = clamp(round(z), 0, Q)
 // and the codes use zr := zq (z hard-rounded at pack time).  Output per thread:
 // 4 bytes (2-bit), 8 bytes (4-bit) or 16 bytes (3-bit, one code per byte).
+// Two fp32 lanes in one 64-bit register, and the packed-pair arithmetic of
+// sm_100 (each lane an IEEE round-to-nearest operation, as the scalar forms).
+__device__ __forceinline__ uint64_t f2_pack(float a, float b) {
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a), "f"(b));
+    return r;
+}
+__device__ __forceinline__ void f2_unpack(uint64_t r, float &a, float &b) {
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(a), "=f"(b) : "l"(r));
+}
+__device__ __forceinline__ uint64_t f2_mul(uint64_t a, uint64_t b) {
+    uint64_t d;
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
+    uint64_t d;
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+__device__ __forceinline__ uint64_t f2_sub(uint64_t a, uint64_t b) {
+    uint64_t d;
+    asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+
 template <int BITS>
 __device__ __forceinline__ void pack_chunk(const float (&w)[16], float sc, float zr, float Q, int64_t e0,
                                            uint8_t *__restrict__ codes) {
@@ -194,6 +220,7 @@ __device__ __forceinline__ void pack_chunk(const float (&w)[16], float sc, float
     // not an exact tie (ties may break toward an odd total, but a tie lies in the
     // near band below and takes the exact path).
     const float mz = __fadd_rn(kRoundMagic, zr);
+    const uint64_t rcp2 = f2_pack(rcp, rcp), mz2 = f2_pack(mz, mz);
     // Each code enters its word as the raw bits of M + code (one multiply-add);
     // the bits of M are taken out once per word at the end.
     uint32_t word[4] = {0u, 0u, 0u, 0u};  // 2-bit: word[0]; 4-bit: word[0..1]; 3-bit: word[0..3]
@@ -201,15 +228,23 @@ __device__ __forceinline__ void pack_chunk(const float (&w)[16], float sc, float
     for (int h = 0; h < 2; ++h) {
         float cm[8];
         bool near = false;
+        // two weights per step: u = RN(w rcp), t = RN(u + M + zr), and the
+        // distance u - (t - M - zr) of u from its rounded value
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
-            const float u = __fmul_rn(w[8 * h + j], rcp);
-            const float t = __fadd_rn(u, mz);
+        for (int j = 0; j < 8; j += 2) {
+            const uint64_t u2 = f2_mul(f2_pack(w[8 * h + j], w[8 * h + j + 1]), rcp2);
+            const uint64_t t2 = f2_add(u2, mz2);
+            const uint64_t r2 = f2_sub(u2, f2_sub(t2, mz2));
+            float t0, t1, r0, r1;
+            f2_unpack(t2, t0, t1);
+            f2_unpack(r2, r0, r1);
             // |u - RN(w / s)| < |u| 2^-22: only a u within that of a half-integer can
             // round differently.  A code that is not clamped has |u| <= Q + zr + 1/2 < 64,
             // so a band of 2^-16 covers it; a clamped code does not depend on it.
-            near |= fabsf(__fsub_rn(u, __fsub_rn(t, mz))) >= 0.5f - 0x1p-16f;
-            cm[j] = fminf(fmaxf(t, lo), hi);
+            near |= fabsf(r0) >= 0.5f - 0x1p-16f;
+            near |= fabsf(r1) >= 0.5f - 0x1p-16f;
+            cm[j] = fminf(fmaxf(t0, lo), hi);
+            cm[j + 1] = fminf(fmaxf(t1, lo), hi);
         }
         if (near) {
 #pragma unroll

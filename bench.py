@@ -661,8 +661,9 @@ def decode_gemv(dev, peaks, budget_bytes=300_000_000):
         out[name] = {"N": N, "K": K, "M": M, "bits": b, "group": g, "us": round(t, 2), "GBps": round(gbs, 1),
                      "frac_hbm": round(gbs / peaks["hbm_gbs"], 4), "bf16_matvec_us": round(tb, 2),
                      "speedup_vs_bf16_matvec": round(tb / t, 2), "layers_cycled": L}
-    out["note"] = ("GPU time per call from a CUDA graph of back-to-back calls (3 kernels per call: X fragments, "
-                   "the streaming kernel, the partial sum); bf16 matvec = torch.matmul on bf16 weights, same method")
+    out["note"] = ("GPU time per call from a CUDA graph of back-to-back calls (the streaming kernel and the partial "
+                   "sum; for layers above the build-mode size also the X-fragment kernel); bf16 matvec = "
+                   "torch.matmul on bf16 weights, same method")
     return out
 
 

@@ -102,9 +102,9 @@ int eqat_version(void);
 /* Bytes of device workspace that the linear entry points need for this shape
  * (0 when none): W-hat (N K elements of dt; fp32 mode also an fp32 N K scratch),
  * and for eqat_dq_linear_fwd at decode sizes (bf16, 1 <= M <= 8, group 64 or
- * 128) the larger of that and the decode path's scratch (X's fragments, group
- * sums of X and per-row-tile partials).  A workspace of only N K * sizeof(dt)
- * bytes still works there: the call then dequantizes W-hat and runs the GEMM. */
+ * 128) the larger of that and the decode path's scratch (per-row-tile partial
+ * sums, at most M N K / 128 bytes, which a W-hat-sized workspace always holds;
+ * a smaller one makes the call dequantize W-hat and run the GEMM instead). */
 size_t eqat_workspace_bytes(int64_t M, int64_t N, int64_t K, int bits, int group, int dt);
 
 /* a1. Per-group min-max initialisation (modelfoundations note, Phase 1):
@@ -163,9 +163,8 @@ eqat_status eqat_fq_linear_bwd(const void *X, const void *W, int dt, const float
 
 /* a8. E2E-QP forward on frozen codes (modelfoundations Phase 2: only
  * dequantization in the graph): Y = X ((W_q - zq) s)^T.  At decode sizes (bf16,
- * 1 <= M <= 8, group 64 or 128, workspace of eqat_workspace_bytes()) the codes are
- * streamed once and W-hat is never written: the inference GEMV of the packed
- * model. */
+ * 1 <= M <= 8, group 64 or 128) the codes are streamed once and W-hat is never
+ * written: the inference GEMV of the packed model. */
 eqat_status eqat_dq_linear_fwd(const void *X, int dt, const uint8_t *codes, const uint8_t *zq,
                                const float *s, void *Y, int64_t M, int64_t N, int64_t K, int bits,
                                int group, void *ws, size_t ws_bytes, eqat_stream_t stream);

@@ -123,16 +123,38 @@ def test_gemv_matches_dequant_gemm_path(orc):
     assert np.abs(outs[0] - outs[1]).max() <= 1e-2 * ref
 
 
-def test_gemv_with_w_hat_sized_workspace_takes_the_gemm_path(orc):
-    """A workspace of only N K bf16 elements (below eqat_workspace_bytes at decode
-    sizes) still gives the right result: the call dequantizes and runs the GEMM."""
-    M, N, K, bits, g = 1, 8, 64, 2, 64
+@pytest.mark.parametrize("shape", [(1, 8, 64), (8, 392, 2304)], ids=lambda s: "x".join(map(str, s)))
+def test_gemv_with_w_hat_sized_workspace(orc, shape):
+    """The smallest workspace the call accepts, N K bf16 elements, holds the decode
+    path's partial sums (at most M N K / 128 bytes) and gives the right result."""
+    M, N, K = shape
+    bits, g = 2, 64
     d = synthetic.draw_linear(np.random.default_rng(11), M, N, K, 0.02, "bf16")
     Xn, Wn = synthetic.as_f32_numpy(d["X"]), synthetic.as_f32_numpy(d["W"])
     s, z = orc.minmax_init(Wn, bits, g)
     packed, zq = orc.pack(Wn, s, z, bits, g)
-    assert eqat.workspace_bytes(M, N, K, bits, g, torch.bfloat16) > N * K * 2
+    assert eqat.workspace_bytes(M, N, K, bits, g, torch.bfloat16) >= N * K * 2
     ws = torch.empty(N * K * 2, dtype=torch.uint8, device="cuda")
     Y = eqat.dq_linear_fwd(d["X"].cuda(), torch.from_numpy(packed).cuda(), torch.from_numpy(zq).cuda(),
                            torch.from_numpy(s).cuda(), bits, g, ws=ws)
     assert_close(to_np(Y), orc.dq_linear_fwd(Xn, packed, zq, s, bits, g), TOL_GEMM, "Y")
+
+
+@pytest.mark.parametrize("M", [1, 2])
+def test_gemv_large_layer_fragment_mode(orc, M):
+    """A layer above the build-mode size (44 MB of codes, s and zq, so the fragments
+    come from the separate X kernel at M = 1 and 2, with eight and four group slots),
+    checked on sampled row tiles: the first, two inner ones and the ragged last.
+    The frozen codes, zq and s are drawn directly (any bytes are valid codes)."""
+    N, K, bits, g = 16392, 8192, 2, 64
+    rng = np.random.default_rng(4100 + M)
+    packed = rng.integers(0, 256, size=(N, K // 4), dtype=np.uint8)
+    zq = rng.integers(0, 4, size=(N, K // g), dtype=np.uint8)
+    s = (rng.random((N, K // g), dtype=np.float32) * 0.01 + 1e-3).astype(np.float32)
+    X = torch.randn(M, K, generator=torch.Generator().manual_seed(M)).to(torch.bfloat16)
+    Y = eqat.dq_linear_fwd(X.cuda(), torch.from_numpy(packed).cuda(), torch.from_numpy(zq).cuda(),
+                           torch.from_numpy(s).cuda(), bits, g)
+    rows = np.r_[0:128, 7040:7168, 12800:12928, 16384:N]
+    Xn = synthetic.as_f32_numpy(X)
+    Y_ref = orc.dq_linear_fwd(Xn, packed[rows], zq[rows], s[rows], bits, g)
+    assert_close(to_np(Y)[:, rows], Y_ref, TOL_GEMM, f"Y sampled rows M={M}")

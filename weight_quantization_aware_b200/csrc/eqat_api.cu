@@ -199,7 +199,7 @@ int eqat_version(void) { return EQAT_VERSION; }
 size_t eqat_workspace_bytes(int64_t M, int64_t N, int64_t K, int bits, int group, int dt) {
     if (N <= 0 || K <= 0 || (dt != EQAT_F32 && dt != EQAT_BF16)) return 0;
     size_t need = ws_need(N, K, dt);
-    // the decode path (bf16, M <= 8) keeps X's fragments and partials here
+    // the decode path (bf16, M <= 8) keeps its per-row-tile partial sums here
     if (dt == EQAT_BF16 && M >= 1 && M <= 8 && (group == 64 || group == 128) && bits >= 2 && bits <= 4)
         need = std::max(need, (eqat::gemv_workspace_bound(M, N, K, bits, group) + 255) & ~static_cast<size_t>(255));
     return need;
@@ -438,8 +438,8 @@ eqat_status eqat_dq_linear_fwd_ex(const void *X, int dt, const uint8_t *codes, c
     const bool f32 = dt == EQAT_F32;
     if (!f32 && M <= 8 && (group == 64 || group == 128) && gemv_enabled() &&
         eqat::gemv_workspace_bytes(M, N, K, bits, group, dev.sm_count) <= ws_bytes) {
-        // decode sizes: stream the codes once, no W-hat in memory (a workspace
-        // sized for W-hat only, below eqat_workspace_bytes, takes the path below)
+        // decode sizes: stream the codes once, no W-hat in memory (the partials
+        // take at most M N K / 128 bytes, inside any workspace check_ws accepts)
         EQAT_CUDA(eqat::launch_dq_gemv(X, codes, zq, s, sdt == EQAT_F16, Y, M, N, K, bits, group, ws, dev, st),
                   "dq GEMV");
         return EQAT_OK;

@@ -6,13 +6,15 @@
 // At M <= 8 the layer is bound by HBM: 2-bit codes are 0.25 B per weight plus
 // 5/g B of s and zq, against 2 B per weight for a bf16 matrix.  The codes are
 // streamed once and W-hat is never formed in memory:
-//   - k_gemv_xprep turns X into the B-operand fragments of mma.sync m16n8k16,
-//     permuted and pre-scaled to match the A registers below, plus the per-group
-//     sums that remove the conversion offset and the zero point (a few KB per
-//     token octet, read from L2 afterwards);
 //   - in k_dq_gemv a producer warp moves 128-row x 128-byte code tiles into a
 //     shared-memory ring with TMA (128-byte swizzle, so the per-lane reads hit
-//     distinct banks), with the matching fragment slice by bulk copy;
+//     distinct banks).  The B-operand fragments of mma.sync m16n8k16 (X permuted
+//     and pre-scaled to match the A registers below) and the per-group sums that
+//     remove the conversion offset and the zero point come in one of two ways:
+//     in build mode the producer warp copies the stage's columns of X with the
+//     code tile and turns them into fragments and sums two stages later; in
+//     fragment mode k_gemv_xprep writes them for all of K beforehand (one more
+//     dependent launch, no per-stage work) and the stages copy their slices;
 //   - eight consumer warps each own 16 rows.  A lane turns 16 codes of a row into
 //     eight bf16x2 registers with one AND-OR per register (the "magic number"
 //     conversion: code bits placed in the mantissa of 128.0 give 128 + code * 4^j
@@ -57,18 +59,28 @@ constexpr int kMaxSets = 8;                // 64-column sets per stage, at most 
 constexpr int kMaxGps = 8;                 // groups per stage, at most (2-bit, g = 64)
 constexpr int kTableSlice = kMaxSets * 1024;  // B fragments of one stage
 constexpr int kXoSlice = kMaxGps * 64;        // {xoff, xsum} x 8 tokens of one stage
-// codes at the start of a stage: 1024-byte aligned for the 128-byte swizzle
-constexpr int kStageBytes = (kCodeTile + kTableSlice + kXoSlice + 1023) / 1024 * 1024;
+constexpr int kXSlice = 8 * 512 * 2;          // the stage's columns of X, 8 tokens (2-bit: 512 columns)
+// A stage slot: codes | fragments | group sums | X columns.  Codes at the start
+// of a slot: 1024-byte aligned for the 128-byte swizzle.
+constexpr int kOffTable = kCodeTile;
+constexpr int kOffXo = kOffTable + kTableSlice;
+constexpr int kOffX = kOffXo + kXoSlice;
+// Fragment mode (the fragments come from k_gemv_xprep) has no X columns in a slot.
+template <bool BUILD>
+constexpr int kStageBytes = (kOffX + (BUILD ? kXSlice : 0) + 1023) / 1024 * 1024;
 constexpr int kStages = 6;
 constexpr int kSlots = 2;                  // s / zq staging slots per consumer warp
 constexpr uint64_t kWaitLimitNs = 4000000000ull;
 
 // Shared-memory layout (after 1024-byte alignment): the stage ring, then the
-// s / zq slots, then the barriers.
-constexpr int kOffSz = kStages * kStageBytes;
+// s / zq slots, then the barriers (full, empty, X-arrived per slot, abort flag).
+template <bool BUILD>
+constexpr int kOffSz = kStages * kStageBytes<BUILD>;
 constexpr int kSzBytes = kConsumers * kSlots * 16 * kMaxGps * 8;
-constexpr int kOffBar = kOffSz + kSzBytes;
-constexpr int kSmemBytes = 1024 + kOffBar + 256;
+template <bool BUILD>
+constexpr int kOffBar = kOffSz<BUILD> + kSzBytes;
+template <bool BUILD>
+constexpr int kSmemBytes = 1024 + kOffBar<BUILD> + 256;
 
 // Codes of one lane for one 64-column set of a row: 16 codes (columns 16t..16t+15
 // of the set).  extract() produces eight bf16x2 registers; register e holds codes
@@ -170,8 +182,9 @@ __device__ __forceinline__ void bulk_load(void *smem_dst, const void *src, uint3
 struct GemvParams {
     const uint8_t *zq;
     const void *s;
-    const uint4 *table;  // B fragments of X: [sets_pad][2][32]
-    const float2 *xso;   // {xoff, xsum}: [groups_pad][8 tokens]
+    const __nv_bfloat16 *X;  // [M][K]
+    const uint4 *table;  // fragment mode only: B fragments of X from k_gemv_xprep, [sets_pad][2][32]
+    const float2 *xso;   // fragment mode only: {xoff, xsum}, [groups_pad][8 tokens]
     float *partials;     // [row_tiles][maxseg][M][kRows]
     int M, N, G;
     int64_t K;
@@ -212,6 +225,82 @@ struct StageCursor {
         }
     }
 };
+
+// The stage's mma fragments (the B operand) and group sums from its columns of
+// X, by the 32 lanes of the producer warp.  Fragment column n = lane / 4 is
+// (slot n / MPC, token n % MPC), MPC = 8 / SL.  Lane (n, t) writes the entries of
+// the sets of the groups of its slot (the group's index within the stage, modulo
+// SL), built from columns 16t .. 16t + 15 of each set: the same entries that lane
+// reads as a consumer.  Entry (set m, ip) holds registers e = 4 ip .. 4 ip + 3, and
+// register e pairs columns lo(e) (low half) and hi(e), scaled by 4^-scale_exp(e).
+// The four lanes of a quad then add up the group's sums: xsum = sum x and
+// xoff = sum 128 4^-j x (j the exponent of the column's code position).  Entries
+// of the other slots, and of tokens beyond M, stay zero (set once).  Columns at or
+// beyond kcols (the end of K) read as zero; kcols is a multiple of 64.
+template <int BITS, int GROUP, int SL>
+__device__ __forceinline__ void build_stage(uint8_t *slot, int M, int kcols, int lane) {
+    using C = Codes<BITS>;
+    constexpr int KS = stage_codes<BITS>();
+    constexpr int SPG = GROUP / 64;
+    constexpr int GPS = KS / GROUP;
+    constexpr int MPC = 8 / SL;
+    const int n = lane >> 2, t = lane & 3;
+    const int sl = n / MPC, tok = n % MPC;
+    uint4 *table = reinterpret_cast<uint4 *>(slot + kOffTable);
+    float2 *xo = reinterpret_cast<float2 *>(slot + kOffXo);
+    const uint4 *xs = reinterpret_cast<const uint4 *>(slot + kOffX);  // [token][KS] bf16
+#pragma unroll
+    for (int i = 0; i < GPS / SL; ++i) {
+        const int gs = sl + SL * i;
+        float xsum = 0.0f, xoff = 0.0f;
+#pragma unroll
+        for (int q = 0; q < SPG; ++q) {
+            const int m = gs * SPG + q;
+            const int c0 = 64 * m + 16 * t;  // the lane's first column in the stage
+            uint32_t xw[8];                  // word k: columns c0 + 2k (low half), c0 + 2k + 1
+            if (tok < M && c0 < kcols) {
+                const uint4 a = xs[(tok * KS + c0) / 8], b = xs[(tok * KS + c0) / 8 + 1];
+                xw[0] = a.x; xw[1] = a.y; xw[2] = a.z; xw[3] = a.w;
+                xw[4] = b.x; xw[5] = b.y; xw[6] = b.z; xw[7] = b.w;
+            } else {
+#pragma unroll
+                for (int k = 0; k < 8; ++k) xw[k] = 0u;
+            }
+            uint32_t r[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+                const int lo = C::lo(e), hi = C::hi(e);
+                // bytes of column lo for the low half, of column hi for the high half
+                const uint32_t sel = (2u * (lo & 1)) | ((2u * (lo & 1) + 1u) << 4) | ((4u + 2u * (hi & 1)) << 8) |
+                                     ((5u + 2u * (hi & 1)) << 12);
+                uint32_t v = __byte_perm(xw[lo >> 1], xw[hi >> 1], sel);
+                if (C::scale_exp(e) != 0) {
+                    const __nv_bfloat162 f = __float2bfloat162_rn(C::scale_exp(e) == 1 ? 0.25f : 0.0625f);
+                    __nv_bfloat162 h = *reinterpret_cast<const __nv_bfloat162 *>(&v);
+                    h = __hmul2(h, f);
+                    v = *reinterpret_cast<const uint32_t *>(&h);
+                }
+                r[e] = v;
+            }
+            table[(m * 2 + 0) * 32 + lane] = make_uint4(r[0], r[1], r[2], r[3]);
+            table[(m * 2 + 1) * 32 + lane] = make_uint4(r[4], r[5], r[6], r[7]);
+#pragma unroll
+            for (int k = 0; k < 8; ++k) {
+                const float x0 = __uint_as_float(xw[k] << 16), x1 = __uint_as_float(xw[k] & 0xFFFF0000u);
+                constexpr float kw[3] = {128.0f, 32.0f, 8.0f};
+                xsum += x0;
+                xsum += x1;
+                xoff = fmaf(x0, kw[C::pos_exp(2 * k)], xoff);
+                xoff = fmaf(x1, kw[C::pos_exp(2 * k + 1)], xoff);
+            }
+        }
+        xsum += __shfl_xor_sync(0xffffffffu, xsum, 1);
+        xsum += __shfl_xor_sync(0xffffffffu, xsum, 2);
+        xoff += __shfl_xor_sync(0xffffffffu, xoff, 1);
+        xoff += __shfl_xor_sync(0xffffffffu, xoff, 2);
+        if (t == 0 && tok < M) xo[gs * 8 + tok] = make_float2(xoff, xsum);
+    }
+}
 
 __device__ __forceinline__ uint32_t bf16x2_bits(float lo, float hi) {
     const __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
@@ -436,7 +525,9 @@ __device__ __forceinline__ void load_codes(const uint8_t *tile, int row, int byt
 }
 
 
-template <int BITS, int GROUP, bool S16, int SL>
+// BUILD: the producer warp builds each stage's fragments from X (build mode);
+// otherwise they come by bulk copy from the table of k_gemv_xprep (fragment mode).
+template <int BITS, int GROUP, bool S16, int SL, bool BUILD>
 __global__ void __launch_bounds__(kThreads, 1)
     k_dq_gemv(const __grid_constant__ CUtensorMap tm_codes, const GemvParams p) {
     using C = Codes<BITS>;
@@ -445,32 +536,50 @@ __global__ void __launch_bounds__(kThreads, 1)
     constexpr int SET_BYTES = 64 * C::kCodeBits / 8;  // code bytes of a set in one row
     constexpr int SPG = GROUP / 64;                   // sets per group
     constexpr int GPS = KS / GROUP;                   // groups per stage
-    constexpr uint32_t TABLE_BYTES = SETS * 1024;
-    constexpr uint32_t XO_BYTES = GPS * 64;
     constexpr int MPC = 8 / SL;  // token columns per slot
     static_assert(SL >= 1 && SL <= 8 && GPS % SL == 0, "slots divide the stage's groups");
     extern __shared__ uint8_t smem_raw[];
     // aligned by an offset from the array itself, so that every pointer below
     // stays in the shared window (shared loads, 32-bit addresses)
     uint8_t *smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
-    float2 *sz = reinterpret_cast<float2 *>(smem + kOffSz);
-    uint64_t *full = reinterpret_cast<uint64_t *>(smem + kOffBar);
+    constexpr int kSlot = kStageBytes<BUILD>;
+    float2 *sz = reinterpret_cast<float2 *>(smem + kOffSz<BUILD>);
+    // Build mode: full[s] = the slot's fragments are built (the producer warp's 32
+    // lanes), xfull[s] = its code tile and X columns have landed (transaction
+    // bytes).  Fragment mode: full[s] = the code tile, fragments and sums have
+    // landed (transaction bytes); xfull is unused.  empty[s]: the consumers are
+    // done with the slot.
+    uint64_t *full = reinterpret_cast<uint64_t *>(smem + kOffBar<BUILD>);
     uint64_t *empty = full + kStages;
-    volatile int *abort_flag = reinterpret_cast<volatile int *>(empty + kStages);
+    uint64_t *xfull = empty + kStages;
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(xfull + kStages);
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < kStages; ++i) {
-            mbar_init(&full[i], 1);
+            mbar_init(&full[i], BUILD ? 32 : 1);
             mbar_init(&empty[i], kConsumers);
+            mbar_init(&xfull[i], 1);
         }
         *abort_flag = 0;
         fence_mbarrier_init();
         tma_prefetch_desc(&tm_codes);
         pdl_allow_dependents();
     }
+    if constexpr (BUILD) {
+        // fragment entries that no stage writes (other slots, tokens beyond M) are zero
+        for (int s = 0; s < kStages; ++s) {
+            uint4 *z = reinterpret_cast<uint4 *>(smem + s * kSlot + kOffTable);
+            for (int i = threadIdx.x; i < (kTableSlice + kXoSlice) / 16; i += kThreads)
+                z[i] = make_uint4(0u, 0u, 0u, 0u);
+        }
+    }
     __syncthreads();
+    // Build mode: X, the codes, s and zq may come from the preceding kernel.  In
+    // fragment mode the preceding kernel is k_gemv_xprep, which waited for them;
+    // the producer waits for k_gemv_xprep itself (below).
+    if constexpr (BUILD) pdl_wait();
 
     const int64_t S = p.total_stages;
     const int64_t x_begin = static_cast<int64_t>(blockIdx.x) * S / gridDim.x;
@@ -478,59 +587,120 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     if (warp == kConsumers) {
         // ------------------------------------------------------------ producer
-        if (elect_one_sync()) {
-            uint32_t armed = 0, armed_parity = 0;
-            bool ok = true;
-            uint32_t it = 0;
-            StageCursor c;
-            c.init(x_begin, p.spr);
-            // The code tiles do not depend on X: the first ring's worth is requested
-            // before waiting for the preceding k_gemv_xprep; the stages' fragments
-            // and sums follow once it has completed.
-            const int pre = static_cast<int>(x_end - x_begin < kStages ? x_end - x_begin : kStages);
-            {
-                StageCursor cp = c;
-                for (int i = 0; i < pre; ++i, cp.next(p.spr)) {
-                    mbar_arrive_expect_tx(&full[i], kCodeTile + TABLE_BYTES + XO_BYTES);
-                    tma_load_2d(smem + i * kStageBytes, &tm_codes, &full[i], cp.ks * kRowBytes, cp.rt * kRows);
-                }
-                armed = (1u << pre) - 1u;  // parity 0
-            }
-            pdl_wait();
-            for (; static_cast<int>(it) < pre; c.next(p.spr), ++it) {
-                uint8_t *stage = smem + it * kStageBytes;
-                bulk_load(stage + kCodeTile, p.table + static_cast<int64_t>(c.ks) * SETS * 64, TABLE_BYTES, &full[it]);
-                bulk_load(stage + kCodeTile + kTableSlice, p.xso + static_cast<int64_t>(c.ks) * GPS * 8, XO_BYTES,
-                          &full[it]);
-            }
-            for (; c.x < x_end; c.next(p.spr), ++it) {
-                const int st = it % kStages;
-                const uint32_t ph = (it / kStages) & 1u;
-                if (!mbar_wait_bounded(&empty[st], ph ^ 1u, abort_flag, p.err, p.wait_limit_ns)) {
-                    ok = false;
-                    break;
-                }
-                const int rt = c.rt, ks = c.ks;
-                uint8_t *stage = smem + st * kStageBytes;
-                mbar_arrive_expect_tx(&full[st], kCodeTile + TABLE_BYTES + XO_BYTES);
-                armed |= 1u << st;
-                armed_parity = (armed_parity & ~(1u << st)) | (ph << st);
-                tma_load_2d(stage, &tm_codes, &full[st], ks * kRowBytes, rt * kRows);
-                bulk_load(stage + kCodeTile, p.table + static_cast<int64_t>(ks) * SETS * 64, TABLE_BYTES, &full[st]);
-                bulk_load(stage + kCodeTile + kTableSlice, p.xso + static_cast<int64_t>(ks) * GPS * 8, XO_BYTES,
-                          &full[st]);
-            }
-            if (!ok) {
-                // let issued copies land before the block can exit
-                for (int st = 0; st < kStages; ++st)
-                    if (armed & (1u << st)) {
-                        const uint32_t a = smem_u32(&full[st]);
-                        const uint64_t t0 = globaltimer_ns();
-                        while (!mbar_try_wait(a, (armed_parity >> st) & 1u) &&
-                               globaltimer_ns() - t0 < 100000000ull) {
-                        }
+        if constexpr (!BUILD) {
+            // Fragment mode: one elected lane requests each stage's code tile (TMA)
+            // and its slices of the fragment table and the group sums (bulk copies) on
+            // full[s].  The code tiles do not depend on X: the first ring's worth is
+            // requested before waiting for the preceding k_gemv_xprep.
+            if (elect_one_sync()) {
+                uint32_t armed = 0, armed_parity = 0;
+                bool ok = true;
+                uint32_t it = 0;
+                StageCursor c;
+                c.init(x_begin, p.spr);
+                constexpr uint32_t kFragBytes = SETS * 1024 + GPS * 64;
+                const int pre = static_cast<int>(x_end - x_begin < kStages ? x_end - x_begin : kStages);
+                {
+                    StageCursor cp = c;
+                    for (int i = 0; i < pre; ++i, cp.next(p.spr)) {
+                        mbar_arrive_expect_tx(&full[i], kCodeTile + kFragBytes);
+                        tma_load_2d(smem + i * kSlot, &tm_codes, &full[i], cp.ks * kRowBytes, cp.rt * kRows);
                     }
+                    armed = (1u << pre) - 1u;  // parity 0
+                }
+                pdl_wait();
+                for (; static_cast<int>(it) < pre; c.next(p.spr), ++it) {
+                    uint8_t *stage = smem + it * kSlot;
+                    bulk_load(stage + kOffTable, p.table + static_cast<int64_t>(c.ks) * SETS * 64, SETS * 1024,
+                              &full[it]);
+                    bulk_load(stage + kOffXo, p.xso + static_cast<int64_t>(c.ks) * GPS * 8, GPS * 64, &full[it]);
+                }
+                for (; c.x < x_end; c.next(p.spr), ++it) {
+                    const int st = it % kStages;
+                    const uint32_t ph = (it / kStages) & 1u;
+                    if (!mbar_wait_bounded(&empty[st], ph ^ 1u, abort_flag, p.err, p.wait_limit_ns)) {
+                        ok = false;
+                        break;
+                    }
+                    uint8_t *stage = smem + st * kSlot;
+                    mbar_arrive_expect_tx(&full[st], kCodeTile + kFragBytes);
+                    armed |= 1u << st;
+                    armed_parity = (armed_parity & ~(1u << st)) | (ph << st);
+                    tma_load_2d(stage, &tm_codes, &full[st], c.ks * kRowBytes, c.rt * kRows);
+                    bulk_load(stage + kOffTable, p.table + static_cast<int64_t>(c.ks) * SETS * 64, SETS * 1024,
+                              &full[st]);
+                    bulk_load(stage + kOffXo, p.xso + static_cast<int64_t>(c.ks) * GPS * 8, GPS * 64, &full[st]);
+                }
+                if (!ok) {
+                    // let issued copies land before the block can exit
+                    for (int st = 0; st < kStages; ++st)
+                        if (armed & (1u << st)) {
+                            const uint32_t a = smem_u32(&full[st]);
+                            const uint64_t t0 = globaltimer_ns();
+                            while (!mbar_try_wait(a, (armed_parity >> st) & 1u) &&
+                                   globaltimer_ns() - t0 < 100000000ull) {
+                            }
+                        }
+                }
             }
+            __syncwarp();
+            return;
+        }
+        // Build mode: lane 0 requests each stage's code tile (TMA) and the stage's
+        // columns of X (one bulk copy per token) on xfull[s].  kLag stages behind,
+        // the whole warp turns those columns into the stage's fragments and group
+        // sums and arrives on full[s].  In the steady state the consumers are
+        // kStages - 1 stages behind the requests, so each stage is built well
+        // before its use.
+        uint32_t armed = 0, armed_parity = 0;
+        bool ok = true;
+        StageCursor ci, cb;
+        ci.init(x_begin, p.spr);
+        cb = ci;
+        const int64_t n = x_end - x_begin;
+        constexpr int kLag = 2;
+        for (int64_t i = 0; i < n + kLag; ++i) {
+            if (i < n) {
+                const int st = static_cast<int>(i % kStages);
+                const uint32_t ph = static_cast<uint32_t>(i / kStages) & 1u;
+                ok = mbar_wait_bounded(&empty[st], ph ^ 1u, abort_flag, p.err, p.wait_limit_ns) && ok;
+                if (!__all_sync(0xffffffffu, ok)) break;
+                if (lane == 0) {
+                    const int64_t k0 = static_cast<int64_t>(ci.ks) * KS;
+                    const uint32_t xbytes = static_cast<uint32_t>((p.K - k0 < KS ? p.K - k0 : KS) * 2);
+                    uint8_t *stage = smem + st * kSlot;
+                    mbar_arrive_expect_tx(&xfull[st], kCodeTile + p.M * xbytes);
+                    armed |= 1u << st;
+                    armed_parity = (armed_parity & ~(1u << st)) | (ph << st);
+                    tma_load_2d(stage, &tm_codes, &xfull[st], ci.ks * kRowBytes, ci.rt * kRows);
+                    for (int tok = 0; tok < p.M; ++tok)
+                        bulk_load(stage + kOffX + tok * KS * 2, p.X + tok * p.K + k0, xbytes, &xfull[st]);
+                }
+                __syncwarp();
+                ci.next(p.spr);
+            }
+            if (i >= kLag) {
+                const int64_t b = i - kLag;
+                const int st = static_cast<int>(b % kStages);
+                const uint32_t ph = static_cast<uint32_t>(b / kStages) & 1u;
+                ok = mbar_wait_bounded(&xfull[st], ph, abort_flag, p.err, p.wait_limit_ns) && ok;
+                if (!__all_sync(0xffffffffu, ok)) break;
+                const int64_t k0 = static_cast<int64_t>(cb.ks) * KS;
+                build_stage<BITS, GROUP, SL>(smem + st * kSlot, p.M, static_cast<int>(p.K - k0 < KS ? p.K - k0 : KS),
+                                             lane);
+                mbar_arrive(&full[st]);
+                cb.next(p.spr);
+            }
+        }
+        if (!ok && lane == 0) {
+            // let issued copies land before the block can exit
+            for (int st = 0; st < kStages; ++st)
+                if (armed & (1u << st)) {
+                    const uint32_t a = smem_u32(&xfull[st]);
+                    const uint64_t t0 = globaltimer_ns();
+                    while (!mbar_try_wait(a, (armed_parity >> st) & 1u) && globaltimer_ns() - t0 < 100000000ull) {
+                    }
+                }
         }
         __syncwarp();
         return;
@@ -571,10 +741,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         pf.next(p.spr);
         const int st = it % kStages;
         const uint32_t ph = (it / kStages) & 1u;
+        // build mode: the code tile (written by TMA), then the fragments (by the
+        // producer warp); fragment mode: all of it by copies on full[st]
+        if constexpr (BUILD) ok = mbar_wait_bounded(&xfull[st], ph, abort_flag, p.err, p.wait_limit_ns) && ok;
         ok = mbar_wait_bounded(&full[st], ph, abort_flag, p.err, p.wait_limit_ns) && ok;
-        const uint8_t *tile = smem + st * kStageBytes;
-        const uint4 *table = reinterpret_cast<const uint4 *>(tile + kCodeTile);
-        const float2 *xo = reinterpret_cast<const float2 *>(tile + kCodeTile + kTableSlice);
+        const uint8_t *tile = smem + st * kSlot;
+        const uint4 *table = reinterpret_cast<const uint4 *>(tile + kOffTable);
+        const float2 *xo = reinterpret_cast<const float2 *>(tile + kOffXo);
         const float2 *szs = szw + (it % kSlots) * (16 * kMaxGps);
         // Runs of SL groups: the four mmas of a set go to four accumulator chains,
         // and the run's groups share them (each in its own columns).
@@ -724,8 +897,18 @@ cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t sme
 struct Plan {
     int spr, row_tiles, maxseg, grid;
     int64_t S;
+    bool build;  // fragments built in the streaming kernel (else by k_gemv_xprep)
     size_t table_bytes, xso_bytes, partial_bytes;
 };
+
+// Build mode saves the k_gemv_xprep launch (about 2.4 us per call on B200) but
+// puts the fragment build (work in proportion to M) on the producer warp's
+// scheduler for every stage.  Measured, it pays for M = 1 below about 32 MB of
+// codes, s and zq, and for M = 2 below about 8 MB; fragment mode elsewhere.
+inline bool build_mode(int64_t M, int64_t N, int64_t K, int bits, int group) {
+    const int64_t bytes = N * K * (bits == 3 ? 8 : bits) / 8 + N * (K / group) * 5;
+    return (M == 1 && bytes <= (int64_t(32) << 20)) || (M == 2 && bytes <= (int64_t(8) << 20));
+}
 
 Plan make_plan(int64_t M, int64_t N, int64_t K, int bits, int group, int sms) {
     Plan pl{};
@@ -740,38 +923,48 @@ Plan make_plan(int64_t M, int64_t N, int64_t K, int bits, int group, int sms) {
         const int c1 = cta_of_stage(static_cast<int64_t>(rt) * pl.spr + pl.spr - 1, pl.S, pl.grid);
         pl.maxseg = std::max(pl.maxseg, c1 - c0 + 1);
     }
+    pl.build = build_mode(M, N, K, bits, group);
     const int64_t sets = static_cast<int64_t>(pl.spr) * (ks / 64);
     const int64_t groups = static_cast<int64_t>(pl.spr) * (ks / group);
-    pl.table_bytes = static_cast<size_t>(sets) * 1024;
-    pl.xso_bytes = (static_cast<size_t>(groups) * 64 + 255) / 256 * 256;
+    pl.table_bytes = pl.build ? 0 : static_cast<size_t>(sets) * 1024;
+    pl.xso_bytes = pl.build ? 0 : (static_cast<size_t>(groups) * 64 + 255) / 256 * 256;
     pl.partial_bytes = static_cast<size_t>(pl.row_tiles) * pl.maxseg * M * kRows * 4;
     return pl;
 }
 
-template <int BITS, int GROUP, bool S16, int SL>
+template <int BITS, int GROUP, bool S16, int SL, bool BUILD>
 cudaError_t launch_main(const CUtensorMap &map, const GemvParams &p, int grid, int dev_id, cudaStream_t st) {
-    auto kern = k_dq_gemv<BITS, GROUP, S16, SL>;
+    auto kern = k_dq_gemv<BITS, GROUP, S16, SL, BUILD>;
     static std::atomic<uint64_t> done{0};
     const uint64_t bit = 1ull << (dev_id & 63);
     if (!(done.load() & bit)) {
-        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes<BUILD>);
         if (e != cudaSuccess) return e;
         done.fetch_or(bit);
     }
-    return launch_pdl(kern, dim3(grid), dim3(kThreads), kSmemBytes, st, map, p);
+    return launch_pdl(kern, dim3(grid), dim3(kThreads), kSmemBytes<BUILD>, st, map, p);
 }
 
 template <int BITS, int GROUP, bool S16>
-cudaError_t launch_slots(int slots, const CUtensorMap &map, const GemvParams &p, int grid, int dev_id,
+cudaError_t launch_slots(int slots, bool build, const CUtensorMap &map, const GemvParams &p, int grid, int dev_id,
                          cudaStream_t st) {
     constexpr int GPS = stage_codes<BITS>() / GROUP;
-    if (slots == 1) return launch_main<BITS, GROUP, S16, 1>(map, p, grid, dev_id, st);
+    constexpr int SL1 = GPS < 8 ? GPS : 8;  // slots at M = 1
+    constexpr int SL2 = GPS < 4 ? GPS : 4;  // slots at M = 2
+    if (build) {
+        // build mode runs at M <= 2 only
+        if (slots == SL1) return launch_main<BITS, GROUP, S16, SL1, true>(map, p, grid, dev_id, st);
+        if constexpr (SL2 != SL1)
+            if (slots == SL2) return launch_main<BITS, GROUP, S16, SL2, true>(map, p, grid, dev_id, st);
+        return cudaErrorInvalidValue;
+    }
+    if (slots == 1) return launch_main<BITS, GROUP, S16, 1, false>(map, p, grid, dev_id, st);
     if constexpr (GPS >= 2)
-        if (slots == 2) return launch_main<BITS, GROUP, S16, 2>(map, p, grid, dev_id, st);
+        if (slots == 2) return launch_main<BITS, GROUP, S16, 2, false>(map, p, grid, dev_id, st);
     if constexpr (GPS >= 4)
-        if (slots == 4) return launch_main<BITS, GROUP, S16, 4>(map, p, grid, dev_id, st);
+        if (slots == 4) return launch_main<BITS, GROUP, S16, 4, false>(map, p, grid, dev_id, st);
     if constexpr (GPS >= 8)
-        if (slots == 8) return launch_main<BITS, GROUP, S16, 8>(map, p, grid, dev_id, st);
+        if (slots == 8) return launch_main<BITS, GROUP, S16, 8, false>(map, p, grid, dev_id, st);
     return cudaErrorInvalidValue;
 }
 
@@ -783,16 +976,19 @@ inline int gemv_slots(int M, int gps) {
 }
 
 template <int BITS, int GROUP>
-cudaError_t launch_all(const CUtensorMap &map, const __nv_bfloat16 *X, GemvParams p, const Plan &pl, bool s_f16,
-                       __nv_bfloat16 *Y, const DeviceInfo &dev, cudaStream_t st) {
+cudaError_t launch_all(const CUtensorMap &map, GemvParams p, const Plan &pl, bool s_f16, __nv_bfloat16 *Y,
+                       const DeviceInfo &dev, cudaStream_t st) {
     constexpr int GPS = stage_codes<BITS>() / GROUP;
     const int slots = gemv_slots(p.M, GPS);
-    const int64_t groups = static_cast<int64_t>(pl.spr) * GPS;
-    cudaError_t e = launch_pdl(k_gemv_xprep<BITS, GROUP>, dim3(static_cast<unsigned>(groups)), dim3(GROUP), 0, st, X,
-                               p.M, p.K, slots, const_cast<uint4 *>(p.table), const_cast<float2 *>(p.xso));
-    if (e != cudaSuccess) return e;
-    e = s_f16 ? launch_slots<BITS, GROUP, true>(slots, map, p, pl.grid, dev.device, st)
-              : launch_slots<BITS, GROUP, false>(slots, map, p, pl.grid, dev.device, st);
+    if (!pl.build) {
+        const int64_t groups = static_cast<int64_t>(pl.spr) * GPS;
+        cudaError_t e = launch_pdl(k_gemv_xprep<BITS, GROUP>, dim3(static_cast<unsigned>(groups)), dim3(GROUP), 0,
+                                   st, p.X, p.M, p.K, slots, const_cast<uint4 *>(p.table),
+                                   const_cast<float2 *>(p.xso));
+        if (e != cudaSuccess) return e;
+    }
+    cudaError_t e = s_f16 ? launch_slots<BITS, GROUP, true>(slots, pl.build, map, p, pl.grid, dev.device, st)
+                          : launch_slots<BITS, GROUP, false>(slots, pl.build, map, p, pl.grid, dev.device, st);
     if (e != cudaSuccess) return e;
     const int64_t MN = static_cast<int64_t>(p.M) * p.N;
     const unsigned rblocks = static_cast<unsigned>(std::min<int64_t>((MN + 255) / 256, 2 * dev.sm_count));
@@ -830,6 +1026,7 @@ cudaError_t launch_dq_gemv(const void *X, const uint8_t *codes, const uint8_t *z
     GemvParams p{};
     p.zq = zq;
     p.s = s;
+    p.X = static_cast<const __nv_bfloat16 *>(X);
     p.table = reinterpret_cast<const uint4 *>(w);
     p.xso = reinterpret_cast<const float2 *>(w + pl.table_bytes);
     p.partials = reinterpret_cast<float *>(w + pl.table_bytes + pl.xso_bytes);
@@ -848,10 +1045,9 @@ cudaError_t launch_dq_gemv(const void *X, const uint8_t *codes, const uint8_t *z
     p.total_stages = pl.S;
     p.err = device_error_word();
     p.wait_limit_ns = kWaitLimitNs;
-    const __nv_bfloat16 *Xb = static_cast<const __nv_bfloat16 *>(X);
     __nv_bfloat16 *Yb = static_cast<__nv_bfloat16 *>(Y);
 #define EQAT_GEMV_CASE(B, GR) \
-    if (bits == B && group == GR) return launch_all<B, GR>(map, Xb, p, pl, s_f16, Yb, dev, st);
+    if (bits == B && group == GR) return launch_all<B, GR>(map, p, pl, s_f16, Yb, dev, st);
     EQAT_GEMV_CASE(2, 64)
     EQAT_GEMV_CASE(2, 128)
     EQAT_GEMV_CASE(3, 64)

@@ -258,6 +258,8 @@ def test_backward_single_contraction_paths(orc):
     (1024, 520, 2048, 2, 64),    # fewer tiles than SMs, long K
     (1024, 1024, 1024, 3, 128),  # grouped backward with one partial wave
     (520, 256, 1536, 2, 32),     # ragged M and N tails, long K
+    (256, 4096, 2048, 2, 64),    # grouped backward whose dX tiles are 16x deeper than its dW-hat tiles
+    (4096, 256, 1024, 2, 64),    # and the other way round
 ], ids=lambda s: "x".join(map(str, s)))
 def test_long_k_partial_wave_launches(orc, shape):
     """Launches of fewer tiles than SMs with long reductions, twice in a row on one

@@ -755,12 +755,24 @@ def calibrate_rows(target_s: float) -> int:
     return int(max(4, min(WORKLOAD.m, (target_s - fixed) / per_row)))
 
 
+def cpu_model() -> str:
+    """The host CPU's model name (first entry of /proc/cpuinfo), for the baseline's record."""
+    try:
+        with open("/proc/cpuinfo") as f:
+            for ln in f:
+                if ln.startswith("model name"):
+                    return ln.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
+
+
 def cpu_baseline(target_s: float = 15.0):
     import oracle
     rows = calibrate_rows(target_s)
     dt, flops, desc = oracle_sample(rows)
     return {"value": round(flops / dt / 1e12, 6), "unit": "TFLOP/s", "cores": oracle.num_threads(),
-            "kind": "oracle", "sample": desc, "seconds": round(dt, 2)}
+            "cpu": cpu_model(), "kind": "oracle", "sample": desc, "seconds": round(dt, 2)}
 
 
 def run_reference(args):
@@ -786,7 +798,7 @@ def run_reference(args):
             "data": "synthetic",
             "config": {"workload": wl.name, "M": wl.m, "N": lin.n, "K": lin.k, "bits": wl.bits, "group": wl.group},
             "cpu_baseline": {"value": round(value, 6), "unit": "TFLOP/s", "cores": oracle.num_threads(),
-                             "kind": "oracle", "sample": desc},
+                             "cpu": cpu_model(), "kind": "oracle", "sample": desc},
             "e2e": {"value": round(value, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
 

@@ -815,6 +815,7 @@ def main():
     ap.add_argument("--no-variants", action="store_true")
     ap.add_argument("--no-gemv", action="store_true")
     ap.add_argument("--gemv-only", action="store_true")
+    ap.add_argument("--gemv-layer", default="70b-gate_proj", choices=["70b-gate_proj", "7b-q_proj"])
     ap.add_argument("--no-blockap", action="store_true")
     ap.add_argument("--blockap-only", action="store_true")
     ap.add_argument("--no-configs", action="store_true")
@@ -833,11 +834,12 @@ def main():
         eqat.load_library()
         print(json.dumps(blockap_block(torch.device("cuda", 0), load_peaks(), steps=2)), flush=True)
         return
-    if args.gemv_only:  # profiling aid: four plain decode GEMV calls, Llama-2-70B gate_proj w2g64, M = 1
+    if args.gemv_only:  # profiling aid: four plain decode GEMV calls at M = 1, w2g64
         torch.cuda.set_device(0)
         eqat.load_library()
         dev = torch.device("cuda", 0)
-        N, K, b, g = 28672, 8192, 2, 64
+        # Llama-2-70B gate_proj (fragment mode), or Llama-2-7B q_proj (build mode)
+        N, K, b, g = (4096, 4096, 2, 64) if args.gemv_layer == "7b-q_proj" else (28672, 8192, 2, 64)
         gen = torch.Generator(device=dev)
         gen.manual_seed(2000 + N)
         c = torch.randint(0, 256, (N, K * b // 8), generator=gen, device=dev, dtype=torch.uint8)

@@ -21,8 +21,8 @@ every rank runs the same step on its own token batch (weak scaling) and the
 weight gradients dW, ds, dz and the E2E ds are summed over ranks with NCCL
 all-reduce inside the step (data-parallel training).
 
---impl reference times the CPU oracle (the only other arm) on a
-bounded sample of the same workload.
+--impl reference times the CPU oracle (the only other arm: the pages hold no
+code to run) on a bounded sample of the same workload.
 """
 from __future__ import annotations
 

@@ -26,7 +26,7 @@
  * fast-math so that no step is fused or reassociated.  Contractions and
  * reductions accumulate in fp64 (fp32 x fp32 products are exact in fp64).
  *
- * Readings where the pages are silent (each one also listed in the design doc):
+ * Readings where the pages are silent:
  *   round()            = round-half-to-even (rintf under the default mode);
  *   W / s              = one correctly rounded fp32 division (never x * (1/s));
  *   s                  = (xmax - xmin) / (2^N - 1) in fp32, then max(s, 1e-5);

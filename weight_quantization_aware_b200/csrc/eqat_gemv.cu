@@ -53,34 +53,15 @@ namespace {
 constexpr int kConsumers = 8;              // consumer warps, 16 rows each
 constexpr int kRows = 16 * kConsumers;     // rows of a tile
 constexpr int kThreads = (kConsumers + 1) * 32;
-constexpr int kRowBytes = 128;             // code bytes of one row per stage
-constexpr int kCodeTile = kRows * kRowBytes;
+constexpr int kRowBytes = 128;             // code bytes of one row per TMA box
 constexpr int kMaxSets = 8;                // 64-column sets per stage, at most (2-bit)
 constexpr int kMaxGps = 8;                 // groups per stage, at most (2-bit, g = 64)
 constexpr int kTableSlice = kMaxSets * 1024;  // B fragments of one stage
 constexpr int kXoSlice = kMaxGps * 64;        // {xoff, xsum} x 8 tokens of one stage
 constexpr int kXSlice = 8 * 512 * 2;          // the stage's columns of X, 8 tokens (2-bit: 512 columns)
-// A stage slot: codes | fragments | group sums | X columns.  Codes at the start
-// of a slot: 1024-byte aligned for the 128-byte swizzle.
-constexpr int kOffTable = kCodeTile;
-constexpr int kOffXo = kOffTable + kTableSlice;
-constexpr int kOffX = kOffXo + kXoSlice;
-// Fragment mode (the fragments come from k_gemv_xprep) has no X columns in a slot.
-template <bool BUILD>
-constexpr int kStageBytes = (kOffX + (BUILD ? kXSlice : 0) + 1023) / 1024 * 1024;
-constexpr int kStages = 6;
 constexpr int kSlots = 2;                  // s / zq staging slots per consumer warp
 constexpr uint64_t kWaitLimitNs = 4000000000ull;
-
-// Shared-memory layout (after 1024-byte alignment): the stage ring, then the
-// s / zq slots, then the barriers (full, empty, X-arrived per slot, abort flag).
-template <bool BUILD>
-constexpr int kOffSz = kStages * kStageBytes<BUILD>;
 constexpr int kSzBytes = kConsumers * kSlots * 16 * kMaxGps * 8;
-template <bool BUILD>
-constexpr int kOffBar = kOffSz<BUILD> + kSzBytes;
-template <bool BUILD>
-constexpr int kSmemBytes = 1024 + kOffBar<BUILD> + 256;
 
 // Codes of one lane for one 64-column set of a row: 16 codes (columns 16t..16t+15
 // of the set).  extract() produces eight bf16x2 registers; register e holds codes
@@ -163,9 +144,48 @@ struct Codes<3> {
 };
 
 // Codes per stage along K: one 128-byte row segment.
+// Code bytes of one row per stage: one 128-byte TMA box, or two for 3-bit codes
+// (stored one per byte), so that a stage still holds four 64-column sets.
+template <int BITS>
+constexpr int stage_row_bytes() {
+    return BITS == 3 ? 2 * kRowBytes : kRowBytes;
+}
+
 template <int BITS>
 constexpr int stage_codes() {
-    return kRowBytes * 8 / Codes<BITS>::kCodeBits;
+    return stage_row_bytes<BITS>() * 8 / Codes<BITS>::kCodeBits;
+}
+
+// A stage slot: codes (one 128-row x 128-byte swizzled tile per box) | fragments |
+// group sums | (build mode) X columns.  Codes at the start of a slot: 1024-byte
+// aligned for the 128-byte swizzle.  The ring has as many slots as fit in shared
+// memory next to the s / zq slots: six, or five / four for the wider 3-bit stage.
+template <int BITS>
+constexpr int kCodeTile = kRows * stage_row_bytes<BITS>();
+template <int BITS>
+constexpr int kOffTable = kCodeTile<BITS>;
+template <int BITS>
+constexpr int kOffXo = kOffTable<BITS> + kTableSlice;
+template <int BITS>
+constexpr int kOffX = kOffXo<BITS> + kXoSlice;
+template <int BITS, bool BUILD>
+constexpr int kStageBytes = (kOffX<BITS> + (BUILD ? kXSlice : 0) + 1023) / 1024 * 1024;
+template <int BITS, bool BUILD>
+constexpr int kStages = BITS == 3 ? (BUILD ? 4 : 5) : 6;
+// Shared-memory layout (after 1024-byte alignment): the stage ring, then the
+// s / zq slots, then the barriers (full, empty, X-arrived per slot, abort flag).
+template <int BITS, bool BUILD>
+constexpr int kOffSz = kStages<BITS, BUILD> * kStageBytes<BITS, BUILD>;
+template <int BITS, bool BUILD>
+constexpr int kOffBar = kOffSz<BITS, BUILD> + kSzBytes;
+template <int BITS, bool BUILD>
+constexpr int kSmemBytes = 1024 + kOffBar<BITS, BUILD> + 256;
+
+// Byte `byte` of row r of a stage's code tiles (box byte / 128, 128-byte swizzle).
+template <int BITS>
+__device__ __forceinline__ uint32_t code_offset(int r, int byte) {
+    return static_cast<uint32_t>((byte >> 7) * (kRows * kRowBytes) + r * kRowBytes +
+                                 ((((byte >> 4) & 7) ^ (r & 7)) << 4) + (byte & 15));
 }
 
 
@@ -246,9 +266,9 @@ __device__ __forceinline__ void build_stage(uint8_t *slot, int M, int kcols, int
     constexpr int MPC = 8 / SL;
     const int n = lane >> 2, t = lane & 3;
     const int sl = n / MPC, tok = n % MPC;
-    uint4 *table = reinterpret_cast<uint4 *>(slot + kOffTable);
-    float2 *xo = reinterpret_cast<float2 *>(slot + kOffXo);
-    const uint4 *xs = reinterpret_cast<const uint4 *>(slot + kOffX);  // [token][KS] bf16
+    uint4 *table = reinterpret_cast<uint4 *>(slot + kOffTable<BITS>);
+    float2 *xo = reinterpret_cast<float2 *>(slot + kOffXo<BITS>);
+    const uint4 *xs = reinterpret_cast<const uint4 *>(slot + kOffX<BITS>);  // [token][KS] bf16
 #pragma unroll
     for (int i = 0; i < GPS / SL; ++i) {
         const int gs = sl + SL * i;
@@ -501,14 +521,9 @@ __device__ __forceinline__ void mma_bf16_z(float (&d)[4], uint32_t a0, uint32_t 
         : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1), "f"(0.0f));
 }
 
-// Byte b of row r of a 128-byte-swizzled code tile.
-__device__ __forceinline__ uint32_t swz(int r, int b) {
-    return static_cast<uint32_t>(r * kRowBytes + ((((b >> 4) ^ (r & 7))) << 4) + (b & 15));
-}
-
 template <int BITS>
 __device__ __forceinline__ void load_codes(const uint8_t *tile, int row, int byte, uint32_t *w) {
-    const uint8_t *ptr = tile + swz(row, byte);
+    const uint8_t *ptr = tile + code_offset<BITS>(row, byte);
     if (Codes<BITS>::kBytes == 4) {
         w[0] = *reinterpret_cast<const uint32_t *>(ptr);
     } else if (Codes<BITS>::kBytes == 8) {
@@ -542,22 +557,32 @@ __global__ void __launch_bounds__(kThreads, 1)
     // aligned by an offset from the array itself, so that every pointer below
     // stays in the shared window (shared loads, 32-bit addresses)
     uint8_t *smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
-    constexpr int kSlot = kStageBytes<BUILD>;
-    float2 *sz = reinterpret_cast<float2 *>(smem + kOffSz<BUILD>);
+    constexpr int NST = kStages<BITS, BUILD>;
+    constexpr int kSlot = kStageBytes<BITS, BUILD>;
+    constexpr int kCT = kCodeTile<BITS>;
+    constexpr int oTable = kOffTable<BITS>, oXo = kOffXo<BITS>, oX = kOffX<BITS>;
+    float2 *sz = reinterpret_cast<float2 *>(smem + kOffSz<BITS, BUILD>);
     // Build mode: full[s] = the slot's fragments are built (the producer warp's 32
     // lanes), xfull[s] = its code tile and X columns have landed (transaction
     // bytes).  Fragment mode: full[s] = the code tile, fragments and sums have
     // landed (transaction bytes); xfull is unused.  empty[s]: the consumers are
     // done with the slot.
-    uint64_t *full = reinterpret_cast<uint64_t *>(smem + kOffBar<BUILD>);
-    uint64_t *empty = full + kStages;
-    uint64_t *xfull = empty + kStages;
-    volatile int *abort_flag = reinterpret_cast<volatile int *>(xfull + kStages);
+    uint64_t *full = reinterpret_cast<uint64_t *>(smem + kOffBar<BITS, BUILD>);
+    uint64_t *empty = full + NST;
+    uint64_t *xfull = empty + NST;
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(xfull + NST);
+    // the code tile of stage (ks, rt): one TMA box per 128 bytes of each row
+    auto load_code_tile = [&](uint8_t *dst, uint64_t *bar, int ks, int rt) {
+#pragma unroll
+        for (int bx = 0; bx < stage_row_bytes<BITS>() / kRowBytes; ++bx)
+            tma_load_2d(dst + bx * (kRows * kRowBytes), &tm_codes, bar, ks * stage_row_bytes<BITS>() + bx * kRowBytes,
+                        rt * kRows);
+    };
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
 
     if (threadIdx.x == 0) {
-        for (int i = 0; i < kStages; ++i) {
+        for (int i = 0; i < NST; ++i) {
             mbar_init(&full[i], BUILD ? 32 : 1);
             mbar_init(&empty[i], kConsumers);
             mbar_init(&xfull[i], 1);
@@ -569,8 +594,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     if constexpr (BUILD) {
         // fragment entries that no stage writes (other slots, tokens beyond M) are zero
-        for (int s = 0; s < kStages; ++s) {
-            uint4 *z = reinterpret_cast<uint4 *>(smem + s * kSlot + kOffTable);
+        for (int s = 0; s < NST; ++s) {
+            uint4 *z = reinterpret_cast<uint4 *>(smem + s * kSlot + oTable);
             for (int i = threadIdx.x; i < (kTableSlice + kXoSlice) / 16; i += kThreads)
                 z[i] = make_uint4(0u, 0u, 0u, 0u);
         }
@@ -599,41 +624,41 @@ __global__ void __launch_bounds__(kThreads, 1)
                 StageCursor c;
                 c.init(x_begin, p.spr);
                 constexpr uint32_t kFragBytes = SETS * 1024 + GPS * 64;
-                const int pre = static_cast<int>(x_end - x_begin < kStages ? x_end - x_begin : kStages);
+                const int pre = static_cast<int>(x_end - x_begin < NST ? x_end - x_begin : NST);
                 {
                     StageCursor cp = c;
                     for (int i = 0; i < pre; ++i, cp.next(p.spr)) {
-                        mbar_arrive_expect_tx(&full[i], kCodeTile + kFragBytes);
-                        tma_load_2d(smem + i * kSlot, &tm_codes, &full[i], cp.ks * kRowBytes, cp.rt * kRows);
+                        mbar_arrive_expect_tx(&full[i], kCT + kFragBytes);
+                        load_code_tile(smem + i * kSlot, &full[i], cp.ks, cp.rt);
                     }
                     armed = (1u << pre) - 1u;  // parity 0
                 }
                 pdl_wait();
                 for (; static_cast<int>(it) < pre; c.next(p.spr), ++it) {
                     uint8_t *stage = smem + it * kSlot;
-                    bulk_load(stage + kOffTable, p.table + static_cast<int64_t>(c.ks) * SETS * 64, SETS * 1024,
+                    bulk_load(stage + oTable, p.table + static_cast<int64_t>(c.ks) * SETS * 64, SETS * 1024,
                               &full[it]);
-                    bulk_load(stage + kOffXo, p.xso + static_cast<int64_t>(c.ks) * GPS * 8, GPS * 64, &full[it]);
+                    bulk_load(stage + oXo, p.xso + static_cast<int64_t>(c.ks) * GPS * 8, GPS * 64, &full[it]);
                 }
                 for (; c.x < x_end; c.next(p.spr), ++it) {
-                    const int st = it % kStages;
-                    const uint32_t ph = (it / kStages) & 1u;
+                    const int st = it % NST;
+                    const uint32_t ph = (it / NST) & 1u;
                     if (!mbar_wait_bounded(&empty[st], ph ^ 1u, abort_flag, p.err, p.wait_limit_ns)) {
                         ok = false;
                         break;
                     }
                     uint8_t *stage = smem + st * kSlot;
-                    mbar_arrive_expect_tx(&full[st], kCodeTile + kFragBytes);
+                    mbar_arrive_expect_tx(&full[st], kCT + kFragBytes);
                     armed |= 1u << st;
                     armed_parity = (armed_parity & ~(1u << st)) | (ph << st);
-                    tma_load_2d(stage, &tm_codes, &full[st], c.ks * kRowBytes, c.rt * kRows);
-                    bulk_load(stage + kOffTable, p.table + static_cast<int64_t>(c.ks) * SETS * 64, SETS * 1024,
+                    load_code_tile(stage, &full[st], c.ks, c.rt);
+                    bulk_load(stage + oTable, p.table + static_cast<int64_t>(c.ks) * SETS * 64, SETS * 1024,
                               &full[st]);
-                    bulk_load(stage + kOffXo, p.xso + static_cast<int64_t>(c.ks) * GPS * 8, GPS * 64, &full[st]);
+                    bulk_load(stage + oXo, p.xso + static_cast<int64_t>(c.ks) * GPS * 8, GPS * 64, &full[st]);
                 }
                 if (!ok) {
                     // let issued copies land before the block can exit
-                    for (int st = 0; st < kStages; ++st)
+                    for (int st = 0; st < NST; ++st)
                         if (armed & (1u << st)) {
                             const uint32_t a = smem_u32(&full[st]);
                             const uint64_t t0 = globaltimer_ns();
@@ -650,7 +675,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         // columns of X (one bulk copy per token) on xfull[s].  kLag stages behind,
         // the whole warp turns those columns into the stage's fragments and group
         // sums and arrives on full[s].  In the steady state the consumers are
-        // kStages - 1 stages behind the requests, so each stage is built well
+        // NST - 1 stages behind the requests, so each stage is built well
         // before its use.
         uint32_t armed = 0, armed_parity = 0;
         bool ok = true;
@@ -661,28 +686,28 @@ __global__ void __launch_bounds__(kThreads, 1)
         constexpr int kLag = 2;
         for (int64_t i = 0; i < n + kLag; ++i) {
             if (i < n) {
-                const int st = static_cast<int>(i % kStages);
-                const uint32_t ph = static_cast<uint32_t>(i / kStages) & 1u;
+                const int st = static_cast<int>(i % NST);
+                const uint32_t ph = static_cast<uint32_t>(i / NST) & 1u;
                 ok = mbar_wait_bounded(&empty[st], ph ^ 1u, abort_flag, p.err, p.wait_limit_ns) && ok;
                 if (!__all_sync(0xffffffffu, ok)) break;
                 if (lane == 0) {
                     const int64_t k0 = static_cast<int64_t>(ci.ks) * KS;
                     const uint32_t xbytes = static_cast<uint32_t>((p.K - k0 < KS ? p.K - k0 : KS) * 2);
                     uint8_t *stage = smem + st * kSlot;
-                    mbar_arrive_expect_tx(&xfull[st], kCodeTile + p.M * xbytes);
+                    mbar_arrive_expect_tx(&xfull[st], kCT + p.M * xbytes);
                     armed |= 1u << st;
                     armed_parity = (armed_parity & ~(1u << st)) | (ph << st);
-                    tma_load_2d(stage, &tm_codes, &xfull[st], ci.ks * kRowBytes, ci.rt * kRows);
+                    load_code_tile(stage, &xfull[st], ci.ks, ci.rt);
                     for (int tok = 0; tok < p.M; ++tok)
-                        bulk_load(stage + kOffX + tok * KS * 2, p.X + tok * p.K + k0, xbytes, &xfull[st]);
+                        bulk_load(stage + oX + tok * KS * 2, p.X + tok * p.K + k0, xbytes, &xfull[st]);
                 }
                 __syncwarp();
                 ci.next(p.spr);
             }
             if (i >= kLag) {
                 const int64_t b = i - kLag;
-                const int st = static_cast<int>(b % kStages);
-                const uint32_t ph = static_cast<uint32_t>(b / kStages) & 1u;
+                const int st = static_cast<int>(b % NST);
+                const uint32_t ph = static_cast<uint32_t>(b / NST) & 1u;
                 ok = mbar_wait_bounded(&xfull[st], ph, abort_flag, p.err, p.wait_limit_ns) && ok;
                 if (!__all_sync(0xffffffffu, ok)) break;
                 const int64_t k0 = static_cast<int64_t>(cb.ks) * KS;
@@ -694,7 +719,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         if (!ok && lane == 0) {
             // let issued copies land before the block can exit
-            for (int st = 0; st < kStages; ++st)
+            for (int st = 0; st < NST; ++st)
                 if (armed & (1u << st)) {
                     const uint32_t a = smem_u32(&xfull[st]);
                     const uint64_t t0 = globaltimer_ns();
@@ -739,15 +764,15 @@ __global__ void __launch_bounds__(kThreads, 1)
     auto stage = [&](SzRegs &load_into, const SzRegs &store_from) {
         load_sz<BITS, GROUP, S16>(p, pf, x_end, warp * 16, lane, load_into);
         pf.next(p.spr);
-        const int st = it % kStages;
-        const uint32_t ph = (it / kStages) & 1u;
+        const int st = it % NST;
+        const uint32_t ph = (it / NST) & 1u;
         // build mode: the code tile (written by TMA), then the fragments (by the
         // producer warp); fragment mode: all of it by copies on full[st]
         if constexpr (BUILD) ok = mbar_wait_bounded(&xfull[st], ph, abort_flag, p.err, p.wait_limit_ns) && ok;
         ok = mbar_wait_bounded(&full[st], ph, abort_flag, p.err, p.wait_limit_ns) && ok;
         const uint8_t *tile = smem + st * kSlot;
-        const uint4 *table = reinterpret_cast<const uint4 *>(tile + kOffTable);
-        const float2 *xo = reinterpret_cast<const float2 *>(tile + kOffXo);
+        const uint4 *table = reinterpret_cast<const uint4 *>(tile + oTable);
+        const float2 *xo = reinterpret_cast<const float2 *>(tile + oXo);
         const float2 *szs = szw + (it % kSlots) * (16 * kMaxGps);
         // Runs of SL groups: the four mmas of a set go to four accumulator chains,
         // and the run's groups share them (each in its own columns).
@@ -938,11 +963,12 @@ cudaError_t launch_main(const CUtensorMap &map, const GemvParams &p, int grid, i
     static std::atomic<uint64_t> done{0};
     const uint64_t bit = 1ull << (dev_id & 63);
     if (!(done.load() & bit)) {
-        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes<BUILD>);
+        cudaError_t e =
+            cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes<BITS, BUILD>);
         if (e != cudaSuccess) return e;
         done.fetch_or(bit);
     }
-    return launch_pdl(kern, dim3(grid), dim3(kThreads), kSmemBytes<BUILD>, st, map, p);
+    return launch_pdl(kern, dim3(grid), dim3(kThreads), kSmemBytes<BITS, BUILD>, st, map, p);
 }
 
 template <int BITS, int GROUP, bool S16>

@@ -144,11 +144,12 @@ struct Codes<3> {
 };
 
 // Codes per stage along K: one 128-byte row segment.
-// Code bytes of one row per stage: one 128-byte TMA box, or two for 3-bit codes
-// (stored one per byte), so that a stage still holds four 64-column sets.
+// Code bytes of one row per stage: one 128-byte TMA box for 2-bit codes (eight
+// 64-column sets), two for 4-bit codes and for 3-bit codes (stored one per byte),
+// so that a stage holds eight or four sets and its fixed cost is shared.
 template <int BITS>
 constexpr int stage_row_bytes() {
-    return BITS == 3 ? 2 * kRowBytes : kRowBytes;
+    return BITS == 2 ? kRowBytes : 2 * kRowBytes;
 }
 
 template <int BITS>
@@ -159,7 +160,7 @@ constexpr int stage_codes() {
 // A stage slot: codes (one 128-row x 128-byte swizzled tile per box) | fragments |
 // group sums | (build mode) X columns.  Codes at the start of a slot: 1024-byte
 // aligned for the 128-byte swizzle.  The ring has as many slots as fit in shared
-// memory next to the s / zq slots: six, or five / four for the wider 3-bit stage.
+// memory next to the s / zq slots: six, or five / four for the two-tile stages.
 template <int BITS>
 constexpr int kCodeTile = kRows * stage_row_bytes<BITS>();
 template <int BITS>
@@ -171,7 +172,7 @@ constexpr int kOffX = kOffXo<BITS> + kXoSlice;
 template <int BITS, bool BUILD>
 constexpr int kStageBytes = (kOffX<BITS> + (BUILD ? kXSlice : 0) + 1023) / 1024 * 1024;
 template <int BITS, bool BUILD>
-constexpr int kStages = BITS == 3 ? (BUILD ? 4 : 5) : 6;
+constexpr int kStages = BITS == 2 ? 6 : (BUILD ? 4 : 5);
 // Shared-memory layout (after 1024-byte alignment): the stage ring, then the
 // s / zq slots, then the barriers (full, empty, X-arrived per slot, abort flag).
 template <int BITS, bool BUILD>

@@ -602,22 +602,26 @@ def blockap_block(dev, peaks, steps=5):
 
 
 def decode_gemv(dev, peaks, budget_bytes=300_000_000):
-    """Batch-1 inference on frozen 2-bit codes (eqat_dq_linear_fwd at M = 1, the
-    decode-size path), against a bf16 matvec (torch.matmul) of the same shape.
+    """Batch-1 inference on frozen 2-, 3- and 4-bit codes (eqat_dq_linear_fwd at
+    M = 1, the decode-size path), against a bf16 matvec (torch.matmul) of the same
+    shape.
     Back-to-back calls over enough distinct layers that their bytes exceed L2,
     captured in a CUDA graph so that host launch cost is excluded; CUDA events
     around three replays.  GB/s = algorithmic bytes (codes + s + zq + X + Y) /
     time per call."""
     out = {}
     side = torch.cuda.Stream(device=dev)
-    for name, N, K in (("llama2-70b-gate_proj", 28672, 8192), ("llama2-7b-q_proj", 4096, 4096)):
-        b, g, M = 2, 64, 1
+    for name, N, K, b, g in (("llama2-70b-gate_proj", 28672, 8192, 2, 64), ("llama2-7b-q_proj", 4096, 4096, 2, 64),
+                             ("llama2-7b-mlp-gate_proj-w3g128", 11008, 4096, 3, 128),
+                             ("llama2-70b-gate_proj-w4g64", 28672, 8192, 4, 64)):
+        M = 1
         G = K // g
-        per = N * K * b // 8 + N * G * 5
+        cb = K * b // 8 if b != 3 else K  # code bytes per row (3-bit: one code per byte)
+        per = N * cb + N * G * 5
         L = max(2, -(-budget_bytes // per))
         gen = torch.Generator(device=dev)
         gen.manual_seed(2000 + N)
-        layers = [(torch.randint(0, 256, (N, K * b // 8), generator=gen, device=dev, dtype=torch.uint8),
+        layers = [(torch.randint(0, 256 if b != 3 else 8, (N, cb), generator=gen, device=dev, dtype=torch.uint8),
                    torch.randint(0, 1 << b, (N, G), generator=gen, device=dev, dtype=torch.uint8),
                    torch.rand(N, G, generator=gen, device=dev) * 0.01 + 1e-3) for _ in range(L)]
         X = torch.randn(M, K, generator=gen, device=dev).to(torch.bfloat16)

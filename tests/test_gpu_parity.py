@@ -101,12 +101,41 @@ def test_fake_quant_and_pack_bit_exact(orc, dtype, trained, bits, g):
         assert_bits_equal(to_np(dq), dq_ref if odt == torch.float32 else bf16_round(dq_ref), "dequant")
 
 
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+@pytest.mark.parametrize("N,K,bits,g", [(8, 96, 2, 32), (8, 640, 3, 128), (40, 1152, 4, 64), (40, 1184, 2, 32),
+                                        (72, 4160, 2, 64)])
+def test_quantizer_ragged_tiles_bit_exact(orc, dtype, N, K, bits, g):
+    """Prepass, pack and dequant where the weight count is not a whole number of the
+    kernels' tiles (and one layer below a single tile), in both quantizer states."""
+    for trained in (False, True):
+        d = synthetic.draw_linear(np.random.default_rng(N * K + bits), 1, N, K, 0.02, dtype)
+        Wn = synthetic.as_f32_numpy(d["W"])
+        s, z = orc.minmax_init(Wn, bits, g)
+        if trained:
+            s, z = synthetic.perturb_quant_params(s, z, N + K)
+        W, sd, zd = d["W"].cuda(), torch.from_numpy(s).cuda(), torch.from_numpy(z).cuda()
+        wh_ref, c_ref, m_ref, _ = orc.fake_quant(Wn, s, z, bits, g)
+        wh, c, m = eqat.fake_quant(W, sd, zd, bits, g)
+        assert_bits_equal(to_np(c), c_ref, "code")
+        assert_bits_equal(to_np(m), m_ref, "mask")
+        assert_bits_equal(to_np(wh), wh_ref if dtype == "f32" else bf16_round(wh_ref), "W_hat")
+        wh_only, _, _ = eqat.fake_quant(W, sd, zd, bits, g, want_code=False, want_mask=False)
+        assert_bits_equal(to_np(wh_only), to_np(wh), "W_hat without codes")
+        p_ref, zq_ref = orc.pack(Wn, s, z, bits, g)
+        p, zq = eqat.pack_codes(W, sd, zd, bits, g)
+        assert_bits_equal(to_np(p), p_ref, "packed codes")
+        assert_bits_equal(to_np(zq), zq_ref, "zq")
+        dq = eqat.dequant_codes(p, zq, sd, K, bits, g, torch.float32)
+        assert_bits_equal(to_np(dq), orc.dequant_packed(p_ref, zq_ref, s, K, bits, g), "dequant")
+
+
 @pytest.mark.parametrize("dtype", ["f32", "bf16"])
 @pytest.mark.parametrize("bits", [2, 3, 4])
 def test_codes_at_and_around_rounding_boundaries_bit_exact(orc, dtype, bits):
     """Weights on, and one or two ulps either side of, half-integer multiples of s:
     the cases where the kernels' reciprocal-multiply decision must hand over to the
-    IEEE division to reproduce round(W/s)."""
+    exact one (a residual test against the half-integer, the IEEE division where that
+    cannot decide) to reproduce round(W/s)."""
     Q = (1 << bits) - 1
     rng = np.random.default_rng(4321 + bits)
     N, K, g = 64, 512, 32

@@ -38,10 +38,6 @@ __device__ __forceinline__ float round_quotient(float w, float s, float rcp, flo
     return r;
 }
 
-// round_quotient for N weights of one group with a single branch: the fast
-// decisions for all N first, then, only if one of them lies within the bound of a
-// rounding boundary, the IEEE division for those.  r[j] = round(RN(w[j]/s)); u[j]
-// as in round_quotient.
 // Round-half-to-even with two full-rate additions: for |x| < 2^22,
 // RN(RN(x + 1.5 * 2^23) - 1.5 * 2^23) == rint(x), because x + 1.5 * 2^23 lies in
 // [2^23, 2^24) where the spacing of fp32 is 1.  (For larger |x| the callers'
@@ -51,39 +47,10 @@ constexpr float kRoundMagic = 12582912.0f;  // 1.5 * 2^23
 
 __device__ __forceinline__ float rint_small(float x) { return __fsub_rn(__fadd_rn(x, kRoundMagic), kRoundMagic); }
 
-// A clamped code c in [0, 255] as an integer: the low mantissa bits of c + 1.5 * 2^23.
-__device__ __forceinline__ uint32_t code_bits(float c) {
-    return static_cast<uint32_t>(__float_as_int(__fadd_rn(c, kRoundMagic))) & 0xFFu;
-}
-
-// Fast decision for one weight in the magic domain: with t = RN(u + M), M =
-// 1.5 * 2^23, t = M + round(u) exactly (|u| < 2^22), so t + zr = M + round(u) + zr
-// exactly and a clamp of t + zr to [M, M + Q] gives M + code.  Returns t + zr
-// (unclamped, for the mask) and sets `near` when u lies within the error bound of
-// a rounding boundary (the caller then takes the exact path for this weight).
-__device__ __forceinline__ float magic_decision(float w, float rcp, float zr, bool &near) {
-    const float u = __fmul_rn(w, rcp);
-    const float t = __fadd_rn(u, kRoundMagic);
-    near |= fabsf(__fsub_rn(u, __fsub_rn(t, kRoundMagic))) >= __fmaf_rn(fabsf(u), -0x1p-21f, 0.5f);
-    return __fadd_rn(t, zr);
-}
-
-// The same decision by the IEEE division (the rare exact path), as M + code:
-// returns M + round(RN(w/s)) + zr for the in-range test and clamps for the code.
-__device__ __forceinline__ float exact_decision(float w, float s, float zr, float Q, bool &inside) {
-    const float q = __fadd_rn(rintf(__fdiv_rn(w, s)), zr);
-    inside = (q >= 0.0f) && (q <= Q);
-    return __fadd_rn(fminf(fmaxf(q, 0.0f), Q), kRoundMagic);
-}
-
-// sum_k bits(M) << (step * k) for k < count, modulo 2^32: what the raw bits of
-// M + code contribute to a packed word beyond the codes themselves.
-__host__ __device__ constexpr uint32_t magic_word(int step, int count) {
-    uint32_t acc = 0;
-    for (int k = 0; k < count; ++k) acc += 0x4B400000u << (step * k);
-    return acc;
-}
-
+// round_quotient for N weights of one group with a single branch: the fast
+// decisions for all N first, then, only if one of them lies within the bound of a
+// rounding boundary, the IEEE division for those.  r[j] = round(RN(w[j]/s)); u[j]
+// as in round_quotient.
 template <int N>
 __device__ __forceinline__ void round_quotients(const float (&w)[N], float s, float rcp, float (&r)[N],
                                                 float (&u)[N]) {
@@ -114,10 +81,6 @@ __device__ __forceinline__ QuantElem quant_elem(float w, float s, float rcp, flo
     e.inside = (q >= 0.0f) && (q <= Q);
     e.c = fminf(fmaxf(q, 0.0f), Q);
     return e;
-}
-
-__device__ __forceinline__ float dequant_elem(float c, float zr, float s) {
-    return __fmul_rn(__fsub_rn(c, zr), s);
 }
 
 // Min-max init of one group (modelfoundations note, Phase 1).

@@ -2,11 +2,12 @@
 // prepass (codes, mask, W-hat), packing to low-bit integers and the E2E-QP
 // dequantization of frozen codes.
 //
-// Every kernel streams its input once with 16-byte loads; a group (g in
-// {32, 64, 128} consecutive in-features of one row) is never split across
-// warps, so per-group reductions are warp shuffles and per-group parameters are
-// read once per thread from L1.  Grids are grid-stride loops sized to a whole
-// number of waves of the SMs.
+// Every kernel streams its input once with coalesced 16-byte loads and keeps a
+// group (g in {32, 64, 128} consecutive in-features of one row) inside one warp:
+// init reduces a group with warp shuffles; the prepass and pack form each group's
+// constants once per warp tile in shared memory and decide two weights per
+// packed-fp32 instruction.  Grids are sized to the resident CTAs of the SMs and
+// loop over the work.
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
@@ -98,93 +99,7 @@ __global__ void __launch_bounds__(kThreads, 4) k_minmax_init(const T *__restrict
     }
 }
 
-// ------------------------------------------------------------------ fake-quant prepass
-// A thread handles U = 2 chunks of 8 consecutive weights (each chunk inside one
-// group) per iteration and issues both loads before any arithmetic.
-template <typename T, typename O, bool CODES>
-__device__ __forceinline__ void fake_quant_chunk(const float (&w)[8], float sc, float zr, float Q,
-                                                 int64_t e0, O *__restrict__ W_hat,
-                                                 uint8_t *__restrict__ code, uint8_t *__restrict__ mask) {
-    const float rcp = __frcp_rn(sc);
-    const float lo = kRoundMagic, hi = __fadd_rn(kRoundMagic, Q);
-    const float mz = __fadd_rn(kRoundMagic, zr);  // W-hat = (M + code - (M + zr)) s
-    float qm[8];
-    bool inside[8];
-    bool near = false;
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-        const float t = magic_decision(w[j], rcp, zr, near);  // M + round(u) + zr
-        inside[j] = (t >= lo) && (t <= hi);
-        qm[j] = fminf(fmaxf(t, lo), hi);
-    }
-    if (near) {
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-            bool nj = false;
-            (void)magic_decision(w[j], rcp, zr, nj);
-            if (nj) qm[j] = exact_decision(w[j], sc, zr, Q, inside[j]);
-        }
-    }
-    float wh[8];
-#pragma unroll
-    for (int j = 0; j < 8; ++j) wh[j] = __fmul_rn(__fsub_rn(qm[j], mz), sc);
-    if (W_hat) store8<O>(W_hat + e0, wh);
-    if (CODES) {
-        uint32_t c_lo = 0, c_hi = 0, m_lo = 0, m_hi = 0;
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-            const uint32_t cb = static_cast<uint32_t>(__float_as_int(qm[j])) & 0xFFu;
-            const uint32_t mb = inside[j] ? 1u : 0u;
-            if (j < 4) {
-                c_lo |= cb << (8 * j);
-                m_lo |= mb << (8 * j);
-            } else {
-                c_hi |= cb << (8 * (j - 4));
-                m_hi |= mb << (8 * (j - 4));
-            }
-        }
-        if (code) *reinterpret_cast<uint2 *>(code + e0) = make_uint2(c_lo, c_hi);
-        if (mask) *reinterpret_cast<uint2 *>(mask + e0) = make_uint2(m_lo, m_hi);
-    }
-}
-
-template <typename T, typename O, bool CODES>
-__global__ void __launch_bounds__(kThreads, 4)
-    k_fake_quant(const T *__restrict__ W, const float *__restrict__ s, const float *__restrict__ z,
-                 int64_t n_chunks, int gshift, float Q, O *__restrict__ W_hat,
-                 uint8_t *__restrict__ code, uint8_t *__restrict__ mask) {
-    constexpr int U = 2;
-    const int64_t nthreads = static_cast<int64_t>(gridDim.x) * kThreads;
-    for (int64_t base = static_cast<int64_t>(blockIdx.x) * kThreads + threadIdx.x; base < n_chunks;
-         base += nthreads * U) {
-        Raw8<T> raw[U];
-        float sc[U], zr[U];
-#pragma unroll
-        for (int u = 0; u < U; ++u) {
-            const int64_t i = base + u * nthreads;
-            if (i < n_chunks) {
-                raw[u] = load_raw8<T>(W + i * 8);
-                const int64_t g = (i * 8) >> gshift;
-                sc[u] = __ldg(s + g);
-                zr[u] = rintf(__ldg(z + g));
-            }
-        }
-#pragma unroll
-        for (int u = 0; u < U; ++u) {
-            const int64_t i = base + u * nthreads;
-            if (i < n_chunks) {
-                float w[8];
-                unpack8(raw[u], w);
-                fake_quant_chunk<T, O, CODES>(w, sc[u], zr[u], Q, i * 8, W_hat, code, mask);
-            }
-        }
-    }
-}
-
-// ------------------------------------------------------------------ pack
-// One thread per 16 consecutive weights (same group).  zq = clamp(round(z), 0, Q)
-// and the codes use zr := zq (z hard-rounded at pack time).  Output per thread:
-// 4 bytes (2-bit), 8 bytes (4-bit) or 16 bytes (3-bit, one code per byte).
+// ------------------------------------------------------------------ packed fp32 pairs
 // Two fp32 lanes in one 64-bit register, and the packed-pair arithmetic of
 // sm_100 (each lane an IEEE round-to-nearest operation, as the scalar forms).
 __device__ __forceinline__ uint64_t f2_pack(float a, float b) {
@@ -211,129 +126,395 @@ __device__ __forceinline__ uint64_t f2_sub(uint64_t a, uint64_t b) {
     return d;
 }
 
-template <int BITS>
-__device__ __forceinline__ void pack_chunk(const float (&w)[16], float sc, float zr, float Q, int64_t e0,
-                                           uint8_t *__restrict__ codes) {
-    const float rcp = __frcp_rn(sc);
-    const float lo = kRoundMagic, hi = __fadd_rn(kRoundMagic, Q);
-    // M + zr is exact; one add of it gives M + zr + round(u) for every u that is
-    // not an exact tie (ties may break toward an odd total, but a tie lies in the
-    // near band below and takes the exact path).
-    const float mz = __fadd_rn(kRoundMagic, zr);
-    const uint64_t rcp2 = f2_pack(rcp, rcp), mz2 = f2_pack(mz, mz);
-    // Each code enters its word as the raw bits of M + code (one multiply-add);
-    // the bits of M are taken out once per word at the end.
-    uint32_t word[4] = {0u, 0u, 0u, 0u};  // 2-bit: word[0]; 4-bit: word[0..1]; 3-bit: word[0..3]
-#pragma unroll
-    for (int h = 0; h < 2; ++h) {
-        float cm[8];
-        bool near = false;
-        // two weights per step: u = RN(w rcp), t = RN(u + M + zr), and the
-        // distance u - (t - M - zr) of u from its rounded value
-#pragma unroll
-        for (int j = 0; j < 8; j += 2) {
-            const uint64_t u2 = f2_mul(f2_pack(w[8 * h + j], w[8 * h + j + 1]), rcp2);
-            const uint64_t t2 = f2_add(u2, mz2);
-            const uint64_t r2 = f2_sub(u2, f2_sub(t2, mz2));
-            float t0, t1, r0, r1;
-            f2_unpack(t2, t0, t1);
-            f2_unpack(r2, r0, r1);
-            // |u - RN(w / s)| < |u| 2^-22: only a u within that of a half-integer can
-            // round differently.  A code that is not clamped has |u| <= Q + zr + 1/2 < 64,
-            // so a band of 2^-16 covers it; a clamped code does not depend on it.
-            near |= fabsf(r0) >= 0.5f - 0x1p-16f;
-            near |= fabsf(r1) >= 0.5f - 0x1p-16f;
-            cm[j] = fminf(fmaxf(t0, lo), hi);
-            cm[j + 1] = fminf(fmaxf(t1, lo), hi);
-        }
-        if (near) {
-#pragma unroll
-            for (int j = 0; j < 8; ++j) {
-                bool nj = false, inside;
-                (void)magic_decision(w[8 * h + j], rcp, zr, nj);
-                if (nj) cm[j] = exact_decision(w[8 * h + j], sc, zr, Q, inside);
-            }
-        }
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-            const uint32_t b = static_cast<uint32_t>(__float_as_int(cm[j]));
-            const int k = 8 * h + j;
-            if (BITS == 2) word[0] += b << (2 * k);
-            else if (BITS == 4) word[k / 8] += b << (4 * (k % 8));
-            else word[k / 4] += b << (8 * (k % 4));
+// Two fp32 values to one f16x2 word (round to nearest; hi in the upper half), and
+// the per-half min / max of f16x2 words.
+__device__ __forceinline__ uint32_t h2_from_f32(float lo, float hi) {
+    uint32_t d;
+    asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(d) : "f"(hi), "f"(lo));
+    return d;
+}
+__device__ __forceinline__ uint32_t h2_clamp(uint32_t a, uint32_t lo, uint32_t hi) {
+    uint32_t d;
+    asm("max.f16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(lo));
+    asm("min.f16x2 %0, %1, %2;" : "=r"(d) : "r"(d), "r"(hi));
+    return d;
+}
+
+// ------------------------------------------------------------------ warp tiles of groups
+// The fake-quant prepass and pack walk the weights in warp tiles of whole groups.
+// A warp first issues the loads of its tile (16-byte loads; lane l takes the
+// 16-weight chunks l, l + 32, ..., so every load instruction is coalesced), then
+// forms the constants of each group of the tile once, one lane per group (s,
+// RN(1/s), zr and the near band), in its own slice of shared memory, and then
+// decides every weight from them.  Warps never wait for one another.
+//
+// A chunk with a weight near a rounding boundary (with min-max init steps, ties of
+// W/s are common: bf16 weights and their group's range) is queued and redone
+// later with the weights reloaded, 32 chunks at a time, so that the exact
+// decisions run on full warps instead of holding up every lane of a warp for one.
+constexpr int kTileThreads = 256;
+constexpr int kTileWarps = kTileThreads / 32;
+constexpr int kTileBlocksPerSm = 3;
+template <typename T>
+constexpr int kChunksPerLane = sizeof(T) == 2 ? 4 : 2;  // 128 bytes of loads in flight per lane
+template <typename T>
+constexpr int kWarpTile = 32 * kChunksPerLane<T> * 16;  // weights; a multiple of every group size
+template <typename T>
+constexpr int kWarpGroups = kWarpTile<T> / 32;  // groups of a tile at most (g = 32)
+template <typename T>
+constexpr int kLaneGroups = (kWarpGroups<T> + 31) / 32;
+
+struct GroupConst {
+    float sc, rcp, zr, band;  // s, RN(1/s), zr, near band (below)
+};
+
+// 16 consecutive elements as stored.
+template <typename T>
+struct Raw16 {
+    Raw8<T> a, b;
+};
+template <typename T>
+__device__ __forceinline__ Raw16<T> load_raw16(const T *p) {
+    return Raw16<T>{load_raw8<T>(p), load_raw8<T>(p + 8)};
+}
+template <typename T>
+__device__ __forceinline__ void unpack16(const Raw16<T> &r, float (&w)[16]) {
+    unpack8(r.a, *reinterpret_cast<float(*)[8]>(&w[0]));
+    unpack8(r.b, *reinterpret_cast<float(*)[8]>(&w[8]));
+}
+
+// Band around the half-integers inside which the fast decision of a weight is not
+// trusted, one per group: |RN(w RN(1/s)) - RN(w / s)| < |u| 2^-22, and a weight
+// whose code is not clamped has |u| <= |zr| + Q + 1/2, so a band of half-width
+// (|zr| + Q + 1) 2^-21 (twice the bound) covers every such weight; a clamped code
+// (or mask) does not change when round(u) is off by one.  A group with |zr| near
+// 2^20 or beyond gets a band that takes every weight to the exact decision.
+__device__ __forceinline__ float near_band(float zr, float Q) {
+    return __fsub_rn(0.5f, __fmul_rn(__fadd_rn(__fadd_rn(fabsf(zr), Q), 1.0f), 0x1p-21f));
+}
+
+// Fast decisions for two weights at once: u = RN(w RN(1/s)) and v = RN(u + M + zr)
+// - (M + zr) = round(u), exact for |u| < 2^22 (beyond that the code is clamped
+// whatever v is), and r = u - v.  A tie of u has |r| = 1/2, inside every band.
+__device__ __forceinline__ void pair_decision(uint64_t w2, uint64_t rcp2, uint64_t mz2, uint64_t &u2, uint64_t &v2,
+                                              float &ra, float &rb) {
+    u2 = f2_mul(w2, rcp2);
+    v2 = f2_sub(f2_add(u2, mz2), mz2);
+    f2_unpack(f2_sub(u2, v2), ra, rb);
+}
+
+// round(RN(w / s)) for one weight, without the division in the usual case.  With
+// u = RN(w RN(1/s)), |w/s - u| < |u| 2^-22 < 2^-8 for |u| < 2^14:
+// - u at least 2^-7 from every half-integer: w/s and RN(w/s) round as u does;
+// - otherwise let h be that half-integer and e = fma(-h, s, w), the rounded
+//   w - h s (its sign is exact).  T = s sp / 2, with sp the spacing of fp32 next
+//   to h on the side of w/s (the side of e; half the spacing above |h| on the
+//   side toward zero when |h| = 1/2, a power of two), is a power-of-two multiple
+//   of s and exact.  RN is monotone and T representable, so |e| < T proves
+//   |w/s - h| < sp / 2: RN(w/s) = h, which rounds half to even; |e| > T proves
+//   RN(w/s) != h, on the side of e, which rounds to that side's integer.  The
+//   IEEE division decides what is left (|e| = T, a tiny s, a large u).
+__device__ __forceinline__ float exact_round(float w, float s, float u) {
+    if (fabsf(u) < 0x1p14f) {
+        const float v = rint_small(u);
+        const float r = __fsub_rn(u, v);
+        if (fabsf(r) < 0.5f - 0x1p-7f) return v;
+        const float h = __fadd_rn(v, copysignf(0.5f, r));
+        const float e = __fmaf_rn(-h, s, w);
+        const float p = __int_as_float((__float_as_int(h) & 0x7F800000) - (24 << 23));  // half the spacing above |h|
+        float T = __fmul_rn(s, p);
+        if (fabsf(h) == 0.5f && ((e > 0.0f) != (h > 0.0f))) T = __fmul_rn(0.5f, T);
+        if (T >= 0x1p-100f) {  // a normal T is the exact product
+            const float ae = fabsf(e);
+            if (ae < T) return rint_small(h);
+            if (ae > T) return e > 0.0f ? __fadd_rn(h, 0.5f) : __fsub_rn(h, 0.5f);
         }
     }
-    if (BITS == 2) {
-        *reinterpret_cast<uint32_t *>(codes + e0 / 4) = word[0] - magic_word(2, 16);
-    } else if (BITS == 4) {
-        *reinterpret_cast<uint2 *>(codes + e0 / 2) =
-            make_uint2(word[0] - magic_word(4, 8), word[1] - magic_word(4, 8));
-    } else {
-        constexpr uint32_t m = magic_word(8, 4);
-        *reinterpret_cast<uint4 *>(codes + e0) = make_uint4(word[0] - m, word[1] - m, word[2] - m, word[3] - m);
+    return __fadd_rn(rintf(__fdiv_rn(w, s)), 0.0f);  // round(-0.3) = +0, as the other branches give
+}
+
+// The constants of the groups of one warp tile: lane l takes groups l, l + 32.
+// With clamp_z (pack) zr = zq = clamp(round(z), 0, Q), written to zq here.
+template <typename T>
+__device__ __forceinline__ void tile_group_consts(const float *__restrict__ s, const float *__restrict__ z,
+                                                  int64_t e_tile, int64_t n, int gshift, float Q, bool clamp_z,
+                                                  int lane, GroupConst *gc, uint8_t *__restrict__ zq) {
+    const int gpt = kWarpTile<T> >> gshift;
+    const int64_t g0 = e_tile >> gshift, n_groups = n >> gshift;
+#pragma unroll
+    for (int k = 0; k < kLaneGroups<T>; ++k) {
+        const int gi = lane + 32 * k;
+        const int64_t g = g0 + gi;
+        if (gi < gpt && g < n_groups) {
+            const float sc = __ldg(s + g);
+            float zr = rintf(__ldg(z + g));
+            if (clamp_z) zr = fminf(fmaxf(zr, 0.0f), Q);
+            if (zq) zq[g] = static_cast<uint8_t>(zr);
+            gc[gi] = GroupConst{sc, __frcp_rn(sc), zr, near_band(zr, Q)};
+        }
     }
 }
 
-// A thread handles U = 2 chunks of 16 consecutive weights (each inside one group)
-// per iteration, loads first.  zq = clamp(round(z), 0, Q) and the codes use
-// zr := zq (z hard-rounded at pack time).  Output per chunk: 4 bytes (2-bit), 8
-// bytes (4-bit) or 16 bytes (3-bit, one code per byte).
-template <typename T, int BITS>
-__global__ void __launch_bounds__(kThreads, 4)
-    k_pack(const T *__restrict__ W, const float *__restrict__ s, const float *__restrict__ z,
-           int64_t n_chunks, int gshift, float Q, uint8_t *__restrict__ codes,
-           uint8_t *__restrict__ zq) {
-    constexpr int U = 2;
-    const int64_t nthreads = static_cast<int64_t>(gridDim.x) * kThreads;
-    for (int64_t base = static_cast<int64_t>(blockIdx.x) * kThreads + threadIdx.x; base < n_chunks;
-         base += nthreads * U) {
-        Raw8<T> raw[U][2];
-        float sc[U], zr[U];
+// A chunk left for the exact pass: where it starts and its group's constants.
+struct PendingChunk {
+    int64_t e0;
+    GroupConst c;
+};
+// Per warp: fewer than 32 entries wait between tiles, and a tile adds at most one
+// per chunk.
+template <typename T>
+constexpr int kQueue = 32 + 32 * kChunksPerLane<T>;
+
+// Walks the warp tiles: chunk(w, group constants, e0, exact) handles the 16
+// weights at e0 and returns true when the fast pass (exact = false) left one of
+// them near a rounding boundary.  Such chunks go to the warp's queue in shared
+// memory; every 32 of them are redone with exact = true, one per lane, with the
+// weights reloaded, and the rest at the end.
+template <typename T, bool CLAMP_Z, typename Chunk>
+__device__ __forceinline__ void walk_warp_tiles(const T *__restrict__ W, const float *__restrict__ s,
+                                                const float *__restrict__ z, int64_t n, int gshift, float Q,
+                                                uint8_t *__restrict__ zq, GroupConst *gc_all,
+                                                PendingChunk *queue_all, Chunk chunk) {
+    constexpr int CPL = kChunksPerLane<T>, WT = kWarpTile<T>;
+    const int lane = threadIdx.x & 31, wib = threadIdx.x >> 5;
+    GroupConst *gc = gc_all + wib * kWarpGroups<T>;
+    PendingChunk *queue = queue_all + wib * kQueue<T>;
+    int queued = 0;  // warp-uniform
+    const int64_t n_tiles = (n + WT - 1) / WT, stride = static_cast<int64_t>(gridDim.x) * kTileWarps;
+    for (int64_t tile = static_cast<int64_t>(blockIdx.x) * kTileWarps + wib; tile < n_tiles; tile += stride) {
+        const int64_t e_tile = tile * WT;
+        const bool last_tile = tile + stride >= n_tiles;
+        Raw16<T> raw[CPL];
 #pragma unroll
-        for (int u = 0; u < U; ++u) {
-            const int64_t i = base + u * nthreads;
-            if (i < n_chunks) {
-                raw[u][0] = load_raw8<T>(W + i * 16);
-                raw[u][1] = load_raw8<T>(W + i * 16 + 8);
-                const int64_t g = (i * 16) >> gshift;
-                sc[u] = __ldg(s + g);
-                zr[u] = fminf(fmaxf(rintf(__ldg(z + g)), 0.0f), Q);
-            }
+        for (int j = 0; j < CPL; ++j) {
+            const int64_t e0 = e_tile + (j * 32 + lane) * 16;
+            if (e0 < n) raw[j] = load_raw16<T>(W + e0);
         }
+        __syncwarp();  // the previous tile's reads of gc are done
+        tile_group_consts<T>(s, z, e_tile, n, gshift, Q, CLAMP_Z, lane, gc, zq);
+        __syncwarp();
 #pragma unroll
-        for (int u = 0; u < U; ++u) {
-            const int64_t i = base + u * nthreads;
-            if (i < n_chunks) {
-                const int64_t e0 = i * 16;
-                if ((e0 & ((int64_t(1) << gshift) - 1)) == 0) zq[e0 >> gshift] = static_cast<uint8_t>(zr[u]);
+        for (int j = 0; j < CPL; ++j) {
+            const int off = (j * 32 + lane) * 16;
+            bool pending = false;
+            if (e_tile + off < n) {
                 float w[16];
-                unpack8(raw[u][0], *reinterpret_cast<float(*)[8]>(&w[0]));
-                unpack8(raw[u][1], *reinterpret_cast<float(*)[8]>(&w[8]));
-                pack_chunk<BITS>(w, sc[u], zr[u], Q, e0, codes);
+                unpack16(raw[j], w);
+                pending = chunk(w, gc[off >> gshift], e_tile + off, false);
             }
+            const uint32_t ballot = __ballot_sync(0xffffffffu, pending);
+            if (pending)
+                queue[queued + __popc(ballot & ((1u << lane) - 1u))] = PendingChunk{e_tile + off, gc[off >> gshift]};
+            queued += __popc(ballot);
+        }
+        // every 32 queued chunks, and the rest after the warp's last tile: the last
+        // `count` entries, one per lane
+        while (queued >= 32 || (last_tile && queued > 0)) {
+            const int count = queued < 32 ? queued : 32;
+            __syncwarp();
+            if (lane < count) {
+                const PendingChunk pc = queue[queued - count + lane];
+                float w[16];
+                unpack16(load_raw16<T>(W + pc.e0), w);
+                (void)chunk(w, pc.c, pc.e0, true);
+            }
+            queued -= count;
+            __syncwarp();
         }
     }
+}
+
+template <typename T>
+int tile_grid(int64_t n, const DeviceInfo &dev) {
+    const int64_t tiles = (n + kWarpTile<T> - 1) / kWarpTile<T>;
+    const int64_t blocks = (tiles + kTileWarps - 1) / kTileWarps;
+    return static_cast<int>(
+        std::max<int64_t>(1, std::min<int64_t>(blocks, static_cast<int64_t>(dev.sm_count) * kTileBlocksPerSm)));
+}
+
+// ------------------------------------------------------------------ fake-quant prepass
+// W-hat = (clamp(round(W/s) + zr, 0, Q) - zr) s = clamp(round(W/s), -zr, Q - zr) s
+// (all integer-valued until the one rounded product), with the code and the
+// straight-through mask 0 <= round(W/s) + zr <= Q when asked for.
+template <typename O, bool CODES>
+__device__ __forceinline__ bool fake_quant_chunk(const float (&w)[16], const GroupConst &c, float Q, int64_t e0,
+                                                 bool exact, O *__restrict__ W_hat, uint8_t *__restrict__ code,
+                                                 uint8_t *__restrict__ mask) {
+    const float mz = __fadd_rn(kRoundMagic, c.zr);
+    const uint64_t rcp2 = f2_pack(c.rcp, c.rcp), mz2 = f2_pack(mz, mz);
+    float v[16];
+    bool near = false;
+#pragma unroll
+    for (int j = 0; j < 16; j += 2) {
+        uint64_t u2, v2;
+        float ra, rb;
+        pair_decision(f2_pack(w[j], w[j + 1]), rcp2, mz2, u2, v2, ra, rb);
+        f2_unpack(v2, v[j], v[j + 1]);
+        if (exact) {
+            float ua, ub;
+            f2_unpack(u2, ua, ub);
+            if (fabsf(ra) >= c.band) v[j] = exact_round(w[j], c.sc, ua);
+            if (fabsf(rb) >= c.band) v[j + 1] = exact_round(w[j + 1], c.sc, ub);
+        } else {
+            near |= fabsf(ra) >= c.band;
+            near |= fabsf(rb) >= c.band;
+        }
+    }
+    if (near) return true;
+    // 0 - zr, not -zr: a clamped code of a group with zr = 0 gives W-hat = +0, as
+    // (c - zr) s does
+    const float vlo = __fsub_rn(0.0f, c.zr), vhi = __fsub_rn(Q, c.zr);
+    uint32_t mbits[4] = {0u, 0u, 0u, 0u};
+#pragma unroll
+    for (int j = 0; j < 16; ++j) {
+        if (CODES) mbits[j / 4] |= ((v[j] >= vlo) && (v[j] <= vhi) ? 1u : 0u) << (8 * (j % 4));
+        v[j] = fminf(fmaxf(v[j], vlo), vhi);
+    }
+    if (W_hat) {
+        const uint64_t s2 = f2_pack(c.sc, c.sc);
+        float wh[16];
+#pragma unroll
+        for (int j = 0; j < 16; j += 2) f2_unpack(f2_mul(f2_pack(v[j], v[j + 1]), s2), wh[j], wh[j + 1]);
+        store8<O>(W_hat + e0, *reinterpret_cast<const float(*)[8]>(&wh[0]));
+        store8<O>(W_hat + e0 + 8, *reinterpret_cast<const float(*)[8]>(&wh[8]));
+    }
+    if (CODES) {
+        // code = v + zr: the low byte of M + zr + v (exact)
+        uint32_t cbits[4] = {0u, 0u, 0u, 0u};
+#pragma unroll
+        for (int j = 0; j < 16; j += 2) {
+            float a, b;
+            f2_unpack(f2_add(f2_pack(v[j], v[j + 1]), mz2), a, b);
+            cbits[j / 4] |= (static_cast<uint32_t>(__float_as_int(a)) & 0xFFu) << (8 * (j % 4));
+            cbits[j / 4] |= (static_cast<uint32_t>(__float_as_int(b)) & 0xFFu) << (8 * (j % 4 + 1));
+        }
+        if (code) *reinterpret_cast<uint4 *>(code + e0) = make_uint4(cbits[0], cbits[1], cbits[2], cbits[3]);
+        if (mask) *reinterpret_cast<uint4 *>(mask + e0) = make_uint4(mbits[0], mbits[1], mbits[2], mbits[3]);
+    }
+    return false;
+}
+
+template <typename T, typename O, bool CODES>
+__global__ void __launch_bounds__(kTileThreads, kTileBlocksPerSm)
+    k_fake_quant(const T *__restrict__ W, const float *__restrict__ s, const float *__restrict__ z, int64_t n,
+                 int gshift, float Q, O *__restrict__ W_hat, uint8_t *__restrict__ code,
+                 uint8_t *__restrict__ mask) {
+    __shared__ GroupConst gc[kTileWarps * kWarpGroups<T>];
+    __shared__ PendingChunk queue[kTileWarps * kQueue<T>];
+    walk_warp_tiles<T, false>(W, s, z, n, gshift, Q, nullptr, gc, queue,
+                              [&](const float (&w)[16], const GroupConst &c, int64_t e0, bool exact) {
+                                  return fake_quant_chunk<O, CODES>(w, c, Q, e0, exact, W_hat, code, mask);
+                              });
+}
+
+// ------------------------------------------------------------------ pack
+// Codes of 16 weights of one group into their packed words (2-bit: one word,
+// code k at bits 2k; 4-bit: two words, 4k; 3-bit: four words, one code per
+// byte).  zr := zq = clamp(round(z), 0, Q) (z hard-rounded at pack time).
+//
+// Two codes per f16x2 word: 1024 + zr + round(u) is an integer that f16 holds
+// exactly, so after a clamp of both halves to [1024, 1024 + Q] the low bits of
+// each half are the code.  The weights of a pair sit 16 bits apart in their
+// packed word (k and k + 8 for 2-bit codes, k and k + 4 for 4-bit, k and k + 2
+// for 3-bit), so one shifted add places both; the bits of 1024 are taken out
+// once per word at the end.
+template <int BITS>
+struct PackLayout {
+    static constexpr int kSlot = BITS == 3 ? 8 : BITS;  // bits per code in a word
+    static constexpr int kPerWord = 32 / kSlot;
+    static constexpr int kWords = 16 / kPerWord;
+    static constexpr int kHalf = kPerWord / 2;  // pair partner distance
+};
+
+// sum over i < count of bits(f16 1024, twice) << (step i), modulo 2^32.
+__host__ __device__ constexpr uint32_t magic_h2_word(int step, int count) {
+    uint32_t acc = 0;
+    for (int i = 0; i < count; ++i) acc += 0x64006400u << (step * i);
+    return acc;
+}
+
+template <int BITS>
+__device__ __forceinline__ bool pack_chunk(const float (&w)[16], const GroupConst &c, float Q, int64_t e0,
+                                           bool exact, uint8_t *__restrict__ codes) {
+    using L = PackLayout<BITS>;
+    const float mz = __fadd_rn(kRoundMagic, c.zr), zk = __fadd_rn(c.zr, 1024.0f);
+    const uint64_t rcp2 = f2_pack(c.rcp, c.rcp), mz2 = f2_pack(mz, mz), zk2 = f2_pack(zk, zk);
+    const uint32_t lo2 = 0x64006400u;  // f16 1024 in both halves
+    const uint32_t qh = 0x6400u + static_cast<uint32_t>(Q);
+    const uint32_t hi2 = qh | (qh << 16);
+    uint32_t word[4];
+    bool near = false;
+#pragma unroll
+    for (int m = 0; m < L::kWords; ++m) {
+        uint32_t acc = 0u;
+#pragma unroll
+        for (int i = 0; i < L::kHalf; ++i) {
+            const int a = m * L::kPerWord + i, b = a + L::kHalf;
+            uint64_t u2, v2;
+            float ra, rb;
+            pair_decision(f2_pack(w[a], w[b]), rcp2, mz2, u2, v2, ra, rb);
+            if (exact) {
+                float ua, ub, va, vb;
+                f2_unpack(u2, ua, ub);
+                f2_unpack(v2, va, vb);
+                if (fabsf(ra) >= c.band) va = exact_round(w[a], c.sc, ua);
+                if (fabsf(rb) >= c.band) vb = exact_round(w[b], c.sc, ub);
+                v2 = f2_pack(va, vb);
+            } else {
+                near |= fabsf(ra) >= c.band;
+                near |= fabsf(rb) >= c.band;
+            }
+            float ea, eb;
+            f2_unpack(f2_add(v2, zk2), ea, eb);
+            acc += h2_clamp(h2_from_f32(ea, eb), lo2, hi2) << (L::kSlot * i);
+        }
+        word[m] = acc - magic_h2_word(L::kSlot, L::kHalf);
+    }
+    if (near) return true;
+    if (BITS == 2) {
+        *reinterpret_cast<uint32_t *>(codes + e0 / 4) = word[0];
+    } else if (BITS == 4) {
+        *reinterpret_cast<uint2 *>(codes + e0 / 2) = make_uint2(word[0], word[1]);
+    } else {
+        *reinterpret_cast<uint4 *>(codes + e0) = make_uint4(word[0], word[1], word[2], word[3]);
+    }
+    return false;
+}
+
+template <typename T, int BITS>
+__global__ void __launch_bounds__(kTileThreads, kTileBlocksPerSm)
+    k_pack(const T *__restrict__ W, const float *__restrict__ s, const float *__restrict__ z, int64_t n, int gshift,
+           float Q, uint8_t *__restrict__ codes, uint8_t *__restrict__ zq) {
+    __shared__ GroupConst gc[kTileWarps * kWarpGroups<T>];
+    __shared__ PendingChunk queue[kTileWarps * kQueue<T>];
+    walk_warp_tiles<T, true>(W, s, z, n, gshift, Q, zq, gc, queue,
+                             [&](const float (&w)[16], const GroupConst &c, int64_t e0, bool exact) {
+                                 return pack_chunk<BITS>(w, c, Q, e0, exact, codes);
+                             });
 }
 
 // ------------------------------------------------------------------ E2E dequant
-// One thread per 16 consecutive codes: W-hat = (W_q - zq) * s (Eq. 2).
+// One thread per 16 consecutive codes: W-hat = (W_q - zq) s (Eq. 2).  A code and
+// zq enter fp32 as the raw bits of M + code and M + zq (exact), so W_q - zq is
+// one subtraction and W-hat one rounded product, two weights per instruction.
 template <int BITS>
-__device__ __forceinline__ void unpack16(const uint8_t *codes, int64_t e0, uint32_t (&c)[16]) {
+__device__ __forceinline__ void codes16_magic(const uint8_t *codes, int64_t e0, float (&f)[16]) {
+    constexpr uint32_t kM = 0x4B400000u;  // bits of M = 1.5 * 2^23
     if (BITS == 2) {
         const uint32_t word = __ldg(reinterpret_cast<const uint32_t *>(codes + e0 / 4));
 #pragma unroll
-        for (int j = 0; j < 16; ++j) c[j] = (word >> (2 * j)) & 3u;
+        for (int j = 0; j < 16; ++j) f[j] = __uint_as_float(((word >> (2 * j)) & 3u) | kM);
     } else if (BITS == 4) {
         const uint2 r = __ldg(reinterpret_cast<const uint2 *>(codes + e0 / 2));
 #pragma unroll
-        for (int j = 0; j < 8; ++j) c[j] = (r.x >> (4 * j)) & 15u;
+        for (int j = 0; j < 8; ++j) f[j] = __uint_as_float(((r.x >> (4 * j)) & 15u) | kM);
 #pragma unroll
-        for (int j = 0; j < 8; ++j) c[8 + j] = (r.y >> (4 * j)) & 15u;
+        for (int j = 0; j < 8; ++j) f[8 + j] = __uint_as_float(((r.y >> (4 * j)) & 15u) | kM);
     } else {
         const uint4 r = __ldg(reinterpret_cast<const uint4 *>(codes + e0));
         const uint32_t w4[4] = {r.x, r.y, r.z, r.w};
 #pragma unroll
-        for (int j = 0; j < 16; ++j) c[j] = (w4[j / 4] >> (8 * (j % 4))) & 0xFFu;
+        for (int j = 0; j < 16; ++j) f[j] = __uint_as_float(((w4[j / 4] >> (8 * (j % 4))) & 0xFFu) | kM);
     }
 }
 
@@ -351,16 +532,16 @@ __global__ void __launch_bounds__(kThreads)
         const int64_t e0 = i * 16;
         const int64_t g = e0 >> gshift;
         const float sc = step_value(s, g);
-        const float zf = static_cast<float>(__ldg(zq + g));
-        uint32_t c[16];
-        unpack16<BITS>(codes, e0, c);
-        float a[8], b[8];
+        const float mz = __uint_as_float(static_cast<uint32_t>(__ldg(zq + g)) | 0x4B400000u);  // M + zq
+        float f[16];
+        codes16_magic<BITS>(codes, e0, f);
+        const uint64_t mz2 = f2_pack(mz, mz), s2 = f2_pack(sc, sc);
+        float wh[16];
 #pragma unroll
-        for (int j = 0; j < 8; ++j) a[j] = dequant_elem(static_cast<float>(c[j]), zf, sc);
-#pragma unroll
-        for (int j = 0; j < 8; ++j) b[j] = dequant_elem(static_cast<float>(c[8 + j]), zf, sc);
-        store8<O>(W_hat + e0, a);
-        store8<O>(W_hat + e0 + 8, b);
+        for (int j = 0; j < 16; j += 2)
+            f2_unpack(f2_mul(f2_sub(f2_pack(f[j], f[j + 1]), mz2), s2), wh[j], wh[j + 1]);
+        store8<O>(W_hat + e0, *reinterpret_cast<const float(*)[8]>(&wh[0]));
+        store8<O>(W_hat + e0 + 8, *reinterpret_cast<const float(*)[8]>(&wh[8]));
     }
 }
 
@@ -381,13 +562,12 @@ template <typename T>
 cudaError_t pack_dispatch(const T *W, const float *s, const float *z, int64_t n, int bits, int group,
                           uint8_t *codes, uint8_t *zq, const DeviceInfo &dev, cudaStream_t st) {
     const int gshift = group_shift(group);
-    const int64_t chunks = n / 16;
-    const int grid = grid_for(chunks, dev);
+    const int grid = tile_grid<T>(n, dev);
     const float Q = static_cast<float>((1 << bits) - 1);
     switch (bits) {
-        case 2: k_pack<T, 2><<<grid, kThreads, 0, st>>>(W, s, z, chunks, gshift, Q, codes, zq); break;
-        case 3: k_pack<T, 3><<<grid, kThreads, 0, st>>>(W, s, z, chunks, gshift, Q, codes, zq); break;
-        case 4: k_pack<T, 4><<<grid, kThreads, 0, st>>>(W, s, z, chunks, gshift, Q, codes, zq); break;
+        case 2: k_pack<T, 2><<<grid, kTileThreads, 0, st>>>(W, s, z, n, gshift, Q, codes, zq); break;
+        case 3: k_pack<T, 3><<<grid, kTileThreads, 0, st>>>(W, s, z, n, gshift, Q, codes, zq); break;
+        case 4: k_pack<T, 4><<<grid, kTileThreads, 0, st>>>(W, s, z, n, gshift, Q, codes, zq); break;
         default: return cudaErrorInvalidValue;
     }
     return cudaGetLastError();
@@ -424,21 +604,21 @@ cudaError_t launch_fake_quant(const void *W, bool w_f32, const float *s, const f
                               int64_t K, int bits, int group, void *W_hat, bool out_f32,
                               uint8_t *code, uint8_t *mask, const DeviceInfo &dev,
                               cudaStream_t st) {
-    const int64_t chunks = N * K / 8;
-    if (chunks == 0) return cudaSuccess;
-    const int grid = grid_for(chunks, dev);
+    const int64_t n = N * K;
+    if (n == 0) return cudaSuccess;
     const float Q = static_cast<float>((1 << bits) - 1);
     using bf = __nv_bfloat16;
     const bool codes = code || mask;
     const int gshift = group_shift(group);
-#define EQAT_FQ_LAUNCH(TW, TO)                                                                          \
-    do {                                                                                                \
-        if (codes)                                                                                      \
-            k_fake_quant<TW, TO, true><<<grid, kThreads, 0, st>>>(static_cast<const TW *>(W), s, z, chunks, \
-                                                                 gshift, Q, static_cast<TO *>(W_hat), code, mask); \
-        else                                                                                            \
-            k_fake_quant<TW, TO, false><<<grid, kThreads, 0, st>>>(static_cast<const TW *>(W), s, z, chunks, \
-                                                                  gshift, Q, static_cast<TO *>(W_hat), code, mask); \
+#define EQAT_FQ_LAUNCH(TW, TO)                                                                              \
+    do {                                                                                                    \
+        const int grid = tile_grid<TW>(n, dev);                                                             \
+        if (codes)                                                                                          \
+            k_fake_quant<TW, TO, true><<<grid, kTileThreads, 0, st>>>(static_cast<const TW *>(W), s, z, n,  \
+                                                                     gshift, Q, static_cast<TO *>(W_hat), code, mask); \
+        else                                                                                                \
+            k_fake_quant<TW, TO, false><<<grid, kTileThreads, 0, st>>>(static_cast<const TW *>(W), s, z, n, \
+                                                                      gshift, Q, static_cast<TO *>(W_hat), code, mask); \
     } while (0)
     if (w_f32 && out_f32)
         EQAT_FQ_LAUNCH(float, float);

@@ -14,6 +14,7 @@
 
 #include <algorithm>
 #include <cstdint>
+#include <type_traits>
 
 #include "eqat_internal.h"
 #include "eqat_qmath.cuh"
@@ -284,28 +285,48 @@ __device__ __forceinline__ void walk_warp_tiles(const T *__restrict__ W, const f
     for (int64_t tile = static_cast<int64_t>(blockIdx.x) * kTileWarps + wib; tile < n_tiles; tile += stride) {
         const int64_t e_tile = tile * WT;
         const bool last_tile = tile + stride >= n_tiles;
+        // A whole tile (every tile but the last of the layer) runs without bounds
+        // checks.
+        const bool whole = e_tile + WT <= n;
         Raw16<T> raw[CPL];
+        if (whole) {
 #pragma unroll
-        for (int j = 0; j < CPL; ++j) {
-            const int64_t e0 = e_tile + (j * 32 + lane) * 16;
-            if (e0 < n) raw[j] = load_raw16<T>(W + e0);
+            for (int j = 0; j < CPL; ++j) raw[j] = load_raw16<T>(W + e_tile + (j * 32 + lane) * 16);
+        } else {
+#pragma unroll
+            for (int j = 0; j < CPL; ++j) {
+                const int64_t e0 = e_tile + (j * 32 + lane) * 16;
+                if (e0 < n) raw[j] = load_raw16<T>(W + e0);
+            }
         }
         __syncwarp();  // the previous tile's reads of gc are done
         tile_group_consts<T>(s, z, e_tile, n, gshift, Q, CLAMP_Z, lane, gc, zq);
         __syncwarp();
+        uint32_t pending = 0u;  // bit j: chunk j left for the exact pass
+        auto fast_pass = [&](auto whole_tag) {
 #pragma unroll
-        for (int j = 0; j < CPL; ++j) {
-            const int off = (j * 32 + lane) * 16;
-            bool pending = false;
-            if (e_tile + off < n) {
-                float w[16];
-                unpack16(raw[j], w);
-                pending = chunk(w, gc[off >> gshift], e_tile + off, false);
+            for (int j = 0; j < CPL; ++j) {
+                const int off = (j * 32 + lane) * 16;
+                if (decltype(whole_tag)::value || e_tile + off < n) {
+                    float w[16];
+                    unpack16(raw[j], w);
+                    if (chunk(w, gc[off >> gshift], e_tile + off, false)) pending |= 1u << j;
+                }
             }
-            const uint32_t ballot = __ballot_sync(0xffffffffu, pending);
-            if (pending)
-                queue[queued + __popc(ballot & ((1u << lane) - 1u))] = PendingChunk{e_tile + off, gc[off >> gshift]};
-            queued += __popc(ballot);
+        };
+        if (whole)
+            fast_pass(std::true_type{});
+        else
+            fast_pass(std::false_type{});
+        if (__any_sync(0xffffffffu, pending != 0u)) {
+#pragma unroll
+            for (int j = 0; j < CPL; ++j) {
+                const int off = (j * 32 + lane) * 16;
+                const bool p = (pending >> j) & 1u;
+                const uint32_t ballot = __ballot_sync(0xffffffffu, p);
+                if (p) queue[queued + __popc(ballot & ((1u << lane) - 1u))] = PendingChunk{e_tile + off, gc[off >> gshift]};
+                queued += __popc(ballot);
+            }
         }
         // every 32 queued chunks, and the rest after the warp's last tile: the last
         // `count` entries, one per lane

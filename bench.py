@@ -90,55 +90,121 @@ def load_traffic():
 
 # ------------------------------------------------------------------------------ clocks
 
-class ClockSampler:
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+CLOCK_REASONS = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
 
-    def __init__(self, index: int):
-        self.index = index
-        self.proc = None
+
+class ClockSampler:
+    """SM clock and clock-event reasons of one GPU, read (never set) through NVML by
+    a background thread every `period_s`, with a wall-clock stamp per sample, so that
+    the samples inside a short timed region can be picked out afterwards.  mark()
+    records the wall clock of the region's ends.  If NVML is unavailable it falls
+    back to `nvidia-smi -lms 200`, which sees only regions longer than its period."""
+
+    def __init__(self, device: torch.device, period_s: float = 0.0005):
+        self.device = device
+        self.period = period_s
+        self.samples = []  # (t, sm_mhz, reasons set)
+        self.marks = {}
+        self.sm_max = None
+        self._stop = None
+        self._thread = None
+        self._smi = None
+        self.source = "none"
+
+    def _nvml_handle(self):
+        import pynvml
+        pynvml.nvmlInit()
+        props = torch.cuda.get_device_properties(self.device)
+        try:
+            bus = f"{props.pci_domain_id:08x}:{props.pci_bus_id:02x}:{props.pci_device_id:02x}.0"
+            return pynvml, pynvml.nvmlDeviceGetHandleByPciBusId(bus.encode())
+        except Exception:  # noqa: BLE001 - fall back to the CUDA ordinal
+            return pynvml, pynvml.nvmlDeviceGetHandleByIndex(self.device.index or 0)
 
     def __enter__(self):
+        import threading
         try:
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                 "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
-        except OSError:
-            self.proc = None
+            nv, h = self._nvml_handle()
+            self.sm_max = float(nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM))
+            bits = {"hw_slowdown": nv.nvmlClocksEventReasonHwSlowdown,
+                    "hw_thermal_slowdown": nv.nvmlClocksEventReasonHwThermalSlowdown,
+                    "sw_thermal_slowdown": nv.nvmlClocksEventReasonSwThermalSlowdown,
+                    "sw_power_cap": nv.nvmlClocksEventReasonSwPowerCap}
+            self._stop = threading.Event()
+
+            def loop():
+                while not self._stop.is_set():
+                    t = time.perf_counter()
+                    try:
+                        mhz = float(nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM))
+                        r = nv.nvmlDeviceGetCurrentClocksEventReasons(h)
+                    except Exception:  # noqa: BLE001
+                        break
+                    self.samples.append((t, mhz, {n for n, b in bits.items() if r & b}))
+                    self._stop.wait(self.period)
+            self._thread = threading.Thread(target=loop, daemon=True)
+            self._thread.start()
+            self.source = "nvml"
+        except Exception:  # noqa: BLE001 - no NVML: nvidia-smi's own sampler
+            fields = ("clocks.sm,clocks.max.sm,clocks_event_reasons.hw_slowdown,"
+                      "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+                      "clocks_event_reasons.sw_power_cap")
+            try:
+                self._smi = subprocess.Popen(
+                    ["nvidia-smi", f"--id={self.device.index or 0}", f"--query-gpu={fields}",
+                     "--format=csv,noheader,nounits", "-lms", "200"],
+                    stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+                self._t0 = time.perf_counter()
+                self.source = "nvidia-smi"
+            except OSError:
+                self._smi = None
         return self
 
-    def __exit__(self, *exc):
-        if self.proc:
-            self.proc.terminate()
-            try:
-                out, _ = self.proc.communicate(timeout=5)
-            except subprocess.TimeoutExpired:
-                self.proc.kill()
-                out, _ = self.proc.communicate()
-            self.lines = [l for l in out.splitlines() if l.strip()]
-        else:
-            self.lines = []
+    def mark(self, name):
+        self.marks[name] = time.perf_counter()
 
-    def summary(self):
-        sm, smax, reasons = [], None, set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for l in self.lines:
-            f = [x.strip() for x in l.split(",")]
-            if len(f) < 9:
-                continue
+    def __exit__(self, *exc):
+        if self._thread is not None:
+            self._stop.set()
+            self._thread.join(timeout=5)
+        if self._smi is not None:
+            self._smi.terminate()
             try:
-                sm.append(float(f[1]))
-                smax = float(f[2])
-            except ValueError:
-                continue
-            for n, v in zip(names, f[5:9]):
-                if v.lower().startswith("active"):
-                    reasons.add(n)
-        if not sm:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0}
-        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": smax, "reasons": sorted(reasons),
-                "samples": len(sm)}
+                out, _ = self._smi.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self._smi.kill()
+                out, _ = self._smi.communicate()
+            # nvidia-smi gives no timestamps here: treat its samples as spread evenly
+            lines = [l for l in out.splitlines() if l.strip()]
+            t1 = time.perf_counter()
+            for i, l in enumerate(lines):
+                f = [x.strip() for x in l.split(",")]
+                try:
+                    mhz, self.sm_max = float(f[0]), float(f[1])
+                except (ValueError, IndexError):
+                    continue
+                rs = {n for n, v in zip(CLOCK_REASONS, f[2:6]) if v.lower().startswith("active")}
+                self.samples.append((self._t0 + (t1 - self._t0) * (i + 0.5) / max(1, len(lines)), mhz, rs))
+
+    def summary(self, start="start", end="end"):
+        """Samples inside [mark start, mark end], plus the last sample before the
+        region and the first after it (the region is often shorter than a few ms)."""
+        t0, t1 = self.marks.get(start), self.marks.get(end)
+        inside = [x for x in self.samples if t0 is not None and t1 is not None and t0 <= x[0] <= t1]
+        before = [x for x in self.samples if t0 is not None and x[0] < t0][-1:]
+        after = [x for x in self.samples if t1 is not None and x[0] > t1][:1]
+        use = inside or (before + after)
+        if not use:
+            return {"sm_mhz": None, "sm_max_mhz": self.sm_max, "reasons": ["unsampled"], "samples": 0,
+                    "source": self.source}
+        reasons = set()
+        for x in use:
+            reasons |= x[2]
+        return {"sm_mhz": statistics.median(x[1] for x in use), "sm_max_mhz": self.sm_max,
+                "reasons": sorted(reasons), "samples": len(inside),
+                "sm_mhz_before": before[0][1] if before else None, "sm_mhz_after": after[0][1] if after else None,
+                "region_ms": round((t1 - t0) * 1e3, 3) if t0 is not None and t1 is not None else None,
+                "source": self.source}
 
 
 # ------------------------------------------------------------------------------ our arm
@@ -201,18 +267,67 @@ class Step:
             allreduce([self.dW, self.ds, self.dz, self.ds2])
 
 
-def phase_bytes(M, N, K, bits, group):
-    """Algorithmic HBM bytes of the two HBM-bound phases (bf16 W)."""
+def code_bytes(N, K, bits):
+    """Bytes of the packed codes: 2-bit 4 per byte, 4-bit 2 per byte, 3-bit one per byte."""
+    return N * K // 4 if bits == 2 else N * K // 2 if bits == 4 else N * K
+
+
+def hbm_bytes(kernel, N, K, bits, group, wbytes=2):
+    """Algorithmic HBM bytes of one launch of an HBM-bound kernel over an [N, K]
+    weight: every input read once and every output written once.
+      init     W, then s and z (fp32)
+      pack     W, s, z, then the codes and zq (uint8)
+      prepass  W, s, z, then W-hat (the weight's dtype)
+      dequant  codes, zq, s, then W-hat"""
     G = K // group
-    init = N * K * 2 + 8 * N * G
-    pack = N * K * 2 + 8 * N * G + N * K * bits // 8 + N * G
-    if bits == 3:
-        pack = N * K * 2 + 8 * N * G + N * K + N * G
-    return init, pack
+    if kernel == "init":
+        return N * K * wbytes + 8 * N * G
+    if kernel == "pack":
+        return N * K * wbytes + 8 * N * G + code_bytes(N, K, bits) + N * G
+    if kernel == "prepass":
+        return 2 * N * K * wbytes + 8 * N * G
+    if kernel == "dequant":
+        return code_bytes(N, K, bits) + 5 * N * G + N * K * wbytes
+    raise ValueError(kernel)
 
 
-def flush_l2(buf):
-    buf.zero_()
+def phase_bytes(M, N, K, bits, group):
+    """Algorithmic HBM bytes of the two HBM-bound phases of the step (bf16 W)."""
+    return hbm_bytes("init", N, K, bits, group), hbm_bytes("pack", N, K, bits, group)
+
+
+class L2Flush:
+    """Leaves L2 holding none of the next kernel's data and no dirty lines: a write
+    of 512 MiB (4x L2), then a read of 256 MiB of another buffer, so the next kernel
+    neither hits in L2 nor first writes back the flush's own dirty lines."""
+
+    def __init__(self, dev):
+        self.w = torch.empty(512 << 20, dtype=torch.uint8, device=dev)
+        self.r = torch.ones(64 << 20, dtype=torch.float32, device=dev)
+
+    def __call__(self):
+        self.w.zero_()
+        self.r.amax()
+
+
+def bench_config(world):
+    """The `config` of both arms' JSON lines (the reference arm prints the same dict)."""
+    wl = WORKLOAD
+    lin = wl.linears[0]
+    return {"workload": wl.name, "M": wl.m, "N": lin.n, "K": lin.k, "bits": wl.bits, "group": wl.group,
+            "flops_per_step": 12 * wl.m * lin.n * lin.k,
+            "l2": "flushed before every step (512 MiB write, then a 256 MiB read of another buffer)",
+            "parallelism": f"dp{world}" if world > 1 else "single-gpu",
+            "step": "+".join(PHASES)}
+
+
+def choose_gemm_peak(peaks, region_s):
+    """The measured bf16 peak that matches how long the kernel ran back to back: the
+    burst figure for a region under a second (the GPU does not reach its power-capped
+    clock in that time), the sustained one for a longer region."""
+    if region_s < 1.0:
+        return peaks["bf16_tflops"], f"bf16 dense, burst (timed region {region_s * 1e3:.1f} ms < 1 s), {peaks['source']}"
+    return peaks["bf16_tflops_sustained"], f"bf16 dense, sustained (timed region {region_s:.1f} s), {peaks['source']}"
 
 
 def run_ours(args):
@@ -234,33 +349,35 @@ def run_ours(args):
     wl = WORKLOAD
     step = Step(wl, rank, wl.bits, wl.group, dev)
     M, N, K = step.M, step.N, step.K
-    flush = torch.empty(512 << 20, dtype=torch.uint8, device=dev)
+    flush = L2Flush(dev)
 
     allreduce = None
     if dist is not None:
         def allreduce(ts):
             dp.allreduce_weight_grads(ts, dist)
 
-    for _ in range(args.warmup):
-        flush_l2(flush)
-        step.run(allreduce=allreduce)
-    torch.cuda.synchronize()
-    if eqat.device_error() != 0:
-        raise RuntimeError("device error word set during warm-up")
-
     nph = len(PHASES)
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(nph + 2)] for _ in range(args.steps)]
-    if dist is not None:
-        dist.barrier()
-    torch.cuda.synchronize()
-    with ClockSampler(local) as clk:
+    with ClockSampler(dev) as clk:
+        for _ in range(args.warmup):
+            flush()
+            step.run(allreduce=allreduce)
+        torch.cuda.synchronize()
+        if eqat.device_error() != 0:
+            raise RuntimeError("device error word set during warm-up")
+        if dist is not None:
+            dist.barrier()
+        torch.cuda.synchronize()
+        clk.mark("start")
         t_wall = time.perf_counter()
         for i in range(args.steps):
-            flush_l2(flush)
+            flush()
             step.run(events=ev[i], allreduce=allreduce)
             ev[i][nph + 1].record()
         torch.cuda.synchronize()
         t_wall = time.perf_counter() - t_wall
+        clk.mark("end")
+        time.sleep(0.01)  # one more sample after the region
     if dist is not None:
         dist.barrier()
     torch.cuda.synchronize()
@@ -283,11 +400,10 @@ def run_ours(args):
     dom_ms = mean[DOMINANT]
     dom_flops = 4 * M * N * K
     achieved = dom_flops / (dom_ms * 1e-3) / 1e12
-    peak = peaks["bf16_tflops_sustained"]
+    peak, peak_kind = choose_gemm_peak(peaks, t_wall)
     init_b, pack_b = phase_bytes(M, N, K, wl.bits, wl.group)
     traffic = load_traffic()
     clocks = clk.summary()
-
     # --------------------------------------------------------------------- e2e (host buffers)
     # Every step copies its inputs (X, W, dY) from pinned host memory and reads its
     # result back: the gradients of the quantization parameters (ds, dz of Block-AP,
@@ -361,6 +477,22 @@ def run_ours(args):
                "note": "inputs X, W, dY copied in every step (double-buffered, overlapping the previous step); "
                        "result read back every step: ds, dz, ds2, codes, zq"}
 
+    # HBM-bound kernels: each timed alone after a clean flush, on the step's layer and
+    # over the seven linears of the Llama-2-70B block
+    hbm = hbm_kernels(step, dev, peaks, flush) if not args.no_hbm else {}
+    ip = initpack_70b_block(dev, peaks) if not args.no_initpack70b else None
+    if ip is not None:
+        for k in ("init", "pack", "prepass", "dequant"):
+            hbm.setdefault(k, {})["llama2-70b-block"] = ip[k]
+    for k, ms, b in (("init", mean["init"], init_b), ("pack", mean["pack"], pack_b)):
+        gbs = b / (ms * 1e-3) / 1e9
+        hbm.setdefault(k, {})["in_step"] = {"GBps": round(gbs, 1), "frac": round(gbs / peaks["hbm_gbs"], 4),
+                                            "bytes": b, "us": round(ms * 1e3, 2)}
+    hbm["peak_GBps"] = peaks["hbm_gbs"]
+    hbm["peak_kind"] = f"copy bandwidth, {peaks['source']}"
+    hbm["note"] = ("algorithmic bytes (each input read once, each output written once) / CUDA-event time; "
+                   "'in_step' inside the timed step, the others alone after a clean L2 flush")
+
     line = {
         "metric": METRIC,
         "value": round(value, 3),
@@ -374,52 +506,84 @@ def run_ours(args):
         "vs_baseline": None,
         "dtype": "bf16",
         "data": "synthetic (seeded N(0,1) activations and gradients, N(0,0.02) weights with 0.1% x10 outliers)",
-        "config": {"workload": wl.name, "M": M, "N": N, "K": K, "bits": wl.bits, "group": wl.group,
-                   "flops_per_step": flops_step, "l2": "flushed before every step (512 MiB write)",
-                   "parallelism": f"dp{world}" if world > 1 else "single-gpu",
-                   "step": "+".join(PHASES)},
+        "config": bench_config(world),
         "roofline": {"bound": "tensor",
                      "kernel": "k_gemm_tc2 grouped backward on CTA pairs: dY W-hat + dY^T X with the fused "
                                "straight-through epilogue",
                      "achieved": round(achieved, 2), "peak": peak, "unit": "TFLOP/s",
                      "frac": round(achieved / peak, 4), "traffic": traffic,
-                     "peak_kind": f"bf16 dense, sustained, {peaks['source']}",
-                     "frac_of_burst_peak": round(achieved / peaks["bf16_tflops"], 4)},
-        "phases_ms": {p: round(v, 4) for p, v in mean.items()},
-        "phase_rates": {
-            "init_GBps": round(init_b / (mean["init"] * 1e-3) / 1e9, 1),
-            "pack_GBps": round(pack_b / (mean["pack"] * 1e-3) / 1e9, 1),
-            "init_frac_hbm": round(init_b / (mean["init"] * 1e-3) / 1e9 / peaks["hbm_gbs"], 4),
-            "pack_frac_hbm": round(pack_b / (mean["pack"] * 1e-3) / 1e9 / peaks["hbm_gbs"], 4),
-            "blockap_fwd_bwd_TFLOPs": round(6 * M * N * K / ((mean["fq_fwd"] + mean["fq_bwd"]) * 1e-3) / 1e12, 2),
-            "e2e_fwd_bwd_TFLOPs": round(6 * M * N * K / ((mean["dq_fwd"] + mean["dq_bwd"]) * 1e-3) / 1e12, 2),
-            "hbm_peak_GBps": peaks["hbm_gbs"],
-        },
+                     "peak_kind": peak_kind,
+                     "frac_of_sustained_peak": round(achieved / peaks["bf16_tflops_sustained"], 4),
+                     "hbm": hbm},
         "gpu_launches": sum(LAUNCHES_PER_STEP.values()) * args.steps,
         "clocks": clocks,
         "wall_s_timed": round(t_wall, 3),
         "e2e": e2e,
+        "phases_ms": {p: round(v, 4) for p, v in mean.items()},
+        "phase_rates": {
+            "blockap_fwd_bwd_TFLOPs": round(6 * M * N * K / ((mean["fq_fwd"] + mean["fq_bwd"]) * 1e-3) / 1e12, 2),
+            "e2e_fwd_bwd_TFLOPs": round(6 * M * N * K / ((mean["dq_fwd"] + mean["dq_bwd"]) * 1e-3) / 1e12, 2),
+        },
     }
-    if not args.no_initpack70b:
-        ip = initpack_70b_block(dev)
-        ip["init_frac_hbm"] = round(ip["init_GBps"] / peaks["hbm_gbs"], 4)
-        ip["pack_frac_hbm"] = round(ip["pack_GBps"] / peaks["hbm_gbs"], 4)
-        line["initpack_70b_block"] = ip
     if not args.no_variants:
         line["variants"] = quantizer_variants(step, dev)
     if not args.no_gemv:
         line["decode_gemv"] = decode_gemv(dev, peaks)
     if not args.no_blockap:
         line["blockap_block"] = blockap_block(dev, peaks)
+    if not args.no_cfg1:
+        line["cfg1_latency"] = cfg1_latency(dev)
     if not args.no_configs:
         line["per_config"] = per_config(dev, peaks)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        line["cpu_baseline"] = cpu_baseline(target_s=args.cpu_seconds)
+        line["cpu_baseline"] = cpu_baseline(target_s=args.cpu_seconds, plan=not args.no_oracle_plan)
     if dist is not None:
         dist.barrier()
         dist.destroy_process_group()
     if rank == 0:
         print(json.dumps(line), flush=True)
+
+
+def timed_alone(fn, flush, reps):
+    """Median CUDA-event time (ms) of fn() over `reps` calls, each after a clean L2 flush."""
+    out = []
+    for r in range(reps + 2):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        flush()
+        e0.record()
+        fn()
+        e1.record()
+        torch.cuda.synchronize()
+        if r >= 2:
+            out.append(e0.elapsed_time(e1))
+    return statistics.median(out)
+
+
+def hbm_kernels(step, dev, peaks, flush, reps=20):
+    """The four HBM-bound quantizer kernels on the step's layer, each launched alone
+    after a clean L2 flush: min-max init, pack, the Block-AP prepass (eqat_fake_quant
+    writing W-hat only: the kernel inside eqat_fq_linear_fwd) and the E2E-QP
+    dequantization (eqat_dequant_codes)."""
+    b, g, N, K = step.bits, step.group, step.N, step.K
+    wh = torch.empty_like(step.W)
+    calls = {
+        "init": lambda: eqat.minmax_init(step.W, b, g, s=step.s, z=step.z),
+        "pack": lambda: eqat.pack_codes(step.W, step.s, step.z, b, g, codes=step.codes, zq=step.zq),
+        "prepass": lambda: eqat.fake_quant(step.W, step.s, step.z, b, g, want_code=False, want_mask=False, W_hat=wh),
+        "dequant": lambda: eqat.dequant_codes(step.codes, step.zq, step.s, K, b, g, out=wh),
+    }
+    out = {}
+    for k, fn in calls.items():
+        ms = timed_alone(fn, flush, reps)
+        byts = hbm_bytes(k, N, K, b, g)
+        gbs = byts / (ms * 1e-3) / 1e9
+        out[k] = {step_layer_name(): {"GBps": round(gbs, 1), "frac": round(gbs / peaks["hbm_gbs"], 4),
+                                      "bytes": byts, "us": round(ms * 1e3, 2)}}
+    return out
+
+
+def step_layer_name():
+    return "llama2-7b-q_proj"
 
 
 def quantizer_variants(step, dev, reps=50):
@@ -472,21 +636,46 @@ def quantizer_variants(step, dev, reps=50):
     return out
 
 
+def fused_linears(wl):
+    """The linears of a workload as they are launched: k_proj and v_proj of the 70B
+    block read the same X and have the same K, so their weights are stored as one
+    [N_k + N_v, K] matrix (k's rows, then v's) and run as one linear, the usual fused
+    k/v projection.  Groups never cross rows, so s, z and the codes of the fused
+    layer are the row-concatenations of the two layers', and every output element is
+    the one the separate layers give (Y_k, Y_v are the column blocks of Y_kv).
+    Returns (name, N, K, [member names])."""
+    lins = list(wl.linears)
+    names = [l.name for l in lins]
+    out = []
+    for l in lins:
+        if l.name == "v_proj" and "k_proj" in names:
+            continue
+        if l.name == "k_proj" and "v_proj" in names:
+            v = lins[names.index("v_proj")]
+            if v.k == l.k:
+                out.append(("kv_proj", l.n + v.n, l.k, ["k_proj", "v_proj"]))
+                continue
+        out.append((l.name, l.n, l.k, [l.name]))
+    return out
+
+
 def per_config(dev, peaks, reps=10):
     """Fake-quant linear forward + backward throughput per linear and per config, for the
     bf16 workloads (Llama-2 7B q_proj; 7B MLP w3g128; 13B E2E-QP w2g64 on packed codes;
-    70B block w2g64).  Block-AP: fq_linear_fwd then fq_linear_bwd (dX, dW, ds, dz, W-hat
-    reused); E2E-QP: dq_linear_fwd then dq_linear_bwd_s (dX, ds).  6 M N K per linear;
-    CUDA events around `reps` back-to-back fwd+bwd pairs after 2 warm ones.  Inputs are
-    drawn on the device (seeded); the per-linear bytes exceed L2 for all but the smallest."""
+    70B block w2g64, k_proj and v_proj as one fused kv linear).  Block-AP: fq_linear_fwd
+    then fq_linear_bwd (dX, dW, ds, dz, W-hat reused); E2E-QP: dq_linear_fwd then
+    dq_linear_bwd_s (dX, ds).  6 M N K per linear; CUDA events around `reps`
+    back-to-back fwd+bwd pairs after 2 warm ones, so each linear's timed region is a
+    few ms and its fraction is of the burst bf16 peak.  Inputs are drawn on the device
+    (seeded); the per-linear bytes exceed L2 for all but the smallest."""
     out = {}
     gen = torch.Generator(device=dev)
+    peak = peaks["bf16_tflops"]
     for idx in (2, 3, 4, 5):
         wl = synthetic.WORKLOADS[idx]
         M, b, g = wl.m, wl.bits, wl.group
         lines, tot_flops, tot_ms = {}, 0, 0.0
-        for lin in wl.linears:
-            N, K = lin.n, lin.k
+        for name, N, K, members in fused_linears(wl):
             gen.manual_seed(4000 + 10 * idx + len(lines))
             X = torch.randn(M, K, generator=gen, device=dev).to(torch.bfloat16)
             W = (torch.randn(N, K, generator=gen, device=dev) * wl.sigma).to(torch.bfloat16)
@@ -516,19 +705,74 @@ def per_config(dev, peaks, reps=10):
             torch.cuda.synchronize()
             ms = e0.elapsed_time(e1) / reps
             fl = 6 * M * N * K
-            lines[lin.name] = {"N": N, "K": K, "us": round(ms * 1e3, 1),
-                               "TFLOPs": round(fl / (ms * 1e-3) / 1e12, 1),
-                               "frac_bf16_sustained": round(fl / (ms * 1e-3) / 1e12 / peaks["bf16_tflops_sustained"], 3)}
+            lines[name] = {"N": N, "K": K, "us": round(ms * 1e3, 1),
+                           "TFLOPs": round(fl / (ms * 1e-3) / 1e12, 1),
+                           "frac_bf16_burst": round(fl / (ms * 1e-3) / 1e12 / peak, 3)}
+            if len(members) > 1:
+                lines[name]["fused"] = "+".join(members)
             tot_flops += fl
             tot_ms += ms
             del X, W, dY, ws, Y, out_b
             torch.cuda.empty_cache()
         out[wl.name] = {"M": M, "bits": b, "group": g, "mode": wl.mode, "linears": lines,
                         "TFLOPs": round(tot_flops / (tot_ms * 1e-3) / 1e12, 1),
-                        "frac_bf16_sustained": round(tot_flops / (tot_ms * 1e-3) / 1e12 /
-                                                     peaks["bf16_tflops_sustained"], 3)}
-    out["note"] = "6 M N K per linear (forward + dX + dW-hat), prepasses included; no L2 flush between calls"
+                        "frac_bf16_burst": round(tot_flops / (tot_ms * 1e-3) / 1e12 / peak, 3)}
+    out["peak_TFLOPs"] = peak
+    out["note"] = ("6 M N K per linear (forward + dX + dW-hat), prepasses included; no L2 flush between calls; "
+                   "fractions of the measured burst bf16 peak (each linear's timed region is a few ms)")
     return out
+
+
+def cfg1_latency(dev, reps=50):
+    """The fp32 parity workload (one linear, M = 128, W [512, 256], w2g64), which is
+    latency-bound: median CUDA-event time of each call of the step, alone (each
+    call synchronised), and of the whole step issued back to back."""
+    wl = synthetic.WORKLOADS[1]
+    d = synthetic.workload_linear(wl, 0)
+    X, W, dY = (d[k].to(dev) for k in ("X", "W", "dY"))
+    M, N, K = X.shape[0], W.shape[0], W.shape[1]
+    b, g = wl.bits, wl.group
+    ws = eqat.workspace(M, N, K, b, g, torch.float32, dev)
+    s, z = eqat.minmax_init(W, b, g)
+    codes, zq = eqat.pack_codes(W, s, z, b, g)
+    bufs = dict(Y=torch.empty(M, N, device=dev), out=(torch.empty(M, K, device=dev), torch.empty(N, K, device=dev),
+                                                     torch.empty_like(s), torch.empty_like(s)),
+                out2=(torch.empty(M, K, device=dev), torch.empty_like(s)))
+    calls = {
+        "init": lambda: eqat.minmax_init(W, b, g, s=s, z=z),
+        "fq_fwd": lambda: eqat.fq_linear_fwd(X, W, s, z, b, g, ws=ws, Y=bufs["Y"]),
+        "fq_bwd": lambda: eqat.fq_linear_bwd(X, W, s, z, dY, b, g, ws=ws, out=bufs["out"], w_hat_in_ws=True),
+        "pack": lambda: eqat.pack_codes(W, s, z, b, g, codes=codes, zq=zq),
+        "dq_fwd": lambda: eqat.dq_linear_fwd(X, codes, zq, s, b, g, ws=ws, Y=bufs["Y"]),
+        "dq_bwd": lambda: eqat.dq_linear_bwd_s(X, codes, zq, s, dY, b, g, ws=ws, out=bufs["out2"], w_hat_in_ws=True),
+    }
+    res = {}
+    for name, fn in calls.items():
+        fn()
+        ts = []
+        for _ in range(reps):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            torch.cuda.synchronize()
+            e0.record()
+            fn()
+            e1.record()
+            torch.cuda.synchronize()
+            ts.append(e0.elapsed_time(e1) * 1e3)
+        res[name + "_us"] = round(statistics.median(ts), 2)
+    ts = []
+    for _ in range(reps):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize()
+        e0.record()
+        for fn in calls.values():
+            fn()
+        e1.record()
+        torch.cuda.synchronize()
+        ts.append(e0.elapsed_time(e1) * 1e3)
+    res["step_us"] = round(statistics.median(ts), 2)
+    res.update(workload=wl.name, dtype="f32", note="median CUDA-event time; each call alone, then the six "
+               "calls issued back to back (host launch cost included: the layer is latency-bound)")
+    return res
 
 
 def blockap_block(dev, peaks, steps=5):
@@ -671,59 +915,53 @@ def decode_gemv(dev, peaks, budget_bytes=300_000_000):
     return out
 
 
-def initpack_70b_block(dev, reps=5):
-    """HBM throughput of min-max init and pack over all seven linears of the
-    Llama-2-70B block (855.6 M bf16 weights, w2g64): algorithmic bytes / event time.
-    Before each launch L2 is flushed by a 512 MiB write and then a 256 MiB read of
-    another buffer, so that the kernel starts on clean lines instead of first
-    writing back the flush's dirty ones.  Weights are seeded N(0, 0.015) with 0.1%
-    x10 outliers, drawn on the device."""
+def initpack_70b_block(dev, peaks, reps=5):
+    """HBM throughput of the four quantizer kernels over all seven linears of the
+    Llama-2-70B block (855.6 M bf16 weights, w2g64): min-max init, pack, the Block-AP
+    prepass (W-hat only) and the E2E-QP dequantization of the packed codes.  Per
+    kernel: sum of algorithmic bytes / sum of median CUDA-event times, each launch
+    alone after a clean L2 flush (a 512 MiB write, then a 256 MiB read of another
+    buffer, so the kernel starts on clean lines instead of first writing back the
+    flush's dirty ones).  Weights are seeded N(0, 0.015) with 0.1% x10 outliers,
+    drawn on the device."""
     wl = synthetic.WORKLOADS[5]
     gen = torch.Generator(device=dev)
     gen.manual_seed(1005)
-    flush = torch.empty(512 << 20, dtype=torch.uint8, device=dev)
-    clean = torch.ones(64 << 20, dtype=torch.float32, device=dev)
-
-    def flush_clean():
-        flush.zero_()
-        clean.amax()
-    t_init = t_pack = 0.0
-    b_init = b_pack = 0
+    flush = L2Flush(dev)
+    kinds = ("init", "pack", "prepass", "dequant")
+    t = dict.fromkeys(kinds, 0.0)
+    nbytes = dict.fromkeys(kinds, 0)
+    b, g = wl.bits, wl.group
     for lin in wl.linears:
         N, K = lin.n, lin.k
         W = torch.randn(N, K, generator=gen, device=dev).mul_(wl.sigma)
         idx = torch.randint(0, N * K, ((N * K) // 1000,), generator=gen, device=dev)
         W.view(-1)[idx] *= 10.0
         W = W.to(torch.bfloat16)
-        G = K // wl.group
+        G = K // g
         s = torch.empty((N, G), dtype=torch.float32, device=dev)
         z = torch.empty_like(s)
-        codes = torch.empty((N, eqat.packed_row_bytes(K, wl.bits)), dtype=torch.uint8, device=dev)
+        codes = torch.empty((N, eqat.packed_row_bytes(K, b)), dtype=torch.uint8, device=dev)
         zq = torch.empty((N, G), dtype=torch.uint8, device=dev)
-        bi, bp = phase_bytes(1, N, K, wl.bits, wl.group)
-        for r in range(reps + 1):
-            e = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
-            flush_clean()
-            e[0].record()
-            eqat.minmax_init(W, wl.bits, wl.group, s=s, z=z)
-            e[1].record()
-            flush_clean()
-            e[2].record()
-            eqat.pack_codes(W, s, z, wl.bits, wl.group, codes=codes, zq=zq)
-            e[3].record()
-            torch.cuda.synchronize()
-            if r:  # first round is warm-up
-                t_init += e[0].elapsed_time(e[1]) / reps
-                t_pack += e[2].elapsed_time(e[3]) / reps
-        b_init += bi
-        b_pack += bp
-        del W, s, z, codes, zq
-    return {"workload": wl.name + " (init+pack of all 7 linears, 855.6 M weights)",
-            "init_GBps": round(b_init / (t_init * 1e-3) / 1e9, 1),
-            "pack_GBps": round(b_pack / (t_pack * 1e-3) / 1e9, 1),
-            "init_ms": round(t_init, 4), "pack_ms": round(t_pack, 4),
-            "init_bytes": b_init, "pack_bytes": b_pack,
-            "l2": "flushed by a 512 MiB write, then a 256 MiB read of another buffer, before each launch"}
+        wh = torch.empty_like(W)
+        calls = {
+            "init": lambda: eqat.minmax_init(W, b, g, s=s, z=z),
+            "pack": lambda: eqat.pack_codes(W, s, z, b, g, codes=codes, zq=zq),
+            "prepass": lambda: eqat.fake_quant(W, s, z, b, g, want_code=False, want_mask=False, W_hat=wh),
+            "dequant": lambda: eqat.dequant_codes(codes, zq, s, K, b, g, out=wh),
+        }
+        for k in kinds:  # in this order: pack and dequant read what init and pack wrote
+            t[k] += timed_alone(calls[k], flush, reps)
+            nbytes[k] += hbm_bytes(k, N, K, b, g)
+        del W, s, z, codes, zq, wh
+    torch.cuda.empty_cache()
+    out = {}
+    for k in kinds:
+        gbs = nbytes[k] / (t[k] * 1e-3) / 1e9
+        out[k] = {"GBps": round(gbs, 1), "frac": round(gbs / peaks["hbm_gbs"], 4), "bytes": nbytes[k],
+                  "us": round(t[k] * 1e3, 1)}
+    out["workload"] = wl.name + " (all 7 linears, 855.6 M weights)"
+    return out
 
 
 # ------------------------------------------------------------------------------ oracle arm
@@ -779,12 +1017,115 @@ def cpu_model() -> str:
     return "unknown"
 
 
-def cpu_baseline(target_s: float = 15.0):
+def cpu_baseline(target_s: float = 15.0, plan: bool = True):
     import oracle
     rows = calibrate_rows(target_s)
     dt, flops, desc = oracle_sample(rows)
-    return {"value": round(flops / dt / 1e12, 6), "unit": "TFLOP/s", "cores": oracle.num_threads(),
-            "cpu": cpu_model(), "kind": "oracle", "sample": desc, "seconds": round(dt, 2)}
+    out = {"value": round(flops / dt / 1e12, 6), "unit": "TFLOP/s", "cores": oracle.num_threads(),
+           "cpu": cpu_model(), "kind": "oracle", "sample": desc, "seconds": round(dt, 2)}
+    if plan:
+        out["configs"] = oracle_plan()
+    return out
+
+
+def oracle_step_cfg1(reps=5):
+    """Median seconds of the oracle's whole step on the fp32 parity workload (one
+    linear, M = 128, W [512, 256], w2g64): init, Block-AP forward and backward, pack,
+    E2E-QP forward and backward, every row."""
+    import oracle
+    wl = synthetic.WORKLOADS[1]
+    d = synthetic.workload_linear(wl, 0)
+    X, W, dY = (synthetic.as_f32_numpy(d[k]) for k in ("X", "W", "dY"))
+    b, g = wl.bits, wl.group
+    ts = []
+    for _ in range(reps + 1):
+        t0 = time.perf_counter()
+        s, z = oracle.minmax_init(W, b, g)
+        oracle.fq_linear_fwd(X, W, s, z, b, g)
+        oracle.fq_linear_bwd(X, W, s, z, dY, b, g)
+        packed, zq = oracle.pack(W, s, z, b, g)
+        oracle.dq_linear_fwd(X, packed, zq, s, b, g)
+        oracle.dq_linear_bwd_s(X, packed, zq, s, dY, b, g)
+        ts.append(time.perf_counter() - t0)
+    return statistics.median(ts[1:]), oracle.num_threads()
+
+
+def oracle_linear_times(wl, li, frac, rng):
+    """Seconds of the oracle on one linear of a workload with a `frac` of the token
+    rows (Y, dX) and of the weight rows (dW-hat and the per-group gradients): init
+    and pack of all weights are timed on their own, the rest in one call chain."""
+    import oracle
+    d = synthetic.workload_linear(wl, li)
+    X, W, dY = (synthetic.as_f32_numpy(d[k]) for k in ("X", "W", "dY"))
+    del d
+    M, N = X.shape[0], W.shape[0]
+    b, g = wl.bits, wl.group
+    r = np.sort(rng.choice(M, max(1, int(round(M * frac))), replace=False))
+    wr = np.sort(rng.choice(N, max(1, int(round(N * frac))), replace=False))
+    t0 = time.perf_counter()
+    s, z = oracle.minmax_init(W, b, g)
+    t1 = time.perf_counter()
+    packed, zq = oracle.pack(W, s, z, b, g)
+    t2 = time.perf_counter()
+    if wl.mode == "e2e_qp":
+        oracle.dq_linear_fwd(X, packed, zq, s, b, g, rows=r)
+        oracle.dq_linear_bwd_s(X, packed, zq, s, dY, b, g, rows=r, wrows=wr)
+    else:
+        oracle.fq_linear_fwd(X, W, s, z, b, g, rows=r)
+        oracle.fq_linear_bwd(X, W, s, z, dY, b, g, rows=r, wrows=wr)
+    t3 = time.perf_counter()
+    return t1 - t0, t2 - t1, t3 - t2
+
+
+def oracle_plan(budget_s: float = 120.0):
+    """The oracle's time on the other workloads: the fp32 parity workload in full, on
+    all host threads and on one; the three large bf16 workloads on a sample, with the
+    full problem's time extrapolated.  For each linear the contraction part is timed
+    at two sample fractions f and 2f of the token and weight rows; its cost is a
+    fixed part (W-hat) plus a part linear in f, so the full time is the straight line
+    through the two points at f = 1.  Init and pack run on every weight.  Workloads
+    that would exceed `budget_s` seconds in all are left out and say so."""
+    out = {}
+    t_all, nthr = oracle_step_cfg1()
+    one = None
+    try:
+        r = subprocess.run([sys.executable, os.path.abspath(__file__), "--oracle-cfg1-only"],
+                           env=dict(os.environ, OMP_NUM_THREADS="1", CUDA_VISIBLE_DEVICES=""),
+                           capture_output=True, text=True, timeout=300)
+        one = json.loads(r.stdout.strip().splitlines()[-1]) if r.returncode == 0 else None
+    except (subprocess.TimeoutExpired, ValueError, IndexError):
+        one = None
+    out[synthetic.WORKLOADS[1].name] = {
+        "what": "whole step, every row (init, Block-AP fwd+bwd, pack, E2E-QP fwd+bwd)",
+        "threads_all": {"ms": round(t_all * 1e3, 3), "threads": nthr},
+        "threads_1": {"ms": round(one["seconds"] * 1e3, 3), "threads": one["threads"]} if one else None,
+        "label": "measured"}
+    t_begin = time.perf_counter()
+    rng = np.random.default_rng(11)
+    for idx, f in ((3, 1 / 256), (4, 1 / 256), (5, 1 / 256)):
+        wl = synthetic.WORKLOADS[idx]
+        if time.perf_counter() - t_begin > budget_s:
+            out[wl.name] = {"label": "not run (time budget of the baseline spent)"}
+            continue
+        t0 = time.perf_counter()
+        full = 0.0
+        init_pack = 0.0
+        for li in range(len(wl.linears)):
+            ti, tp, tc1 = oracle_linear_times(wl, li, f, rng)
+            _, _, tc2 = oracle_linear_times(wl, li, 2 * f, rng)
+            slope = max((tc2 - tc1) / f, 0.0)
+            fixed = max(tc1 - slope * f, 0.0)
+            full += ti + tp + fixed + slope
+            init_pack += ti + tp
+        out[wl.name] = {"seconds_full": round(full, 2), "label": "extrapolated",
+                        "init_pack_seconds": round(init_pack, 2),
+                        "seconds_spent": round(time.perf_counter() - t0, 2),
+                        "sample": f"per linear: init+pack of every weight; fwd, dX and weight-side gradients on "
+                                  f"{f:.5f} and {2 * f:.5f} of the token and weight rows, extrapolated to all rows",
+                        "flops_full": wl.flops_per_step(),
+                        "TFLOPs_extrapolated": round(wl.flops_per_step() / full / 1e12, 6),
+                        "threads": nthr}
+    return out
 
 
 def run_reference(args):
@@ -808,7 +1149,7 @@ def run_reference(args):
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(sec * 1e3, 2),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic",
-            "config": {"workload": wl.name, "M": wl.m, "N": lin.n, "K": lin.k, "bits": wl.bits, "group": wl.group},
+            "config": bench_config(args.gpus),
             "cpu_baseline": {"value": round(value, 6), "unit": "TFLOP/s", "cores": oracle.num_threads(),
                              "cpu": cpu_model(), "kind": "oracle", "sample": desc},
             "e2e": {"value": round(value, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
@@ -834,7 +1175,15 @@ def main():
     ap.add_argument("--configs-only", action="store_true")
     ap.add_argument("--initpack70b-only", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--no-hbm", action="store_true")
+    ap.add_argument("--no-cfg1", action="store_true")
+    ap.add_argument("--no-oracle-plan", action="store_true")
+    ap.add_argument("--oracle-cfg1-only", action="store_true")
     args = ap.parse_args()
+    if args.oracle_cfg1_only:  # the oracle's fp32 parity step, in a process of its own (its thread count)
+        sec, thr = oracle_step_cfg1()
+        print(json.dumps({"seconds": sec, "threads": thr}), flush=True)
+        return
     args.warmup = max(3, args.warmup)  # timing rule: at least 3 untimed warm-up steps
     if args.configs_only:  # the per-config table alone
         torch.cuda.set_device(0)
@@ -869,7 +1218,7 @@ def main():
     if args.initpack70b_only:  # profiling aid: just the 70B-block init/pack measurement
         torch.cuda.set_device(0)
         eqat.load_library()
-        print(json.dumps(initpack_70b_block(torch.device("cuda", 0), reps=1)), flush=True)
+        print(json.dumps(initpack_70b_block(torch.device("cuda", 0), load_peaks(), reps=1)), flush=True)
         return
     if args.impl == "reference":
         run_reference(args)

@@ -279,7 +279,10 @@ double eqat_cosine_lr(double lr0, double lr_min, int64_t step, int64_t total);
  * fp32 weights); larger layers are rejected with EQAT_ERR_WORKSPACE before
  * anything is launched.  The first call on a device looks up the array's device
  * address (cudaGetSymbolAddress), so make that first call before any stream
- * capture.  Every call shares the one array: calls whose kernels overlap on the
+ * capture.  That address is cached per device for the life of the process, so a
+ * cudaDeviceReset (or any reset of the primary context) is not supported once
+ * this entry point has run on that device: later calls would use the stale
+ * address.  Every call shares the one array: calls whose kernels overlap on the
  * GPU (other streams, other host threads) race on it and must be serialised by
  * the caller.  Arguments, layout and the result are those of eqat_fq_linear_fwd. */
 #define EQAT_NOALLOC_SCRATCH_BYTES 33554432u

@@ -169,3 +169,39 @@ def test_blockap_entry_points_argument_errors(lib):
     assert abs(eqat.cosine_lr(1e-4, 0.0, 0, 10) - 1e-4) < 1e-18
     assert abs(eqat.cosine_lr(1e-4, 0.0, 10, 10)) < 1e-18
     assert abs(eqat.cosine_lr(1e-4, 1e-6, 5, 10) - (1e-6 + (1e-4 - 1e-6) / 2)) < 1e-15
+
+
+def test_binding_refuses_wrong_shapes_before_the_library():
+    """The C ABI sees only pointers and sizes, so the binding must refuse an
+    undersized or mis-shaped buffer itself (it would be read or written out of
+    bounds on the device).  The checks run before the device checks, so they are
+    exercised here on CPU tensors."""
+    import torch
+    bf, f32, u8 = torch.bfloat16, torch.float32, torch.uint8
+    M, N, K, g, b = 8, 16, 128, 64, 2
+    X, W = torch.zeros(M, K, dtype=bf), torch.zeros(N, K, dtype=bf)
+    s, z = torch.zeros(N, K // g, dtype=f32), torch.zeros(N, K // g, dtype=f32)
+    codes, zq = torch.zeros(N, K // 4, dtype=u8), torch.zeros(N, K // g, dtype=u8)
+    Y_bad = torch.zeros(M, N - 8, dtype=bf)
+    cases = [
+        lambda: eqat.fq_linear_fwd_noalloc(X, W, s, z, b, g, Y=Y_bad),
+        lambda: eqat.fq_linear_fwd(X, W, s, z, b, g, Y=Y_bad),
+        lambda: eqat.fq_linear_fwd(X, W, s[:, :1], z, b, g),
+        lambda: eqat.fq_linear_fwd(X, torch.zeros(N, K - 64, dtype=bf), s, z, b, g),
+        lambda: eqat.fq_linear_bwd(X, W, s, z, torch.zeros(M, N + 8, dtype=bf), b, g),
+        lambda: eqat.fq_linear_bwd(X, W, s, z, torch.zeros(M, N, dtype=bf), b, g,
+                                   out=(torch.zeros(M, K - 8, dtype=bf), None, None, None)),
+        lambda: eqat.dq_linear_fwd(X, codes[:, :-1], zq, s, b, g),
+        lambda: eqat.dq_linear_fwd(X, codes, zq[:-8], s, b, g),
+        lambda: eqat.dq_linear_bwd_s(X, codes, zq, s, torch.zeros(M, N, dtype=bf), b, g,
+                                     out=(None, torch.zeros(N, 1, dtype=f32))),
+        lambda: eqat.dq_linear_bwd(X, codes, zq, s, Y_bad, b, g),
+        lambda: eqat.fq_linear_fwd_mse(X, W, s, z, Y_bad, b, g),
+        lambda: eqat.pack_codes(W, s, z, b, g, codes=torch.zeros(N, K // 8, dtype=u8)),
+        lambda: eqat.minmax_init(W, b, g, s=torch.zeros(N, 1, dtype=f32)),
+        lambda: eqat.fake_quant(W, s[:8], z, b, g),
+        lambda: eqat.dequant_codes(codes, zq, s[:, :1], K, b, g),
+    ]
+    for i, call in enumerate(cases):
+        with pytest.raises(ValueError, match="shape|in-features|2-D"):
+            call()

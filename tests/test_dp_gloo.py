@@ -79,7 +79,11 @@ def reducer_worker(rank, world, port, out):
         for i, ts in enumerate(layers):
             red.submit(ts + [None], tag=i)
         red.wait()
-        out[rank] = ([[t.numpy() for t in ts] for ts in before], [[t.numpy() for t in ts] for ts in layers], red.order)
+        # the helper with op="mean" scales the same way as the reducer
+        meaned = [t.clone() for t in before[0]]
+        dp.allreduce_weight_grads(meaned + [None], dist, op="mean")
+        out[rank] = ([[t.numpy() for t in ts] for ts in before], [[t.numpy() for t in ts] for ts in layers], red.order,
+                     [t.numpy() for t in meaned])
     finally:
         dist.destroy_process_group()
 
@@ -92,8 +96,10 @@ def test_overlapped_reducer_averages_each_layer_in_order():
     mp.spawn(reducer_worker, args=(world, free_port(), out), nprocs=world, join=True)
     before = [out[r][0] for r in range(world)]
     for r in range(world):
-        _, after, order = out[r]
+        _, after, order, meaned = out[r]
         assert order == [0, 1, 2]
+        for j in range(3):
+            np.testing.assert_array_equal(meaned[j], after[0][j])
         for i in range(3):
             for j in range(3):
                 mean = (before[0][i][j] + before[1][i][j]) / 2

@@ -157,6 +157,73 @@ def test_blockap_steps_match_oracle(orc):
         assert (to_np(L.W) == bf16_round(to_np(L.W_master))).all()
 
 
+def test_blockap_steps_trained_state_match_oracle_per_element(orc):
+    """Three composed steps from a trained-like state (s shrunk, z shifted: a few
+    percent of the weights clamp, so dz != 0 and z must move), with a per-element
+    bound on the moves of W, s and z against the oracle.
+
+    Elements whose oracle gradient stays well away from zero at every step (at least
+    a tenth of that step's largest gradient of the tensor) must move as the oracle's
+    do to within a tenth of one learning-rate step per step; there the bf16 GEMMs'
+    error cannot flip the sign of Adam's update.  The rest (gradients within
+    rounding of zero) keep the global bound of one flipped update per step."""
+    cfg = BlockAPConfig(bits=2, group=64, total_steps=10, weight_decay=0.0)
+    M = 192
+    shapes = [(136, 256), (264, 384)]
+    rng = np.random.default_rng(123)
+    lin, Xs, Ts, ref = [], [], [], []
+    for i, (N, K) in enumerate(shapes):
+        d = synthetic.draw_linear(rng, M, N, K, 0.02, "bf16")
+        Xn, Wn = synthetic.as_f32_numpy(d["X"]), synthetic.as_f32_numpy(d["W"])
+        T = fp_target(Xn, Wn, "bf16")
+        L = QuantLinearState.from_weight(d["W"].float().cuda(), cfg.bits, cfg.group, M)
+        s0, z0 = orc.minmax_init(Wn, cfg.bits, cfg.group)
+        s0, z0 = synthetic.perturb_quant_params(s0, z0, 31 + i)
+        L.s.copy_(torch.from_numpy(s0))
+        L.z.copy_(torch.from_numpy(z0))
+        lin.append(L)
+        Xs.append(d["X"].cuda())
+        Ts.append(T.cuda())
+        ref.append({"X": Xn, "T": synthetic.as_f32_numpy(T), "W": Wn.copy(), "s": s0.copy(), "z": z0.copy(),
+                    "mW": np.zeros_like(Wn), "vW": np.zeros_like(Wn), "ms": np.zeros_like(s0),
+                    "vs": np.zeros_like(s0), "mz": np.zeros_like(z0), "vz": np.zeros_like(z0),
+                    "g": {"W": [], "s": [], "z": []}})
+    start = [(r["W"].copy(), r["s"].copy(), r["z"].copy()) for r in ref]
+    for t in range(1, 4):
+        blockap_step(lin, Xs, Ts, cfg, t)
+        lr_w = orc.cosine_lr(cfg.lr_w, cfg.lr_min, t - 1, cfg.total_steps)
+        lr_q = orc.cosine_lr(cfg.lr_q, cfg.lr_min, t - 1, cfg.total_steps)
+        for r in ref:
+            Wb = bf16_round(r["W"])
+            Y = orc.fq_linear_fwd(r["X"], Wb, r["s"], r["z"], cfg.bits, cfg.group)
+            _, dY = orc.mse_grad(Y, r["T"])
+            dwh = orc.linear_dwhat(dY.astype(np.float32), r["X"])
+            dW, ds, dz = orc.ste_grads(Wb, r["s"], r["z"], dwh, cfg.bits, cfg.group)
+            for name, g in (("W", dW), ("s", ds), ("z", dz)):
+                r["g"][name].append(np.asarray(g, dtype=np.float64))
+            r["W"], r["mW"], r["vW"] = orc.adamw(r["W"], dW, r["mW"], r["vW"], lr_w, 0.9, 0.999, 1e-8, 0.0, t)
+            r["s"], r["ms"], r["vs"] = orc.adamw(r["s"], ds, r["ms"], r["vs"], lr_q, 0.9, 0.999, 1e-8, 0.0, t)
+            r["z"], r["mz"], r["vz"] = orc.adamw(r["z"], dz, r["mz"], r["vz"], lr_q, 0.9, 0.999, 1e-8, 0.0, t)
+    for i, (L, r) in enumerate(zip(lin, ref)):
+        assert np.abs(np.stack(r["g"]["z"])).max() > 0, "the trained-state case must clamp"
+        for name, got, lr in (("W", to_np(L.W_master), cfg.lr_w), ("s", to_np(L.s), cfg.lr_q),
+                              ("z", to_np(L.z), cfg.lr_q)):
+            st = start[i][{"W": 0, "s": 1, "z": 2}[name]]
+            move_g, move_r = got - st, r[name] - st
+            gs = np.stack(r["g"][name])  # [steps, ...]
+            scale = np.abs(gs).reshape(gs.shape[0], -1).max(axis=1).reshape((-1,) + (1,) * (gs.ndim - 1))
+            firm = (np.abs(gs) >= 0.1 * scale).all(axis=0)
+            err = np.abs(move_g - move_r)
+            assert firm.mean() > 0.05, f"{name}: too few elements with firm gradients ({firm.mean():.3f})"
+            assert err[firm].max() <= 0.1 * 3 * lr, \
+                f"{name}: move error {err[firm].max():.3e} on firm elements > {0.3 * lr:.3e}"
+            assert err.max() <= 2.01 * 3 * lr
+            if name == "z":
+                moved = firm & (np.abs(move_r) > 0.5 * lr)
+                assert moved.any() and (np.abs(move_g[moved]) > 0.5 * lr).all(), "z must move where the oracle's does"
+        assert (to_np(L.W) == bf16_round(to_np(L.W_master))).all()
+
+
 def test_blockap_step_with_overlapped_reducer_single_rank():
     """The NCCL stream plumbing of the overlapped gradient exchange, on one rank (the mean
     over one rank is the identity): the step gives the same state as without it."""

@@ -131,6 +131,30 @@ def _req(t, name, dtype=None):
     return t
 
 
+def _shape(t, name, shape):
+    """Refuses a tensor whose shape is not `shape` before any pointer reaches the
+    library: the C ABI sees only pointers and sizes, so an undersized buffer would
+    otherwise be read or written out of bounds on the device."""
+    if t is None:
+        return
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
+
+
+def _linear_shapes(X, W_rows, K_w, group):
+    """(M, N, K, G) of a linear layer; X is [M, K] and the weight side [N, K_w]."""
+    if X.dim() != 2:
+        raise ValueError(f"X must be 2-D [M, K], got shape {tuple(X.shape)}")
+    M, K = X.shape
+    if K_w != K:
+        raise ValueError(f"the weight has {K_w} in-features, X has {K}")
+    if group <= 0 or K % group:
+        raise ValueError(f"K = {K} is not a multiple of group = {group}")
+    return M, W_rows, K, K // group
+
+
 def packed_row_bytes(K: int, bits: int) -> int:
     return K // 4 if bits == 2 else K // 2 if bits == 4 else K
 
@@ -155,20 +179,26 @@ def _ws(ws, M, N, K, bits, group, dtype, device):
 
 def minmax_init(W, bits, group, s=None, z=None):
     """Per-group min-max init: returns (s, z) fp32 [N, K/group]."""
-    _req(W, "W")
     N, K = W.shape
     G = K // group if group else 0
+    _shape(s, "s", (N, G)); _shape(z, "z", (N, G))
+    _req(W, "W")
     s = torch.empty((N, G), dtype=torch.float32, device=W.device) if s is None else _req(s, "s", torch.float32)
     z = torch.empty((N, G), dtype=torch.float32, device=W.device) if z is None else _req(z, "z", torch.float32)
     _call("eqat_minmax_init", _p(W), _dt(W), N, K, bits, group, _p(s), _p(z), _stream())
     return s, z
 
 
-def fake_quant(W, s, z, bits, group, want_w_hat=True, want_code=True, want_mask=True):
-    """Quantizer prepass: returns (W_hat (W's dtype), code uint8, mask uint8), None where not wanted."""
-    _req(W, "W"); _req(s, "s", torch.float32); _req(z, "z", torch.float32)
+def fake_quant(W, s, z, bits, group, want_w_hat=True, want_code=True, want_mask=True, W_hat=None):
+    """Quantizer prepass: returns (W_hat (W's dtype), code uint8, mask uint8), None where not wanted.
+    W_hat, if given, receives the fake-quantized weight (it is then always written)."""
     N, K = W.shape
-    wh = torch.empty_like(W) if want_w_hat else None
+    _shape(s, "s", (N, K // group)); _shape(z, "z", (N, K // group)); _shape(W_hat, "W_hat", (N, K))
+    _req(W, "W"); _req(s, "s", torch.float32); _req(z, "z", torch.float32)
+    if W_hat is not None:
+        wh = _req(W_hat, "W_hat", W.dtype)
+    else:
+        wh = torch.empty_like(W) if want_w_hat else None
     code = torch.empty((N, K), dtype=torch.uint8, device=W.device) if want_code else None
     mask = torch.empty((N, K), dtype=torch.uint8, device=W.device) if want_mask else None
     _call("eqat_fake_quant", _p(W), _dt(W), _p(s), _p(z), N, K, bits, group, _p(wh), _p(code), _p(mask),
@@ -178,8 +208,10 @@ def fake_quant(W, s, z, bits, group, want_w_hat=True, want_code=True, want_mask=
 
 def pack_codes(W, s, z, bits, group, codes=None, zq=None):
     """Pack to low-bit integers: returns (codes uint8 [N, row_bytes], zq uint8 [N, K/group])."""
-    _req(W, "W"); _req(s, "s", torch.float32); _req(z, "z", torch.float32)
     N, K = W.shape
+    _shape(s, "s", (N, K // group)); _shape(z, "z", (N, K // group))
+    _shape(codes, "codes", (N, packed_row_bytes(K, bits))); _shape(zq, "zq", (N, K // group))
+    _req(W, "W"); _req(s, "s", torch.float32); _req(z, "z", torch.float32)
     if codes is None:
         codes = torch.empty((N, packed_row_bytes(K, bits)), dtype=torch.uint8, device=W.device)
     if zq is None:
@@ -189,19 +221,49 @@ def pack_codes(W, s, z, bits, group, codes=None, zq=None):
     return codes, zq
 
 
-def dequant_codes(codes, zq, s, K, bits, group, dtype=torch.bfloat16):
-    """E2E-QP dequant of frozen codes: W_hat = (W_q - zq) s, [N, K] of `dtype`.
-    s is fp32 or fp16 (fp16 step-size storage)."""
-    _req(codes, "codes", torch.uint8); _req(zq, "zq", torch.uint8); _req(s, "s")
+def dequant_codes(codes, zq, s, K, bits, group, dtype=torch.bfloat16, out=None):
+    """E2E-QP dequant of frozen codes: W_hat = (W_q - zq) s, [N, K] of `dtype` (or into
+    `out`, whose dtype then decides).  s is fp32 or fp16 (fp16 step-size storage)."""
     N = codes.shape[0]
-    wh = torch.empty((N, K), dtype=dtype, device=codes.device)
+    _shape(codes, "codes", (N, packed_row_bytes(K, bits))); _shape(zq, "zq", (N, K // group))
+    _shape(s, "s", (N, K // group)); _shape(out, "out", (N, K))
+    _req(codes, "codes", torch.uint8); _req(zq, "zq", torch.uint8); _req(s, "s")
+    wh = torch.empty((N, K), dtype=dtype, device=codes.device) if out is None else _req(out, "out")
     _call("eqat_dequant_codes_ex", _p(codes), _p(zq), _p(s), _sdt(s), N, K, bits, group, _p(wh), _dt(wh),
           _stream())
     return wh
 
 
+def _fq_shapes(X, W, s, z, group, **mn):
+    """Shapes of a Block-AP call: W [N, K], s and z [N, K/group], and each [M, N]
+    tensor of `mn` (Y, dY, T)."""
+    if W.dim() != 2:
+        raise ValueError(f"W must be 2-D [N, K], got shape {tuple(W.shape)}")
+    M, N, K, G = _linear_shapes(X, W.shape[0], W.shape[1], group)
+    _shape(s, "s", (N, G)); _shape(z, "z", (N, G))
+    for name, t in mn.items():
+        _shape(t, name, (M, N))
+    return M, N, K, G
+
+
+def _dq_shapes(X, codes, zq, s, bits, group, **mn):
+    """Shapes of an E2E-QP call: codes [N, packed row bytes of K], zq and s
+    [N, K/group], and each [M, N] tensor of `mn`."""
+    if codes.dim() != 2:
+        raise ValueError(f"codes must be 2-D [N, row bytes], got shape {tuple(codes.shape)}")
+    if X.dim() != 2:
+        raise ValueError(f"X must be 2-D [M, K], got shape {tuple(X.shape)}")
+    M, N, K, G = _linear_shapes(X, codes.shape[0], X.shape[1], group)
+    _shape(codes, "codes", (N, packed_row_bytes(K, bits)))
+    _shape(zq, "zq", (N, G)); _shape(s, "s", (N, G))
+    for name, t in mn.items():
+        _shape(t, name, (M, N))
+    return M, N, K, G
+
+
 def fq_linear_fwd(X, W, s, z, bits, group, ws=None, Y=None):
     """Block-AP forward Y = X W_hat^T."""
+    _fq_shapes(X, W, s, z, group, Y=Y)
     _req(X, "X"); _req(W, "W", X.dtype); _req(s, "s", torch.float32); _req(z, "z", torch.float32)
     M, K = X.shape
     N = W.shape[0]
@@ -217,6 +279,9 @@ def fq_linear_fwd_noalloc(X, W, s, z, bits, group, Y):
     the library's static 32 MiB device scratch (N*K*sizeof(dtype) must fit).  The
     output Y is the caller's.  Calls that overlap on the GPU share that scratch and
     race; serialise them."""
+    if Y is None:
+        raise ValueError("Y is required: this entry point allocates nothing")
+    _fq_shapes(X, W, s, z, group, Y=Y)
     _req(X, "X"); _req(W, "W", X.dtype); _req(s, "s", torch.float32); _req(z, "z", torch.float32)
     _req(Y, "Y", X.dtype)
     M, K = X.shape
@@ -231,6 +296,10 @@ def fq_linear_bwd(X, W, s, z, dY, bits, group, need_dx=True, need_dw=True, need_
     """Block-AP straight-through backward: returns (dX, dW, ds, dz), None where not requested.
     w_hat_in_ws=True reuses the W-hat that fq_linear_fwd left in `ws` (same W, s, z).
     clamp_pass=True lets the clamp pass the gradient too (EQAT_GRAD_CLAMP_PASS)."""
+    M, N, K, G = _fq_shapes(X, W, s, z, group, dY=dY)
+    if out is not None:
+        _shape(out[0], "dX", (M, K)); _shape(out[1], "dW", (N, K))
+        _shape(out[2], "ds", (N, G)); _shape(out[3], "dz", (N, G))
     _req(X, "X"); _req(W, "W", X.dtype); _req(s, "s", torch.float32); _req(z, "z", torch.float32)
     _req(dY, "dY", X.dtype)
     M, K = X.shape
@@ -255,6 +324,7 @@ def fq_linear_bwd(X, W, s, z, dY, bits, group, need_dx=True, need_dw=True, need_
 
 def dq_linear_fwd(X, codes, zq, s, bits, group, ws=None, Y=None):
     """E2E-QP forward on frozen codes: Y = X ((W_q - zq) s)^T; s fp32 or fp16."""
+    _dq_shapes(X, codes, zq, s, bits, group, Y=Y)
     _req(X, "X"); _req(codes, "codes", torch.uint8); _req(zq, "zq", torch.uint8); _req(s, "s")
     M, K = X.shape
     N = codes.shape[0]
@@ -269,6 +339,9 @@ def dq_linear_bwd_s(X, codes, zq, s, dY, bits, group, need_dx=True, need_ds=True
                     w_hat_in_ws=False):
     """E2E-QP backward (scales only): returns (dX, ds).  w_hat_in_ws=True reuses the
     W-hat that dq_linear_fwd left in `ws`."""
+    M, N, K, G = _dq_shapes(X, codes, zq, s, bits, group, dY=dY)
+    if out is not None:
+        _shape(out[0], "dX", (M, K)); _shape(out[1], "ds", (N, G))
     _req(X, "X"); _req(codes, "codes", torch.uint8); _req(zq, "zq", torch.uint8); _req(s, "s", torch.float32)
     _req(dY, "dY", X.dtype)
     M, K = X.shape
@@ -290,6 +363,9 @@ def dq_linear_bwd(X, codes, zq, s, dY, bits, group, need_dx=True, need_ds=True, 
                   out=None, w_hat_in_ws=False):
     """E2E-QP backward with the zero-point gradient: returns (dX, ds, dz), None where not
     requested; dz = -s sum_group dY^T X.  s fp32 or fp16."""
+    M, N, K, G = _dq_shapes(X, codes, zq, s, bits, group, dY=dY)
+    if out is not None:
+        _shape(out[0], "dX", (M, K)); _shape(out[1], "ds", (N, G)); _shape(out[2], "dz", (N, G))
     _req(X, "X"); _req(codes, "codes", torch.uint8); _req(zq, "zq", torch.uint8); _req(s, "s")
     _req(dY, "dY", X.dtype)
     M, K = X.shape
@@ -312,6 +388,8 @@ def dq_linear_bwd(X, codes, zq, s, dY, bits, group, need_dx=True, need_ds=True, 
 def fq_linear_fwd_mse(X, W, s, z, T, bits, group, ws=None, dY=None, loss=None):
     """Block-AP forward against the full-precision output T, Y not stored: returns
     (dY = 2 (Y - T) / (M N), loss = mean (Y - T)^2 as a 1-element fp64 CUDA tensor)."""
+    M, N, K, G = _fq_shapes(X, W, s, z, group, T=T, dY=dY)
+    _shape(loss, "loss", (1,))
     _req(X, "X"); _req(W, "W", X.dtype); _req(s, "s", torch.float32); _req(z, "z", torch.float32)
     _req(T, "T", X.dtype)
     M, K = X.shape

@@ -3,7 +3,18 @@
 Every rank holds the same W, s, z (or frozen codes) and its own batch of tokens.
 The forward and the input gradient are rank-local; the weight-side gradients
 dW, ds, dz (Block-AP) and ds (E2E-QP) are sums over tokens, hence over ranks, and
-are the layer's one exchange: an all-reduce (sum) after the backward.
+are the layer's one exchange: an all-reduce after the backward.
+
+The two helpers scale differently, on purpose:
+
+* allreduce_weight_grads(..., op="sum") SUMS over ranks (the default): the
+  gradient of a loss that is a sum over every rank's tokens (the bench step's
+  dY is a per-token gradient, so the sum is the full-batch gradient).
+* OverlappedGradReducer AVERAGES over ranks: the Block-AP loss is a mean over
+  tokens, and each rank's dY already carries 1 / (its own tokens), so the mean of
+  the ranks' gradients is the gradient of the mean over all tokens.
+
+allreduce_weight_grads(..., op="mean") gives the reducer's scaling in one call.
 """
 from __future__ import annotations
 
@@ -22,11 +33,18 @@ def rank_batch(wl: synthetic.Workload, li: int, rank: int, m: int | None = None)
     return d
 
 
-def allreduce_weight_grads(tensors, dist, group=None) -> None:
-    """Sums the weight-side gradients over ranks in place (None entries skipped)."""
+def allreduce_weight_grads(tensors, dist, group=None, op: str = "sum") -> None:
+    """All-reduces the weight-side gradients over ranks in place (None entries
+    skipped): op="sum" adds them, op="mean" adds them and divides by the number
+    of ranks (the scaling of OverlappedGradReducer)."""
+    if op not in ("sum", "mean"):
+        raise ValueError(f"op must be 'sum' or 'mean', got {op!r}")
+    world = dist.get_world_size(group)
     for t in tensors:
         if t is not None:
             dist.all_reduce(t, op=dist.ReduceOp.SUM, group=group)
+            if op == "mean" and world > 1:
+                t.mul_(1.0 / world)
 
 
 class OverlappedGradReducer:

@@ -162,10 +162,12 @@ def test_blockap_steps_trained_state_match_oracle_per_element(orc):
     percent of the weights clamp, so dz != 0 and z must move), with a per-element
     bound on the moves of W, s and z against the oracle.
 
-    Elements whose oracle gradient stays well away from zero at every step (at least
-    a tenth of that step's largest gradient of the tensor) must move as the oracle's
-    do to within a tenth of one learning-rate step per step; there the bf16 GEMMs'
-    error cannot flip the sign of Adam's update.  The rest (gradients within
+    Elements whose oracle gradient stays well away from zero at every step must move
+    as the oracle's do to within a tenth of one learning-rate step per step; there the
+    kernels' error cannot flip the sign of Adam's update.  "Well away" is measured
+    against each tensor's own largest gradient at that step, at the scale of its
+    tolerance: a tenth of it for dW (bf16 GEMM, 2e-2 of the largest), a hundredth for
+    ds and dz (fp32 reductions, 1e-3 of the largest).  The rest (gradients within
     rounding of zero) keep the global bound of one flipped update per step."""
     cfg = BlockAPConfig(bits=2, group=64, total_steps=10, weight_decay=0.0)
     M = 192
@@ -206,15 +208,15 @@ def test_blockap_steps_trained_state_match_oracle_per_element(orc):
             r["z"], r["mz"], r["vz"] = orc.adamw(r["z"], dz, r["mz"], r["vz"], lr_q, 0.9, 0.999, 1e-8, 0.0, t)
     for i, (L, r) in enumerate(zip(lin, ref)):
         assert np.abs(np.stack(r["g"]["z"])).max() > 0, "the trained-state case must clamp"
-        for name, got, lr in (("W", to_np(L.W_master), cfg.lr_w), ("s", to_np(L.s), cfg.lr_q),
-                              ("z", to_np(L.z), cfg.lr_q)):
+        for name, got, lr, frac in (("W", to_np(L.W_master), cfg.lr_w, 0.1), ("s", to_np(L.s), cfg.lr_q, 0.01),
+                                    ("z", to_np(L.z), cfg.lr_q, 0.01)):
             st = start[i][{"W": 0, "s": 1, "z": 2}[name]]
             move_g, move_r = got - st, r[name] - st
             gs = np.stack(r["g"][name])  # [steps, ...]
             scale = np.abs(gs).reshape(gs.shape[0], -1).max(axis=1).reshape((-1,) + (1,) * (gs.ndim - 1))
-            firm = (np.abs(gs) >= 0.1 * scale).all(axis=0)
+            firm = (np.abs(gs) >= frac * scale).all(axis=0)
             err = np.abs(move_g - move_r)
-            assert firm.mean() > 0.05, f"{name}: too few elements with firm gradients ({firm.mean():.3f})"
+            assert firm.sum() >= 16, f"{name}: too few elements with firm gradients ({firm.sum()} of {firm.size})"
             assert err[firm].max() <= 0.1 * 3 * lr, \
                 f"{name}: move error {err[firm].max():.3e} on firm elements > {0.3 * lr:.3e}"
             assert err.max() <= 2.01 * 3 * lr

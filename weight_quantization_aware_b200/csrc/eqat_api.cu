@@ -131,6 +131,52 @@ bool gemv_enabled() {
     return on;
 }
 
+// Dequantize on load in the E2E-QP contractions (bf16): the pair GEMM makes W-hat
+// from the codes in shared memory instead of reading a W-hat that the dequantize
+// kernel wrote to the workspace.  Each B tile is converted once per 256-row M tile,
+// so the conversion work is M / 256 times the dequantize kernel's, while the HBM it
+// saves (a 2-byte W-hat written and read back, 0.25-1 byte codes read instead) does
+// not grow with M.  Measured on B200 (forward, w2g64 / w3g128): with one M tile
+// (M <= 256) it is 1.5x faster on a 13824 x 5120 layer, 1.2x on 28672 x 8192, about
+// even on 11008 x 4096 (3-bit) and 0.8x on 4096 x 4096, where few N tiles leave most
+// SMs idle;
+// at M >= 512 the dequantize + GEMM path wins (0.55-0.9x at M = 4096).  So it is used
+// for M <= 256 on layers of 2^25 weights or more.  The decision depends only on the
+// shapes, so a backward with w_hat_in_ws takes the same path as its forward.
+// EQAT_DQ_ONLOAD=1 uses it wherever the code layout allows, EQAT_DQ_ONLOAD=0 never
+// (measurement aids and the tests' way to compare the two paths).
+int onload_mode() {
+    static const int mode = [] {
+        const char *v = std::getenv("EQAT_DQ_ONLOAD");
+        if (v && v[0] == '0') return 0;
+        if (v && v[0] == '1') return 1;
+        return -1;  // by shape
+    }();
+    return mode;
+}
+
+bool use_onload(int64_t M, int64_t N, int64_t K, int bits, int group) {
+    if (!eqat::cvt_supported(N, K, bits, group)) return false;
+    const int mode = onload_mode();
+    if (mode >= 0) return mode == 1;
+    return M <= 256 && N * K >= (int64_t(1) << 25);
+}
+
+eqat::CvtArgs cvt_args(const uint8_t *codes, const uint8_t *zq, const void *s, int sdt, int64_t N, int64_t K,
+                       int bits, int group) {
+    eqat::CvtArgs c;
+    c.on = true;
+    c.codes = codes;
+    c.zq = zq;
+    c.s = s;
+    c.s_f16 = sdt == EQAT_F16;
+    c.bits = bits;
+    c.group = group;
+    c.w_rows = N;
+    c.w_cols = K;
+    return c;
+}
+
 int64_t code_bytes(int64_t N, int64_t K, int bits) {
     return bits == 2 ? N * (K / 4) : bits == 4 ? N * (K / 2) : N * K;
 }
@@ -444,13 +490,20 @@ eqat_status eqat_dq_linear_fwd_ex(const void *X, int dt, const uint8_t *codes, c
                   "dq GEMV");
         return EQAT_OK;
     }
-    EQAT_CUDA(eqat::launch_dequant(codes, zq, s, sdt == EQAT_F16, N, K, bits, group, ws, f32, dev, st),
-              "dequant prepass");
     EpiArgs epi;
     epi.kind = Epi::kStore;
     epi.out = Y;
     epi.ldo = N;
     epi.out_f32 = f32;
+    if (!f32 && use_onload(M, N, K, bits, group)) {
+        // W-hat made from the codes inside the contraction, never written to HBM
+        eqat::GemmProblem g{Operand{X, K, false}, Operand{nullptr, K, false}, M, N, K, epi};
+        g.cvt = cvt_args(codes, zq, s, sdt, N, K, bits, group);
+        EQAT_CUDA(eqat::launch_gemm_tc_group(&g, 1, dev, st), "dq forward contraction (dequantize on load)");
+        return EQAT_OK;
+    }
+    EQAT_CUDA(eqat::launch_dequant(codes, zq, s, sdt == EQAT_F16, N, K, bits, group, ws, f32, dev, st),
+              "dequant prepass");
     EQAT_CUDA(contract(dt, Operand{X, K, false}, Operand{ws, K, false}, M, N, K, epi, nullptr, dev, st),
               "dq forward contraction");
     return EQAT_OK;
@@ -510,7 +563,8 @@ eqat_status eqat_dq_linear_bwd(const void *X, int dt, const uint8_t *codes, cons
         if (N == 0) {
             EQAT_CUDA(zero(dX, static_cast<size_t>(M * K) * esize(dt), st), "memset dX");
         } else {
-            if (!w_hat_in_ws)
+            const bool onload = !f32 && use_onload(M, N, K, bits, group);
+            if (!w_hat_in_ws && !onload)
                 EQAT_CUDA(eqat::launch_dequant(codes, zq, s, sdt == EQAT_F16, N, K, bits, group, ws, f32, dev, st),
                           "dequant prepass");
             EpiArgs epi;
@@ -518,7 +572,10 @@ eqat_status eqat_dq_linear_bwd(const void *X, int dt, const uint8_t *codes, cons
             epi.out = dX;
             epi.ldo = K;
             epi.out_f32 = f32;
-            probs[np++] = eqat::GemmProblem{Operand{dY, N, false}, Operand{ws, K, true}, M, K, N, epi};
+            probs[np] = eqat::GemmProblem{Operand{dY, N, false}, Operand{ws, K, true}, M, K, N, epi};
+            // dX = dY W-hat with W-hat made from the codes on load (MN-major B)
+            if (onload) probs[np].cvt = cvt_args(codes, zq, s, sdt, N, K, bits, group);
+            ++np;
         }
     }
     if (np == 0) return EQAT_OK;

@@ -82,6 +82,14 @@ struct Prob {
     int group;
     int gshift;  // log2(group)
     float Q;
+    // B made on load from packed codes (pair kernel, CVT variants): W-hat [w_rows, w_cols]
+    // = (W_q - zq) s, converted in shared memory from the code tile that B's tensor map
+    // (then a map of the codes) brings in
+    int b_cvt;
+    int w_rows, w_cols, w_groups;
+    const uint8_t *cvt_zq;
+    const void *cvt_s;
+    int cvt_s_f16;
 };
 
 struct KParams {
@@ -91,6 +99,7 @@ struct KParams {
     int split_begin;  // pair kernel, one problem: tiles from here on are halves (-1: none)
     int *err;
     uint64_t wait_limit_ns;
+    int cvt_cluster_scope;  // converter hand-off: release/acquire at cluster (1) or CTA (0) scope
 };
 
 struct SharedCtl {
@@ -106,6 +115,8 @@ struct SharedCtl {
 struct SharedCtl2 {
     uint64_t full[6];
     uint64_t empty[6];
+    uint64_t cfull[6];     // this CTA's code tile of the stage has landed (CVT variants)
+    uint64_t cvt_full[6];  // the leader's: both CTAs' B tiles of the stage are converted
     uint64_t acc_full[2];
     uint64_t acc_empty[2];
     uint64_t drain;
@@ -562,20 +573,275 @@ __global__ void __launch_bounds__((4 + EPI_WARPS) * 32, 1)
 //   acc_full[a]  each CTA's: the leader's commit after a tile's last MMA (multicast)
 //   acc_empty[a] the leader's: both CTAs' epilogue threads arrive after draining
 constexpr int BM2 = 256;              // rows of a pair tile
-constexpr int STAGES2 = 6;
 constexpr int A_HALF = 128 * BK * 2;  // this CTA's 128 rows of A per stage
-constexpr int STAGE2_BYTES = A_HALF + 128 * BK * 2;  // + up to 128 rows of B
-constexpr int SMEM2_BYTES = 1024 + STAGES2 * STAGE2_BYTES + 256;
+constexpr int B_HALF = 128 * BK * 2;  // up to 128 rows of B per stage
 
-template <int EPI0, int EPI1, int BITS, int EPI_WARPS>
-__global__ void __launch_bounds__((4 + EPI_WARPS) * 32, 1)
+// Stage layout of the pair kernel.  CVT variants add a slot for the stage's packed
+// code tile (128 rows x 64 codes at most) behind A and B and four converter warps.
+template <int CVT, int BITS>
+struct PairCfg {
+    static constexpr int CODE_BITS = BITS == 3 ? 8 : BITS;  // stored bits per code (3-bit: one byte)
+    static constexpr int CODE_SLOT = CVT ? 128 * 8 * CODE_BITS : 0;
+    static constexpr int STAGE = A_HALF + B_HALF + CODE_SLOT;
+    static constexpr int STAGES = (CVT && CODE_BITS > 2) ? 5 : 6;
+    // Converter warps: one per ring slot; warp w converts every stage of slot w, a whole
+    // stage per warp, so that all the ring's stages can be in conversion at once and
+    // each warp has the time of STAGES stages of MMA for one of its own.
+    static constexpr int CVT_WARPS = CVT ? STAGES : 0;
+    // Epilogue warps: the plain store and the E2E ds epilogue keep up with four.
+    static constexpr int EPI_WARPS = CVT ? 4 : 8;
+    // Per converter warp: the group constants (s, zq as fp32) of the stage it converts,
+    // two per B tile row (the two 32-code halves of its 64 codes).
+    static constexpr int CONST_BYTES = CVT_WARPS * 256 * 8;
+    static constexpr int SMEM = 1024 + STAGES * STAGE + CONST_BYTES + 256;
+};
+static_assert(PairCfg<1, 3>::SMEM <= 232448 && PairCfg<1, 2>::SMEM <= 232448 && PairCfg<1, 4>::SMEM <= 232448,
+              "pair kernel stages exceed the shared memory of a CTA");
+static_assert(sizeof(SharedCtl2) <= 256, "control block exceeds its slot");
+
+// ------------------------------------------------------------------ dequantize on load
+// Eq. 2 on the way into the MMA (modelfoundations note, Phase 2: only dequantization
+// sits in the E2E-QP graph): the B tile W-hat = (W_q - zq) s of a stage is made in
+// shared memory from the stage's packed code tile, in the 128-byte-swizzled layout a
+// TMA load of bf16 W-hat would have produced, so the MMA descriptors do not change.
+//
+// A B tile row ("row" below) is 64 consecutive in-features k of one W-hat row n: for
+// the forward (K-major B) row r of the tile is n = n0 + r over the stage's k range; for
+// the input gradient (MN-major B) row b*64 + r is n = k0 + r (the contraction index)
+// over the columns n0 + 64 b ...  Its codes are 8 * CODE_BITS contiguous bytes.
+//
+// Exactness.  With 0 <= m < 2^23 the fp32 number with bits 0x4B000000 | m is exactly
+// 2^23 + m.  A code c at bit offset CB*i of a 16-bit half word, masked in place, gives
+// f = 2^23 + c 2^(CB i); o_i = 2^23 + zq 2^(CB i) likewise (zq <= 15 keeps both below
+// 2^24), so f - o_i = (c - zq) 2^(CB i) exactly, and multiplying by s 2^(-CB i) (exact:
+// a power-of-two scaling of a normal s) rounds once to RN((c - zq) s), the fp32 product
+// of Eq. 2.  cvt.rn.bf16x2.f32 then rounds it to the bf16 operand as the dequantize
+// kernel does.  Two weights per packed-fp32 instruction.
+template <int BITS>
+struct CodeFmt {
+    static constexpr int CB = BITS == 3 ? 8 : BITS;  // stored bits per code
+    static constexpr int PER_UNIT = 128 / CB;        // codes in one 16-byte unit: 64, 32, 16
+    static constexpr int PER_HALF = 16 / CB;         // codes in a 16-bit half word: 8, 4, 2
+    static constexpr int UPR = CB / 2;               // 16-byte units per 64-code row: 1, 2, 4
+    static constexpr uint32_t MASK = (1u << CB) - 1u;
+};
+
+__device__ __forceinline__ uint64_t cf2_pack(float a, float b) {
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a), "f"(b));
+    return r;
+}
+__device__ __forceinline__ uint64_t cf2_sub(uint64_t a, uint64_t b) {
+    uint64_t d;
+    asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+__device__ __forceinline__ uint64_t cf2_mul(uint64_t a, uint64_t b) {
+    uint64_t d;
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+// Two fp32 lanes (lo, hi) to one bf16x2 word, round to nearest even (lo in the low half).
+__device__ __forceinline__ uint32_t cf2_to_bf16x2(uint64_t v) {
+    uint32_t d;
+    asm("{\n"
+        ".reg .f32 lo, hi;\n"
+        "mov.b64 {lo, hi}, %1;\n"
+        "cvt.rn.bf16x2.f32 %0, hi, lo;\n"
+        "}\n"
+        : "=r"(d)
+        : "l"(v));
+    return d;
+}
+
+// The constants of one group for the codes of a half word: o_i, s_i as packed pairs
+// (i, i + 1).
+template <int BITS>
+struct GroupPairs {
+    uint64_t off[CodeFmt<BITS>::PER_HALF / 2];
+    uint64_t sc[CodeFmt<BITS>::PER_HALF / 2];
+    __device__ __forceinline__ void set(float s, uint32_t zq) {
+        using F = CodeFmt<BITS>;
+#pragma unroll
+        for (int i = 0; i < F::PER_HALF; i += 2) {
+            const float o0 = __uint_as_float(0x4B000000u + (zq << (F::CB * i)));
+            const float o1 = __uint_as_float(0x4B000000u + (zq << (F::CB * (i + 1))));
+            const float s0 = __fmul_rn(s, __uint_as_float(static_cast<uint32_t>(127 - F::CB * i) << 23));
+            const float s1 = __fmul_rn(s, __uint_as_float(static_cast<uint32_t>(127 - F::CB * (i + 1)) << 23));
+            off[i / 2] = cf2_pack(o0, o1);
+            sc[i / 2] = cf2_pack(s0, s1);
+        }
+    }
+};
+
+// W-hat of the PER_HALF codes of half word h (codes at bit offsets CB*i) as
+// PER_HALF / 2 bf16x2 words, code order.
+template <int BITS>
+__device__ __forceinline__ void convert_half(uint32_t h, const GroupPairs<BITS> &gp, uint32_t *out) {
+    using F = CodeFmt<BITS>;
+#pragma unroll
+    for (int i = 0; i < F::PER_HALF; i += 2) {
+        const float a = __uint_as_float((h & (F::MASK << (F::CB * i))) | 0x4B000000u);
+        const float b = __uint_as_float((h & (F::MASK << (F::CB * (i + 1)))) | 0x4B000000u);
+        out[i / 2] = cf2_to_bf16x2(cf2_mul(cf2_sub(cf2_pack(a, b), gp.off[i / 2]), gp.sc[i / 2]));
+    }
+}
+
+// A 16-byte unit of the stage's code tile (units are numbered by their offset in the tile).
+// Where a unit lies (tile row, first 16-byte chunk of the row it fills, W-hat n and k).
+struct UnitPos {
+    int row, chunk, n, k;
+};
+
+template <int BITS>
+__device__ __forceinline__ UnitPos unit_pos(int u, int b_mn, int half, int n0, int k0) {
+    using F = CodeFmt<BITS>;
+    UnitPos p;
+    if (!b_mn) {
+        const int r = u / F::UPR, q = u % F::UPR;
+        p.row = r;
+        p.chunk = q * (F::PER_UNIT / 8);
+        p.n = n0 + r;
+        p.k = k0 + q * F::PER_UNIT;
+    } else {
+        const int per_row = half * F::CB / 128;  // units per code row (contraction index)
+        const int r = u / per_row, w = u % per_row;
+        const int b = w / F::UPR, q = w % F::UPR;
+        p.row = b * 64 + r;
+        p.chunk = q * (F::PER_UNIT / 8);
+        p.n = k0 + r;
+        p.k = n0 + 64 * b + q * F::PER_UNIT;
+    }
+    return p;
+}
+
+// Where the group constants of B tile row `row`, code half `hsub` (codes 32 hsub ..
+// 32 hsub + 31 of the row's 64) come from: W-hat row n and in-feature k.
+__device__ __forceinline__ void row_half_pos(int row, int hsub, int b_mn, int n0, int k0, int &n, int &k) {
+    if (!b_mn) {
+        n = n0 + row;
+        k = k0 + 32 * hsub;
+    } else {
+        n = k0 + (row & 63);
+        k = n0 + 64 * (row >> 6) + 32 * hsub;
+    }
+}
+
+// The stage's constants, gathered by one warp into registers a stage ahead: entry
+// e = lane + 32 i is (row e / 2, half e % 2) of the B tile; s = 0 and zq = 0 where the
+// row or the in-feature lies outside W-hat.
+constexpr int kConstPerLane = 256 / 32;
+
+struct StageConsts {
+    float s[kConstPerLane];
+    uint32_t zq[kConstPerLane];
+};
+
+// With groups of 64 or more the two halves of a row share their group: entries
+// e = lane + 32 i, i < 4, are then rows (one load per row) and stand for both halves.
+__device__ __forceinline__ void gather_consts(const Prob &pr, int b_mn, int half, int n0, int k0, int lane,
+                                              StageConsts &c) {
+    const bool per_row = pr.gshift > 5;
+#pragma unroll
+    for (int i = 0; i < kConstPerLane; ++i) {
+        const int e = lane + 32 * i;
+        c.s[i] = 0.0f;
+        c.zq[i] = 0u;
+        if (per_row ? (e < half) : (e < 2 * half)) {
+            int n, k;
+            if (per_row)
+                row_half_pos(e, 0, b_mn, n0, k0, n, k);
+            else
+                row_half_pos(e >> 1, e & 1, b_mn, n0, k0, n, k);
+            if (n < pr.w_rows && k < pr.w_cols) {
+                const int64_t gi = static_cast<int64_t>(n) * pr.w_groups + (k >> pr.gshift);
+                c.s[i] = pr.cvt_s_f16 ? __half2float(__ldg(static_cast<const __half *>(pr.cvt_s) + gi))
+                                      : __ldg(static_cast<const float *>(pr.cvt_s) + gi);
+                c.zq[i] = __ldg(pr.cvt_zq + gi);
+            }
+        }
+    }
+}
+
+// One warp converts a whole stage: code units u = lane, lane + 32, ... of the stage's
+// code tile into the B slot.  `tab` holds the stage's constants (float2 {s, zq} per
+// entry, written by this warp just before).
+template <int BITS>
+__device__ __forceinline__ void convert_stage_warp(const uint8_t *codes_smem, uint8_t *b_smem, int b_mn, int half,
+                                                   bool two_groups, int lane, const float2 *tab) {
+    using F = CodeFmt<BITS>;
+    const int units = half * F::CB / 2;
+#pragma unroll 2
+    for (int u = lane; u < units; u += 32) {
+        const UnitPos p = unit_pos<BITS>(u, b_mn, half, 0, 0);
+        const uint4 raw = *reinterpret_cast<const uint4 *>(codes_smem + 16 * u);
+        const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
+        uint8_t *row = b_smem + p.row * 128;
+        const int sw = p.row & 7;
+        // the unit's codes start at code 8 * p.chunk of the row: half 0 or 1 of it
+        const int h0 = (8 * p.chunk) >> 5;
+        GroupPairs<BITS> gp;
+        float2 c = tab[2 * p.row + h0];
+        gp.set(c.x, static_cast<uint32_t>(c.y));
+        constexpr int HALVES_PER_CHUNK = 8 / F::PER_HALF;
+#pragma unroll
+        for (int cc = 0; cc < F::PER_UNIT / 8; ++cc) {
+            if (BITS == 2 && cc == 4 && two_groups) {  // codes 32..63 of the row: another group of 32
+                c = tab[2 * p.row + 1];
+                gp.set(c.x, static_cast<uint32_t>(c.y));
+            }
+            uint32_t o[4];
+#pragma unroll
+            for (int hh = 0; hh < HALVES_PER_CHUNK; ++hh) {
+                const int hidx = cc * HALVES_PER_CHUNK + hh;  // half word index in the unit
+                const uint32_t word = w[hidx >> 1];
+                const uint32_t h = (hidx & 1) ? (word >> 16) : (word & 0xFFFFu);
+                convert_half<BITS>(h, gp, o + hh * (F::PER_HALF / 2));
+            }
+            const int pos = (p.chunk + cc) ^ sw;
+            *reinterpret_cast<uint4 *>(row + pos * 16) = make_uint4(o[0], o[1], o[2], o[3]);
+        }
+    }
+}
+
+// The converter warps' walk over the launch's stages, in the order of the producer and
+// the MMA issuer: (tile, k block) with the global stage counter `it`.
+struct StageWalk {
+    int t, kb, nkb;
+    uint32_t it;
+    TileInfo ti;
+};
+
+// ---------------------------------------------------------------------------- CTA pairs
+// The same grouped GEMM on pairs of SMs (cta_group::2, cluster of two CTAs):
+// one tcgen05.mma covers a 256-row tile, each CTA stages its 128 rows of A and
+// half of the tile's B columns, the even CTA issues the MMAs, and each CTA's
+// tensor memory holds its 128 accumulator rows.  Per SM, a 256 x bn pair tile
+// reads a third less operand data from shared memory per FLOP than a 128 x bn
+// tile of one CTA (B is split between the two SMs), the limiter of the one-CTA
+// kernel.  Protocol:
+//   full[s]      the leader's: armed by the leader with both CTAs' bytes, completed
+//                by both CTAs' TMA loads (each into its own shared memory)
+//   empty[s]     each CTA's: the leader's MMA commit arrives on both (multicast)
+//   acc_full[a]  each CTA's: the leader's commit after a tile's last MMA (multicast)
+//   acc_empty[a] the leader's: both CTAs' epilogue threads arrive after draining
+// CVT variants, for the stages of a problem whose B is made from codes on load:
+//   cfull[s]     each CTA's: its own TMA load of the stage's code tile
+//   cvt_full[s]  the leader's: one arrival per converter warp of both CTAs once the
+//                warp's part of the B tile is written and fenced for the tensor core;
+//                the MMA issuer waits on it besides full[s] (which then counts A only)
+template <int EPI0, int EPI1, int BITS, int EPI_WARPS, int CVT>
+__global__ void __launch_bounds__((4 + EPI_WARPS + PairCfg<CVT, BITS>::CVT_WARPS) * 32, 1)
     k_gemm_tc2(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUtensorMap tmB0,
                const __grid_constant__ CUtensorMap tmA1, const __grid_constant__ CUtensorMap tmB1,
                const KParams p) {
+    using C = PairCfg<CVT, BITS>;
+    constexpr int STAGES2 = C::STAGES;
+    constexpr int STAGE2_BYTES = C::STAGE;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                 ~static_cast<uintptr_t>(1023));
-    SharedCtl2 *ctl = reinterpret_cast<SharedCtl2 *>(smem + STAGES2 * STAGE2_BYTES);
+    SharedCtl2 *ctl = reinterpret_cast<SharedCtl2 *>(smem + STAGES2 * STAGE2_BYTES + C::CONST_BYTES);
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
     const uint32_t rank = cluster_rank();
@@ -586,6 +852,8 @@ __global__ void __launch_bounds__((4 + EPI_WARPS) * 32, 1)
         for (int i = 0; i < STAGES2; ++i) {
             mbar_init(&ctl->full[i], 1);
             mbar_init(&ctl->empty[i], 1);
+            mbar_init(&ctl->cfull[i], 1);
+            mbar_init(&ctl->cvt_full[i], 2);  // one converter warp of each CTA
         }
         for (int i = 0; i < 2; ++i) {
             mbar_init(&ctl->acc_full[i], 1);
@@ -618,7 +886,9 @@ __global__ void __launch_bounds__((4 + EPI_WARPS) * 32, 1)
         // ---------------------------------------------------------- TMA producer (both CTAs)
         if (elect_one_sync()) {
             uint32_t it = 0;
-            uint32_t armed = 0, armed_parity = 0;
+            uint32_t armed = 0, armed_parity = 0;     // the leader's full barriers with a phase armed
+            uint32_t carmed = 0, carmed_parity = 0;   // this CTA's code barriers with a phase armed
+            uint32_t cuse = 0;                        // per stage: parity of its next code phase
             bool ok = true;
             for (int t = pair; ok && t < p.total_tiles; t += npairs) {
                 const TileInfo ti = tile_info(p, t);
@@ -628,6 +898,7 @@ __global__ void __launch_bounds__((4 + EPI_WARPS) * 32, 1)
                 const CUtensorMap *mb = (pi || ti.narrow) ? &tmB1 : &tmB0;
                 const int a_mn = pi ? p.pr[1].a_mn : p.pr[0].a_mn;
                 const int b_mn = pi ? p.pr[1].b_mn : p.pr[0].b_mn;
+                const bool cvt = CVT && (pi ? p.pr[1].b_cvt : p.pr[0].b_cvt);
                 const int nkb = ((pi ? p.pr[1].GK : p.pr[0].GK) + BK - 1) / BK;
                 const int half = ti.bn / 2;
                 const int m0 = ti.tm * BM2 + 128 * static_cast<int>(rank);
@@ -642,7 +913,7 @@ __global__ void __launch_bounds__((4 + EPI_WARPS) * 32, 1)
                     uint8_t *sa = smem + st * STAGE2_BYTES;
                     uint8_t *sb = sa + A_HALF;
                     if (leader) {
-                        mbar_arrive_expect_tx(&ctl->full[st], 2 * (A_HALF + half * BK * 2));
+                        mbar_arrive_expect_tx(&ctl->full[st], 2 * (A_HALF + (cvt ? 0 : half * BK * 2)));
                         armed |= 1u << st;
                         armed_parity = (armed_parity & ~(1u << st)) | (ph << st);
                     }
@@ -655,7 +926,22 @@ __global__ void __launch_bounds__((4 + EPI_WARPS) * 32, 1)
                     } else {
                         tma_load_2d_pair(sa, ma, bar, k0, m0);
                     }
-                    if (b_mn) {
+                    if (cvt) {
+                        // this CTA's code tile, on its own barrier: K-major rows n0.. at
+                        // byte k0 * CB / 8; MN-major rows k0.. (the contraction index) at
+                        // byte n0 * CB / 8
+                        constexpr int CBITS = CodeFmt<BITS>::CB;
+                        const uint32_t cph = (cuse >> st) & 1u;
+                        cuse ^= 1u << st;
+                        mbar_arrive_expect_tx(&ctl->cfull[st], half * 8 * CBITS);
+                        carmed |= 1u << st;
+                        carmed_parity = (carmed_parity & ~(1u << st)) | (cph << st);
+                        uint8_t *sc = sb + B_HALF;
+                        if (b_mn)
+                            tma_load_2d(sc, mb, &ctl->cfull[st], n0 * CBITS / 8, k0);
+                        else
+                            tma_load_2d(sc, mb, &ctl->cfull[st], k0 * CBITS / 8, n0);
+                    } else if (b_mn) {
                         for (int b = 0; b < half / MN_BOX; ++b)
                             tma_load_2d_pair(sb + b * MN_BOX_BYTES, mb, bar, n0 + b * MN_BOX, k0);
                     } else {
@@ -669,6 +955,15 @@ __global__ void __launch_bounds__((4 + EPI_WARPS) * 32, 1)
                 const uint64_t t0 = globaltimer_ns();
                 while (globaltimer_ns() - t0 < 2000000ull) {
                 }
+                // This CTA's code copies count on its own barriers: let them land.
+                for (int st = 0; st < STAGES2; ++st)
+                    if (carmed & (1u << st)) {
+                        const uint32_t a = smem_u32(&ctl->cfull[st]);
+                        const uint64_t t1 = globaltimer_ns();
+                        while (!mbar_try_wait(a, (carmed_parity >> st) & 1u) &&
+                               globaltimer_ns() - t1 < 100000000ull) {
+                        }
+                    }
             }
             if (!ok && leader) {
                 // Let the pair's copies already issued land before the blocks exit.
@@ -687,12 +982,14 @@ __global__ void __launch_bounds__((4 + EPI_WARPS) * 32, 1)
         // ---------------------------------------------------------- MMA issuer (the leader)
         if (leader && elect_one_sync()) {
             uint32_t it = 0, local = 0;
+            uint32_t cuse = 0;  // per stage: parity of its next converted phase
             bool ok = true, issued = false;
             for (int t = pair; ok && t < p.total_tiles; t += npairs, ++local) {
                 const TileInfo ti = tile_info(p, t);
                 const int pi = ti.pi;
                 const int a_mn = pi ? p.pr[1].a_mn : p.pr[0].a_mn;
                 const int b_mn = pi ? p.pr[1].b_mn : p.pr[0].b_mn;
+                const bool cvt = CVT && (pi ? p.pr[1].b_cvt : p.pr[0].b_cvt);
                 const int nkb = ((pi ? p.pr[1].GK : p.pr[0].GK) + BK - 1) / BK;
                 const uint32_t idesc = idesc_bf16_f32(BM2, ti.bn, a_mn != 0, b_mn != 0);
                 const uint32_t a_step = a_mn ? UK * 128 : UK * 2, a_lbo = a_mn ? MN_BOX_BYTES : 16;
@@ -711,6 +1008,19 @@ __global__ void __launch_bounds__((4 + EPI_WARPS) * 32, 1)
                     if (!mbar_wait_bounded(&ctl->full[st], ph, abort_flag, p.err, p.wait_limit_ns)) {
                         ok = false;
                         break;
+                    }
+                    if (cvt) {
+                        const uint32_t cph = (cuse >> st) & 1u;
+                        cuse ^= 1u << st;
+                        const bool w = p.cvt_cluster_scope
+                                           ? mbar_wait_bounded<true>(&ctl->cvt_full[st], cph, abort_flag, p.err,
+                                                                     p.wait_limit_ns)
+                                           : mbar_wait_bounded<false>(&ctl->cvt_full[st], cph, abort_flag, p.err,
+                                                                      p.wait_limit_ns);
+                        if (!w) {
+                            ok = false;
+                            break;
+                        }
                     }
                     tc_fence_after();
                     const uint32_t sa = smem_u32(smem + st * STAGE2_BYTES);
@@ -736,7 +1046,7 @@ __global__ void __launch_bounds__((4 + EPI_WARPS) * 32, 1)
             }
         }
         __syncwarp();
-    } else if (warp >= 4) {
+    } else if (warp >= 4 && warp < 4 + EPI_WARPS) {
         // ---------------------------------------------------------- epilogue (both CTAs)
         const int ew = warp - 4;
         const int quad = warp & 3;
@@ -759,6 +1069,95 @@ __global__ void __launch_bounds__((4 + EPI_WARPS) * 32, 1)
                 drain_accumulator<EPI1, BITS>(p.pr[1], taddr, row, ti.n0, half_slice * cols, (half_slice + 1) * cols);
             tc_fence_before();
             mbar_arrive_cluster(acc_empty0 + 8u * acc);
+        }
+    } else if (CVT && warp >= 4 + EPI_WARPS) {
+        // ---------------------------------------------------------- converters (both CTAs)
+        // Warp cw converts the stages of B-from-codes problems whose global stage
+        // counter is cw modulo CVT_WARPS (so it owns the ring slots cw, cw + CVT_WARPS,
+        // ...: each slot's phases are waited on in order by one warp).  It gathers the
+        // group constants of its next stage into registers before it waits for the
+        // current one, so their L2 latency hides behind the other warps' stages.
+        constexpr int CW = C::CVT_WARPS;
+        const int cw = warp - (4 + EPI_WARPS);
+        float2 *tab = reinterpret_cast<float2 *>(smem + STAGES2 * STAGE2_BYTES) + cw * 256;
+        const uint32_t cvt_full0 = map_to_rank(&ctl->cvt_full[0], 0);
+        uint32_t cuse = 0;  // per owned slot: parity of its next code phase
+        // this warp's next stage at or after (t, kb)
+        auto seek = [&](StageWalk &w) -> bool {
+            while (w.t < p.total_tiles) {
+                if (w.kb == 0) {
+                    w.ti = tile_info(p, w.t);
+                    w.nkb = ((w.ti.pi ? p.pr[1].GK : p.pr[0].GK) + BK - 1) / BK;
+                }
+                const bool cvt = w.ti.pi ? p.pr[1].b_cvt : p.pr[0].b_cvt;
+                if (cvt) {
+                    const int skip = (cw - static_cast<int>(w.it % CW) + CW) % CW;
+                    if (w.kb + skip < w.nkb) {
+                        w.kb += skip;
+                        w.it += static_cast<uint32_t>(skip);
+                        return true;
+                    }
+                }
+                w.it += static_cast<uint32_t>(w.nkb - w.kb);  // the rest of this tile
+                w.t += npairs;
+                w.kb = 0;
+            }
+            return false;
+        };
+        auto consts = [&](const StageWalk &w, StageConsts &c) {
+            const Prob &pr = w.ti.pi ? p.pr[1] : p.pr[0];
+            const int half = w.ti.bn / 2;
+            gather_consts(pr, pr.b_mn, half, w.ti.n0 + half * static_cast<int>(rank), w.kb * BK, lane, c);
+        };
+        StageWalk cur{pair, 0, 0, 0u, TileInfo{}};
+        bool have = seek(cur);
+        StageConsts c_cur, c_nxt;
+        if (have) consts(cur, c_cur);
+        while (have) {
+            StageWalk nxt = cur;
+            ++nxt.kb;
+            ++nxt.it;
+            if (nxt.kb >= nxt.nkb) {
+                nxt.t += npairs;
+                nxt.kb = 0;
+            }
+            const bool have_nxt = seek(nxt);
+            if (have_nxt) consts(nxt, c_nxt);
+            const int st = cur.it % STAGES2;
+            const uint32_t cph = (cuse >> st) & 1u;
+            cuse ^= 1u << st;
+            const Prob &pr = cur.ti.pi ? p.pr[1] : p.pr[0];
+            const int half = cur.ti.bn / 2;
+            // the constants into the warp's table (the previous stage's reads are done)
+            __syncwarp();
+            if (pr.gshift > 5) {
+#pragma unroll
+                for (int i = 0; i < kConstPerLane / 2; ++i) {
+                    const float2 v = make_float2(c_cur.s[i], static_cast<float>(c_cur.zq[i]));
+                    tab[2 * (lane + 32 * i)] = v;
+                    tab[2 * (lane + 32 * i) + 1] = v;
+                }
+            } else {
+#pragma unroll
+                for (int i = 0; i < kConstPerLane; ++i)
+                    tab[lane + 32 * i] = make_float2(c_cur.s[i], static_cast<float>(c_cur.zq[i]));
+            }
+            __syncwarp();
+            const bool ok = mbar_wait_bounded(&ctl->cfull[st], cph, abort_flag, p.err, p.wait_limit_ns);
+            if (!__all_sync(0xffffffffu, ok)) break;
+            uint8_t *sb = smem + st * STAGE2_BYTES + A_HALF;
+            convert_stage_warp<BITS>(sb + B_HALF, sb, pr.b_mn, half, pr.gshift == 5, lane, tab);
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+                if (p.cvt_cluster_scope)
+                    mbar_arrive_cluster(cvt_full0 + 8u * static_cast<uint32_t>(st));
+                else
+                    mbar_arrive_cluster_cta_scope(cvt_full0 + 8u * static_cast<uint32_t>(st));
+            }
+            cur = nxt;
+            have = have_nxt;
+            c_cur = c_nxt;
         }
     }
 
@@ -812,6 +1211,31 @@ cudaError_t make_map(CUtensorMap &map, const Operand &op, int64_t rows, int64_t 
     return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 
+int code_bits_stored(int bits) { return bits == 3 ? 8 : bits; }
+
+// The packed codes of W-hat [w_rows, w_cols] as a 2-D byte tensor, one box per stage and
+// CTA: K-major (forward) 64 codes of `half` rows; MN-major (input gradient) `half`
+// codes of 64 rows (the contraction index).  No swizzle: the converter warps read it.
+cudaError_t make_code_map(CUtensorMap &map, const CvtArgs &c, bool mn_major, int half) {
+    const int cb = code_bits_stored(c.bits);
+    const uint64_t row_bytes = static_cast<uint64_t>(c.w_cols) * cb / 8;
+    cuuint64_t dims[2] = {row_bytes, static_cast<cuuint64_t>(c.w_rows)};
+    cuuint64_t strides[1] = {row_bytes};
+    cuuint32_t box[2];
+    if (mn_major) {
+        box[0] = static_cast<cuuint32_t>(half * cb / 8);
+        box[1] = BK;
+    } else {
+        box[0] = static_cast<cuuint32_t>(BK * cb / 8);
+        box[1] = static_cast<cuuint32_t>(half);
+    }
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = g_encode(&map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t *>(c.codes), dims, strides,
+                          box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                          CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
 constexpr int kEpiWarps = 8;
 
 template <int EPI0, int EPI1, int BITS>
@@ -831,21 +1255,22 @@ cudaError_t launch_variant(const CUtensorMap (&maps)[4], const KParams &p, int g
     return cudaGetLastError();
 }
 
-template <int EPI0, int EPI1, int BITS>
+template <int EPI0, int EPI1, int BITS, int CVT = 0>
 cudaError_t launch_pair_variant(const CUtensorMap (&maps)[4], const KParams &p, int grid, int dev_id,
                                 cudaStream_t st) {
-    auto kern = k_gemm_tc2<EPI0, EPI1, BITS, kEpiWarps>;
+    using C = PairCfg<CVT, BITS>;
+    auto kern = k_gemm_tc2<EPI0, EPI1, BITS, C::EPI_WARPS, CVT>;
     static std::atomic<uint64_t> done{0};
     const uint64_t bit = 1ull << (dev_id & 63);
     if (!(done.load() & bit)) {
-        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM2_BYTES);
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
         if (e != cudaSuccess) return e;
         done.fetch_or(bit);
     }
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(static_cast<unsigned>(grid), 1, 1);
-    cfg.blockDim = dim3((4 + kEpiWarps) * 32, 1, 1);
-    cfg.dynamicSmemBytes = SMEM2_BYTES;
+    cfg.blockDim = dim3((4 + C::EPI_WARPS + C::CVT_WARPS) * 32, 1, 1);
+    cfg.dynamicSmemBytes = C::SMEM;
     cfg.stream = st;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -865,6 +1290,15 @@ cudaError_t launch_pair_variant(const CUtensorMap (&maps)[4], const KParams &p, 
     }
     cfg.gridDim.x = static_cast<unsigned>(std::min(grid, 2 * n));
     return cudaLaunchKernelEx(&cfg, kern, maps[0], maps[1], maps[2], maps[3], p);
+}
+
+// EQAT_CVT_SCOPE=cta: converter hand-off at CTA scope (measurement aid).
+bool cvt_scope_cluster() {
+    static const bool on = [] {
+        const char *v = std::getenv("EQAT_CVT_SCOPE");
+        return !(v && v[0] == 'c' && v[1] == 't');
+    }();
+    return on;
 }
 
 // EQAT_GEMM_SPLIT_TAIL=0 keeps the last wave whole (measurement aid).
@@ -892,7 +1326,12 @@ cudaError_t fill_prob(Prob &q, const GemmProblem &g, int tile_begin, int bn, int
     cudaError_t e;
     const bool pair = tile_m == BM2;
     if ((e = make_map(ma, g.A, GM, GK, BM)) != cudaSuccess) return e;
-    if ((e = make_map(mb, g.B, GN, GK, pair ? bn / 2 : bn)) != cudaSuccess) return e;
+    if (g.cvt.on) {
+        if (!pair) return cudaErrorInvalidValue;
+        if ((e = make_code_map(mb, g.cvt, g.B.mn_major, bn / 2)) != cudaSuccess) return e;
+    } else if ((e = make_map(mb, g.B, GN, GK, pair ? bn / 2 : bn)) != cudaSuccess) {
+        return e;
+    }
     q = Prob{};
     q.GM = static_cast<int>(GM);
     q.GN = static_cast<int>(GN);
@@ -926,6 +1365,18 @@ cudaError_t fill_prob(Prob &q, const GemmProblem &g, int tile_begin, int bn, int
     q.group = epi.group;
     q.gshift = epi.group == 32 ? 5 : epi.group == 64 ? 6 : 7;
     q.Q = static_cast<float>((1 << epi.bits) - 1);
+    if (g.cvt.on) {
+        if (g.cvt.w_rows > INT32_MAX || g.cvt.w_cols > INT32_MAX) return cudaErrorInvalidValue;
+        q.b_cvt = 1;
+        q.w_rows = static_cast<int>(g.cvt.w_rows);
+        q.w_cols = static_cast<int>(g.cvt.w_cols);
+        q.w_groups = static_cast<int>(g.cvt.w_cols / g.cvt.group);
+        q.cvt_zq = g.cvt.zq;
+        q.cvt_s = g.cvt.s;
+        q.cvt_s_f16 = g.cvt.s_f16 ? 1 : 0;
+        q.gshift = g.cvt.group == 32 ? 5 : g.cvt.group == 64 ? 6 : 7;
+        q.group = g.cvt.group;
+    }
     return cudaSuccess;
 }
 
@@ -967,10 +1418,13 @@ Tiling choose_tiling(const GemmProblem *probs, int nprob, int sms) {
         const double cost = pair ? (bn == 256 ? 0.89 : 0.89 * 0.66) : (bn == 256 ? 1.0 : 0.72);
         return static_cast<double>(waves) * cost;
     };
-    Tiling best{false, 256};
+    bool need_pair = false;  // B made from codes on load: the pair kernel only
+    for (int i = 0; i < nprob; ++i) need_pair |= probs[i].cvt.on;
+    Tiling best{need_pair, 256};
     double best_t = 1e300;
     for (int pair = 0; pair < 2; ++pair) {
-        if (forced_pair >= 0 && pair != (forced_pair != 0)) continue;
+        if (need_pair && !pair) continue;
+        if (!need_pair && forced_pair >= 0 && pair != (forced_pair != 0)) continue;
         for (int bn = 256; bn >= 128; bn -= 128) {
             if (bn == 128 && (!narrow_ok || forced_bn == 256)) continue;
             if (bn == 256 && forced_bn == 128 && narrow_ok) continue;
@@ -987,6 +1441,14 @@ Tiling choose_tiling(const GemmProblem *probs, int nprob, int sms) {
 }  // namespace
 
 int *device_error_word() { return device_error_ptr(); }
+
+bool cvt_supported(int64_t w_rows, int64_t w_cols, int bits, int group) {
+    if (w_rows <= 0 || w_cols <= 0 || w_rows > INT32_MAX || w_cols > INT32_MAX) return false;
+    if (bits != 2 && bits != 3 && bits != 4) return false;
+    if (group != 32 && group != 64 && group != 128) return false;
+    const int64_t row_bytes = w_cols * code_bits_stored(bits) / 8;
+    return w_cols % group == 0 && row_bytes % 16 == 0;
+}
 
 cudaError_t encode_map_2d(CUtensorMap &map, CUtensorMapDataType type, const void *base, uint64_t inner,
                           uint64_t outer, uint64_t stride_bytes, uint32_t box_inner, uint32_t box_outer,
@@ -1044,7 +1506,9 @@ cudaError_t launch_gemm_tc_group(const GemmProblem *probs, int nprob, const Devi
         (probs[0].epi.kind == Epi::kStore || probs[0].epi.kind == Epi::kMse || probs[0].epi.group <= 64)) {
         const int full = tiles / units, tail = tiles % units;
         if (full >= 1 && tail > 0 && 2 * tail <= units) {
-            if ((e = make_map(maps[3], probs[0].B, probs[0].GN, probs[0].GK, bn / 4)) != cudaSuccess) return e;
+            e = probs[0].cvt.on ? make_code_map(maps[3], probs[0].cvt, false, bn / 4)
+                                : make_map(maps[3], probs[0].B, probs[0].GN, probs[0].GK, bn / 4);
+            if (e != cudaSuccess) return e;
             p.split_begin = full * units;
             p.total_tiles = full * units + 2 * tail;
         }
@@ -1052,6 +1516,33 @@ cudaError_t launch_gemm_tc_group(const GemmProblem *probs, int nprob, const Devi
     p.err = device_error_ptr();
     if (!p.err) return cudaErrorInvalidSymbol;
     p.wait_limit_ns = kWaitLimitNs;
+    p.cvt_cluster_scope = cvt_scope_cluster() ? 1 : 0;
+    bool any_cvt = false;
+    int cvt_bits = 2;
+    for (int i = 0; i < nprob; ++i)
+        if (probs[i].cvt.on) {
+            if (any_cvt && probs[i].cvt.bits != cvt_bits) return cudaErrorInvalidValue;
+            any_cvt = true;
+            cvt_bits = probs[i].cvt.bits;
+        }
+    if (pair && any_cvt) {
+        // B from codes: the E2E-QP forward (one problem, plain store) or backward
+        // (the ds epilogue on dY^T X, then dX = dY W-hat with W-hat made on load)
+        const int grid = 2 * std::min(p.total_tiles, units);
+        if (probs[0].epi.kind == Epi::kE2eDs && probs[0].epi.bits != cvt_bits) return cudaErrorInvalidValue;
+        const bool ds = probs[0].epi.kind == Epi::kE2eDs;
+        if (!ds && (probs[0].epi.kind != Epi::kStore || nprob > 1)) return cudaErrorInvalidValue;
+        switch (cvt_bits) {
+            case 2: return ds ? launch_pair_variant<2, 0, 2, 1>(maps, p, grid, dev.device, st)
+                              : launch_pair_variant<0, 0, 2, 1>(maps, p, grid, dev.device, st);
+            case 3: return ds ? launch_pair_variant<2, 0, 3, 1>(maps, p, grid, dev.device, st)
+                              : launch_pair_variant<0, 0, 3, 1>(maps, p, grid, dev.device, st);
+            case 4: return ds ? launch_pair_variant<2, 0, 4, 1>(maps, p, grid, dev.device, st)
+                              : launch_pair_variant<0, 0, 4, 1>(maps, p, grid, dev.device, st);
+            default: return cudaErrorInvalidValue;
+        }
+    }
+    if (any_cvt) return cudaErrorInvalidValue;
     if (pair) {
         const int grid = 2 * std::min(p.total_tiles, units);
         switch (probs[0].epi.kind) {

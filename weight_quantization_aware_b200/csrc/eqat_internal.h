@@ -79,12 +79,32 @@ struct EpiArgs {
     int group = 64;
 };
 
+// B made on load from packed codes (E2E-QP, Eq. 2): W-hat[w_rows, w_cols] =
+// (W_q - zq) s, converted in shared memory inside the pair GEMM instead of being
+// written to HBM first.  B.mn_major says how W-hat enters the contraction (K-major for
+// the forward, MN-major for the input gradient); B.ptr and B.ld are ignored.
+struct CvtArgs {
+    bool on = false;
+    const uint8_t *codes = nullptr;  // [w_rows, code_row_bytes(w_cols, bits)]
+    const uint8_t *zq = nullptr;     // [w_rows, w_cols / group]
+    const void *s = nullptr;         // [w_rows, w_cols / group], fp32 or fp16 (s_f16)
+    bool s_f16 = false;
+    int bits = 2;
+    int group = 64;
+    int64_t w_rows = 0, w_cols = 0;
+};
+
 struct GemmProblem {
     Operand A;
     Operand B;
     int64_t GM, GN, GK;
     EpiArgs epi;
+    CvtArgs cvt = {};
 };
+
+// Whether the pair GEMM can make this W-hat from its codes on load: the code rows must
+// be a whole number of 16-byte units for the tensor map (2-bit: w_cols % 64 == 0).
+bool cvt_supported(int64_t w_rows, int64_t w_cols, int bits, int group);
 
 // bf16 operands on tcgen05 tensor cores, fp32 accumulation in tensor memory.
 // A grouped launch runs the tiles of up to two contractions in one persistent

@@ -71,18 +71,44 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar_addr, uint32_t parity
     return ok != 0;
 }
 
+// The same test with acquire semantics at cluster scope: the phase was completed by
+// arrivals (release.cluster) of threads of the other CTA of a pair, whose earlier
+// shared-memory writes the caller then reads (or hands to the tensor core).
+__device__ __forceinline__ bool mbar_try_wait_cluster(uint32_t bar_addr, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n"
+        ".reg .pred P1;\n"
+        "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 P1, [%1], %2;\n"
+        "selp.b32 %0, 1, 0, P1;\n"
+        "}\n"
+        : "=r"(ok)
+        : "r"(bar_addr), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+// Makes this thread's generic-proxy writes to shared memory visible to later
+// async-proxy operations (TMA, tcgen05.mma operand reads).
+__device__ __forceinline__ void fence_proxy_async_smem() {
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
 // Waits until the phase of `bar` with the given parity has completed.  The wait
 // is bounded: after `limit_ns` nanoseconds it records kDevErrTimeout in *err,
 // raises the block-wide abort flag and returns false.  It also returns false as
 // soon as another thread of the block has raised the abort flag.
+// CLUSTER_ACQ selects the cluster-scope acquire (mbar_try_wait_cluster).
+template <bool CLUSTER_ACQ = false>
 __device__ __forceinline__ bool mbar_wait_bounded(uint64_t *bar, uint32_t parity,
                                                   volatile int *abort_flag, int *err,
                                                   uint64_t limit_ns) {
     const uint32_t a = smem_u32(bar);
-    if (mbar_try_wait(a, parity)) return true;
+    auto test = [&] { return CLUSTER_ACQ ? mbar_try_wait_cluster(a, parity) : mbar_try_wait(a, parity); };
+    if (test()) return true;
     const uint64_t t0 = globaltimer_ns();
     for (uint32_t i = 1;; ++i) {
-        if (mbar_try_wait(a, parity)) return true;
+        if (test()) return true;
         if ((i & 63u) == 0u) {
             if (*abort_flag) return false;
             if (globaltimer_ns() - t0 > limit_ns) {
@@ -228,6 +254,11 @@ __device__ __forceinline__ uint32_t map_to_rank(const void *p, uint32_t rank) {
 
 __device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
     asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+}
+
+// Arrive on an mbarrier of either CTA of the pair with release semantics at CTA scope.
+__device__ __forceinline__ void mbar_arrive_cluster_cta_scope(uint32_t cluster_addr) {
+    asm volatile("mbarrier.arrive.release.cta.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
 }
 
 // 2-D tile load into this CTA's shared memory whose completion is counted on an

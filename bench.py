@@ -909,9 +909,10 @@ def decode_gemv(dev, peaks, budget_bytes=300_000_000):
         out[name] = {"N": N, "K": K, "M": M, "bits": b, "group": g, "us": round(t, 2), "GBps": round(gbs, 1),
                      "frac_hbm": round(gbs / peaks["hbm_gbs"], 4), "bf16_matvec_us": round(tb, 2),
                      "speedup_vs_bf16_matvec": round(tb / t, 2), "layers_cycled": L}
-    out["note"] = ("GPU time per call from a CUDA graph of back-to-back calls (the streaming kernel and the partial "
-                   "sum; for layers above the build-mode size also the X-fragment kernel); bf16 matvec = "
-                   "torch.matmul on bf16 weights, same method")
+    out["note"] = ("GPU time per call from a CUDA graph of back-to-back calls: one kernel for layers with few row "
+                   "tiles (clusters sum the partials on chip), else the streaming kernel and the partial sum, and "
+                   "above the build-mode size also the X-fragment kernel; bf16 matvec = torch.matmul on bf16 "
+                   "weights, same method")
     return out
 
 
@@ -1174,6 +1175,7 @@ def main():
     ap.add_argument("--no-configs", action="store_true")
     ap.add_argument("--configs-only", action="store_true")
     ap.add_argument("--initpack70b-only", action="store_true")
+    ap.add_argument("--dq-only", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-hbm", action="store_true")
     ap.add_argument("--no-cfg1", action="store_true")
@@ -1214,6 +1216,22 @@ def main():
         if eqat.device_error() != 0:
             raise RuntimeError("device error word set")
         print(json.dumps({"gemv_only": "ok"}), flush=True)
+        return
+    if args.dq_only:  # profiling aid: one E2E-QP forward and backward on the step's workload
+        torch.cuda.set_device(0)
+        eqat.load_library()
+        dev = torch.device("cuda", 0)
+        step = Step(WORKLOAD, 0, WORKLOAD.bits, WORKLOAD.group, dev)
+        b, g = step.bits, step.group
+        eqat.minmax_init(step.W, b, g, s=step.s, z=step.z)
+        eqat.pack_codes(step.W, step.s, step.z, b, g, codes=step.codes, zq=step.zq)
+        eqat.dq_linear_fwd(step.X, step.codes, step.zq, step.s, b, g, ws=step.ws, Y=step.Y2)
+        eqat.dq_linear_bwd_s(step.X, step.codes, step.zq, step.s, step.dY, b, g, ws=step.ws,
+                             out=(step.dX2, step.ds2), w_hat_in_ws=True)
+        torch.cuda.synchronize()
+        if eqat.device_error() != 0:
+            raise RuntimeError("device error word set")
+        print(json.dumps({"dq_only": "ok"}), flush=True)
         return
     if args.initpack70b_only:  # profiling aid: just the 70B-block init/pack measurement
         torch.cuda.set_device(0)

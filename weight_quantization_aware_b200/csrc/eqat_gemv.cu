@@ -33,7 +33,10 @@
 // into equal contiguous ranges, one per CTA, so each CTA streams along K of the
 // same rows (whole DRAM pages, s / zq sectors reused at once).  A CTA writes one
 // fp32 partial per row tile it touches; k_gemv_reduce sums the partials of each
-// row tile in CTA order (deterministic).
+// row tile in CTA order (deterministic).  Layers with few row tiles (build mode)
+// instead give each row tile a cluster of C CTAs that split its K range; the
+// CTAs leave their partials in shared memory and the cluster's rank 0 sums them in
+// rank order through distributed shared memory and writes Y: one kernel per call.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
@@ -207,6 +210,8 @@ struct GemvParams {
     const uint4 *table;  // fragment mode only: B fragments of X from k_gemv_xprep, [sets_pad][2][32]
     const float2 *xso;   // fragment mode only: {xoff, xsum}, [groups_pad][8 tokens]
     float *partials;     // [row_tiles][maxseg][M][kRows]
+    __nv_bfloat16 *Y;    // cluster mode: written by each cluster's rank 0
+    int clu;             // cluster mode: CTAs per row tile (the cluster size)
     int M, N, G;
     int64_t K;
     int spr;             // stages per row tile (along K)
@@ -543,7 +548,8 @@ __device__ __forceinline__ void load_codes(const uint8_t *tile, int row, int byt
 
 // BUILD: the producer warp builds each stage's fragments from X (build mode);
 // otherwise they come by bulk copy from the table of k_gemv_xprep (fragment mode).
-template <int BITS, int GROUP, bool S16, int SL, bool BUILD>
+// CLU: cluster mode (grid = row tiles x p.clu, one row tile per cluster).
+template <int BITS, int GROUP, bool S16, int SL, bool BUILD, bool CLU>
 __global__ void __launch_bounds__(kThreads, 1)
     k_dq_gemv(const __grid_constant__ CUtensorMap tm_codes, const GemvParams p) {
     using C = Codes<BITS>;
@@ -571,7 +577,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint64_t *full = reinterpret_cast<uint64_t *>(smem + kOffBar<BITS, BUILD>);
     uint64_t *empty = full + NST;
     uint64_t *xfull = empty + NST;
-    volatile int *abort_flag = reinterpret_cast<volatile int *>(xfull + NST);
+    // cluster mode: red_full (rank 0's) counts the consumer warps of the cluster whose
+    // partials are in shared memory; red_done (each CTA's) rank 0's warps, once read
+    uint64_t *red_full = xfull + NST;
+    uint64_t *red_done = red_full + 1;
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(red_done + 1);
     // the code tile of stage (ks, rt): one TMA box per 128 bytes of each row
     auto load_code_tile = [&](uint8_t *dst, uint64_t *bar, int ks, int rt) {
 #pragma unroll
@@ -588,6 +598,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(&empty[i], kConsumers);
             mbar_init(&xfull[i], 1);
         }
+        if (CLU) {
+            mbar_init(red_full, kConsumers * p.clu);
+            mbar_init(red_done, kConsumers);
+        }
         *abort_flag = 0;
         fence_mbarrier_init();
         tma_prefetch_desc(&tm_codes);
@@ -602,6 +616,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
     }
     __syncthreads();
+    if constexpr (CLU) cluster_sync();  // every CTA's barriers exist before any remote arrival
     // Build mode: X, the codes, s and zq may come from the preceding kernel.  In
     // fragment mode the preceding kernel is k_gemv_xprep, which waited for them;
     // the producer waits for k_gemv_xprep itself (below).
@@ -842,9 +857,6 @@ __global__ void __launch_bounds__(kThreads, 1)
             // this CTA is done with row tile rt: its partial goes to slot
             // (rt, cta - first cta of rt).  The lanes of a quad that hold the
             // same tokens in different slots are summed first.
-            const int seg = static_cast<int>(blockIdx.x) -
-                            cta_of_stage(static_cast<int64_t>(rt) * p.spr, S, static_cast<int>(gridDim.x));
-            float *P = p.partials + (static_cast<int64_t>(rt) * p.maxseg + seg) * p.M * kRows;
             float v[4] = {y[0], y[1], y[2], y[3]};
             if constexpr (MPC == 1) {
                 v[0] += v[1];
@@ -859,15 +871,36 @@ __global__ void __launch_bounds__(kThreads, 1)
                     v[i] += __shfl_xor_sync(0xffffffffu, v[i], 2);
                 }
             }
-            if (slot0 == 0) {
-                const int m0 = tok0, m1 = tok0 + 1;
-                if (m0 < p.M) {
-                    P[m0 * kRows + row_a] = v[0];
-                    P[m0 * kRows + row_b] = v[2];
+            if constexpr (CLU) {
+                // cluster mode (one row tile per CTA): into this warp's s / zq
+                // area, which no stage reads any more: [token][16 rows]
+                __syncwarp();
+                float *Pw = reinterpret_cast<float *>(szw);
+                if (slot0 == 0) {
+                    const int m0 = tok0, m1 = tok0 + 1;
+                    if (m0 < p.M) {
+                        Pw[m0 * 16 + r0] = v[0];
+                        Pw[m0 * 16 + r0 + 8] = v[2];
+                    }
+                    if (MPC > 1 && m1 < p.M) {
+                        Pw[m1 * 16 + r0] = v[1];
+                        Pw[m1 * 16 + r0 + 8] = v[3];
+                    }
                 }
-                if (MPC > 1 && m1 < p.M) {
-                    P[m1 * kRows + row_a] = v[1];
-                    P[m1 * kRows + row_b] = v[3];
+            } else {
+                const int seg = static_cast<int>(blockIdx.x) -
+                                cta_of_stage(static_cast<int64_t>(rt) * p.spr, S, static_cast<int>(gridDim.x));
+                float *P = p.partials + (static_cast<int64_t>(rt) * p.maxseg + seg) * p.M * kRows;
+                if (slot0 == 0) {
+                    const int m0 = tok0, m1 = tok0 + 1;
+                    if (m0 < p.M) {
+                        P[m0 * kRows + row_a] = v[0];
+                        P[m0 * kRows + row_b] = v[2];
+                    }
+                    if (MPC > 1 && m1 < p.M) {
+                        P[m1 * kRows + row_a] = v[1];
+                        P[m1 * kRows + row_b] = v[3];
+                    }
                 }
             }
             y[0] = y[1] = y[2] = y[3] = 0.0f;
@@ -880,6 +913,39 @@ __global__ void __launch_bounds__(kThreads, 1)
         stage(sb_, sc_);
         if (cur.x >= x_end) break;
         stage(sc_, sa_);
+    }
+    if constexpr (CLU) {
+        // Each warp's partial of this CTA's K range is in its s / zq area.  Rank 0's
+        // warp w sums warp w's partials of the cluster's CTAs in rank order and
+        // writes its 16 rows of Y; the other CTAs keep their shared memory until
+        // rank 0 is done with it.
+        const uint32_t rank = cluster_rank();
+        __syncwarp();
+        if (lane == 0) mbar_arrive_cluster(map_to_rank(red_full, 0));
+        if (rank == 0) {
+            ok = mbar_wait_bounded<true>(red_full, 0, abort_flag, p.err, p.wait_limit_ns) && ok;
+            if (__all_sync(0xffffffffu, ok)) {
+                const int rt = static_cast<int>(x_begin / p.spr);
+                const uint32_t base = smem_u32(szw);
+                for (int i = lane; i < p.M * 16; i += 32) {
+                    const int m = i >> 4, rr = i & 15;
+                    float a = 0.0f;
+                    for (int c = 0; c < p.clu; ++c) {
+                        uint32_t addr;
+                        asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(addr) : "r"(base + 4u * i), "r"(c));
+                        float v;
+                        asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(addr) : "memory");
+                        a += v;
+                    }
+                    const int n = rt * kRows + warp * 16 + rr;
+                    if (n < p.N) p.Y[static_cast<int64_t>(m) * p.N + n] = __float2bfloat16_rn(a);
+                }
+            }
+            __syncwarp();
+            if (lane > 0 && lane < p.clu) mbar_arrive_cluster(map_to_rank(red_done, lane));
+        } else {
+            (void)mbar_wait_bounded<true>(red_done, 0, abort_flag, p.err, p.wait_limit_ns);
+        }
     }
     (void)ok;
 }
@@ -924,6 +990,7 @@ struct Plan {
     int spr, row_tiles, maxseg, grid;
     int64_t S;
     bool build;  // fragments built in the streaming kernel (else by k_gemv_xprep)
+    int clu;     // build mode with few row tiles: CTAs per row tile (cluster), else 1
     size_t table_bytes, xso_bytes, partial_bytes;
 };
 
@@ -950,6 +1017,19 @@ Plan make_plan(int64_t M, int64_t N, int64_t K, int bits, int group, int sms) {
         pl.maxseg = std::max(pl.maxseg, c1 - c0 + 1);
     }
     pl.build = build_mode(M, N, K, bits, group);
+    // Cluster mode: when two CTAs per row tile still fit on the SMs at once, each row
+    // tile gets a cluster of C CTAs (a power of two, at most 8 and at most its stages)
+    // and the partial sums never leave the chip: no second kernel.
+    pl.clu = 1;
+    if (pl.build && static_cast<int64_t>(pl.row_tiles) * 2 <= sms) {
+        int c = 2;
+        while (c * 2 <= 8 && c * 2 <= pl.spr && static_cast<int64_t>(pl.row_tiles) * c * 2 <= sms) c *= 2;
+        if (c <= pl.spr) {
+            pl.clu = c;
+            pl.grid = pl.row_tiles * c;
+            pl.maxseg = c;
+        }
+    }
     const int64_t sets = static_cast<int64_t>(pl.spr) * (ks / 64);
     const int64_t groups = static_cast<int64_t>(pl.spr) * (ks / group);
     pl.table_bytes = pl.build ? 0 : static_cast<size_t>(sets) * 1024;
@@ -960,7 +1040,33 @@ Plan make_plan(int64_t M, int64_t N, int64_t K, int bits, int group, int sms) {
 
 template <int BITS, int GROUP, bool S16, int SL, bool BUILD>
 cudaError_t launch_main(const CUtensorMap &map, const GemvParams &p, int grid, int dev_id, cudaStream_t st) {
-    auto kern = k_dq_gemv<BITS, GROUP, S16, SL, BUILD>;
+    if (BUILD && p.clu > 1) {
+        auto kern = k_dq_gemv<BITS, GROUP, S16, SL, BUILD, true>;
+        static std::atomic<uint64_t> done{0};
+        const uint64_t bit = 1ull << (dev_id & 63);
+        if (!(done.load() & bit)) {
+            cudaError_t e =
+                cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes<BITS, BUILD>);
+            if (e != cudaSuccess) return e;
+            done.fetch_or(bit);
+        }
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(grid);
+        cfg.blockDim = dim3(kThreads);
+        cfg.dynamicSmemBytes = kSmemBytes<BITS, BUILD>;
+        cfg.stream = st;
+        cudaLaunchAttribute attr[2];
+        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[0].val.programmaticStreamSerializationAllowed = 1;
+        attr[1].id = cudaLaunchAttributeClusterDimension;
+        attr[1].val.clusterDim.x = static_cast<unsigned>(p.clu);
+        attr[1].val.clusterDim.y = 1;
+        attr[1].val.clusterDim.z = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 2;
+        return cudaLaunchKernelEx(&cfg, kern, map, p);
+    }
+    auto kern = k_dq_gemv<BITS, GROUP, S16, SL, BUILD, false>;
     static std::atomic<uint64_t> done{0};
     const uint64_t bit = 1ull << (dev_id & 63);
     if (!(done.load() & bit)) {
@@ -1014,9 +1120,12 @@ cudaError_t launch_all(const CUtensorMap &map, GemvParams p, const Plan &pl, boo
                                    const_cast<float2 *>(p.xso));
         if (e != cudaSuccess) return e;
     }
+    p.clu = pl.clu;
+    p.Y = Y;
     cudaError_t e = s_f16 ? launch_slots<BITS, GROUP, true>(slots, pl.build, map, p, pl.grid, dev.device, st)
                           : launch_slots<BITS, GROUP, false>(slots, pl.build, map, p, pl.grid, dev.device, st);
     if (e != cudaSuccess) return e;
+    if (pl.clu > 1) return cudaSuccess;  // rank 0 of each cluster wrote Y
     const int64_t MN = static_cast<int64_t>(p.M) * p.N;
     const unsigned rblocks = static_cast<unsigned>(std::min<int64_t>((MN + 255) / 256, 2 * dev.sm_count));
     return launch_pdl(k_gemv_reduce, dim3(rblocks), dim3(256), 0, st, static_cast<const float *>(p.partials), p.M,

@@ -171,29 +171,17 @@ __device__ __forceinline__ TileInfo tile_info(const KParams &p, int t) {
 template <int EPI, int BITS>
 struct Epilogue;
 
+// Each epilogue kind computes the row's 32 values of a chunk; those with an output
+// matrix (kinds 0, 1 and 3) leave them in o[], which drain_accumulator writes out.
+// Rows at or beyond GM and columns at or beyond GN compute nothing that is stored.
+
 // D -> bf16 output.
 template <int BITS>
 struct Epilogue<0, BITS> {
     float acc_s = 0.0f, acc_z = 0.0f;
-    __device__ __forceinline__ void chunk(const Prob &p, int row, int col, const float (&v)[32]) {
-        if (row >= p.GM) return;
-        __nv_bfloat16 *out = static_cast<__nv_bfloat16 *>(p.out) + static_cast<int64_t>(row) * p.ldo + col;
-        if (col + 32 <= p.GN) {
-            uint4 *o = reinterpret_cast<uint4 *>(out);
+    __device__ __forceinline__ void chunk(const Prob &, int, int, const float (&v)[32], float (&o)[32]) {
 #pragma unroll
-            for (int q = 0; q < 4; ++q) {
-                uint4 r;
-                r.x = pack_bf16x2(v[8 * q + 0], v[8 * q + 1]);
-                r.y = pack_bf16x2(v[8 * q + 2], v[8 * q + 3]);
-                r.z = pack_bf16x2(v[8 * q + 4], v[8 * q + 5]);
-                r.w = pack_bf16x2(v[8 * q + 6], v[8 * q + 7]);
-                o[q] = r;
-            }
-        } else {
-#pragma unroll
-            for (int j = 0; j < 32; ++j)
-                if (col + j < p.GN) out[j] = __float2bfloat16_rn(v[j]);
-        }
+        for (int j = 0; j < 32; ++j) o[j] = v[j];
     }
 };
 
@@ -203,8 +191,13 @@ struct Epilogue<0, BITS> {
 template <int BITS>
 struct Epilogue<1, BITS> {
     float acc_s = 0.0f, acc_z = 0.0f;
-    __device__ __forceinline__ void chunk(const Prob &p, int row, int col, const float (&v)[32]) {
-        if (row >= p.GM || col >= p.GN) return;
+    __device__ __forceinline__ void chunk(const Prob &p, int row, int col, const float (&v)[32],
+                                          float (&dwv)[32]) {
+        if (row >= p.GM || col >= p.GN) {
+#pragma unroll
+            for (int j = 0; j < 32; ++j) dwv[j] = 0.0f;
+            return;
+        }
         const int64_t K = p.GN;
         const int64_t G = K >> p.gshift;
         const int64_t gi = static_cast<int64_t>(row) * G + (col >> p.gshift);
@@ -212,7 +205,6 @@ struct Epilogue<1, BITS> {
         const float rcp = __frcp_rn(sc);
         const float zr = rintf(__ldg(p.z + gi));
         const int64_t e0 = static_cast<int64_t>(row) * K + col;
-        float dwv[32];
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
             float w[8];
@@ -231,12 +223,6 @@ struct Epilogue<1, BITS> {
                 dwv[8 * q + j] = inside ? d : 0.0f;
             }
         }
-        if (p.dW) {
-            __nv_bfloat16 *o = static_cast<__nv_bfloat16 *>(p.dW) + e0;
-#pragma unroll
-            for (int q = 0; q < 4; ++q)
-                store8<__nv_bfloat16>(o + 8 * q, *reinterpret_cast<const float(*)[8]>(&dwv[8 * q]));
-        }
         if (((col + 32) & (p.group - 1)) == 0) {
             if (p.ds) p.ds[gi] = acc_s;
             if (p.dz) p.dz[gi] = -sc * acc_z;
@@ -251,7 +237,7 @@ struct Epilogue<1, BITS> {
 template <int BITS>
 struct Epilogue<2, BITS> {
     float acc_s = 0.0f, acc_z = 0.0f;
-    __device__ __forceinline__ void chunk(const Prob &p, int row, int col, const float (&v)[32]) {
+    __device__ __forceinline__ void chunk(const Prob &p, int row, int col, const float (&v)[32], float (&)[32]) {
         if (row >= p.GM || col >= p.GN) return;
         const int64_t K = p.GN;
         const int64_t G = K >> p.gshift;
@@ -301,33 +287,36 @@ struct Epilogue<2, BITS> {
 template <int BITS>
 struct Epilogue<3, BITS> {
     float acc_s = 0.0f, acc_z = 0.0f;
-    __device__ __forceinline__ void chunk(const Prob &p, int row, int col, const float (&v)[32]) {
-        if (row >= p.GM) return;
+    __device__ __forceinline__ void chunk(const Prob &p, int row, int col, const float (&v)[32], float (&o)[32]) {
+        if (row >= p.GM) {
+#pragma unroll
+            for (int j = 0; j < 32; ++j) o[j] = 0.0f;
+            return;
+        }
         const int64_t off = static_cast<int64_t>(row) * p.ldo + col;
         const __nv_bfloat16 *T = static_cast<const __nv_bfloat16 *>(p.target) + off;
-        __nv_bfloat16 *out = static_cast<__nv_bfloat16 *>(p.out) + off;
         if (col + 32 <= p.GN) {
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
                 float t[8];
                 load8<__nv_bfloat16>(T + 8 * q, t);
-                float r[8];
 #pragma unroll
                 for (int j = 0; j < 8; ++j) {
                     const float d = __fsub_rn(v[8 * q + j], t[j]);
                     acc_s = fmaf(d, d, acc_s);
-                    r[j] = __fmul_rn(d, p.mse_scale);
+                    o[8 * q + j] = __fmul_rn(d, p.mse_scale);
                 }
-                store8<__nv_bfloat16>(out + 8 * q, r);
             }
         } else {
 #pragma unroll
-            for (int j = 0; j < 32; ++j)
+            for (int j = 0; j < 32; ++j) {
+                o[j] = 0.0f;
                 if (col + j < p.GN) {
                     const float d = __fsub_rn(v[j], __bfloat162float(T[j]));
                     acc_s = fmaf(d, d, acc_s);
-                    out[j] = __float2bfloat16_rn(__fmul_rn(d, p.mse_scale));
+                    o[j] = __fmul_rn(d, p.mse_scale);
                 }
+            }
         }
     }
 };
@@ -343,17 +332,87 @@ __device__ __forceinline__ void finish_drain(const Prob &p, float acc) {
     }
 }
 
+// The output of one epilogue warp: 32 rows x 32 columns of bf16 per chunk.  With a
+// tensor map (CTA-pair kernel) the warp writes the chunk into its 2 KB of shared
+// memory in the 64-byte-swizzled layout of the map's box, and lane 0 stores it with
+// a TMA: the lanes do not wait on the stores, and each leaves the SM as whole
+// sectors (a lane owns one output row, so direct stores touch 32 rows per
+// instruction).  The TMA clips rows and columns beyond the matrix.  Without a map
+// (one-CTA kernel) the lanes store their rows directly.
+struct OutStage {
+    uint8_t *buf;            // this warp's staging buffer (512-byte aligned)
+    const CUtensorMap *map;  // nullptr: direct stores
+    bool pending;            // a TMA store may still read buf
+};
+
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap *map, const void *smem_src, int32_t c0, int32_t c1) {
+    asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
+                     reinterpret_cast<uint64_t>(map)),
+                 "r"(smem_u32(smem_src)), "r"(c0), "r"(c1)
+                 : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_read_all() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+
+template <int EPI>
+constexpr bool kHasOut = EPI == 0 || EPI == 1 || EPI == 3;
+
+__device__ __forceinline__ void write_chunk(OutStage &os, void *dst, int64_t ld, int64_t GM, int64_t GN, int row0,
+                                            int col, const float (&o)[32]) {
+    const int lane = threadIdx.x & 31;
+    uint32_t w[16];
+#pragma unroll
+    for (int j = 0; j < 16; ++j) w[j] = pack_bf16x2(o[2 * j], o[2 * j + 1]);
+    if (os.map) {
+        if (os.pending) {  // the previous chunk's store has read the buffer
+            if (lane == 0) bulk_wait_read_all();
+            __syncwarp();
+        }
+        uint8_t *rp = os.buf + lane * 64;
+        const int sw = (lane >> 1) & 3;  // 64-byte swizzle: 16-byte unit q of row r at q ^ ((r >> 1) & 3)
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+            *reinterpret_cast<uint4 *>(rp + ((q ^ sw) << 4)) = make_uint4(w[4 * q], w[4 * q + 1], w[4 * q + 2], w[4 * q + 3]);
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0 && row0 < GM && col < GN) {
+            tma_store_2d(os.map, os.buf, col, row0);
+            bulk_commit();
+        }
+        os.pending = true;
+        return;
+    }
+    const int row = row0 + lane;
+    if (row >= GM || col >= GN) return;
+    __nv_bfloat16 *out = static_cast<__nv_bfloat16 *>(dst) + row * ld + col;
+    if (col + 32 <= GN) {
+        uint4 *q4 = reinterpret_cast<uint4 *>(out);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) q4[q] = make_uint4(w[4 * q], w[4 * q + 1], w[4 * q + 2], w[4 * q + 3]);
+    } else {
+#pragma unroll
+        for (int j = 0; j < 32; ++j)
+            if (col + j < GN) out[j] = __float2bfloat16_rn(o[j]);
+    }
+}
+
 // Drains one accumulator (this warp's 32 rows, columns [c_begin, c_end)) through
-// the epilogue of kind EPI.
+// the epilogue of kind EPI.  row = row0 + lane.
 template <int EPI, int BITS>
-__device__ __forceinline__ void drain_accumulator(const Prob &pr, uint32_t taddr, int row, int col0,
-                                                  int c_begin, int c_end) {
+__device__ __forceinline__ void drain_accumulator(const Prob &pr, uint32_t taddr, int row0, int col0,
+                                                  int c_begin, int c_end, OutStage &os) {
     Epilogue<EPI, BITS> epi;
+    const int row = row0 + (threadIdx.x & 31);
+    void *dst = EPI == 1 ? pr.dW : pr.out;
+    const int64_t ld = EPI == 1 ? static_cast<int64_t>(pr.GN) : pr.ldo;
 #pragma unroll 1
     for (int c0 = c_begin; c0 < c_end; c0 += 32) {
         float v[32];
         tmem_ld_32cols(taddr + c0, v);
-        epi.chunk(pr, row, col0 + c0, v);
+        float o[32];
+        epi.chunk(pr, row, col0 + c0, v, o);
+        if (kHasOut<EPI> && dst) write_chunk(os, dst, ld, pr.GM, pr.GN, row0, col0 + c0, o);
     }
     finish_drain<EPI>(pr, epi.acc_s);
 }
@@ -538,14 +597,15 @@ __global__ void __launch_bounds__((4 + EPI_WARPS) * 32, 1)
             tc_fence_after();
             int tm, tn;
             const int pi = tile_coords(p, t, tm, tn);
-            const int row = tm * BM + quad * 32 + lane;
+            const int row0 = tm * BM + quad * 32;
             const uint32_t taddr = tmem_base + acc * ACC_COLS + ((quad * 32) << 16);
             const int bn = pi ? p.pr[1].bn : p.pr[0].bn;
             const int cols = bn / SLICES;  // a multiple of 64, hence of every group size
+            OutStage os{nullptr, nullptr, false};  // direct stores
             if (pi == 0)
-                drain_accumulator<EPI0, BITS>(p.pr[0], taddr, row, tn * bn, half * cols, (half + 1) * cols);
+                drain_accumulator<EPI0, BITS>(p.pr[0], taddr, row0, tn * bn, half * cols, (half + 1) * cols, os);
             else
-                drain_accumulator<EPI1, BITS>(p.pr[1], taddr, row, tn * bn, half * cols, (half + 1) * cols);
+                drain_accumulator<EPI1, BITS>(p.pr[1], taddr, row0, tn * bn, half * cols, (half + 1) * cols, os);
             tc_fence_before();
             mbar_arrive(&ctl->acc_empty[acc]);
         }
@@ -593,7 +653,9 @@ struct PairCfg {
     // Per converter warp: the group constants (s, zq as fp32) of the stage it converts,
     // two per B tile row (the two 32-code halves of its 64 codes).
     static constexpr int CONST_BYTES = CVT_WARPS * 256 * 8;
-    static constexpr int SMEM = 1024 + STAGES * STAGE + CONST_BYTES + 256;
+    // Per epilogue warp: one 32 x 32 bf16 output chunk on its way to a TMA store.
+    static constexpr int OUT_BYTES = EPI_WARPS * 2048;
+    static constexpr int SMEM = 1024 + STAGES * STAGE + CONST_BYTES + OUT_BYTES + 256;
 };
 static_assert(PairCfg<1, 3>::SMEM <= 232448 && PairCfg<1, 2>::SMEM <= 232448 && PairCfg<1, 4>::SMEM <= 232448,
               "pair kernel stages exceed the shared memory of a CTA");
@@ -834,14 +896,17 @@ template <int EPI0, int EPI1, int BITS, int EPI_WARPS, int CVT>
 __global__ void __launch_bounds__((4 + EPI_WARPS + PairCfg<CVT, BITS>::CVT_WARPS) * 32, 1)
     k_gemm_tc2(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUtensorMap tmB0,
                const __grid_constant__ CUtensorMap tmA1, const __grid_constant__ CUtensorMap tmB1,
+               const __grid_constant__ CUtensorMap tmO0, const __grid_constant__ CUtensorMap tmO1,
                const KParams p) {
     using C = PairCfg<CVT, BITS>;
+    static_assert(EPI_WARPS == C::EPI_WARPS, "the staging area is sized for C::EPI_WARPS epilogue warps");
     constexpr int STAGES2 = C::STAGES;
     constexpr int STAGE2_BYTES = C::STAGE;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                 ~static_cast<uintptr_t>(1023));
-    SharedCtl2 *ctl = reinterpret_cast<SharedCtl2 *>(smem + STAGES2 * STAGE2_BYTES + C::CONST_BYTES);
+    SharedCtl2 *ctl =
+        reinterpret_cast<SharedCtl2 *>(smem + STAGES2 * STAGE2_BYTES + C::CONST_BYTES + C::OUT_BYTES);
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
     const uint32_t rank = cluster_rank();
@@ -1053,6 +1118,7 @@ __global__ void __launch_bounds__((4 + EPI_WARPS + PairCfg<CVT, BITS>::CVT_WARPS
         const int half_slice = ew >> 2;
         constexpr int SLICES = EPI_WARPS / 4;
         uint32_t local = 0;
+        OutStage os{smem + STAGES2 * STAGE2_BYTES + C::CONST_BYTES + ew * 2048, nullptr, false};
         for (int t = pair; t < p.total_tiles; t += npairs, ++local) {
             const uint32_t acc = local & 1u;
             const uint32_t aph = (local >> 1) & 1u;
@@ -1060,16 +1126,20 @@ __global__ void __launch_bounds__((4 + EPI_WARPS + PairCfg<CVT, BITS>::CVT_WARPS
             if (!__all_sync(0xffffffffu, ok)) break;
             tc_fence_after();
             const TileInfo ti = tile_info(p, t);
-            const int row = ti.tm * BM2 + 128 * static_cast<int>(rank) + quad * 32 + lane;
+            const int row0 = ti.tm * BM2 + 128 * static_cast<int>(rank) + quad * 32;
             const uint32_t taddr = tmem_base + acc * ACC_COLS + ((quad * 32) << 16);
             const int cols = ti.bn / SLICES;
+            os.map = ti.pi ? &tmO1 : &tmO0;
             if (ti.pi == 0)
-                drain_accumulator<EPI0, BITS>(p.pr[0], taddr, row, ti.n0, half_slice * cols, (half_slice + 1) * cols);
+                drain_accumulator<EPI0, BITS>(p.pr[0], taddr, row0, ti.n0, half_slice * cols, (half_slice + 1) * cols, os);
             else
-                drain_accumulator<EPI1, BITS>(p.pr[1], taddr, row, ti.n0, half_slice * cols, (half_slice + 1) * cols);
+                drain_accumulator<EPI1, BITS>(p.pr[1], taddr, row0, ti.n0, half_slice * cols, (half_slice + 1) * cols, os);
             tc_fence_before();
             mbar_arrive_cluster(acc_empty0 + 8u * acc);
         }
+        // the warp's output stores have completed (and read their shared memory)
+        if (lane == 0) bulk_wait_all();
+        __syncwarp();
     } else if (CVT && warp >= 4 + EPI_WARPS) {
         // ---------------------------------------------------------- converters (both CTAs)
         // Warp cw converts the stages of B-from-codes problems whose global stage
@@ -1236,10 +1306,23 @@ cudaError_t make_code_map(CUtensorMap &map, const CvtArgs &c, bool mn_major, int
     return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 
+// A bf16 output matrix [rows, cols] (row stride ld elements) as the target of the
+// epilogue's TMA stores: one box of 32 x 32 per warp and chunk, 64-byte swizzle.
+cudaError_t make_out_map(CUtensorMap &map, const void *ptr, int64_t rows, int64_t cols, int64_t ld) {
+    cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
+    cuuint64_t strides[1] = {static_cast<cuuint64_t>(ld) * 2};
+    cuuint32_t box[2] = {32, 32};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = g_encode(&map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(ptr), dims, strides, box,
+                          estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B,
+                          CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
 constexpr int kEpiWarps = 8;
 
 template <int EPI0, int EPI1, int BITS>
-cudaError_t launch_variant(const CUtensorMap (&maps)[4], const KParams &p, int grid, int dev_id,
+cudaError_t launch_variant(const CUtensorMap (&maps)[6], const KParams &p, int grid, int dev_id,
                            cudaStream_t st) {
     auto kern = k_gemm_tc<EPI0, EPI1, BITS, kEpiWarps>;
     // The shared-memory opt-in is a per-device function attribute; setting it
@@ -1256,7 +1339,7 @@ cudaError_t launch_variant(const CUtensorMap (&maps)[4], const KParams &p, int g
 }
 
 template <int EPI0, int EPI1, int BITS, int CVT = 0>
-cudaError_t launch_pair_variant(const CUtensorMap (&maps)[4], const KParams &p, int grid, int dev_id,
+cudaError_t launch_pair_variant(const CUtensorMap (&maps)[6], const KParams &p, int grid, int dev_id,
                                 cudaStream_t st) {
     using C = PairCfg<CVT, BITS>;
     auto kern = k_gemm_tc2<EPI0, EPI1, BITS, C::EPI_WARPS, CVT>;
@@ -1289,7 +1372,7 @@ cudaError_t launch_pair_variant(const CUtensorMap (&maps)[4], const KParams &p, 
         resident[dev_id & 63].store(n);
     }
     cfg.gridDim.x = static_cast<unsigned>(std::min(grid, 2 * n));
-    return cudaLaunchKernelEx(&cfg, kern, maps[0], maps[1], maps[2], maps[3], p);
+    return cudaLaunchKernelEx(&cfg, kern, maps[0], maps[1], maps[2], maps[3], maps[4], maps[5], p);
 }
 
 // EQAT_CVT_SCOPE=cta: converter hand-off at CTA scope (measurement aid).
@@ -1476,7 +1559,7 @@ cudaError_t launch_gemm_tc_group(const GemmProblem *probs, int nprob, const Devi
     }
     cudaError_t e = get_encode();
     if (e != cudaSuccess) return e;
-    CUtensorMap maps[4];
+    CUtensorMap maps[6];  // A, B of problem 0; A, B of problem 1; the outputs of problems 0 and 1
     KParams p{};
     int tiles = 0;
     const Tiling tiling = choose_tiling(probs, nprob, dev.sm_count);
@@ -1494,6 +1577,18 @@ cudaError_t launch_gemm_tc_group(const GemmProblem *probs, int nprob, const Devi
     if (nprob == 1) {  // unused slots still travel as kernel parameters
         maps[2] = maps[0];
         maps[3] = maps[1];
+    }
+    // The epilogue's output matrices (bf16 store, MSE and straight-through dW).
+    for (int i = 0; i < 2; ++i) {
+        maps[4 + i] = maps[0];  // placeholder: no output matrix
+        if (i >= nprob) continue;
+        const EpiArgs &ea = probs[i].epi;
+        if (ea.kind == Epi::kStore || ea.kind == Epi::kMse) {
+            if ((e = make_out_map(maps[4 + i], ea.out, probs[i].GM, probs[i].GN, ea.ldo)) != cudaSuccess) return e;
+        } else if (ea.kind == Epi::kFqGrad && ea.dW) {
+            if ((e = make_out_map(maps[4 + i], ea.dW, probs[i].GM, probs[i].GN, probs[i].GN)) != cudaSuccess)
+                return e;
+        }
     }
     p.nprob = nprob;
     p.total_tiles = tiles;

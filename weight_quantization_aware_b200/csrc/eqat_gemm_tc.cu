@@ -638,7 +638,7 @@ constexpr int B_HALF = 128 * BK * 2;  // up to 128 rows of B per stage
 
 // Stage layout of the pair kernel.  CVT variants add a slot for the stage's packed
 // code tile (128 rows x 64 codes at most) behind A and B and four converter warps.
-template <int CVT, int BITS>
+template <int CVT, int BITS, int EW = 8>
 struct PairCfg {
     static constexpr int CODE_BITS = BITS == 3 ? 8 : BITS;  // stored bits per code (3-bit: one byte)
     static constexpr int CODE_SLOT = CVT ? 128 * 8 * CODE_BITS : 0;
@@ -648,8 +648,10 @@ struct PairCfg {
     // stage per warp, so that all the ring's stages can be in conversion at once and
     // each warp has the time of STAGES stages of MMA for one of its own.
     static constexpr int CVT_WARPS = CVT ? STAGES : 0;
-    // Epilogue warps: the plain store and the E2E ds epilogue keep up with four.
-    static constexpr int EPI_WARPS = CVT ? 4 : 8;
+    // Epilogue warps: the plain store and the E2E ds epilogue keep up with four next to
+    // the converters; otherwise EW (8, or 16 for the straight-through epilogue of a
+    // shallow contraction, chosen per launch).
+    static constexpr int EPI_WARPS = CVT ? 4 : EW;
     // Per converter warp: the group constants (s, zq as fp32) of the stage it converts,
     // two per B tile row (the two 32-code halves of its 64 codes).
     static constexpr int CONST_BYTES = CVT_WARPS * 256 * 8;
@@ -657,7 +659,8 @@ struct PairCfg {
     static constexpr int OUT_BYTES = EPI_WARPS * 2048;
     static constexpr int SMEM = 1024 + STAGES * STAGE + CONST_BYTES + OUT_BYTES + 256;
 };
-static_assert(PairCfg<1, 3>::SMEM <= 232448 && PairCfg<1, 2>::SMEM <= 232448 && PairCfg<1, 4>::SMEM <= 232448,
+static_assert(PairCfg<1, 3>::SMEM <= 232448 && PairCfg<1, 2>::SMEM <= 232448 && PairCfg<1, 4>::SMEM <= 232448 &&
+                  PairCfg<0, 2, 16>::SMEM <= 232448,
               "pair kernel stages exceed the shared memory of a CTA");
 static_assert(sizeof(SharedCtl2) <= 256, "control block exceeds its slot");
 
@@ -893,12 +896,12 @@ struct StageWalk {
 //                warp's part of the B tile is written and fenced for the tensor core;
 //                the MMA issuer waits on it besides full[s] (which then counts A only)
 template <int EPI0, int EPI1, int BITS, int EPI_WARPS, int CVT>
-__global__ void __launch_bounds__((4 + EPI_WARPS + PairCfg<CVT, BITS>::CVT_WARPS) * 32, 1)
+__global__ void __launch_bounds__((4 + EPI_WARPS + PairCfg<CVT, BITS, EPI_WARPS>::CVT_WARPS) * 32, 1)
     k_gemm_tc2(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUtensorMap tmB0,
                const __grid_constant__ CUtensorMap tmA1, const __grid_constant__ CUtensorMap tmB1,
                const __grid_constant__ CUtensorMap tmO0, const __grid_constant__ CUtensorMap tmO1,
                const KParams p) {
-    using C = PairCfg<CVT, BITS>;
+    using C = PairCfg<CVT, BITS, EPI_WARPS>;
     static_assert(EPI_WARPS == C::EPI_WARPS, "the staging area is sized for C::EPI_WARPS epilogue warps");
     constexpr int STAGES2 = C::STAGES;
     constexpr int STAGE2_BYTES = C::STAGE;
@@ -1128,12 +1131,19 @@ __global__ void __launch_bounds__((4 + EPI_WARPS + PairCfg<CVT, BITS>::CVT_WARPS
             const TileInfo ti = tile_info(p, t);
             const int row0 = ti.tm * BM2 + 128 * static_cast<int>(rank) + quad * 32;
             const uint32_t taddr = tmem_base + acc * ACC_COLS + ((quad * 32) << 16);
-            const int cols = ti.bn / SLICES;
+            // a slice holds whole groups where the epilogue reduces over groups (then
+            // some warps may have none)
+            const Prob &pe = ti.pi ? p.pr[1] : p.pr[0];
+            const bool reduces = ti.pi ? (EPI1 == 1 || EPI1 == 2) : (EPI0 == 1 || EPI0 == 2);
+            int cols = ti.bn / SLICES;
+            if (reduces && cols < pe.group) cols = pe.group;
+            const int c_begin = half_slice * cols;
+            const int c_end = c_begin + cols < ti.bn ? c_begin + cols : ti.bn;
             os.map = ti.pi ? &tmO1 : &tmO0;
             if (ti.pi == 0)
-                drain_accumulator<EPI0, BITS>(p.pr[0], taddr, row0, ti.n0, half_slice * cols, (half_slice + 1) * cols, os);
+                drain_accumulator<EPI0, BITS>(p.pr[0], taddr, row0, ti.n0, c_begin, c_end, os);
             else
-                drain_accumulator<EPI1, BITS>(p.pr[1], taddr, row0, ti.n0, half_slice * cols, (half_slice + 1) * cols, os);
+                drain_accumulator<EPI1, BITS>(p.pr[1], taddr, row0, ti.n0, c_begin, c_end, os);
             tc_fence_before();
             mbar_arrive_cluster(acc_empty0 + 8u * acc);
         }
@@ -1338,10 +1348,10 @@ cudaError_t launch_variant(const CUtensorMap (&maps)[6], const KParams &p, int g
     return cudaGetLastError();
 }
 
-template <int EPI0, int EPI1, int BITS, int CVT = 0>
+template <int EPI0, int EPI1, int BITS, int CVT = 0, int EW = 8>
 cudaError_t launch_pair_variant(const CUtensorMap (&maps)[6], const KParams &p, int grid, int dev_id,
                                 cudaStream_t st) {
-    using C = PairCfg<CVT, BITS>;
+    using C = PairCfg<CVT, BITS, CVT ? 4 : EW>;
     auto kern = k_gemm_tc2<EPI0, EPI1, BITS, C::EPI_WARPS, CVT>;
     static std::atomic<uint64_t> done{0};
     const uint64_t bit = 1ull << (dev_id & 63);
@@ -1645,6 +1655,11 @@ cudaError_t launch_gemm_tc_group(const GemmProblem *probs, int nprob, const Devi
                 if (nprob > 1) return cudaErrorInvalidValue;
                 return launch_pair_variant<0, 0, 2>(maps, p, grid, dev.device, st);
             case Epi::kFqGrad:
+                // The straight-through epilogue outlasts a main loop 2048 deep with eight
+                // warps (per-tile timestamps on the 70B gate backward: 13.7 us against
+                // 10 us); sixteen keep up there (3% off that backward) but cost 1.7% on
+                // 4096-deep contractions, where eight already hide behind the main loop.
+                if (probs[0].GK <= 2048) return launch_pair_variant<1, 0, 2, 0, 16>(maps, p, grid, dev.device, st);
                 return launch_pair_variant<1, 0, 2>(maps, p, grid, dev.device, st);
             case Epi::kE2eDs:
                 switch (probs[0].epi.bits) {

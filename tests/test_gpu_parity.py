@@ -129,6 +129,37 @@ def test_quantizer_ragged_tiles_bit_exact(orc, dtype, N, K, bits, g):
         assert_bits_equal(to_np(dq), orc.dequant_packed(p_ref, zq_ref, s, K, bits, g), "dequant")
 
 
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+def test_w_hat_outputs_aligned_to_16_bytes_only(orc, dtype):
+    """W-hat written into a buffer that starts 16 bytes past a 32-byte boundary (the
+    ABI asks for 16): the prepass and the dequantize kernel then store each 16-weight
+    chunk as two 16-byte halves instead of one 32-byte store.  Both give the oracle's
+    values, bit for bit, and leave the bytes around the view untouched."""
+    N, K, bits, g = 40, 1152, 2, 64
+    d = synthetic.draw_linear(np.random.default_rng(77), 1, N, K, 0.02, dtype)
+    Wn = synthetic.as_f32_numpy(d["W"])
+    s, z = synthetic.perturb_quant_params(*orc.minmax_init(Wn, bits, g), 5)
+    W, sd, zd = d["W"].cuda(), torch.from_numpy(s).cuda(), torch.from_numpy(z).cuda()
+    wh_ref = orc.fake_quant(Wn, s, z, bits, g)[0]
+    p_ref, zq_ref = orc.pack(Wn, s, z, bits, g)
+    p, zq = eqat.pack_codes(W, sd, zd, bits, g)
+    tdt = W.dtype
+    shift = 16 // W.element_size()
+    for which in ("fake_quant", "dequant"):
+        buf = torch.full((N * K + 2 * shift,), 7.0, dtype=tdt, device="cuda")
+        view = buf[shift:shift + N * K].view(N, K)
+        assert view.data_ptr() % 32 == 16
+        if which == "fake_quant":
+            eqat.fake_quant(W, sd, zd, bits, g, want_code=False, want_mask=False, W_hat=view)
+            ref = wh_ref
+        else:
+            eqat.dequant_codes(p, zq, sd, K, bits, g, out=view)
+            ref = orc.dequant_packed(p_ref, zq_ref, s, K, bits, g)
+        assert_bits_equal(to_np(view), ref if dtype == "f32" else bf16_round(ref), which)
+        edge = to_np(buf)
+        assert (edge[:shift] == 7.0).all() and (edge[shift + N * K:] == 7.0).all(), f"{which} wrote outside its view"
+
+
 @pytest.mark.parametrize("dtype", ["f32", "bf16"])
 @pytest.mark.parametrize("bits", [2, 3, 4])
 def test_codes_at_and_around_rounding_boundaries_bit_exact(orc, dtype, bits):

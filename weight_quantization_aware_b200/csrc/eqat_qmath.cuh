@@ -190,4 +190,45 @@ __device__ __forceinline__ void store8<float>(float *p, const float (&v)[8]) {
     reinterpret_cast<float4 *>(p)[1] = make_float4(v[4], v[5], v[6], v[7]);
 }
 
+// 32 bytes from 8 registers in one instruction (p 32-byte aligned).
+__device__ __forceinline__ void st_global_v8(void *p, uint32_t a, uint32_t b, uint32_t c, uint32_t d, uint32_t e,
+                                             uint32_t f, uint32_t g, uint32_t h) {
+    asm volatile("st.global.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(p), "r"(a), "r"(b), "r"(c),
+                 "r"(d), "r"(e), "r"(f), "r"(g), "r"(h)
+                 : "memory");
+}
+
+// 16 consecutive values. With V8 (p 32-byte aligned) every store instruction
+// writes whole 32-byte sectors: a warp whose lanes store 32 consecutive bytes each
+// as two 16-byte halves leaves every sector half written by each instruction, and
+// such stores stream at about half the rate of whole-sector ones on B200 (3.5
+// against 6.1-6.8 TB/s over a 1 GiB buffer).  Without V8, two 16-byte stores.
+template <typename T, bool V8>
+__device__ __forceinline__ void store16(T *p, const float (&v)[16]);
+
+template <>
+__device__ __forceinline__ void store16<__nv_bfloat16, true>(__nv_bfloat16 *p, const float (&v)[16]) {
+    st_global_v8(p, pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]), pack_bf16x2(v[4], v[5]),
+                 pack_bf16x2(v[6], v[7]), pack_bf16x2(v[8], v[9]), pack_bf16x2(v[10], v[11]),
+                 pack_bf16x2(v[12], v[13]), pack_bf16x2(v[14], v[15]));
+}
+template <>
+__device__ __forceinline__ void store16<float, true>(float *p, const float (&v)[16]) {
+#pragma unroll
+    for (int h = 0; h < 2; ++h)
+        st_global_v8(p + 8 * h, __float_as_uint(v[8 * h]), __float_as_uint(v[8 * h + 1]), __float_as_uint(v[8 * h + 2]),
+                     __float_as_uint(v[8 * h + 3]), __float_as_uint(v[8 * h + 4]), __float_as_uint(v[8 * h + 5]),
+                     __float_as_uint(v[8 * h + 6]), __float_as_uint(v[8 * h + 7]));
+}
+template <>
+__device__ __forceinline__ void store16<__nv_bfloat16, false>(__nv_bfloat16 *p, const float (&v)[16]) {
+    store8<__nv_bfloat16>(p, *reinterpret_cast<const float(*)[8]>(&v[0]));
+    store8<__nv_bfloat16>(p + 8, *reinterpret_cast<const float(*)[8]>(&v[8]));
+}
+template <>
+__device__ __forceinline__ void store16<float, false>(float *p, const float (&v)[16]) {
+    store8<float>(p, *reinterpret_cast<const float(*)[8]>(&v[0]));
+    store8<float>(p + 8, *reinterpret_cast<const float(*)[8]>(&v[8]));
+}
+
 }  // namespace eqat

@@ -357,7 +357,7 @@ int tile_grid(int64_t n, const DeviceInfo &dev) {
 // W-hat = (clamp(round(W/s) + zr, 0, Q) - zr) s = clamp(round(W/s), -zr, Q - zr) s
 // (all integer-valued until the one rounded product), with the code and the
 // straight-through mask 0 <= round(W/s) + zr <= Q when asked for.
-template <typename O, bool CODES>
+template <typename O, bool CODES, bool V8>
 __device__ __forceinline__ bool fake_quant_chunk(const float (&w)[16], const GroupConst &c, float Q, int64_t e0,
                                                  bool exact, O *__restrict__ W_hat, uint8_t *__restrict__ code,
                                                  uint8_t *__restrict__ mask) {
@@ -396,8 +396,7 @@ __device__ __forceinline__ bool fake_quant_chunk(const float (&w)[16], const Gro
         float wh[16];
 #pragma unroll
         for (int j = 0; j < 16; j += 2) f2_unpack(f2_mul(f2_pack(v[j], v[j + 1]), s2), wh[j], wh[j + 1]);
-        store8<O>(W_hat + e0, *reinterpret_cast<const float(*)[8]>(&wh[0]));
-        store8<O>(W_hat + e0 + 8, *reinterpret_cast<const float(*)[8]>(&wh[8]));
+        store16<O, V8>(W_hat + e0, wh);
     }
     if (CODES) {
         // code = v + zr: the low byte of M + zr + v (exact)
@@ -415,7 +414,8 @@ __device__ __forceinline__ bool fake_quant_chunk(const float (&w)[16], const Gro
     return false;
 }
 
-template <typename T, typename O, bool CODES>
+// V8: W_hat is 32-byte aligned (whole-sector stores).
+template <typename T, typename O, bool CODES, bool V8>
 __global__ void __launch_bounds__(kTileThreads, kTileBlocksPerSm)
     k_fake_quant(const T *__restrict__ W, const float *__restrict__ s, const float *__restrict__ z, int64_t n,
                  int gshift, float Q, O *__restrict__ W_hat, uint8_t *__restrict__ code,
@@ -424,7 +424,7 @@ __global__ void __launch_bounds__(kTileThreads, kTileBlocksPerSm)
     __shared__ PendingChunk queue[kTileWarps * kQueue<T>];
     walk_warp_tiles<T, false>(W, s, z, n, gshift, Q, nullptr, gc, queue,
                               [&](const float (&w)[16], const GroupConst &c, int64_t e0, bool exact) {
-                                  return fake_quant_chunk<O, CODES>(w, c, Q, e0, exact, W_hat, code, mask);
+                                  return fake_quant_chunk<O, CODES, V8>(w, c, Q, e0, exact, W_hat, code, mask);
                               });
 }
 
@@ -543,7 +543,8 @@ __device__ __forceinline__ float step_value(const float *s, int64_t g) { return 
 __device__ __forceinline__ float step_value(const __half *s, int64_t g) { return __half2float(__ldg(s + g)); }
 
 // S: fp32 step sizes, or fp16 ones (fp16 step-size storage), widened exactly.
-template <int BITS, typename O, typename S>
+// V8: W_hat is 32-byte aligned (whole-sector stores).
+template <int BITS, typename O, typename S, bool V8>
 __global__ void __launch_bounds__(kThreads)
     k_dequant(const uint8_t *__restrict__ codes, const uint8_t *__restrict__ zq,
               const S *__restrict__ s, int64_t n_chunks, int gshift, O *__restrict__ W_hat) {
@@ -561,8 +562,7 @@ __global__ void __launch_bounds__(kThreads)
 #pragma unroll
         for (int j = 0; j < 16; j += 2)
             f2_unpack(f2_mul(f2_sub(f2_pack(f[j], f[j + 1]), mz2), s2), wh[j], wh[j + 1]);
-        store8<O>(W_hat + e0, *reinterpret_cast<const float(*)[8]>(&wh[0]));
-        store8<O>(W_hat + e0 + 8, *reinterpret_cast<const float(*)[8]>(&wh[8]));
+        store16<O, V8>(W_hat + e0, wh);
     }
 }
 
@@ -594,20 +594,30 @@ cudaError_t pack_dispatch(const T *W, const float *s, const float *z, int64_t n,
     return cudaGetLastError();
 }
 
-template <typename O, typename S>
-cudaError_t dequant_dispatch(const uint8_t *codes, const uint8_t *zq, const S *s, int64_t n,
-                             int bits, int group, O *W_hat, const DeviceInfo &dev,
-                             cudaStream_t st) {
+template <typename O, typename S, bool V8>
+cudaError_t dequant_dispatch_v(const uint8_t *codes, const uint8_t *zq, const S *s, int64_t n,
+                               int bits, int group, O *W_hat, const DeviceInfo &dev,
+                               cudaStream_t st) {
     const int gshift = group_shift(group);
     const int64_t chunks = n / 16;
     const int grid = grid_for(chunks, dev);
     switch (bits) {
-        case 2: k_dequant<2, O, S><<<grid, kThreads, 0, st>>>(codes, zq, s, chunks, gshift, W_hat); break;
-        case 3: k_dequant<3, O, S><<<grid, kThreads, 0, st>>>(codes, zq, s, chunks, gshift, W_hat); break;
-        case 4: k_dequant<4, O, S><<<grid, kThreads, 0, st>>>(codes, zq, s, chunks, gshift, W_hat); break;
+        case 2: k_dequant<2, O, S, V8><<<grid, kThreads, 0, st>>>(codes, zq, s, chunks, gshift, W_hat); break;
+        case 3: k_dequant<3, O, S, V8><<<grid, kThreads, 0, st>>>(codes, zq, s, chunks, gshift, W_hat); break;
+        case 4: k_dequant<4, O, S, V8><<<grid, kThreads, 0, st>>>(codes, zq, s, chunks, gshift, W_hat); break;
         default: return cudaErrorInvalidValue;
     }
     return cudaGetLastError();
+}
+
+inline bool aligned32(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 31u) == 0; }
+
+template <typename O, typename S>
+cudaError_t dequant_dispatch(const uint8_t *codes, const uint8_t *zq, const S *s, int64_t n,
+                             int bits, int group, O *W_hat, const DeviceInfo &dev,
+                             cudaStream_t st) {
+    if (aligned32(W_hat)) return dequant_dispatch_v<O, S, true>(codes, zq, s, n, bits, group, W_hat, dev, st);
+    return dequant_dispatch_v<O, S, false>(codes, zq, s, n, bits, group, W_hat, dev, st);
 }
 
 }  // namespace
@@ -631,15 +641,20 @@ cudaError_t launch_fake_quant(const void *W, bool w_f32, const float *s, const f
     using bf = __nv_bfloat16;
     const bool codes = code || mask;
     const int gshift = group_shift(group);
+    const bool v8 = aligned32(W_hat);
+#define EQAT_FQ_LAUNCH_V(TW, TO, CODES, V8)                                                                  \
+    k_fake_quant<TW, TO, CODES, V8><<<tile_grid<TW>(n, dev), kTileThreads, 0, st>>>(                        \
+        static_cast<const TW *>(W), s, z, n, gshift, Q, static_cast<TO *>(W_hat), code, mask)
 #define EQAT_FQ_LAUNCH(TW, TO)                                                                              \
     do {                                                                                                    \
-        const int grid = tile_grid<TW>(n, dev);                                                             \
-        if (codes)                                                                                          \
-            k_fake_quant<TW, TO, true><<<grid, kTileThreads, 0, st>>>(static_cast<const TW *>(W), s, z, n,  \
-                                                                     gshift, Q, static_cast<TO *>(W_hat), code, mask); \
+        if (codes && v8)                                                                                    \
+            EQAT_FQ_LAUNCH_V(TW, TO, true, true);                                                           \
+        else if (codes)                                                                                     \
+            EQAT_FQ_LAUNCH_V(TW, TO, true, false);                                                          \
+        else if (v8)                                                                                        \
+            EQAT_FQ_LAUNCH_V(TW, TO, false, true);                                                          \
         else                                                                                                \
-            k_fake_quant<TW, TO, false><<<grid, kTileThreads, 0, st>>>(static_cast<const TW *>(W), s, z, n, \
-                                                                      gshift, Q, static_cast<TO *>(W_hat), code, mask); \
+            EQAT_FQ_LAUNCH_V(TW, TO, false, false);                                                         \
     } while (0)
     if (w_f32 && out_f32)
         EQAT_FQ_LAUNCH(float, float);
@@ -650,6 +665,7 @@ cudaError_t launch_fake_quant(const void *W, bool w_f32, const float *s, const f
     else
         EQAT_FQ_LAUNCH(bf, bf);
 #undef EQAT_FQ_LAUNCH
+#undef EQAT_FQ_LAUNCH_V
     return cudaGetLastError();
 }
 

@@ -131,6 +131,25 @@ eqat_status eqat_pack_codes(const void *W, int wdt, const float *s, const float 
                             int64_t K, int bits, int group, uint8_t *codes, uint8_t *zq,
                             eqat_stream_t stream);
 
+/* a1 and a7 over the weight matrices of a whole block in one launch per eight
+ * layers (the 70B Block-AP sweep initialises and packs all seven linears of a
+ * decoder block together; small layers then share the waves of large ones
+ * instead of paying a launch ramp and tail each).  Layer i has W[i] [N[i], K[i]]
+ * and the outputs of eqat_minmax_init / eqat_pack_codes for it; results equal n
+ * single calls, bit for bit.  W, N, K, s, z, codes, zq are HOST arrays of n
+ * entries (0 <= n <= EQAT_MAX_MULTI) holding device pointers and sizes; every
+ * layer has dtype wdt and the same bits and group.  The layers' buffers must not
+ * overlap.  Arguments are checked layer by layer before any launch; an error
+ * launches nothing. */
+#define EQAT_MAX_MULTI 64
+eqat_status eqat_minmax_init_multi(int n, const void *const *W, int wdt, const int64_t *N, const int64_t *K,
+                                   int bits, int group, float *const *s, float *const *z,
+                                   eqat_stream_t stream);
+eqat_status eqat_pack_codes_multi(int n, const void *const *W, int wdt, const float *const *s,
+                                  const float *const *z, const int64_t *N, const int64_t *K, int bits,
+                                  int group, uint8_t *const *codes, uint8_t *const *zq,
+                                  eqat_stream_t stream);
+
 /* a3 (E2E-QP). Eq. 2 on frozen codes: W_hat = (W_q - zq) * s, dtype dt. */
 eqat_status eqat_dequant_codes(const uint8_t *codes, const uint8_t *zq, const float *s, int64_t N,
                                int64_t K, int bits, int group, void *W_hat, int dt,

@@ -135,6 +135,41 @@ def test_variant_entry_points_argument_errors(lib):
                                   16, 16, 64, 2, 64, P(0), 0, 0, st) == OK
 
 
+def test_multi_layer_entry_points_argument_errors(lib):
+    """Layer-by-layer validation of the block-wide init and pack: a bad layer
+    anywhere refuses the whole call before any launch."""
+    st = None
+    VP, I64 = ctypes.c_void_p, ctypes.c_int64
+
+    def arr(t, xs):
+        return (t * len(xs))(*xs)
+
+    def pack(n=2, W=(FAKE, FAKE), s=(FAKE, FAKE), z=(FAKE, FAKE), N=(16, 8), K=(64, 128), codes=(FAKE, FAKE),
+             zq=(FAKE, FAKE), bits=2, group=64):
+        return lib.eqat_pack_codes_multi(n, arr(VP, W), 1, arr(VP, s), arr(VP, z), arr(I64, N), arr(I64, K),
+                                         bits, group, arr(VP, codes), arr(VP, zq), st)
+
+    def init(n=2, W=(FAKE, FAKE), N=(16, 8), K=(64, 128), s=(FAKE, FAKE), z=(FAKE, FAKE), group=64):
+        return lib.eqat_minmax_init_multi(n, arr(VP, W), 1, arr(I64, N), arr(I64, K), 2, group, arr(VP, s),
+                                          arr(VP, z), st)
+
+    assert pack(n=-1) == SHAPE
+    assert pack(n=65) == SHAPE
+    assert lib.eqat_pack_codes_multi(1, None, 1, None, None, None, None, 2, 64, None, None, st) == NULL
+    assert pack(N=(16, 12)) == SHAPE            # second layer: N not a multiple of 8
+    assert pack(K=(64, 96)) == SHAPE            # second layer: K not a multiple of g
+    assert pack(codes=(FAKE, 0)) == NULL
+    assert pack(zq=(FAKE + 4, FAKE)) == ALIGN
+    assert pack(bits=5) == UNSUP
+    assert pack(N=(0, 0)) == OK                 # nothing to pack, no device touched
+    assert pack(n=0) == OK
+    assert init(N=(16, 12)) == SHAPE
+    assert init(s=(FAKE, 0)) == NULL
+    assert init(W=(FAKE + 2, FAKE)) == ALIGN
+    assert init(group=48) == UNSUP
+    assert init(N=(0, 0)) == OK
+
+
 def test_binding_refuses_cpu_tensors():
     import torch
     W = torch.zeros(16, 64, dtype=torch.bfloat16)

@@ -78,6 +78,36 @@ def test_minmax_init_degenerate_groups(orc):
         assert_bits_equal(to_np(m), m_ref, "mask")
 
 
+@pytest.mark.parametrize("bits", [2, 3, 4])
+def test_codes_for_extreme_step_sizes_bit_exact(orc, bits):
+    """Groups whose W/s leaves every fp32 shortcut range: u = W/s between -2.5e7 and
+    -1.26e7 (where M + zr + u is negative but its bits, read as an integer and
+    reduced by those of M, would wrap around), below -2^31, above 2^22, and plain
+    ones beside them.  Codes clamp to 0 or Q exactly as the definition says, in the
+    prepass (code, mask, W-hat) and in pack."""
+    g = 64
+    rng = np.random.default_rng(600 + bits)
+    W = rng.standard_normal((8, 8 * g)).astype(np.float32)
+    W = torch.from_numpy(W).to(torch.bfloat16).float().numpy()
+    Q = (1 << bits) - 1
+    steps = np.array([1 / 1.5e7, 1 / 1.9e7, 1e-9, 1e-30, 3e-8, 0.4, 1 / 1.3e7, 2.0], np.float32)
+    s = np.tile(steps, (8, 1))
+    s = np.roll(s, 3, axis=1) * np.float32(1)
+    z = rng.uniform(0, Q, (8, 8)).astype(np.float32)
+    Wd, sd, zd = torch.from_numpy(W).to(torch.bfloat16).cuda(), torch.from_numpy(s).cuda(), torch.from_numpy(z).cuda()
+    u = W.reshape(8, 8, g) / s[:, :, None]
+    assert ((u > -2.5e7) & (u < -1.26e7)).sum() > 100 and (u < -2.0 ** 31).any() and (u > 2.0 ** 22).any()
+    wh_ref, c_ref, m_ref, _ = orc.fake_quant(W, s, z, bits, g)
+    wh, c, m = eqat.fake_quant(Wd, sd, zd, bits, g)
+    assert_bits_equal(to_np(c), c_ref, "code")
+    assert_bits_equal(to_np(m), m_ref, "mask")
+    assert_bits_equal(to_np(wh), bf16_round(wh_ref), "W_hat")
+    p_ref, zq_ref = orc.pack(W, s, z, bits, g)
+    p, zq = eqat.pack_codes(Wd, sd, zd, bits, g)
+    assert_bits_equal(to_np(zq), zq_ref, "zq")
+    assert_bits_equal(to_np(p), p_ref, "packed codes")
+
+
 @pytest.mark.parametrize("dtype", ["bf16", "f32"])
 @pytest.mark.parametrize("trained", [False, True])
 @pytest.mark.parametrize("bits,g", [(2, 64), (3, 128), (4, 32)])
@@ -127,6 +157,46 @@ def test_quantizer_ragged_tiles_bit_exact(orc, dtype, N, K, bits, g):
         assert_bits_equal(to_np(zq), zq_ref, "zq")
         dq = eqat.dequant_codes(p, zq, sd, K, bits, g, torch.float32)
         assert_bits_equal(to_np(dq), orc.dequant_packed(p_ref, zq_ref, s, K, bits, g), "dequant")
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+@pytest.mark.parametrize("bits,g", [(2, 64), (3, 128), (4, 32)])
+def test_multi_layer_init_and_pack_bit_exact(orc, dtype, bits, g):
+    """min-max init and pack of several layers in one call (tiles and units
+    numbered through the layers, one launch per eight layers): the results of
+    every layer equal the oracle's, bit for bit.  Eleven layers (two launches),
+    of unlike shapes: one below a single warp tile, ragged tile counts, an empty
+    layer in the middle, and one whose rows are the concatenation of two others."""
+    shapes = [(8, 256), (40, 1152), (72, 4224), (16, 128), (0, 512), (264, 1024), (8, 128 * 5),
+              (136, 512), (48, 2048), (24, 384), (16, 1024)]
+    rng = np.random.default_rng(800 + bits + g)
+    Ws, Wns = [], []
+    for i, (N, K) in enumerate(shapes):
+        d = synthetic.draw_linear(rng, 1, N, K, 0.02, dtype)
+        Ws.append(d["W"].cuda())
+        Wns.append(synthetic.as_f32_numpy(d["W"]))
+    ss, zs = eqat.minmax_init_multi(Ws, bits, g)
+    refs = [orc.minmax_init(Wn, bits, g) if Wn.size else (np.zeros((0, Wn.shape[1] // g), np.float32),) * 2
+            for Wn in Wns]
+    for i, (s_ref, z_ref) in enumerate(refs):
+        assert_bits_equal(to_np(ss[i]), s_ref, f"s[{i}]")
+        assert_bits_equal(to_np(zs[i]), z_ref, f"z[{i}]")
+    # trained-state steps on every other layer, so clamped codes occur too
+    sp, zp = [], []
+    for i, (s_ref, z_ref) in enumerate(refs):
+        if i % 2 and s_ref.size:
+            s_ref, z_ref = synthetic.perturb_quant_params(s_ref, z_ref, i)
+        sp.append(s_ref)
+        zp.append(z_ref)
+    codes, zqs = eqat.pack_codes_multi(Ws, [torch.from_numpy(a).cuda() for a in sp],
+                                       [torch.from_numpy(a).cuda() for a in zp], bits, g)
+    for i, Wn in enumerate(Wns):
+        if not Wn.size:
+            assert codes[i].numel() == 0
+            continue
+        p_ref, zq_ref = orc.pack(Wn, sp[i], zp[i], bits, g)
+        assert_bits_equal(to_np(codes[i]), p_ref, f"codes[{i}]")
+        assert_bits_equal(to_np(zqs[i]), zq_ref, f"zq[{i}]")
 
 
 @pytest.mark.parametrize("dtype", ["bf16", "f32"])

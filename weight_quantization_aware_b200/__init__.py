@@ -49,6 +49,8 @@ def load_library():
         "eqat_minmax_init": [P, I, I64, I64, I, I, P, P, P],
         "eqat_fake_quant": [P, I, P, P, I64, I64, I, I, P, P, P, P],
         "eqat_pack_codes": [P, I, P, P, I64, I64, I, I, P, P, P],
+        "eqat_minmax_init_multi": [I, P, I, P, P, I, I, P, P, P],
+        "eqat_pack_codes_multi": [I, P, I, P, P, P, P, I, I, P, P, P],
         "eqat_dequant_codes": [P, P, P, I64, I64, I, I, P, I, P],
         "eqat_fq_linear_fwd": [P, P, I, P, P, P, I64, I64, I64, I, I, P, SZ, P],
         "eqat_fq_linear_bwd": [P, P, I, P, P, P, P, P, P, P, I64, I64, I64, I, I, P, SZ, I, P],
@@ -187,6 +189,78 @@ def minmax_init(W, bits, group, s=None, z=None):
     z = torch.empty((N, G), dtype=torch.float32, device=W.device) if z is None else _req(z, "z", torch.float32)
     _call("eqat_minmax_init", _p(W), _dt(W), N, K, bits, group, _p(s), _p(z), _stream())
     return s, z
+
+
+def _ptr_array(ts):
+    return (ctypes.c_void_p * max(1, len(ts)))(*[_p(t) for t in ts])
+
+
+def _i64_array(xs):
+    return (ctypes.c_int64 * max(1, len(xs)))(*xs)
+
+
+def _same_kind(Ws):
+    if not Ws:
+        return None
+    dt = Ws[0].dtype
+    for i, W in enumerate(Ws):
+        if W.dim() != 2:
+            raise ValueError(f"W[{i}] must be 2-D")
+        if W.dtype != dt:
+            raise TypeError(f"W[{i}] is {W.dtype}, W[0] is {dt}: one dtype per call")
+        _req(W, f"W[{i}]")
+    return dt
+
+
+def minmax_init_multi(Ws, bits, group, ss=None, zs=None):
+    """min-max init of several weight matrices (the linears of a block) in one
+    launch per eight layers: returns lists (s, z) as minmax_init gives per layer."""
+    Ws = list(Ws)
+    _same_kind(Ws)
+    ss = [None] * len(Ws) if ss is None else list(ss)
+    zs = [None] * len(Ws) if zs is None else list(zs)
+    if len(ss) != len(Ws) or len(zs) != len(Ws):
+        raise ValueError("one s and one z per W")
+    for i, W in enumerate(Ws):
+        N, K = W.shape
+        G = K // group if group else 0
+        _shape(ss[i], f"s[{i}]", (N, G)); _shape(zs[i], f"z[{i}]", (N, G))
+        ss[i] = torch.empty((N, G), dtype=torch.float32, device=W.device) if ss[i] is None else \
+            _req(ss[i], f"s[{i}]", torch.float32)
+        zs[i] = torch.empty((N, G), dtype=torch.float32, device=W.device) if zs[i] is None else \
+            _req(zs[i], f"z[{i}]", torch.float32)
+    if Ws:
+        _call("eqat_minmax_init_multi", len(Ws), _ptr_array(Ws), _dt(Ws[0]),
+              _i64_array([W.shape[0] for W in Ws]), _i64_array([W.shape[1] for W in Ws]), bits, group,
+              _ptr_array(ss), _ptr_array(zs), _stream())
+    return ss, zs
+
+
+def pack_codes_multi(Ws, ss, zs, bits, group, codes=None, zqs=None):
+    """pack of several weight matrices (the linears of a block) in one launch per
+    eight layers: returns lists (codes, zq) as pack_codes gives per layer."""
+    Ws, ss, zs = list(Ws), list(ss), list(zs)
+    _same_kind(Ws)
+    codes = [None] * len(Ws) if codes is None else list(codes)
+    zqs = [None] * len(Ws) if zqs is None else list(zqs)
+    if not (len(ss) == len(zs) == len(codes) == len(zqs) == len(Ws)):
+        raise ValueError("one s, z, codes and zq per W")
+    for i, W in enumerate(Ws):
+        N, K = W.shape
+        G = K // group
+        _shape(ss[i], f"s[{i}]", (N, G)); _shape(zs[i], f"z[{i}]", (N, G))
+        _shape(codes[i], f"codes[{i}]", (N, packed_row_bytes(K, bits))); _shape(zqs[i], f"zq[{i}]", (N, G))
+        _req(ss[i], f"s[{i}]", torch.float32); _req(zs[i], f"z[{i}]", torch.float32)
+        if codes[i] is None:
+            codes[i] = torch.empty((N, packed_row_bytes(K, bits)), dtype=torch.uint8, device=W.device)
+        if zqs[i] is None:
+            zqs[i] = torch.empty((N, G), dtype=torch.uint8, device=W.device)
+        _req(codes[i], f"codes[{i}]", torch.uint8); _req(zqs[i], f"zq[{i}]", torch.uint8)
+    if Ws:
+        _call("eqat_pack_codes_multi", len(Ws), _ptr_array(Ws), _dt(Ws[0]), _ptr_array(ss), _ptr_array(zs),
+              _i64_array([W.shape[0] for W in Ws]), _i64_array([W.shape[1] for W in Ws]), bits, group,
+              _ptr_array(codes), _ptr_array(zqs), _stream())
+    return codes, zqs
 
 
 def fake_quant(W, s, z, bits, group, want_w_hat=True, want_code=True, want_mask=True, W_hat=None):

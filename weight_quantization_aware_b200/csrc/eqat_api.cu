@@ -10,6 +10,7 @@
 #include <cstdlib>
 #include <cstring>
 #include <mutex>
+#include <vector>
 
 #include "../../include/eqat.h"
 #include "eqat_internal.h"
@@ -306,6 +307,82 @@ eqat_status eqat_pack_codes(const void *W, int wdt, const float *s, const float 
     EQAT_CUDA(eqat::launch_pack(W, wdt == EQAT_F32, s, z, N, K, bits, group, codes, zq, dev,
                                 reinterpret_cast<cudaStream_t>(stream)),
               "pack_codes");
+    return EQAT_OK;
+}
+
+// n layers of one multi-layer call: at most EQAT_MAX_MULTI, host arrays present.
+eqat_status check_multi(int n, const void *a, const void *b, const void *c) {
+    if (n < 0 || n > EQAT_MAX_MULTI) return fail(EQAT_ERR_SHAPE, "layer count must be 0..EQAT_MAX_MULTI");
+    if (n > 0 && (!a || !b || !c)) return fail(EQAT_ERR_NULL, "a layer array is NULL");
+    return EQAT_OK;
+}
+
+eqat_status eqat_minmax_init_multi(int n, const void *const *W, int wdt, const int64_t *N, const int64_t *K,
+                                   int bits, int group, float *const *s, float *const *z,
+                                   eqat_stream_t stream) {
+    DeviceInfo dev;
+    EQAT_TRY(check_dtype(wdt));
+    EQAT_TRY(check_multi(n, W, N, K));
+    EQAT_TRY(check_multi(n, s, z, W));
+    std::vector<eqat::QuantLayerArgs> layers(static_cast<size_t>(n));
+    for (int i = 0; i < n; ++i) {
+        EQAT_TRY(check_common(0, N[i], K[i], bits, group));
+        const int64_t ng = N[i] * (K[i] / group);
+        EQAT_TRY(check_ptr(W[i], N[i] * K[i], "W[i]"));
+        EQAT_TRY(check_ptr(s[i], ng, "s[i]"));
+        EQAT_TRY(check_ptr(z[i], ng, "z[i]"));
+        eqat::QuantLayerArgs &a = layers[static_cast<size_t>(i)];
+        a = eqat::QuantLayerArgs{};
+        a.W = W[i];
+        a.s_out = s[i];
+        a.z_out = z[i];
+        a.N = N[i];
+        a.K = K[i];
+    }
+    int64_t total = 0;
+    for (const auto &a : layers) total += a.N * a.K;
+    if (total == 0) return EQAT_OK;
+    EQAT_TRY(get_device(dev));
+    EQAT_CUDA(eqat::launch_minmax_init_multi(layers.data(), n, wdt == EQAT_F32, bits, group, dev,
+                                             reinterpret_cast<cudaStream_t>(stream)),
+              "minmax_init_multi");
+    return EQAT_OK;
+}
+
+eqat_status eqat_pack_codes_multi(int n, const void *const *W, int wdt, const float *const *s,
+                                  const float *const *z, const int64_t *N, const int64_t *K, int bits, int group,
+                                  uint8_t *const *codes, uint8_t *const *zq, eqat_stream_t stream) {
+    DeviceInfo dev;
+    EQAT_TRY(check_dtype(wdt));
+    EQAT_TRY(check_multi(n, W, N, K));
+    EQAT_TRY(check_multi(n, s, z, W));
+    EQAT_TRY(check_multi(n, codes, zq, W));
+    std::vector<eqat::QuantLayerArgs> layers(static_cast<size_t>(n));
+    for (int i = 0; i < n; ++i) {
+        EQAT_TRY(check_common(0, N[i], K[i], bits, group));
+        const int64_t ng = N[i] * (K[i] / group);
+        EQAT_TRY(check_ptr(W[i], N[i] * K[i], "W[i]"));
+        EQAT_TRY(check_ptr(s[i], ng, "s[i]"));
+        EQAT_TRY(check_ptr(z[i], ng, "z[i]"));
+        EQAT_TRY(check_ptr(codes[i], code_bytes(N[i], K[i], bits), "codes[i]"));
+        EQAT_TRY(check_ptr(zq[i], ng, "zq[i]"));
+        eqat::QuantLayerArgs &a = layers[static_cast<size_t>(i)];
+        a = eqat::QuantLayerArgs{};
+        a.W = W[i];
+        a.s = s[i];
+        a.z = z[i];
+        a.codes = codes[i];
+        a.zq = zq[i];
+        a.N = N[i];
+        a.K = K[i];
+    }
+    int64_t total = 0;
+    for (const auto &a : layers) total += a.N * a.K;
+    if (total == 0) return EQAT_OK;
+    EQAT_TRY(get_device(dev));
+    EQAT_CUDA(eqat::launch_pack_multi(layers.data(), n, wdt == EQAT_F32, bits, group, dev,
+                                      reinterpret_cast<cudaStream_t>(stream)),
+              "pack_codes_multi");
     return EQAT_OK;
 }
 

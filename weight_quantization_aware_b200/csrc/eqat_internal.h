@@ -20,6 +20,22 @@ cudaError_t current_device_info(DeviceInfo &info);
 
 // ---------------------------------------------------------------- HBM kernels
 // All element counts are validated by the caller; every launch goes on `st`.
+
+// One weight matrix of a multi-layer init or pack: W [N, K]; init writes s_out,
+// z_out; pack reads s, z and writes codes, zq.
+struct QuantLayerArgs {
+    const void *W;
+    const float *s, *z;
+    float *s_out, *z_out;
+    uint8_t *codes, *zq;
+    int64_t N, K;
+};
+// Every layer of one call in one launch (up to eight per launch); empty layers
+// are skipped.
+cudaError_t launch_minmax_init_multi(const QuantLayerArgs *layers, int n, bool w_f32, int bits, int group,
+                                     const DeviceInfo &dev, cudaStream_t st);
+cudaError_t launch_pack_multi(const QuantLayerArgs *layers, int n, bool w_f32, int bits, int group,
+                              const DeviceInfo &dev, cudaStream_t st);
 cudaError_t launch_minmax_init(const void *W, bool w_f32, int64_t N, int64_t K, int bits, int group,
                                float *s, float *z, const DeviceInfo &dev, cudaStream_t st);
 cudaError_t launch_fake_quant(const void *W, bool w_f32, const float *s, const float *z, int64_t N,

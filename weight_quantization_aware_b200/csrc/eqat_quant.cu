@@ -39,19 +39,49 @@ inline int grid_for(int64_t work_items, const DeviceInfo &dev, int per_thread = 
 // A thread holds 8 consecutive weights of one group; TPG = G/8 threads cover a
 // group and reduce min/max with xor shuffles; UNROLL independent groups per
 // thread keep 128 bytes (bf16) of loads in flight per thread.
-template <typename T, int G>
-__global__ void __launch_bounds__(kThreads, 4) k_minmax_init(const T *__restrict__ W, int64_t n_groups,
-                                                             float Q, float *__restrict__ s,
-                                                             float *__restrict__ z) {
+//
+// One launch covers NL weight matrices (NL = 1, or the linears of a block): the
+// warps walk units of GPW * UNROLL groups, numbered through the layers in order
+// (a unit never spans two layers), so small layers share the waves of large ones
+// instead of paying a launch ramp and tail each.
+constexpr int kInitUnroll = 4;  // 16-byte words in flight per thread
+template <int G>
+constexpr int kInitUnit = (32 / (G / 8)) * kInitUnroll;  // groups per warp unit
+
+template <typename T, int NL>
+struct InitLayers {
+    const T *W[NL];
+    float *s[NL];
+    float *z[NL];
+    int64_t n_groups[NL];
+    int64_t unit_end[NL];  // units of layers 0..i; entries past the last layer repeat it
+};
+
+template <typename T, int G, int NL>
+__global__ void __launch_bounds__(kThreads, 4) k_minmax_init(const __grid_constant__ InitLayers<T, NL> L, float Q) {
     constexpr int TPG = G / 8;
     constexpr int GPW = 32 / TPG;  // groups per warp per unrolled slot
-    constexpr int UNROLL = 4;  // 16-byte words in flight per thread
+    constexpr int UNROLL = kInitUnroll;
     const int lane = threadIdx.x & 31;
     const int sub = lane % TPG;
     const int slot = lane / TPG;
     const int64_t warp = (static_cast<int64_t>(blockIdx.x) * kThreads + threadIdx.x) >> 5;
     const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * kThreads) >> 5;
-    for (int64_t base = warp * (GPW * UNROLL); base < n_groups; base += nwarps * (GPW * UNROLL)) {
+    const int64_t n_units = L.unit_end[NL - 1];
+    int li = 0;
+    int64_t unit_begin = 0;
+    for (int64_t unit = warp; unit < n_units; unit += nwarps) {
+        if constexpr (NL > 1) {
+            while (unit >= L.unit_end[li]) {
+                unit_begin = L.unit_end[li];
+                ++li;
+            }
+        }
+        const T *__restrict__ W = L.W[li];
+        float *__restrict__ s = L.s[li];
+        float *__restrict__ z = L.z[li];
+        const int64_t n_groups = L.n_groups[li];
+        const int64_t base = (unit - unit_begin) * (GPW * UNROLL);
         Raw8<T> raw[UNROLL];
 #pragma unroll
         for (int u = 0; u < UNROLL; ++u) {
@@ -156,14 +186,21 @@ __device__ __forceinline__ uint32_t h2_clamp(uint32_t a, uint32_t lo, uint32_t h
 constexpr int kTileThreads = 256;
 constexpr int kTileWarps = kTileThreads / 32;
 constexpr int kTileBlocksPerSm = 3;
+// CPL: 16-weight chunks per lane and warp tile (two or three 16-byte loads each in
+// flight per lane).  Three for bf16 weights in the prepass and in multi-layer pack;
+// four in single-layer pack.  The choice is measured (70B block, w2g64): with four,
+// the prepass and multi-layer pack spill a few registers at the 80 that three CTAs
+// per SM allow and lose 2-4%; single-layer pack runs 3.5% faster with four.
 template <typename T>
-constexpr int kChunksPerLane = sizeof(T) == 2 ? 4 : 2;  // 128 bytes of loads in flight per lane
-template <typename T>
-constexpr int kWarpTile = 32 * kChunksPerLane<T> * 16;  // weights; a multiple of every group size
-template <typename T>
-constexpr int kWarpGroups = kWarpTile<T> / 32;  // groups of a tile at most (g = 32)
-template <typename T>
-constexpr int kLaneGroups = (kWarpGroups<T> + 31) / 32;
+constexpr int kChunksPerLane = sizeof(T) == 2 ? 3 : 2;
+template <typename T, int NL>
+constexpr int kPackChunksPerLane = (sizeof(T) == 2 && NL == 1) ? 4 : kChunksPerLane<T>;
+template <int CPL>
+constexpr int kWarpTile = 32 * CPL * 16;  // weights; a multiple of every group size
+template <int CPL>
+constexpr int kWarpGroups = kWarpTile<CPL> / 32;  // groups of a tile at most (g = 32)
+template <int CPL>
+constexpr int kLaneGroups = (kWarpGroups<CPL> + 31) / 32;
 
 struct GroupConst {
     float sc, rcp, zr, band;  // s, RN(1/s), zr, near band (below)
@@ -236,14 +273,14 @@ __device__ __forceinline__ float exact_round(float w, float s, float u) {
 
 // The constants of the groups of one warp tile: lane l takes groups l, l + 32.
 // With clamp_z (pack) zr = zq = clamp(round(z), 0, Q), written to zq here.
-template <typename T>
+template <int CPL>
 __device__ __forceinline__ void tile_group_consts(const float *__restrict__ s, const float *__restrict__ z,
                                                   int64_t e_tile, int64_t n, int gshift, float Q, bool clamp_z,
                                                   int lane, GroupConst *gc, uint8_t *__restrict__ zq) {
-    const int gpt = kWarpTile<T> >> gshift;
+    const int gpt = kWarpTile<CPL> >> gshift;
     const int64_t g0 = e_tile >> gshift, n_groups = n >> gshift;
 #pragma unroll
-    for (int k = 0; k < kLaneGroups<T>; ++k) {
+    for (int k = 0; k < kLaneGroups<CPL>; ++k) {
         const int gi = lane + 32 * k;
         const int64_t g = g0 + gi;
         if (gi < gpt && g < n_groups) {
@@ -256,34 +293,57 @@ __device__ __forceinline__ void tile_group_consts(const float *__restrict__ s, c
     }
 }
 
-// A chunk left for the exact pass: where it starts and its group's constants.
+// A chunk left for the exact pass: where it starts (the layer in the top byte)
+// and its group's constants.
 struct PendingChunk {
     int64_t e0;
     GroupConst c;
 };
+constexpr int kLayerShift = 56;
 // Per warp: fewer than 32 entries wait between tiles, and a tile adds at most one
 // per chunk.
-template <typename T>
-constexpr int kQueue = 32 + 32 * kChunksPerLane<T>;
+template <int CPL>
+constexpr int kQueue = 32 + 32 * CPL;
 
 // Walks the warp tiles: chunk(w, group constants, e0, exact) handles the 16
 // weights at e0 and returns true when the fast pass (exact = false) left one of
 // them near a rounding boundary.  Such chunks go to the warp's queue in shared
 // memory; every 32 of them are redone with exact = true, one per lane, with the
 // weights reloaded, and the rest at the end.
-template <typename T, bool CLAMP_Z, typename Chunk>
-__device__ __forceinline__ void walk_warp_tiles(const T *__restrict__ W, const float *__restrict__ s,
-                                                const float *__restrict__ z, int64_t n, int gshift, float Q,
-                                                uint8_t *__restrict__ zq, GroupConst *gc_all,
-                                                PendingChunk *queue_all, Chunk chunk) {
-    constexpr int CPL = kChunksPerLane<T>, WT = kWarpTile<T>;
+//
+// The tiles are numbered through NL weight matrices in order (NL = 1, or the
+// linears of a block in one launch); chunk() also receives the layer.
+template <typename T, int NL>
+struct TileLayers {
+    const T *W[NL];
+    const float *s[NL];
+    const float *z[NL];
+    uint8_t *zq[NL];     // pack: zq out (NULL otherwise)
+    uint8_t *codes[NL];  // pack: codes out
+    int64_t n[NL];
+    int32_t tile_end[NL];  // warp tiles of layers 0..i (< 2^31); entries past the last layer repeat it
+};
+
+template <typename T, bool CLAMP_Z, int NL, int CPL, typename Chunk>
+__device__ __forceinline__ void walk_warp_tiles(const TileLayers<T, NL> &L, int gshift, float Q,
+                                                GroupConst *gc_all, PendingChunk *queue_all, Chunk chunk) {
+    constexpr int WT = kWarpTile<CPL>;
     const int lane = threadIdx.x & 31, wib = threadIdx.x >> 5;
-    GroupConst *gc = gc_all + wib * kWarpGroups<T>;
-    PendingChunk *queue = queue_all + wib * kQueue<T>;
+    GroupConst *gc = gc_all + wib * kWarpGroups<CPL>;
+    PendingChunk *queue = queue_all + wib * kQueue<CPL>;
     int queued = 0;  // warp-uniform
-    const int64_t n_tiles = (n + WT - 1) / WT, stride = static_cast<int64_t>(gridDim.x) * kTileWarps;
-    for (int64_t tile = static_cast<int64_t>(blockIdx.x) * kTileWarps + wib; tile < n_tiles; tile += stride) {
-        const int64_t e_tile = tile * WT;
+    // tile indices: 32-bit with several layers (fewer live registers), 64-bit with one
+    using TI = std::conditional_t<(NL > 1), int32_t, int64_t>;
+    const TI n_tiles = NL > 1 ? L.tile_end[NL - 1] : (L.n[0] + WT - 1) / WT;
+    const TI stride = static_cast<TI>(gridDim.x) * kTileWarps;
+    int li = 0;
+    for (TI tile = static_cast<TI>(blockIdx.x) * kTileWarps + wib; tile < n_tiles; tile += stride) {
+        if constexpr (NL > 1) {
+            while (tile >= L.tile_end[li]) ++li;
+        }
+        const T *__restrict__ W = L.W[li];
+        const int64_t n = L.n[li];
+        const int64_t e_tile = static_cast<int64_t>(NL > 1 && li > 0 ? tile - L.tile_end[li > 0 ? li - 1 : 0] : tile) * WT;
         const bool last_tile = tile + stride >= n_tiles;
         // A whole tile (every tile but the last of the layer) runs without bounds
         // checks.
@@ -300,7 +360,7 @@ __device__ __forceinline__ void walk_warp_tiles(const T *__restrict__ W, const f
             }
         }
         __syncwarp();  // the previous tile's reads of gc are done
-        tile_group_consts<T>(s, z, e_tile, n, gshift, Q, CLAMP_Z, lane, gc, zq);
+        tile_group_consts<CPL>(L.s[li], L.z[li], e_tile, n, gshift, Q, CLAMP_Z, lane, gc, L.zq[li]);
         __syncwarp();
         uint32_t pending = 0u;  // bit j: chunk j left for the exact pass
         auto fast_pass = [&](auto whole_tag) {
@@ -310,7 +370,7 @@ __device__ __forceinline__ void walk_warp_tiles(const T *__restrict__ W, const f
                 if (decltype(whole_tag)::value || e_tile + off < n) {
                     float w[16];
                     unpack16(raw[j], w);
-                    if (chunk(w, gc[off >> gshift], e_tile + off, false)) pending |= 1u << j;
+                    if (chunk(w, gc[off >> gshift], e_tile + off, false, li)) pending |= 1u << j;
                 }
             }
         };
@@ -324,7 +384,10 @@ __device__ __forceinline__ void walk_warp_tiles(const T *__restrict__ W, const f
                 const int off = (j * 32 + lane) * 16;
                 const bool p = (pending >> j) & 1u;
                 const uint32_t ballot = __ballot_sync(0xffffffffu, p);
-                if (p) queue[queued + __popc(ballot & ((1u << lane) - 1u))] = PendingChunk{e_tile + off, gc[off >> gshift]};
+                if (p)
+                    queue[queued + __popc(ballot & ((1u << lane) - 1u))] = PendingChunk{
+                        NL > 1 ? (e_tile + off) | (static_cast<int64_t>(li) << kLayerShift) : e_tile + off,
+                        gc[off >> gshift]};
                 queued += __popc(ballot);
             }
         }
@@ -335,9 +398,11 @@ __device__ __forceinline__ void walk_warp_tiles(const T *__restrict__ W, const f
             __syncwarp();
             if (lane < count) {
                 const PendingChunk pc = queue[queued - count + lane];
+                const int pl = NL > 1 ? static_cast<int>(pc.e0 >> kLayerShift) : 0;
+                const int64_t e0 = NL > 1 ? pc.e0 & ((int64_t{1} << kLayerShift) - 1) : pc.e0;
                 float w[16];
-                unpack16(load_raw16<T>(W + pc.e0), w);
-                (void)chunk(w, pc.c, pc.e0, true);
+                unpack16(load_raw16<T>(L.W[pl] + e0), w);
+                (void)chunk(w, pc.c, e0, true, pl);
             }
             queued -= count;
             __syncwarp();
@@ -345,9 +410,14 @@ __device__ __forceinline__ void walk_warp_tiles(const T *__restrict__ W, const f
     }
 }
 
-template <typename T>
-int tile_grid(int64_t n, const DeviceInfo &dev) {
-    const int64_t tiles = (n + kWarpTile<T> - 1) / kWarpTile<T>;
+template <int CPL>
+__host__ __device__ __forceinline__ int64_t warp_tiles(int64_t n) {
+    return (n + kWarpTile<CPL> - 1) / kWarpTile<CPL>;
+}
+
+template <int CPL>
+int tile_grid(int64_t n, const DeviceInfo &dev, int64_t tiles = -1) {
+    if (tiles < 0) tiles = warp_tiles<CPL>(n);
     const int64_t blocks = (tiles + kTileWarps - 1) / kTileWarps;
     return static_cast<int>(
         std::max<int64_t>(1, std::min<int64_t>(blocks, static_cast<int64_t>(dev.sm_count) * kTileBlocksPerSm)));
@@ -420,12 +490,21 @@ __global__ void __launch_bounds__(kTileThreads, kTileBlocksPerSm)
     k_fake_quant(const T *__restrict__ W, const float *__restrict__ s, const float *__restrict__ z, int64_t n,
                  int gshift, float Q, O *__restrict__ W_hat, uint8_t *__restrict__ code,
                  uint8_t *__restrict__ mask) {
-    __shared__ GroupConst gc[kTileWarps * kWarpGroups<T>];
-    __shared__ PendingChunk queue[kTileWarps * kQueue<T>];
-    walk_warp_tiles<T, false>(W, s, z, n, gshift, Q, nullptr, gc, queue,
-                              [&](const float (&w)[16], const GroupConst &c, int64_t e0, bool exact) {
-                                  return fake_quant_chunk<O, CODES, V8>(w, c, Q, e0, exact, W_hat, code, mask);
-                              });
+    constexpr int CPL = kChunksPerLane<T>;
+    __shared__ GroupConst gc[kTileWarps * kWarpGroups<CPL>];
+    __shared__ PendingChunk queue[kTileWarps * kQueue<CPL>];
+    TileLayers<T, 1> L;
+    L.W[0] = W;
+    L.s[0] = s;
+    L.z[0] = z;
+    L.zq[0] = nullptr;
+    L.codes[0] = nullptr;
+    L.n[0] = n;
+    L.tile_end[0] = static_cast<int32_t>(warp_tiles<CPL>(n));
+    walk_warp_tiles<T, false, 1, CPL>(L, gshift, Q, gc, queue,
+                                 [&](const float (&w)[16], const GroupConst &c, int64_t e0, bool exact, int) {
+                                     return fake_quant_chunk<O, CODES, V8>(w, c, Q, e0, exact, W_hat, code, mask);
+                                 });
 }
 
 // ------------------------------------------------------------------ pack
@@ -502,16 +581,29 @@ __device__ __forceinline__ bool pack_chunk(const float (&w)[16], const GroupCons
     return false;
 }
 
-template <typename T, int BITS>
+template <typename T, int BITS, int NL>
 __global__ void __launch_bounds__(kTileThreads, kTileBlocksPerSm)
-    k_pack(const T *__restrict__ W, const float *__restrict__ s, const float *__restrict__ z, int64_t n, int gshift,
-           float Q, uint8_t *__restrict__ codes, uint8_t *__restrict__ zq) {
-    __shared__ GroupConst gc[kTileWarps * kWarpGroups<T>];
-    __shared__ PendingChunk queue[kTileWarps * kQueue<T>];
-    walk_warp_tiles<T, true>(W, s, z, n, gshift, Q, zq, gc, queue,
-                             [&](const float (&w)[16], const GroupConst &c, int64_t e0, bool exact) {
-                                 return pack_chunk<BITS>(w, c, Q, e0, exact, codes);
-                             });
+    k_pack(const __grid_constant__ TileLayers<T, NL> L, int gshift, float Q) {
+    constexpr int CPL = kPackChunksPerLane<T, NL>;
+    __shared__ GroupConst gc[kTileWarps * kWarpGroups<CPL>];
+    __shared__ PendingChunk queue[kTileWarps * kQueue<CPL>];
+    // Several layers: the table goes to shared memory, where a layer's entries are
+    // read per tile instead of being held in registers.
+    if constexpr (NL > 1) {
+        __shared__ TileLayers<T, NL> Ls;
+        constexpr int kWords = sizeof(TileLayers<T, NL>) / 8;
+        for (int i = threadIdx.x; i < kWords; i += kTileThreads)
+            reinterpret_cast<uint64_t *>(&Ls)[i] = reinterpret_cast<const uint64_t *>(&L)[i];
+        __syncthreads();
+        walk_warp_tiles<T, true, NL, CPL>(Ls, gshift, Q, gc, queue,
+                                          [&](const float (&w)[16], const GroupConst &c, int64_t e0, bool exact,
+                                              int li) { return pack_chunk<BITS>(w, c, Q, e0, exact, Ls.codes[li]); });
+    } else {
+        walk_warp_tiles<T, true, 1, CPL>(L, gshift, Q, gc, queue,
+                                         [&](const float (&w)[16], const GroupConst &c, int64_t e0, bool exact, int) {
+                                             return pack_chunk<BITS>(w, c, Q, e0, exact, L.codes[0]);
+                                         });
+    }
 }
 
 // ------------------------------------------------------------------ E2E dequant
@@ -566,32 +658,88 @@ __global__ void __launch_bounds__(kThreads)
     }
 }
 
-template <typename T>
-cudaError_t minmax_dispatch(const T *W, int64_t n_groups, int group, float Q, float *s, float *z,
-                            const DeviceInfo &dev, cudaStream_t st) {
-    const int grid = grid_for(n_groups * group, dev, 8 * 4);
+// Layers per multi-layer launch (a Llama block has seven linears); more are
+// launched in batches of this many.
+constexpr int kMultiLayers = 8;
+
+// One launch over layers a[0..n) (1 <= n <= NL, every layer non-empty).
+template <typename T, int G, int NL>
+cudaError_t minmax_launch(const QuantLayerArgs *a, int n, float Q, const DeviceInfo &dev, cudaStream_t st) {
+    InitLayers<T, NL> L{};
+    int64_t units = 0, weights = 0;
+    for (int i = 0; i < NL; ++i) {
+        const QuantLayerArgs &x = a[i < n ? i : n - 1];
+        const int64_t ng = x.N * (x.K / G);
+        L.W[i] = static_cast<const T *>(x.W);
+        L.s[i] = x.s_out;
+        L.z[i] = x.z_out;
+        L.n_groups[i] = ng;
+        if (i < n) {
+            units += (ng + kInitUnit<G> - 1) / kInitUnit<G>;
+            weights += ng * G;
+        }
+        L.unit_end[i] = units;
+    }
+    k_minmax_init<T, G, NL><<<grid_for(weights, dev, 8 * 4), kThreads, 0, st>>>(L, Q);
+    return cudaGetLastError();
+}
+
+template <typename T, int NL>
+cudaError_t minmax_dispatch(const QuantLayerArgs *a, int n, int group, float Q, const DeviceInfo &dev,
+                            cudaStream_t st) {
     switch (group) {
-        case 32: k_minmax_init<T, 32><<<grid, kThreads, 0, st>>>(W, n_groups, Q, s, z); break;
-        case 64: k_minmax_init<T, 64><<<grid, kThreads, 0, st>>>(W, n_groups, Q, s, z); break;
-        case 128: k_minmax_init<T, 128><<<grid, kThreads, 0, st>>>(W, n_groups, Q, s, z); break;
+        case 32: return minmax_launch<T, 32, NL>(a, n, Q, dev, st);
+        case 64: return minmax_launch<T, 64, NL>(a, n, Q, dev, st);
+        case 128: return minmax_launch<T, 128, NL>(a, n, Q, dev, st);
+        default: return cudaErrorInvalidValue;
+    }
+}
+
+template <typename T, int NL>
+cudaError_t pack_dispatch(const QuantLayerArgs *a, int n, int bits, int group, const DeviceInfo &dev,
+                          cudaStream_t st) {
+    TileLayers<T, NL> L{};
+    int64_t tiles = 0;
+    for (int i = 0; i < NL; ++i) {
+        const QuantLayerArgs &x = a[i < n ? i : n - 1];
+        L.W[i] = static_cast<const T *>(x.W);
+        L.s[i] = x.s;
+        L.z[i] = x.z;
+        L.zq[i] = x.zq;
+        L.codes[i] = x.codes;
+        L.n[i] = x.N * x.K;
+        if (i < n) tiles += warp_tiles<kPackChunksPerLane<T, NL>>(x.N * x.K);
+        if (tiles > INT32_MAX) return cudaErrorInvalidValue;  // beyond any device memory
+        L.tile_end[i] = static_cast<int32_t>(tiles);
+    }
+    const int gshift = group_shift(group);
+    const int grid = tile_grid<kPackChunksPerLane<T, NL>>(0, dev, tiles);
+    const float Q = static_cast<float>((1 << bits) - 1);
+    switch (bits) {
+        case 2: k_pack<T, 2, NL><<<grid, kTileThreads, 0, st>>>(L, gshift, Q); break;
+        case 3: k_pack<T, 3, NL><<<grid, kTileThreads, 0, st>>>(L, gshift, Q); break;
+        case 4: k_pack<T, 4, NL><<<grid, kTileThreads, 0, st>>>(L, gshift, Q); break;
         default: return cudaErrorInvalidValue;
     }
     return cudaGetLastError();
 }
 
-template <typename T>
-cudaError_t pack_dispatch(const T *W, const float *s, const float *z, int64_t n, int bits, int group,
-                          uint8_t *codes, uint8_t *zq, const DeviceInfo &dev, cudaStream_t st) {
-    const int gshift = group_shift(group);
-    const int grid = tile_grid<T>(n, dev);
-    const float Q = static_cast<float>((1 << bits) - 1);
-    switch (bits) {
-        case 2: k_pack<T, 2><<<grid, kTileThreads, 0, st>>>(W, s, z, n, gshift, Q, codes, zq); break;
-        case 3: k_pack<T, 3><<<grid, kTileThreads, 0, st>>>(W, s, z, n, gshift, Q, codes, zq); break;
-        case 4: k_pack<T, 4><<<grid, kTileThreads, 0, st>>>(W, s, z, n, gshift, Q, codes, zq); break;
-        default: return cudaErrorInvalidValue;
+// Drops empty layers, then one launch per kMultiLayers layers (single-layer
+// kernels for one layer).
+template <typename Launch>
+cudaError_t for_layer_batches(const QuantLayerArgs *layers, int n, Launch launch) {
+    QuantLayerArgs batch[kMultiLayers];
+    int m = 0;
+    for (int i = 0; i < n; ++i) {
+        if (layers[i].N * layers[i].K == 0) continue;
+        batch[m++] = layers[i];
+        if (m == kMultiLayers || i == n - 1) {
+            const cudaError_t e = launch(batch, m);
+            if (e != cudaSuccess) return e;
+            m = 0;
+        }
     }
-    return cudaGetLastError();
+    return m ? launch(batch, m) : cudaSuccess;
 }
 
 template <typename O, typename S, bool V8>
@@ -622,13 +770,28 @@ cudaError_t dequant_dispatch(const uint8_t *codes, const uint8_t *zq, const S *s
 
 }  // namespace
 
+cudaError_t launch_minmax_init_multi(const QuantLayerArgs *layers, int n, bool w_f32, int bits, int group,
+                                     const DeviceInfo &dev, cudaStream_t st) {
+    const float Q = static_cast<float>((1 << bits) - 1);
+    return for_layer_batches(layers, n, [&](const QuantLayerArgs *b, int m) {
+        using bf = __nv_bfloat16;
+        if (m == 1)
+            return w_f32 ? minmax_dispatch<float, 1>(b, 1, group, Q, dev, st)
+                         : minmax_dispatch<bf, 1>(b, 1, group, Q, dev, st);
+        return w_f32 ? minmax_dispatch<float, kMultiLayers>(b, m, group, Q, dev, st)
+                     : minmax_dispatch<bf, kMultiLayers>(b, m, group, Q, dev, st);
+    });
+}
+
 cudaError_t launch_minmax_init(const void *W, bool w_f32, int64_t N, int64_t K, int bits, int group,
                                float *s, float *z, const DeviceInfo &dev, cudaStream_t st) {
-    const int64_t n_groups = N * (K / group);
-    if (n_groups == 0) return cudaSuccess;
-    const float Q = static_cast<float>((1 << bits) - 1);
-    if (w_f32) return minmax_dispatch(static_cast<const float *>(W), n_groups, group, Q, s, z, dev, st);
-    return minmax_dispatch(static_cast<const __nv_bfloat16 *>(W), n_groups, group, Q, s, z, dev, st);
+    QuantLayerArgs a{};
+    a.W = W;
+    a.s_out = s;
+    a.z_out = z;
+    a.N = N;
+    a.K = K;
+    return launch_minmax_init_multi(&a, 1, w_f32, bits, group, dev, st);
 }
 
 cudaError_t launch_fake_quant(const void *W, bool w_f32, const float *s, const float *z, int64_t N,
@@ -637,13 +800,14 @@ cudaError_t launch_fake_quant(const void *W, bool w_f32, const float *s, const f
                               cudaStream_t st) {
     const int64_t n = N * K;
     if (n == 0) return cudaSuccess;
+    if (warp_tiles<kChunksPerLane<float>>(n) > INT32_MAX) return cudaErrorInvalidValue;  // beyond any memory
     const float Q = static_cast<float>((1 << bits) - 1);
     using bf = __nv_bfloat16;
     const bool codes = code || mask;
     const int gshift = group_shift(group);
     const bool v8 = aligned32(W_hat);
 #define EQAT_FQ_LAUNCH_V(TW, TO, CODES, V8)                                                                  \
-    k_fake_quant<TW, TO, CODES, V8><<<tile_grid<TW>(n, dev), kTileThreads, 0, st>>>(                        \
+    k_fake_quant<TW, TO, CODES, V8><<<tile_grid<kChunksPerLane<TW>>(n, dev), kTileThreads, 0, st>>>(                        \
         static_cast<const TW *>(W), s, z, n, gshift, Q, static_cast<TO *>(W_hat), code, mask)
 #define EQAT_FQ_LAUNCH(TW, TO)                                                                              \
     do {                                                                                                    \
@@ -669,13 +833,30 @@ cudaError_t launch_fake_quant(const void *W, bool w_f32, const float *s, const f
     return cudaGetLastError();
 }
 
+cudaError_t launch_pack_multi(const QuantLayerArgs *layers, int n, bool w_f32, int bits, int group,
+                              const DeviceInfo &dev, cudaStream_t st) {
+    return for_layer_batches(layers, n, [&](const QuantLayerArgs *b, int m) {
+        using bf = __nv_bfloat16;
+        if (m == 1)
+            return w_f32 ? pack_dispatch<float, 1>(b, 1, bits, group, dev, st)
+                         : pack_dispatch<bf, 1>(b, 1, bits, group, dev, st);
+        return w_f32 ? pack_dispatch<float, kMultiLayers>(b, m, bits, group, dev, st)
+                     : pack_dispatch<bf, kMultiLayers>(b, m, bits, group, dev, st);
+    });
+}
+
 cudaError_t launch_pack(const void *W, bool w_f32, const float *s, const float *z, int64_t N,
                         int64_t K, int bits, int group, uint8_t *codes, uint8_t *zq,
                         const DeviceInfo &dev, cudaStream_t st) {
-    const int64_t n = N * K;
-    if (n == 0) return cudaSuccess;
-    if (w_f32) return pack_dispatch(static_cast<const float *>(W), s, z, n, bits, group, codes, zq, dev, st);
-    return pack_dispatch(static_cast<const __nv_bfloat16 *>(W), s, z, n, bits, group, codes, zq, dev, st);
+    QuantLayerArgs a{};
+    a.W = W;
+    a.s = s;
+    a.z = z;
+    a.codes = codes;
+    a.zq = zq;
+    a.N = N;
+    a.K = K;
+    return launch_pack_multi(&a, 1, w_f32, bits, group, dev, st);
 }
 
 cudaError_t launch_dequant(const uint8_t *codes, const uint8_t *zq, const void *s, bool s_f16, int64_t N,

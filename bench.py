@@ -484,6 +484,8 @@ def run_ours(args):
     if ip is not None:
         for k in ("init", "pack", "prepass", "dequant"):
             hbm.setdefault(k, {})["llama2-70b-block"] = ip[k]
+        for k in ("init", "pack"):
+            hbm[k]["llama2-70b-block_per_layer"] = ip[k + "_per_layer"]
     for k, ms, b in (("init", mean["init"], init_b), ("pack", mean["pack"], pack_b)):
         gbs = b / (ms * 1e-3) / 1e9
         hbm.setdefault(k, {})["in_step"] = {"GBps": round(gbs, 1), "frac": round(gbs / peaks["hbm_gbs"], 4),
@@ -919,48 +921,70 @@ def decode_gemv(dev, peaks, budget_bytes=300_000_000):
 def initpack_70b_block(dev, peaks, reps=5):
     """HBM throughput of the four quantizer kernels over all seven linears of the
     Llama-2-70B block (855.6 M bf16 weights, w2g64): min-max init, pack, the Block-AP
-    prepass (W-hat only) and the E2E-QP dequantization of the packed codes.  Per
-    kernel: sum of algorithmic bytes / sum of median CUDA-event times, each launch
-    alone after a clean L2 flush (a 512 MiB write, then a 256 MiB read of another
-    buffer, so the kernel starts on clean lines instead of first writing back the
-    flush's dirty ones).  Weights are seeded N(0, 0.015) with 0.1% x10 outliers,
-    drawn on the device."""
+    prepass (W-hat only) and the E2E-QP dequantization of the packed codes.
+
+    Init and pack of the block are one call each (eqat_minmax_init_multi,
+    eqat_pack_codes_multi: the sweep initialises and packs all seven linears
+    together); they are also timed layer by layer ("<kernel>_per_layer": sum of the
+    seven single-layer calls).  The prepass and dequant run once per linear inside
+    the training step, so they are timed layer by layer only.  GB/s = algorithmic
+    bytes / median CUDA-event time, each call alone after a clean L2 flush (a 512 MiB
+    write, then a 256 MiB read of another buffer, so the kernel starts on clean lines
+    instead of first writing back the flush's dirty ones).  Weights are seeded
+    N(0, 0.015) with 0.1% x10 outliers, drawn on the device."""
     wl = synthetic.WORKLOADS[5]
     gen = torch.Generator(device=dev)
     gen.manual_seed(1005)
     flush = L2Flush(dev)
-    kinds = ("init", "pack", "prepass", "dequant")
-    t = dict.fromkeys(kinds, 0.0)
-    nbytes = dict.fromkeys(kinds, 0)
     b, g = wl.bits, wl.group
+    Ws, ss, zs, codes, zqs = [], [], [], [], []
     for lin in wl.linears:
         N, K = lin.n, lin.k
         W = torch.randn(N, K, generator=gen, device=dev).mul_(wl.sigma)
         idx = torch.randint(0, N * K, ((N * K) // 1000,), generator=gen, device=dev)
         W.view(-1)[idx] *= 10.0
-        W = W.to(torch.bfloat16)
+        Ws.append(W.to(torch.bfloat16))
+        del W, idx
         G = K // g
-        s = torch.empty((N, G), dtype=torch.float32, device=dev)
-        z = torch.empty_like(s)
-        codes = torch.empty((N, eqat.packed_row_bytes(K, b)), dtype=torch.uint8, device=dev)
-        zq = torch.empty((N, G), dtype=torch.uint8, device=dev)
-        wh = torch.empty_like(W)
+        ss.append(torch.empty((N, G), dtype=torch.float32, device=dev))
+        zs.append(torch.empty((N, G), dtype=torch.float32, device=dev))
+        codes.append(torch.empty((N, eqat.packed_row_bytes(K, b)), dtype=torch.uint8, device=dev))
+        zqs.append(torch.empty((N, G), dtype=torch.uint8, device=dev))
+    wh = torch.empty(max(W.numel() for W in Ws), dtype=torch.bfloat16, device=dev)
+    kinds = ("init", "pack", "prepass", "dequant")
+    t = dict.fromkeys(kinds, 0.0)
+    nbytes = dict.fromkeys(kinds, 0)
+    for i, lin in enumerate(wl.linears):
+        N, K = lin.n, lin.k
+        W, s, z = Ws[i], ss[i], zs[i]
+        whi = wh[:N * K].view(N, K)
         calls = {
             "init": lambda: eqat.minmax_init(W, b, g, s=s, z=z),
-            "pack": lambda: eqat.pack_codes(W, s, z, b, g, codes=codes, zq=zq),
-            "prepass": lambda: eqat.fake_quant(W, s, z, b, g, want_code=False, want_mask=False, W_hat=wh),
-            "dequant": lambda: eqat.dequant_codes(codes, zq, s, K, b, g, out=wh),
+            "pack": lambda: eqat.pack_codes(W, s, z, b, g, codes=codes[i], zq=zqs[i]),
+            "prepass": lambda: eqat.fake_quant(W, s, z, b, g, want_code=False, want_mask=False, W_hat=whi),
+            "dequant": lambda: eqat.dequant_codes(codes[i], zqs[i], s, K, b, g, out=whi),
         }
         for k in kinds:  # in this order: pack and dequant read what init and pack wrote
             t[k] += timed_alone(calls[k], flush, reps)
             nbytes[k] += hbm_bytes(k, N, K, b, g)
-        del W, s, z, codes, zq, wh
+    block = {
+        "init": timed_alone(lambda: eqat.minmax_init_multi(Ws, b, g, ss, zs), flush, reps),
+        "pack": timed_alone(lambda: eqat.pack_codes_multi(Ws, ss, zs, b, g, codes, zqs), flush, reps),
+    }
+    del Ws, ss, zs, codes, zqs, wh
     torch.cuda.empty_cache()
+
+    def entry(ms, byts, how):
+        gbs = byts / (ms * 1e-3) / 1e9
+        return {"GBps": round(gbs, 1), "frac": round(gbs / peaks["hbm_gbs"], 4), "bytes": byts,
+                "us": round(ms * 1e3, 1), "how": how}
+
     out = {}
-    for k in kinds:
-        gbs = nbytes[k] / (t[k] * 1e-3) / 1e9
-        out[k] = {"GBps": round(gbs, 1), "frac": round(gbs / peaks["hbm_gbs"], 4), "bytes": nbytes[k],
-                  "us": round(t[k] * 1e3, 1)}
+    for k in ("init", "pack"):
+        out[k] = entry(block[k], nbytes[k], "one call for the seven linears")
+        out[k + "_per_layer"] = entry(t[k], nbytes[k], "seven single-layer calls")
+    for k in ("prepass", "dequant"):
+        out[k] = entry(t[k], nbytes[k], "seven single-layer calls")
     out["workload"] = wl.name + " (all 7 linears, 855.6 M weights)"
     return out
 
@@ -1175,6 +1199,7 @@ def main():
     ap.add_argument("--no-configs", action="store_true")
     ap.add_argument("--configs-only", action="store_true")
     ap.add_argument("--initpack70b-only", action="store_true")
+    ap.add_argument("--quant-multi-only", action="store_true")
     ap.add_argument("--dq-only", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-hbm", action="store_true")
@@ -1232,6 +1257,21 @@ def main():
         if eqat.device_error() != 0:
             raise RuntimeError("device error word set")
         print(json.dumps({"dq_only": "ok"}), flush=True)
+        return
+    if args.quant_multi_only:  # profiling aid: block-wide init and pack once each, Llama-2-7B block shapes
+        torch.cuda.set_device(0)
+        eqat.load_library()
+        dev = torch.device("cuda", 0)
+        gen = torch.Generator(device=dev)
+        gen.manual_seed(1007)
+        shapes = [(4096, 4096)] * 4 + [(11008, 4096), (11008, 4096), (4096, 11008)]
+        Ws = [(torch.randn(N, K, generator=gen, device=dev) * 0.02).to(torch.bfloat16) for N, K in shapes]
+        ss, zs = eqat.minmax_init_multi(Ws, 2, 64)
+        eqat.pack_codes_multi(Ws, ss, zs, 2, 64)
+        torch.cuda.synchronize()
+        if eqat.device_error() != 0:
+            raise RuntimeError("device error word set")
+        print(json.dumps({"quant_multi_only": "ok", "weights": sum(N * K for N, K in shapes)}), flush=True)
         return
     if args.initpack70b_only:  # profiling aid: just the 70B-block init/pack measurement
         torch.cuda.set_device(0)

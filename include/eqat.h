@@ -181,9 +181,15 @@ eqat_status eqat_fq_linear_bwd(const void *X, const void *W, int dt, const float
                                void *ws, size_t ws_bytes, int w_hat_in_ws, eqat_stream_t stream);
 
 /* a8. E2E-QP forward on frozen codes (modelfoundations Phase 2: only
- * dequantization in the graph): Y = X ((W_q - zq) s)^T.  At decode sizes (bf16,
- * 1 <= M <= 8, group 64 or 128) the codes are streamed once and W-hat is never
- * written: the inference GEMV of the packed model. */
+ * dequantization in the graph): Y = X ((W_q - zq) s)^T.  With a workspace, W-hat
+ * is dequantized into it first and stays there for eqat_dq_linear_bwd_s
+ * (w_hat_in_ws = 1).  In bf16 mode ws may be NULL (ws_bytes 0): W-hat is then made
+ * from the codes inside the contraction and kept nowhere (forward-only use; a
+ * backward after it takes w_hat_in_ws = 0).  That needs rows of codes a multiple of
+ * 16 bytes (K * bits / 8, or K for 3-bit codes); otherwise a NULL workspace is
+ * EQAT_ERR_WORKSPACE.  At decode sizes (bf16, 1 <= M <= 8, group 64 or 128, with a
+ * workspace) the codes are streamed once and W-hat is never written: the inference
+ * GEMV of the packed model. */
 eqat_status eqat_dq_linear_fwd(const void *X, int dt, const uint8_t *codes, const uint8_t *zq,
                                const float *s, void *Y, int64_t M, int64_t N, int64_t K, int bits,
                                int group, void *ws, size_t ws_bytes, eqat_stream_t stream);

@@ -108,6 +108,11 @@ def test_other_entry_points_argument_errors(lib):
                                   P(FAKE), 1 << 20, st) == SHAPE
     assert lib.eqat_dq_linear_bwd_s(P(FAKE), 1, P(FAKE), P(FAKE), P(FAKE), P(FAKE), P(0), P(0),
                                     16, 16, 64, 2, 64, P(0), 0, 0, st) == OK
+    # no workspace: only a bf16 forward whose code rows are a multiple of 16 bytes may do without one
+    assert lib.eqat_dq_linear_fwd(P(FAKE), 0, P(FAKE), P(FAKE), P(FAKE), P(FAKE), 16, 16, 64, 2, 64,
+                                  P(0), 0, st) == WS
+    assert lib.eqat_dq_linear_fwd(P(FAKE), 1, P(FAKE), P(FAKE), P(FAKE), P(FAKE), 16, 16, 32, 2, 32,
+                                  P(0), 0, st) == WS
     assert lib.eqat_selftest_bounded_wait(10, st) == SHAPE
 
 

@@ -11,7 +11,8 @@ Both paths are forced in fresh processes (EQAT_DQ_ONLOAD=1 / 0, CTA-pair tiles) 
 the same inputs.  Shapes cover 2-, 3- and 4-bit codes, groups of 32, 64 and 128 (a
 2-bit group of 32 splits a 16-byte code unit), ragged M, N and K, fp16 step sizes,
 and both N-tile widths the wave model picks.  A last case checks the default choice:
-a large layer at a small M takes the on-load path, a training-size M the other."""
+a forward without a workspace takes the on-load path, one with a workspace and
+every backward the other."""
 import os
 import subprocess
 import sys
@@ -114,32 +115,41 @@ def test_onload_equals_dequantize_path_and_oracle(orc, forced, i):
     assert_close(on[i]["dz"], dz_ref, TOL_RED, "dz")
 
 
-def test_default_choice_by_shape(orc, tmp_path):
-    """A 13824 x 5120 layer (Llama-2-13B gate_proj) at 64 tokens takes the on-load path by
-    default (equal bit for bit to the forced on-load run) and matches the oracle; at 512
-    tokens it takes the dequantize path.  The backward reuses the workspace flag of a
-    training step and must give the same results either way."""
+def test_default_choice_by_workspace(orc, tmp_path):
+    """By default the forward makes W-hat on load exactly when it gets no workspace
+    (keep_w_hat=False): its results then equal, bit for bit, the forced on-load
+    run's.  With a workspace it dequantizes into it, equal to the forced dequantize
+    run, and a backward reusing that W-hat equals the forced dequantize backward;
+    the backward never makes W-hat on load by default, also after a forward without
+    a workspace (w_hat_in_ws=False).  Layer: 13824 x 5120 (Llama-2-13B gate_proj) at
+    64 and 512 tokens; everything also matches the oracle."""
     N, K, bits, g = 13824, 5120, 2, 64
-    for M, mode in ((64, "1"), (512, "0")):
+    for M in (64, 512):
         Xn, dYn, packed, zq, s = make_case(orc, M, N, K, bits, g, "f32", 900 + M)
         X = torch.from_numpy(Xn).to(torch.bfloat16).cuda()
         dY = torch.from_numpy(dYn).to(torch.bfloat16).cuda()
         codes_d, zq_d, s_d = (torch.from_numpy(a).cuda() for a in (packed, zq, s))
         ws = eqat.workspace(M, N, K, bits, g, torch.bfloat16)
-        Y = eqat.dq_linear_fwd(X, codes_d, zq_d, s_d, bits, g, ws=ws)
-        dX, ds, dz = eqat.dq_linear_bwd(X, codes_d, zq_d, s_d, dY, bits, g, ws=ws, w_hat_in_ws=True)
+        Y_nows = eqat.dq_linear_fwd(X, codes_d, zq_d, s_d, bits, g, keep_w_hat=False)
+        dX_a, ds_a, dz_a = eqat.dq_linear_bwd(X, codes_d, zq_d, s_d, dY, bits, g, ws=ws, w_hat_in_ws=False)
+        Y_ws = eqat.dq_linear_fwd(X, codes_d, zq_d, s_d, bits, g, ws=ws)
+        dX_b, ds_b, dz_b = eqat.dq_linear_bwd(X, codes_d, zq_d, s_d, dY, bits, g, ws=ws, w_hat_in_ws=True)
         torch.cuda.synchronize()
         assert eqat.device_error() == 0
         p = tmp_path / f"m{M}.npz"
         np.savez(p, X=Xn, dY=dYn, codes=packed, zq=zq, s=s, bits=bits, group=g)
-        ref = run_forced(mode, [p])[0]
-        for name, got in (("Y", Y), ("dX", dX), ("ds", ds), ("dz", dz)):
-            assert np.array_equal(to_np(got), ref[name]), f"M={M} {name}: not the expected path's result"
+        on = run_forced("1", [p])[0]
+        off = run_forced("0", [p])[0]
+        assert np.array_equal(to_np(Y_nows), on["Y"]), f"M={M}: forward without a workspace is not the on-load one"
+        assert np.array_equal(to_np(Y_ws), off["Y"]), f"M={M}: forward with a workspace is not the dequantize one"
+        for name, a, b in (("dX", dX_a, dX_b), ("ds", ds_a, ds_b), ("dz", dz_a, dz_b)):
+            assert np.array_equal(to_np(a), off[name]), f"M={M} {name}: backward after a workspace-free forward"
+            assert np.array_equal(to_np(b), off[name]), f"M={M} {name}: backward reusing the forward's W-hat"
         rows = np.sort(np.random.default_rng(3).choice(M, min(M, 32), replace=False))
         wrows = np.sort(np.random.default_rng(4).choice(N, 256, replace=False))
         Y_ref = orc.dq_linear_fwd(Xn, packed, zq, s, bits, g, rows=rows)
         dX_ref, ds_ref, dz_ref = orc.dq_linear_bwd(Xn, packed, zq, s, dYn, bits, g, rows=rows, wrows=wrows)
-        assert_close(to_np(Y)[rows], Y_ref, TOL_GEMM, "Y")
-        assert_close(to_np(dX)[rows], dX_ref, TOL_GEMM, "dX")
-        assert_close(to_np(ds)[wrows], ds_ref, TOL_RED, "ds")
-        assert_close(to_np(dz)[wrows], dz_ref, TOL_RED, "dz")
+        assert_close(to_np(Y_nows)[rows], Y_ref, TOL_GEMM, "Y")
+        assert_close(to_np(dX_b)[rows], dX_ref, TOL_GEMM, "dX")
+        assert_close(to_np(ds_b)[wrows], ds_ref, TOL_RED, "ds")
+        assert_close(to_np(dz_b)[wrows], dz_ref, TOL_RED, "dz")

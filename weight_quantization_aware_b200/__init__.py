@@ -396,16 +396,24 @@ def fq_linear_bwd(X, W, s, z, dY, bits, group, need_dx=True, need_dw=True, need_
     return dX, dW, ds, dz
 
 
-def dq_linear_fwd(X, codes, zq, s, bits, group, ws=None, Y=None):
-    """E2E-QP forward on frozen codes: Y = X ((W_q - zq) s)^T; s fp32 or fp16."""
+def dq_linear_fwd(X, codes, zq, s, bits, group, ws=None, Y=None, keep_w_hat=True):
+    """E2E-QP forward on frozen codes: Y = X ((W_q - zq) s)^T; s fp32 or fp16.
+    keep_w_hat=False passes no workspace (ws must be None): W-hat is made from the
+    codes inside the contraction and kept nowhere (forward-only use)."""
     _dq_shapes(X, codes, zq, s, bits, group, Y=Y)
     _req(X, "X"); _req(codes, "codes", torch.uint8); _req(zq, "zq", torch.uint8); _req(s, "s")
     M, K = X.shape
     N = codes.shape[0]
     Y = torch.empty((M, N), dtype=X.dtype, device=X.device) if Y is None else _req(Y, "Y", X.dtype)
-    ws = _ws(ws, M, N, K, bits, group, X.dtype, X.device)
+    if keep_w_hat:
+        ws = _ws(ws, M, N, K, bits, group, X.dtype, X.device)
+        wsp, wsn = _p(ws), ws.numel()
+    else:
+        if ws is not None:
+            raise ValueError("keep_w_hat=False takes no workspace")
+        wsp, wsn = None, 0
     _call("eqat_dq_linear_fwd_ex", _p(X), _dt(X), _p(codes), _p(zq), _p(s), _sdt(s), _p(Y), M, N, K, bits,
-          group, _p(ws), ws.numel(), _stream())
+          group, wsp, wsn, _stream())
     return Y
 
 

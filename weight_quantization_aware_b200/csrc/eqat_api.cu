@@ -137,30 +137,37 @@ bool gemv_enabled() {
 // kernel wrote to the workspace.  Each B tile is converted once per 256-row M tile,
 // so the conversion work is M / 256 times the dequantize kernel's, while the HBM it
 // saves (a 2-byte W-hat written and read back, 0.25-1 byte codes read instead) does
-// not grow with M.  Measured on B200 (forward, w2g64 / w3g128): with one M tile
-// (M <= 256) it is 1.5x faster on a 13824 x 5120 layer, 1.2x on 28672 x 8192, about
-// even on 11008 x 4096 (3-bit) and 0.8x on 4096 x 4096, where few N tiles leave most
-// SMs idle;
-// at M >= 512 the dequantize + GEMM path wins (0.55-0.9x at M = 4096).  So it is used
-// for M <= 256 on layers of 2^25 weights or more.  The decision depends only on the
-// shapes, so a backward with w_hat_in_ws takes the same path as its forward.
-// EQAT_DQ_ONLOAD=1 uses it wherever the code layout allows, EQAT_DQ_ONLOAD=0 never
-// (measurement aids and the tests' way to compare the two paths).
+// not grow with M.  Measured on B200, forward alone: at M <= 256 it is 0.89-0.98x the
+// time of dequantize + GEMM on 2-bit layers of 2^25 weights or more (13824 x 5120,
+// 28672 x 8192), 1.03-1.26x on 3- and 4-bit layers and 1.3x on 4096 x 4096; at
+// M >= 512 1.2-2.3x.  In the backward (dX = dY W-hat with W-hat made on load, an
+// MN-major B) it is far slower: a forward + backward pair on the 70B gate at M = 64
+// takes 777 us against 499 us when the forward dequantizes into the workspace and
+// the backward reuses that W-hat.
+// So: the forward makes W-hat on load only when the caller passes no workspace (a
+// forward without one keeps nothing for a backward, and the dequantize path needs
+// one); with a workspace it dequantizes into it.  The backward never makes W-hat on
+// load.  EQAT_DQ_ONLOAD=1 uses it in both wherever the code layout allows,
+// EQAT_DQ_ONLOAD=0 never (measurement aids and the tests' way to compare the paths).
 int onload_mode() {
     static const int mode = [] {
         const char *v = std::getenv("EQAT_DQ_ONLOAD");
         if (v && v[0] == '0') return 0;
         if (v && v[0] == '1') return 1;
-        return -1;  // by shape
+        return -1;  // by the rule above
     }();
     return mode;
 }
 
-bool use_onload(int64_t M, int64_t N, int64_t K, int bits, int group) {
+bool fwd_onload(int64_t N, int64_t K, int bits, int group, bool have_ws) {
     if (!eqat::cvt_supported(N, K, bits, group)) return false;
     const int mode = onload_mode();
     if (mode >= 0) return mode == 1;
-    return M <= 256 && N * K >= (int64_t(1) << 25);
+    return !have_ws;
+}
+
+bool bwd_onload(int64_t N, int64_t K, int bits, int group) {
+    return eqat::cvt_supported(N, K, bits, group) && onload_mode() == 1;
 }
 
 eqat::CvtArgs cvt_args(const uint8_t *codes, const uint8_t *zq, const void *s, int sdt, int64_t N, int64_t K,
@@ -552,14 +559,16 @@ eqat_status eqat_dq_linear_fwd_ex(const void *X, int dt, const uint8_t *codes, c
     EQAT_TRY(check_ptr(Y, M * N, "Y"));
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     if (M * N == 0) return EQAT_OK;
-    if (K > 0) EQAT_TRY(check_ws(ws, ws_bytes, N, K, dt));
+    const bool f32 = dt == EQAT_F32;
+    // no workspace: W-hat made on load (bf16, a code layout the converter takes)
+    const bool onload = K > 0 && !f32 && fwd_onload(N, K, bits, group, ws != nullptr);
+    if (K > 0 && !(onload && ws == nullptr)) EQAT_TRY(check_ws(ws, ws_bytes, N, K, dt));
     EQAT_TRY(get_device(dev));
     if (K == 0) {
         EQAT_CUDA(zero(Y, static_cast<size_t>(M * N) * esize(dt), st), "memset Y");
         return EQAT_OK;
     }
-    const bool f32 = dt == EQAT_F32;
-    if (!f32 && M <= 8 && (group == 64 || group == 128) && gemv_enabled() &&
+    if (ws && !f32 && M <= 8 && (group == 64 || group == 128) && gemv_enabled() &&
         eqat::gemv_workspace_bytes(M, N, K, bits, group, dev.sm_count) <= ws_bytes) {
         // decode sizes: stream the codes once, no W-hat in memory (the partials
         // take at most M N K / 128 bytes, inside any workspace check_ws accepts)
@@ -572,7 +581,7 @@ eqat_status eqat_dq_linear_fwd_ex(const void *X, int dt, const uint8_t *codes, c
     epi.out = Y;
     epi.ldo = N;
     epi.out_f32 = f32;
-    if (!f32 && use_onload(M, N, K, bits, group)) {
+    if (onload) {
         // W-hat made from the codes inside the contraction, never written to HBM
         eqat::GemmProblem g{Operand{X, K, false}, Operand{nullptr, K, false}, M, N, K, epi};
         g.cvt = cvt_args(codes, zq, s, sdt, N, K, bits, group);
@@ -640,7 +649,7 @@ eqat_status eqat_dq_linear_bwd(const void *X, int dt, const uint8_t *codes, cons
         if (N == 0) {
             EQAT_CUDA(zero(dX, static_cast<size_t>(M * K) * esize(dt), st), "memset dX");
         } else {
-            const bool onload = !f32 && use_onload(M, N, K, bits, group);
+            const bool onload = !f32 && bwd_onload(N, K, bits, group);
             if (!w_hat_in_ws && !onload)
                 EQAT_CUDA(eqat::launch_dequant(codes, zq, s, sdt == EQAT_F16, N, K, bits, group, ws, f32, dev, st),
                           "dequant prepass");

@@ -31,6 +31,7 @@
 #include <mutex>
 
 #include "eqat_internal.h"
+#include "eqat_pdl.cuh"
 #include "eqat_ptx.cuh"
 #include "eqat_qmath.cuh"
 
@@ -429,7 +430,6 @@ __global__ void __launch_bounds__((4 + EPI_WARPS) * 32, 1)
                                                 ~static_cast<uintptr_t>(1023));
     SharedCtl *ctl = reinterpret_cast<SharedCtl *>(smem + STAGES * STAGE_BYTES);
     const int warp = threadIdx.x >> 5;
-    const int lane = threadIdx.x & 31;
     constexpr int EPI_THREADS = EPI_WARPS * 32;
 
     if (threadIdx.x == 0) {
@@ -451,6 +451,11 @@ __global__ void __launch_bounds__((4 + EPI_WARPS) * 32, 1)
             tma_prefetch_desc(&tmB1);
         }
     }
+    // A programmatic dependent (eqat_pdl.cuh): everything above touched only this
+    // CTA's shared memory and the kernel parameters; tensor and global memory come
+    // after the preceding kernel has completed.
+    pdl_wait();
+    if (threadIdx.x == 0) pdl_allow_dependents();
     if (warp == 2) {
         tmem_alloc(&ctl->tmem_base, TMEM_COLS);
         tmem_relinquish();
@@ -937,6 +942,11 @@ __global__ void __launch_bounds__((4 + EPI_WARPS + PairCfg<CVT, BITS, EPI_WARPS>
             tma_prefetch_desc(&tmB1);
         }
     }
+    // A programmatic dependent (eqat_pdl.cuh): everything above touched only this
+    // CTA's shared memory and the kernel parameters; tensor and global memory come
+    // after the preceding kernel has completed.
+    pdl_wait();
+    if (threadIdx.x == 0) pdl_allow_dependents();
     if (warp == 2) {
         tmem_alloc_pair(&ctl->tmem_base, TMEM_COLS);
         tmem_relinquish_pair();
@@ -1157,7 +1167,7 @@ __global__ void __launch_bounds__((4 + EPI_WARPS + PairCfg<CVT, BITS, EPI_WARPS>
         // ...: each slot's phases are waited on in order by one warp).  It gathers the
         // group constants of its next stage into registers before it waits for the
         // current one, so their L2 latency hides behind the other warps' stages.
-        constexpr int CW = C::CVT_WARPS;
+        constexpr int CW = C::CVT_WARPS > 0 ? C::CVT_WARPS : 1;  // never 0 where this role runs (CVT)
         const int cw = warp - (4 + EPI_WARPS);
         float2 *tab = reinterpret_cast<float2 *>(smem + STAGES2 * STAGE2_BYTES) + cw * 256;
         const uint32_t cvt_full0 = map_to_rank(&ctl->cvt_full[0], 0);
@@ -1344,8 +1354,8 @@ cudaError_t launch_variant(const CUtensorMap (&maps)[6], const KParams &p, int g
         if (e != cudaSuccess) return e;
         done.fetch_or(bit);
     }
-    kern<<<grid, (4 + kEpiWarps) * 32, SMEM_BYTES, st>>>(maps[0], maps[1], maps[2], maps[3], p);
-    return cudaGetLastError();
+    return launch_pdl(kern, dim3(grid), dim3((4 + kEpiWarps) * 32), SMEM_BYTES, st, maps[0], maps[1], maps[2],
+                      maps[3], p);
 }
 
 template <int EPI0, int EPI1, int BITS, int CVT = 0, int EW = 8>
@@ -1381,8 +1391,8 @@ cudaError_t launch_pair_variant(const CUtensorMap (&maps)[6], const KParams &p, 
         if (n <= 0) return cudaErrorInvalidConfiguration;
         resident[dev_id & 63].store(n);
     }
-    cfg.gridDim.x = static_cast<unsigned>(std::min(grid, 2 * n));
-    return cudaLaunchKernelEx(&cfg, kern, maps[0], maps[1], maps[2], maps[3], maps[4], maps[5], p);
+    return launch_pdl_ex(kern, dim3(static_cast<unsigned>(std::min(grid, 2 * n))), cfg.blockDim, C::SMEM, st,
+                         attr[0], maps[0], maps[1], maps[2], maps[3], maps[4], maps[5], p);
 }
 
 // EQAT_CVT_SCOPE=cta: converter hand-off at CTA scope (measurement aid).

@@ -48,6 +48,7 @@
 #include <cstdlib>
 
 #include "eqat_internal.h"
+#include "eqat_pdl.cuh"
 #include "eqat_ptx.cuh"
 
 namespace eqat {
@@ -228,11 +229,6 @@ __host__ __device__ __forceinline__ int cta_of_stage(int64_t x, int64_t S, int g
     return static_cast<int>(((x + 1) * grid - 1) / S);
 }
 
-// Programmatic dependent launch: a kernel launched with programmatic stream
-// serialization may start before its predecessor ends; pdl_wait() blocks the
-// calling thread until the predecessor has completed and its writes are visible.
-__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
-__device__ __forceinline__ void pdl_allow_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
 
 // Stage x = rt * spr + ks, advanced without divisions.
 struct StageCursor {
@@ -968,22 +964,6 @@ __global__ void k_gemv_reduce(const float *__restrict__ partials, int M, int N, 
             a += partials[((static_cast<int64_t>(rt) * maxseg + (c - c0)) * M + m) * kRows + row];
         Y[i] = __float2bfloat16_rn(a);
     }
-}
-
-// Launch with programmatic stream serialization (may overlap the predecessor).
-template <typename... KArgs, typename... Args>
-cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st, Args... args) {
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = grid;
-    cfg.blockDim = block;
-    cfg.dynamicSmemBytes = smem;
-    cfg.stream = st;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, kern, args...);
 }
 
 struct Plan {

@@ -17,6 +17,7 @@
 #include <type_traits>
 
 #include "eqat_internal.h"
+#include "eqat_pdl.cuh"
 #include "eqat_qmath.cuh"
 
 namespace eqat {
@@ -24,6 +25,14 @@ namespace {
 
 constexpr int kThreads = 256;
 constexpr int kBlocksPerSm = 8;
+
+// Every kernel here is launched as a programmatic dependent (eqat_pdl.cuh): it
+// waits for the preceding kernel before its first global access, then lets its
+// own dependents be scheduled.
+__device__ __forceinline__ void begin_dependent() {
+    pdl_wait();
+    pdl_allow_dependents();
+}
 
 // log2 of the group size (32, 64 or 128): index arithmetic by shifts, not division.
 inline int group_shift(int group) { return group == 32 ? 5 : group == 64 ? 6 : 7; }
@@ -59,6 +68,7 @@ struct InitLayers {
 
 template <typename T, int G, int NL>
 __global__ void __launch_bounds__(kThreads, 4) k_minmax_init(const __grid_constant__ InitLayers<T, NL> L, float Q) {
+    begin_dependent();
     constexpr int TPG = G / 8;
     constexpr int GPW = 32 / TPG;  // groups per warp per unrolled slot
     constexpr int UNROLL = kInitUnroll;
@@ -490,6 +500,7 @@ __global__ void __launch_bounds__(kTileThreads, kTileBlocksPerSm)
     k_fake_quant(const T *__restrict__ W, const float *__restrict__ s, const float *__restrict__ z, int64_t n,
                  int gshift, float Q, O *__restrict__ W_hat, uint8_t *__restrict__ code,
                  uint8_t *__restrict__ mask) {
+    begin_dependent();
     constexpr int CPL = kChunksPerLane<T>;
     __shared__ GroupConst gc[kTileWarps * kWarpGroups<CPL>];
     __shared__ PendingChunk queue[kTileWarps * kQueue<CPL>];
@@ -584,6 +595,7 @@ __device__ __forceinline__ bool pack_chunk(const float (&w)[16], const GroupCons
 template <typename T, int BITS, int NL>
 __global__ void __launch_bounds__(kTileThreads, kTileBlocksPerSm)
     k_pack(const __grid_constant__ TileLayers<T, NL> L, int gshift, float Q) {
+    begin_dependent();
     constexpr int CPL = kPackChunksPerLane<T, NL>;
     __shared__ GroupConst gc[kTileWarps * kWarpGroups<CPL>];
     __shared__ PendingChunk queue[kTileWarps * kQueue<CPL>];
@@ -640,6 +652,7 @@ template <int BITS, typename O, typename S, bool V8>
 __global__ void __launch_bounds__(kThreads)
     k_dequant(const uint8_t *__restrict__ codes, const uint8_t *__restrict__ zq,
               const S *__restrict__ s, int64_t n_chunks, int gshift, O *__restrict__ W_hat) {
+    begin_dependent();
     const int64_t stride = static_cast<int64_t>(gridDim.x) * kThreads;
     for (int64_t i = static_cast<int64_t>(blockIdx.x) * kThreads + threadIdx.x; i < n_chunks;
          i += stride) {
@@ -680,8 +693,7 @@ cudaError_t minmax_launch(const QuantLayerArgs *a, int n, float Q, const DeviceI
         }
         L.unit_end[i] = units;
     }
-    k_minmax_init<T, G, NL><<<grid_for(weights, dev, 8 * 4), kThreads, 0, st>>>(L, Q);
-    return cudaGetLastError();
+    return launch_pdl(k_minmax_init<T, G, NL>, dim3(grid_for(weights, dev, 8 * 4)), dim3(kThreads), 0, st, L, Q);
 }
 
 template <typename T, int NL>
@@ -716,12 +728,11 @@ cudaError_t pack_dispatch(const QuantLayerArgs *a, int n, int bits, int group, c
     const int grid = tile_grid<kPackChunksPerLane<T, NL>>(0, dev, tiles);
     const float Q = static_cast<float>((1 << bits) - 1);
     switch (bits) {
-        case 2: k_pack<T, 2, NL><<<grid, kTileThreads, 0, st>>>(L, gshift, Q); break;
-        case 3: k_pack<T, 3, NL><<<grid, kTileThreads, 0, st>>>(L, gshift, Q); break;
-        case 4: k_pack<T, 4, NL><<<grid, kTileThreads, 0, st>>>(L, gshift, Q); break;
+        case 2: return launch_pdl(k_pack<T, 2, NL>, dim3(grid), dim3(kTileThreads), 0, st, L, gshift, Q);
+        case 3: return launch_pdl(k_pack<T, 3, NL>, dim3(grid), dim3(kTileThreads), 0, st, L, gshift, Q);
+        case 4: return launch_pdl(k_pack<T, 4, NL>, dim3(grid), dim3(kTileThreads), 0, st, L, gshift, Q);
         default: return cudaErrorInvalidValue;
     }
-    return cudaGetLastError();
 }
 
 // Drops empty layers, then one launch per kMultiLayers layers (single-layer
@@ -750,12 +761,11 @@ cudaError_t dequant_dispatch_v(const uint8_t *codes, const uint8_t *zq, const S 
     const int64_t chunks = n / 16;
     const int grid = grid_for(chunks, dev);
     switch (bits) {
-        case 2: k_dequant<2, O, S, V8><<<grid, kThreads, 0, st>>>(codes, zq, s, chunks, gshift, W_hat); break;
-        case 3: k_dequant<3, O, S, V8><<<grid, kThreads, 0, st>>>(codes, zq, s, chunks, gshift, W_hat); break;
-        case 4: k_dequant<4, O, S, V8><<<grid, kThreads, 0, st>>>(codes, zq, s, chunks, gshift, W_hat); break;
+        case 2: return launch_pdl(k_dequant<2, O, S, V8>, dim3(grid), dim3(kThreads), 0, st, codes, zq, s, chunks, gshift, W_hat);
+        case 3: return launch_pdl(k_dequant<3, O, S, V8>, dim3(grid), dim3(kThreads), 0, st, codes, zq, s, chunks, gshift, W_hat);
+        case 4: return launch_pdl(k_dequant<4, O, S, V8>, dim3(grid), dim3(kThreads), 0, st, codes, zq, s, chunks, gshift, W_hat);
         default: return cudaErrorInvalidValue;
     }
-    return cudaGetLastError();
 }
 
 inline bool aligned32(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 31u) == 0; }
@@ -807,30 +817,25 @@ cudaError_t launch_fake_quant(const void *W, bool w_f32, const float *s, const f
     const int gshift = group_shift(group);
     const bool v8 = aligned32(W_hat);
 #define EQAT_FQ_LAUNCH_V(TW, TO, CODES, V8)                                                                  \
-    k_fake_quant<TW, TO, CODES, V8><<<tile_grid<kChunksPerLane<TW>>(n, dev), kTileThreads, 0, st>>>(                        \
-        static_cast<const TW *>(W), s, z, n, gshift, Q, static_cast<TO *>(W_hat), code, mask)
+    launch_pdl(k_fake_quant<TW, TO, CODES, V8>, dim3(tile_grid<kChunksPerLane<TW>>(n, dev)), dim3(kTileThreads), 0, \
+               st, static_cast<const TW *>(W), s, z, n, gshift, Q, static_cast<TO *>(W_hat), code, mask)
 #define EQAT_FQ_LAUNCH(TW, TO)                                                                              \
-    do {                                                                                                    \
-        if (codes && v8)                                                                                    \
-            EQAT_FQ_LAUNCH_V(TW, TO, true, true);                                                           \
-        else if (codes)                                                                                     \
-            EQAT_FQ_LAUNCH_V(TW, TO, true, false);                                                          \
-        else if (v8)                                                                                        \
-            EQAT_FQ_LAUNCH_V(TW, TO, false, true);                                                          \
-        else                                                                                                \
-            EQAT_FQ_LAUNCH_V(TW, TO, false, false);                                                         \
-    } while (0)
+    (codes && v8 ? EQAT_FQ_LAUNCH_V(TW, TO, true, true)                                                     \
+     : codes     ? EQAT_FQ_LAUNCH_V(TW, TO, true, false)                                                    \
+     : v8        ? EQAT_FQ_LAUNCH_V(TW, TO, false, true)                                                    \
+                 : EQAT_FQ_LAUNCH_V(TW, TO, false, false))
+    cudaError_t e;
     if (w_f32 && out_f32)
-        EQAT_FQ_LAUNCH(float, float);
+        e = EQAT_FQ_LAUNCH(float, float);
     else if (w_f32)
-        EQAT_FQ_LAUNCH(float, bf);
+        e = EQAT_FQ_LAUNCH(float, bf);
     else if (out_f32)
-        EQAT_FQ_LAUNCH(bf, float);
+        e = EQAT_FQ_LAUNCH(bf, float);
     else
-        EQAT_FQ_LAUNCH(bf, bf);
+        e = EQAT_FQ_LAUNCH(bf, bf);
 #undef EQAT_FQ_LAUNCH
 #undef EQAT_FQ_LAUNCH_V
-    return cudaGetLastError();
+    return e;
 }
 
 cudaError_t launch_pack_multi(const QuantLayerArgs *layers, int n, bool w_f32, int bits, int group,

@@ -1220,6 +1220,7 @@ def main():
     ap.add_argument("--configs-only", action="store_true")
     ap.add_argument("--initpack70b-only", action="store_true")
     ap.add_argument("--quant-multi-only", action="store_true")
+    ap.add_argument("--quant-gate-only", action="store_true")
     ap.add_argument("--dq-only", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-hbm", action="store_true")
@@ -1277,6 +1278,23 @@ def main():
         if eqat.device_error() != 0:
             raise RuntimeError("device error word set")
         print(json.dumps({"dq_only": "ok"}), flush=True)
+        return
+    if args.quant_gate_only:  # profiling aid: init, prepass, pack, dequant once each on the 70B gate_proj
+        torch.cuda.set_device(0)
+        eqat.load_library()
+        dev = torch.device("cuda", 0)
+        gen = torch.Generator(device=dev)
+        gen.manual_seed(1008)
+        W = (torch.randn(28672, 8192, generator=gen, device=dev) * 0.015).to(torch.bfloat16)
+        s_, z_ = eqat.minmax_init(W, 2, 64)
+        wh = torch.empty_like(W)
+        eqat.fake_quant(W, s_, z_, 2, 64, want_code=False, want_mask=False, W_hat=wh)
+        codes, zq = eqat.pack_codes(W, s_, z_, 2, 64)
+        eqat.dequant_codes(codes, zq, s_, 8192, 2, 64, out=wh)
+        torch.cuda.synchronize()
+        if eqat.device_error() != 0:
+            raise RuntimeError("device error word set")
+        print(json.dumps({"quant_gate_only": "ok"}), flush=True)
         return
     if args.quant_multi_only:  # profiling aid: block-wide init and pack once each, Llama-2-7B block shapes
         torch.cuda.set_device(0)

@@ -29,6 +29,10 @@
 #include <cstdint>
 #include <cstdlib>
 #include <mutex>
+#include <queue>
+#include <type_traits>
+#include <utility>
+#include <vector>
 
 #include "eqat_internal.h"
 #include "eqat_pdl.cuh"
@@ -102,6 +106,50 @@ struct KParams {
     uint64_t wait_limit_ns;
     int cvt_cluster_scope;  // converter hand-off: release/acquire at cluster (1) or CTA (0) scope
 };
+
+// The tiles of a pair launch are dealt round-robin (pair q takes q, q + npairs, ...)
+// unless the launch carries a TileSched: a host-made deal, pair q taking
+// tile[begin[q] .. begin[q + 1]).  Used for grouped launches whose two problems
+// have tiles of very different cost (a dW-hat contraction 2048 deep beside a dX
+// contraction 8192-28672 deep), where round-robin leaves some pairs one long tile
+// more than others and no fewer short ones.
+constexpr int kSchedTiles = 8192;
+constexpr int kSchedPairs = 128;
+struct TileSched {
+    uint16_t begin[kSchedPairs + 1];
+    uint16_t tile[kSchedTiles];
+};
+struct NoSched {
+    int unused;
+};
+template <int SCHED>
+using SchedParam = typename std::conditional<SCHED != 0, TileSched, NoSched>::type;
+// kernel parameters of a scheduled pair launch: six tensor maps, KParams, the deal
+static_assert(6 * sizeof(CUtensorMap) + sizeof(KParams) + sizeof(TileSched) <= 32000,
+              "a scheduled pair launch must fit the kernel-parameter limit");
+
+// This pair's tiles: positions first, first + step, ... below end; tile_at maps a
+// position to the tile.
+template <int SCHED>
+__device__ __forceinline__ void sched_range(const SchedParam<SCHED> &sc, int total_tiles, int pair, int npairs,
+                                            int &first, int &end, int &step) {
+    if constexpr (SCHED != 0) {
+        first = sc.begin[pair];
+        end = sc.begin[pair + 1];
+        step = 1;
+    } else {
+        first = pair;
+        end = total_tiles;
+        step = npairs;
+    }
+}
+template <int SCHED>
+__device__ __forceinline__ int sched_tile(const SchedParam<SCHED> &sc, int i) {
+    if constexpr (SCHED != 0)
+        return sc.tile[i];
+    else
+        return i;
+}
 
 struct SharedCtl {
     uint64_t full[STAGES];
@@ -900,12 +948,12 @@ struct StageWalk {
 //   cvt_full[s]  the leader's: one arrival per converter warp of both CTAs once the
 //                warp's part of the B tile is written and fenced for the tensor core;
 //                the MMA issuer waits on it besides full[s] (which then counts A only)
-template <int EPI0, int EPI1, int BITS, int EPI_WARPS, int CVT>
+template <int EPI0, int EPI1, int BITS, int EPI_WARPS, int CVT, int SCHED>
 __global__ void __launch_bounds__((4 + EPI_WARPS + PairCfg<CVT, BITS, EPI_WARPS>::CVT_WARPS) * 32, 1)
     k_gemm_tc2(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUtensorMap tmB0,
                const __grid_constant__ CUtensorMap tmA1, const __grid_constant__ CUtensorMap tmB1,
                const __grid_constant__ CUtensorMap tmO0, const __grid_constant__ CUtensorMap tmO1,
-               const KParams p) {
+               const KParams p, const __grid_constant__ SchedParam<SCHED> sched) {
     using C = PairCfg<CVT, BITS, EPI_WARPS>;
     static_assert(EPI_WARPS == C::EPI_WARPS, "the staging area is sized for C::EPI_WARPS epilogue warps");
     constexpr int STAGES2 = C::STAGES;
@@ -968,8 +1016,10 @@ __global__ void __launch_bounds__((4 + EPI_WARPS + PairCfg<CVT, BITS, EPI_WARPS>
             uint32_t carmed = 0, carmed_parity = 0;   // this CTA's code barriers with a phase armed
             uint32_t cuse = 0;                        // per stage: parity of its next code phase
             bool ok = true;
-            for (int t = pair; ok && t < p.total_tiles; t += npairs) {
-                const TileInfo ti = tile_info(p, t);
+            int w_first, w_end, w_step;
+            sched_range<SCHED>(sched, p.total_tiles, pair, npairs, w_first, w_end, w_step);
+            for (int w = w_first; ok && w < w_end; w += w_step) {
+                const TileInfo ti = tile_info(p, sched_tile<SCHED>(sched, w));
                 const int pi = ti.pi;
                 const CUtensorMap *ma = pi ? &tmA1 : &tmA0;
                 // the halves of a split wave take B through the second map (half the box rows)
@@ -1062,8 +1112,10 @@ __global__ void __launch_bounds__((4 + EPI_WARPS + PairCfg<CVT, BITS, EPI_WARPS>
             uint32_t it = 0, local = 0;
             uint32_t cuse = 0;  // per stage: parity of its next converted phase
             bool ok = true, issued = false;
-            for (int t = pair; ok && t < p.total_tiles; t += npairs, ++local) {
-                const TileInfo ti = tile_info(p, t);
+            int w_first, w_end, w_step;
+            sched_range<SCHED>(sched, p.total_tiles, pair, npairs, w_first, w_end, w_step);
+            for (int w = w_first; ok && w < w_end; w += w_step, ++local) {
+                const TileInfo ti = tile_info(p, sched_tile<SCHED>(sched, w));
                 const int pi = ti.pi;
                 const int a_mn = pi ? p.pr[1].a_mn : p.pr[0].a_mn;
                 const int b_mn = pi ? p.pr[1].b_mn : p.pr[0].b_mn;
@@ -1132,13 +1184,15 @@ __global__ void __launch_bounds__((4 + EPI_WARPS + PairCfg<CVT, BITS, EPI_WARPS>
         constexpr int SLICES = EPI_WARPS / 4;
         uint32_t local = 0;
         OutStage os{smem + STAGES2 * STAGE2_BYTES + C::CONST_BYTES + ew * 2048, nullptr, false};
-        for (int t = pair; t < p.total_tiles; t += npairs, ++local) {
+        int w_first, w_end, w_step;
+        sched_range<SCHED>(sched, p.total_tiles, pair, npairs, w_first, w_end, w_step);
+        for (int w = w_first; w < w_end; w += w_step, ++local) {
             const uint32_t acc = local & 1u;
             const uint32_t aph = (local >> 1) & 1u;
             const bool ok = mbar_wait_bounded(&ctl->acc_full[acc], aph, abort_flag, p.err, p.wait_limit_ns);
             if (!__all_sync(0xffffffffu, ok)) break;
             tc_fence_after();
-            const TileInfo ti = tile_info(p, t);
+            const TileInfo ti = tile_info(p, sched_tile<SCHED>(sched, w));
             const int row0 = ti.tm * BM2 + 128 * static_cast<int>(rank) + quad * 32;
             const uint32_t taddr = tmem_base + acc * ACC_COLS + ((quad * 32) << 16);
             // a slice holds whole groups where the epilogue reduces over groups (then
@@ -1358,11 +1412,61 @@ cudaError_t launch_variant(const CUtensorMap (&maps)[6], const KParams &p, int g
                       maps[3], p);
 }
 
-template <int EPI0, int EPI1, int BITS, int CVT = 0, int EW = 8>
+// Tile costs of a two-problem launch, for a host-made deal (tile_cost per tile of
+// problem 0 and problem 1).
+struct SchedSpec {
+    int tiles0, tiles1;
+    int cost0, cost1;
+};
+
+// Longest tiles first, each to the least-loaded pair (ties: the lowest pair); a pair
+// takes its tiles in the order dealt.  The last deal is kept: a training loop
+// launches the same shapes over and over.
+bool build_sched(const SchedSpec &sp, int npairs, TileSched &out) {
+    const int total = sp.tiles0 + sp.tiles1;
+    if (npairs < 1 || npairs > kSchedPairs || total > kSchedTiles) return false;
+    static std::mutex mu;
+    static SchedSpec last{};
+    static int last_pairs = 0;
+    static TileSched cached;
+    std::lock_guard<std::mutex> lock(mu);
+    if (last_pairs == npairs && last.tiles0 == sp.tiles0 && last.tiles1 == sp.tiles1 && last.cost0 == sp.cost0 &&
+        last.cost1 == sp.cost1) {
+        out = cached;
+        return true;
+    }
+    std::vector<std::vector<uint16_t>> lists(static_cast<size_t>(npairs));
+    using Load = std::pair<int64_t, int>;  // (load, pair): the smallest on top
+    std::priority_queue<Load, std::vector<Load>, std::greater<Load>> heap;
+    for (int q = 0; q < npairs; ++q) heap.push({0, q});
+    const bool first1 = sp.cost1 > sp.cost0;
+    for (int k = 0; k < 2; ++k) {
+        const int prob = (k == 0) == first1 ? 1 : 0;
+        const int n = prob ? sp.tiles1 : sp.tiles0, base = prob ? sp.tiles0 : 0, cost = prob ? sp.cost1 : sp.cost0;
+        for (int i = 0; i < n; ++i) {
+            const Load top = heap.top();
+            heap.pop();
+            lists[static_cast<size_t>(top.second)].push_back(static_cast<uint16_t>(base + i));
+            heap.push({top.first + cost, top.second});
+        }
+    }
+    int pos = 0;
+    for (int q = 0; q < npairs; ++q) {
+        out.begin[q] = static_cast<uint16_t>(pos);
+        for (uint16_t t : lists[static_cast<size_t>(q)]) out.tile[pos++] = t;
+    }
+    for (int q = npairs; q <= kSchedPairs; ++q) out.begin[q] = static_cast<uint16_t>(pos);
+    last = sp;
+    last_pairs = npairs;
+    cached = out;
+    return true;
+}
+
+template <int EPI0, int EPI1, int BITS, int CVT = 0, int EW = 8, int SCHED = 0>
 cudaError_t launch_pair_variant(const CUtensorMap (&maps)[6], const KParams &p, int grid, int dev_id,
-                                cudaStream_t st) {
+                                cudaStream_t st, const SchedSpec *spec = nullptr) {
     using C = PairCfg<CVT, BITS, CVT ? 4 : EW>;
-    auto kern = k_gemm_tc2<EPI0, EPI1, BITS, C::EPI_WARPS, CVT>;
+    auto kern = k_gemm_tc2<EPI0, EPI1, BITS, C::EPI_WARPS, CVT, SCHED>;
     static std::atomic<uint64_t> done{0};
     const uint64_t bit = 1ull << (dev_id & 63);
     if (!(done.load() & bit)) {
@@ -1391,8 +1495,22 @@ cudaError_t launch_pair_variant(const CUtensorMap (&maps)[6], const KParams &p, 
         if (n <= 0) return cudaErrorInvalidConfiguration;
         resident[dev_id & 63].store(n);
     }
-    return launch_pdl_ex(kern, dim3(static_cast<unsigned>(std::min(grid, 2 * n))), cfg.blockDim, C::SMEM, st,
-                         attr[0], maps[0], maps[1], maps[2], maps[3], maps[4], maps[5], p);
+    const int launched = std::min(grid, 2 * n);
+    SchedParam<SCHED> sc{};
+    if constexpr (SCHED != 0) {
+        if (!spec || !build_sched(*spec, launched / 2, sc)) return cudaErrorInvalidValue;
+    }
+    return launch_pdl_ex(kern, dim3(static_cast<unsigned>(launched)), cfg.blockDim, C::SMEM, st, attr[0], maps[0],
+                         maps[1], maps[2], maps[3], maps[4], maps[5], p, sc);
+}
+
+// EQAT_GEMM_SCHED=0: grouped launches deal tiles round-robin always (measurement aid).
+bool sched_disabled() {
+    static const bool off = [] {
+        const char *v = std::getenv("EQAT_GEMM_SCHED");
+        return v && v[0] == '0';
+    }();
+    return off;
 }
 
 // EQAT_CVT_SCOPE=cta: converter hand-off at CTA scope (measurement aid).
@@ -1660,6 +1778,21 @@ cudaError_t launch_gemm_tc_group(const GemmProblem *probs, int nprob, const Devi
     if (any_cvt) return cudaErrorInvalidValue;
     if (pair) {
         const int grid = 2 * std::min(p.total_tiles, units);
+        // Two problems whose tiles differ in cost by 2x or more (main-loop k-blocks,
+        // or the reducing epilogue's time where that is longer, about 24 k-blocks)
+        // get a host-made deal instead of round-robin.
+        SchedSpec spec{};
+        bool sched = false;
+        if (nprob == 2 && !sched_disabled()) {
+            auto cost = [](const Prob &q, bool reduces) {
+                const int nkb = (q.GK + BK - 1) / BK;
+                return reduces ? std::max(nkb, 24) : nkb;
+            };
+            spec = SchedSpec{p.pr[0].tiles_m * p.pr[0].tiles_n, p.pr[1].tiles_m * p.pr[1].tiles_n,
+                             cost(p.pr[0], probs[0].epi.kind != Epi::kStore), cost(p.pr[1], probs[1].epi.kind != Epi::kStore)};
+            const int lo = std::min(spec.cost0, spec.cost1), hi = std::max(spec.cost0, spec.cost1);
+            sched = hi >= 2 * lo && spec.tiles0 + spec.tiles1 <= kSchedTiles;
+        }
         switch (probs[0].epi.kind) {
             case Epi::kStore:
                 if (nprob > 1) return cudaErrorInvalidValue;
@@ -1669,13 +1802,19 @@ cudaError_t launch_gemm_tc_group(const GemmProblem *probs, int nprob, const Devi
                 // warps (per-tile timestamps on the 70B gate backward: 13.7 us against
                 // 10 us); sixteen keep up there (3% off that backward) but cost 1.7% on
                 // 4096-deep contractions, where eight already hide behind the main loop.
-                if (probs[0].GK <= 2048) return launch_pair_variant<1, 0, 2, 0, 16>(maps, p, grid, dev.device, st);
-                return launch_pair_variant<1, 0, 2>(maps, p, grid, dev.device, st);
+                if (probs[0].GK <= 2048)
+                    return sched ? launch_pair_variant<1, 0, 2, 0, 16, 1>(maps, p, grid, dev.device, st, &spec)
+                                 : launch_pair_variant<1, 0, 2, 0, 16>(maps, p, grid, dev.device, st);
+                return sched ? launch_pair_variant<1, 0, 2, 0, 8, 1>(maps, p, grid, dev.device, st, &spec)
+                             : launch_pair_variant<1, 0, 2>(maps, p, grid, dev.device, st);
             case Epi::kE2eDs:
                 switch (probs[0].epi.bits) {
-                    case 2: return launch_pair_variant<2, 0, 2>(maps, p, grid, dev.device, st);
-                    case 3: return launch_pair_variant<2, 0, 3>(maps, p, grid, dev.device, st);
-                    case 4: return launch_pair_variant<2, 0, 4>(maps, p, grid, dev.device, st);
+                    case 2: return sched ? launch_pair_variant<2, 0, 2, 0, 8, 1>(maps, p, grid, dev.device, st, &spec)
+                                         : launch_pair_variant<2, 0, 2>(maps, p, grid, dev.device, st);
+                    case 3: return sched ? launch_pair_variant<2, 0, 3, 0, 8, 1>(maps, p, grid, dev.device, st, &spec)
+                                         : launch_pair_variant<2, 0, 3>(maps, p, grid, dev.device, st);
+                    case 4: return sched ? launch_pair_variant<2, 0, 4, 0, 8, 1>(maps, p, grid, dev.device, st, &spec)
+                                         : launch_pair_variant<2, 0, 4>(maps, p, grid, dev.device, st);
                     default: return cudaErrorInvalidValue;
                 }
             case Epi::kMse:
